@@ -1,0 +1,341 @@
+#!/usr/bin/env python
+"""Benchmark of the Gated Delta Rule chunked forward on B200.
+
+One step = one forward pass (chunk table, prologue, intra-chunk, state pass,
+output) over the one-layer prefill workload: B = 1, T = 32768 tokens,
+Nqk = 16, Nv = 32, Dk = Dv = 128, L = 128, bf16 q/k/v/beta, fp32 g, inputs
+already resident in HBM.  Every rank of a multi-GPU run processes its own
+batch (independent problems, weak scaling, no collective on the data path).
+
+FLOPs per token (dense tensor-core work, counted once per qk-head where the
+product is shared by the v-heads of a group):
+    F = Nv (4 L Dv + 2 L Dk + 6 Dk Dv) + Nqk (4 L Dk)    (= 7,340,032 at this size)
+i.e. per chunk and v-head: U = T (beta V), W = T (beta e^gamma K), W S, Q S,
+P U', K^T U'; per chunk and qk-head: K K^T and Q K^T.  The triangular solve
+and the masked halves are not counted.
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the fp64 CPU
+oracle (the reference arm) on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_deltanet_linear_17_b200 import dist as gdist  # noqa: E402
+from gated_deltanet_linear_17_b200 import inputs  # noqa: E402
+
+METRIC = "GDN fwd tokens/s @Nv32 D128 S32K; % bf16 TC roofline; short-seq HBM GB/s"
+WORKLOAD = "prefill_s32k"
+L = D = 128
+
+
+def flops_per_token(Nqk, Nv):
+    return Nv * (4 * L * D + 2 * L * D + 6 * D * D) + Nqk * (4 * L * D)
+
+
+def stage_work(T, Nqk, Nv):
+    """Algorithmic work of one launch of each stage: (bound, amount, unit)."""
+    return {
+        "chunk_map": ("hbm", 0.0, "GB/s"),
+        # q and k read and written back normalised (fp16), g and beta read, gamma and beta written
+        "prologue": ("hbm", T * (4 * Nqk * D * 2 + Nv * 4 + Nv * 2 + 2 * Nv * 4), "GB/s"),
+        "intra": ("tensor", T * (Nv * (2 * L * D + 2 * L * D) + Nqk * 2 * L * D), "TFLOP/s"),
+        "state": ("tensor", T * Nv * 4 * D * D, "TFLOP/s"),
+        "output": ("tensor", T * (Nv * (2 * D * D + 2 * L * D) + Nqk * 2 * L * D), "TFLOP/s"),
+    }
+
+
+def short_bytes(inp):
+    """HBM bytes of the short-sequence pass: state read + write plus per-token I/O."""
+    per_tok = 2 * inp.Nqk * D * 2 + inp.Nv * D * 2 + inp.Nv * 4 + inp.Nv * 2 + inp.Nv * D * 2
+    return 2 * inp.B * inp.Nv * D * D * 4 + inp.T * per_tok
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            uuid = str(device_index)
+        self.target = uuid
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="gdn_clocks_", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.target, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 7:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx = float(parts[1])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[3:7]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_sample(inp, tokens):
+    """Time the fp64 oracle on the first `tokens` tokens of a one-sequence batch (all v-heads)."""
+    import oracle
+    n = min(tokens, inp.T)
+    t0 = time.perf_counter()
+    _, _, threads = oracle.recurrent(inp.q[:n], inp.k[:n], inp.v[:n], inp.g[:n], inp.beta[:n],
+                                     torch.tensor([0, n], dtype=torch.int32), None, None,
+                                     scale=inp.scale, eps=inp.eps, return_threads=True)
+    dt = time.perf_counter() - t0
+    return n / dt, threads, dt, n
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 CPU oracle, timed as it stands on the host cores."""
+    if rank != 0:
+        return 0
+    inp = inputs.config(WORKLOAD)
+    tok = args.ref_tokens
+    for _ in range(args.warmup):
+        cpu_oracle_sample(inp, min(tok, 256))
+    t0 = time.perf_counter()
+    threads = 0
+    for _ in range(args.steps):
+        _, threads, _, n = cpu_oracle_sample(inp, tok)
+    dt = time.perf_counter() - t0
+    value = args.steps * n / dt
+    sample = f"first {n} tokens of the {inp.T}-token sequence, all {inp.Nv} v-heads, per step"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(inp),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(inp):
+    return {"workload": f"{WORKLOAD}: one-layer prefill, B={inp.B} T={inp.T} Nqk={inp.Nqk} Nv={inp.Nv} "
+                        f"D=128 L=128", "B": inp.B, "T": inp.T, "Nqk": inp.Nqk, "Nv": inp.Nv, "D": 128, "L": 128,
+            "flop_per_token": flops_per_token(inp.Nqk, inp.Nv),
+            "l2": "inputs larger than L2 (q, k, v, out = 805 MB per step; no flush)",
+            "parallelism": "independent batch per GPU (weak scaling, no data-path collective)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-tokens", type=int, default=8192, help="tokens of the CPU-oracle baseline sample")
+    ap.add_argument("--ref-tokens", type=int, default=2048, help="tokens per step of the reference arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-short", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        rank, _, world = gdist.env_rank()
+        return run_reference(args, rank, world)
+
+    import gated_deltanet_linear_17_b200 as gdn
+    rank, local, world = gdist.init("nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+
+    host = inputs.config(WORKLOAD, seed=inputs.CONFIGS[WORKLOAD]["seed"] + rank)
+    inp = host.to(dev)
+    T, B, Nqk, Nv = inp.T, inp.B, inp.Nqk, inp.Nv
+    st = gdn.Stages(T, B, Nqk, Nv, dev)
+    out = torch.empty(T, Nv, D, dtype=torch.bfloat16, device=dev)
+    fin = torch.empty(B, Nv, D, D, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    names = ["chunk_map", "prologue", "intra", "state", "output"]
+
+    def step(evs=None):
+        calls = [lambda: st.chunk_map(inp.cu_seqlens),
+                 lambda: st.prologue(inp.q, inp.k, inp.g, inp.beta, inp.scale, inp.eps),
+                 lambda: st.intra(inp.v),
+                 lambda: st.state(inp.state_pool, inp.state_indices, fin),
+                 lambda: st.output(out)]
+        for i, c in enumerate(calls):
+            if evs is not None:
+                evs[i].record(stream)
+            c()
+        if evs is not None:
+            evs[len(calls)].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
+    clk = ClockSampler(local) if rank == 0 else None
+    if clk:
+        clk.start()
+    gdist.barrier()
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        step(evs[k])
+    torch.cuda.synchronize()
+    gdist.barrier()
+    clocks = clk.stop() if clk else None
+
+    total_ms = evs[0][0].elapsed_time(evs[-1][-1])
+    stage_ms = {n: sum(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps)) / args.steps
+                for i, n in enumerate(names)}
+    ms = gdist.max_over_ranks(total_ms / args.steps, device=dev)
+    value = world * T / (ms / 1e3)
+    F = flops_per_token(Nqk, Nv)
+    tc_frac = F * T / (ms / 1e3) / (peaks["bf16_tflops"] * 1e12)
+
+    work = stage_work(T, Nqk, Nv)
+    dom = max(names, key=lambda n: stage_ms[n])
+    bound, amount, unit = work[dom]
+    sec = stage_ms[dom] / 1e3
+    if bound == "hbm":
+        achieved, peak = amount / sec / 1e9, peaks["hbm_gbs"]
+    else:
+        achieved, peak = amount / sec / 1e12, peaks["bf16_tflops"]
+    roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": None,
+                "peak_source": f"{peaks['source']} (burst bf16 / STREAM copy)",
+                "per_launch": f"{amount:.4g} {'bytes' if bound == 'hbm' else 'FLOP'} per launch"}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; see inputs.CONFIGS)",
+            "config": workload_config(inp), "tc_frac": tc_frac,
+            "stages_ms": {n: round(v, 5) for n, v in stage_ms.items()}, "roofline": roofline,
+            "gpu_launches": len(names) * args.steps, "clocks": clocks}
+
+    # ---- short-sequence state-pool pass (HBM-bound)
+    if not args.no_short:
+        sh = inputs.config("short_pool_b256", seed=inputs.CONFIGS["short_pool_b256"]["seed"] + rank).to(dev)
+        so = torch.empty(sh.T, sh.Nv, D, dtype=torch.bfloat16, device=dev)
+        sf = torch.empty(sh.B, sh.Nv, D, D, dtype=torch.float32, device=dev)
+        ms_len = sh.max_seqlen
+
+        def sstep():
+            gdn.chunk_fwd(sh.q, sh.k, sh.v, sh.g, sh.beta, sh.cu_seqlens, sh.state_pool, sh.state_indices,
+                          scale=sh.scale, eps=sh.eps, max_seqlen=ms_len, out=so, final_state=sf)
+        for _ in range(args.warmup):
+            sstep()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            sstep()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        sms = gdist.max_over_ranks(e0.elapsed_time(e1) / args.steps, device=dev)
+        nb = short_bytes(sh)
+        gbs = nb / (sms / 1e3) / 1e9
+        line["short_seq"] = {"workload": f"short_pool_b256: B={sh.B} lens 1..8 (T={sh.T}), Nqk={sh.Nqk}, "
+                                         f"Nv={sh.Nv}, fp32 pool [512,{sh.Nv},128,128]",
+                             "ms": sms, "bytes": nb, "GB/s": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+                             "tokens/s": world * sh.T / (sms / 1e3), "kernel": "short_kernel",
+                             "l2": "state traffic 1.07 GB per step > L2"}
+        line["gpu_launches"] += args.steps
+        del sh, so, sf
+
+    # ---- end to end from pinned host buffers through the public call
+    if not args.no_e2e:
+        pin = lambda t: None if t is None else t.pin_memory()
+        hq, hk, hv, hg, hb, hc = (pin(getattr(host, n)) for n in ("q", "k", "v", "g", "beta", "cu_seqlens"))
+        oh = torch.empty(T, Nv, D, dtype=torch.bfloat16, pin_memory=True)
+        fh = torch.empty(B, Nv, D, D, dtype=torch.float32, pin_memory=True)
+        ws = st.ws
+        for _ in range(max(1, args.warmup // 2)):
+            gdn.chunk_fwd_host(hq, hk, hv, hg, hb, hc, scale=host.scale, eps=host.eps, device=dev,
+                               out_host=oh, final_host=fh, workspace=ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        gdist.barrier()
+        e0.record(stream)
+        h2d = d2h = 0
+        for _ in range(args.steps):
+            _, _, h2d, d2h = gdn.chunk_fwd_host(hq, hk, hv, hg, hb, hc, scale=host.scale, eps=host.eps, device=dev,
+                                                out_host=oh, final_host=fh, workspace=ws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = gdist.max_over_ranks(e0.elapsed_time(e1) / args.steps, device=dev)
+        line["e2e"] = {"value": world * T / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "ms_per_step": ems}
+        line["gpu_launches"] += 5 * args.steps
+
+    # ---- CPU oracle baseline (rank 0, one GPU only)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, threads, dt, n = cpu_oracle_sample(host, args.cpu_tokens)
+        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": f"first {n} of {T} tokens, all {Nv} v-heads ({dt:.1f} s wall)"}
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if torch.distributed.is_initialized():
+        gdist.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,302 @@
+"""ctypes binding of ``libgdn.so`` (include/gdn.h, include/gdn_stages.h).
+
+Argument marshalling only: shapes and dtypes are checked, torch supplies the
+device memory and the current stream, and every step of the computation runs
+in the library's CUDA kernels.  There is no fallback: if the library is
+missing or a tensor is not on a CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdn.so")
+HEAD_DIM = 128
+CHUNK = 128
+SHORT_MAX = 16
+
+GDN_OK, GDN_ERR_NULL_ARG, GDN_ERR_BAD_SHAPE, GDN_ERR_UNSUPPORTED = 0, 1, 2, 3
+GDN_ERR_ALIGNMENT, GDN_ERR_WORKSPACE, GDN_ERR_CUDA, GDN_ERR_OVERLAP = 4, 5, 6, 7
+
+_lib = None
+
+
+class _Layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in
+                ("total", "status", "chunk_info", "seq_chunk0", "qn", "kn", "gcum", "betaf", "U", "W", "Up", "Sc")] + \
+               [("max_chunks", ctypes.c_int64)]
+
+
+def lib():
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m gated_deltanet_linear_17_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        p, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+        L.gdn_status_string.restype = ctypes.c_char_p
+        L.gdn_status_string.argtypes = [ctypes.c_int]
+        L.gdn_version.restype = ctypes.c_int
+        L.gdn_chunk_fwd_workspace_bytes.restype = sz
+        L.gdn_chunk_fwd_workspace_bytes.argtypes = [i64, i32, i32, i32]
+        L.gdn_workspace_layout.restype = ctypes.c_int
+        L.gdn_workspace_layout.argtypes = [i64, i32, i32, i32, ctypes.POINTER(_Layout)]
+        L.gdn_chunk_fwd.restype = ctypes.c_int
+        L.gdn_chunk_fwd.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, i32, p, sz, p]
+        L.gdn_short_fwd.restype = ctypes.c_int
+        L.gdn_short_fwd.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, p]
+        L.gdn_stage_chunk_map.restype = ctypes.c_int
+        L.gdn_stage_chunk_map.argtypes = [p, i64, i32, i32, i32, p, sz, p]
+        L.gdn_stage_prologue.restype = ctypes.c_int
+        L.gdn_stage_prologue.argtypes = [p, p, p, p, f32, f32, i64, i32, i32, i32, p, sz, p]
+        L.gdn_stage_intra.restype = ctypes.c_int
+        L.gdn_stage_intra.argtypes = [p, i64, i32, i32, i32, p, sz, p]
+        L.gdn_stage_state.restype = ctypes.c_int
+        L.gdn_stage_state.argtypes = [p, p, p, i64, i32, i32, i32, i32, p, sz, p]
+        L.gdn_stage_output.restype = ctypes.c_int
+        L.gdn_stage_output.argtypes = [p, i64, i32, i32, i32, p, sz, p]
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().gdn_status_string(int(code)).decode()
+
+
+def _check(code: int, what: str):
+    if code == GDN_OK:
+        return
+    msg = f"{what}: {status_string(code)}"
+    if code in (GDN_ERR_BAD_SHAPE, GDN_ERR_UNSUPPORTED, GDN_ERR_NULL_ARG, GDN_ERR_OVERLAP, GDN_ERR_WORKSPACE,
+                GDN_ERR_ALIGNMENT):
+        raise ValueError(msg)
+    raise RuntimeError(msg)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype, shape, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise RuntimeError(f"{name} must be on a CUDA device (got {t.device})")
+    if device is not None and t.device != device:
+        raise RuntimeError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise RuntimeError(f"{name} must be {dtype} (got {t.dtype})")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def workspace_bytes(T: int, B: int, Nqk: int, Nv: int) -> int:
+    return int(lib().gdn_chunk_fwd_workspace_bytes(T, B, Nqk, Nv))
+
+
+def workspace_layout(T: int, B: int, Nqk: int, Nv: int) -> dict:
+    lay = _Layout()
+    _check(lib().gdn_workspace_layout(T, B, Nqk, Nv, ctypes.byref(lay)), "gdn_workspace_layout")
+    return {n: getattr(lay, n) for n, _ in _Layout._fields_}
+
+
+def _resolve(q, k, v, g, beta, cu_seqlens, state_pool, state_indices):
+    if q.dim() != 3 or v.dim() != 3:
+        raise ValueError("q/k must be [T, Nqk, 128] and v [T, Nv, 128]")
+    T, Nqk, Dk = q.shape
+    Nv = v.shape[1]
+    if Dk != HEAD_DIM or v.shape[2] != HEAD_DIM:
+        raise ValueError(f"head dimension must be {HEAD_DIM}")
+    if Nv % Nqk != 0:
+        raise ValueError(f"Nv ({Nv}) must be a multiple of Nqk ({Nqk})")
+    B = cu_seqlens.shape[0] - 1
+    dev = q.device
+    _need(q, "q", torch.bfloat16, (T, Nqk, HEAD_DIM), dev)
+    _need(k, "k", torch.bfloat16, (T, Nqk, HEAD_DIM), dev)
+    _need(v, "v", torch.bfloat16, (T, Nv, HEAD_DIM), dev)
+    _need(g, "g", torch.float32, (T, Nv), dev)
+    _need(beta, "beta", torch.bfloat16, (T, Nv), dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), dev)
+    P = 0
+    if state_pool is not None:
+        P = state_pool.shape[0]
+        _need(state_pool, "state_pool", torch.float32, (P, Nv, HEAD_DIM, HEAD_DIM), dev)
+    if state_indices is not None:
+        _need(state_indices, "state_indices", torch.int32, (B,), dev)
+    return T, B, Nqk, Nv, P, dev
+
+
+def chunk_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None, scale=None, eps=1e-6,
+              max_seqlen: int = 0, out=None, final_state=None, output_final_state=True, workspace=None,
+              stream=None):
+    """Gated Delta Rule forward through ``gdn_chunk_fwd``; returns (out, final_state).
+
+    q, k [T, Nqk, 128] bf16; v [T, Nv, 128] bf16; g [T, Nv] fp32; beta [T, Nv]
+    bf16; cu_seqlens [B+1] int32; state_pool [P, Nv, 128, 128] fp32 or None;
+    state_indices [B] int32 or None.  All on one CUDA device.  ``max_seqlen``
+    in 1..16 selects the fused short-sequence kernel."""
+    T, B, Nqk, Nv, P, dev = _resolve(q, k, v, g, beta, cu_seqlens, state_pool, state_indices)
+    if out is None:
+        out = torch.empty(T, Nv, HEAD_DIM, dtype=torch.bfloat16, device=dev)
+    else:
+        _need(out, "out", torch.bfloat16, (T, Nv, HEAD_DIM), dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(B, Nv, HEAD_DIM, HEAD_DIM, dtype=torch.float32, device=dev)
+    elif final_state is not None:
+        _need(final_state, "final_state", torch.float32, (B, Nv, HEAD_DIM, HEAD_DIM), dev)
+    short = 1 <= int(max_seqlen) <= SHORT_MAX
+    if workspace is None and not short and B > 0:
+        workspace = torch.empty(workspace_bytes(T, B, Nqk, Nv), dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    sc = 0.0 if scale is None else float(scale)
+    rc = lib().gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), _ptr(state_pool),
+                             _ptr(state_indices), sc, float(eps), _ptr(out), _ptr(final_state), T, B, Nqk, Nv, P,
+                             int(max_seqlen), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "gdn_chunk_fwd")
+    return out, final_state
+
+
+def short_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None, scale=None, eps=1e-6,
+              out=None, final_state=None, stream=None):
+    """The fused short-sequence kernel directly (``gdn_short_fwd``)."""
+    T, B, Nqk, Nv, P, dev = _resolve(q, k, v, g, beta, cu_seqlens, state_pool, state_indices)
+    if out is None:
+        out = torch.empty(T, Nv, HEAD_DIM, dtype=torch.bfloat16, device=dev)
+    if final_state is None:
+        final_state = torch.empty(B, Nv, HEAD_DIM, HEAD_DIM, dtype=torch.float32, device=dev)
+    sc = 0.0 if scale is None else float(scale)
+    rc = lib().gdn_short_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), _ptr(state_pool),
+                             _ptr(state_indices), sc, float(eps), _ptr(out), _ptr(final_state), T, B, Nqk, Nv, P,
+                             _stream(stream))
+    _check(rc, "gdn_short_fwd")
+    return out, final_state
+
+
+class Stages:
+    """The five kernels of the chunked path as separate calls on one workspace.
+
+    After ``run_all`` (or the individual calls in order) the intermediates are
+    readable through the typed views ``U``, ``W``, ``Up``, ``Sc``, ``qn``, ``kn``,
+    ``gcum``, ``betaf``, ``chunk_info`` and ``status`` (U, W, Up, Sc, qn, kn in fp16)."""
+
+    def __init__(self, T, B, Nqk, Nv, device):
+        self.T, self.B, self.Nqk, self.Nv = int(T), int(B), int(Nqk), int(Nv)
+        self.layout = workspace_layout(T, B, Nqk, Nv)
+        self.ws = torch.zeros(self.layout["total"], dtype=torch.uint8, device=device)
+        self.nbytes = self.layout["total"]
+        self.NC = int(self.layout["max_chunks"])
+
+    def _view(self, name, dtype, shape):
+        off = self.layout[name]
+        n = int(math.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
+        return self.ws[off:off + n].view(dtype).view(*shape)
+
+    @property
+    def U(self):
+        return self._view("U", torch.float16, (self.NC, self.Nv, CHUNK, HEAD_DIM))
+
+    @property
+    def W(self):
+        return self._view("W", torch.float16, (self.NC, self.Nv, CHUNK, HEAD_DIM))
+
+    @property
+    def Up(self):
+        return self._view("Up", torch.float16, (self.NC, self.Nv, CHUNK, HEAD_DIM))
+
+    @property
+    def Sc(self):
+        return self._view("Sc", torch.float16, (self.NC, self.Nv, HEAD_DIM, HEAD_DIM))
+
+    @property
+    def qn(self):
+        return self._view("qn", torch.float16, (self.T, self.Nqk, HEAD_DIM))
+
+    @property
+    def kn(self):
+        return self._view("kn", torch.float16, (self.T, self.Nqk, HEAD_DIM))
+
+    @property
+    def gcum(self):
+        return self._view("gcum", torch.float32, (self.Nv, self.T))
+
+    @property
+    def betaf(self):
+        return self._view("betaf", torch.float32, (self.Nv, self.T))
+
+    @property
+    def chunk_info(self):
+        return self._view("chunk_info", torch.int32, (self.NC, 4))
+
+    @property
+    def status(self):
+        return self._view("status", torch.int32, (4,))
+
+    def chunk_map(self, cu_seqlens, stream=None):
+        _check(lib().gdn_stage_chunk_map(_ptr(cu_seqlens), self.T, self.B, self.Nqk, self.Nv, _ptr(self.ws),
+                                         self.nbytes, _stream(stream)), "gdn_stage_chunk_map")
+
+    def prologue(self, q, k, g, beta, scale=None, eps=1e-6, stream=None):
+        sc = 0.0 if scale is None else float(scale)
+        _check(lib().gdn_stage_prologue(_ptr(q), _ptr(k), _ptr(g), _ptr(beta), sc, float(eps), self.T, self.B,
+                                        self.Nqk, self.Nv, _ptr(self.ws), self.nbytes, _stream(stream)),
+               "gdn_stage_prologue")
+
+    def intra(self, v, stream=None):
+        _check(lib().gdn_stage_intra(_ptr(v), self.T, self.B, self.Nqk, self.Nv, _ptr(self.ws), self.nbytes,
+                                     _stream(stream)), "gdn_stage_intra")
+
+    def state(self, state_pool=None, state_indices=None, final_state=None, stream=None):
+        P = 0 if state_pool is None else int(state_pool.shape[0])
+        _check(lib().gdn_stage_state(_ptr(state_pool), _ptr(state_indices), _ptr(final_state), self.T, self.B,
+                                     self.Nqk, self.Nv, P, _ptr(self.ws), self.nbytes, _stream(stream)),
+               "gdn_stage_state")
+
+    def output(self, out, stream=None):
+        _check(lib().gdn_stage_output(_ptr(out), self.T, self.B, self.Nqk, self.Nv, _ptr(self.ws), self.nbytes,
+                                      _stream(stream)), "gdn_stage_output")
+
+    def run_all(self, q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None, scale=None, eps=1e-6,
+                out=None, final_state=None, stream=None):
+        dev = q.device
+        if out is None:
+            out = torch.empty(self.T, self.Nv, HEAD_DIM, dtype=torch.bfloat16, device=dev)
+        if final_state is None:
+            final_state = torch.empty(self.B, self.Nv, HEAD_DIM, HEAD_DIM, dtype=torch.float32, device=dev)
+        self.chunk_map(cu_seqlens, stream)
+        self.prologue(q, k, g, beta, scale, eps, stream)
+        self.intra(v, stream)
+        self.state(state_pool, state_indices, final_state, stream)
+        self.output(out, stream)
+        return out, final_state
+
+
+def chunk_fwd_host(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None, scale=None, eps=1e-6,
+                   max_seqlen: int = 0, device="cuda", out_host=None, final_host=None, workspace=None):
+    """End-to-end call from host tensors: copies the inputs to the device,
+    runs ``gdn_chunk_fwd`` and copies out and final_state back (into the given
+    pinned host buffers when provided).  Returns (out, final_state, h2d_bytes, d2h_bytes)."""
+    host = [q, k, v, g, beta, cu_seqlens, state_pool, state_indices]
+    dev = [None if t is None else t.to(device, non_blocking=True) for t in host]
+    h2d = sum(t.numel() * t.element_size() for t in host if t is not None)
+    o, f = chunk_fwd(*dev, scale=scale, eps=eps, max_seqlen=max_seqlen, workspace=workspace)
+    if out_host is None:
+        out_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    if final_host is None:
+        final_host = torch.empty(f.shape, dtype=f.dtype, pin_memory=True)
+    out_host.copy_(o, non_blocking=True)
+    final_host.copy_(f, non_blocking=True)
+    d2h = o.numel() * o.element_size() + f.numel() * f.element_size()
+    return out_host, final_host, h2d, d2h

@@ -1,0 +1,162 @@
+// Device helpers shared by the Gated Delta Rule kernels (sm_100a).
+//
+// Shared-memory tiles of bf16 are stored with 16-byte chunks XOR-swizzled by
+// row, so that eight ldmatrix row addresses of one 8x8 matrix always land in
+// eight different bank groups:
+//   256-byte rows (128 bf16): chunk' = chunk ^ (row & 7)
+//    64-byte rows ( 32 bf16): chunk' = chunk ^ ((row >> 1) & 3)
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "gdn_internal.h"
+
+namespace gdn {
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------- swizzled tiles
+
+// byte offset of 16-byte chunk `c` of row `r` in a tile with 256-byte rows
+__device__ __forceinline__ uint32_t sw256(int r, int c) { return (r << 8) + ((c ^ (r & 7)) << 4); }
+// byte offset of 16-byte chunk `c` of row `r` in a tile with 64-byte rows
+__device__ __forceinline__ uint32_t sw64(int r, int c) { return (r << 6) + ((c ^ ((r >> 1) & 3)) << 4); }
+// byte offset of bf16 element (r, col) in those tiles
+__device__ __forceinline__ uint32_t el256(int r, int col) { return sw256(r, col >> 3) + ((col & 7) << 1); }
+__device__ __forceinline__ uint32_t el64(int r, int col) { return sw64(r, col >> 3) + ((col & 7) << 1); }
+
+// ---------------------------------------------------------------- async copies
+
+// 16-byte global->shared copy; when !valid the destination is zero-filled and
+// nothing is read (src must still be a mapped address, callers pass a base pointer)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid)
+{
+    const int n = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// ---------------------------------------------------------------- ldmatrix / mma
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                        uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                          uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// D += A(16x16, row) * B(16x8, col), fp16 inputs, fp32 accumulate
+__device__ __forceinline__ void mma16816(float *d, const uint32_t *a, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Lane addresses for ldmatrix.x4 on a 256-byte-row swizzled tile.
+//  A operand, tile holds A[m][k] (k contiguous): 16x16 block at (m0, k0)
+__device__ __forceinline__ uint32_t a_rowmajor_256(uint32_t base, int m0, int k0, int lane)
+{
+    const int r = m0 + (lane & 15);
+    const int c = (k0 >> 3) + (lane >> 4);
+    return base + sw256(r, c);
+}
+//  A operand, tile holds A^T[k][m] (m contiguous): 16x16 block at (m0, k0), use ldsm_x4_t
+__device__ __forceinline__ uint32_t a_colmajor_256(uint32_t base, int m0, int k0, int lane)
+{
+    const int mi = lane >> 3;
+    const int r = k0 + (lane & 7) + ((mi >> 1) << 3);
+    const int c = (m0 >> 3) + (mi & 1);
+    return base + sw256(r, c);
+}
+//  B operand, tile holds B^T[n][k] (k contiguous): n-tiles n0 and n0+8, k block k0; ldsm_x4
+//  gives {b0,b1} of n-tile n0 then {b0,b1} of n-tile n0+8
+__device__ __forceinline__ uint32_t b_nmajor_256(uint32_t base, int n0, int k0, int lane)
+{
+    const int r = n0 + (lane & 7) + ((lane >> 4) << 3);
+    const int c = (k0 >> 3) + ((lane >> 3) & 1);
+    return base + sw256(r, c);
+}
+//  B operand, tile holds B[k][n] (n contiguous): same fragment order, use ldsm_x4_t
+__device__ __forceinline__ uint32_t b_kmajor_256(uint32_t base, int n0, int k0, int lane)
+{
+    const int r = k0 + (lane & 7) + (((lane >> 3) & 1) << 3);
+    const int c = (n0 >> 3) + (lane >> 4);
+    return base + sw256(r, c);
+}
+//  B operand from a 64-byte-row tile B[k][n] (n contiguous, 32 columns), use ldsm_x4_t
+__device__ __forceinline__ uint32_t b_kmajor_64(uint32_t base, int n0, int k0, int lane)
+{
+    const int r = k0 + (lane & 7) + (((lane >> 3) & 1) << 3);
+    const int c = (n0 >> 3) + (lane >> 4);
+    return base + sw64(r, c);
+}
+
+// ---------------------------------------------------------------- conversions
+
+__device__ __forceinline__ float bf2f(uint16_t x) { return __uint_as_float(static_cast<uint32_t>(x) << 16); }
+__device__ __forceinline__ uint16_t f2bf(float x)
+{
+    __nv_bfloat16 h = __float2bfloat16_rn(x);
+    return *reinterpret_cast<uint16_t *>(&h);
+}
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi)
+{
+    return static_cast<uint32_t>(f2bf(lo)) | (static_cast<uint32_t>(f2bf(hi)) << 16);
+}
+// two floats -> packed fp16 pair (round to nearest even), low half first
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi)
+{
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ float2 unpack_h2(uint32_t x)
+{
+    return __half22float2(*reinterpret_cast<const __half2 *>(&x));
+}
+// packed bf16 pair -> packed fp16 pair (exact for magnitudes in fp16's normal range)
+__device__ __forceinline__ uint32_t bf2_to_h2(uint32_t x)
+{
+    return pack_h2(__uint_as_float(x << 16), __uint_as_float(x & 0xffff0000u));
+}
+
+__device__ __forceinline__ float warp_sum(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// chunk table row: sequence, first token, tokens, chunk index within the sequence
+struct ChunkInfo {
+    int seq, start, len, idx;
+};
+
+__device__ __forceinline__ ChunkInfo load_chunk(const int4 *info, int c)
+{
+    const int4 v = info[c];
+    return ChunkInfo{v.x, v.y, v.z, v.w};
+}
+
+}  // namespace gdn

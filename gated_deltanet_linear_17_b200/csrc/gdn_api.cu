@@ -1,0 +1,298 @@
+// Host side of the C ABI (include/gdn.h, include/gdn_stages.h): argument
+// checks, workspace layout and the launch sequence on the caller's stream.
+#include <math.h>
+#include <string.h>
+
+#include "gdn.h"
+#include "gdn_internal.h"
+#include "gdn_stages.h"
+
+using gdn::Workspace;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t max_chunks(int64_t T, int32_t B) { return (T + 127 * (int64_t)B) / gdn::L; }
+
+int fill_layout(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, gdn_workspace_layout_t *lay)
+{
+    if (T < 0 || B < 0 || Nqk <= 0 || Nv <= 0) return GDN_ERR_BAD_SHAPE;
+    const int64_t NC = max_chunks(T, B);
+    const size_t tile = (size_t)gdn::L * gdn::D * 2;
+    size_t off = 0;
+    lay->status = off;
+    off = align256(off + 16);
+    lay->chunk_info = off;
+    off = align256(off + (size_t)NC * 16);
+    lay->seq_chunk0 = off;
+    off = align256(off + (size_t)(B + 1) * 4);
+    lay->qn = off;
+    off = align256(off + (size_t)Nqk * T * gdn::D * 2);
+    lay->kn = off;
+    off = align256(off + (size_t)Nqk * T * gdn::D * 2);
+    lay->gcum = off;
+    off = align256(off + (size_t)Nv * T * 4);
+    lay->betaf = off;
+    off = align256(off + (size_t)Nv * T * 4);
+    lay->U = off;
+    off += (size_t)NC * Nv * tile;
+    lay->W = off;
+    off += (size_t)NC * Nv * tile;
+    lay->Up = off;
+    off += (size_t)NC * Nv * tile;
+    lay->Sc = off;
+    off += (size_t)NC * Nv * tile;
+    lay->total = align256(off);
+    lay->max_chunks = NC;
+    return GDN_OK;
+}
+
+Workspace views(void *base, const gdn_workspace_layout_t &lay)
+{
+    char *p = static_cast<char *>(base);
+    Workspace w;
+    w.status = reinterpret_cast<int32_t *>(p + lay.status);
+    w.chunk_info = reinterpret_cast<int4 *>(p + lay.chunk_info);
+    w.seq_chunk0 = reinterpret_cast<int32_t *>(p + lay.seq_chunk0);
+    w.qn = reinterpret_cast<uint16_t *>(p + lay.qn);
+    w.kn = reinterpret_cast<uint16_t *>(p + lay.kn);
+    w.gcum = reinterpret_cast<float *>(p + lay.gcum);
+    w.betaf = reinterpret_cast<float *>(p + lay.betaf);
+    w.U = reinterpret_cast<uint16_t *>(p + lay.U);
+    w.W = reinterpret_cast<uint16_t *>(p + lay.W);
+    w.Up = reinterpret_cast<uint16_t *>(p + lay.Up);
+    w.Sc = reinterpret_cast<uint16_t *>(p + lay.Sc);
+    w.NC = static_cast<int>(lay.max_chunks);
+    return w;
+}
+
+// sizes shared by every entry point
+int check_sizes(int64_t T, int32_t B, int32_t Nqk, int32_t Nv)
+{
+    if (T < 0 || B < 0 || Nqk <= 0 || Nv <= 0) return GDN_ERR_BAD_SHAPE;
+    if (Nv % Nqk != 0) return GDN_ERR_BAD_SHAPE;
+    if (T >= (int64_t(1) << 31) || Nqk > 64 || Nv > 256) return GDN_ERR_UNSUPPORTED;
+    if (max_chunks(T, B) >= (int64_t(1) << 31) / 256) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+int check_workspace(void *ws, size_t bytes, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
+                    gdn_workspace_layout_t *lay)
+{
+    int rc = fill_layout(T, B, Nqk, Nv, lay);
+    if (rc) return rc;
+    if (!ws) return GDN_ERR_NULL_ARG;
+    if (!aligned16(ws)) return GDN_ERR_ALIGNMENT;
+    if (bytes < lay->total) return GDN_ERR_WORKSPACE;
+    return GDN_OK;
+}
+
+bool overlap(const void *a, size_t na, const void *b, size_t nb)
+{
+    const char *x = static_cast<const char *>(a), *y = static_cast<const char *>(b);
+    return a && b && na && nb && x < y + nb && y < x + na;
+}
+
+float resolve_scale(float scale) { return scale > 0.f ? scale : 1.0f / sqrtf((float)gdn::D); }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+// arguments of the whole forward (shared by gdn_chunk_fwd and gdn_short_fwd)
+int check_forward(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                  const uint16_t *beta, const int32_t *cu, const float *pool, const int32_t *idx,
+                  const uint16_t *out, const float *final_state, int64_t T, int32_t B, int32_t Nqk,
+                  int32_t Nv, int32_t P)
+{
+    int rc = check_sizes(T, B, Nqk, Nv);
+    if (rc) return rc;
+    if (P < 0) return GDN_ERR_BAD_SHAPE;
+    if (B == 0) return GDN_OK;
+    if (!cu) return GDN_ERR_NULL_ARG;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !out)) return GDN_ERR_NULL_ARG;
+    if (pool && P == 0) return GDN_ERR_BAD_SHAPE;
+    if (pool && !idx && P < B) return GDN_ERR_BAD_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(pool) ||
+        !aligned16(final_state))
+        return GDN_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(g) & 3u) || (reinterpret_cast<uintptr_t>(beta) & 1u) ||
+        (reinterpret_cast<uintptr_t>(cu) & 3u) || (reinterpret_cast<uintptr_t>(idx) & 3u))
+        return GDN_ERR_ALIGNMENT;
+    const size_t sbytes = (size_t)gdn::D * gdn::D * 4 * Nv;
+    if (overlap(final_state, sbytes * B, pool, sbytes * P)) return GDN_ERR_OVERLAP;
+    const size_t obytes = (size_t)T * Nv * gdn::D * 2;
+    if (overlap(out, obytes, q, (size_t)T * Nqk * gdn::D * 2) ||
+        overlap(out, obytes, k, (size_t)T * Nqk * gdn::D * 2) || overlap(out, obytes, v, obytes))
+        return GDN_ERR_OVERLAP;
+    return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *gdn_status_string(int status)
+{
+    switch (status) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_NULL_ARG: return "GDN_ERR_NULL_ARG: a required pointer is NULL";
+    case GDN_ERR_BAD_SHAPE: return "GDN_ERR_BAD_SHAPE: invalid sizes";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: sizes beyond the supported limits";
+    case GDN_ERR_ALIGNMENT: return "GDN_ERR_ALIGNMENT: pointer not aligned";
+    case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE: workspace too small";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA: CUDA call failed";
+    case GDN_ERR_OVERLAP: return "GDN_ERR_OVERLAP: an output overlaps an input";
+    default: return "GDN_ERR_UNKNOWN";
+    }
+}
+
+int gdn_version(void) { return kVersion; }
+
+int gdn_workspace_layout(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, gdn_workspace_layout_t *layout)
+{
+    if (!layout) return GDN_ERR_NULL_ARG;
+    return fill_layout(T, B, Nqk, Nv, layout);
+}
+
+size_t gdn_chunk_fwd_workspace_bytes(int64_t T, int32_t B, int32_t Nqk, int32_t Nv)
+{
+    gdn_workspace_layout_t lay;
+    if (fill_layout(T, B, Nqk, Nv, &lay)) return 0;
+    return lay.total;
+}
+
+int gdn_stage_chunk_map(const int32_t *cu_seqlens, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
+                        void *workspace, size_t workspace_bytes, void *stream)
+{
+    int rc = check_sizes(T, B, Nqk, Nv);
+    if (rc) return rc;
+    gdn_workspace_layout_t lay;
+    if ((rc = check_workspace(workspace, workspace_bytes, T, B, Nqk, Nv, &lay))) return rc;
+    if (B == 0) return GDN_OK;
+    if (!cu_seqlens) return GDN_ERR_NULL_ARG;
+    const Workspace w = views(workspace, lay);
+    return cuda_status(gdn::launch_chunk_map(cu_seqlens, B, (int)T, w.NC, w, (cudaStream_t)stream));
+}
+
+int gdn_stage_prologue(const uint16_t *q, const uint16_t *k, const float *g, const uint16_t *beta,
+                       float scale, float eps, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
+                       void *workspace, size_t workspace_bytes, void *stream)
+{
+    int rc = check_sizes(T, B, Nqk, Nv);
+    if (rc) return rc;
+    gdn_workspace_layout_t lay;
+    if ((rc = check_workspace(workspace, workspace_bytes, T, B, Nqk, Nv, &lay))) return rc;
+    if (B == 0 || T == 0) return GDN_OK;
+    if (!q || !k || !g || !beta) return GDN_ERR_NULL_ARG;
+    if (!aligned16(q) || !aligned16(k)) return GDN_ERR_ALIGNMENT;
+    const Workspace w = views(workspace, lay);
+    return cuda_status(gdn::launch_prologue(q, k, g, beta, resolve_scale(scale), eps, (int)T, Nqk, Nv, w.NC,
+                                            w, (cudaStream_t)stream));
+}
+
+int gdn_stage_intra(const uint16_t *v, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, void *workspace,
+                    size_t workspace_bytes, void *stream)
+{
+    int rc = check_sizes(T, B, Nqk, Nv);
+    if (rc) return rc;
+    gdn_workspace_layout_t lay;
+    if ((rc = check_workspace(workspace, workspace_bytes, T, B, Nqk, Nv, &lay))) return rc;
+    if (B == 0 || T == 0) return GDN_OK;
+    if (!v) return GDN_ERR_NULL_ARG;
+    if (!aligned16(v)) return GDN_ERR_ALIGNMENT;
+    const Workspace w = views(workspace, lay);
+    return cuda_status(gdn::launch_intra(v, (int)T, Nqk, Nv, w.NC, w, (cudaStream_t)stream));
+}
+
+int gdn_stage_state(const float *state_pool, const int32_t *state_indices, float *final_state, int64_t T,
+                    int32_t B, int32_t Nqk, int32_t Nv, int32_t P, void *workspace, size_t workspace_bytes,
+                    void *stream)
+{
+    int rc = check_sizes(T, B, Nqk, Nv);
+    if (rc) return rc;
+    if (P < 0) return GDN_ERR_BAD_SHAPE;
+    gdn_workspace_layout_t lay;
+    if ((rc = check_workspace(workspace, workspace_bytes, T, B, Nqk, Nv, &lay))) return rc;
+    if (B == 0) return GDN_OK;
+    if (state_pool && P == 0) return GDN_ERR_BAD_SHAPE;
+    if (state_pool && !state_indices && P < B) return GDN_ERR_BAD_SHAPE;
+    if (!aligned16(state_pool) || !aligned16(final_state)) return GDN_ERR_ALIGNMENT;
+    const size_t sbytes = (size_t)gdn::D * gdn::D * 4 * Nv;
+    if (overlap(final_state, sbytes * B, state_pool, sbytes * P)) return GDN_ERR_OVERLAP;
+    const Workspace w = views(workspace, lay);
+    return cuda_status(gdn::launch_state(state_pool, state_indices, final_state, (int)T, B, Nqk, Nv, w,
+                                         (cudaStream_t)stream));
+}
+
+int gdn_stage_output(uint16_t *out, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, void *workspace,
+                     size_t workspace_bytes, void *stream)
+{
+    int rc = check_sizes(T, B, Nqk, Nv);
+    if (rc) return rc;
+    gdn_workspace_layout_t lay;
+    if ((rc = check_workspace(workspace, workspace_bytes, T, B, Nqk, Nv, &lay))) return rc;
+    if (B == 0 || T == 0) return GDN_OK;
+    if (!out) return GDN_ERR_NULL_ARG;
+    if (!aligned16(out)) return GDN_ERR_ALIGNMENT;
+    const Workspace w = views(workspace, lay);
+    return cuda_status(gdn::launch_output(out, (int)T, Nqk, Nv, w.NC, w, (cudaStream_t)stream));
+}
+
+int gdn_short_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                  const uint16_t *beta, const int32_t *cu_seqlens, const float *state_pool,
+                  const int32_t *state_indices, float scale, float eps, uint16_t *out,
+                  float *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
+                  void *stream)
+{
+    int rc = check_forward(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, out, final_state, T, B,
+                           Nqk, Nv, P);
+    if (rc || B == 0) return rc;
+    return cuda_status(gdn::launch_short(q, k, v, g, beta, cu_seqlens, state_pool, state_indices,
+                                         resolve_scale(scale), eps, out, final_state, (int)T, B, Nqk, Nv,
+                                         (cudaStream_t)stream));
+}
+
+int gdn_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                  const uint16_t *beta, const int32_t *cu_seqlens, const float *state_pool,
+                  const int32_t *state_indices, float scale, float eps, uint16_t *out,
+                  float *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
+                  int32_t max_seqlen, void *workspace, size_t workspace_bytes, void *stream)
+{
+    int rc = check_forward(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, out, final_state, T, B,
+                           Nqk, Nv, P);
+    if (rc || B == 0) return rc;
+    const cudaStream_t st = (cudaStream_t)stream;
+    const float sc = resolve_scale(scale);
+    if (max_seqlen >= 1 && max_seqlen <= GDN_SHORT_MAX)
+        return cuda_status(gdn::launch_short(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, sc, eps,
+                                             out, final_state, (int)T, B, Nqk, Nv, st));
+
+    gdn_workspace_layout_t lay;
+    if ((rc = fill_layout(T, B, Nqk, Nv, &lay))) return rc;
+    bool owned = false;
+    if (!workspace) {
+        if (cudaMallocAsync(&workspace, lay.total, st) != cudaSuccess) return GDN_ERR_CUDA;
+        owned = true;
+    } else {
+        if (!aligned16(workspace)) return GDN_ERR_ALIGNMENT;
+        if (workspace_bytes < lay.total) return GDN_ERR_WORKSPACE;
+    }
+    const Workspace w = views(workspace, lay);
+    const int Ti = (int)T;
+    cudaError_t e = gdn::launch_chunk_map(cu_seqlens, B, Ti, w.NC, w, st);
+    if (e == cudaSuccess) e = gdn::launch_prologue(q, k, g, beta, sc, eps, Ti, Nqk, Nv, w.NC, w, st);
+    if (e == cudaSuccess) e = gdn::launch_intra(v, Ti, Nqk, Nv, w.NC, w, st);
+    if (e == cudaSuccess) e = gdn::launch_state(state_pool, state_indices, final_state, Ti, B, Nqk, Nv, w, st);
+    if (e == cudaSuccess) e = gdn::launch_output(out, Ti, Nqk, Nv, w.NC, w, st);
+    if (owned) {
+        cudaError_t f = cudaFreeAsync(workspace, st);
+        if (e == cudaSuccess) e = f;
+    }
+    return cuda_status(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,39 @@
+// Internal declarations shared by the host API and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gdn {
+
+constexpr int L = 128;  // chunk length
+constexpr int D = 128;  // head dimension (Dk = Dv)
+
+// Typed views of the workspace regions (layout: gdn_workspace_layout in gdn_stages.h)
+struct Workspace {
+    int32_t *status;
+    int4 *chunk_info;
+    int32_t *seq_chunk0;
+    uint16_t *qn, *kn;  // fp16 [T][Nqk][128]: scale * q / |q|, k / |k|
+    float *gcum, *betaf;
+    uint16_t *U, *W, *Up, *Sc;
+    int NC;  // max chunks
+};
+
+cudaError_t launch_chunk_map(const int32_t *cu, int B, int T, int NC, const Workspace &ws,
+                             cudaStream_t st);
+cudaError_t launch_prologue(const uint16_t *q, const uint16_t *k, const float *g, const uint16_t *beta,
+                            float scale, float eps, int T, int Nqk, int Nv, int NC, const Workspace &ws,
+                            cudaStream_t st);
+cudaError_t launch_intra(const uint16_t *v, int T, int Nqk, int Nv, int NC, const Workspace &ws,
+                         cudaStream_t st);
+cudaError_t launch_state(const float *pool, const int32_t *idx, float *final_state, int T, int B, int Nqk,
+                         int Nv, const Workspace &ws, cudaStream_t st);
+cudaError_t launch_output(uint16_t *out, int T, int Nqk, int Nv, int NC, const Workspace &ws, cudaStream_t st);
+cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                         const uint16_t *beta, const int32_t *cu, const float *pool, const int32_t *idx,
+                         float scale, float eps, uint16_t *out, float *final_state, int T, int B, int Nqk,
+                         int Nv, cudaStream_t st);
+
+}  // namespace gdn

@@ -1,0 +1,121 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) Gated Delta Rule chunked forward.
+ *
+ * The operator is the chunked Gated Delta Rule forward of the page
+ * "Qwen3Next Samples" (chunk_gated_delta_rule: "Function Prototype",
+ * "Parameter Description", "Mathematical Formulas"): q/k L2 normalisation,
+ * per-chunk gate cumulative sum, decay mask, pre-attention matrix, the
+ * unit-lower-triangular inverse, value/key cumulative decay, recurrent state
+ * attention and the state update, over a packed batch of variable-length
+ * sequences.  It computes exactly (up to rounding) the token recurrence of the
+ * page "lite_boost.ops.recurrent_gated_delta_rule" (algorithm flow):
+ *
+ *     S = exp(g_t) S;  kv = S^T kh_t;  S += kh_t (beta_t (v_t - kv))^T;  o_t = S^T qh_t
+ *
+ * with kh = k / sqrt(|k|^2 + eps), qh = scale * q / sqrt(|q|^2 + eps), per
+ * sequence and v-head, v-head h reading qk-head h / (Nv / Nqk).  The initial
+ * state comes from a slot pool as on the decode page (state, ssm_state_indices)
+ * with one slot per sequence.
+ *
+ * Fixed sizes: head dimension Dk = Dv = 128 and chunk length L = 128 (both
+ * fixed on the "Qwen3Next Samples" page, "Parameter Description/Constraints").
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named "device" are device memory owned by the caller; the
+ *     library keeps no pointer after a call returns.  All tensors are dense,
+ *     row-major, contiguous.
+ *   - bf16 tensors are passed as uint16_t* holding the raw bfloat16 bits.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call only enqueues work on `stream` and returns; it never synchronises.
+ *     Argument errors are returned before anything is enqueued.  A launch
+ *     failure returns GDN_ERR_CUDA; a fault inside a kernel surfaces at the
+ *     caller's next synchronisation, as with any CUDA launch.
+ *   - Values are not validated on the device: gates are expected <= 0 and
+ *     beta in [0, 1] (the decode page leaves both unchecked on purpose, since
+ *     a reduction over the inputs would cost a pass on the inference path);
+ *     state_indices must lie in [0, P).
+ *   - Return value: a gdn_status_t code (0 = success).
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDN_HEAD_DIM 128 /* Dk = Dv */
+#define GDN_CHUNK 128    /* L */
+#define GDN_SHORT_MAX 16 /* max_seqlen at or below which the fused short-sequence kernel runs */
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_NULL_ARG = 1,    /* a required pointer is NULL                              */
+    GDN_ERR_BAD_SHAPE = 2,   /* negative size, Nv not a multiple of Nqk, P < B without indices */
+    GDN_ERR_UNSUPPORTED = 3, /* size beyond what the kernels handle (see each entry)     */
+    GDN_ERR_ALIGNMENT = 4,   /* a pointer breaks the 16-byte alignment rule              */
+    GDN_ERR_WORKSPACE = 5,   /* caller workspace smaller than gdn_chunk_fwd_workspace_bytes */
+    GDN_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed                     */
+    GDN_ERR_OVERLAP = 7      /* an output buffer overlaps an input buffer                */
+} gdn_status_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *gdn_status_string(int status);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int gdn_version(void);
+
+/*
+ * Bytes of device workspace that the chunked path of gdn_chunk_fwd needs for
+ * these sizes (the fused short-sequence path needs none).  The workspace holds
+ * the per-chunk intermediates of the chunked form: the chunk table, inverse
+ * norms, cumulative gates, U, W, U' and the chunk-entry states; its layout is
+ * given by gdn_workspace_layout (gdn_stages.h).
+ */
+size_t gdn_chunk_fwd_workspace_bytes(int64_t T, int32_t B, int32_t Nqk, int32_t Nv);
+
+/*
+ * gdn_chunk_fwd -- the whole forward pass.
+ *
+ *   q, k          device bf16 [T, Nqk, 128]   queries / keys (normalised in the op)
+ *   v             device bf16 [T, Nv, 128]
+ *   g             device fp32 [T, Nv]         log-space gate per token and v-head
+ *   beta          device bf16 [T, Nv]
+ *   cu_seqlens    device int32 [B+1]          cu[0] = 0, non-decreasing, cu[B] = T;
+ *                                             sequence b holds tokens cu[b] .. cu[b+1]-1
+ *   state_pool    device fp32 [P, Nv, 128 (Dk), 128 (Dv)], or NULL for zero initial states
+ *   state_indices device int32 [B]            slot of each sequence in state_pool, or
+ *                                             NULL for slot b (then P >= B is required)
+ *   scale         query scale; <= 0 selects 1/sqrt(128)
+ *   eps           L2-norm epsilon (inside the square root; 1e-6 on the prefill page)
+ *   out           device bf16 [T, Nv, 128]    written for every token
+ *   final_state   device fp32 [B, Nv, 128 (Dk), 128 (Dv)], or NULL (not written);
+ *                 must not overlap state_pool
+ *   T, B, Nqk, Nv, P   sizes (T = cu[B]); Nv % Nqk == 0
+ *   max_seqlen    longest sequence if known, else 0.  A value in 1..GDN_SHORT_MAX
+ *                 selects the fused short-sequence kernel (token recurrence on
+ *                 the state held on chip); any other value selects the chunked
+ *                 kernels.  Both paths are correct for any lengths; the hint
+ *                 only chooses the faster one.
+ *   workspace     device buffer of workspace_bytes >= gdn_chunk_fwd_workspace_bytes,
+ *                 or NULL: the call then allocates and frees it stream-ordered
+ *                 (cudaMallocAsync / cudaFreeAsync on `stream`).
+ *
+ * Alignment: q, k, v, out, state_pool, final_state and workspace 16-byte aligned.
+ * Limits: T < 2^31, Nqk <= 64, Nv <= 256 (else GDN_ERR_UNSUPPORTED).
+ * B == 0 is a no-op.  A sequence of length 0 writes no output and copies its
+ * initial state to final_state.
+ */
+int gdn_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                  const uint16_t *beta, const int32_t *cu_seqlens, const float *state_pool,
+                  const int32_t *state_indices, float scale, float eps, uint16_t *out,
+                  float *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
+                  int32_t max_seqlen, void *workspace, size_t workspace_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

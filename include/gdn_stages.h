@@ -1,0 +1,150 @@
+/*
+ * gdn_stages.h -- the kernels of gdn_chunk_fwd as separate C-ABI calls.
+ *
+ * gdn_chunk_fwd (gdn.h) is exactly gdn_stage_chunk_map, gdn_stage_prologue,
+ * gdn_stage_intra, gdn_stage_state and gdn_stage_output enqueued in that order
+ * on one stream with one workspace.  The stages are exposed so that each
+ * kernel can be checked against the chunked form's intermediates and timed on
+ * its own.  Conventions (device pointers, bf16 as uint16_t bits, asynchronous
+ * on `stream`, status codes, alignment) are those of gdn.h.  Every stage takes
+ * the sizes (T, B, Nqk, Nv) and the workspace that the chunk map was built
+ * with; a stage reads the workspace regions that earlier stages wrote.
+ *
+ * Notation (page "Qwen3Next Samples", "Mathematical Formulas"; the state is
+ * held as S[Dk, Dv] as on the decode page): per chunk of L = 128 tokens of one
+ * sequence and v-head, gamma = chunk-local cumulative gate, Gamma_ij =
+ * exp(gamma_i - gamma_j), kh/qh the normalised keys/queries, beta the update
+ * rates.  A_ij = beta_i (kh_i . kh_j) Gamma_ij for j < i (the page's A with
+ * its negative mask is -A); T = (I + A)^-1; U = T diag(beta) V;
+ * W = T diag(beta e^gamma) Kh; S_c is the state entering chunk c;
+ * U' = U - W S_c; S_{c+1} = e^{gamma_last} S_c + (Kh * e^{gamma_last - gamma})^T U';
+ * o = diag(e^gamma) Qh S_c + (Qh Kh^T * Gamma * tril) U'.
+ */
+#ifndef GDN_STAGES_H_
+#define GDN_STAGES_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "gdn.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * Byte offsets of the workspace regions (each 256-byte aligned) for given
+ * sizes.  NC = max_chunks = floor((T + 127 B) / 128), an upper bound on the
+ * number of chunks of any packing of T tokens into B sequences.
+ *   status      int32[4]: [0] cu_seqlens error bits (1: cu[0] != 0, 2: decreasing,
+ *               4: cu[B] != T), [1] number of chunks
+ *   chunk_info  int32[NC][4]: sequence, first token, tokens in the chunk (1..128),
+ *               chunk index within its sequence; rows past the last chunk hold -1
+ *   seq_chunk0  int32[B+1]: first chunk of each sequence, [B] = number of chunks
+ *   qn          fp16 [T][Nqk][128]: scale * q / sqrt(|q|^2 + eps)
+ *   kn          fp16 [T][Nqk][128]: k / sqrt(|k|^2 + eps)
+ *   gcum        fp32 [Nv][T]: chunk-local cumulative gate gamma
+ *   betaf       fp32 [Nv][T]: beta widened to fp32
+ *   U, W, Up    fp16 [NC][Nv][128 (L)][128]: U, W (columns Dk) and U' of each chunk
+ *   Sc          fp16 [NC][Nv][128 (Dk)][128 (Dv)]: state entering each chunk
+ * The tensor-core products take fp16 operands (11-bit significand) with fp32
+ * accumulation; fp16 holds the normalised q and k exactly enough and keeps
+ * the max-abs error of the pass well inside the tolerance, where bf16
+ * operands did not.  Values derived from v (U, U', S) must stay below 65504 in
+ * magnitude.
+ */
+typedef struct {
+    size_t total;
+    size_t status;
+    size_t chunk_info;
+    size_t seq_chunk0;
+    size_t qn;
+    size_t kn;
+    size_t gcum;
+    size_t betaf;
+    size_t U;
+    size_t W;
+    size_t Up;
+    size_t Sc;
+    int64_t max_chunks;
+} gdn_workspace_layout_t;
+
+/* Fill *layout for these sizes; GDN_ERR_BAD_SHAPE on negative sizes. */
+int gdn_workspace_layout(int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
+                         gdn_workspace_layout_t *layout);
+
+/*
+ * Chunk table from cu_seqlens (device int32 [B+1]): splits every sequence
+ * into chunks of 128 tokens starting at its first token, the last chunk taking
+ * the remainder ("Qwen3Next Samples": L = 128, act_seq_len).  Token ranges
+ * are clamped to [0, T) so that a malformed cu_seqlens can never make a later
+ * stage read or write out of bounds; the error bits in status say why.
+ */
+int gdn_stage_chunk_map(const int32_t *cu_seqlens, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Prologue: per token and qk-head the L2-normalised q (times scale) and k
+ * ("L2 Normalization", eps inside the square root) in fp16, per chunk and
+ * v-head the cumulative gate ("Gate Cumulative Sum") restarting at every chunk
+ * start, and beta widened to fp32.  Reads q, k [T, Nqk, 128] bf16, g [T, Nv]
+ * fp32, beta [T, Nv] bf16; writes qn, kn, gcum, betaf.  scale <= 0 selects
+ * 1/sqrt(128).
+ */
+int gdn_stage_prologue(const uint16_t *q, const uint16_t *k, const float *g, const uint16_t *beta,
+                       float scale, float eps, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Intra-chunk: per (chunk, v-head) forms A ("Pre-Attention Matrix"), solves
+ * T = (I + A)^-1 by blocked forward substitution ("Matrix Inversion" with the
+ * block merge of inverse_pto / inverse_matmul), and computes U and W ("Value
+ * and Key Cumulative Decay").  Reads v [T, Nv, 128] bf16 and the prologue's
+ * outputs; writes U, W.
+ */
+int gdn_stage_intra(const uint16_t *v, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, void *workspace,
+                    size_t workspace_bytes, void *stream);
+
+/*
+ * Inter-chunk state passing: per (sequence, v-head, 32-column slice of Dv),
+ * serially over the sequence's chunks, U' = U - W S and
+ * S <- e^{gamma_last} S + (Kh * e^{gamma_last - gamma})^T U' ("Recurrent State
+ * Attention" v', "State Update" with k_gexp), the state kept in fp32 on chip.
+ * S starts from state_pool[state_indices[b]] (or slot b, or zero without a
+ * pool).  Reads kn, gcum, U, W; writes Sc and Up for every chunk and
+ * final_state (if not NULL).
+ */
+int gdn_stage_state(const float *state_pool, const int32_t *state_indices, float *final_state, int64_t T,
+                    int32_t B, int32_t Nqk, int32_t Nv, int32_t P, void *workspace, size_t workspace_bytes,
+                    void *stream);
+
+/*
+ * Output: per (chunk, v-head) o = diag(e^gamma) Qh S_c + (Qh Kh^T * Gamma * tril) U'
+ * ("Recurrent State Attention": o_inter and o_chunk; tril includes the
+ * diagonal).  Reads qn, kn, gcum, Sc, Up; writes out [T, Nv, 128] bf16 for
+ * every token of every chunk.
+ */
+int gdn_stage_output(uint16_t *out, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, void *workspace,
+                     size_t workspace_bytes, void *stream);
+
+/*
+ * Fused short-sequence forward: the token recurrence of the decode page
+ * ("lite_boost.ops.recurrent_gated_delta_rule", algorithm flow, for up to 8
+ * tokens per call there) run with each (sequence, v-head, 32-column slice)
+ * state held in registers: one pass reads the initial state from the pool,
+ * applies the sequence's tokens and writes out and final_state.  Correct for
+ * any length (cost grows linearly with it); gdn_chunk_fwd routes here when
+ * 1 <= max_seqlen <= GDN_SHORT_MAX.  Same arguments as gdn_chunk_fwd without
+ * the workspace.
+ */
+int gdn_short_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                  const uint16_t *beta, const int32_t *cu_seqlens, const float *state_pool,
+                  const int32_t *state_indices, float scale, float eps, uint16_t *out,
+                  float *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
+                  void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_STAGES_H_ */

@@ -127,6 +127,8 @@ def chunked(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None, s
                 qn = scale * l2norm(q[c0:c1, hq], eps)
                 kn = l2norm(k[c0:c1, hq], eps)
                 r = chunk_intermediates(qn, kn, v[c0:c1, h], g[c0:c1, h], beta[c0:c1, h], S)
+                if keep:
+                    r["qn"], r["kn"] = qn, kn
                 out[c0:c1, slot] = r["o"]
                 S = r["S_new"]
                 if keep:

@@ -1,0 +1,119 @@
+"""The C-ABI library loads, exports every symbol its headers declare, and
+rejects bad arguments before touching a GPU (CPU only: no call here enqueues work)."""
+from __future__ import annotations
+
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import gated_deltanet_linear_17_b200 as gdn
+from gated_deltanet_linear_17_b200 import _binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        for m in re.finditer(r"\b(gdn_[a-z0-9_]+)\s*\(", text):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(B.LIB_PATH):
+        pytest.skip("libgdn.so not built")
+    return gdn.lib()
+
+
+def test_headers_declare_entry_points():
+    names = _declared()
+    for n in ("gdn_chunk_fwd", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string", "gdn_short_fwd",
+              "gdn_stage_intra", "gdn_stage_state", "gdn_stage_output", "gdn_stage_prologue"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, f"declared but not exported: {missing}"
+
+
+def test_status_strings(lib):
+    for code in range(0, 8):
+        assert gdn.status_string(code).startswith("GDN_")
+    assert "UNKNOWN" in gdn.status_string(99)
+
+
+def test_workspace_layout_regions_disjoint_and_aligned(lib):
+    lay = gdn.workspace_layout(4048, 4, 4, 8)
+    assert lay["max_chunks"] == (4048 + 127 * 4) // 128
+    regions = ["status", "chunk_info", "seq_chunk0", "qn", "kn", "gcum", "betaf", "U", "W", "Up", "Sc"]
+    offs = [lay[r] for r in regions]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    tile = 128 * 128 * 2
+    assert lay["W"] - lay["U"] == lay["max_chunks"] * 8 * tile
+    assert lay["total"] >= lay["Sc"] + lay["max_chunks"] * 8 * tile
+    assert gdn.workspace_bytes(4048, 4, 4, 8) == lay["total"]
+
+
+def test_max_chunks_is_an_upper_bound():
+    # floor((T + 127 B) / 128) >= sum(ceil(len / 128)) for every packing
+    import random
+    r = random.Random(0)
+    for _ in range(2000):
+        Bn = r.randint(1, 12)
+        lens = [r.choice([0, 1, 127, 128, 129, r.randint(0, 700)]) for _ in range(Bn)]
+        T = sum(lens)
+        assert sum((n + 127) // 128 for n in lens) <= (T + 127 * Bn) // 128
+
+
+def _call(lib, **over):
+    M = 1 << 20  # fake, disjoint, 16-byte aligned addresses (never dereferenced)
+    a = dict(q=1 * M, k=2 * M, v=3 * M, g=4 * M, beta=5 * M, cu=6 * M, pool=None, idx=None, scale=0.0,
+             eps=1e-6, out=7 * M, fin=None, T=8, B=1, Nqk=2, Nv=4, P=0, max_seqlen=0, ws=None, wsb=0,
+             stream=None)
+    a.update(over)
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.gdn_chunk_fwd(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["g"]), vp(a["beta"]), vp(a["cu"]),
+                             vp(a["pool"]), vp(a["idx"]), a["scale"], a["eps"], vp(a["out"]), vp(a["fin"]),
+                             a["T"], a["B"], a["Nqk"], a["Nv"], a["P"], a["max_seqlen"], vp(a["ws"]), a["wsb"],
+                             vp(a["stream"]))
+
+
+def test_argument_errors_before_any_launch(lib):
+    # These return before any CUDA call (the fake addresses are never dereferenced).
+    assert _call(lib, Nv=3) == B.GDN_ERR_BAD_SHAPE            # Nv not a multiple of Nqk
+    assert _call(lib, T=-1) == B.GDN_ERR_BAD_SHAPE
+    assert _call(lib, Nqk=0) == B.GDN_ERR_BAD_SHAPE
+    assert _call(lib, P=-1) == B.GDN_ERR_BAD_SHAPE
+    assert _call(lib, q=None) == B.GDN_ERR_NULL_ARG
+    assert _call(lib, cu=None) == B.GDN_ERR_NULL_ARG
+    assert _call(lib, q=(1 << 20) + 8) == B.GDN_ERR_ALIGNMENT  # not 16-byte aligned
+    assert _call(lib, out=3 << 20) == B.GDN_ERR_OVERLAP           # out aliases v
+    assert _call(lib, pool=9 << 20, P=1, B=2) == B.GDN_ERR_BAD_SHAPE   # P < B without indices
+    assert _call(lib, pool=9 << 20, P=1, fin=9 << 20) == B.GDN_ERR_OVERLAP
+    assert _call(lib, Nqk=128, Nv=128) == B.GDN_ERR_UNSUPPORTED
+    assert _call(lib, T=1 << 31) == B.GDN_ERR_UNSUPPORTED
+    assert _call(lib, B=0) == B.GDN_OK                        # empty batch: nothing to do
+    assert _call(lib, ws=8 << 20, wsb=10) == B.GDN_ERR_WORKSPACE  # caller workspace too small
+    assert _call(lib, ws=(8 << 20) + 4, wsb=1 << 40) == B.GDN_ERR_ALIGNMENT
+
+
+def test_stage_argument_errors(lib):
+    vp = ctypes.c_void_p
+    assert lib.gdn_stage_intra(vp(16), 8, 1, 2, 4, None, 0, None) == B.GDN_ERR_NULL_ARG
+    assert lib.gdn_stage_intra(vp(16), 8, 1, 2, 4, vp(16), 10, None) == B.GDN_ERR_WORKSPACE
+    assert lib.gdn_stage_output(vp(16), 8, 1, 2, 3, vp(16), 1 << 30, None) == B.GDN_ERR_BAD_SHAPE
+
+
+def test_python_layer_refuses_cpu_tensors():
+    import torch
+    from gated_deltanet_linear_17_b200 import inputs
+    inp = inputs.make([5], 1, 2, seed=0)
+    with pytest.raises(RuntimeError):
+        gdn.chunk_fwd(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens)
