@@ -189,6 +189,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-short", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="override the prefill length (profiling on a smaller case; not a bench line)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -202,7 +204,13 @@ def main():
     dev = torch.device("cuda", local)
     peaks = load_peaks()
 
-    host = inputs.config(WORKLOAD, seed=inputs.CONFIGS[WORKLOAD]["seed"] + rank)
+    if args.seq_len:
+        rec = dict(inputs.CONFIGS[WORKLOAD])
+        rec["lens"] = [args.seq_len]
+        rec["seed"] += rank
+        host = inputs.make(name=f"{WORKLOAD}@{args.seq_len}", **rec)
+    else:
+        host = inputs.config(WORKLOAD, seed=inputs.CONFIGS[WORKLOAD]["seed"] + rank)
     inp = host.to(dev)
     T, B, Nqk, Nv = inp.T, inp.B, inp.Nqk, inp.Nv
     st = gdn.Stages(T, B, Nqk, Nv, dev)
