@@ -22,6 +22,8 @@ SHORT_MAX = 16
 
 GDN_OK, GDN_ERR_NULL_ARG, GDN_ERR_BAD_SHAPE, GDN_ERR_UNSUPPORTED = 0, 1, 2, 3
 GDN_ERR_ALIGNMENT, GDN_ERR_WORKSPACE, GDN_ERR_CUDA, GDN_ERR_OVERLAP = 4, 5, 6, 7
+GDN_ERR_SCRATCH_LIMIT = 8
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
 
@@ -49,6 +51,8 @@ def lib():
         L.gdn_workspace_layout.argtypes = [i64, i32, i32, i32, ctypes.POINTER(_Layout)]
         L.gdn_chunk_fwd.restype = ctypes.c_int
         L.gdn_chunk_fwd.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, i32, p, sz, p]
+        L.gdn_chunk_fwd_noalloc.restype = ctypes.c_int
+        L.gdn_chunk_fwd_noalloc.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, i32, p]
         L.gdn_short_fwd.restype = ctypes.c_int
         L.gdn_short_fwd.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, p]
         L.gdn_stage_chunk_map.restype = ctypes.c_int
@@ -74,7 +78,7 @@ def _check(code: int, what: str):
         return
     msg = f"{what}: {status_string(code)}"
     if code in (GDN_ERR_BAD_SHAPE, GDN_ERR_UNSUPPORTED, GDN_ERR_NULL_ARG, GDN_ERR_OVERLAP, GDN_ERR_WORKSPACE,
-                GDN_ERR_ALIGNMENT):
+                GDN_ERR_ALIGNMENT, GDN_ERR_SCRATCH_LIMIT):
         raise ValueError(msg)
     raise RuntimeError(msg)
 
@@ -166,6 +170,27 @@ def chunk_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None,
                              _ptr(state_indices), sc, float(eps), _ptr(out), _ptr(final_state), T, B, Nqk, Nv, P,
                              int(max_seqlen), _ptr(workspace), ws_bytes, _stream(stream))
     _check(rc, "gdn_chunk_fwd")
+    return out, final_state
+
+
+def chunk_fwd_noalloc(q, k, v, g, beta, cu_seqlens, out, final_state=None, state_pool=None, state_indices=None,
+                      scale=None, eps=1e-6, max_seqlen: int = 0, stream=None):
+    """``gdn_chunk_fwd_noalloc``: the forward pass with no device allocation at all.
+
+    For callers that may not allocate device memory: the caller passes every
+    input and output (``out``, and ``final_state`` or None), and the library
+    runs on its static per-GPU scratch (64 MiB); sizes that need more raise
+    ValueError (GDN_ERR_SCRATCH_LIMIT).  Calls that may overlap on the GPU
+    share that scratch and must be ordered on one stream."""
+    T, B, Nqk, Nv, P, dev = _resolve(q, k, v, g, beta, cu_seqlens, state_pool, state_indices)
+    _need(out, "out", torch.bfloat16, (T, Nv, HEAD_DIM), dev)
+    if final_state is not None:
+        _need(final_state, "final_state", torch.float32, (B, Nv, HEAD_DIM, HEAD_DIM), dev)
+    sc = 0.0 if scale is None else float(scale)
+    rc = lib().gdn_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+                                     _ptr(state_pool), _ptr(state_indices), sc, float(eps), _ptr(out),
+                                     _ptr(final_state), T, B, Nqk, Nv, P, int(max_seqlen), _stream(stream))
+    _check(rc, "gdn_chunk_fwd_noalloc")
     return out, final_state
 
 

@@ -146,6 +146,8 @@ const char *gdn_status_string(int status)
     case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE: workspace too small";
     case GDN_ERR_CUDA: return "GDN_ERR_CUDA: CUDA call failed";
     case GDN_ERR_OVERLAP: return "GDN_ERR_OVERLAP: an output overlaps an input";
+    case GDN_ERR_SCRATCH_LIMIT:
+        return "GDN_ERR_SCRATCH_LIMIT: these sizes need more workspace than the library's static scratch";
     default: return "GDN_ERR_UNKNOWN";
     }
 }

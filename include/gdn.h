@@ -49,6 +49,7 @@ extern "C" {
 #define GDN_HEAD_DIM 128 /* Dk = Dv */
 #define GDN_CHUNK 128    /* L */
 #define GDN_SHORT_MAX 16 /* max_seqlen at or below which the fused short-sequence kernel runs */
+#define GDN_NOALLOC_SCRATCH_BYTES (64u << 20) /* static workspace of gdn_chunk_fwd_noalloc, per GPU */
 
 typedef enum {
     GDN_OK = 0,
@@ -58,7 +59,9 @@ typedef enum {
     GDN_ERR_ALIGNMENT = 4,   /* a pointer breaks the 16-byte alignment rule              */
     GDN_ERR_WORKSPACE = 5,   /* caller workspace smaller than gdn_chunk_fwd_workspace_bytes */
     GDN_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed                     */
-    GDN_ERR_OVERLAP = 7      /* an output buffer overlaps an input buffer                */
+    GDN_ERR_OVERLAP = 7,     /* an output buffer overlaps an input buffer                */
+    GDN_ERR_SCRATCH_LIMIT = 8 /* gdn_chunk_fwd_noalloc: the sizes need more workspace than
+                                 GDN_NOALLOC_SCRATCH_BYTES                                 */
 } gdn_status_t;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -113,6 +116,42 @@ int gdn_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
                   const int32_t *state_indices, float scale, float eps, uint16_t *out,
                   float *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
                   int32_t max_seqlen, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd for callers that cannot allocate
+ * device memory.  The pages have no counterpart of this call.
+ *
+ * Some callers cannot call cudaMalloc or cudaMallocAsync and cannot hand over
+ * a workspace either: code running inside a host framework that owns every
+ * byte of device memory and forbids allocation while it executes (an inference
+ * engine's plugin or custom-op enqueue, a serving runtime that reserved the
+ * whole GPU for its state pools up front), or an interface with no place for a
+ * workspace argument.  This call takes the same arguments as gdn_chunk_fwd
+ * without the workspace and allocates nothing: the chunked path runs on a
+ * static device buffer of GDN_NOALLOC_SCRATCH_BYTES (64 MiB) inside this
+ * library.  Every GPU on which the library's code is loaded holds one such
+ * buffer until the process exits.
+ *
+ * Limit: sizes whose chunked-path workspace (gdn_chunk_fwd_workspace_bytes)
+ * exceeds 64 MiB are rejected with GDN_ERR_SCRATCH_LIMIT before anything is
+ * enqueued (at Nqk = 16, Nv = 32 that is about 1500 tokens in one sequence).
+ * The fused short-sequence path (1 <= max_seqlen <= GDN_SHORT_MAX) uses no
+ * workspace and has no such limit.
+ *
+ * The buffer used is the one of the calling thread's current device; `stream`
+ * must belong to that device.  The first call on a device looks up the
+ * buffer's device address (cudaGetSymbolAddress) and keeps it; make that first
+ * call before any stream capture.  All calls on one device share the buffer,
+ * which keeps whatever the previous call left in it (no call depends on it
+ * starting at zero): calls that can overlap on the GPU (unordered streams,
+ * several host threads) race on it and corrupt each other's results, so
+ * order them on one stream.
+ */
+int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                          const uint16_t *beta, const int32_t *cu_seqlens, const float *state_pool,
+                          const int32_t *state_indices, float scale, float eps, uint16_t *out,
+                          float *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
+                          int32_t max_seqlen, void *stream);
 
 #ifdef __cplusplus
 }

@@ -44,7 +44,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in range(0, 8):
+    for code in range(0, 9):
         assert gdn.status_string(code).startswith("GDN_")
     assert "UNKNOWN" in gdn.status_string(99)
 
