@@ -50,8 +50,8 @@ def stage_work(T, Nqk, Nv):
     """Algorithmic work of one launch of each stage: (bound, amount, unit)."""
     return {
         "chunk_map": ("hbm", 0.0, "GB/s"),
-        # q and k read and written back normalised (fp16), g and beta read, gamma and beta written
-        "prologue": ("hbm", T * (4 * Nqk * D * 2 + Nv * 4 + Nv * 2 + 2 * Nv * 4), "GB/s"),
+        # q and k read once, g and beta read, norm factors / gamma / beta written
+        "prologue": ("hbm", T * (2 * Nqk * D * 2 + Nv * 4 + Nv * 2 + 2 * Nqk * 4 + 2 * Nv * 4), "GB/s"),
         "intra": ("tensor", T * (Nv * (2 * L * D + 2 * L * D) + Nqk * 2 * L * D), "TFLOP/s"),
         "state": ("tensor", T * Nv * 4 * D * D, "TFLOP/s"),
         "output": ("tensor", T * (Nv * (2 * D * D + 2 * L * D) + Nqk * 2 * L * D), "TFLOP/s"),
@@ -222,9 +222,9 @@ def main():
     def step(evs=None):
         calls = [lambda: st.chunk_map(inp.cu_seqlens),
                  lambda: st.prologue(inp.q, inp.k, inp.g, inp.beta, inp.scale, inp.eps),
-                 lambda: st.intra(inp.v),
-                 lambda: st.state(inp.state_pool, inp.state_indices, fin),
-                 lambda: st.output(out)]
+                 lambda: st.intra(inp.k, inp.v),
+                 lambda: st.state(inp.k, inp.state_pool, inp.state_indices, fin),
+                 lambda: st.output(inp.q, inp.k, out)]
         for i, c in enumerate(calls):
             if evs is not None:
                 evs[i].record(stream)

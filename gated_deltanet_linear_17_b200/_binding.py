@@ -30,7 +30,7 @@ _lib = None
 
 class _Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
-                ("total", "status", "chunk_info", "seq_chunk0", "qn", "kn", "gcum", "betaf", "U", "W", "Up", "Sc")] + \
+                ("total", "status", "chunk_info", "seq_chunk0", "rq", "rk", "gcum", "betaf", "U", "W", "Up", "Sc")] + \
                [("max_chunks", ctypes.c_int64)]
 
 
@@ -60,11 +60,11 @@ def lib():
         L.gdn_stage_prologue.restype = ctypes.c_int
         L.gdn_stage_prologue.argtypes = [p, p, p, p, f32, f32, i64, i32, i32, i32, p, sz, p]
         L.gdn_stage_intra.restype = ctypes.c_int
-        L.gdn_stage_intra.argtypes = [p, i64, i32, i32, i32, p, sz, p]
+        L.gdn_stage_intra.argtypes = [p, p, i64, i32, i32, i32, p, sz, p]
         L.gdn_stage_state.restype = ctypes.c_int
-        L.gdn_stage_state.argtypes = [p, p, p, i64, i32, i32, i32, i32, p, sz, p]
+        L.gdn_stage_state.argtypes = [p, p, p, p, i64, i32, i32, i32, i32, p, sz, p]
         L.gdn_stage_output.restype = ctypes.c_int
-        L.gdn_stage_output.argtypes = [p, i64, i32, i32, i32, p, sz, p]
+        L.gdn_stage_output.argtypes = [p, p, p, i64, i32, i32, i32, p, sz, p]
         _lib = L
     return _lib
 
@@ -214,8 +214,8 @@ class Stages:
     """The five kernels of the chunked path as separate calls on one workspace.
 
     After ``run_all`` (or the individual calls in order) the intermediates are
-    readable through the typed views ``U``, ``W``, ``Up``, ``Sc``, ``qn``, ``kn``,
-    ``gcum``, ``betaf``, ``chunk_info`` and ``status`` (U, W, Up, Sc, qn, kn in fp16)."""
+    readable through the typed views ``U``, ``W``, ``Up``, ``Sc``, ``rq``, ``rk``,
+    ``gcum``, ``betaf``, ``chunk_info`` and ``status`` (U, W, Up, Sc in fp16)."""
 
     def __init__(self, T, B, Nqk, Nv, device):
         self.T, self.B, self.Nqk, self.Nv = int(T), int(B), int(Nqk), int(Nv)
@@ -246,12 +246,12 @@ class Stages:
         return self._view("Sc", torch.float16, (self.NC, self.Nv, HEAD_DIM, HEAD_DIM))
 
     @property
-    def qn(self):
-        return self._view("qn", torch.float16, (self.T, self.Nqk, HEAD_DIM))
+    def rq(self):
+        return self._view("rq", torch.float32, (self.Nqk, self.T))
 
     @property
-    def kn(self):
-        return self._view("kn", torch.float16, (self.T, self.Nqk, HEAD_DIM))
+    def rk(self):
+        return self._view("rk", torch.float32, (self.Nqk, self.T))
 
     @property
     def gcum(self):
@@ -279,19 +279,19 @@ class Stages:
                                         self.Nqk, self.Nv, _ptr(self.ws), self.nbytes, _stream(stream)),
                "gdn_stage_prologue")
 
-    def intra(self, v, stream=None):
-        _check(lib().gdn_stage_intra(_ptr(v), self.T, self.B, self.Nqk, self.Nv, _ptr(self.ws), self.nbytes,
+    def intra(self, k, v, stream=None):
+        _check(lib().gdn_stage_intra(_ptr(k), _ptr(v), self.T, self.B, self.Nqk, self.Nv, _ptr(self.ws), self.nbytes,
                                      _stream(stream)), "gdn_stage_intra")
 
-    def state(self, state_pool=None, state_indices=None, final_state=None, stream=None):
+    def state(self, k, state_pool=None, state_indices=None, final_state=None, stream=None):
         P = 0 if state_pool is None else int(state_pool.shape[0])
-        _check(lib().gdn_stage_state(_ptr(state_pool), _ptr(state_indices), _ptr(final_state), self.T, self.B,
-                                     self.Nqk, self.Nv, P, _ptr(self.ws), self.nbytes, _stream(stream)),
+        _check(lib().gdn_stage_state(_ptr(k), _ptr(state_pool), _ptr(state_indices), _ptr(final_state), self.T,
+                                     self.B, self.Nqk, self.Nv, P, _ptr(self.ws), self.nbytes, _stream(stream)),
                "gdn_stage_state")
 
-    def output(self, out, stream=None):
-        _check(lib().gdn_stage_output(_ptr(out), self.T, self.B, self.Nqk, self.Nv, _ptr(self.ws), self.nbytes,
-                                      _stream(stream)), "gdn_stage_output")
+    def output(self, q, k, out, stream=None):
+        _check(lib().gdn_stage_output(_ptr(q), _ptr(k), _ptr(out), self.T, self.B, self.Nqk, self.Nv,
+                                      _ptr(self.ws), self.nbytes, _stream(stream)), "gdn_stage_output")
 
     def run_all(self, q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None, scale=None, eps=1e-6,
                 out=None, final_state=None, stream=None):
@@ -302,9 +302,9 @@ class Stages:
             final_state = torch.empty(self.B, self.Nv, HEAD_DIM, HEAD_DIM, dtype=torch.float32, device=dev)
         self.chunk_map(cu_seqlens, stream)
         self.prologue(q, k, g, beta, scale, eps, stream)
-        self.intra(v, stream)
-        self.state(state_pool, state_indices, final_state, stream)
-        self.output(out, stream)
+        self.intra(k, v, stream)
+        self.state(k, state_pool, state_indices, final_state, stream)
+        self.output(q, k, out, stream)
         return out, final_state
 
 

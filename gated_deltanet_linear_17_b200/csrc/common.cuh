@@ -148,6 +148,22 @@ __device__ __forceinline__ float warp_sum(float x)
     return x;
 }
 
+// convert one 16-byte chunk of 8 bf16 values in shared memory to 8 fp16 values in place
+__device__ __forceinline__ void bf16_chunk_to_fp16(uint8_t *p)
+{
+    uint4 w = *reinterpret_cast<const uint4 *>(p);
+    w = make_uint4(bf2_to_h2(w.x), bf2_to_h2(w.y), bf2_to_h2(w.z), bf2_to_h2(w.w));
+    *reinterpret_cast<uint4 *>(p) = w;
+}
+
+// split x into an fp16 pair (hi, lo) with hi + lo = x to ~22 significant bits
+__device__ __forceinline__ void split_h2(float x0, float x1, uint32_t &hi, uint32_t &lo)
+{
+    hi = pack_h2(x0, x1);
+    const float2 h = unpack_h2(hi);
+    lo = pack_h2(x0 - h.x, x1 - h.y);
+}
+
 // chunk table row: sequence, first token, tokens, chunk index within the sequence
 struct ChunkInfo {
     int seq, start, len, idx;

@@ -31,10 +31,10 @@ int fill_layout(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, gdn_workspace_lay
     off = align256(off + (size_t)NC * 16);
     lay->seq_chunk0 = off;
     off = align256(off + (size_t)(B + 1) * 4);
-    lay->qn = off;
-    off = align256(off + (size_t)Nqk * T * gdn::D * 2);
-    lay->kn = off;
-    off = align256(off + (size_t)Nqk * T * gdn::D * 2);
+    lay->rq = off;
+    off = align256(off + (size_t)Nqk * T * 4);
+    lay->rk = off;
+    off = align256(off + (size_t)Nqk * T * 4);
     lay->gcum = off;
     off = align256(off + (size_t)Nv * T * 4);
     lay->betaf = off;
@@ -59,8 +59,8 @@ Workspace views(void *base, const gdn_workspace_layout_t &lay)
     w.status = reinterpret_cast<int32_t *>(p + lay.status);
     w.chunk_info = reinterpret_cast<int4 *>(p + lay.chunk_info);
     w.seq_chunk0 = reinterpret_cast<int32_t *>(p + lay.seq_chunk0);
-    w.qn = reinterpret_cast<uint16_t *>(p + lay.qn);
-    w.kn = reinterpret_cast<uint16_t *>(p + lay.kn);
+    w.rq = reinterpret_cast<float *>(p + lay.rq);
+    w.rk = reinterpret_cast<float *>(p + lay.rk);
     w.gcum = reinterpret_cast<float *>(p + lay.gcum);
     w.betaf = reinterpret_cast<float *>(p + lay.betaf);
     w.U = reinterpret_cast<uint16_t *>(p + lay.U);
@@ -196,23 +196,23 @@ int gdn_stage_prologue(const uint16_t *q, const uint16_t *k, const float *g, con
                                             w, (cudaStream_t)stream));
 }
 
-int gdn_stage_intra(const uint16_t *v, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, void *workspace,
-                    size_t workspace_bytes, void *stream)
+int gdn_stage_intra(const uint16_t *k, const uint16_t *v, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
+                    void *workspace, size_t workspace_bytes, void *stream)
 {
     int rc = check_sizes(T, B, Nqk, Nv);
     if (rc) return rc;
     gdn_workspace_layout_t lay;
     if ((rc = check_workspace(workspace, workspace_bytes, T, B, Nqk, Nv, &lay))) return rc;
     if (B == 0 || T == 0) return GDN_OK;
-    if (!v) return GDN_ERR_NULL_ARG;
-    if (!aligned16(v)) return GDN_ERR_ALIGNMENT;
+    if (!k || !v) return GDN_ERR_NULL_ARG;
+    if (!aligned16(k) || !aligned16(v)) return GDN_ERR_ALIGNMENT;
     const Workspace w = views(workspace, lay);
-    return cuda_status(gdn::launch_intra(v, (int)T, Nqk, Nv, w.NC, w, (cudaStream_t)stream));
+    return cuda_status(gdn::launch_intra(k, v, (int)T, Nqk, Nv, w.NC, w, (cudaStream_t)stream));
 }
 
-int gdn_stage_state(const float *state_pool, const int32_t *state_indices, float *final_state, int64_t T,
-                    int32_t B, int32_t Nqk, int32_t Nv, int32_t P, void *workspace, size_t workspace_bytes,
-                    void *stream)
+int gdn_stage_state(const uint16_t *k, const float *state_pool, const int32_t *state_indices, float *final_state,
+                    int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P, void *workspace,
+                    size_t workspace_bytes, void *stream)
 {
     int rc = check_sizes(T, B, Nqk, Nv);
     if (rc) return rc;
@@ -220,28 +220,29 @@ int gdn_stage_state(const float *state_pool, const int32_t *state_indices, float
     gdn_workspace_layout_t lay;
     if ((rc = check_workspace(workspace, workspace_bytes, T, B, Nqk, Nv, &lay))) return rc;
     if (B == 0) return GDN_OK;
+    if (T > 0 && !k) return GDN_ERR_NULL_ARG;
     if (state_pool && P == 0) return GDN_ERR_BAD_SHAPE;
     if (state_pool && !state_indices && P < B) return GDN_ERR_BAD_SHAPE;
-    if (!aligned16(state_pool) || !aligned16(final_state)) return GDN_ERR_ALIGNMENT;
+    if (!aligned16(k) || !aligned16(state_pool) || !aligned16(final_state)) return GDN_ERR_ALIGNMENT;
     const size_t sbytes = (size_t)gdn::D * gdn::D * 4 * Nv;
     if (overlap(final_state, sbytes * B, state_pool, sbytes * P)) return GDN_ERR_OVERLAP;
     const Workspace w = views(workspace, lay);
-    return cuda_status(gdn::launch_state(state_pool, state_indices, final_state, (int)T, B, Nqk, Nv, w,
+    return cuda_status(gdn::launch_state(k, state_pool, state_indices, final_state, (int)T, B, Nqk, Nv, w,
                                          (cudaStream_t)stream));
 }
 
-int gdn_stage_output(uint16_t *out, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, void *workspace,
-                     size_t workspace_bytes, void *stream)
+int gdn_stage_output(const uint16_t *q, const uint16_t *k, uint16_t *out, int64_t T, int32_t B, int32_t Nqk,
+                     int32_t Nv, void *workspace, size_t workspace_bytes, void *stream)
 {
     int rc = check_sizes(T, B, Nqk, Nv);
     if (rc) return rc;
     gdn_workspace_layout_t lay;
     if ((rc = check_workspace(workspace, workspace_bytes, T, B, Nqk, Nv, &lay))) return rc;
     if (B == 0 || T == 0) return GDN_OK;
-    if (!out) return GDN_ERR_NULL_ARG;
-    if (!aligned16(out)) return GDN_ERR_ALIGNMENT;
+    if (!q || !k || !out) return GDN_ERR_NULL_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(out)) return GDN_ERR_ALIGNMENT;
     const Workspace w = views(workspace, lay);
-    return cuda_status(gdn::launch_output(out, (int)T, Nqk, Nv, w.NC, w, (cudaStream_t)stream));
+    return cuda_status(gdn::launch_output(q, k, out, (int)T, Nqk, Nv, w.NC, w, (cudaStream_t)stream));
 }
 
 int gdn_short_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
@@ -287,9 +288,9 @@ int gdn_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
     const int Ti = (int)T;
     cudaError_t e = gdn::launch_chunk_map(cu_seqlens, B, Ti, w.NC, w, st);
     if (e == cudaSuccess) e = gdn::launch_prologue(q, k, g, beta, sc, eps, Ti, Nqk, Nv, w.NC, w, st);
-    if (e == cudaSuccess) e = gdn::launch_intra(v, Ti, Nqk, Nv, w.NC, w, st);
-    if (e == cudaSuccess) e = gdn::launch_state(state_pool, state_indices, final_state, Ti, B, Nqk, Nv, w, st);
-    if (e == cudaSuccess) e = gdn::launch_output(out, Ti, Nqk, Nv, w.NC, w, st);
+    if (e == cudaSuccess) e = gdn::launch_intra(k, v, Ti, Nqk, Nv, w.NC, w, st);
+    if (e == cudaSuccess) e = gdn::launch_state(k, state_pool, state_indices, final_state, Ti, B, Nqk, Nv, w, st);
+    if (e == cudaSuccess) e = gdn::launch_output(q, k, out, Ti, Nqk, Nv, w.NC, w, st);
     if (owned) {
         cudaError_t f = cudaFreeAsync(workspace, st);
         if (e == cudaSuccess) e = f;

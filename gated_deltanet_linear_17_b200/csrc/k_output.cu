@@ -4,8 +4,10 @@
 //   o_inter = (q (.) exp(g_cum)) S^T
 //   o_chunk = o_inter + (q k^T (.) D_decay (.) T_tril) (v_out - v')
 // with S held as [Dk, Dv] (so S^T there is S here), T_tril including the
-// diagonal, and v_out - v' = U' from the state kernel.  q (normalised and
-// scaled) and k (normalised) come from the prologue in fp16; all tensor-core
+// diagonal, and v_out - v' = U' from the state kernel.  The raw bf16 q and k
+// rows are converted to fp16 in place once they land (exact); the
+// normalisation and the query scale enter as the prologue's fp32 factors rq,
+// rk, applied to the q k^T product and to the rows of q S.  All tensor-core
 // operands are fp16 with fp32 accumulation.  Each warp owns 16 rows of the chunk.
 #include "common.cuh"
 #include "gdn_internal.h"
@@ -14,12 +16,12 @@ namespace gdn {
 
 constexpr int kOutThreads = 256;
 constexpr int OO_Q = 0, OO_K = 32768, OO_S = 65536, OO_U = 98304, OO_P = 131072, OO_VEC = 163840;
-constexpr int kOutSmem = OO_VEC + 128 * 4;
+constexpr int kOutSmem = OO_VEC + 3 * 128 * 4;
 
 __global__ void __launch_bounds__(kOutThreads, 1) output_kernel(
-    const uint16_t *__restrict__ qn, const uint16_t *__restrict__ kn, uint16_t *__restrict__ out, int T,
-    int Nqk, int Nv, const int4 *__restrict__ info, const float *__restrict__ gcum,
-    const uint16_t *__restrict__ Up, const uint16_t *__restrict__ Sc)
+    const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, uint16_t *__restrict__ out, int T,
+    int Nqk, int Nv, const int4 *__restrict__ info, const float *__restrict__ rq, const float *__restrict__ rk,
+    const float *__restrict__ gcum, const uint16_t *__restrict__ Up, const uint16_t *__restrict__ Sc)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int c = blockIdx.x, h = blockIdx.y;
@@ -34,20 +36,31 @@ __global__ void __launch_bounds__(kOutThreads, 1) output_kernel(
                    us = smem_addr(smem + OO_U), ps = smem_addr(smem + OO_P);
     uint8_t *Ps = smem + OO_P;
     float *gam = reinterpret_cast<float *>(smem + OO_VEC);
+    float *rqv = gam + 128, *rkv = gam + 256;
 
     const size_t tile = (size_t)(c * Nv + h) * L * D;
     for (int e = tid; e < 128 * 16; e += kOutThreads) {
         const int r = e >> 4, cc = e & 15;
         const bool ok = r < n;
         const int t = t0 + (ok ? r : 0);
-        cp_async16(qs + sw256(r, cc), qn + ((size_t)t * Nqk + hq) * D + cc * 8, ok);
-        cp_async16(ks + sw256(r, cc), kn + ((size_t)t * Nqk + hq) * D + cc * 8, ok);
+        cp_async16(qs + sw256(r, cc), q + ((size_t)t * Nqk + hq) * D + cc * 8, ok);
+        cp_async16(ks + sw256(r, cc), k + ((size_t)t * Nqk + hq) * D + cc * 8, ok);
         cp_async16(ss + sw256(r, cc), Sc + tile + r * D + cc * 8, true);
         cp_async16(us + sw256(r, cc), Up + tile + r * D + cc * 8, true);
     }
     cp_async_commit();
-    if (tid < 128) gam[tid] = gcum[(size_t)h * T + t0 + min(tid, n - 1)];
+    if (tid < 128) {
+        const int i = tid;
+        gam[i] = gcum[(size_t)h * T + t0 + min(i, n - 1)];
+        rqv[i] = i < n ? rq[(size_t)hq * T + t0 + i] : 0.f;
+        rkv[i] = i < n ? rk[(size_t)hq * T + t0 + i] : 0.f;
+    }
     cp_async_wait<0>();
+    // the q and k rows this thread copied have landed: convert them to fp16 in place
+    for (int e = tid; e < 128 * 16; e += kOutThreads) {
+        bf16_chunk_to_fp16(smem + OO_Q + sw256(e >> 4, e & 15));
+        bf16_chunk_to_fp16(smem + OO_K + sw256(e >> 4, e & 15));
+    }
     __syncthreads();
 
     const int m0 = wid * 16;
@@ -77,15 +90,16 @@ __global__ void __launch_bounds__(kOutThreads, 1) output_kernel(
                 const int row = m0 + gid + hf * 8;
                 const int col = nt * 8 + tig * 2;
                 float p0 = 0.f, p1 = 0.f;
-                if (col <= row) p0 = acc[nt][2 * hf] * __expf(gam[row] - gam[col]);
-                if (col + 1 <= row) p1 = acc[nt][2 * hf + 1] * __expf(gam[row] - gam[col + 1]);
+                const float fr = rqv[row];
+                if (col <= row) p0 = fr * rkv[col] * acc[nt][2 * hf] * __expf(gam[row] - gam[col]);
+                if (col + 1 <= row) p1 = fr * rkv[col + 1] * acc[nt][2 * hf + 1] * __expf(gam[row] - gam[col + 1]);
                 *reinterpret_cast<uint32_t *>(Ps + el256(row, col)) = pack_h2(p0, p1);
             }
         }
     }
     __syncwarp();
 
-    // ---- o = diag(e^gamma) Qh S_c + P U'
+    // ---- o = diag(rq e^gamma) Q S_c + P U'
 #pragma unroll
     for (int i = 0; i < 16; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
 #pragma unroll
@@ -101,8 +115,8 @@ __global__ void __launch_bounds__(kOutThreads, 1) output_kernel(
         }
     }
     {
-        const float f0 = __expf(gam[m0 + gid]);
-        const float f1 = __expf(gam[m0 + gid + 8]);
+        const float f0 = rqv[m0 + gid] * __expf(gam[m0 + gid]);
+        const float f1 = rqv[m0 + gid + 8] * __expf(gam[m0 + gid + 8]);
 #pragma unroll
         for (int nt = 0; nt < 16; ++nt) {
             acc[nt][0] *= f0;
@@ -135,13 +149,14 @@ __global__ void __launch_bounds__(kOutThreads, 1) output_kernel(
     }
 }
 
-cudaError_t launch_output(uint16_t *out, int T, int Nqk, int Nv, int NC, const Workspace &ws, cudaStream_t st)
+cudaError_t launch_output(const uint16_t *q, const uint16_t *k, uint16_t *out, int T, int Nqk, int Nv, int NC,
+                          const Workspace &ws, cudaStream_t st)
 {
     if (NC == 0) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kOutSmem);
     if (e != cudaSuccess) return e;
-    output_kernel<<<dim3(NC, Nv), kOutThreads, kOutSmem, st>>>(ws.qn, ws.kn, out, T, Nqk, Nv, ws.chunk_info,
+    output_kernel<<<dim3(NC, Nv), kOutThreads, kOutSmem, st>>>(q, k, out, T, Nqk, Nv, ws.chunk_info, ws.rq, ws.rk,
                                                                 ws.gcum, ws.Up, ws.Sc);
     return cudaGetLastError();
 }

@@ -3,14 +3,15 @@
 // chunk_map: one CTA turns cu_seqlens into the table of 128-token chunks
 //   ("Qwen3Next Samples": chunk length L = 128, act_seq_len as cumulative
 //   sequence lengths).
-// prologue : per chunk, the L2-normalised q (times the query scale) and k
-//   ("L2 Normalization", eps inside the square root) in fp16, the chunk-local
-//   cumulative gate ("Gate Cumulative Sum") and beta in fp32, the gate and beta
-//   laid out head-major ([head][token]) so that later kernels read one chunk of
-//   one head as a contiguous run.  Bound by HBM: it streams q and k once.
-//   Normalised rows lie in [-1, 1], so fp16 (11-bit significand) holds them
-//   with 8x less rounding than bf16; the tensor-core products downstream use
-//   fp16 operands throughout.
+// prologue : per chunk, the L2 normalisation of q (times the query scale) and
+//   of k ("L2 Normalization", eps inside the square root) as fp32 factors
+//   rq = scale / sqrt(|q|^2 + eps), rk = 1 / sqrt(|k|^2 + eps), the chunk-local
+//   cumulative gate ("Gate Cumulative Sum") and beta in fp32, all laid out
+//   head-major ([head][token]) so that later kernels read one chunk of one head
+//   as a contiguous run.  The factors are applied where q and k are consumed
+//   (as fp32 row/column scalings around tensor-core products on the raw rows,
+//   which convert exactly from bf16 to fp16), so no rounded normalised copy of
+//   q or k is ever made.  Bound by HBM: it streams q and k once.
 #include "common.cuh"
 #include "gdn_internal.h"
 
@@ -86,11 +87,13 @@ __global__ void __launch_bounds__(kMapThreads) chunk_map_kernel(const int32_t *_
 
 constexpr int kProThreads = 256;
 constexpr int kHeadGroup = 32;  // v-heads per pass of the gate scan
+constexpr int kProSplit = 4;    // CTAs per chunk: each normalises a quarter of the chunk's rows
+constexpr int kRowsInFlight = 4; // rows each half-warp loads before reducing
 
 __global__ void __launch_bounds__(kProThreads) prologue_kernel(
     const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, const float *__restrict__ g,
     const uint16_t *__restrict__ beta, float scale, float eps, int T, int Nqk, int Nv,
-    const int4 *__restrict__ info, uint16_t *__restrict__ qn, uint16_t *__restrict__ kn,
+    const int4 *__restrict__ info, float *__restrict__ rq, float *__restrict__ rk,
     float *__restrict__ gcum, float *__restrict__ betaf)
 {
     __shared__ float gs[L][kHeadGroup + 1];
@@ -98,9 +101,10 @@ __global__ void __launch_bounds__(kProThreads) prologue_kernel(
     if (ci.seq < 0) return;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int n = ci.len, t0 = ci.start;
+    const int part = blockIdx.y;
 
-    // ---- gates: chunk-local inclusive cumsum of g per v-head, beta to fp32
-    for (int hg = 0; hg < Nv; hg += kHeadGroup) {
+    // ---- gates (first CTA of the chunk): chunk-local inclusive cumsum of g per v-head, beta to fp32
+    for (int hg = 0; part == 0 && hg < Nv; hg += kHeadGroup) {
         const int nh = min(kHeadGroup, Nv - hg);
         for (int e = tid; e < L * kHeadGroup; e += kProThreads) {
             const int i = e / kHeadGroup, j = e % kHeadGroup;
@@ -129,41 +133,46 @@ __global__ void __launch_bounds__(kProThreads) prologue_kernel(
         }
         __syncthreads();
     }
-    for (int e = tid; e < n * Nv; e += kProThreads) {
+    for (int e = tid; part == 0 && e < n * Nv; e += kProThreads) {
         const int i = e / Nv, h = e % Nv;
         betaf[(size_t)h * T + t0 + i] = bf2f(beta[(size_t)(t0 + i) * Nv + h]);
     }
 
-    // ---- L2 normalisation: a half-warp per 128-element row, 16 bytes per lane
+    // ---- L2 norms: a half-warp per 128-element row, 16 bytes per lane,
+    //      kRowsInFlight rows loaded before any is reduced
     const int rows = n * Nqk;  // rows of q (and of k) in this chunk, contiguous in memory
     const int half = lane >> 4, hl = lane & 15;
-    for (int r0 = wid * 2; r0 < 2 * rows; r0 += (kProThreads / 32) * 2) {
-        const int r = r0 + half;  // r < rows: q row, else k row
-        const bool valid = r < 2 * rows;
-        const bool isk = r >= rows;
-        const int rr = isk ? r - rows : r;
-        const size_t off = ((size_t)t0 * Nqk + rr) * D + hl * 8;
-        uint4 w = make_uint4(0u, 0u, 0u, 0u);
-        if (valid) w = *reinterpret_cast<const uint4 *>((isk ? k : q) + off);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-        float x[8];
-        float ss = 0.f;
+    const int stride = kProSplit * (kProThreads / 32) * 2 * kRowsInFlight;
+    for (int rbase = (part * (kProThreads / 32) + wid) * 2 * kRowsInFlight; rbase < 2 * rows; rbase += stride) {
+        uint4 w[kRowsInFlight];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            x[2 * u] = __uint_as_float(ws[u] << 16);
-            x[2 * u + 1] = __uint_as_float(ws[u] & 0xffff0000u);
-            ss += x[2 * u] * x[2 * u] + x[2 * u + 1] * x[2 * u + 1];
+        for (int u = 0; u < kRowsInFlight; ++u) {
+            const int r = rbase + 2 * u + half;  // r < rows: q row, else k row
+            const bool isk = r >= rows;
+            const int rr = isk ? r - rows : r;
+            w[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (r < 2 * rows)
+                w[u] = __ldg(reinterpret_cast<const uint4 *>((isk ? k : q) + ((size_t)t0 * Nqk + rr) * D + hl * 8));
         }
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if (valid) {
-            const float f = (isk ? 1.0f : scale) / sqrtf(ss + eps);
-            uint4 o;
-            o.x = pack_h2(x[0] * f, x[1] * f);
-            o.y = pack_h2(x[2] * f, x[3] * f);
-            o.z = pack_h2(x[4] * f, x[5] * f);
-            o.w = pack_h2(x[6] * f, x[7] * f);
-            *reinterpret_cast<uint4 *>((isk ? kn : qn) + off) = o;
+        for (int u = 0; u < kRowsInFlight; ++u) {
+            const int r = rbase + 2 * u + half;
+            const bool isk = r >= rows;
+            const int rr = isk ? r - rows : r;
+            const uint32_t ws[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+            float ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float a = __uint_as_float(ws[e] << 16), b = __uint_as_float(ws[e] & 0xffff0000u);
+                ss += a * a + b * b;
+            }
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            if (r < 2 * rows && hl == 0) {
+                const int i = rr / Nqk, hq = rr % Nqk;
+                const float f = (isk ? 1.0f : scale) / sqrtf(ss + eps);
+                (isk ? rk : rq)[(size_t)hq * T + t0 + i] = f;
+            }
         }
     }
 }
@@ -180,8 +189,8 @@ cudaError_t launch_prologue(const uint16_t *q, const uint16_t *k, const float *g
                             cudaStream_t st)
 {
     if (NC == 0) return cudaSuccess;
-    prologue_kernel<<<NC, kProThreads, 0, st>>>(q, k, g, beta, scale, eps, T, Nqk, Nv, ws.chunk_info,
-                                                ws.qn, ws.kn, ws.gcum, ws.betaf);
+    prologue_kernel<<<dim3(NC, kProSplit), kProThreads, 0, st>>>(q, k, g, beta, scale, eps, T, Nqk, Nv, ws.chunk_info,
+                                                ws.rq, ws.rk, ws.gcum, ws.betaf);
     return cudaGetLastError();
 }
 

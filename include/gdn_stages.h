@@ -41,16 +41,17 @@ extern "C" {
  *   chunk_info  int32[NC][4]: sequence, first token, tokens in the chunk (1..128),
  *               chunk index within its sequence; rows past the last chunk hold -1
  *   seq_chunk0  int32[B+1]: first chunk of each sequence, [B] = number of chunks
- *   qn          fp16 [T][Nqk][128]: scale * q / sqrt(|q|^2 + eps)
- *   kn          fp16 [T][Nqk][128]: k / sqrt(|k|^2 + eps)
+ *   rq          fp32 [Nqk][T]: scale / sqrt(|q|^2 + eps)
+ *   rk          fp32 [Nqk][T]: 1 / sqrt(|k|^2 + eps)
  *   gcum        fp32 [Nv][T]: chunk-local cumulative gate gamma
  *   betaf       fp32 [Nv][T]: beta widened to fp32
  *   U, W, Up    fp16 [NC][Nv][128 (L)][128]: U, W (columns Dk) and U' of each chunk
  *   Sc          fp16 [NC][Nv][128 (Dk)][128 (Dv)]: state entering each chunk
  * The tensor-core products take fp16 operands (11-bit significand) with fp32
- * accumulation; fp16 holds the normalised q and k exactly enough and keeps
- * the max-abs error of the pass well inside the tolerance, where bf16
- * operands did not.  Values derived from v (U, U', S) must stay below 65504 in
+ * accumulation: the raw bf16 q, k, v convert to fp16 exactly (magnitudes in
+ * [2^-14, 65504]), the L2 norms enter as fp32 scalings, and the state update's
+ * second operand is split into two fp16 halves; bf16 operands missed the
+ * max-abs bound.  Values derived from v (U, U', S) must stay below 65504 in
  * magnitude.
  */
 typedef struct {
@@ -58,8 +59,8 @@ typedef struct {
     size_t status;
     size_t chunk_info;
     size_t seq_chunk0;
-    size_t qn;
-    size_t kn;
+    size_t rq;
+    size_t rk;
     size_t gcum;
     size_t betaf;
     size_t U;
@@ -84,12 +85,12 @@ int gdn_stage_chunk_map(const int32_t *cu_seqlens, int64_t T, int32_t B, int32_t
                         void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * Prologue: per token and qk-head the L2-normalised q (times scale) and k
- * ("L2 Normalization", eps inside the square root) in fp16, per chunk and
- * v-head the cumulative gate ("Gate Cumulative Sum") restarting at every chunk
- * start, and beta widened to fp32.  Reads q, k [T, Nqk, 128] bf16, g [T, Nv]
- * fp32, beta [T, Nv] bf16; writes qn, kn, gcum, betaf.  scale <= 0 selects
- * 1/sqrt(128).
+ * Prologue: per token and qk-head the L2 normalisation factors of q (times
+ * scale) and k ("L2 Normalization", eps inside the square root), per chunk
+ * and v-head the cumulative gate ("Gate Cumulative Sum") restarting at every
+ * chunk start, and beta widened to fp32.  Reads q, k [T, Nqk, 128] bf16,
+ * g [T, Nv] fp32, beta [T, Nv] bf16; writes rq, rk, gcum, betaf.
+ * scale <= 0 selects 1/sqrt(128).
  */
 int gdn_stage_prologue(const uint16_t *q, const uint16_t *k, const float *g, const uint16_t *beta,
                        float scale, float eps, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
@@ -99,11 +100,11 @@ int gdn_stage_prologue(const uint16_t *q, const uint16_t *k, const float *g, con
  * Intra-chunk: per (chunk, v-head) forms A ("Pre-Attention Matrix"), solves
  * T = (I + A)^-1 by blocked forward substitution ("Matrix Inversion" with the
  * block merge of inverse_pto / inverse_matmul), and computes U and W ("Value
- * and Key Cumulative Decay").  Reads v [T, Nv, 128] bf16 and the prologue's
- * outputs; writes U, W.
+ * and Key Cumulative Decay").  Reads k [T, Nqk, 128], v [T, Nv, 128] (bf16)
+ * and the prologue's outputs; writes U, W.
  */
-int gdn_stage_intra(const uint16_t *v, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, void *workspace,
-                    size_t workspace_bytes, void *stream);
+int gdn_stage_intra(const uint16_t *k, const uint16_t *v, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
+                    void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Inter-chunk state passing: per (sequence, v-head, 32-column slice of Dv),
@@ -111,21 +112,21 @@ int gdn_stage_intra(const uint16_t *v, int64_t T, int32_t B, int32_t Nqk, int32_
  * S <- e^{gamma_last} S + (Kh * e^{gamma_last - gamma})^T U' ("Recurrent State
  * Attention" v', "State Update" with k_gexp), the state kept in fp32 on chip.
  * S starts from state_pool[state_indices[b]] (or slot b, or zero without a
- * pool).  Reads kn, gcum, U, W; writes Sc and Up for every chunk and
- * final_state (if not NULL).
+ * pool).  Reads k [T, Nqk, 128] bf16, rk, gcum, U, W; writes Sc and Up for
+ * every chunk and final_state (if not NULL).
  */
-int gdn_stage_state(const float *state_pool, const int32_t *state_indices, float *final_state, int64_t T,
-                    int32_t B, int32_t Nqk, int32_t Nv, int32_t P, void *workspace, size_t workspace_bytes,
-                    void *stream);
+int gdn_stage_state(const uint16_t *k, const float *state_pool, const int32_t *state_indices, float *final_state,
+                    int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P, void *workspace,
+                    size_t workspace_bytes, void *stream);
 
 /*
  * Output: per (chunk, v-head) o = diag(e^gamma) Qh S_c + (Qh Kh^T * Gamma * tril) U'
  * ("Recurrent State Attention": o_inter and o_chunk; tril includes the
- * diagonal).  Reads qn, kn, gcum, Sc, Up; writes out [T, Nv, 128] bf16 for
- * every token of every chunk.
+ * diagonal).  Reads q, k [T, Nqk, 128] bf16, rq, rk, gcum, Sc, Up; writes
+ * out [T, Nv, 128] bf16 for every token of every chunk.
  */
-int gdn_stage_output(uint16_t *out, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, void *workspace,
-                     size_t workspace_bytes, void *stream);
+int gdn_stage_output(const uint16_t *q, const uint16_t *k, uint16_t *out, int64_t T, int32_t B, int32_t Nqk,
+                     int32_t Nv, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Fused short-sequence forward: the token recurrence of the decode page

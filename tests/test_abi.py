@@ -52,7 +52,7 @@ def test_status_strings(lib):
 def test_workspace_layout_regions_disjoint_and_aligned(lib):
     lay = gdn.workspace_layout(4048, 4, 4, 8)
     assert lay["max_chunks"] == (4048 + 127 * 4) // 128
-    regions = ["status", "chunk_info", "seq_chunk0", "qn", "kn", "gcum", "betaf", "U", "W", "Up", "Sc"]
+    regions = ["status", "chunk_info", "seq_chunk0", "rq", "rk", "gcum", "betaf", "U", "W", "Up", "Sc"]
     offs = [lay[r] for r in regions]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     tile = 128 * 128 * 2
@@ -106,9 +106,9 @@ def test_argument_errors_before_any_launch(lib):
 
 def test_stage_argument_errors(lib):
     vp = ctypes.c_void_p
-    assert lib.gdn_stage_intra(vp(16), 8, 1, 2, 4, None, 0, None) == B.GDN_ERR_NULL_ARG
-    assert lib.gdn_stage_intra(vp(16), 8, 1, 2, 4, vp(16), 10, None) == B.GDN_ERR_WORKSPACE
-    assert lib.gdn_stage_output(vp(16), 8, 1, 2, 3, vp(16), 1 << 30, None) == B.GDN_ERR_BAD_SHAPE
+    assert lib.gdn_stage_intra(vp(16), vp(16), 8, 1, 2, 4, None, 0, None) == B.GDN_ERR_NULL_ARG
+    assert lib.gdn_stage_intra(vp(16), vp(16), 8, 1, 2, 4, vp(16), 10, None) == B.GDN_ERR_WORKSPACE
+    assert lib.gdn_stage_output(vp(16), vp(16), vp(16), 8, 1, 2, 3, vp(16), 1 << 30, None) == B.GDN_ERR_BAD_SHAPE
 
 
 def test_python_layer_refuses_cpu_tensors():

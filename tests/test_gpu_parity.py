@@ -94,7 +94,7 @@ def test_stages_match_chunked_intermediates():
     got = {n: [] for n in names}
     ref = {n: [] for n in names}
     gam_g, gam_r, kh_g, kh_r, qh_g, qh_r = [], [], [], [], [], []
-    kn, qn, gcum = st.kn.cpu().double().numpy(), st.qn.cpu().double().numpy(), st.gcum.cpu().double()
+    rk, rq, gcum = st.rk.cpu().double().numpy(), st.rq.cpu().double().numpy(), st.gcum.cpu().double()
     G = inp.Nv // inp.Nqk
     for (b, h, ci), r in kept.items():
         c = seq_first[b] + ci
@@ -108,15 +108,15 @@ def test_stages_match_chunked_intermediates():
         hq = h // G
         gam_g.append(gcum[h, t0:t0 + n].numpy())
         gam_r.append(r["g_cum"])
-        kh_g.append(kn[t0:t0 + n, hq])
+        kh_g.append(X["k"][t0:t0 + n, hq] * rk[hq, t0:t0 + n, None])
         kh_r.append(r["kn"])
-        qh_g.append(qn[t0:t0 + n, hq])
+        qh_g.append(X["q"][t0:t0 + n, hq] * rq[hq, t0:t0 + n, None])
         qh_r.append(r["qn"])
     cat = lambda xs: np.concatenate([x.reshape(-1) for x in xs])
     assert_close(cat(gam_g), cat(gam_r), "gcum", rel_l2=1e-5, max_abs_rms=1e-5)
-    # fp16 storage of values in [-1, 1]: relative rounding <= 2^-11
-    assert_close(cat(kh_g), cat(kh_r), "k normalised", rel_l2=1e-3, max_abs_rms=1e-2)
-    assert_close(cat(qh_g), cat(qh_r), "q normalised and scaled", rel_l2=1e-3, max_abs_rms=1e-2)
+    # fp32 normalisation factors applied to the exact raw rows
+    assert_close(cat(kh_g), cat(kh_r), "k normalised", rel_l2=1e-5, max_abs_rms=1e-5)
+    assert_close(cat(qh_g), cat(qh_r), "q normalised and scaled", rel_l2=1e-5, max_abs_rms=1e-5)
     for nm in names:  # fp16 intermediates: their own storage rounding is allowed per element
         assert_close(cat(got[nm]), cat(ref[nm]), f"stage {nm}", ulp=helpers.FP16_HALF_ULP)
     _check(inp, out, fin, what="stages")
