@@ -40,6 +40,11 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool v
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n)
                  : "memory");
 }
+// 4-byte global->shared copy (always valid)
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait()
@@ -69,6 +74,16 @@ __device__ __forceinline__ void mma16816(float *d, const uint32_t *a, uint32_t b
 {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D += A(16x16, row) * B(16x8, col), bf16 inputs, fp32 accumulate
+__device__ __forceinline__ void mma16816_bf16(float *d, const uint32_t *a, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -156,12 +171,12 @@ __device__ __forceinline__ void bf16_chunk_to_fp16(uint8_t *p)
     *reinterpret_cast<uint4 *>(p) = w;
 }
 
-// split x into an fp16 pair (hi, lo) with hi + lo = x to ~22 significant bits
-__device__ __forceinline__ void split_h2(float x0, float x1, uint32_t &hi, uint32_t &lo)
+// split x into a bf16 pair (hi, lo) with hi + lo = x to ~16 significant bits
+__device__ __forceinline__ void split_bf2(float x0, float x1, uint32_t &hi, uint32_t &lo)
 {
-    hi = pack_h2(x0, x1);
-    const float2 h = unpack_h2(hi);
-    lo = pack_h2(x0 - h.x, x1 - h.y);
+    hi = pack_bf2(x0, x1);
+    const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xffff0000u);
+    lo = pack_bf2(x0 - h0, x1 - h1);
 }
 
 // chunk table row: sequence, first token, tokens, chunk index within the sequence

@@ -19,11 +19,11 @@
 // runs the whole block recurrence on them by itself, on tensor cores, with no
 // CTA-wide barrier inside the solve.  X overwrites R in place.
 //
-// The raw bf16 k and v rows are converted to fp16 while staged (exact: bf16's
-// 8-bit significand fits fp16's 11 bits); the L2 normalisation of k enters as
-// the prologue's fp32 factors rk, applied to the Kh Kh^T product and to the
-// right-hand side.  Tensor-core operands are fp16 with fp32 accumulation; U and
-// W are stored in fp16.
+// The raw bf16 k and v rows are staged as they are; K K^T is a bf16 product of
+// exact inputs, and the L2 normalisation of k enters as the prologue's fp32
+// factors rk, applied to that product and to the right-hand side.  The solve
+// itself runs on fp16 operands (the brackets and X overwrite the bf16
+// right-hand side in place), with fp32 accumulation; U and W are stored in fp16.
 #include "common.cuh"
 #include "gdn_internal.h"
 
@@ -32,7 +32,7 @@ namespace gdn {
 constexpr int kIntraThreads = 256;
 
 // shared memory (bytes)
-constexpr int OFF_RX = 0;                 // fp16 [128][256]: [V | Kh], then [U | W]; 512-byte rows
+constexpr int OFF_RX = 0;                 // [128][256]: bf16 [V | K], then fp16 [U | W]; 512-byte rows
 constexpr int OFF_AP = 65536;             // fp16 [128][128]: Ap off-diagonal blocks (256-byte rows)
 constexpr int OFF_TD = OFF_AP + 32768;    // fp16 8 x [16][16]: T_ii (32-byte rows)
 constexpr int OFF_DS = OFF_TD + 4096;     // fp32 8 x [16][16]: per-warp diagonal block scratch
@@ -60,18 +60,16 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     float *gam = reinterpret_cast<float *>(smem + OFF_VEC);
     float *bet = gam + 128, *egam = gam + 256, *rkv = gam + 384;
 
-    // ---- stage [V | K] as fp16 (rows past the chunk are zero)
+    // ---- stage [V | K] (rows past the chunk are zero) with async copies
     for (int e = tid; e < 128 * 32; e += kIntraThreads) {
         const int r = e >> 5, cc = e & 31;
-        uint4 w = make_uint4(0u, 0u, 0u, 0u);
-        if (r < n) {
-            const uint16_t *src = cc < 16 ? v + ((size_t)(t0 + r) * Nv + h) * D + cc * 8
-                                          : k + ((size_t)(t0 + r) * Nqk + hq) * D + (cc - 16) * 8;
-            w = __ldg(reinterpret_cast<const uint4 *>(src));
-            w = make_uint4(bf2_to_h2(w.x), bf2_to_h2(w.y), bf2_to_h2(w.z), bf2_to_h2(w.w));
-        }
-        *reinterpret_cast<uint4 *>(smem + OFF_RX + sw512(r, cc)) = w;
+        const bool ok = r < n;
+        const int t = t0 + (ok ? r : 0);
+        const uint16_t *src = cc < 16 ? v + ((size_t)t * Nv + h) * D + cc * 8
+                                      : k + ((size_t)t * Nqk + hq) * D + (cc - 16) * 8;
+        cp_async16(rx + sw512(r, cc), src, ok);
     }
+    cp_async_commit();
     if (tid < 128) {
         const int i = tid;
         const float gi = gcum[(size_t)h * T + t0 + min(i, n - 1)];
@@ -80,6 +78,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
         bet[i] = i < n ? betaf[(size_t)h * T + t0 + i] : 0.f;
         rkv[i] = i < n ? rk[(size_t)hq * T + t0 + i] : 0.f;
     }
+    cp_async_wait<0>();
     __syncthreads();
 
     const int m0 = wid * 16;  // this warp's row block in the KK^T step
@@ -101,8 +100,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
                     const int r = np * 16 + (lane & 7) + ((lane >> 4) << 3);
                     uint32_t b0, b1, b2, b3;
                     ldsm_x4(rx + sw512(r, 16 + (kk >> 3) + ((lane >> 3) & 1)), b0, b1, b2, b3);
-                    mma16816(acc[2 * np], a, b0, b1);
-                    mma16816(acc[2 * np + 1], a, b2, b3);
+                    mma16816_bf16(acc[2 * np], a, b0, b1);
+                    mma16816_bf16(acc[2 * np + 1], a, b2, b3);
                 }
             }
         }
@@ -166,9 +165,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt) {
                     const uint32_t off = sw512(row, cb + nt) + tig * 4;
-                    const float2 x = unpack_h2(*reinterpret_cast<const uint32_t *>(smem + OFF_RX + off));
-                    acc[nt][2 * hf] = x.x * f;
-                    acc[nt][2 * hf + 1] = x.y * f;
+                    const uint32_t x = *reinterpret_cast<const uint32_t *>(smem + OFF_RX + off);  // bf16 pair
+                    acc[nt][2 * hf] = __uint_as_float(x << 16) * f;
+                    acc[nt][2 * hf + 1] = __uint_as_float(x & 0xffff0000u) * f;
                 }
             }
             // + sum_{j<i} Ap_ij X_j

@@ -4,18 +4,21 @@
 //   o_inter = (q (.) exp(g_cum)) S^T
 //   o_chunk = o_inter + (q k^T (.) D_decay (.) T_tril) (v_out - v')
 // with S held as [Dk, Dv] (so S^T there is S here), T_tril including the
-// diagonal, and v_out - v' = U' from the state kernel.  The raw bf16 q and k
-// rows are converted to fp16 in place once they land (exact); the
-// normalisation and the query scale enter as the prologue's fp32 factors rq,
-// rk, applied to the q k^T product and to the rows of q S.  All tensor-core
-// operands are fp16 with fp32 accumulation.  Each warp owns 16 rows of the chunk.
+// diagonal, and v_out - v' = U' from the state kernel.  q k^T is a bf16
+// product of the raw rows (exact inputs); q is then converted to fp16 in place
+// (exact) for the q S product with the fp16 state.  The normalisation and the
+// query scale enter as the prologue's fp32 factors rq, rk, applied to the
+// q k^T product and to the rows of q S.  Accumulation is fp32.  Each warp owns 16 rows of the chunk;
+// its rows of P = (q k^T) (.) Gamma (.) tril never leave registers: the
+// accumulator fragments of two adjacent 8-column tiles are exactly the A
+// fragment of one 16-wide k step of the P U' product.
 #include "common.cuh"
 #include "gdn_internal.h"
 
 namespace gdn {
 
 constexpr int kOutThreads = 256;
-constexpr int OO_Q = 0, OO_K = 32768, OO_S = 65536, OO_U = 98304, OO_P = 131072, OO_VEC = 163840;
+constexpr int OO_Q = 0, OO_K = 32768, OO_S = 65536, OO_U = 98304, OO_VEC = 131072;
 constexpr int kOutSmem = OO_VEC + 3 * 128 * 4;
 
 __global__ void __launch_bounds__(kOutThreads, 1) output_kernel(
@@ -33,8 +36,7 @@ __global__ void __launch_bounds__(kOutThreads, 1) output_kernel(
     const int gid = lane >> 2, tig = lane & 3;
 
     const uint32_t qs = smem_addr(smem + OO_Q), ks = smem_addr(smem + OO_K), ss = smem_addr(smem + OO_S),
-                   us = smem_addr(smem + OO_U), ps = smem_addr(smem + OO_P);
-    uint8_t *Ps = smem + OO_P;
+                   us = smem_addr(smem + OO_U);
     float *gam = reinterpret_cast<float *>(smem + OO_VEC);
     float *rqv = gam + 128, *rkv = gam + 256;
 
@@ -56,11 +58,6 @@ __global__ void __launch_bounds__(kOutThreads, 1) output_kernel(
         rkv[i] = i < n ? rk[(size_t)hq * T + t0 + i] : 0.f;
     }
     cp_async_wait<0>();
-    // the q and k rows this thread copied have landed: convert them to fp16 in place
-    for (int e = tid; e < 128 * 16; e += kOutThreads) {
-        bf16_chunk_to_fp16(smem + OO_Q + sw256(e >> 4, e & 15));
-        bf16_chunk_to_fp16(smem + OO_K + sw256(e >> 4, e & 15));
-    }
     __syncthreads();
 
     const int m0 = wid * 16;
@@ -77,27 +74,32 @@ __global__ void __launch_bounds__(kOutThreads, 1) output_kernel(
             if (np <= wid) {
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4(b_nmajor_256(ks, np * 16, kk, lane), b0, b1, b2, b3);
-                mma16816(acc[2 * np], a, b0, b1);
-                mma16816(acc[2 * np + 1], a, b2, b3);
+                mma16816_bf16(acc[2 * np], a, b0, b1);
+                mma16816_bf16(acc[2 * np + 1], a, b2, b3);
             }
         }
     }
+    __syncthreads();  // every warp is done with the bf16 q rows
+    // q to fp16 in place for the q S product (each thread converts the chunks it copied)
+    for (int e = tid; e < 128 * 16; e += kOutThreads) bf16_chunk_to_fp16(smem + OO_Q + sw256(e >> 4, e & 15));
+    __syncthreads();
+    // P as fp16 A fragments: pa[j] is k block j (columns 16j..16j+15) of this warp's 16 rows
+    uint32_t pa[8][4];
 #pragma unroll
     for (int nt = 0; nt < 16; ++nt) {
-        if ((nt >> 1) <= wid) {
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                const int row = m0 + gid + hf * 8;
-                const int col = nt * 8 + tig * 2;
-                float p0 = 0.f, p1 = 0.f;
+        for (int hf = 0; hf < 2; ++hf) {
+            const int row = m0 + gid + hf * 8;
+            const int col = nt * 8 + tig * 2;
+            float p0 = 0.f, p1 = 0.f;
+            if ((nt >> 1) <= wid) {
                 const float fr = rqv[row];
                 if (col <= row) p0 = fr * rkv[col] * acc[nt][2 * hf] * __expf(gam[row] - gam[col]);
                 if (col + 1 <= row) p1 = fr * rkv[col + 1] * acc[nt][2 * hf + 1] * __expf(gam[row] - gam[col + 1]);
-                *reinterpret_cast<uint32_t *>(Ps + el256(row, col)) = pack_h2(p0, p1);
             }
+            pa[nt >> 1][(nt & 1) * 2 + hf] = pack_h2(p0, p1);
         }
     }
-    __syncwarp();
 
     // ---- o = diag(rq e^gamma) Q S_c + P U'
 #pragma unroll
@@ -125,15 +127,16 @@ __global__ void __launch_bounds__(kOutThreads, 1) output_kernel(
             acc[nt][3] *= f1;
         }
     }
-    for (int kk = 0; kk < (wid + 1) * 16; kk += 16) {
-        uint32_t a[4];
-        ldsm_x4(a_rowmajor_256(ps, m0, kk, lane), a[0], a[1], a[2], a[3]);
 #pragma unroll
-        for (int np = 0; np < 8; ++np) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(b_kmajor_256(us, np * 16, kk, lane), b0, b1, b2, b3);
-            mma16816(acc[2 * np], a, b0, b1);
-            mma16816(acc[2 * np + 1], a, b2, b3);
+    for (int j = 0; j < 8; ++j) {
+        if (j <= wid) {
+#pragma unroll
+            for (int np = 0; np < 8; ++np) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(b_kmajor_256(us, np * 16, j * 16, lane), b0, b1, b2, b3);
+                mma16816(acc[2 * np], pa[j], b0, b1);
+                mma16816(acc[2 * np + 1], pa[j], b2, b3);
+            }
         }
     }
 #pragma unroll
