@@ -54,7 +54,7 @@ def lib():
         L.gdn_chunk_fwd_noalloc.restype = ctypes.c_int
         L.gdn_chunk_fwd_noalloc.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, i32, p]
         L.gdn_selftest_umma.restype = ctypes.c_int
-        L.gdn_selftest_umma.argtypes = [p, p, p, i32, i32, i32, p, p]
+        L.gdn_selftest_umma.argtypes = [p, p, p, i32, i32, i32, i32, i32, p, p]
         L.gdn_short_fwd.restype = ctypes.c_int
         L.gdn_short_fwd.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, p]
         L.gdn_stage_chunk_map.restype = ctypes.c_int

@@ -1,8 +1,8 @@
 // Self-test of the tcgen05 path (test hook, include/gdn_testing.h): one CTA
-// computes C[128, N] = A[128, K] B[N, K]^T with both operands staged K-major
-// with the 128-byte swizzle, the product accumulated in TMEM and read back
-// with tcgen05.ld -- the same descriptor, swizzle and TMEM conventions that
-// the state kernel uses.
+// computes C[128, N] = sum_k A(m, k) B(n, k) with each operand staged either
+// K-major (128-byte swizzle) or MN-major (128-byte swizzle, or 64-byte for
+// N = 32), the product accumulated in TMEM and read back with tcgen05.ld --
+// the descriptor, swizzle and TMEM conventions that the kernels build on.
 #include "common.cuh"
 #include "gdn_internal.h"
 #include "gdn_testing.h"
@@ -12,7 +12,7 @@ namespace gdn {
 
 __global__ void __launch_bounds__(128, 1)
     umma_selftest_kernel(const uint16_t *__restrict__ A, const uint16_t *__restrict__ Bm, float *__restrict__ C,
-                         int N, int K, int bf16, int32_t *__restrict__ status)
+                         int N, int K, int bf16, int a_mn, int b_mn, int32_t *__restrict__ status)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // the swizzle atoms need 1024-byte alignment of the shared-memory address itself
@@ -25,15 +25,36 @@ __global__ void __launch_bounds__(128, 1)
     uint32_t *slot = reinterpret_cast<uint32_t *>(bar + 1);
     const uint32_t ncols = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
 
-    for (int e = tid; e < 128 * (K / 8); e += 128) {
-        const int r = e / (K / 8), c = e % (K / 8);
-        *reinterpret_cast<uint4 *>(sA + (c / 8) * 128 * 128 + tc::sw128c(r, c % 8)) =
-            *reinterpret_cast<const uint4 *>(A + (size_t)r * K + c * 8);
+    if (!a_mn) {  // A given as [128][K]
+        for (int e = tid; e < 128 * (K / 8); e += 128) {
+            const int r = e / (K / 8), c = e % (K / 8);
+            *reinterpret_cast<uint4 *>(sA + (c / 8) * 128 * 128 + tc::sw128c(r, c % 8)) =
+                *reinterpret_cast<const uint4 *>(A + (size_t)r * K + c * 8);
+        }
+    } else {      // A given as [K][128]: K rows of two 64-element MN halves
+        for (int e = tid; e < K * 16; e += 128) {
+            const int r = e / 16, c = e % 16;
+            *reinterpret_cast<uint4 *>(sA + (c / 8) * K * 128 + tc::sw128c(r, c % 8)) =
+                *reinterpret_cast<const uint4 *>(A + (size_t)r * 128 + c * 8);
+        }
     }
-    for (int e = tid; e < N * (K / 8); e += 128) {
-        const int r = e / (K / 8), c = e % (K / 8);
-        *reinterpret_cast<uint4 *>(sB + (c / 8) * N * 128 + tc::sw128c(r, c % 8)) =
-            *reinterpret_cast<const uint4 *>(Bm + (size_t)r * K + c * 8);
+    if (!b_mn) {  // B given as [N][K]
+        for (int e = tid; e < N * (K / 8); e += 128) {
+            const int r = e / (K / 8), c = e % (K / 8);
+            *reinterpret_cast<uint4 *>(sB + (c / 8) * N * 128 + tc::sw128c(r, c % 8)) =
+                *reinterpret_cast<const uint4 *>(Bm + (size_t)r * K + c * 8);
+        }
+    } else if (N == 32) {  // B given as [K][32]: 64-byte K rows, 64-byte swizzle
+        for (int e = tid; e < K * 4; e += 128) {
+            const int r = e / 4, c = e % 4;
+            *reinterpret_cast<uint4 *>(sB + sw64(r, c)) = *reinterpret_cast<const uint4 *>(Bm + (size_t)r * 32 + c * 8);
+        }
+    } else {      // B given as [K][N]: K rows of N/64 MN halves of 128 bytes
+        for (int e = tid; e < K * (N / 8); e += 128) {
+            const int r = e / (N / 8), c = e % (N / 8);
+            *reinterpret_cast<uint4 *>(sB + (c / 8) * K * 128 + tc::sw128c(r, c % 8)) =
+                *reinterpret_cast<const uint4 *>(Bm + (size_t)r * N + c * 8);
+        }
     }
     if (tid == 0) {
         tc::mbar_init(smem_addr(bar), 1);
@@ -47,10 +68,14 @@ __global__ void __launch_bounds__(128, 1)
     const uint32_t tmem = *slot;
 
     if (tid == 0) {
-        const uint32_t idesc = tc::idesc_f16(128, N, bf16 != 0, bf16 != 0);
+        const uint32_t idesc = tc::idesc_f16(128, N, bf16 != 0, bf16 != 0, a_mn != 0, b_mn != 0);
+        const uint32_t a0 = smem_addr(sA), b0 = smem_addr(sB);
         for (int kk = 0; kk < K / 16; ++kk) {
-            const uint64_t ad = tc::desc_k128(smem_addr(sA) + (kk / 4) * 128 * 128 + (kk % 4) * 32);
-            const uint64_t bd = tc::desc_k128(smem_addr(sB) + (kk / 4) * N * 128 + (kk % 4) * 32);
+            const uint64_t ad = a_mn ? tc::desc_mn(a0 + kk * 2048, K * 128, 1024, 2)
+                                     : tc::desc_k128(a0 + (kk / 4) * 128 * 128 + (kk % 4) * 32);
+            const uint64_t bd = !b_mn     ? tc::desc_k128(b0 + (kk / 4) * N * 128 + (kk % 4) * 32)
+                                : N == 32 ? tc::desc_mn(b0 + kk * 1024, 0, 512, 4)
+                                          : tc::desc_mn(b0 + kk * 2048, K * 128, 1024, 2);
             tc::mma_f16(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
         }
         tc::commit(smem_addr(bar));
@@ -76,13 +101,13 @@ __global__ void __launch_bounds__(128, 1)
 }  // namespace gdn
 
 extern "C" int gdn_selftest_umma(const uint16_t *A, const uint16_t *B, float *C, int32_t N, int32_t K,
-                                 int32_t bf16, int32_t *status, void *stream)
+                                 int32_t bf16, int32_t a_mn, int32_t b_mn, int32_t *status, void *stream)
 {
     if (!A || !B || !C || !status) return GDN_ERR_NULL_ARG;
     if (!(N == 32 || N == 64 || N == 128 || N == 256) || !(K == 64 || K == 128)) return GDN_ERR_BAD_SHAPE;
     const int smem = (K / 64) * (128 + N) * 128 + 64 + 1024;
     cudaError_t e = cudaFuncSetAttribute(gdn::umma_selftest_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
-    gdn::umma_selftest_kernel<<<1, 128, smem, (cudaStream_t)stream>>>(A, B, C, N, K, bf16, status);
+    gdn::umma_selftest_kernel<<<1, 128, smem, (cudaStream_t)stream>>>(A, B, C, N, K, bf16, a_mn, b_mn, status);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

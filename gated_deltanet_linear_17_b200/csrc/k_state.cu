@@ -1,211 +1,287 @@
-// Inter-chunk state passing: one CTA per (sequence, v-head, 32-column slice of Dv).
+// Inter-chunk state passing on the Blackwell tensor core: one CTA (8 warps) per
+// (sequence, v-head, 32-column slice of Dv).
 //
 // Page "Qwen3Next Samples", "Recurrent State Attention" and "State Update",
 // with the state held as S[Dk, Dv]:
 //   v'    = k_cumdecay S                 -> U' = U - W S
 //   S_new = S exp(g_last) + k_gexp^T (v_out - v'),  k_gexp = kh (.) exp(g_last - g_cum)
-// g_last is the cumulative gate at the chunk's last valid token.  The CTA
-// walks its sequence's chunks in order; the fp32 state slice [128 x 32] never
-// leaves registers (16 warps, each 16 rows of Dk x 16 columns).  Each step writes the fp16 state
-// entering the chunk (S_c) and U' for the output kernel.  The next chunk's W,
-// k and U tiles are prefetched with cp.async while the current one computes.
-// The state update multiplies the raw bf16 k rows (exact) by the decayed U'
-// operand Ub = diag(rk e^{g_last - gamma}) U', with the normalisation 1/|k|
-// folded in; Ub is split into two bf16 halves (hi + lo, ~16 significant bits)
-// so the update keeps near-fp32 accuracy.  W S uses fp16 operands;
-// accumulation is fp32 throughout.
+// g_last is the cumulative gate at the chunk's last valid token.  The CTA walks
+// its sequence's chunks in order.  Warp w owns rows 32(w%4)..32(w%4)+31 and
+// columns 16(w/4)..16(w/4)+15 of the slice: each thread keeps 16 fp32 values of
+// one row of the state S in registers for the whole sequence, and handles the
+// same 16 values of one row of U'.  Per chunk:
+//   1. W S     -- tcgen05.mma M=128 (L), N=32, K=128 (Dk), fp16: A = W
+//                 (K-major), B = S (MN-major, as the threads store it); fp32
+//                 accumulator in TMEM.
+//   2. U' = U - W S (tcgen05.ld), written to Up; the decayed operand
+//      Ub = diag(rk e^{g_last - gamma}) U' is split into bf16 hi + lo (~16
+//      significant bits) and stored row-wise (MN-major).
+//   3. K^T Ub  -- tcgen05.mma M=128 (Dk), N=32, K=128 (L), bf16: A = the raw k
+//                 tile read MN-major (no transpose), B = Ub hi then lo, both
+//                 accumulated into a second TMEM tile.
+//   4. S = e^{g_last} S + K^T Ub (tcgen05.ld); S in fp16 becomes the next B
+//      operand and, as the state entering the next chunk, goes to Sc.
+// The next chunk's W, k, U, gamma and 1/|k| are prefetched with cp.async.  One
+// thread issues the MMAs and waits for their completion (an mbarrier arrival
+// from tcgen05.commit); a CTA barrier passes the outcome on.  Every wait is
+// bounded: if one gives up, the CTA sets bit 0 of status[2] in the workspace,
+// stops, lets its MMAs drain and frees its tensor memory.
 #include "common.cuh"
 #include "gdn_internal.h"
+#include "tc100.cuh"
 
 namespace gdn {
 
-constexpr int kStateThreads = 512;
+constexpr int kStateThreads = 256;
 constexpr int DVT = 32;  // Dv columns per CTA
 
-// per stage: W [128][128] fp16, K [128][128] bf16, U slice [128][32] fp16, gam[128], rkv[128]
-constexpr int ST_W = 0, ST_K = 32768, ST_U = 65536, ST_G = 73728, ST_R = 74240;
-constexpr int kStageBytes = 74752;
-constexpr int OFF_SB = 2 * kStageBytes;      // fp16 [128 (Dk)][32] state operand
-constexpr int OFF_UB = OFF_SB + 128 * 64;    // bf16 [128 (L)][32] decayed U' operand, high half
-constexpr int OFF_UL = OFF_UB + 128 * 64;    // bf16 [128 (L)][32] decayed U' operand, low half
-constexpr int kStateSmem = OFF_UL + 128 * 64;
+// shared memory, relative to a 1024-byte aligned base (bytes)
+constexpr int ST_W = 0;             // fp16 W, K-major over Dk, 128B swizzle: 2 halves x 128 rows x 128 B
+constexpr int ST_K = 32768;         // bf16 k, MN-major over Dk (K rows = L), 128B swizzle: 2 halves x 128 x 128 B
+constexpr int ST_U = 65536;         // fp16 U slice [L][32], 64-byte rows, 64B swizzle
+constexpr int ST_G = 73728;         // fp32 gamma[128]
+constexpr int ST_R = 74240;         // fp32 1/|k| [128]
+constexpr int kStageBytes = 75776;  // rounded up to a multiple of 1024
+constexpr int OFF_S = 2 * kStageBytes;  // fp16 S [Dk][32], MN-major, 64B swizzle
+constexpr int OFF_UH = OFF_S + 8192;    // bf16 Ub high half [L][32], MN-major, 64B swizzle
+constexpr int OFF_UL = OFF_UH + 8192;   // bf16 Ub low half
+constexpr int OFF_BAR = OFF_UL + 8192;  // 2 mbarriers + TMEM address slot
+constexpr int kStateSmem = OFF_BAR + 64 + 1024;  // + alignment slack
 
 __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
     const uint16_t *__restrict__ k, const float *__restrict__ pool, const int32_t *__restrict__ idx,
     float *__restrict__ final_state, int T, int Nqk, int Nv, const int4 *__restrict__ info,
     const int32_t *__restrict__ seq_chunk0, const float *__restrict__ rk, const float *__restrict__ gcum,
     const uint16_t *__restrict__ U, const uint16_t *__restrict__ W, uint16_t *__restrict__ Up,
-    uint16_t *__restrict__ Sc)
+    uint16_t *__restrict__ Sc, int32_t *__restrict__ status)
 {
-    extern __shared__ __align__(1024) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
+    const uint32_t sbase = smem_addr(smem);
     const int b = blockIdx.x, h = blockIdx.y, col0 = blockIdx.z * DVT;
     const int hq = h / (Nv / Nqk);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int gid = lane >> 2, tig = lane & 3;
-    // warp = (row block, column half): 16 rows (of Dk for the state, of L for U') x 16 columns
-    const int r0 = (wid & 7) * 16, cb = (wid >> 3) * 16;
+    const int quarter = wid & 3, half = wid >> 2;
+    const int row = quarter * 32 + lane;  // row of the state (Dk) and of U' (L)
+    const int cbase = half * 16;          // first of this thread's 16 columns in the slice
     const int c_begin = seq_chunk0[b], c_end = seq_chunk0[b + 1];
-    // tokens of the sequence (the chunks of a sequence are consecutive 128-token runs)
     const int seq_t0 = c_begin < c_end ? info[c_begin].y : 0;
     const int seq_t1 = c_begin < c_end ? info[c_end - 1].y + info[c_end - 1].z : 0;
 
-    // state slice: s[nt][e] is S[r0 + gid + 8*(e>>1)][col0 + cb + nt*8 + tig*2 + (e&1)]
-    float s[2][4];
-    {
-        const float *src = nullptr;
-        if (pool) {
-            const int slot = idx ? idx[b] : b;
-            src = pool + ((size_t)slot * Nv + h) * D * D;
-        }
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                const int row = r0 + gid + hf * 8;
-                const int col = col0 + cb + nt * 8 + tig * 2;
-                float2 x = make_float2(0.f, 0.f);
-                if (src) x = *reinterpret_cast<const float2 *>(src + (size_t)row * D + col);
-                s[nt][2 * hf] = x.x;
-                s[nt][2 * hf + 1] = x.y;
-            }
+    const uint32_t bar_ws = sbase + OFF_BAR, bar_up = sbase + OFF_BAR + 8;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 16);
+    if (tid == 0) {
+        tc::mbar_init(bar_ws, 1);
+        tc::mbar_init(bar_up, 1);
+        tc::mbar_init_fence();
     }
+    if (wid == 0) tc::tmem_alloc(smem_addr(tslot), 64);
 
+    // initial state: this thread's 16 values
+    float s[16];
+    if (pool) {
+        const int slot = idx ? idx[b] : b;
+        const float4 *src =
+            reinterpret_cast<const float4 *>(pool + (((size_t)slot * Nv + h) * D + row) * D + col0 + cbase);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 x = src[j];
+            s[4 * j] = x.x;
+            s[4 * j + 1] = x.y;
+            s[4 * j + 2] = x.z;
+            s[4 * j + 3] = x.w;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) s[j] = 0.f;
+    }
+    // S in fp16 as the MN-major B operand: row `row`, 16-byte chunks (cbase/8, cbase/8 + 1)
+    auto store_state_operand = [&]() {
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+            *reinterpret_cast<uint4 *>(smem + OFF_S + sw64(row, (cbase >> 3) + j)) =
+                make_uint4(pack_h2(s[8 * j], s[8 * j + 1]), pack_h2(s[8 * j + 2], s[8 * j + 3]),
+                           pack_h2(s[8 * j + 4], s[8 * j + 5]), pack_h2(s[8 * j + 6], s[8 * j + 7]));
+    };
+    store_state_operand();
+
+    // per-thread constant parts of the prefetch addresses
+    const int wr = tid >> 4, wc = tid & 15;  // W / k pieces: rows wr + 16 j, chunk wc
+    const uint32_t w_dst = (uint32_t)((wc >> 3) * 16384) + tc::sw128c(wr, wc & 7);
+    const int ur = tid >> 2, uc = tid & 3;   // U pieces: rows ur + 64 j, chunk uc
+    const uint32_t u_dst = sw64(ur, uc);
     auto issue = [&](int c, int st) {
         const int cstart = seq_t0 + (c - c_begin) * L, clen = min(L, seq_t1 - cstart);
-        uint8_t *base = smem + st * kStageBytes;
-        const uint32_t wsa = smem_addr(base + ST_W), ksa = smem_addr(base + ST_K), usa = smem_addr(base + ST_U);
-        const uint16_t *wsrc = W + (size_t)(c * Nv + h) * L * D;
-        const uint16_t *usrc = U + (size_t)(c * Nv + h) * L * D + col0;
-        for (int e = tid; e < 128 * 16; e += kStateThreads) {
-            const int r = e >> 4, cc = e & 15;
-            cp_async16(wsa + sw256(r, cc), wsrc + r * D + cc * 8, true);
-            const bool ok = r < clen;
-            const int t = cstart + (ok ? r : 0);
-            cp_async16(ksa + sw256(r, cc), k + ((size_t)t * Nqk + hq) * D + cc * 8, ok);
+        const uint32_t base = sbase + st * kStageBytes;
+        const uint16_t *wsrc = W + (size_t)(c * Nv + h) * L * D + wr * D + wc * 8;
+        const uint16_t *ksrc = k + ((size_t)cstart * Nqk + hq) * D + wc * 8;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int r = wr + 16 * j;
+            cp_async16(base + ST_W + w_dst + j * 2048, wsrc + (size_t)j * 16 * D, true);
+            const bool valid = r < clen;
+            cp_async16(base + ST_K + w_dst + j * 2048, ksrc + (size_t)(valid ? r : 0) * Nqk * D, valid);
         }
-        {
-            const int r = tid >> 2, cc = tid & 3;  // 512 pieces: one per thread
-            cp_async16(usa + sw64(r, cc), usrc + r * D + cc * 8, true);
-        }
-        // gamma (clamped to the last valid row) and 1/|k| (rows past the chunk read a real row; they
-        // multiply zero rows of U' and K)
+        const uint16_t *usrc = U + (size_t)(c * Nv + h) * L * D + col0 + ur * D + uc * 8;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) cp_async16(base + ST_U + u_dst + j * 4096, usrc + (size_t)j * 64 * D, true);
         if (tid < 128) {
+            // gamma (clamped to the last valid row) and 1/|k|; rows past the chunk multiply zeros
             const int i = min(tid, clen - 1);
-            cp_async4(smem_addr(base + ST_G) + tid * 4, gcum + (size_t)h * T + cstart + i);
-            cp_async4(smem_addr(base + ST_R) + tid * 4, rk + (size_t)hq * T + cstart + i);
+            cp_async4(base + ST_G + tid * 4, gcum + (size_t)h * T + cstart + i);
+            cp_async4(base + ST_R + tid * 4, rk + (size_t)hq * T + cstart + i);
         }
     };
 
-    uint8_t *Sb = smem + OFF_SB, *Ub = smem + OFF_UB, *Ul = smem + OFF_UL;
-    const uint32_t sba = smem_addr(Sb), uba = smem_addr(Ub), ula = smem_addr(Ul);
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tslot;  // columns [0, 32): W S; [32, 64): K^T Ub
+    const uint32_t t_mine = tmem + ((uint32_t)(quarter * 32) << 16) + cbase;
+    const uint32_t idesc_ws = tc::idesc_f16(128, 32, false, false, false, true);
+    const uint32_t idesc_up = tc::idesc_f16(128, 32, true, true, true, true);
+    bool ok = true;
 
     if (c_begin < c_end) issue(c_begin, 0);
     cp_async_commit();
     for (int c = c_begin, it = 0; c < c_end; ++c, ++it) {
         const int st = it & 1;
+        const uint32_t parity = (uint32_t)(it & 1);
         if (c + 1 < c_end) issue(c + 1, st ^ 1);
         cp_async_commit();
         cp_async_wait<1>();
-
         const int clen = min(L, seq_t1 - (seq_t0 + (c - c_begin) * L));
         uint8_t *base = smem + st * kStageBytes;
-        const uint32_t wsa = smem_addr(base + ST_W), ksa = smem_addr(base + ST_K);
-        const uint8_t *Us = base + ST_U;
+        const uint32_t abase = sbase + st * kStageBytes;
         const float *gam = reinterpret_cast<const float *>(base + ST_G);
         const float *rkv = reinterpret_cast<const float *>(base + ST_R);
         const size_t tile = (size_t)(c * Nv + h) * L * D;
 
-        // (1) state entering the chunk: fp16 copy to shared (MMA operand) and to Sc
+        // state entering the chunk -> Sc (fp16)
+        {
+            uint4 *dst = reinterpret_cast<uint4 *>(Sc + tile + (size_t)row * D + col0 + cbase);
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                const int row = r0 + gid + hf * 8;
-                const int col = cb + nt * 8 + tig * 2;
-                const uint32_t p = pack_h2(s[nt][2 * hf], s[nt][2 * hf + 1]);
-                *reinterpret_cast<uint32_t *>(Sb + el64(row, col)) = p;
-                *reinterpret_cast<uint32_t *>(Sc + tile + (size_t)row * D + col0 + col) = p;
-            }
-        __syncthreads();
-
-        // (2) WS = W S for L rows r0..r0+15, columns cb..cb+15 (K = Dk)
-        float wsacc[2][4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) wsacc[nt][0] = wsacc[nt][1] = wsacc[nt][2] = wsacc[nt][3] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < D; kk += 16) {
-            uint32_t a[4], b0, b1, b2, b3;
-            ldsm_x4(a_rowmajor_256(wsa, r0, kk, lane), a[0], a[1], a[2], a[3]);
-            ldsm_x4_t(b_kmajor_64(sba, cb, kk, lane), b0, b1, b2, b3);
-            mma16816(wsacc[0], a, b0, b1);
-            mma16816(wsacc[1], a, b2, b3);
+            for (int j = 0; j < 2; ++j)
+                dst[j] = make_uint4(pack_h2(s[8 * j], s[8 * j + 1]), pack_h2(s[8 * j + 2], s[8 * j + 3]),
+                                    pack_h2(s[8 * j + 4], s[8 * j + 5]), pack_h2(s[8 * j + 6], s[8 * j + 7]));
         }
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
 
-        // (3) U' = U - W S -> Up; Ub = diag(rk e^{g_last - gamma}) U' as hi + lo (operand of the update)
-        const float gl = gam[clen - 1];
+        // (1) W S
+        if (tid == 0) {
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            const int row = r0 + gid + hf * 8;
+            for (int kk = 0; kk < 8; ++kk)
+                tc::mma_f16(tmem, tc::desc_k128(abase + ST_W + (kk >> 2) * 16384 + (kk & 3) * 32),
+                            tc::desc_mn(sbase + OFF_S + kk * 1024, 0, 512, 4), idesc_ws, kk > 0 ? 1u : 0u);
+            tc::commit(bar_ws);
+        }
+        {
+            bool w_ok = true;
+            if (tid == 0) w_ok = tc::mbar_wait_bounded(bar_ws, parity);
+            tc::fence_before_sync();
+            ok = __syncthreads_and(w_ok) != 0;
+            tc::fence_after_sync();
+        }
+        if (!ok) break;
+
+        // (2) U' = U - W S -> Up; Ub hi / lo
+        {
+            float ws[16];
+            tc::tmem_ld16(t_mine, ws);
+            const float gl = gam[clen - 1];
             const float sc = rkv[row] * __expf(gl - gam[row]);
+            uint4 *updst = reinterpret_cast<uint4 *>(Up + tile + (size_t)row * D + col0 + cbase);
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const int col = cb + nt * 8 + tig * 2;
-                const float2 u = unpack_h2(*reinterpret_cast<const uint32_t *>(Us + el64(row, col)));
-                const float p0 = u.x - wsacc[nt][2 * hf];
-                const float p1 = u.y - wsacc[nt][2 * hf + 1];
-                *reinterpret_cast<uint32_t *>(Up + tile + (size_t)row * D + col0 + col) = pack_h2(p0, p1);
-                uint32_t hi, lo;
-                split_bf2(p0 * sc, p1 * sc, hi, lo);
-                *reinterpret_cast<uint32_t *>(Ub + el64(row, col)) = hi;
-                *reinterpret_cast<uint32_t *>(Ul + el64(row, col)) = lo;
+            for (int j = 0; j < 2; ++j) {
+                const uint4 uu = *reinterpret_cast<const uint4 *>(base + ST_U + sw64(row, (cbase >> 3) + j));
+                const uint32_t w4[4] = {uu.x, uu.y, uu.z, uu.w};
+                uint32_t o4[4], h4[4], l4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 u = unpack_h2(w4[e]);
+                    const float p0 = u.x - ws[8 * j + 2 * e], p1 = u.y - ws[8 * j + 2 * e + 1];
+                    o4[e] = pack_h2(p0, p1);
+                    split_bf2(p0 * sc, p1 * sc, h4[e], l4[e]);
+                }
+                updst[j] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                *reinterpret_cast<uint4 *>(smem + OFF_UH + sw64(row, (cbase >> 3) + j)) =
+                    make_uint4(h4[0], h4[1], h4[2], h4[3]);
+                *reinterpret_cast<uint4 *>(smem + OFF_UL + sw64(row, (cbase >> 3) + j)) =
+                    make_uint4(l4[0], l4[1], l4[2], l4[3]);
             }
         }
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
         __syncthreads();
+        tc::fence_after_sync();
 
-        // (4) S = e^{g_last} S + K^T (Ub_hi + Ub_lo) for Dk rows r0..r0+15, columns cb..cb+15 (K = L)
-        const float dg = __expf(gl);
+        // (3) K^T (Ub_hi + Ub_lo)
+        if (tid == 0) {
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) s[nt][e] *= dg;
-#pragma unroll
-        for (int kk = 0; kk < L; kk += 16) {
-            uint32_t a[4], b0, b1, b2, b3;
-            ldsm_x4_t(a_colmajor_256(ksa, r0, kk, lane), a[0], a[1], a[2], a[3]);
-            ldsm_x4_t(b_kmajor_64(uba, cb, kk, lane), b0, b1, b2, b3);
-            mma16816_bf16(s[0], a, b0, b1);
-            mma16816_bf16(s[1], a, b2, b3);
-            ldsm_x4_t(b_kmajor_64(ula, cb, kk, lane), b0, b1, b2, b3);
-            mma16816_bf16(s[0], a, b0, b1);
-            mma16816_bf16(s[1], a, b2, b3);
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t ad = tc::desc_mn(abase + ST_K + kk * 2048, 16384, 1024, 2);
+                tc::mma_f16(tmem + 32, ad, tc::desc_mn(sbase + OFF_UH + kk * 1024, 0, 512, 4), idesc_up,
+                            kk > 0 ? 1u : 0u);
+                tc::mma_f16(tmem + 32, ad, tc::desc_mn(sbase + OFF_UL + kk * 1024, 0, 512, 4), idesc_up, 1u);
+            }
+            tc::commit(bar_up);
         }
-        __syncthreads();
+        {
+            bool w_ok = true;
+            if (tid == 0) w_ok = tc::mbar_wait_bounded(bar_up, parity);
+            tc::fence_before_sync();
+            ok = __syncthreads_and(w_ok) != 0;
+            tc::fence_after_sync();
+        }
+        if (!ok) break;
+
+        // (4) S = e^{g_last} S + K^T Ub; the next chunk's B operand
+        {
+            float up[16];
+            tc::tmem_ld16(t_mine + 32, up);
+            const float dg = __expf(gam[clen - 1]);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) s[j] = dg * s[j] + up[j];
+        }
+        store_state_operand();
+        tc::fence_before_sync();
+        __syncthreads();  // stage `st`, Ub and the TMEM tiles are free for the next chunk
+        tc::fence_after_sync();
     }
     cp_async_wait<0>();
 
-    if (final_state) {
-        float *dst = final_state + ((size_t)b * Nv + h) * D * D;
+    if (!ok) {
+        if (tid == 0) {
+            atomicOr(status + 2, 1);
+            // give the MMAs already issued time to finish before the tensor memory is released
+            tc::mbar_wait_bounded(bar_ws, 0);
+            tc::mbar_wait_bounded(bar_up, 0);
+        }
+    } else if (final_state) {
+        float4 *dst =
+            reinterpret_cast<float4 *>(final_state + (((size_t)b * Nv + h) * D + row) * D + col0 + cbase);
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                const int row = r0 + gid + hf * 8;
-                const int col = col0 + cb + nt * 8 + tig * 2;
-                *reinterpret_cast<float2 *>(dst + (size_t)row * D + col) = make_float2(s[nt][2 * hf], s[nt][2 * hf + 1]);
-            }
+        for (int j = 0; j < 4; ++j) dst[j] = make_float4(s[4 * j], s[4 * j + 1], s[4 * j + 2], s[4 * j + 3]);
     }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (wid == 0) tc::tmem_dealloc(tmem, 64);
 }
 
 cudaError_t launch_state(const uint16_t *k, const float *pool, const int32_t *idx, float *final_state, int T, int B,
                          int Nqk, int Nv, const Workspace &ws, cudaStream_t st)
 {
     if (B == 0) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kStateSmem);
+    cudaError_t e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStateSmem);
     if (e != cudaSuccess) return e;
     state_kernel<<<dim3(B, Nv, D / DVT), kStateThreads, kStateSmem, st>>>(
         k, pool, idx, final_state, T, Nqk, Nv, ws.chunk_info, ws.seq_chunk0, ws.rk, ws.gcum, ws.U, ws.W, ws.Up,
-        ws.Sc);
+        ws.Sc, ws.status);
     return cudaGetLastError();
 }
 

@@ -1,12 +1,21 @@
 // Blackwell (sm_100a) tensor-core helpers: TMEM allocation, tcgen05.mma with
 // shared-memory descriptors, tcgen05.commit to an mbarrier, tcgen05.ld.
 //
-// Operand tiles are K-major with the 128-byte swizzle: a tile of R rows and
-// 64 16-bit elements (128 bytes) of K is stored row after row, and inside each
+// K-major operand tiles use the 128-byte swizzle: a tile of R rows and 64
+// 16-bit elements (128 bytes) of K is stored row after row, and inside each
 // 8-row, 1024-byte atom the 16-byte chunk c of row r sits at chunk c ^ (r & 7).
 // A K extent of 128 elements is two such tiles ("K halves") one after the
 // other.  One MMA consumes 16 elements of K (32 bytes of each row), so the
 // descriptor of k step kk starts (kk % 4) * 32 bytes into K half kk / 4.
+//
+// MN-major operand tiles store rows of K: each K row holds the M (or N)
+// elements contiguously.  With the 128-byte swizzle a K row carries 64
+// elements (128 bytes) and M = 128 is two such "MN halves" one after the
+// other (leading byte offset = the size of one half); 8 K rows form a
+// 1024-byte atom (stride byte offset 1024), chunk c of K row r at c ^ (r & 7).
+// With the 64-byte swizzle a K row carries 32 elements (64 bytes), 8 K rows
+// form a 512-byte atom (stride byte offset 512), chunk c of K row r at
+// c ^ ((r >> 1) & 3).  One MMA consumes 16 K rows = two atoms.
 // Every tile must start on a 1024-byte boundary.
 #pragma once
 
@@ -37,11 +46,27 @@ __device__ __forceinline__ uint64_t desc_k128(uint32_t smem_byte_addr)
     return d;
 }
 
-// instruction descriptor of kind::f16 with fp32 accumulation, both operands K-major
-__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_bf16, bool b_bf16)
+// shared-memory matrix descriptor of an MN-major operand: `swz` is 2 (128-byte
+// swizzle) or 4 (64-byte swizzle); lbo = bytes between MN blocks, sbo = bytes
+// between 8-row K groups
+__device__ __forceinline__ uint64_t desc_mn(uint32_t smem_byte_addr, uint32_t lbo, uint32_t sbo, uint32_t swz)
 {
-    return (1u << 4) | ((a_bf16 ? 1u : 0u) << 7) | ((b_bf16 ? 1u : 0u) << 10) | ((uint32_t)(N >> 3) << 17) |
-           ((uint32_t)(M >> 4) << 24);
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_byte_addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)swz << 61;
+    return d;
+}
+
+// instruction descriptor of kind::f16 with fp32 accumulation; a_mn / b_mn select
+// MN-major (transposed) operands
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_bf16, bool b_bf16, bool a_mn = false,
+                                                 bool b_mn = false)
+{
+    return (1u << 4) | ((a_bf16 ? 1u : 0u) << 7) | ((b_bf16 ? 1u : 0u) << 10) | ((a_mn ? 1u : 0u) << 15) |
+           ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -93,6 +118,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v)
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 32 lanes x 16 consecutive fp32 columns: lane i of the warp gets row (lane base + i)
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v)
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // ------------------------------------------------------------------ mbarrier

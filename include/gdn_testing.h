@@ -1,13 +1,14 @@
 /*
  * gdn_testing.h -- test hooks of the library (not part of the operator).
  *
- * gdn_selftest_umma: one CTA computes C[128, N] = A[128, K] B[N, K]^T on the
- * Blackwell tensor core (tcgen05.mma, operands K-major with the 128-byte
- * swizzle in shared memory, fp32 accumulator in tensor memory, read back with
- * tcgen05.ld).  It checks the descriptor and layout conventions that the
- * kernels build on, in isolation.
- *   A       device fp16 (bf16 = 0) or bf16 (bf16 = 1) [128, K], row-major
- *   B       device, same type, [N, K], row-major
+ * gdn_selftest_umma: one CTA computes C[128, N] = sum_k A(m, k) B(n, k) on
+ * the Blackwell tensor core (tcgen05.mma from swizzled shared-memory tiles,
+ * fp32 accumulator in tensor memory, read back with tcgen05.ld).  It checks
+ * the descriptor and layout conventions that the kernels build on, in
+ * isolation, for K-major and MN-major operands.
+ *   A       device fp16 (bf16 = 0) or bf16 (bf16 = 1): [128, K] row-major
+ *           (a_mn = 0, K-major) or [K, 128] row-major (a_mn = 1, MN-major)
+ *   B       device, same type: [N, K] (b_mn = 0) or [K, N] (b_mn = 1)
  *   C       device fp32 [128, N]
  *   N       32, 64, 128 or 256;  K  64 or 128
  *   status  device int32, set to 1 if the completion wait gave up (0 is not
@@ -26,7 +27,7 @@ extern "C" {
 #endif
 
 int gdn_selftest_umma(const uint16_t *A, const uint16_t *B, float *C, int32_t N, int32_t K, int32_t bf16,
-                      int32_t *status, void *stream);
+                      int32_t a_mn, int32_t b_mn, int32_t *status, void *stream);
 
 #ifdef __cplusplus
 }
