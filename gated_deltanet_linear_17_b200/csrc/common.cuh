@@ -138,7 +138,8 @@ __device__ __forceinline__ uint16_t f2bf(float x)
 }
 __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi)
 {
-    return static_cast<uint32_t>(f2bf(lo)) | (static_cast<uint32_t>(f2bf(hi)) << 16);
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
 }
 // two floats -> packed fp16 pair (round to nearest even), low half first
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi)

@@ -21,7 +21,10 @@
 //                 accumulated into a second TMEM tile.
 //   4. S = e^{g_last} S + K^T Ub (tcgen05.ld); S in fp16 becomes the next B
 //      operand and, as the state entering the next chunk, goes to Sc.
-// The next chunk's W, k, U, gamma and 1/|k| are prefetched with cp.async.  One
+// The next chunk's W, k, U, gamma and 1/|k| are prefetched with cp.async while
+// the W S product runs, and each product is split into independent
+// accumulation chains (partial sums over halves of K, and the hi / lo halves of
+// Ub) that are added after one TMEM read, to shorten the serial chain.  One
 // thread issues the MMAs and waits for their completion (an mbarrier arrival
 // from tcgen05.commit); a CTA barrier passes the outcome on.  Every wait is
 // bounded: if one gives up, the CTA sets bit 0 of status[2] in the workspace,
@@ -75,7 +78,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
         tc::mbar_init(bar_up, 1);
         tc::mbar_init_fence();
     }
-    if (wid == 0) tc::tmem_alloc(smem_addr(tslot), 64);
+    if (wid == 0) tc::tmem_alloc(smem_addr(tslot), 256);
 
     // initial state: this thread's 16 values
     float s[16];
@@ -133,32 +136,51 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
         }
     };
 
+    if (c_begin < c_end) issue(c_begin, 0);
+    cp_async_commit();
+    cp_async_wait<0>();
     tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    const uint32_t tmem = *tslot;  // columns [0, 32): W S; [32, 64): K^T Ub
+    // TMEM columns: [0, 64) W S as two partial sums over the Dk halves;
+    // [64, 192) K^T Ub as four partial sums (L half x hi / lo)
+    const uint32_t tmem = *tslot;
     const uint32_t t_mine = tmem + ((uint32_t)(quarter * 32) << 16) + cbase;
     const uint32_t idesc_ws = tc::idesc_f16(128, 32, false, false, false, true);
     const uint32_t idesc_up = tc::idesc_f16(128, 32, true, true, true, true);
+    // Operand descriptors of k step 0 of each tile; the start-address field holds
+    // (byte address >> 4) and every address stays below 256 KiB, so the
+    // descriptor of a k step is the base descriptor plus (byte offset >> 4).
+    const uint64_t dW0 = tc::desc_k128(sbase + ST_W), dK0 = tc::desc_mn(sbase + ST_K, 16384, 1024, 2);
+    const uint64_t dS = tc::desc_mn(sbase + OFF_S, 0, 512, 4);
+    const uint64_t dUH = tc::desc_mn(sbase + OFF_UH, 0, 512, 4), dUL = tc::desc_mn(sbase + OFF_UL, 0, 512, 4);
     bool ok = true;
 
-    if (c_begin < c_end) issue(c_begin, 0);
-    cp_async_commit();
+    // Each iteration starts with the chunk's data and the state operand in
+    // shared memory (made visible to the tensor core before the barrier at the
+    // end of the previous iteration).
     for (int c = c_begin, it = 0; c < c_end; ++c, ++it) {
         const int st = it & 1;
         const uint32_t parity = (uint32_t)(it & 1);
-        if (c + 1 < c_end) issue(c + 1, st ^ 1);
-        cp_async_commit();
-        cp_async_wait<1>();
         const int clen = min(L, seq_t1 - (seq_t0 + (c - c_begin) * L));
         uint8_t *base = smem + st * kStageBytes;
-        const uint32_t abase = sbase + st * kStageBytes;
         const float *gam = reinterpret_cast<const float *>(base + ST_G);
         const float *rkv = reinterpret_cast<const float *>(base + ST_R);
         const size_t tile = (size_t)(c * Nv + h) * L * D;
 
-        // state entering the chunk -> Sc (fp16)
+        const uint64_t stage_off = (uint64_t)((st * kStageBytes) >> 4);
+        // (1) W S: two independent accumulation chains (Dk halves)
+        if (tid == 0) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                tc::mma_f16(tmem + (kk >> 2) * 32, dW0 + stage_off + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                            dS + (uint64_t)((kk * 1024) >> 4), idesc_ws, (kk & 3) ? 1u : 0u);
+            tc::commit(bar_ws);
+        }
+        // while it runs: prefetch the next chunk, write the entering state, read U and the row factor
+        if (c + 1 < c_end) issue(c + 1, st ^ 1);
+        cp_async_commit();
         {
             uint4 *dst = reinterpret_cast<uint4 *>(Sc + tile + (size_t)row * D + col0 + cbase);
 #pragma unroll
@@ -166,19 +188,12 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
                 dst[j] = make_uint4(pack_h2(s[8 * j], s[8 * j + 1]), pack_h2(s[8 * j + 2], s[8 * j + 3]),
                                     pack_h2(s[8 * j + 4], s[8 * j + 5]), pack_h2(s[8 * j + 6], s[8 * j + 7]));
         }
-        tc::fence_proxy_async();
-        tc::fence_before_sync();
-        __syncthreads();
-        tc::fence_after_sync();
-
-        // (1) W S
-        if (tid == 0) {
+        const float gl = gam[clen - 1];
+        const float sc = rkv[row] * __expf(gl - gam[row]);
+        const float dg = __expf(gl);
+        uint4 uu[2];
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                tc::mma_f16(tmem, tc::desc_k128(abase + ST_W + (kk >> 2) * 16384 + (kk & 3) * 32),
-                            tc::desc_mn(sbase + OFF_S + kk * 1024, 0, 512, 4), idesc_ws, kk > 0 ? 1u : 0u);
-            tc::commit(bar_ws);
-        }
+        for (int j = 0; j < 2; ++j) uu[j] = *reinterpret_cast<const uint4 *>(base + ST_U + sw64(row, (cbase >> 3) + j));
         {
             bool w_ok = true;
             if (tid == 0) w_ok = tc::mbar_wait_bounded(bar_ws, parity);
@@ -190,20 +205,19 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
 
         // (2) U' = U - W S -> Up; Ub hi / lo
         {
-            float ws[16];
+            float ws[16], ws2[16];
             tc::tmem_ld16(t_mine, ws);
-            const float gl = gam[clen - 1];
-            const float sc = rkv[row] * __expf(gl - gam[row]);
+            tc::tmem_ld16(t_mine + 32, ws2);
             uint4 *updst = reinterpret_cast<uint4 *>(Up + tile + (size_t)row * D + col0 + cbase);
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                const uint4 uu = *reinterpret_cast<const uint4 *>(base + ST_U + sw64(row, (cbase >> 3) + j));
-                const uint32_t w4[4] = {uu.x, uu.y, uu.z, uu.w};
+                const uint32_t w4[4] = {uu[j].x, uu[j].y, uu[j].z, uu[j].w};
                 uint32_t o4[4], h4[4], l4[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 u = unpack_h2(w4[e]);
-                    const float p0 = u.x - ws[8 * j + 2 * e], p1 = u.y - ws[8 * j + 2 * e + 1];
+                    const int i0 = 8 * j + 2 * e;
+                    const float p0 = u.x - (ws[i0] + ws2[i0]), p1 = u.y - (ws[i0 + 1] + ws2[i0 + 1]);
                     o4[e] = pack_h2(p0, p1);
                     split_bf2(p0 * sc, p1 * sc, h4[e], l4[e]);
                 }
@@ -219,14 +233,14 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
         __syncthreads();
         tc::fence_after_sync();
 
-        // (3) K^T (Ub_hi + Ub_lo)
+        // (3) K^T (Ub_hi + Ub_lo): four independent chains (L half x hi / lo)
         if (tid == 0) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t ad = tc::desc_mn(abase + ST_K + kk * 2048, 16384, 1024, 2);
-                tc::mma_f16(tmem + 32, ad, tc::desc_mn(sbase + OFF_UH + kk * 1024, 0, 512, 4), idesc_up,
-                            kk > 0 ? 1u : 0u);
-                tc::mma_f16(tmem + 32, ad, tc::desc_mn(sbase + OFF_UL + kk * 1024, 0, 512, 4), idesc_up, 1u);
+                const uint64_t ad = dK0 + stage_off + (uint64_t)((kk * 2048) >> 4);
+                const uint32_t acc = (kk & 3) ? 1u : 0u;
+                tc::mma_f16(tmem + 64 + (kk >> 2) * 32, ad, dUH + (uint64_t)((kk * 1024) >> 4), idesc_up, acc);
+                tc::mma_f16(tmem + 128 + (kk >> 2) * 32, ad, dUL + (uint64_t)((kk * 1024) >> 4), idesc_up, acc);
             }
             tc::commit(bar_up);
         }
@@ -241,15 +255,19 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
 
         // (4) S = e^{g_last} S + K^T Ub; the next chunk's B operand
         {
-            float up[16];
-            tc::tmem_ld16(t_mine + 32, up);
-            const float dg = __expf(gam[clen - 1]);
+            float p0[16], p1[16], p2[16], p3[16];
+            tc::tmem_ld16(t_mine + 64, p0);
+            tc::tmem_ld16(t_mine + 96, p1);
+            tc::tmem_ld16(t_mine + 128, p2);
+            tc::tmem_ld16(t_mine + 160, p3);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) s[j] = dg * s[j] + up[j];
+            for (int j = 0; j < 16; ++j) s[j] = dg * s[j] + ((p0[j] + p1[j]) + (p2[j] + p3[j]));
         }
         store_state_operand();
+        cp_async_wait<0>();  // the next chunk's data
+        tc::fence_proxy_async();
         tc::fence_before_sync();
-        __syncthreads();  // stage `st`, Ub and the TMEM tiles are free for the next chunk
+        __syncthreads();
         tc::fence_after_sync();
     }
     cp_async_wait<0>();
@@ -270,7 +288,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    if (wid == 0) tc::tmem_dealloc(tmem, 64);
+    if (wid == 0) tc::tmem_dealloc(tmem, 256);
 }
 
 cudaError_t launch_state(const uint16_t *k, const float *pool, const int32_t *idx, float *final_state, int T, int B,
