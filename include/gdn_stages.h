@@ -37,9 +37,9 @@ extern "C" {
  * sizes.  NC = max_chunks = floor((T + 127 B) / 128), an upper bound on the
  * number of chunks of any packing of T tokens into B sequences.
  *   status      int32[4]: [0] cu_seqlens error bits (1: cu[0] != 0, 2: decreasing,
- *               4: cu[B] != T), [1] number of chunks, [2] bit 0: a tensor-core
- *               completion wait of the state pass gave up (its results are then
- *               incomplete); the caller clears [2] if it wants to read it
+ *               4: cu[B] != T), [1] number of chunks, [2] tensor-core completion
+ *               waits that gave up (bit 0: state pass, bit 1: output; the
+ *               results are then incomplete); the caller clears [2] to read it
  *   chunk_info  int32[NC][4]: sequence, first token, tokens in the chunk (1..128),
  *               chunk index within its sequence; rows past the last chunk hold -1
  *   seq_chunk0  int32[B+1]: first chunk of each sequence, [B] = number of chunks

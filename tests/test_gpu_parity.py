@@ -167,6 +167,15 @@ def test_beta_zero_gives_exact_zeros():
     assert torch.count_nonzero(out) == 0 and torch.count_nonzero(fin) == 0
 
 
+@pytest.mark.parametrize("gate", [("uniform_neg", 30.0, 5.0), ("zero",)], ids=["strong_decay", "no_decay"])
+def test_gate_extremes(gate):
+    """Gates far below zero (e^gamma underflows inside a chunk) and gates of exactly zero."""
+    inp = inputs.make([300, 17, 129], Nqk=2, Nv=4, g=gate, state=("normal", 0.02, 3, "perm"), seed=14)
+    out, fin = _gpu(inp)
+    assert torch.isfinite(out.float()).all() and torch.isfinite(fin).all()
+    _check(inp, out, fin, what=f"gate {gate[0]}")
+
+
 def test_every_output_written_once_nan_canary():
     inp = inputs.make([130, 0, 77], Nqk=2, Nv=2, seed=9)
     d = inp.to(DEV)
