@@ -30,7 +30,7 @@ _lib = None
 
 class _Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
-                ("total", "status", "chunk_info", "seq_chunk0", "rq", "rk", "gcum", "betaf", "U", "W", "Up", "Sc")] + \
+                ("total", "status", "chunk_info", "seq_chunk0", "rq", "rk", "gcum", "betaf", "U", "W", "Mk", "Sc", "fa")] + \
                [("max_chunks", ctypes.c_int64)]
 
 
@@ -216,8 +216,9 @@ class Stages:
     """The five kernels of the chunked path as separate calls on one workspace.
 
     After ``run_all`` (or the individual calls in order) the intermediates are
-    readable through the typed views ``U``, ``W``, ``Up``, ``Sc``, ``rq``, ``rk``,
-    ``gcum``, ``betaf``, ``chunk_info`` and ``status`` (U, W, Up, Sc in fp16)."""
+    readable through the typed views ``U``, ``W``, ``Mk``, ``Sc``, ``rq``,
+    ``rk``, ``gcum``, ``betaf``, ``chunk_info`` and ``status`` (U, W, Mk, Sc
+    in fp16)."""
 
     def __init__(self, T, B, Nqk, Nv, device):
         self.T, self.B, self.Nqk, self.Nv = int(T), int(B), int(Nqk), int(Nv)
@@ -240,8 +241,8 @@ class Stages:
         return self._view("W", torch.float16, (self.NC, self.Nv, CHUNK, HEAD_DIM))
 
     @property
-    def Up(self):
-        return self._view("Up", torch.float16, (self.NC, self.Nv, CHUNK, HEAD_DIM))
+    def Mk(self):
+        return self._view("Mk", torch.float16, (self.NC, self.Nv, HEAD_DIM, HEAD_DIM))
 
     @property
     def Sc(self):

@@ -43,10 +43,12 @@ int fill_layout(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, gdn_workspace_lay
     off += (size_t)NC * Nv * tile;
     lay->W = off;
     off += (size_t)NC * Nv * tile;
-    lay->Up = off;
+    lay->Mk = off;
     off += (size_t)NC * Nv * tile;
     lay->Sc = off;
     off += (size_t)NC * Nv * tile;
+    lay->fa = off;
+    off += (size_t)NC * Nv * gdn::kFaStride * 4;
     lay->total = align256(off);
     lay->max_chunks = NC;
     return GDN_OK;
@@ -65,8 +67,9 @@ Workspace views(void *base, const gdn_workspace_layout_t &lay)
     w.betaf = reinterpret_cast<float *>(p + lay.betaf);
     w.U = reinterpret_cast<uint16_t *>(p + lay.U);
     w.W = reinterpret_cast<uint16_t *>(p + lay.W);
-    w.Up = reinterpret_cast<uint16_t *>(p + lay.Up);
+    w.Mk = reinterpret_cast<uint16_t *>(p + lay.Mk);
     w.Sc = reinterpret_cast<uint16_t *>(p + lay.Sc);
+    w.fa = reinterpret_cast<float *>(p + lay.fa);
     w.NC = static_cast<int>(lay.max_chunks);
     return w;
 }

@@ -9,6 +9,7 @@ namespace gdn {
 
 constexpr int L = 128;  // chunk length
 constexpr int D = 128;  // head dimension (Dk = Dv)
+constexpr int kFaStride = 132;  // floats per (chunk, v-head) record of the state-update factors (16-byte multiple)
 
 // Typed views of the workspace regions (layout: gdn_workspace_layout in gdn_stages.h)
 struct Workspace {
@@ -17,7 +18,8 @@ struct Workspace {
     int32_t *seq_chunk0;
     float *rq, *rk;     // fp32 [Nqk][T]: scale / |q|, 1 / |k| (eps inside the square root)
     float *gcum, *betaf;
-    uint16_t *U, *W, *Up, *Sc;
+    uint16_t *U, *W, *Mk, *Sc;
+    float *fa;  // [NC][Nv][kFaStride]: rk_t e^{gamma_L - gamma_t} (t < 128), e^{gamma_L} at 128
     int NC;  // max chunks
 };
 

@@ -3,9 +3,12 @@
 //
 // Page "Qwen3Next Samples", "Recurrent State Attention":
 //   o_inter = (q (.) exp(g_cum)) S^T
-//   o_chunk = o_inter + (q k^T (.) D_decay (.) T_tril) (v_out - v')
+//   o_chunk = o_inter + (q k^T (.) D_decay (.) T_tril) (v_out - v'),  v' = k_cumdecay S
 // with S held as [Dk, Dv] (so S^T there is S here), T_tril including the
-// diagonal, and v_out - v' = U' from the state kernel.  Warp w handles rows
+// diagonal, v_out = U and k_cumdecay = W.  With P = q k^T (.) D_decay (.) T_tril
+// and Q' = diag(e^gamma) q this is regrouped as
+//   o = (Q' - P W) S_c + P U,
+// so the chunk's state S_c enters one product.  Warp w handles rows
 // 32(w%4)..32(w%4)+31 and, in the epilogues, one half of the columns.  Steps:
 //   1. q k^T     -- tcgen05.mma M=128, N=128, K=128 on the raw bf16 rows (exact
 //                   inputs), both K-major; fp32 accumulator in TMEM.
@@ -17,11 +20,12 @@
 //      gamma_j), both factors <= 1, so a row needs one exponential per block;
 //      only the 32-column chunk on a warp's diagonal takes one per element.
 //      Chunks above all of a warp's rows are written as zeros without reading
-//      TMEM.  q is rescaled in place to Q' = diag(rq e^gamma) q in fp16
-//      (|Q'| <= scale).
-//   3. O = Q' S_c + P U' for Dv columns 0..63, then 64..127 -- 16 tcgen05.mma
-//      each (N = 64); the second half's S_c and U' load while the first half
-//      is stored.
+//      TMEM.
+//   3. Z = P W  -- M=128, N=128, K=128, fp16 (W read MN-major); then
+//      Qw = diag(rq e^gamma) q - Z in fp16, in place of q.
+//   4. O = Qw S_c + P U for Dv columns 0..63, then 64..127 -- 16 tcgen05.mma
+//      each (N = 64); S_c and U are staged one column half at a time in the
+//      buffer W used, and each half is stored while the next one loads.
 // One thread issues the MMAs and waits for their completion (mbarrier arrival
 // from tcgen05.commit, bounded wait); a CTA barrier passes the outcome on.  If
 // a wait gives up, the CTA sets bit 1 of status[2] in the workspace and skips
@@ -34,10 +38,10 @@ namespace gdn {
 
 constexpr int kOutThreads = 256;
 // shared memory, relative to a 1024-byte aligned base
-constexpr int OO_Q = 0;         // q (bf16) then Q' (fp16): K-major over Dk, 2 halves x 128 rows x 128 B
+constexpr int OO_Q = 0;         // q (bf16) then Qw (fp16): K-major over Dk, 2 halves x 128 rows x 128 B
 constexpr int OO_K = 32768;     // k (bf16), K-major over Dk; then P (fp16), K-major over j
-constexpr int OO_S = 65536;     // S_c[:, half] (fp16) [Dk][64], MN-major: 128 rows x 128 B
-constexpr int OO_U = 81920;     // U'[:, half] (fp16) [L][64], MN-major
+constexpr int OO_X = 65536;     // W (fp16) [L][Dk] in two 64-column blocks (MN-major B of P W); then
+                                // S_c[:, half] (fp16) [Dk][64] and, 16 KiB on, U[:, half] (fp16) [L][64]
 constexpr int OO_VEC = 98304;   // gam, rqv, rkv, kfe (rk_j e^{gamma_je - gamma_j})
 constexpr int OO_BAR = OO_VEC + 4 * 512;
 constexpr int kOutSmem = OO_BAR + 64 + 1024;
@@ -48,8 +52,8 @@ __device__ __forceinline__ uint32_t t128(int r, int c) { return (uint32_t)((c >>
 __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, uint16_t *__restrict__ out, int T, int Nqk,
     int Nv, const int4 *__restrict__ info, const float *__restrict__ rq, const float *__restrict__ rk,
-    const float *__restrict__ gcum, const uint16_t *__restrict__ Up, const uint16_t *__restrict__ Sc,
-    int32_t *__restrict__ status)
+    const float *__restrict__ gcum, const uint16_t *__restrict__ U, const uint16_t *__restrict__ W,
+    const uint16_t *__restrict__ Sc, int32_t *__restrict__ status)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
@@ -64,20 +68,20 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     const int row = quarter * 32 + lane;
     float *gam = reinterpret_cast<float *>(smem + OO_VEC);
     float *rqv = gam + 128, *rkv = gam + 256, *kfe = gam + 384;
-    const uint32_t bar_qk = sbase + OO_BAR, bar_o = sbase + OO_BAR + 8;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + OO_BAR + 16);
+    const uint32_t bar_qk = sbase + OO_BAR, bar_z = sbase + OO_BAR + 8, bar_o = sbase + OO_BAR + 16;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + OO_BAR + 24);
     const size_t tile = (size_t)(c * Nv + h) * L * D;
 
-    // S_c and U' columns [64 hf, 64 hf + 64) into the MN-major buffers
+    // S_c and U columns [64 hf, 64 hf + 64) into the MN-major buffers
     auto load_su = [&](int hf) {
         for (int e = tid; e < 128 * 8; e += kOutThreads) {
             const int r = e >> 3, cc = e & 7;
-            cp_async16(sbase + OO_S + tc::sw128c(r, cc), Sc + tile + (size_t)r * D + hf * 64 + cc * 8, true);
-            cp_async16(sbase + OO_U + tc::sw128c(r, cc), Up + tile + (size_t)r * D + hf * 64 + cc * 8, true);
+            cp_async16(sbase + OO_X + tc::sw128c(r, cc), Sc + tile + (size_t)r * D + hf * 64 + cc * 8, true);
+            cp_async16(sbase + OO_X + 16384 + tc::sw128c(r, cc), U + tile + (size_t)r * D + hf * 64 + cc * 8, true);
         }
     };
 
-    // ---- async loads: q, k rows of the chunk (zero past n), S_c / U' first half, gamma, rq, rk
+    // ---- async loads: q, k rows of the chunk (zero past n), W, gamma, rq, rk
     for (int e = tid; e < 128 * 16; e += kOutThreads) {
         const int r = e >> 4, cc = e & 15;
         const bool ok = r < n;
@@ -85,8 +89,8 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         const uint32_t off = t128(r, cc);
         cp_async16(sbase + OO_Q + off, q + ((size_t)t * Nqk + hq) * D + cc * 8, ok);
         cp_async16(sbase + OO_K + off, k + ((size_t)t * Nqk + hq) * D + cc * 8, ok);
+        cp_async16(sbase + OO_X + off, W + tile + (size_t)r * D + cc * 8, true);
     }
-    load_su(0);
     if (tid < 128) {
         const int i = min(tid, n - 1);
         cp_async4(smem_addr(gam + tid), gcum + (size_t)h * T + t0 + i);
@@ -96,6 +100,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     cp_async_commit();
     if (tid == 0) {
         tc::mbar_init(bar_qk, 1);
+        tc::mbar_init(bar_z, 1);
         tc::mbar_init(bar_o, 1);
         tc::mbar_init_fence();
     }
@@ -105,7 +110,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    const uint32_t tmem = *tslot;  // columns [0, 128): q k^T; [128, 192), [192, 256): O halves
+    const uint32_t tmem = *tslot;  // columns [0, 128): q k^T, then O; [128, 256): Z = P W
     const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
     bool ok = true;
     uint32_t last_bar = bar_qk, last_par = 0;  // the most recent commit (thread 0)
@@ -116,23 +121,28 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         ok = __syncthreads_and(w_ok) != 0;
         tc::fence_after_sync();
     };
+    auto sync_operands = [&]() {  // generic-proxy shared-memory writes -> tensor core
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+    };
+    // descriptor of K step kk of a K-major tile with two 64-column K halves
+    auto kmaj = [](uint64_t d, int kk) { return d + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4); };
 
     // ---- (1) q k^T
     if (tid == 0) {
         const uint64_t dq = tc::desc_k128(sbase + OO_Q), dk = tc::desc_k128(sbase + OO_K);
         const uint32_t idesc = tc::idesc_f16(128, 128, true, true);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-            tc::mma_f16(tmem, dq + off, dk + off, idesc, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 8; ++kk) tc::mma_f16(tmem, kmaj(dq, kk), kmaj(dk, kk), idesc, kk > 0 ? 1u : 0u);
         tc::commit(bar_qk);
     }
     if (tid < 128) kfe[tid] = rkv[tid] * __expf(gam[tid | 15] - gam[tid]);
     wait_mma(bar_qk, 0);
 
     if (ok) {
-        // ---- (2) P, this thread's 64 columns of its row (fp16 over the k tile); Q' (in place)
+        // ---- (2) P, this thread's 64 columns of its row (fp16 over the k tile)
         const float gi = gam[row], fr = rqv[row];
         const int rlo = quarter * 32;  // first row of this warp
 #pragma unroll 1
@@ -173,39 +183,58 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
                 }
             }
         }
-        const float qf = fr * __expf(gi);
-#pragma unroll 4
-        for (int cc = half * 8; cc < half * 8 + 8; ++cc) {
-            uint4 *p = reinterpret_cast<uint4 *>(smem + OO_Q + t128(row, cc));
-            const uint4 w = *p;
-            const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
-            uint32_t o4[4];
+        sync_operands();
+
+        // ---- (3) Z = P W, then Qw = diag(rq e^gamma) q - Z over q
+        if (tid == 0) {
+            const uint64_t dp = tc::desc_k128(sbase + OO_K), dw = tc::desc_mn(sbase + OO_X, 16384, 1024, 2);
+            const uint32_t idesc = tc::idesc_f16(128, 128, false, false, false, true);
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                o4[e] = pack_h2(__uint_as_float(w4[e] << 16) * qf, __uint_as_float(w4[e] & 0xffff0000u) * qf);
-            *p = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+            for (int kk = 0; kk < 8; ++kk)
+                tc::mma_f16(tmem + 128, kmaj(dp, kk), dw + (uint64_t)((kk * 2048) >> 4), idesc, kk > 0 ? 1u : 0u);
+            tc::commit(bar_z);
+            last_bar = bar_z;
         }
-        tc::fence_proxy_async();
-        tc::fence_before_sync();
-        __syncthreads();
-        tc::fence_after_sync();
+        wait_mma(bar_z, 0);
+    }
+    if (ok) {
+        load_su(0);  // W is consumed
+        cp_async_commit();
+        const float qf = rqv[row] * __expf(gam[row]);
+#pragma unroll 1
+        for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
+            float z[32];
+            tc::tmem_ld32(t_row + 128 + j0, z);
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                uint4 *p = reinterpret_cast<uint4 *>(smem + OO_Q + t128(row, (j0 >> 3) + c4));
+                const uint4 w = *p;
+                const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+                uint32_t o4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    o4[e] = pack_h2(__uint_as_float(w4[e] << 16) * qf - z[c4 * 8 + 2 * e],
+                                    __uint_as_float(w4[e] & 0xffff0000u) * qf - z[c4 * 8 + 2 * e + 1]);
+                *p = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+            }
+        }
+        cp_async_wait<0>();
+        sync_operands();
 
         const uint64_t dq = tc::desc_k128(sbase + OO_Q), dp = tc::desc_k128(sbase + OO_K);
-        const uint64_t ds = tc::desc_mn(sbase + OO_S, 16384, 1024, 2), du = tc::desc_mn(sbase + OO_U, 16384, 1024, 2);
+        const uint64_t ds = tc::desc_mn(sbase + OO_X, 16384, 1024, 2), du = tc::desc_mn(sbase + OO_X + 16384, 16384, 1024, 2);
         const uint32_t idesc = tc::idesc_f16(128, 64, false, false, false, true);
 #pragma unroll 1
         for (int hf = 0; hf < 2 && ok; ++hf) {
-            // ---- (3) O[:, 64 hf : 64 hf + 64] = Q' S_c + P U'
+            // ---- (4) O[:, 64 hf : 64 hf + 64] = Qw S_c + P U
             if (tid == 0) {
-                const uint32_t dst = tmem + 128 + hf * 64;
+                const uint32_t dst = tmem + hf * 64;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_f16(dst, dq + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                                ds + (uint64_t)((kk * 2048) >> 4), idesc, kk > 0 ? 1u : 0u);
+                    tc::mma_f16(dst, kmaj(dq, kk), ds + (uint64_t)((kk * 2048) >> 4), idesc, kk > 0 ? 1u : 0u);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_f16(dst, dp + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                                du + (uint64_t)((kk * 2048) >> 4), idesc, 1u);
+                    tc::mma_f16(dst, kmaj(dp, kk), du + (uint64_t)((kk * 2048) >> 4), idesc, 1u);
                 tc::commit(bar_o);
                 last_bar = bar_o;
                 last_par = (uint32_t)hf;
@@ -216,10 +245,10 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
                 load_su(1);
                 cp_async_commit();
             }
-            // ---- (4) this thread's 32 columns of the half, to bf16 (TMEM reads are warp-collective)
+            // ---- this thread's 32 columns of the half, to bf16 (TMEM reads are warp-collective)
             {
                 float a[32];
-                tc::tmem_ld32(t_row + 128 + hf * 64 + half * 32, a);
+                tc::tmem_ld32(t_row + hf * 64 + half * 32, a);
                 if (row < n) {
                     uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)(t0 + row) * Nv + h) * D + hf * 64 + half * 32);
 #pragma unroll
@@ -231,10 +260,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
             }
             if (hf == 0) {
                 cp_async_wait<0>();
-                tc::fence_proxy_async();
-                tc::fence_before_sync();
-                __syncthreads();
-                tc::fence_after_sync();
+                sync_operands();
             }
         }
     }
@@ -256,7 +282,7 @@ cudaError_t launch_output(const uint16_t *q, const uint16_t *k, uint16_t *out, i
     cudaError_t e = cudaFuncSetAttribute(output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
     if (e != cudaSuccess) return e;
     output_kernel<<<dim3(NC, Nv), kOutThreads, kOutSmem, st>>>(q, k, out, T, Nqk, Nv, ws.chunk_info, ws.rq, ws.rk,
-                                                                ws.gcum, ws.Up, ws.Sc, ws.status);
+                                                                ws.gcum, ws.U, ws.W, ws.Sc, ws.status);
     return cudaGetLastError();
 }
 

@@ -38,7 +38,8 @@ extern "C" {
  * number of chunks of any packing of T tokens into B sequences.
  *   status      int32[4]: [0] cu_seqlens error bits (1: cu[0] != 0, 2: decreasing,
  *               4: cu[B] != T), [1] number of chunks, [2] tensor-core completion
- *               waits that gave up (bit 0: state pass, bit 1: output; the
+ *               waits that gave up (bit 0: state pass, bit 1: output, bit 2:
+ *               intra-chunk; the
  *               results are then incomplete); the caller clears [2] to read it
  *   chunk_info  int32[NC][4]: sequence, first token, tokens in the chunk (1..128),
  *               chunk index within its sequence; rows past the last chunk hold -1
@@ -47,8 +48,12 @@ extern "C" {
  *   rk          fp32 [Nqk][T]: 1 / sqrt(|k|^2 + eps)
  *   gcum        fp32 [Nv][T]: chunk-local cumulative gate gamma
  *   betaf       fp32 [Nv][T]: beta widened to fp32
- *   U, W, Up    fp16 [NC][Nv][128 (L)][128]: U, W (columns Dk) and U' of each chunk
+ *   U, W        fp16 [NC][Nv][128 (L)][128]: U and W (columns Dk) of each chunk
+ *   Mk          fp16 [NC][Nv][128 (Dk)][128 (Dk)]: Mk = k_gexp^T W, the factor of
+ *               the state update that multiplies the state
  *   Sc          fp16 [NC][Nv][128 (Dk)][128 (Dv)]: state entering each chunk
+ *   fa          fp32 [NC][Nv][132]: per chunk rk_t e^{gamma_L - gamma_t} for its
+ *               rows t < 128 (0 past the chunk), e^{gamma_L} at 128, zeros after
  * The tensor-core products take fp16 operands (11-bit significand) with fp32
  * accumulation: the raw bf16 q, k, v convert to fp16 exactly (magnitudes in
  * [2^-14, 65504]), the L2 norms enter as fp32 scalings, and the state update's
@@ -67,8 +72,9 @@ typedef struct {
     size_t betaf;
     size_t U;
     size_t W;
-    size_t Up;
+    size_t Mk;
     size_t Sc;
+    size_t fa;
     int64_t max_chunks;
 } gdn_workspace_layout_t;
 
@@ -103,19 +109,19 @@ int gdn_stage_prologue(const uint16_t *q, const uint16_t *k, const float *g, con
  * T = (I + A)^-1 by blocked forward substitution ("Matrix Inversion" with the
  * block merge of inverse_pto / inverse_matmul), and computes U and W ("Value
  * and Key Cumulative Decay").  Reads k [T, Nqk, 128], v [T, Nv, 128] (bf16)
- * and the prologue's outputs; writes U, W.
+ * and the prologue's outputs; writes U, W and Mk = k_gexp^T W with
+ * k_gexp = Kh * exp(g_last - g_cum) ("State Update").
  */
 int gdn_stage_intra(const uint16_t *k, const uint16_t *v, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
                     void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Inter-chunk state passing: per (sequence, v-head, 32-column slice of Dv),
- * serially over the sequence's chunks, U' = U - W S and
- * S <- e^{gamma_last} S + (Kh * e^{gamma_last - gamma})^T U' ("Recurrent State
- * Attention" v', "State Update" with k_gexp), the state kept in fp32 on chip.
+ * serially over the sequence's chunks, S <- e^{gamma_last} S + k_gexp^T U - Mk S
+ * ("State Update" with v' = W S regrouped), the state kept in fp32 on chip.
  * S starts from state_pool[state_indices[b]] (or slot b, or zero without a
- * pool).  Reads k [T, Nqk, 128] bf16, rk, gcum, U, W; writes Sc and Up for
- * every chunk and final_state (if not NULL).
+ * pool).  Reads k [T, Nqk, 128] bf16, rk, gcum, U and Mk; writes Sc for every
+ * chunk and final_state (if not NULL).
  */
 int gdn_stage_state(const uint16_t *k, const float *state_pool, const int32_t *state_indices, float *final_state,
                     int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P, void *workspace,
@@ -124,7 +130,7 @@ int gdn_stage_state(const uint16_t *k, const float *state_pool, const int32_t *s
 /*
  * Output: per (chunk, v-head) o = diag(e^gamma) Qh S_c + (Qh Kh^T * Gamma * tril) U'
  * ("Recurrent State Attention": o_inter and o_chunk; tril includes the
- * diagonal).  Reads q, k [T, Nqk, 128] bf16, rq, rk, gcum, Sc, Up; writes
+ * diagonal).  Reads q, k [T, Nqk, 128] bf16, rq, rk, gcum, Sc, U' (in U); writes
  * out [T, Nv, 128] bf16 for every token of every chunk.
  */
 int gdn_stage_output(const uint16_t *q, const uint16_t *k, uint16_t *out, int64_t T, int32_t B, int32_t Nqk,

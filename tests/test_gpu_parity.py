@@ -78,8 +78,13 @@ def test_stages_match_chunked_intermediates():
     inp = inputs.make([200, 129, 1, 128], Nqk=2, Nv=4, state=("normal", 0.02, 6, "perm"), seed=11)
     d = inp.to(DEV)
     st = gdn.Stages(inp.T, inp.B, inp.Nqk, inp.Nv, DEV)
-    out, fin = st.run_all(d.q, d.k, d.v, d.g, d.beta, d.cu_seqlens, d.state_pool, d.state_indices,
-                          scale=inp.scale, eps=inp.eps)
+    out = torch.empty(inp.T, inp.Nv, 128, dtype=torch.bfloat16, device=DEV)
+    fin = torch.empty(inp.B, inp.Nv, 128, 128, dtype=torch.float32, device=DEV)
+    st.chunk_map(d.cu_seqlens)
+    st.prologue(d.q, d.k, d.g, d.beta, inp.scale, inp.eps)
+    st.intra(d.k, d.v)
+    st.state(d.k, d.state_pool, d.state_indices, fin)
+    st.output(d.q, d.k, out)
     torch.cuda.synchronize()
     X = {n: oracle.as_numpy_exact(getattr(inp, n)) for n in ("q", "k", "v", "g", "beta")}
     _, _, kept = oracle.chunked(X["q"], X["k"], X["v"], X["g"], X["beta"], inp.cu_seqlens.numpy(),
@@ -90,7 +95,8 @@ def test_stages_match_chunked_intermediates():
     for c in range(info.shape[0]):
         if info[c, 0] >= 0 and info[c, 3] == 0:
             seq_first[int(info[c, 0])] = c
-    names = {"U": "v_out", "W": "k_cumdecay", "Up": "v_new", "Sc": "S_in"}
+    names = {"U": "v_out", "W": "k_cumdecay", "Sc": "S_in", "Mk": None}
+    per_token = {"U", "W"}
     got = {n: [] for n in names}
     ref = {n: [] for n in names}
     gam_g, gam_r, kh_g, kh_r, qh_g, qh_r = [], [], [], [], [], []
@@ -101,10 +107,13 @@ def test_stages_match_chunked_intermediates():
         n = r["o"].shape[0]
         t0 = int(info[c, 1])
         assert int(info[c, 2]) == n
+        # the factor of the state update that multiplies S ("State Update": k_gexp^T k_cumdecay)
+        k_gexp = r["kn"] * np.exp(r["g_cum"][-1] - r["g_cum"])[:, None]
+        derived = {"Mk": k_gexp.T @ r["k_cumdecay"]}
         for nm, key in names.items():
             t = getattr(st, nm)[c, h].cpu().double().numpy()
-            got[nm].append(t if nm == "Sc" else t[:n])
-            ref[nm].append(r[key])
+            got[nm].append(t[:n] if nm in per_token else t)
+            ref[nm].append(r[key] if key else derived[nm])
         hq = h // G
         gam_g.append(gcum[h, t0:t0 + n].numpy())
         gam_r.append(r["g_cum"])
@@ -119,6 +128,7 @@ def test_stages_match_chunked_intermediates():
     assert_close(cat(qh_g), cat(qh_r), "q normalised and scaled", rel_l2=1e-5, max_abs_rms=1e-5)
     for nm in names:  # fp16 intermediates: their own storage rounding is allowed per element
         assert_close(cat(got[nm]), cat(ref[nm]), f"stage {nm}", ulp=helpers.FP16_HALF_ULP)
+    assert int(st.status.cpu()[2]) == 0
     _check(inp, out, fin, what="stages")
 
 

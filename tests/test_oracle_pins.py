@@ -330,3 +330,18 @@ def test_chunk_intermediates_identities():
         _close(r["v_new"], r["v_out"] - r["k_cumdecay"] @ r["S_in"], 1e-12, "v_new")
         n = r["o"].shape[0]
         _close(r["o"], o_rec[c * 32:c * 32 + n, 0], 1e-10, "chunk o")
+
+
+def test_state_update_split_into_state_free_parts():
+    """The state update regrouped as e^{g_last} S + N - Mk S, with N = k_gexp^T v_out and
+    Mk = k_gexp^T k_cumdecay (the form the GPU state pass iterates), closes each chunk
+    exactly as the page's update does, partial last chunk included."""
+    p = _random_problem(23, [75, 32], Nqk=1, Nv=2, D=8, with_pool=True, P=2)
+    _, _, kept = oracle.chunked(**p, C=32, keep=True)
+    assert any(r["o"].shape[0] < 32 for r in kept.values())
+    for r in kept.values():
+        k_gexp = r["kn"] * np.exp(r["g_cum"][-1] - r["g_cum"])[:, None]
+        N = k_gexp.T @ r["v_out"]
+        Mk = k_gexp.T @ r["k_cumdecay"]
+        S = r["S_in"]
+        _close(np.exp(r["g_cum"][-1]) * S + N - Mk @ S, r["S_new"], 1e-12, "regrouped state update")
