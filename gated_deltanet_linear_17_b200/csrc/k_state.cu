@@ -1,6 +1,6 @@
 // Inter-chunk state passing on the Blackwell tensor core: one CTA per
-// (sequence, v-head, 32-column slice of Dv), 8 epilogue warps and one warp
-// that moves data (TMA) and issues the tensor-core work.
+// (sequence, v-head, 32-column slice of Dv), 8 epilogue warps, one warp that
+// issues the tensor-core work and one that moves data with TMA.
 //
 // Page "Qwen3Next Samples", "Recurrent State Attention" and "State Update",
 // with the state held as S[Dk, Dv]:
@@ -17,13 +17,13 @@
 // whole sequence.  Per chunk c:
 //   issue warp: Mk S_c (tcgen05.mma M=128, N=32, K=128, fp16; A = Mk K-major,
 //               B = S_c MN-major as the threads store it; two accumulation
-//               chains over the halves of K), committed to an mbarrier; a TMA
-//               store of S_c (fp16) to Sc; once Mk S_c has completed, TMA loads
-//               of chunk c+2 (Mk, the raw k rows, the U slice and the factors)
-//               into the freed stage; once the epilogue warps have staged its
-//               operand, Kt of chunk c+1 = K^T Ub (M=128, N=64, K=128, bf16; A =
-//               the raw k tile read MN-major, B = [Ub_hi | Ub_lo]) into one of
-//               two TMEM buffers.
+//               chains over the halves of K), committed to an mbarrier; then,
+//               once the epilogue warps have staged its operand, Kt of chunk
+//               c+1 = K^T Ub (M=128, N=64, K=128, bf16; A = the raw k tile read
+//               MN-major, B = [Ub_hi | Ub_lo]) into one of two TMEM buffers.
+//   data warp:  a TMA store of S_c (fp16) to Sc; once Mk S_c has completed, TMA
+//               loads of chunk c+2 (Mk, the raw k rows, the U slice and the
+//               factors) into the freed stage.
 //   epilogue:   Ub = diag(f) U of chunk c+1 split into bf16 hi + lo (~16
 //               significant bits; k is exact in bf16); wait for Mk S_c (its
 //               commit also covers Kt of chunk c, issued before it);
@@ -41,7 +41,7 @@
 
 namespace gdn {
 
-constexpr int kStateThreads = 288;  // 8 epilogue warps + the data / issue warp
+constexpr int kStateThreads = 320;  // 8 epilogue warps, the issue warp, the data warp
 constexpr int DVT = 32;             // Dv columns per CTA
 
 // shared memory, relative to a 1024-byte aligned base (bytes); two stages
@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
     const int b = blockIdx.x, h = blockIdx.y, col0 = blockIdx.z * DVT;
     const int hq = h / (Nv / Nqk);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const bool issuer = wid == 8;
+    const bool issuer = wid == 8, producer = wid == 9, epi = wid < 8;
     const int quarter = wid & 3, half = (wid >> 2) & 1;
     const int row = quarter * 32 + lane;  // row of the state (Dk) and of Ub (L)
     const int cbase = half * 16;          // first of this thread's 16 columns in the slice
@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
     if (wid == 0) tc::tmem_alloc(smem_addr(tslot), kTmemCols);
     __syncthreads();
 
-    // TMA fill of stage st with chunk c (issue lane)
+    // TMA fill of stage st with chunk c (data lane)
     int fills[2] = {0, 0};
     auto fill = [&](int c, int st) {
         const uint32_t base = sbase + st * kStage, full = bar_full + 8 * st;
@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
 
     // initial state: this thread's 16 values
     float s[16];
-    if (!issuer && pool) {
+    if (epi && pool) {
         const int slot = idx ? idx[b] : b;
         const float4 *src =
             reinterpret_cast<const float4 *>(pool + (((size_t)slot * Nv + h) * D + row) * D + col0 + cbase);
@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
 
     bool ok = true;
     float dg = 1.f;  // e^{g_last} of the chunk in flight (epilogue warps)
-    if (issuer) {
+    if (producer) {
         if (lane == 0) {
             tma::prefetch_map(&tm_mk);
             tma::prefetch_map(&tm_k);
@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
             if (c_begin < c_end) fill(c_begin, 0);
             if (c_begin + 1 < c_end) fill(c_begin + 1, 1);
         }
-    } else {
+    } else if (epi) {
         store_state_operand(0);
         if (c_begin < c_end) {
             ok = warp_wait(bar_full, 0, lane);
@@ -224,7 +224,6 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
         const int st = it & 1;
         const bool has_next = c + 1 < c_end;
         if (issuer) {
-            bool w_ok = true;
             if (lane == 0) {
                 if (it == 0) issue_kt(0);  // the first chunk's Kt, before its chain product
                 const uint64_t so = (uint64_t)((st * kStage) >> 4), sb = (uint64_t)((st * 8192) >> 4);
@@ -234,12 +233,6 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
                                 dS0 + sb + (uint64_t)((kk * 1024) >> 4), idesc_m, (kk & 3) ? 1u : 0u);
                 tc::commit(bar_m);
                 issued = true;
-                // the state entering chunk c, from its operand copy
-                tma::store_2d(&tm_sc, col0, (c * Nv + h) * L, sbase + OFF_S + st * 8192);
-                tma::commit_group();
-                // stage st is free once Mk S_c (and Kt_c before it) has completed
-                w_ok = tc::mbar_wait_bounded(bar_m, (uint32_t)(it & 1));
-                if (w_ok && c + 2 < c_end) fill(c + 2, st);
             }
             __syncwarp();
             if (has_next) {
@@ -247,9 +240,19 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
                 if (lane == 0) issue_kt(st ^ 1);
                 __syncwarp();
             }
-            if (lane == 0) tma::wait_read_all();  // the store of S_c has read its buffer
+        } else if (producer) {
+            bool w_ok = true;
+            if (lane == 0) {
+                // the state entering chunk c, from its operand copy
+                tma::store_2d(&tm_sc, col0, (c * Nv + h) * L, sbase + OFF_S + st * 8192);
+                tma::commit_group();
+                // stage st is free once Mk S_c (and Kt_c before it) has completed
+                w_ok = tc::mbar_wait_bounded(bar_m, (uint32_t)(it & 1));
+                if (w_ok && c + 2 < c_end) fill(c + 2, st);
+                tma::wait_read_all();  // the store of S_c has read its buffer
+            }
             ok = __shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0) != 0;
-        } else {
+        } else {  // epilogue warps
             float dg_next = 1.f;
             if (has_next) {
                 const bool f_ok = warp_wait(bar_full + 8 * (st ^ 1), (uint32_t)(((it + 1) >> 1) & 1), lane);
@@ -278,18 +281,18 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
     }
 
     // copies and MMAs still in flight land before shared and tensor memory are released
-    if (issuer && lane == 0) {
+    if (producer && lane == 0) {
         for (int st = 0; st < 2; ++st)
             if (fills[st] > 0) tc::mbar_wait_bounded(bar_full + 8 * st, (uint32_t)((fills[st] - 1) & 1));
-        if (!ok && issued) {  // a commit covers every MMA issued before it
-            tc::commit(bar_d);
-            tc::mbar_wait_bounded(bar_d, 0);
-        }
         tma::wait_all();
+    }
+    if (issuer && lane == 0 && !ok && issued) {  // a commit covers every MMA issued before it
+        tc::commit(bar_d);
+        tc::mbar_wait_bounded(bar_d, 0);
     }
     if (!ok) {
         if (tid == 0) atomicOr(status + 2, 1);
-    } else if (final_state && !issuer) {
+    } else if (final_state && epi) {
         float4 *dst =
             reinterpret_cast<float4 *>(final_state + (((size_t)b * Nv + h) * D + row) * D + col0 + cbase);
 #pragma unroll
