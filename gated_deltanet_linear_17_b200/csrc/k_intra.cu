@@ -85,9 +85,11 @@ __device__ __forceinline__ void warp_store16(const float (&acc)[2][4], uint8_t *
 }
 
 __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
-    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, int T, int Nqk, int Nv,
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_w,
+    const __grid_constant__ CUtensorMap tm_mk, int T, int Nqk, int Nv,
     const int4 *__restrict__ info, const float *__restrict__ rk, const float *__restrict__ gcum,
-    const float *__restrict__ betaf, uint16_t *__restrict__ U, uint16_t *__restrict__ W, uint16_t *__restrict__ Mk,
+    const float *__restrict__ betaf,
     float *__restrict__ fa, int32_t *__restrict__ status)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -105,7 +107,6 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     float *bet = gam + 128, *rkv = gam + 256, *kfe = gam + 384;
     const uint32_t bar_ld = sbase + OFF_BAR, bar_mma = sbase + OFF_BAR + 8, bar_d = sbase + OFF_BAR + 16;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 24);
-    const size_t tile = (size_t)(c * Nv + h) * L * D;
 
     if (tid == 0) {
         tc::mbar_init(bar_ld, 1);
@@ -191,7 +192,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
 
     // ---- (2) Ap = -strict_tril(diag(beta rk) (k k^T) diag(rk) (.) Gamma): this thread's row and 64 columns.
     // Blocks left of the row's diagonal 16-block go to the A tile in fp16; the diagonal block goes to the
-    // fp32 scratch (block b at OFF_X + 1024 b); blocks right of it are zero.
+    // fp32 scratch (block b at OFF_X + 1024 b, element (r, c) at r * 16 + (c ^ (r >> 1))); blocks right
+    // of it are zero.
     float *dsc = reinterpret_cast<float *>(smem + OFF_X);
     if (ok) {
         const float gi = gam[row], fr = -bet[row] * rkv[row];
@@ -206,18 +208,43 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
             }
             float a[32];
             tc::tmem_ld32(t_row + j0, a);
+            if (j0 == quarter * 32) {
+                // The warp's diagonal chunk (warp-uniform): every lane takes its 32 values element by
+                // element.  Lanes 0-15 have their diagonal block at columns j0..j0+15, lanes 16-31 at
+                // j0+16..; the block left of it (lanes 16-31, columns j0..j0+15) goes to the fp16 tile.
+                float v[32];
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int j = j0 + jj;
+                    v[jj] = j < row ? fr * rkv[j] * __expf(fminf(gi - gam[j], 0.f)) * a[jj] : 0.f;
+                }
+                const bool hi = lane >= 16;
+                float *drow = dsc + (rb >> 4) * 256 + (row - rb) * 16;
+                const int sw = (row - rb) >> 1;  // bank swizzle of the fp32 diagonal blocks
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) drow[jj ^ sw] = hi ? v[16 + jj] : v[jj];
+#pragma unroll
+                for (int q16 = 0; q16 < 2; ++q16) {
+                    const bool left = q16 == 0 && hi;
+#pragma unroll
+                    for (int q8 = 0; q8 < 2; ++q8) {
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int jj = q16 * 16 + q8 * 8 + 2 * e;
+                            w4[e] = left ? pack_h2(v[jj], v[jj + 1]) : 0u;
+                        }
+                        *reinterpret_cast<uint4 *>(smem + OFF_A + t128(row, (j0 >> 3) + 2 * q16 + q8)) =
+                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
+                }
+                continue;
+            }
+            // a chunk left of the warp's rows: the decay factored per 16-column block
 #pragma unroll
             for (int q16 = 0; q16 < 2; ++q16) {
                 const int jb = j0 + q16 * 16;
-                if (jb == rb) {  // the diagonal block, kept in fp32
-#pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) {
-                        const int j = jb + jj;
-                        dsc[(rb >> 4) * 256 + (row - rb) * 16 + jj] =
-                            j < row ? fr * rkv[j] * __expf(fminf(gi - gam[j], 0.f)) * a[q16 * 16 + jj] : 0.f;
-                    }
-                }
-                const float eb = jb < rb ? fr * __expf(gi - gam[jb + 15]) : 0.f;  // 0 on and right of the diagonal
+                const float eb = fr * __expf(gi - gam[jb + 15]);
 #pragma unroll
                 for (int q8 = 0; q8 < 2; ++q8) {
                     uint32_t w4[4];
@@ -255,7 +282,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
             float val = (i == cidx) ? 1.f : 0.f;
 #pragma unroll
             for (int j = 0; j < i; ++j)
-                if (j >= cidx) val += ds[i * 16 + j] * tcol[j];
+                if (j >= cidx) val += ds[i * 16 + (j ^ (i >> 1))] * tcol[j];
             tcol[i] = (i < cidx) ? 0.f : val;
         }
         const int col = wid * 16 + cidx;
@@ -330,19 +357,18 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     }
     if (ok && tid == 0) load_k();  // the k rows again, for k_gexp (the first use of the tile is over)
     if (ok) {
-        // W (warps 0-3) and U (warps 4-7) rows to global in fp16; W also to the v tile as Mk's B operand
-        uint16_t *grow = (half ? U : W) + tile + (size_t)row * D;
+        // W (warps 0-3) into the v tile, where it is also Mk's B operand, and U (warps 4-7) into the
+        // A tile, in fp16; both leave for global memory by TMA
+        uint8_t *dst = smem + (half ? OFF_A : OFF_V);
 #pragma unroll 1
         for (int j0 = 0; j0 < 128; j0 += 32) {
             float a[32];
             tc::tmem_ld32(t_row + half * 128 + j0, a);
 #pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {
-                const uint4 w = make_uint4(pack_h2(a[8 * q8], a[8 * q8 + 1]), pack_h2(a[8 * q8 + 2], a[8 * q8 + 3]),
-                                           pack_h2(a[8 * q8 + 4], a[8 * q8 + 5]), pack_h2(a[8 * q8 + 6], a[8 * q8 + 7]));
-                reinterpret_cast<uint4 *>(grow)[(j0 >> 3) + q8] = w;
-                if (!half) *reinterpret_cast<uint4 *>(smem + OFF_V + t128(row, (j0 >> 3) + q8)) = w;
-            }
+            for (int q8 = 0; q8 < 4; ++q8)
+                *reinterpret_cast<uint4 *>(dst + t128(row, (j0 >> 3) + q8)) =
+                    make_uint4(pack_h2(a[8 * q8], a[8 * q8 + 1]), pack_h2(a[8 * q8 + 2], a[8 * q8 + 3]),
+                               pack_h2(a[8 * q8 + 4], a[8 * q8 + 5]), pack_h2(a[8 * q8 + 6], a[8 * q8 + 7]));
         }
         // the state pass's per-row factors rk_t e^{g_last - gamma_t} (0 past the chunk) and e^{g_last}
         if (tid < kFaStride) {
@@ -350,6 +376,17 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
             fa[(size_t)(c * Nv + h) * kFaStride + tid] =
                 tid < 128 ? rkv[tid] * __expf(gl - gam[tid]) : (tid == 128 ? __expf(gl) : 0.f);
         }
+    }
+
+    const int trow = (c * Nv + h) * L;  // first row of the chunk's tiles in the workspace
+    tc::fence_proxy_async();
+    __syncthreads();
+    if (ok && tid == 0) {
+        tma::store_2d(&tm_w, 0, trow, sbase + OFF_V);
+        tma::store_2d(&tm_w, 64, trow, sbase + OFF_V + 16384);
+        tma::store_2d(&tm_u, 0, trow, sbase + OFF_A);
+        tma::store_2d(&tm_u, 64, trow, sbase + OFF_A + 16384);
+        tma::commit_group();
     }
 
     // ---- (5) k_gexp = fp16(rk e^{g_last - gamma} k) over the reloaded k rows (zero past the chunk), then Mk
@@ -384,17 +421,23 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     }
     if (ok) wait_bar(bar_mma, mma_phase);
     if (ok) {
-        // warp w: row 32 (w % 4) + lane of Mk, columns 64 (w / 4) .. +63
-        uint4 *dst = reinterpret_cast<uint4 *>(Mk + tile + (size_t)row * D + half * 64);
+        // warp w: row 32 (w % 4) + lane of Mk, columns 64 (w / 4) .. +63, into the (consumed) k tile
 #pragma unroll 1
         for (int j0 = 0; j0 < 64; j0 += 32) {
             float a[32];
             tc::tmem_ld32(t_row + half * 64 + j0, a);
 #pragma unroll
             for (int q8 = 0; q8 < 4; ++q8)
-                dst[(j0 >> 3) + q8] =
+                *reinterpret_cast<uint4 *>(smem + OFF_K + t128(row, half * 8 + (j0 >> 3) + q8)) =
                     make_uint4(pack_h2(a[8 * q8], a[8 * q8 + 1]), pack_h2(a[8 * q8 + 2], a[8 * q8 + 3]),
                                pack_h2(a[8 * q8 + 4], a[8 * q8 + 5]), pack_h2(a[8 * q8 + 6], a[8 * q8 + 7]));
+        }
+        tc::fence_proxy_async();
+        __syncthreads();
+        if (tid == 0) {
+            tma::store_2d(&tm_mk, 0, trow, sbase + OFF_K);
+            tma::store_2d(&tm_mk, 64, trow, sbase + OFF_K + 16384);
+            tma::commit_group();
         }
     } else if (tid == 0) {
         atomicOr(status + 2, 4);
@@ -405,6 +448,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
         tc::mbar_wait_bounded(bar_ld, 0);
         tc::mbar_wait_bounded(bar_ld, 1);
     }
+    if (tid == 0) tma::wait_all();  // the stores have read shared memory and completed
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -415,18 +459,26 @@ cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, int T, int Nqk, i
                          cudaStream_t st)
 {
     if (NC == 0 || T == 0) return cudaSuccess;
-    if ((uint64_t)T >= (1ull << 31)) return cudaErrorInvalidValue;
-    CUtensorMap m_k, m_v;
+    const uint64_t trows = (uint64_t)NC * Nv * L;  // TMA coordinates are 32-bit signed
+    if ((uint64_t)T >= (1ull << 31) || trows >= (1ull << 31)) return cudaErrorInvalidValue;
+    CUtensorMap m_k, m_v, m_u, m_w, m_mk;
     cudaError_t e = tma::map2d(&m_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, (uint64_t)Nqk * D, (uint64_t)T,
                                (uint64_t)Nqk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     if (e == cudaSuccess)
         e = tma::map2d(&m_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, (uint64_t)Nv * D, (uint64_t)T, (uint64_t)Nv * D * 2,
                        64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e == cudaSuccess)
+        e = tma::map2d(&m_u, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws.U, D, trows, D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e == cudaSuccess)
+        e = tma::map2d(&m_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws.W, D, trows, D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e == cudaSuccess)
+        e = tma::map2d(&m_mk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws.Mk, D, trows, D * 2, 64, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kIntraSmem);
     if (e != cudaSuccess) return e;
-    intra_kernel<<<dim3(NC, Nv), kIntraThreads, kIntraSmem, st>>>(m_k, m_v, T, Nqk, Nv, ws.chunk_info, ws.rk, ws.gcum,
-                                                                   ws.betaf, ws.U, ws.W, ws.Mk, ws.fa, ws.status);
+    intra_kernel<<<dim3(NC, Nv), kIntraThreads, kIntraSmem, st>>>(m_k, m_v, m_u, m_w, m_mk, T, Nqk, Nv, ws.chunk_info, ws.rk, ws.gcum,
+                                                                   ws.betaf, ws.fa, ws.status);
     return cudaGetLastError();
 }
 
