@@ -10,6 +10,8 @@
 //   o = (Q' - P W) S_c + P U,
 // so the chunk's state S_c enters one product.  Warp w handles rows
 // 32(w%4)..32(w%4)+31 and, in the epilogues, one half of the columns.  Steps:
+//   0. TMA loads of the raw q and k rows and of W; rows past a short chunk are
+//      zeroed after the load.
 //   1. q k^T     -- tcgen05.mma M=128, N=128, K=128 on the raw bf16 rows (exact
 //                   inputs), both K-major; fp32 accumulator in TMEM.
 //   2. P = rq_i rk_j exp(gamma_i - gamma_j) (q k^T)_ij for j <= i, else 0, read
@@ -24,36 +26,42 @@
 //   3. Z = P W  -- M=128, N=128, K=128, fp16 (W read MN-major); then
 //      Qw = diag(rq e^gamma) q - Z in fp16, in place of q.
 //   4. O = Qw S_c + P U for Dv columns 0..63, then 64..127 -- 16 tcgen05.mma
-//      each (N = 64); S_c and U are staged one column half at a time in the
-//      buffer W used, and each half is stored while the next one loads.
-// One thread issues the MMAs and waits for their completion (mbarrier arrival
-// from tcgen05.commit, bounded wait); a CTA barrier passes the outcome on.  If
-// a wait gives up, the CTA sets bit 1 of status[2] in the workspace and skips
-// the rest of its chunk after letting its MMAs drain.
+//      each (N = 64), both halves kept in TMEM; S_c and U arrive one column half
+//      at a time by TMA in the buffer W used.
+//   5. O in bf16 is staged over the consumed Qw tile and leaves by TMA for a
+//      full chunk; a short chunk's rows are stored by the threads, so rows of
+//      the next sequence are never written.
+// One thread issues the MMAs and copies and waits for their completion
+// (mbarriers, bounded waits); a CTA barrier passes the outcome on.  If a wait
+// gives up, the CTA sets bit 1 of status[2] in the workspace and skips the rest
+// of its chunk after letting its copies and MMAs drain.
 #include "common.cuh"
 #include "gdn_internal.h"
 #include "tc100.cuh"
+#include "tma.cuh"
 
 namespace gdn {
 
 constexpr int kOutThreads = 256;
-// shared memory, relative to a 1024-byte aligned base
-constexpr int OO_Q = 0;         // q (bf16) then Qw (fp16): K-major over Dk, 2 halves x 128 rows x 128 B
-constexpr int OO_K = 32768;     // k (bf16), K-major over Dk; then P (fp16), K-major over j
-constexpr int OO_X = 65536;     // W (fp16) [L][Dk] in two 64-column blocks (MN-major B of P W); then
-                                // S_c[:, half] (fp16) [Dk][64] and, 16 KiB on, U[:, half] (fp16) [L][64]
-constexpr int OO_VEC = 98304;   // gam, rqv, rkv, kfe (rk_j e^{gamma_je - gamma_j})
+// shared memory, relative to a 1024-byte aligned base; 128 x 128 16-bit tiles are
+// two 64-column halves of 128-byte rows with the 128-byte swizzle
+constexpr int OO_Q = 0;        // q (bf16) -> Qw (fp16), K-major over Dk -> O (bf16) for the store
+constexpr int OO_K = 32768;    // k (bf16), K-major over Dk -> P (fp16), K-major over j
+constexpr int OO_X = 65536;    // W (fp16) [L][Dk] (MN-major B of P W) -> S_c[:, half] [Dk][64] and,
+                               // 16 KiB on, U[:, half] [L][64] (fp16, MN-major)
+constexpr int OO_VEC = 98304;  // gam, rqv, rkv, kfe (rk_j e^{gamma_je - gamma_j})
 constexpr int OO_BAR = OO_VEC + 4 * 512;
 constexpr int kOutSmem = OO_BAR + 64 + 1024;
 
-// byte offset of 16-byte chunk c (0..15) of row r in a 128-row, 128-element tile
+// byte offset of 16-byte chunk c (0..15) of row r in a 128 x 128 tile
 __device__ __forceinline__ uint32_t t128(int r, int c) { return (uint32_t)((c >> 3) * 16384) + tc::sw128c(r, c & 7); }
 
 __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
-    const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, uint16_t *__restrict__ out, int T, int Nqk,
-    int Nv, const int4 *__restrict__ info, const float *__restrict__ rq, const float *__restrict__ rk,
-    const float *__restrict__ gcum, const uint16_t *__restrict__ U, const uint16_t *__restrict__ W,
-    const uint16_t *__restrict__ Sc, int32_t *__restrict__ status)
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sc,
+    const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_out, uint16_t *__restrict__ out,
+    int T, int Nqk, int Nv, const int4 *__restrict__ info, const float *__restrict__ rq, const float *__restrict__ rk,
+    const float *__restrict__ gcum, int32_t *__restrict__ status)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
@@ -68,57 +76,48 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     const int row = quarter * 32 + lane;
     float *gam = reinterpret_cast<float *>(smem + OO_VEC);
     float *rqv = gam + 128, *rkv = gam + 256, *kfe = gam + 384;
-    const uint32_t bar_qk = sbase + OO_BAR, bar_z = sbase + OO_BAR + 8, bar_o = sbase + OO_BAR + 16;
+    const uint32_t bar_ld = sbase + OO_BAR, bar_mma = sbase + OO_BAR + 8, bar_d = sbase + OO_BAR + 16;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + OO_BAR + 24);
-    const size_t tile = (size_t)(c * Nv + h) * L * D;
+    const int trow = (c * Nv + h) * L;  // first row of the chunk's tiles in the workspace
 
-    // S_c and U columns [64 hf, 64 hf + 64) into the MN-major buffers
-    auto load_su = [&](int hf) {
-        for (int e = tid; e < 128 * 8; e += kOutThreads) {
-            const int r = e >> 3, cc = e & 7;
-            cp_async16(sbase + OO_X + tc::sw128c(r, cc), Sc + tile + (size_t)r * D + hf * 64 + cc * 8, true);
-            cp_async16(sbase + OO_X + 16384 + tc::sw128c(r, cc), U + tile + (size_t)r * D + hf * 64 + cc * 8, true);
-        }
-    };
-
-    // ---- async loads: q, k rows of the chunk (zero past n), W, gamma, rq, rk
-    for (int e = tid; e < 128 * 16; e += kOutThreads) {
-        const int r = e >> 4, cc = e & 15;
-        const bool ok = r < n;
-        const int t = t0 + (ok ? r : 0);
-        const uint32_t off = t128(r, cc);
-        cp_async16(sbase + OO_Q + off, q + ((size_t)t * Nqk + hq) * D + cc * 8, ok);
-        cp_async16(sbase + OO_K + off, k + ((size_t)t * Nqk + hq) * D + cc * 8, ok);
-        cp_async16(sbase + OO_X + off, W + tile + (size_t)r * D + cc * 8, true);
-    }
-    if (tid < 128) {
-        const int i = min(tid, n - 1);
-        cp_async4(smem_addr(gam + tid), gcum + (size_t)h * T + t0 + i);
-        cp_async4(smem_addr(rqv + tid), rq + (size_t)hq * T + t0 + i);
-        cp_async4(smem_addr(rkv + tid), rk + (size_t)hq * T + t0 + i);
-    }
-    cp_async_commit();
     if (tid == 0) {
-        tc::mbar_init(bar_qk, 1);
-        tc::mbar_init(bar_z, 1);
-        tc::mbar_init(bar_o, 1);
+        tc::mbar_init(bar_ld, 1);
+        tc::mbar_init(bar_mma, 1);
+        tc::mbar_init(bar_d, 1);
         tc::mbar_init_fence();
     }
     if (wid == 0) tc::tmem_alloc(smem_addr(tslot), 256);
-    cp_async_wait<0>();
-    tc::fence_proxy_async();
-    tc::fence_before_sync();
     __syncthreads();
-    tc::fence_after_sync();
-    const uint32_t tmem = *tslot;  // columns [0, 128): q k^T, then O; [128, 256): Z = P W
-    const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
+    if (tid == 0) {  // one arrival and 96 KiB for the first phase of bar_ld
+        tma::expect_tx(bar_ld, 98304);
+        tma::load_2d(sbase + OO_Q, &tm_q, hq * D, t0, bar_ld);
+        tma::load_2d(sbase + OO_Q + 16384, &tm_q, hq * D + 64, t0, bar_ld);
+        tma::load_2d(sbase + OO_K, &tm_k, hq * D, t0, bar_ld);
+        tma::load_2d(sbase + OO_K + 16384, &tm_k, hq * D + 64, t0, bar_ld);
+        tma::load_2d(sbase + OO_X, &tm_w, 0, trow, bar_ld);
+        tma::load_2d(sbase + OO_X + 16384, &tm_w, 64, trow, bar_ld);
+    }
+    if (tid < 128) {
+        const int i = min(tid, n - 1);
+        gam[tid] = gcum[(size_t)h * T + t0 + i];
+        rqv[tid] = rq[(size_t)hq * T + t0 + i];
+        rkv[tid] = rk[(size_t)hq * T + t0 + i];
+    }
+    // S_c and U columns [64 hf, 64 hf + 64) into the MN-major buffers (thread 0), on bar_ld
+    int ld_issued = 1;  // load phases issued on bar_ld (thread 0)
+    auto load_su = [&](int hf) {
+        ++ld_issued;
+        tma::expect_tx(bar_ld, 32768);
+        tma::load_2d(sbase + OO_X, &tm_sc, hf * 64, trow, bar_ld);
+        tma::load_2d(sbase + OO_X + 16384, &tm_u, hf * 64, trow, bar_ld);
+    };
     bool ok = true;
-    uint32_t last_bar = bar_qk, last_par = 0;  // the most recent commit (thread 0)
-    auto wait_mma = [&](uint32_t bar, uint32_t parity) {
+    uint32_t ld_phase = 0;
+    auto wait_bar = [&](uint32_t bar, uint32_t parity) {  // bounded, outcome shared with the CTA
         bool w_ok = true;
         if (tid == 0) w_ok = tc::mbar_wait_bounded(bar, parity);
         tc::fence_before_sync();
-        ok = __syncthreads_and(w_ok) != 0;
+        ok = __syncthreads_and(w_ok) != 0 && ok;
         tc::fence_after_sync();
     };
     auto sync_operands = [&]() {  // generic-proxy shared-memory writes -> tensor core
@@ -130,16 +129,29 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     // descriptor of K step kk of a K-major tile with two 64-column K halves
     auto kmaj = [](uint64_t d, int kk) { return d + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4); };
 
+    wait_bar(bar_ld, ld_phase);
+    ld_phase ^= 1;
+    if (n < L) {  // q and k rows past the chunk belong to the next sequence (W is zero there)
+        for (int e = tid; e < (L - n) * 32; e += kOutThreads) {
+            const int r = n + (e >> 5), tl = (e >> 4) & 1, blk = (e >> 3) & 1, cc = e & 7;
+            *reinterpret_cast<uint4 *>(smem + (tl ? OO_K : OO_Q) + blk * 16384 + r * 128 + cc * 16) =
+                make_uint4(0, 0, 0, 0);
+        }
+    }
+    if (tid < 128) kfe[tid] = rkv[tid] * __expf(gam[tid | 15] - gam[tid]);
+    sync_operands();
+    const uint32_t tmem = *tslot;  // columns [0, 128): q k^T, then O; [128, 256): Z = P W
+    const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
+
     // ---- (1) q k^T
-    if (tid == 0) {
+    if (ok && tid == 0) {
         const uint64_t dq = tc::desc_k128(sbase + OO_Q), dk = tc::desc_k128(sbase + OO_K);
         const uint32_t idesc = tc::idesc_f16(128, 128, true, true);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) tc::mma_f16(tmem, kmaj(dq, kk), kmaj(dk, kk), idesc, kk > 0 ? 1u : 0u);
-        tc::commit(bar_qk);
+        tc::commit(bar_mma);
     }
-    if (tid < 128) kfe[tid] = rkv[tid] * __expf(gam[tid | 15] - gam[tid]);
-    wait_mma(bar_qk, 0);
+    if (ok) wait_bar(bar_mma, 0);
 
     if (ok) {
         // ---- (2) P, this thread's 64 columns of its row (fp16 over the k tile)
@@ -183,23 +195,21 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
                 }
             }
         }
-        sync_operands();
-
-        // ---- (3) Z = P W, then Qw = diag(rq e^gamma) q - Z over q
-        if (tid == 0) {
-            const uint64_t dp = tc::desc_k128(sbase + OO_K), dw = tc::desc_mn(sbase + OO_X, 16384, 1024, 2);
-            const uint32_t idesc = tc::idesc_f16(128, 128, false, false, false, true);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                tc::mma_f16(tmem + 128, kmaj(dp, kk), dw + (uint64_t)((kk * 2048) >> 4), idesc, kk > 0 ? 1u : 0u);
-            tc::commit(bar_z);
-            last_bar = bar_z;
-        }
-        wait_mma(bar_z, 0);
     }
+    sync_operands();
+
+    // ---- (3) Z = P W into TMEM columns [128, 256), then Qw = diag(rq e^gamma) q - Z over q
+    if (ok && tid == 0) {
+        const uint64_t dp = tc::desc_k128(sbase + OO_K), dw = tc::desc_mn(sbase + OO_X, 16384, 1024, 2);
+        const uint32_t idesc = tc::idesc_f16(128, 128, false, false, false, true);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+            tc::mma_f16(tmem + 128, kmaj(dp, kk), dw + (uint64_t)((kk * 2048) >> 4), idesc, kk > 0 ? 1u : 0u);
+        tc::commit(bar_mma);
+    }
+    if (ok) wait_bar(bar_mma, 1);
+    if (ok && tid == 0) load_su(0);  // W is consumed
     if (ok) {
-        load_su(0);  // W is consumed
-        cp_async_commit();
         const float qf = rqv[row] * __expf(gam[row]);
 #pragma unroll 1
         for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
@@ -218,16 +228,19 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
                 *p = make_uint4(o4[0], o4[1], o4[2], o4[3]);
             }
         }
-        cp_async_wait<0>();
-        sync_operands();
+    }
 
+    // ---- (4) O[:, 64 hf : 64 hf + 64] = Qw S_c + P U into TMEM columns [64 hf, 64 hf + 64)
+    {
         const uint64_t dq = tc::desc_k128(sbase + OO_Q), dp = tc::desc_k128(sbase + OO_K);
         const uint64_t ds = tc::desc_mn(sbase + OO_X, 16384, 1024, 2), du = tc::desc_mn(sbase + OO_X + 16384, 16384, 1024, 2);
         const uint32_t idesc = tc::idesc_f16(128, 64, false, false, false, true);
 #pragma unroll 1
-        for (int hf = 0; hf < 2 && ok; ++hf) {
-            // ---- (4) O[:, 64 hf : 64 hf + 64] = Qw S_c + P U
-            if (tid == 0) {
+        for (int hf = 0; hf < 2; ++hf) {
+            if (ok) wait_bar(bar_ld, ld_phase);  // S_c and U of this column half have landed
+            ld_phase ^= 1;
+            sync_operands();
+            if (ok && tid == 0) {
                 const uint32_t dst = tmem + hf * 64;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
@@ -235,40 +248,53 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_f16(dst, kmaj(dp, kk), du + (uint64_t)((kk * 2048) >> 4), idesc, 1u);
-                tc::commit(bar_o);
-                last_bar = bar_o;
-                last_par = (uint32_t)hf;
+                tc::commit(bar_mma);
             }
-            wait_mma(bar_o, (uint32_t)hf);
-            if (!ok) break;
-            if (hf == 0) {  // the buffers are free: start the second half's loads
-                load_su(1);
-                cp_async_commit();
-            }
-            // ---- this thread's 32 columns of the half, to bf16 (TMEM reads are warp-collective)
-            {
-                float a[32];
-                tc::tmem_ld32(t_row + hf * 64 + half * 32, a);
-                if (row < n) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)(t0 + row) * Nv + h) * D + hf * 64 + half * 32);
-#pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8)
-                        dst[q8] = make_uint4(pack_bf2(a[q8 * 8], a[q8 * 8 + 1]), pack_bf2(a[q8 * 8 + 2], a[q8 * 8 + 3]),
-                                             pack_bf2(a[q8 * 8 + 4], a[q8 * 8 + 5]),
-                                             pack_bf2(a[q8 * 8 + 6], a[q8 * 8 + 7]));
-                }
-            }
-            if (hf == 0) {
-                cp_async_wait<0>();
-                sync_operands();
-            }
+            if (ok) wait_bar(bar_mma, (uint32_t)hf);  // third and fourth phases of bar_mma
+            if (ok && hf == 0 && tid == 0) load_su(1);  // the buffers are free
         }
     }
-    cp_async_wait<0>();
-    if (!ok && tid == 0) {  // let the MMAs drain before TMEM is freed (a commit covers all earlier MMAs)
+
+    // ---- (5) O to bf16: a full chunk through shared memory (over Qw) and TMA, a short one row by row
+    if (ok) {
+        const bool full = n == L;
+#pragma unroll 1
+        for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
+            float a[32];
+            tc::tmem_ld32(t_row + j0, a);
+            uint4 w[4];
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8)
+                w[q8] = make_uint4(pack_bf2(a[q8 * 8], a[q8 * 8 + 1]), pack_bf2(a[q8 * 8 + 2], a[q8 * 8 + 3]),
+                                   pack_bf2(a[q8 * 8 + 4], a[q8 * 8 + 5]), pack_bf2(a[q8 * 8 + 6], a[q8 * 8 + 7]));
+            if (full) {
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8)
+                    *reinterpret_cast<uint4 *>(smem + OO_Q + t128(row, (j0 >> 3) + q8)) = w[q8];
+            } else if (row < n) {
+                uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)(t0 + row) * Nv + h) * D + j0);
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) dst[q8] = w[q8];
+            }
+        }
+        if (full) {
+            tc::fence_proxy_async();
+            __syncthreads();
+            if (tid == 0) {
+                tma::store_2d(&tm_out, h * D, t0, sbase + OO_Q);
+                tma::store_2d(&tm_out, h * D + 64, t0, sbase + OO_Q + 16384);
+                tma::commit_group();
+            }
+        }
+    } else if (tid == 0) {
         atomicOr(status + 2, 2);
-        tc::mbar_wait_bounded(last_bar, last_par);
+        // copies and MMAs still in flight land before shared and tensor memory are released:
+        // a commit covers every MMA issued before it; then the last load phase issued
+        tc::commit(bar_d);
+        tc::mbar_wait_bounded(bar_d, 0);
+        tc::mbar_wait_bounded(bar_ld, (uint32_t)((ld_issued - 1) & 1));
     }
+    if (tid == 0) tma::wait_all();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -278,11 +304,23 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
 cudaError_t launch_output(const uint16_t *q, const uint16_t *k, uint16_t *out, int T, int Nqk, int Nv, int NC,
                           const Workspace &ws, cudaStream_t st)
 {
-    if (NC == 0) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
+    if (NC == 0 || T == 0) return cudaSuccess;
+    const uint64_t trows = (uint64_t)NC * Nv * L;  // TMA coordinates are 32-bit signed
+    if ((uint64_t)T >= (1ull << 31) || trows >= (1ull << 31)) return cudaErrorInvalidValue;
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, HF = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+    CUtensorMap m_q, m_k, m_w, m_sc, m_u, m_out;
+    cudaError_t e = tma::map2d(&m_q, BF, q, (uint64_t)Nqk * D, (uint64_t)T, (uint64_t)Nqk * D * 2, 64, 128, SW);
+    if (e == cudaSuccess) e = tma::map2d(&m_k, BF, k, (uint64_t)Nqk * D, (uint64_t)T, (uint64_t)Nqk * D * 2, 64, 128, SW);
+    if (e == cudaSuccess) e = tma::map2d(&m_w, HF, ws.W, D, trows, D * 2, 64, 128, SW);
+    if (e == cudaSuccess) e = tma::map2d(&m_sc, HF, ws.Sc, D, trows, D * 2, 64, 128, SW);
+    if (e == cudaSuccess) e = tma::map2d(&m_u, HF, ws.U, D, trows, D * 2, 64, 128, SW);
+    if (e == cudaSuccess) e = tma::map2d(&m_out, BF, out, (uint64_t)Nv * D, (uint64_t)T, (uint64_t)Nv * D * 2, 64, 128, SW);
     if (e != cudaSuccess) return e;
-    output_kernel<<<dim3(NC, Nv), kOutThreads, kOutSmem, st>>>(q, k, out, T, Nqk, Nv, ws.chunk_info, ws.rq, ws.rk,
-                                                                ws.gcum, ws.U, ws.W, ws.Sc, ws.status);
+    e = cudaFuncSetAttribute(output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
+    if (e != cudaSuccess) return e;
+    output_kernel<<<dim3(NC, Nv), kOutThreads, kOutSmem, st>>>(m_q, m_k, m_w, m_sc, m_u, m_out, out, T, Nqk, Nv,
+                                                                ws.chunk_info, ws.rq, ws.rk, ws.gcum, ws.status);
     return cudaGetLastError();
 }
 
