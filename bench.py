@@ -1,8 +1,8 @@
 #!/usr/bin/env python
 """Benchmark of the Gated Delta Rule chunked forward on B200.
 
-One step = one forward pass (chunk table, prologue, intra-chunk, state pass,
-output) over the one-layer prefill workload: B = 1, T = 32768 tokens,
+One step = one forward pass (chunk table, intra-chunk, state pass, output)
+over the one-layer prefill workload: B = 1, T = 32768 tokens,
 Nqk = 16, Nv = 32, Dk = Dv = 128, L = 128, bf16 q/k/v/beta, fp32 g, inputs
 already resident in HBM.  Every rank of a multi-GPU run processes its own
 batch (independent problems, weak scaling, no collective on the data path).
@@ -50,8 +50,6 @@ def stage_work(T, Nqk, Nv):
     """Algorithmic work of one launch of each stage: (bound, amount, unit)."""
     return {
         "chunk_map": ("hbm", 0.0, "GB/s"),
-        # q and k read once, g and beta read, norm factors / gamma / beta written
-        "prologue": ("hbm", T * (2 * Nqk * D * 2 + Nv * 4 + Nv * 2 + 2 * Nqk * 4 + 2 * Nv * 4), "GB/s"),
         "intra": ("tensor", T * (Nv * (2 * L * D + 2 * L * D) + Nqk * 2 * L * D), "TFLOP/s"),
         "state": ("tensor", T * Nv * 4 * D * D, "TFLOP/s"),
         "output": ("tensor", T * (Nv * (2 * D * D + 2 * L * D) + Nqk * 2 * L * D), "TFLOP/s"),
@@ -217,14 +215,13 @@ def main():
     out = torch.empty(T, Nv, D, dtype=torch.bfloat16, device=dev)
     fin = torch.empty(B, Nv, D, D, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
-    names = ["chunk_map", "prologue", "intra", "state", "output"]
+    names = ["chunk_map", "intra", "state", "output"]
 
     def step(evs=None):
         calls = [lambda: st.chunk_map(inp.cu_seqlens),
-                 lambda: st.prologue(inp.q, inp.k, inp.g, inp.beta, inp.scale, inp.eps),
-                 lambda: st.intra(inp.k, inp.v),
+                 lambda: st.intra(inp.k, inp.v, inp.g, inp.beta, inp.eps),
                  lambda: st.state(inp.k, inp.state_pool, inp.state_indices, fin),
-                 lambda: st.output(inp.q, inp.k, out)]
+                 lambda: st.output(inp.q, inp.k, inp.g, out, inp.scale, inp.eps)]
         for i, c in enumerate(calls):
             if evs is not None:
                 evs[i].record(stream)

@@ -59,14 +59,12 @@ def lib():
         L.gdn_short_fwd.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, p]
         L.gdn_stage_chunk_map.restype = ctypes.c_int
         L.gdn_stage_chunk_map.argtypes = [p, i64, i32, i32, i32, p, sz, p]
-        L.gdn_stage_prologue.restype = ctypes.c_int
-        L.gdn_stage_prologue.argtypes = [p, p, p, p, f32, f32, i64, i32, i32, i32, p, sz, p]
         L.gdn_stage_intra.restype = ctypes.c_int
-        L.gdn_stage_intra.argtypes = [p, p, i64, i32, i32, i32, p, sz, p]
+        L.gdn_stage_intra.argtypes = [p, p, p, p, f32, i64, i32, i32, i32, p, sz, p]
         L.gdn_stage_state.restype = ctypes.c_int
         L.gdn_stage_state.argtypes = [p, p, p, p, i64, i32, i32, i32, i32, p, sz, p]
         L.gdn_stage_output.restype = ctypes.c_int
-        L.gdn_stage_output.argtypes = [p, p, p, i64, i32, i32, i32, p, sz, p]
+        L.gdn_stage_output.argtypes = [p, p, p, f32, f32, p, i64, i32, i32, i32, p, sz, p]
         _lib = L
     return _lib
 
@@ -213,7 +211,7 @@ def short_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None,
 
 
 class Stages:
-    """The five kernels of the chunked path as separate calls on one workspace.
+    """The four kernels of the chunked path as separate calls on one workspace.
 
     After ``run_all`` (or the individual calls in order) the intermediates are
     readable through the typed views ``U``, ``W``, ``Mk``, ``Sc``, ``rq``,
@@ -276,15 +274,9 @@ class Stages:
         _check(lib().gdn_stage_chunk_map(_ptr(cu_seqlens), self.T, self.B, self.Nqk, self.Nv, _ptr(self.ws),
                                          self.nbytes, _stream(stream)), "gdn_stage_chunk_map")
 
-    def prologue(self, q, k, g, beta, scale=None, eps=1e-6, stream=None):
-        sc = 0.0 if scale is None else float(scale)
-        _check(lib().gdn_stage_prologue(_ptr(q), _ptr(k), _ptr(g), _ptr(beta), sc, float(eps), self.T, self.B,
-                                        self.Nqk, self.Nv, _ptr(self.ws), self.nbytes, _stream(stream)),
-               "gdn_stage_prologue")
-
-    def intra(self, k, v, stream=None):
-        _check(lib().gdn_stage_intra(_ptr(k), _ptr(v), self.T, self.B, self.Nqk, self.Nv, _ptr(self.ws), self.nbytes,
-                                     _stream(stream)), "gdn_stage_intra")
+    def intra(self, k, v, g, beta, eps=1e-6, stream=None):
+        _check(lib().gdn_stage_intra(_ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(eps), self.T, self.B, self.Nqk,
+                                     self.Nv, _ptr(self.ws), self.nbytes, _stream(stream)), "gdn_stage_intra")
 
     def state(self, k, state_pool=None, state_indices=None, final_state=None, stream=None):
         P = 0 if state_pool is None else int(state_pool.shape[0])
@@ -292,9 +284,10 @@ class Stages:
                                      self.B, self.Nqk, self.Nv, P, _ptr(self.ws), self.nbytes, _stream(stream)),
                "gdn_stage_state")
 
-    def output(self, q, k, out, stream=None):
-        _check(lib().gdn_stage_output(_ptr(q), _ptr(k), _ptr(out), self.T, self.B, self.Nqk, self.Nv,
-                                      _ptr(self.ws), self.nbytes, _stream(stream)), "gdn_stage_output")
+    def output(self, q, k, g, out, scale=None, eps=1e-6, stream=None):
+        sc = 0.0 if scale is None else float(scale)
+        _check(lib().gdn_stage_output(_ptr(q), _ptr(k), _ptr(g), sc, float(eps), _ptr(out), self.T, self.B, self.Nqk,
+                                      self.Nv, _ptr(self.ws), self.nbytes, _stream(stream)), "gdn_stage_output")
 
     def run_all(self, q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None, scale=None, eps=1e-6,
                 out=None, final_state=None, stream=None):
@@ -304,10 +297,9 @@ class Stages:
         if final_state is None:
             final_state = torch.empty(self.B, self.Nv, HEAD_DIM, HEAD_DIM, dtype=torch.float32, device=dev)
         self.chunk_map(cu_seqlens, stream)
-        self.prologue(q, k, g, beta, scale, eps, stream)
-        self.intra(k, v, stream)
+        self.intra(k, v, g, beta, eps, stream)
         self.state(k, state_pool, state_indices, final_state, stream)
-        self.output(q, k, out, stream)
+        self.output(q, k, g, out, scale, eps, stream)
         return out, final_state
 
 

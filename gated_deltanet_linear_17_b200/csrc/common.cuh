@@ -191,4 +191,50 @@ __device__ __forceinline__ ChunkInfo load_chunk(const int4 *info, int c)
     return ChunkInfo{v.x, v.y, v.z, v.w};
 }
 
+// Chunk-local cumulative gate ("Gate Cumulative Sum"): gam[i] = sum_{j <= i} g[t0 + j][h]
+// over the chunk's n rows; rows i >= n add nothing, so they repeat the last valid
+// value.  Every thread of the CTA calls it (it holds barriers); threads 0..127
+// produce gam[i]; wsum is 4 floats of shared scratch.  The kernels that need the
+// gate all use this function, so they see the same fp32 values bit for bit.
+__device__ __forceinline__ void chunk_gamma(const float *__restrict__ g, int Nv, int h, int t0, int n, float *gam,
+                                            float *wsum)
+{
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    float x = (tid < 128 && tid < n) ? g[(size_t)(t0 + tid) * Nv + h] : 0.f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (tid < 128 && lane == 31) wsum[w] = x;
+    __syncthreads();
+    if (tid < 128) {
+        float pre = 0.f;
+        for (int j = 0; j < w; ++j) pre += wsum[j];
+        gam[tid] = x + pre;
+    }
+    __syncthreads();
+}
+
+// 1 / sqrt(|x_r|^2 + eps) for row r of a 128 x 128 16-bit tile of raw bf16 rows
+// stored as two 64-column halves of 128-byte rows with the 128-byte swizzle
+// ("L2 Normalization", eps inside the square root).  Same summation order in
+// every kernel that calls it.
+__device__ __forceinline__ float row_inv_norm(const uint8_t *tile, int r, float eps)
+{
+    float s = 0.f;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        const uint4 x = *reinterpret_cast<const uint4 *>(tile + (c >> 3) * 16384 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+        const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float a = __uint_as_float(w4[e] << 16), b = __uint_as_float(w4[e] & 0xffff0000u);
+            s = fmaf(a, a, s);
+            s = fmaf(b, b, s);
+        }
+    }
+    return 1.0f / sqrtf(s + eps);
+}
+
 }  // namespace gdn

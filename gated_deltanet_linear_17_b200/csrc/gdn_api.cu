@@ -183,34 +183,18 @@ int gdn_stage_chunk_map(const int32_t *cu_seqlens, int64_t T, int32_t B, int32_t
     return cuda_status(gdn::launch_chunk_map(cu_seqlens, B, (int)T, w.NC, w, (cudaStream_t)stream));
 }
 
-int gdn_stage_prologue(const uint16_t *q, const uint16_t *k, const float *g, const uint16_t *beta,
-                       float scale, float eps, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
-                       void *workspace, size_t workspace_bytes, void *stream)
+int gdn_stage_intra(const uint16_t *k, const uint16_t *v, const float *g, const uint16_t *beta, float eps, int64_t T,
+                    int32_t B, int32_t Nqk, int32_t Nv, void *workspace, size_t workspace_bytes, void *stream)
 {
     int rc = check_sizes(T, B, Nqk, Nv);
     if (rc) return rc;
     gdn_workspace_layout_t lay;
     if ((rc = check_workspace(workspace, workspace_bytes, T, B, Nqk, Nv, &lay))) return rc;
     if (B == 0 || T == 0) return GDN_OK;
-    if (!q || !k || !g || !beta) return GDN_ERR_NULL_ARG;
-    if (!aligned16(q) || !aligned16(k)) return GDN_ERR_ALIGNMENT;
-    const Workspace w = views(workspace, lay);
-    return cuda_status(gdn::launch_prologue(q, k, g, beta, resolve_scale(scale), eps, (int)T, Nqk, Nv, w.NC,
-                                            w, (cudaStream_t)stream));
-}
-
-int gdn_stage_intra(const uint16_t *k, const uint16_t *v, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
-                    void *workspace, size_t workspace_bytes, void *stream)
-{
-    int rc = check_sizes(T, B, Nqk, Nv);
-    if (rc) return rc;
-    gdn_workspace_layout_t lay;
-    if ((rc = check_workspace(workspace, workspace_bytes, T, B, Nqk, Nv, &lay))) return rc;
-    if (B == 0 || T == 0) return GDN_OK;
-    if (!k || !v) return GDN_ERR_NULL_ARG;
+    if (!k || !v || !g || !beta) return GDN_ERR_NULL_ARG;
     if (!aligned16(k) || !aligned16(v)) return GDN_ERR_ALIGNMENT;
     const Workspace w = views(workspace, lay);
-    return cuda_status(gdn::launch_intra(k, v, (int)T, Nqk, Nv, w.NC, w, (cudaStream_t)stream));
+    return cuda_status(gdn::launch_intra(k, v, g, beta, eps, (int)T, Nqk, Nv, w.NC, w, (cudaStream_t)stream));
 }
 
 int gdn_stage_state(const uint16_t *k, const float *state_pool, const int32_t *state_indices, float *final_state,
@@ -234,18 +218,20 @@ int gdn_stage_state(const uint16_t *k, const float *state_pool, const int32_t *s
                                          (cudaStream_t)stream));
 }
 
-int gdn_stage_output(const uint16_t *q, const uint16_t *k, uint16_t *out, int64_t T, int32_t B, int32_t Nqk,
-                     int32_t Nv, void *workspace, size_t workspace_bytes, void *stream)
+int gdn_stage_output(const uint16_t *q, const uint16_t *k, const float *g, float scale, float eps, uint16_t *out,
+                     int64_t T, int32_t B, int32_t Nqk, int32_t Nv, void *workspace, size_t workspace_bytes,
+                     void *stream)
 {
     int rc = check_sizes(T, B, Nqk, Nv);
     if (rc) return rc;
     gdn_workspace_layout_t lay;
     if ((rc = check_workspace(workspace, workspace_bytes, T, B, Nqk, Nv, &lay))) return rc;
     if (B == 0 || T == 0) return GDN_OK;
-    if (!q || !k || !out) return GDN_ERR_NULL_ARG;
+    if (!q || !k || !g || !out) return GDN_ERR_NULL_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(out)) return GDN_ERR_ALIGNMENT;
     const Workspace w = views(workspace, lay);
-    return cuda_status(gdn::launch_output(q, k, out, (int)T, Nqk, Nv, w.NC, w, (cudaStream_t)stream));
+    return cuda_status(gdn::launch_output(q, k, g, resolve_scale(scale), eps, out, (int)T, Nqk, Nv, w.NC, w,
+                                          (cudaStream_t)stream));
 }
 
 int gdn_short_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
@@ -290,10 +276,9 @@ int gdn_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
     const Workspace w = views(workspace, lay);
     const int Ti = (int)T;
     cudaError_t e = gdn::launch_chunk_map(cu_seqlens, B, Ti, w.NC, w, st);
-    if (e == cudaSuccess) e = gdn::launch_prologue(q, k, g, beta, sc, eps, Ti, Nqk, Nv, w.NC, w, st);
-    if (e == cudaSuccess) e = gdn::launch_intra(k, v, Ti, Nqk, Nv, w.NC, w, st);
+    if (e == cudaSuccess) e = gdn::launch_intra(k, v, g, beta, eps, Ti, Nqk, Nv, w.NC, w, st);
     if (e == cudaSuccess) e = gdn::launch_state(k, state_pool, state_indices, final_state, Ti, B, Nqk, Nv, w, st);
-    if (e == cudaSuccess) e = gdn::launch_output(q, k, out, Ti, Nqk, Nv, w.NC, w, st);
+    if (e == cudaSuccess) e = gdn::launch_output(q, k, g, sc, eps, out, Ti, Nqk, Nv, w.NC, w, st);
     if (owned) {
         cudaError_t f = cudaFreeAsync(workspace, st);
         if (e == cudaSuccess) e = f;

@@ -25,15 +25,12 @@ struct Workspace {
 
 cudaError_t launch_chunk_map(const int32_t *cu, int B, int T, int NC, const Workspace &ws,
                              cudaStream_t st);
-cudaError_t launch_prologue(const uint16_t *q, const uint16_t *k, const float *g, const uint16_t *beta,
-                            float scale, float eps, int T, int Nqk, int Nv, int NC, const Workspace &ws,
-                            cudaStream_t st);
-cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, int T, int Nqk, int Nv, int NC, const Workspace &ws,
-                         cudaStream_t st);
+cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, const float *g, const uint16_t *beta, float eps, int T,
+                         int Nqk, int Nv, int NC, const Workspace &ws, cudaStream_t st);
 cudaError_t launch_state(const uint16_t *k, const float *pool, const int32_t *idx, float *final_state, int T, int B,
                          int Nqk, int Nv, const Workspace &ws, cudaStream_t st);
-cudaError_t launch_output(const uint16_t *q, const uint16_t *k, uint16_t *out, int T, int Nqk, int Nv, int NC,
-                          const Workspace &ws, cudaStream_t st);
+cudaError_t launch_output(const uint16_t *q, const uint16_t *k, const float *g, float scale, float eps, uint16_t *out,
+                          int T, int Nqk, int Nv, int NC, const Workspace &ws, cudaStream_t st);
 cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                          const uint16_t *beta, const int32_t *cu, const float *pool, const int32_t *idx,
                          float scale, float eps, uint16_t *out, float *final_state, int T, int B, int Nqk,

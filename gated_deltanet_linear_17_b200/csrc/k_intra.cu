@@ -87,10 +87,9 @@ __device__ __forceinline__ void warp_store16(const float (&acc)[2][4], uint8_t *
 __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_w,
-    const __grid_constant__ CUtensorMap tm_mk, int T, int Nqk, int Nv,
-    const int4 *__restrict__ info, const float *__restrict__ rk, const float *__restrict__ gcum,
-    const float *__restrict__ betaf,
-    float *__restrict__ fa, int32_t *__restrict__ status)
+    const __grid_constant__ CUtensorMap tm_mk, const float *__restrict__ g, const uint16_t *__restrict__ beta,
+    float eps, int T, int Nqk, int Nv, const int4 *__restrict__ info, float *__restrict__ rk_out,
+    float *__restrict__ gcum_out, float *__restrict__ betaf_out, float *__restrict__ fa, int32_t *__restrict__ status)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
@@ -129,12 +128,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
         tma::load_2d(sbase + OFF_K, &tm_k, hq * D, t0, bar_ld);
         tma::load_2d(sbase + OFF_K + 16384, &tm_k, hq * D + 64, t0, bar_ld);
     }
-    if (tid < 128) {
-        const int i = tid;
-        gam[i] = gcum[(size_t)h * T + t0 + min(i, n - 1)];
-        bet[i] = i < n ? betaf[(size_t)h * T + t0 + i] : 0.f;
-        rkv[i] = i < n ? rk[(size_t)hq * T + t0 + i] : 0.f;
-    }
+    // chunk-local cumulative gate and beta while the rows load
+    chunk_gamma(g, Nv, h, t0, n, gam, reinterpret_cast<float *>(smem + OFF_BAR + 32));
+    if (tid < 128) bet[tid] = tid < n ? bf2f(beta[(size_t)(t0 + tid) * Nv + h]) : 0.f;
     // zero the rows of a tile past the chunk (they belong to the next sequence)
     auto zero_tail = [&](int off) {
         for (int e = tid; e < (L - n) * 16; e += kIntraThreads) {
@@ -162,7 +158,6 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
         zero_tail(OFF_K);
         zero_tail(OFF_V);
     }
-    if (tid < 128) kfe[tid] = rkv[tid] * __expf(gam[tid | 15] - gam[tid]);
     sync_operands();
     const uint32_t tmem = *tslot;
     const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -176,7 +171,18 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
         for (int kk = 0; kk < 8; ++kk) tc::mma_f16(tmem, kmaj(dk, kk), kmaj(dk, kk), idesc, kk > 0 ? 1u : 0u);
         tc::commit(bar_mma);
     }
-    // meanwhile: diag(beta) v in fp16, in place
+    // meanwhile: 1/|k| of the valid rows ("L2 Normalization") and the decay factors ...
+    if (tid < 128) {
+        rkv[tid] = tid < n ? row_inv_norm(smem + OFF_K, tid, eps) : 0.f;
+        if (tid < n) {  // for inspection through the stage interface
+            gcum_out[(size_t)h * T + t0 + tid] = gam[tid];
+            betaf_out[(size_t)h * T + t0 + tid] = bet[tid];
+            if (h % (Nv / Nqk) == 0) rk_out[(size_t)hq * T + t0 + tid] = rkv[tid];
+        }
+    }
+    __syncthreads();
+    if (tid < 128) kfe[tid] = rkv[tid] * __expf(gam[tid | 15] - gam[tid]);
+    // ... and diag(beta) v in fp16, in place
     for (int e = tid; e < 128 * 16; e += kIntraThreads) {
         const int r = e >> 4, cc = e & 15;
         uint4 *p = reinterpret_cast<uint4 *>(smem + OFF_V + t128(r, cc));
@@ -455,8 +461,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     if (wid == 0) tc::tmem_dealloc(tmem, 256);
 }
 
-cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, int T, int Nqk, int Nv, int NC, const Workspace &ws,
-                         cudaStream_t st)
+cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, const float *g, const uint16_t *beta, float eps, int T,
+                         int Nqk, int Nv, int NC, const Workspace &ws, cudaStream_t st)
 {
     if (NC == 0 || T == 0) return cudaSuccess;
     const uint64_t trows = (uint64_t)NC * Nv * L;  // TMA coordinates are 32-bit signed
@@ -477,8 +483,9 @@ cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, int T, int Nqk, i
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kIntraSmem);
     if (e != cudaSuccess) return e;
-    intra_kernel<<<dim3(NC, Nv), kIntraThreads, kIntraSmem, st>>>(m_k, m_v, m_u, m_w, m_mk, T, Nqk, Nv, ws.chunk_info, ws.rk, ws.gcum,
-                                                                   ws.betaf, ws.fa, ws.status);
+    intra_kernel<<<dim3(NC, Nv), kIntraThreads, kIntraSmem, st>>>(m_k, m_v, m_u, m_w, m_mk, g, beta, eps, T, Nqk, Nv,
+                                                                   ws.chunk_info, ws.rk, ws.gcum, ws.betaf, ws.fa,
+                                                                   ws.status);
     return cudaGetLastError();
 }
 

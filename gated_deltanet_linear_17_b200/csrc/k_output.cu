@@ -60,8 +60,8 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sc,
     const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_out, uint16_t *__restrict__ out,
-    int T, int Nqk, int Nv, const int4 *__restrict__ info, const float *__restrict__ rq, const float *__restrict__ rk,
-    const float *__restrict__ gcum, int32_t *__restrict__ status)
+    const float *__restrict__ g, float scale, float eps, int T, int Nqk, int Nv, const int4 *__restrict__ info,
+    float *__restrict__ rq_out, int32_t *__restrict__ status)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
@@ -97,12 +97,8 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         tma::load_2d(sbase + OO_X, &tm_w, 0, trow, bar_ld);
         tma::load_2d(sbase + OO_X + 16384, &tm_w, 64, trow, bar_ld);
     }
-    if (tid < 128) {
-        const int i = min(tid, n - 1);
-        gam[tid] = gcum[(size_t)h * T + t0 + i];
-        rqv[tid] = rq[(size_t)hq * T + t0 + i];
-        rkv[tid] = rk[(size_t)hq * T + t0 + i];
-    }
+    // chunk-local cumulative gate while the rows load
+    chunk_gamma(g, Nv, h, t0, n, gam, reinterpret_cast<float *>(smem + OO_BAR + 32));
     // S_c and U columns [64 hf, 64 hf + 64) into the MN-major buffers (thread 0), on bar_ld
     int ld_issued = 1;  // load phases issued on bar_ld (thread 0)
     auto load_su = [&](int hf) {
@@ -138,7 +134,6 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
                 make_uint4(0, 0, 0, 0);
         }
     }
-    if (tid < 128) kfe[tid] = rkv[tid] * __expf(gam[tid | 15] - gam[tid]);
     sync_operands();
     const uint32_t tmem = *tslot;  // columns [0, 128): q k^T, then O; [128, 256): Z = P W
     const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -151,6 +146,14 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         for (int kk = 0; kk < 8; ++kk) tc::mma_f16(tmem, kmaj(dq, kk), kmaj(dk, kk), idesc, kk > 0 ? 1u : 0u);
         tc::commit(bar_mma);
     }
+    // while it runs: scale/|q| and 1/|k| of the valid rows ("L2 Normalization") and the decay factors
+    if (tid < 128) {
+        rqv[tid] = tid < n ? scale * row_inv_norm(smem + OO_Q, tid, eps) : 0.f;
+        rkv[tid] = tid < n ? row_inv_norm(smem + OO_K, tid, eps) : 0.f;
+        if (tid < n && h % (Nv / Nqk) == 0) rq_out[(size_t)hq * T + t0 + tid] = rqv[tid];  // for inspection
+    }
+    __syncthreads();
+    if (tid < 128) kfe[tid] = rkv[tid] * __expf(gam[tid | 15] - gam[tid]);
     if (ok) wait_bar(bar_mma, 0);
 
     if (ok) {
@@ -301,8 +304,8 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     if (wid == 0) tc::tmem_dealloc(tmem, 256);
 }
 
-cudaError_t launch_output(const uint16_t *q, const uint16_t *k, uint16_t *out, int T, int Nqk, int Nv, int NC,
-                          const Workspace &ws, cudaStream_t st)
+cudaError_t launch_output(const uint16_t *q, const uint16_t *k, const float *g, float scale, float eps, uint16_t *out,
+                          int T, int Nqk, int Nv, int NC, const Workspace &ws, cudaStream_t st)
 {
     if (NC == 0 || T == 0) return cudaSuccess;
     const uint64_t trows = (uint64_t)NC * Nv * L;  // TMA coordinates are 32-bit signed
@@ -319,8 +322,8 @@ cudaError_t launch_output(const uint16_t *q, const uint16_t *k, uint16_t *out, i
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
     if (e != cudaSuccess) return e;
-    output_kernel<<<dim3(NC, Nv), kOutThreads, kOutSmem, st>>>(m_q, m_k, m_w, m_sc, m_u, m_out, out, T, Nqk, Nv,
-                                                                ws.chunk_info, ws.rq, ws.rk, ws.gcum, ws.status);
+    output_kernel<<<dim3(NC, Nv), kOutThreads, kOutSmem, st>>>(m_q, m_k, m_w, m_sc, m_u, m_out, out, g, scale, eps, T,
+                                                                Nqk, Nv, ws.chunk_info, ws.rq, ws.status);
     return cudaGetLastError();
 }
 

@@ -1,8 +1,8 @@
 /*
  * gdn_stages.h -- the kernels of gdn_chunk_fwd as separate C-ABI calls.
  *
- * gdn_chunk_fwd (gdn.h) is exactly gdn_stage_chunk_map, gdn_stage_prologue,
- * gdn_stage_intra, gdn_stage_state and gdn_stage_output enqueued in that order
+ * gdn_chunk_fwd (gdn.h) is exactly gdn_stage_chunk_map, gdn_stage_intra,
+ * gdn_stage_state and gdn_stage_output enqueued in that order
  * on one stream with one workspace.  The stages are exposed so that each
  * kernel can be checked against the chunked form's intermediates and timed on
  * its own.  Conventions (device pointers, bf16 as uint16_t bits, asynchronous
@@ -93,48 +93,41 @@ int gdn_stage_chunk_map(const int32_t *cu_seqlens, int64_t T, int32_t B, int32_t
                         void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * Prologue: per token and qk-head the L2 normalisation factors of q (times
- * scale) and k ("L2 Normalization", eps inside the square root), per chunk
- * and v-head the cumulative gate ("Gate Cumulative Sum") restarting at every
- * chunk start, and beta widened to fp32.  Reads q, k [T, Nqk, 128] bf16,
- * g [T, Nv] fp32, beta [T, Nv] bf16; writes rq, rk, gcum, betaf.
- * scale <= 0 selects 1/sqrt(128).
+ * Intra-chunk: per (chunk, v-head) the L2 normalisation factors of k ("L2
+ * Normalization", eps inside the square root), the cumulative gate ("Gate
+ * Cumulative Sum") restarting at every chunk start, A ("Pre-Attention
+ * Matrix"), T = (I + A)^-1 by the block merge of inverse_pto / inverse_matmul
+ * ("Matrix Inversion"), U and W ("Value and Key Cumulative Decay"), and
+ * Mk = k_gexp^T W with k_gexp = Kh * exp(g_last - g_cum) ("State Update").
+ * Reads k [T, Nqk, 128], v [T, Nv, 128] (bf16), g [T, Nv] fp32, beta [T, Nv]
+ * bf16; writes U, W, Mk, fa, and rk, gcum, betaf (for inspection).
  */
-int gdn_stage_prologue(const uint16_t *q, const uint16_t *k, const float *g, const uint16_t *beta,
-                       float scale, float eps, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
-                       void *workspace, size_t workspace_bytes, void *stream);
-
-/*
- * Intra-chunk: per (chunk, v-head) forms A ("Pre-Attention Matrix"), solves
- * T = (I + A)^-1 by blocked forward substitution ("Matrix Inversion" with the
- * block merge of inverse_pto / inverse_matmul), and computes U and W ("Value
- * and Key Cumulative Decay").  Reads k [T, Nqk, 128], v [T, Nv, 128] (bf16)
- * and the prologue's outputs; writes U, W and Mk = k_gexp^T W with
- * k_gexp = Kh * exp(g_last - g_cum) ("State Update").
- */
-int gdn_stage_intra(const uint16_t *k, const uint16_t *v, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
-                    void *workspace, size_t workspace_bytes, void *stream);
+int gdn_stage_intra(const uint16_t *k, const uint16_t *v, const float *g, const uint16_t *beta, float eps,
+                    int64_t T, int32_t B, int32_t Nqk, int32_t Nv, void *workspace, size_t workspace_bytes,
+                    void *stream);
 
 /*
  * Inter-chunk state passing: per (sequence, v-head, 32-column slice of Dv),
  * serially over the sequence's chunks, S <- e^{gamma_last} S + k_gexp^T U - Mk S
  * ("State Update" with v' = W S regrouped), the state kept in fp32 on chip.
  * S starts from state_pool[state_indices[b]] (or slot b, or zero without a
- * pool).  Reads k [T, Nqk, 128] bf16, rk, gcum, U and Mk; writes Sc for every
- * chunk and final_state (if not NULL).
+ * pool).  Reads k [T, Nqk, 128] bf16, fa, U and Mk; writes Sc for every chunk
+ * and final_state (if not NULL).
  */
 int gdn_stage_state(const uint16_t *k, const float *state_pool, const int32_t *state_indices, float *final_state,
                     int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P, void *workspace,
                     size_t workspace_bytes, void *stream);
 
 /*
- * Output: per (chunk, v-head) o = diag(e^gamma) Qh S_c + (Qh Kh^T * Gamma * tril) U'
- * ("Recurrent State Attention": o_inter and o_chunk; tril includes the
- * diagonal).  Reads q, k [T, Nqk, 128] bf16, rq, rk, gcum, Sc, U' (in U); writes
- * out [T, Nv, 128] bf16 for every token of every chunk.
+ * Output: per (chunk, v-head) o = (diag(e^gamma) Qh - P W) S_c + P U with
+ * P = Qh Kh^T * Gamma * tril ("Recurrent State Attention": o_inter and
+ * o_chunk regrouped; tril includes the diagonal).  Reads q, k [T, Nqk, 128]
+ * bf16, g [T, Nv] fp32, W, U, Sc; writes out [T, Nv, 128] bf16 for every token
+ * of every chunk, and rq (for inspection).  scale <= 0 selects 1/sqrt(128).
  */
-int gdn_stage_output(const uint16_t *q, const uint16_t *k, uint16_t *out, int64_t T, int32_t B, int32_t Nqk,
-                     int32_t Nv, void *workspace, size_t workspace_bytes, void *stream);
+int gdn_stage_output(const uint16_t *q, const uint16_t *k, const float *g, float scale, float eps, uint16_t *out,
+                     int64_t T, int32_t B, int32_t Nqk, int32_t Nv, void *workspace, size_t workspace_bytes,
+                     void *stream);
 
 /*
  * Fused short-sequence forward: the token recurrence of the decode page

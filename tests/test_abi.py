@@ -34,7 +34,7 @@ def lib():
 def test_headers_declare_entry_points():
     names = _declared()
     for n in ("gdn_chunk_fwd", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string", "gdn_short_fwd",
-              "gdn_stage_intra", "gdn_stage_state", "gdn_stage_output", "gdn_stage_prologue"):
+              "gdn_stage_intra", "gdn_stage_state", "gdn_stage_output"):
         assert n in names
 
 
@@ -107,9 +107,10 @@ def test_argument_errors_before_any_launch(lib):
 
 def test_stage_argument_errors(lib):
     vp = ctypes.c_void_p
-    assert lib.gdn_stage_intra(vp(16), vp(16), 8, 1, 2, 4, None, 0, None) == B.GDN_ERR_NULL_ARG
-    assert lib.gdn_stage_intra(vp(16), vp(16), 8, 1, 2, 4, vp(16), 10, None) == B.GDN_ERR_WORKSPACE
-    assert lib.gdn_stage_output(vp(16), vp(16), vp(16), 8, 1, 2, 3, vp(16), 1 << 30, None) == B.GDN_ERR_BAD_SHAPE
+    x = vp(16)
+    assert lib.gdn_stage_intra(x, x, x, x, 1e-6, 8, 1, 2, 4, None, 0, None) == B.GDN_ERR_NULL_ARG
+    assert lib.gdn_stage_intra(x, x, x, x, 1e-6, 8, 1, 2, 4, x, 10, None) == B.GDN_ERR_WORKSPACE
+    assert lib.gdn_stage_output(x, x, x, 0.0, 1e-6, x, 8, 1, 2, 3, x, 1 << 30, None) == B.GDN_ERR_BAD_SHAPE
 
 
 def test_python_layer_refuses_cpu_tensors():

@@ -81,10 +81,9 @@ def test_stages_match_chunked_intermediates():
     out = torch.empty(inp.T, inp.Nv, 128, dtype=torch.bfloat16, device=DEV)
     fin = torch.empty(inp.B, inp.Nv, 128, 128, dtype=torch.float32, device=DEV)
     st.chunk_map(d.cu_seqlens)
-    st.prologue(d.q, d.k, d.g, d.beta, inp.scale, inp.eps)
-    st.intra(d.k, d.v)
+    st.intra(d.k, d.v, d.g, d.beta, inp.eps)
     st.state(d.k, d.state_pool, d.state_indices, fin)
-    st.output(d.q, d.k, out)
+    st.output(d.q, d.k, d.g, out, inp.scale, inp.eps)
     torch.cuda.synchronize()
     X = {n: oracle.as_numpy_exact(getattr(inp, n)) for n in ("q", "k", "v", "g", "beta")}
     _, _, kept = oracle.chunked(X["q"], X["k"], X["v"], X["g"], X["beta"], inp.cu_seqlens.numpy(),
