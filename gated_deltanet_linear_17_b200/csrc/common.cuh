@@ -218,23 +218,28 @@ __device__ __forceinline__ void chunk_gamma(const float *__restrict__ g, int Nv,
 
 // 1 / sqrt(|x_r|^2 + eps) for row r of a 128 x 128 16-bit tile of raw bf16 rows
 // stored as two 64-column halves of 128-byte rows with the 128-byte swizzle
-// ("L2 Normalization", eps inside the square root).  Same summation order in
-// every kernel that calls it.
-__device__ __forceinline__ float row_inv_norm(const uint8_t *tile, int r, float eps)
+// ("L2 Normalization", eps inside the square root).  Two adjacent lanes share a
+// row (part = lane & 1): part 0 sums the first 64 columns, part 1 the last 64, each
+// 16-byte chunk in an order that keeps a quarter-warp on eight distinct bank
+// groups, with four partial sums; both lanes get the result.  Same summation
+// order in every kernel that calls it.
+__device__ __forceinline__ float row_inv_norm_pair(const uint8_t *tile, int r, int part, float eps)
 {
-    float s = 0.f;
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-        const uint4 x = *reinterpret_cast<const uint4 *>(tile + (c >> 3) * 16384 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+    for (int i = 0; i < 8; ++i) {
+        const int cc = i ^ (part << 2);  // column chunk within the half
+        const uint4 x = *reinterpret_cast<const uint4 *>(tile + part * 16384 + r * 128 + ((cc ^ (r & 7)) << 4));
         const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const float a = __uint_as_float(w4[e] << 16), b = __uint_as_float(w4[e] & 0xffff0000u);
-            s = fmaf(a, a, s);
-            s = fmaf(b, b, s);
+            s[e] = fmaf(b, b, fmaf(a, a, s[e]));
         }
     }
-    return 1.0f / sqrtf(s + eps);
+    float t = (s[0] + s[1]) + (s[2] + s[3]);
+    t += __shfl_xor_sync(0xffffffffu, t, 1);
+    return 1.0f / sqrtf(t + eps);
 }
 
 }  // namespace gdn

@@ -84,6 +84,34 @@ __device__ __forceinline__ void warp_store16(const float (&acc)[2][4], uint8_t *
         }
 }
 
+// Rewrite a 128 x 128 tile of raw bf16 rows in place as fp16 rows scaled by fac(r),
+// rows from nvalid on as zeros; all 256 threads, thread t at chunk t % 16 of rows
+// t / 16 + 16 i: the eight loads are issued before any conversion
+template <typename F>
+__device__ __forceinline__ void scale_rows_f16(uint8_t *tile, int tid, int nvalid, F fac)
+{
+    uint4 x[8];
+    float f[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int r = (tid >> 4) + 16 * i;
+        x[i] = *reinterpret_cast<const uint4 *>(tile + t128(r, tid & 15));
+        f[i] = fac(r);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int r = (tid >> 4) + 16 * i;
+        const float m = f[i];
+        *reinterpret_cast<uint4 *>(tile + t128(r, tid & 15)) =
+            r < nvalid
+                ? make_uint4(pack_h2(__uint_as_float(x[i].x << 16) * m, __uint_as_float(x[i].x & 0xffff0000u) * m),
+                             pack_h2(__uint_as_float(x[i].y << 16) * m, __uint_as_float(x[i].y & 0xffff0000u) * m),
+                             pack_h2(__uint_as_float(x[i].z << 16) * m, __uint_as_float(x[i].z & 0xffff0000u) * m),
+                             pack_h2(__uint_as_float(x[i].w << 16) * m, __uint_as_float(x[i].w & 0xffff0000u) * m))
+                : make_uint4(0, 0, 0, 0);
+    }
+}
+
 __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_w,
@@ -172,26 +200,21 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
         tc::commit(bar_mma);
     }
     // meanwhile: 1/|k| of the valid rows ("L2 Normalization") and the decay factors ...
-    if (tid < 128) {
-        rkv[tid] = tid < n ? row_inv_norm(smem + OFF_K, tid, eps) : 0.f;
-        if (tid < n) {  // for inspection through the stage interface
-            gcum_out[(size_t)h * T + t0 + tid] = gam[tid];
-            betaf_out[(size_t)h * T + t0 + tid] = bet[tid];
-            if (h % (Nv / Nqk) == 0) rk_out[(size_t)hq * T + t0 + tid] = rkv[tid];
-        }
+    {
+        const int r = tid >> 1;  // two lanes per row
+        const float x = row_inv_norm_pair(smem + OFF_K, r, tid & 1, eps);
+        if ((tid & 1) == 0) rkv[r] = r < n ? x : 0.f;
     }
-    __syncthreads();
-    if (tid < 128) kfe[tid] = rkv[tid] * __expf(gam[tid | 15] - gam[tid]);
+    if (tid < n) {  // for inspection through the stage interface
+        gcum_out[(size_t)h * T + t0 + tid] = gam[tid];
+        betaf_out[(size_t)h * T + t0 + tid] = bet[tid];
+    }
     // ... and diag(beta) v in fp16, in place
-    for (int e = tid; e < 128 * 16; e += kIntraThreads) {
-        const int r = e >> 4, cc = e & 15;
-        uint4 *p = reinterpret_cast<uint4 *>(smem + OFF_V + t128(r, cc));
-        const float f = bet[r];
-        const uint4 x = *p;
-        *p = make_uint4(pack_h2(__uint_as_float(x.x << 16) * f, __uint_as_float(x.x & 0xffff0000u) * f),
-                        pack_h2(__uint_as_float(x.y << 16) * f, __uint_as_float(x.y & 0xffff0000u) * f),
-                        pack_h2(__uint_as_float(x.z << 16) * f, __uint_as_float(x.z & 0xffff0000u) * f),
-                        pack_h2(__uint_as_float(x.w << 16) * f, __uint_as_float(x.w & 0xffff0000u) * f));
+    scale_rows_f16(smem + OFF_V, tid, L, [&](int r) { return bet[r]; });
+    __syncthreads();
+    if (tid < 128) {
+        kfe[tid] = rkv[tid] * __expf(gam[tid | 15] - gam[tid]);
+        if (tid < n && h % (Nv / Nqk) == 0) rk_out[(size_t)hq * T + t0 + tid] = rkv[tid];
     }
     wait_bar(bar_mma, mma_phase);
     mma_phase ^= 1;
@@ -215,34 +238,31 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
             float a[32];
             tc::tmem_ld32(t_row + j0, a);
             if (j0 == quarter * 32) {
-                // The warp's diagonal chunk (warp-uniform): every lane takes its 32 values element by
-                // element.  Lanes 0-15 have their diagonal block at columns j0..j0+15, lanes 16-31 at
-                // j0+16..; the block left of it (lanes 16-31, columns j0..j0+15) goes to the fp16 tile.
-                float v[32];
-#pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int j = j0 + jj;
-                    v[jj] = j < row ? fr * rkv[j] * __expf(fminf(gi - gam[j], 0.f)) * a[jj] : 0.f;
-                }
+                // The warp's diagonal chunk (warp-uniform).  Lanes 0-15 have their diagonal block at
+                // columns j0..j0+15 and nothing below the diagonal right of it; lanes 16-31 have it at
+                // j0+16.. and the block left of it at j0..j0+15.  The diagonal block takes the decay
+                // element by element into the fp32 scratch; the left block takes the block factor into
+                // the fp16 tile, where the diagonal blocks are written later as T_ii.
                 const bool hi = lane >= 16;
                 float *drow = dsc + (rb >> 4) * 256 + (row - rb) * 16;
                 const int sw = (row - rb) >> 1;  // bank swizzle of the fp32 diagonal blocks
 #pragma unroll
-                for (int jj = 0; jj < 16; ++jj) drow[jj ^ sw] = hi ? v[16 + jj] : v[jj];
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int j = rb + jj;
+                    const float x = hi ? a[16 + jj] : a[jj];
+                    drow[jj ^ sw] = j < row ? fr * rkv[j] * __expf(fminf(gi - gam[j], 0.f)) * x : 0.f;
+                }
+                const float eb = hi ? fr * __expf(gi - gam[j0 + 15]) : 0.f;
 #pragma unroll
-                for (int q16 = 0; q16 < 2; ++q16) {
-                    const bool left = q16 == 0 && hi;
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    uint32_t w4[4];
 #pragma unroll
-                    for (int q8 = 0; q8 < 2; ++q8) {
-                        uint32_t w4[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int jj = q16 * 16 + q8 * 8 + 2 * e;
-                            w4[e] = left ? pack_h2(v[jj], v[jj + 1]) : 0u;
-                        }
-                        *reinterpret_cast<uint4 *>(smem + OFF_A + t128(row, (j0 >> 3) + 2 * q16 + q8)) =
-                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    for (int e = 0; e < 4; ++e) {
+                        const int jj = q8 * 8 + 2 * e, j = j0 + jj;
+                        w4[e] = (q8 < 2 && hi) ? pack_h2(eb * kfe[j] * a[jj], eb * kfe[j + 1] * a[jj + 1]) : 0u;
                     }
+                    *reinterpret_cast<uint4 *>(smem + OFF_A + t128(row, (j0 >> 3) + q8)) =
+                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
                 continue;
             }
@@ -265,16 +285,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
             }
         }
         // diag(beta e^gamma rk) k in fp16, in place (the k k^T product is complete)
-        for (int e = tid; e < 128 * 16; e += kIntraThreads) {
-            const int r = e >> 4, cc = e & 15;
-            uint4 *p = reinterpret_cast<uint4 *>(smem + OFF_K + t128(r, cc));
-            const float f = bet[r] * __expf(gam[r]) * rkv[r];
-            const uint4 x = *p;
-            *p = make_uint4(pack_h2(__uint_as_float(x.x << 16) * f, __uint_as_float(x.x & 0xffff0000u) * f),
-                            pack_h2(__uint_as_float(x.y << 16) * f, __uint_as_float(x.y & 0xffff0000u) * f),
-                            pack_h2(__uint_as_float(x.z << 16) * f, __uint_as_float(x.z & 0xffff0000u) * f),
-                            pack_h2(__uint_as_float(x.w << 16) * f, __uint_as_float(x.w & 0xffff0000u) * f));
-        }
+        scale_rows_f16(smem + OFF_K, tid, L, [&](int r) { return bet[r] * __expf(gam[r]) * rkv[r]; });
     }
     __syncthreads();
 
@@ -399,20 +410,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     if (ok) wait_bar(bar_ld, 1);
     if (ok) {
         const float gl = gam[127];
-        for (int e = tid; e < 128 * 16; e += kIntraThreads) {
-            const int r = e >> 4, cc = e & 15;
-            uint4 *p = reinterpret_cast<uint4 *>(smem + OFF_K + t128(r, cc));
-            if (r >= n) {
-                *p = make_uint4(0, 0, 0, 0);
-                continue;
-            }
-            const float f = rkv[r] * __expf(gl - gam[r]);
-            const uint4 x = *p;
-            *p = make_uint4(pack_h2(__uint_as_float(x.x << 16) * f, __uint_as_float(x.x & 0xffff0000u) * f),
-                            pack_h2(__uint_as_float(x.y << 16) * f, __uint_as_float(x.y & 0xffff0000u) * f),
-                            pack_h2(__uint_as_float(x.z << 16) * f, __uint_as_float(x.z & 0xffff0000u) * f),
-                            pack_h2(__uint_as_float(x.w << 16) * f, __uint_as_float(x.w & 0xffff0000u) * f));
-        }
+        scale_rows_f16(smem + OFF_K, tid, n, [&](int r) { return rkv[r] * __expf(gl - gam[r]); });
     }
     sync_operands();
     // Mk = k_gexp^T W: A = k_gexp read MN-major (Dk contiguous), B = W MN-major; TMEM columns [0, 128)
@@ -454,7 +452,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
         tc::mbar_wait_bounded(bar_ld, 0);
         tc::mbar_wait_bounded(bar_ld, 1);
     }
-    if (tid == 0) tma::wait_all();  // the stores have read shared memory and completed
+    if (tid == 0) tma::wait_read_all();  // the stores have read shared memory (the grid's end publishes them)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();

@@ -147,13 +147,20 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         tc::commit(bar_mma);
     }
     // while it runs: scale/|q| and 1/|k| of the valid rows ("L2 Normalization") and the decay factors
-    if (tid < 128) {
-        rqv[tid] = tid < n ? scale * row_inv_norm(smem + OO_Q, tid, eps) : 0.f;
-        rkv[tid] = tid < n ? row_inv_norm(smem + OO_K, tid, eps) : 0.f;
-        if (tid < n && h % (Nv / Nqk) == 0) rq_out[(size_t)hq * T + t0 + tid] = rqv[tid];  // for inspection
+    {
+        const int r = tid >> 1;  // two lanes per row
+        const float xq = row_inv_norm_pair(smem + OO_Q, r, tid & 1, eps);
+        const float xk = row_inv_norm_pair(smem + OO_K, r, tid & 1, eps);
+        if ((tid & 1) == 0) {
+            rqv[r] = r < n ? scale * xq : 0.f;
+            rkv[r] = r < n ? xk : 0.f;
+        }
     }
     __syncthreads();
-    if (tid < 128) kfe[tid] = rkv[tid] * __expf(gam[tid | 15] - gam[tid]);
+    if (tid < 128) {
+        kfe[tid] = rkv[tid] * __expf(gam[tid | 15] - gam[tid]);
+        if (tid < n && h % (Nv / Nqk) == 0) rq_out[(size_t)hq * T + t0 + tid] = rqv[tid];  // for inspection
+    }
     if (ok) wait_bar(bar_mma, 0);
 
     if (ok) {
@@ -170,28 +177,48 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
             }
             float a[32];
             tc::tmem_ld32(t_row + j0, a);
-            const bool diag = j0 == rlo;  // warp-uniform
+            if (j0 == rlo) {
+                // The warp's diagonal chunk (warp-uniform).  Lanes 0-15 have their diagonal block at
+                // columns j0..j0+15 and zeros right of it; lanes 16-31 have it at j0+16.. and the block
+                // left of it at j0..j0+15.  The diagonal block takes the decay element by element, the
+                // left block the block factor.
+                const bool hi = lane >= 16;
+                const int rb = row & ~15;
+                float pd[16];
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int j = rb + jj;
+                    const float x = hi ? a[16 + jj] : a[jj];
+                    pd[jj] = j <= row ? fr * rkv[j] * __expf(fminf(gi - gam[j], 0.f)) * x : 0.f;
+                }
+                const float eb = hi ? fr * __expf(gi - gam[j0 + 15]) : 0.f;
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int jj = q8 * 8 + 2 * e, j = j0 + jj, d = jj & 15;
+                        const uint32_t left = pack_h2(eb * kfe[j] * a[jj], eb * kfe[j + 1] * a[jj + 1]);
+                        const uint32_t dg = pack_h2(pd[d], pd[d + 1]);
+                        w4[e] = q8 < 2 ? (hi ? left : dg) : (hi ? dg : 0u);
+                    }
+                    *reinterpret_cast<uint4 *>(smem + OO_K + t128(row, (j0 >> 3) + q8)) =
+                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+                continue;
+            }
+            // a chunk left of the warp's rows: the decay factored per 16-column block
 #pragma unroll
             for (int q16 = 0; q16 < 2; ++q16) {
                 const int jb = j0 + q16 * 16;
-                const float eb = diag ? 0.f : fr * __expf(gi - gam[jb + 15]);
+                const float eb = fr * __expf(gi - gam[jb + 15]);
 #pragma unroll
                 for (int q8 = 0; q8 < 2; ++q8) {
                     uint32_t w4[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        float p[2];
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int jj = q16 * 16 + q8 * 8 + 2 * e + u, j = j0 + jj;
-                            float f;
-                            if (diag)
-                                f = j <= row ? fr * rkv[j] * __expf(fminf(gi - gam[j], 0.f)) : 0.f;
-                            else
-                                f = eb * kfe[j];
-                            p[u] = f * a[jj];
-                        }
-                        w4[e] = pack_h2(p[0], p[1]);
+                        const int jj = q16 * 16 + q8 * 8 + 2 * e, j = j0 + jj;
+                        w4[e] = pack_h2(eb * kfe[j] * a[jj], eb * kfe[j + 1] * a[jj + 1]);
                     }
                     *reinterpret_cast<uint4 *>(smem + OO_K + t128(row, (jb >> 3) + q8)) =
                         make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -297,7 +324,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         tc::mbar_wait_bounded(bar_d, 0);
         tc::mbar_wait_bounded(bar_ld, (uint32_t)((ld_issued - 1) & 1));
     }
-    if (tid == 0) tma::wait_all();
+    if (tid == 0) tma::wait_read_all();  // the stores have read shared memory (the grid's end publishes them)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();

@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
     if (producer && lane == 0) {
         for (int st = 0; st < 2; ++st)
             if (fills[st] > 0) tc::mbar_wait_bounded(bar_full + 8 * st, (uint32_t)((fills[st] - 1) & 1));
-        tma::wait_all();
+        tma::wait_read_all();  // the stores have read shared memory (the grid's end publishes them)
     }
     if (issuer && lane == 0 && !ok && issued) {  // a commit covers every MMA issued before it
         tc::commit(bar_d);
