@@ -216,6 +216,28 @@ __device__ __forceinline__ void chunk_gamma(const float *__restrict__ g, int Nv,
     __syncthreads();
 }
 
+// Largest gate span gamma_first - gamma_last of a 16-row block for which a row's
+// decay inside the block is taken as e^{gamma_i - gamma_last} e^{gamma_last - gamma_j}:
+// the first factor stays below e^64 and the second above e^-64, both normal fp32.
+// Wider spans take e^{gamma_i - gamma_j} element by element.
+constexpr float kSpanMax = 64.f;
+
+// d[0..N) = s[0..N) from shared memory in 16-byte loads (s 16-byte aligned).  Loading
+// a row's per-column factors into registers ahead of the row's stores keeps the
+// loads from being ordered after stores the compiler cannot tell apart from them.
+template <int N>
+__device__ __forceinline__ void lds_vec(float (&d)[N], const float *s)
+{
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+        const float4 x = reinterpret_cast<const float4 *>(s)[i];
+        d[4 * i] = x.x;
+        d[4 * i + 1] = x.y;
+        d[4 * i + 2] = x.z;
+        d[4 * i + 3] = x.w;
+    }
+}
+
 // 1 / sqrt(|x_r|^2 + eps) for row r of a 128 x 128 16-bit tile of raw bf16 rows
 // stored as two 64-column halves of 128-byte rows with the 128-byte swizzle
 // ("L2 Normalization", eps inside the square root).  Two adjacent lanes share a

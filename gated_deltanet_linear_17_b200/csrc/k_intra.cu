@@ -14,7 +14,8 @@
 //   1. k k^T     -- tcgen05.mma M=128, N=128, K=128, bf16 (exact inputs); the L2
 //                   norms enter as the fp32 factors rk.
 //   2. Ap from TMEM in fp16 (the diagonal 16x16 blocks in fp32); the decay is
-//      factored per 16-column block as in the output kernel.
+//      factored per 16-column block as in the output kernel, the diagonal
+//      blocks included unless their gate span exceeds kSpanMax.
 //   3. T_ii by forward substitution (fp32), then the three merge levels with
 //      mma.sync on fp16 operands, in place over Ap.
 //   4. [W | U] = T [diag(beta e^gamma rk) k | diag(beta) v] -- one tcgen05.mma
@@ -221,8 +222,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
 
     // ---- (2) Ap = -strict_tril(diag(beta rk) (k k^T) diag(rk) (.) Gamma): this thread's row and 64 columns.
     // Blocks left of the row's diagonal 16-block go to the A tile in fp16; the diagonal block goes to the
-    // fp32 scratch (block b at OFF_X + 1024 b, element (r, c) at r * 16 + (c ^ (r >> 1))); blocks right
-    // of it are zero.
+    // fp32 scratch (block b at OFF_X + 1024 b, row r at 64 r bytes, its 16-byte group q at position
+    // q ^ ((r >> 1) & 3)); blocks right of it are zero.
     float *dsc = reinterpret_cast<float *>(smem + OFF_X);
     if (ok) {
         const float gi = gam[row], fr = -bet[row] * rkv[row];
@@ -240,26 +241,42 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
             if (j0 == quarter * 32) {
                 // The warp's diagonal chunk (warp-uniform).  Lanes 0-15 have their diagonal block at
                 // columns j0..j0+15 and nothing below the diagonal right of it; lanes 16-31 have it at
-                // j0+16.. and the block left of it at j0..j0+15.  The diagonal block takes the decay
-                // element by element into the fp32 scratch; the left block takes the block factor into
-                // the fp16 tile, where the diagonal blocks are written later as T_ii.
+                // j0+16.. and the block left of it at j0..j0+15.  The diagonal block goes to the fp32
+                // scratch, its decay element by element only when its gate span is too wide for the
+                // block factor; the left block goes to the fp16 tile, where the diagonal blocks are
+                // written later as T_ii.
                 const bool hi = lane >= 16;
-                float *drow = dsc + (rb >> 4) * 256 + (row - rb) * 16;
-                const int sw = (row - rb) >> 1;  // bank swizzle of the fp32 diagonal blocks
-#pragma unroll
-                for (int jj = 0; jj < 16; ++jj) {
-                    const int j = rb + jj;
-                    const float x = hi ? a[16 + jj] : a[jj];
-                    drow[jj ^ sw] = j < row ? fr * rkv[j] * __expf(fminf(gi - gam[j], 0.f)) * x : 0.f;
-                }
+                float kf[16], dv[16];
+                lds_vec(kf, kfe + j0);  // the left block's column factors (lanes 16-31)
                 const float eb = hi ? fr * __expf(gi - gam[j0 + 15]) : 0.f;
+                const float gl = gam[rb + 15];
+                if (gam[rb] - gl <= kSpanMax) {  // half-warp-uniform
+                    float kd[16];
+                    lds_vec(kd, kfe + rb);
+                    const float ed = fr * __expf(gi - gl);
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) dv[jj] = rb + jj < row ? ed * kd[jj] * (hi ? a[16 + jj] : a[jj]) : 0.f;
+                } else {
+                    float rkj[16], gmj[16];
+                    lds_vec(rkj, rkv + rb);
+                    lds_vec(gmj, gam + rb);
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj)
+                        dv[jj] = rb + jj < row ? fr * rkj[jj] * __expf(fminf(gi - gmj[jj], 0.f)) * (hi ? a[16 + jj] : a[jj])
+                                               : 0.f;
+                }
+                // row r of block b at OFF_X + 1024 b + 64 r, 16-byte group q at position q ^ ((r >> 1) & 3)
+                float4 *drow = reinterpret_cast<float4 *>(dsc + (rb >> 4) * 256 + (row - rb) * 16);
+                const int sw = ((row - rb) >> 1) & 3;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) drow[q ^ sw] = make_float4(dv[4 * q], dv[4 * q + 1], dv[4 * q + 2], dv[4 * q + 3]);
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8) {
                     uint32_t w4[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int jj = q8 * 8 + 2 * e, j = j0 + jj;
-                        w4[e] = (q8 < 2 && hi) ? pack_h2(eb * kfe[j] * a[jj], eb * kfe[j + 1] * a[jj + 1]) : 0u;
+                        const int jj = (q8 & 1) * 8 + 2 * e;
+                        w4[e] = (q8 < 2 && hi) ? pack_h2(eb * kf[jj] * a[jj], eb * kf[jj + 1] * a[jj + 1]) : 0u;
                     }
                     *reinterpret_cast<uint4 *>(smem + OFF_A + t128(row, (j0 >> 3) + q8)) =
                         make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -267,17 +284,20 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
                 continue;
             }
             // a chunk left of the warp's rows: the decay factored per 16-column block
+            float kf[32];
+            lds_vec(kf, kfe + j0);
+            const float eb2[2] = {fr * __expf(gi - gam[j0 + 15]), fr * __expf(gi - gam[j0 + 31])};
 #pragma unroll
             for (int q16 = 0; q16 < 2; ++q16) {
                 const int jb = j0 + q16 * 16;
-                const float eb = fr * __expf(gi - gam[jb + 15]);
+                const float eb = eb2[q16];
 #pragma unroll
                 for (int q8 = 0; q8 < 2; ++q8) {
                     uint32_t w4[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int jj = q16 * 16 + q8 * 8 + 2 * e, j = j0 + jj;
-                        w4[e] = pack_h2(eb * kfe[j] * a[jj], eb * kfe[j + 1] * a[jj + 1]);
+                        const int jj = q16 * 16 + q8 * 8 + 2 * e;
+                        w4[e] = pack_h2(eb * kf[jj] * a[jj], eb * kf[jj + 1] * a[jj + 1]);
                     }
                     *reinterpret_cast<uint4 *>(smem + OFF_A + t128(row, (jb >> 3) + q8)) =
                         make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -293,14 +313,28 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     if (ok && lane < 16) {
         const float *ds = dsc + wid * 256;
         const int cidx = lane;
-        float tcol[16];
+        float tcol[16];  // T_ii = I + Ap_ii T_ii, row by row; tcol[j] = 0 above the diagonal
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            float val = (i == cidx) ? 1.f : 0.f;
+            float nr[16];
 #pragma unroll
-            for (int j = 0; j < i; ++j)
-                if (j >= cidx) val += ds[i * 16 + (j ^ (i >> 1))] * tcol[j];
-            tcol[i] = (i < cidx) ? 0.f : val;
+            for (int q = 0; q < 4; ++q)
+                if (4 * q < i) {
+                    const float4 x = reinterpret_cast<const float4 *>(ds + i * 16)[q ^ ((i >> 1) & 3)];
+                    nr[4 * q] = x.x;
+                    nr[4 * q + 1] = x.y;
+                    nr[4 * q + 2] = x.z;
+                    nr[4 * q + 3] = x.w;
+                }
+            float s0 = i == cidx ? 1.f : 0.f, s1 = 0.f;
+#pragma unroll
+            for (int j = 0; j < i; ++j) {
+                if (j & 1)
+                    s1 = fmaf(nr[j], tcol[j], s1);
+                else
+                    s0 = fmaf(nr[j], tcol[j], s0);
+            }
+            tcol[i] = i < cidx ? 0.f : s0 + s1;
         }
         const int col = wid * 16 + cidx;
 #pragma unroll

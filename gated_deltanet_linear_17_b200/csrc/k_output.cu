@@ -19,10 +19,12 @@
 //      tile.  Since the gates are <= 0, gamma does not increase along the
 //      chunk.  For a 16-column block below the diagonal the decay is factored
 //      at the block's last column je as exp(gamma_i - gamma_je) exp(gamma_je -
-//      gamma_j), both factors <= 1, so a row needs one exponential per block;
-//      only the 32-column chunk on a warp's diagonal takes one per element.
-//      Chunks above all of a warp's rows are written as zeros without reading
-//      TMEM.
+//      gamma_j), both factors <= 1, so a row needs one exponential per block.
+//      A row's own diagonal block takes the same split at its last row, where
+//      the first factor is >= 1; it stays below e^kSpanMax unless the block's
+//      gate span is wider, and then that block takes one exponential per
+//      element.  Chunks above all of a warp's rows are written as zeros without
+//      reading TMEM.
 //   3. Z = P W  -- M=128, N=128, K=128, fp16 (W read MN-major); then
 //      Qw = diag(rq e^gamma) q - Z in fp16, in place of q.
 //   4. O = Qw S_c + P U for Dv columns 0..63, then 64..127 -- 16 tcgen05.mma
@@ -180,25 +182,36 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
             if (j0 == rlo) {
                 // The warp's diagonal chunk (warp-uniform).  Lanes 0-15 have their diagonal block at
                 // columns j0..j0+15 and zeros right of it; lanes 16-31 have it at j0+16.. and the block
-                // left of it at j0..j0+15.  The diagonal block takes the decay element by element, the
-                // left block the block factor.
+                // left of it at j0..j0+15.  Both blocks take the block factor, the diagonal one element
+                // by element when its gate span is too wide for it.
                 const bool hi = lane >= 16;
                 const int rb = row & ~15;
-                float pd[16];
-#pragma unroll
-                for (int jj = 0; jj < 16; ++jj) {
-                    const int j = rb + jj;
-                    const float x = hi ? a[16 + jj] : a[jj];
-                    pd[jj] = j <= row ? fr * rkv[j] * __expf(fminf(gi - gam[j], 0.f)) * x : 0.f;
-                }
+                float kf[16], pd[16];
+                lds_vec(kf, kfe + j0);  // the left block's column factors (lanes 16-31)
                 const float eb = hi ? fr * __expf(gi - gam[j0 + 15]) : 0.f;
+                const float gl = gam[rb + 15];
+                if (gam[rb] - gl <= kSpanMax) {  // half-warp-uniform
+                    float kd[16];
+                    lds_vec(kd, kfe + rb);
+                    const float ed = fr * __expf(gi - gl);
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) pd[jj] = rb + jj <= row ? ed * kd[jj] * (hi ? a[16 + jj] : a[jj]) : 0.f;
+                } else {
+                    float rkj[16], gmj[16];
+                    lds_vec(rkj, rkv + rb);
+                    lds_vec(gmj, gam + rb);
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj)
+                        pd[jj] = rb + jj <= row ? fr * rkj[jj] * __expf(fminf(gi - gmj[jj], 0.f)) * (hi ? a[16 + jj] : a[jj])
+                                                : 0.f;
+                }
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8) {
                     uint32_t w4[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int jj = q8 * 8 + 2 * e, j = j0 + jj, d = jj & 15;
-                        const uint32_t left = pack_h2(eb * kfe[j] * a[jj], eb * kfe[j + 1] * a[jj + 1]);
+                        const int jj = q8 * 8 + 2 * e, d = jj & 15;
+                        const uint32_t left = pack_h2(eb * kf[d] * a[jj], eb * kf[d + 1] * a[jj + 1]);
                         const uint32_t dg = pack_h2(pd[d], pd[d + 1]);
                         w4[e] = q8 < 2 ? (hi ? left : dg) : (hi ? dg : 0u);
                     }
@@ -208,17 +221,20 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
                 continue;
             }
             // a chunk left of the warp's rows: the decay factored per 16-column block
+            float kf[32];
+            lds_vec(kf, kfe + j0);
+            const float eb2[2] = {fr * __expf(gi - gam[j0 + 15]), fr * __expf(gi - gam[j0 + 31])};
 #pragma unroll
             for (int q16 = 0; q16 < 2; ++q16) {
                 const int jb = j0 + q16 * 16;
-                const float eb = fr * __expf(gi - gam[jb + 15]);
+                const float eb = eb2[q16];
 #pragma unroll
                 for (int q8 = 0; q8 < 2; ++q8) {
                     uint32_t w4[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int jj = q16 * 16 + q8 * 8 + 2 * e, j = j0 + jj;
-                        w4[e] = pack_h2(eb * kfe[j] * a[jj], eb * kfe[j + 1] * a[jj + 1]);
+                        const int jj = q16 * 16 + q8 * 8 + 2 * e;
+                        w4[e] = pack_h2(eb * kf[jj] * a[jj], eb * kf[jj + 1] * a[jj + 1]);
                     }
                     *reinterpret_cast<uint4 *>(smem + OO_K + t128(row, (jb >> 3) + q8)) =
                         make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -245,10 +261,13 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
             float z[32];
             tc::tmem_ld32(t_row + 128 + j0, z);
+            uint4 qv[4];
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) qv[c4] = *reinterpret_cast<const uint4 *>(smem + OO_Q + t128(row, (j0 >> 3) + c4));
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {
                 uint4 *p = reinterpret_cast<uint4 *>(smem + OO_Q + t128(row, (j0 >> 3) + c4));
-                const uint4 w = *p;
+                const uint4 w = qv[c4];
                 const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
                 uint32_t o4[4];
 #pragma unroll

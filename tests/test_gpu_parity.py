@@ -176,9 +176,12 @@ def test_beta_zero_gives_exact_zeros():
     assert torch.count_nonzero(out) == 0 and torch.count_nonzero(fin) == 0
 
 
-@pytest.mark.parametrize("gate", [("uniform_neg", 30.0, 5.0), ("zero",)], ids=["strong_decay", "no_decay"])
+@pytest.mark.parametrize("gate", [("uniform_neg", 30.0, 5.0), ("uniform_neg", 1.5, 3.5), ("zero",)],
+                         ids=["strong_decay", "span_near_64", "no_decay"])
 def test_gate_extremes(gate):
-    """Gates far below zero (e^gamma underflows inside a chunk) and gates of exactly zero."""
+    """Gates far below zero (e^gamma underflows inside a chunk), gates whose span over a
+    16-row block straddles the kernels' switch to element-by-element decays, and gates
+    of exactly zero."""
     inp = inputs.make([300, 17, 129], Nqk=2, Nv=4, g=gate, state=("normal", 0.02, 3, "perm"), seed=14)
     out, fin = _gpu(inp)
     assert torch.isfinite(out.float()).all() and torch.isfinite(fin).all()
