@@ -15,8 +15,8 @@
 //   1. q k^T     -- tcgen05.mma M=128, N=128, K=128 on the raw bf16 rows (exact
 //                   inputs), both K-major; fp32 accumulator in TMEM.
 //   2. P = rq_i rk_j exp(gamma_i - gamma_j) (q k^T)_ij for j <= i, else 0, read
-//      from TMEM and stored in fp16 as a K-major A tile over the now unused k
-//      tile.  Since the gates are <= 0, gamma does not increase along the
+//      from TMEM and written back to TMEM in fp16 pairs, where it is the A
+//      operand of both products with P.  Since the gates are <= 0, gamma does not increase along the
 //      chunk.  For a 16-column block below the diagonal the decay is factored
 //      at the block's last column je as exp(gamma_i - gamma_je) exp(gamma_je -
 //      gamma_j), both factors <= 1, so a row needs one exponential per block.
@@ -25,11 +25,11 @@
 //      gate span is wider, and then that block takes one exponential per
 //      element.  Chunks above all of a warp's rows are written as zeros without
 //      reading TMEM.
-//   3. Z = P W  -- M=128, N=128, K=128, fp16 (W read MN-major); then
-//      Qw = diag(rq e^gamma) q - Z in fp16, in place of q.
-//   4. O = Qw S_c + P U for Dv columns 0..63, then 64..127 -- 16 tcgen05.mma
-//      each (N = 64), both halves kept in TMEM; S_c and U arrive one column half
-//      at a time by TMA in the buffer W used.
+//   3. S_c starts loading into the k tile, free once q k^T is done.  Z = P W
+//      -- M=128, N=128, K=128, fp16 (W read MN-major); then U starts loading
+//      into W's tile, and Qw = diag(rq e^gamma) q - Z in fp16, in place of q.
+//   4. O = Qw S_c + P U -- 16 tcgen05.mma (N = 128); the eight on U are issued
+//      once it has landed, while the eight on S_c run.
 //   5. O in bf16 is staged over the consumed Qw tile and leaves by TMA for a
 //      full chunk; a short chunk's rows are stored by the threads, so rows of
 //      the next sequence are never written.
@@ -48,11 +48,10 @@ constexpr int kOutThreads = 256;
 // shared memory, relative to a 1024-byte aligned base; 128 x 128 16-bit tiles are
 // two 64-column halves of 128-byte rows with the 128-byte swizzle
 constexpr int OO_Q = 0;        // q (bf16) -> Qw (fp16), K-major over Dk -> O (bf16) for the store
-constexpr int OO_K = 32768;    // k (bf16), K-major over Dk -> P (fp16), K-major over j
-constexpr int OO_X = 65536;    // W (fp16) [L][Dk] (MN-major B of P W) -> S_c[:, half] [Dk][64] and,
-                               // 16 KiB on, U[:, half] [L][64] (fp16, MN-major)
+constexpr int OO_K = 32768;    // k (bf16), K-major over Dk -> S_c (fp16) [Dk][Dv], MN-major B of Qw S_c
+constexpr int OO_X = 65536;    // W (fp16) [L][Dk], MN-major B of P W -> U (fp16) [L][Dv], MN-major B of P U
 constexpr int OO_VEC = 98304;  // gam, rqv, rkv, kfe (rk_j e^{gamma_je - gamma_j})
-constexpr int OO_BAR = OO_VEC + 4 * 512;
+constexpr int OO_BAR = OO_VEC + 4 * 512;  // mbarriers, TMEM slot, scan sums (64 bytes)
 constexpr int kOutSmem = OO_BAR + 64 + 1024;
 
 // byte offset of 16-byte chunk c (0..15) of row r in a 128 x 128 tile
@@ -80,12 +79,15 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     float *rqv = gam + 128, *rkv = gam + 256, *kfe = gam + 384;
     const uint32_t bar_ld = sbase + OO_BAR, bar_mma = sbase + OO_BAR + 8, bar_d = sbase + OO_BAR + 16;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + OO_BAR + 24);
+    const uint32_t bar_s = sbase + OO_BAR + 48, bar_u = sbase + OO_BAR + 56;  // S_c and U loads
     const int trow = (c * Nv + h) * L;  // first row of the chunk's tiles in the workspace
 
     if (tid == 0) {
         tc::mbar_init(bar_ld, 1);
         tc::mbar_init(bar_mma, 1);
         tc::mbar_init(bar_d, 1);
+        tc::mbar_init(bar_s, 1);
+        tc::mbar_init(bar_u, 1);
         tc::mbar_init_fence();
     }
     if (wid == 0) tc::tmem_alloc(smem_addr(tslot), 256);
@@ -101,16 +103,14 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     }
     // chunk-local cumulative gate while the rows load
     chunk_gamma(g, Nv, h, t0, n, gam, reinterpret_cast<float *>(smem + OO_BAR + 32));
-    // S_c and U columns [64 hf, 64 hf + 64) into the MN-major buffers (thread 0), on bar_ld
-    int ld_issued = 1;  // load phases issued on bar_ld (thread 0)
-    auto load_su = [&](int hf) {
-        ++ld_issued;
-        tma::expect_tx(bar_ld, 32768);
-        tma::load_2d(sbase + OO_X, &tm_sc, hf * 64, trow, bar_ld);
-        tma::load_2d(sbase + OO_X + 16384, &tm_u, hf * 64, trow, bar_ld);
+    // S_c, then U, as MN-major [128][128] tiles (two 64-column halves), each on its own barrier (thread 0)
+    bool s_issued = false, u_issued = false;
+    auto load_tile = [&](uint32_t dst, const CUtensorMap *m, uint32_t bar) {
+        tma::expect_tx(bar, 32768);
+        tma::load_2d(dst, m, 0, trow, bar);
+        tma::load_2d(dst + 16384, m, 64, trow, bar);
     };
     bool ok = true;
-    uint32_t ld_phase = 0;
     auto wait_bar = [&](uint32_t bar, uint32_t parity) {  // bounded, outcome shared with the CTA
         bool w_ok = true;
         if (tid == 0) w_ok = tc::mbar_wait_bounded(bar, parity);
@@ -127,8 +127,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     // descriptor of K step kk of a K-major tile with two 64-column K halves
     auto kmaj = [](uint64_t d, int kk) { return d + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4); };
 
-    wait_bar(bar_ld, ld_phase);
-    ld_phase ^= 1;
+    wait_bar(bar_ld, 0);
     if (n < L) {  // q and k rows past the chunk belong to the next sequence (W is zero there)
         for (int e = tid; e < (L - n) * 32; e += kOutThreads) {
             const int r = n + (e >> 5), tl = (e >> 4) & 1, blk = (e >> 3) & 1, cc = e & 7;
@@ -137,7 +136,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         }
     }
     sync_operands();
-    const uint32_t tmem = *tslot;  // columns [0, 128): q k^T, then O; [128, 256): Z = P W
+    const uint32_t tmem = *tslot;  // columns [0, 128): q k^T, then Z = P W, then O; [128, 192): P (fp16 pairs)
     const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
 
     // ---- (1) q k^T
@@ -166,15 +165,17 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     if (ok) wait_bar(bar_mma, 0);
 
     if (ok) {
-        // ---- (2) P, this thread's 64 columns of its row (fp16 over the k tile)
+        // ---- (2) P, this thread's 64 columns of its row, in fp16 pairs into TMEM columns [128, 192)
         const float gi = gam[row], fr = rqv[row];
         const int rlo = quarter * 32;  // first row of this warp
 #pragma unroll 1
         for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
+            uint32_t pw[16];  // columns j0 .. j0 + 31 of the row, two to a word
+            const uint32_t t_p = t_row + 128 + (j0 >> 1);
             if (j0 > rlo + 31) {  // above the diagonal for every row of the warp
 #pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8)
-                    *reinterpret_cast<uint4 *>(smem + OO_K + t128(row, (j0 >> 3) + c8)) = make_uint4(0, 0, 0, 0);
+                for (int e = 0; e < 16; ++e) pw[e] = 0u;
+                tc::tmem_st16(t_p, pw);
                 continue;
             }
             float a[32];
@@ -207,17 +208,15 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
                 }
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8) {
-                    uint32_t w4[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int jj = q8 * 8 + 2 * e, d = jj & 15;
                         const uint32_t left = pack_h2(eb * kf[d] * a[jj], eb * kf[d + 1] * a[jj + 1]);
                         const uint32_t dg = pack_h2(pd[d], pd[d + 1]);
-                        w4[e] = q8 < 2 ? (hi ? left : dg) : (hi ? dg : 0u);
+                        pw[q8 * 4 + e] = q8 < 2 ? (hi ? left : dg) : (hi ? dg : 0u);
                     }
-                    *reinterpret_cast<uint4 *>(smem + OO_K + t128(row, (j0 >> 3) + q8)) =
-                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
+                tc::tmem_st16(t_p, pw);
                 continue;
             }
             // a chunk left of the warp's rows: the decay factored per 16-column block
@@ -226,41 +225,42 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
             const float eb2[2] = {fr * __expf(gi - gam[j0 + 15]), fr * __expf(gi - gam[j0 + 31])};
 #pragma unroll
             for (int q16 = 0; q16 < 2; ++q16) {
-                const int jb = j0 + q16 * 16;
                 const float eb = eb2[q16];
 #pragma unroll
-                for (int q8 = 0; q8 < 2; ++q8) {
-                    uint32_t w4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int jj = q16 * 16 + q8 * 8 + 2 * e;
-                        w4[e] = pack_h2(eb * kf[jj] * a[jj], eb * kf[jj + 1] * a[jj + 1]);
-                    }
-                    *reinterpret_cast<uint4 *>(smem + OO_K + t128(row, (jb >> 3) + q8)) =
-                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                for (int e = 0; e < 8; ++e) {
+                    const int jj = q16 * 16 + 2 * e;
+                    pw[q16 * 8 + e] = pack_h2(eb * kf[jj] * a[jj], eb * kf[jj + 1] * a[jj + 1]);
                 }
             }
+            tc::tmem_st16(t_p, pw);
         }
+        tc::tmem_wait_st();
     }
     sync_operands();
 
-    // ---- (3) Z = P W into TMEM columns [128, 256), then Qw = diag(rq e^gamma) q - Z over q
+    // ---- (3) S_c starts loading over the consumed k tile; Z = P W (P from TMEM) into TMEM columns
+    // [0, 128); U then loads over the consumed W; Qw = diag(rq e^gamma) q - Z in fp16, in place of q
+    const uint32_t idesc_n128 = tc::idesc_f16(128, 128, false, false, false, true);
     if (ok && tid == 0) {
-        const uint64_t dp = tc::desc_k128(sbase + OO_K), dw = tc::desc_mn(sbase + OO_X, 16384, 1024, 2);
-        const uint32_t idesc = tc::idesc_f16(128, 128, false, false, false, true);
+        load_tile(sbase + OO_K, &tm_sc, bar_s);
+        s_issued = true;
+        const uint64_t dw = tc::desc_mn(sbase + OO_X, 16384, 1024, 2);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-            tc::mma_f16(tmem + 128, kmaj(dp, kk), dw + (uint64_t)((kk * 2048) >> 4), idesc, kk > 0 ? 1u : 0u);
+            tc::mma_f16_ts(tmem, tmem + 128 + kk * 8, dw + (uint64_t)((kk * 2048) >> 4), idesc_n128, kk > 0 ? 1u : 0u);
         tc::commit(bar_mma);
     }
     if (ok) wait_bar(bar_mma, 1);
-    if (ok && tid == 0) load_su(0);  // W is consumed
+    if (ok && tid == 0) {
+        load_tile(sbase + OO_X, &tm_u, bar_u);
+        u_issued = true;
+    }
     if (ok) {
         const float qf = rqv[row] * __expf(gam[row]);
 #pragma unroll 1
         for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
             float z[32];
-            tc::tmem_ld32(t_row + 128 + j0, z);
+            tc::tmem_ld32(t_row + j0, z);
             uint4 qv[4];
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) qv[c4] = *reinterpret_cast<const uint4 *>(smem + OO_Q + t128(row, (j0 >> 3) + c4));
@@ -278,30 +278,31 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
             }
         }
     }
+    sync_operands();
 
-    // ---- (4) O[:, 64 hf : 64 hf + 64] = Qw S_c + P U into TMEM columns [64 hf, 64 hf + 64)
+    // ---- (4) O = Qw S_c + P U into TMEM columns [0, 128): 8 MMAs on S_c, then 8 on U once it has landed
+    if (ok) wait_bar(bar_s, 0);
     {
-        const uint64_t dq = tc::desc_k128(sbase + OO_Q), dp = tc::desc_k128(sbase + OO_K);
-        const uint64_t ds = tc::desc_mn(sbase + OO_X, 16384, 1024, 2), du = tc::desc_mn(sbase + OO_X + 16384, 16384, 1024, 2);
-        const uint32_t idesc = tc::idesc_f16(128, 64, false, false, false, true);
-#pragma unroll 1
-        for (int hf = 0; hf < 2; ++hf) {
-            if (ok) wait_bar(bar_ld, ld_phase);  // S_c and U of this column half have landed
-            ld_phase ^= 1;
-            sync_operands();
-            if (ok && tid == 0) {
-                const uint32_t dst = tmem + hf * 64;
+        bool w_ok = true;
+        if (ok && tid == 0) {
+            const uint64_t dq = tc::desc_k128(sbase + OO_Q), ds = tc::desc_mn(sbase + OO_K, 16384, 1024, 2);
+            const uint64_t du = tc::desc_mn(sbase + OO_X, 16384, 1024, 2);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                tc::mma_f16(tmem, kmaj(dq, kk), ds + (uint64_t)((kk * 2048) >> 4), idesc_n128, kk > 0 ? 1u : 0u);
+            w_ok = tc::mbar_wait_bounded(bar_u, 0);
+            if (w_ok) {
+                tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_f16(dst, kmaj(dq, kk), ds + (uint64_t)((kk * 2048) >> 4), idesc, kk > 0 ? 1u : 0u);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_f16(dst, kmaj(dp, kk), du + (uint64_t)((kk * 2048) >> 4), idesc, 1u);
-                tc::commit(bar_mma);
+                    tc::mma_f16_ts(tmem, tmem + 128 + kk * 8, du + (uint64_t)((kk * 2048) >> 4), idesc_n128, 1u);
             }
-            if (ok) wait_bar(bar_mma, (uint32_t)hf);  // third and fourth phases of bar_mma
-            if (ok && hf == 0 && tid == 0) load_su(1);  // the buffers are free
+            tc::commit(bar_mma);
+            w_ok = w_ok && tc::mbar_wait_bounded(bar_mma, 0);  // third phase of bar_mma
         }
+        tc::fence_before_sync();
+        ok = __syncthreads_and(w_ok) != 0 && ok;
+        tc::fence_after_sync();
     }
 
     // ---- (5) O to bf16: a full chunk through shared memory (over Qw) and TMA, a short one row by row
@@ -341,7 +342,9 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         // a commit covers every MMA issued before it; then the last load phase issued
         tc::commit(bar_d);
         tc::mbar_wait_bounded(bar_d, 0);
-        tc::mbar_wait_bounded(bar_ld, (uint32_t)((ld_issued - 1) & 1));
+        tc::mbar_wait_bounded(bar_ld, 0);
+        if (s_issued) tc::mbar_wait_bounded(bar_s, 0);
+        if (u_issued) tc::mbar_wait_bounded(bar_u, 0);
     }
     if (tid == 0) tma::wait_read_all();  // the stores have read shared memory (the grid's end publishes them)
     tc::fence_before_sync();

@@ -1,5 +1,6 @@
 // Blackwell (sm_100a) tensor-core helpers: TMEM allocation, tcgen05.mma with
-// shared-memory descriptors, tcgen05.commit to an mbarrier, tcgen05.ld.
+// shared-memory descriptors (A also from TMEM), tcgen05.commit to an mbarrier,
+// tcgen05.ld and tcgen05.st.
 //
 // K-major operand tiles use the 128-byte swizzle: a tile of R rows and 64
 // 16-bit elements (128 bytes) of K is stored row after row, and inside each
@@ -79,6 +80,19 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_
         : "memory");
 }
 
+// the same with A read from tensor memory: row m of A in lane m of a_tmem, its K
+// elements two to a 32-bit column (the lower half holds the even element), so K
+// step kk of 16 elements starts 8 columns further on; A is K-major
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // all previously issued MMAs of this thread arrive on the mbarrier when complete
 __device__ __forceinline__ void commit(uint32_t mbar_addr)
 {
@@ -119,6 +133,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v)
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+
+// 32 lanes x 16 consecutive 32-bit columns from registers: lane i of the warp
+// writes row (lane base + i); tmem_wait_st() before the data is used elsewhere
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *v)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 32 lanes x 16 consecutive fp32 columns: lane i of the warp gets row (lane base + i)
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v)
