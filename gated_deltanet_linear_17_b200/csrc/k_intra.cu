@@ -54,20 +54,28 @@ __device__ __forceinline__ uint32_t t128(int r, int c) { return (uint32_t)((c >>
 __device__ __forceinline__ uint32_t x64(int r, int c) { return tc::sw128c(r, c); }
 
 // One warp: acc (a 16 x 16 fp32 tile, two m16n8 fragments) += A[am0.., ak0 + k] B[bk0 + k, bn0..]
-// for k in [0, K) in steps of 16; A and B are fp16 tiles addressed by the offset
-// functions fa_ (row, chunk) and fb_ (row, chunk).
-template <typename FA, typename FB>
+// for k in [0, 16 steps) in steps of 16 (steps <= KMAX); A and B are fp16 tiles addressed by
+// the offset functions fa_ (row, chunk) and fb_ (row, chunk).  Every fragment load is issued
+// before the first MMA.
+template <int KMAX, typename FA, typename FB>
 __device__ __forceinline__ void warp_mm(float (&acc)[2][4], uint32_t abase, FA fa_, int am0, int ak0, uint32_t bbase,
-                                        FB fb_, int bk0, int bn0, int K, int lane)
+                                        FB fb_, int bk0, int bn0, int steps, int lane)
 {
-    for (int kk = 0; kk < K; kk += 16) {
-        uint32_t a[4], b0, b1, b2, b3;
-        ldsm_x4(abase + fa_(am0 + (lane & 15), ((ak0 + kk) >> 3) + (lane >> 4)), a[0], a[1], a[2], a[3]);
-        ldsm_x4_t(bbase + fb_(bk0 + kk + (lane & 7) + (((lane >> 3) & 1) << 3), (bn0 >> 3) + (lane >> 4)), b0, b1, b2,
-                  b3);
-        mma16816(acc[0], a, b0, b1);
-        mma16816(acc[1], a, b2, b3);
-    }
+    uint32_t a[KMAX][4], b[KMAX][4];
+#pragma unroll
+    for (int s = 0; s < KMAX; ++s)
+        if (s < steps) {
+            const int kk = 16 * s;
+            ldsm_x4(abase + fa_(am0 + (lane & 15), ((ak0 + kk) >> 3) + (lane >> 4)), a[s][0], a[s][1], a[s][2], a[s][3]);
+            ldsm_x4_t(bbase + fb_(bk0 + kk + (lane & 7) + (((lane >> 3) & 1) << 3), (bn0 >> 3) + (lane >> 4)), b[s][0],
+                      b[s][1], b[s][2], b[s][3]);
+        }
+#pragma unroll
+    for (int s = 0; s < KMAX; ++s)
+        if (s < steps) {
+            mma16816(acc[0], a[s], b[s][0], b[s][1]);
+            mma16816(acc[1], a[s], b[s][2], b[s][3]);
+        }
 }
 
 // store a warp's 16 x 16 fp32 tile in fp16 at rows m0.., columns n0.. of a tile with offsets f_(row, chunk)
@@ -355,11 +363,11 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
         if (wid < 4) {
             const int a = 32 * wid, bb = a + 16;
             float acc[2][4] = {};
-            warp_mm(acc, aA, fA, bb, a, aA, fA, a, a, 16, lane);
+            warp_mm<1>(acc, aA, fA, bb, a, aA, fA, a, a, 1, lane);
             warp_store16(acc, pX, fX, 16 * wid, 0, lane);
             __syncwarp();
             float acc2[2][4] = {};
-            warp_mm(acc2, aA, fA, bb, bb, aX, fX, 16 * wid, 0, 16, lane);
+            warp_mm<1>(acc2, aA, fA, bb, bb, aX, fX, 16 * wid, 0, 1, lane);
             warp_store16(acc2, pA, fA, bb, a, lane);
         }
         __syncthreads();
@@ -368,26 +376,30 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
             const int p = wid >> 2, mi = (wid >> 1) & 1, ni = wid & 1;
             const int a = 64 * p, bb = a + 32;
             float acc[2][4] = {};
-            warp_mm(acc, aA, fA, bb + 16 * mi, a + 16 * ni, aA, fA, a + 16 * ni, a + 16 * ni, 32 - 16 * ni, lane);
+            warp_mm<2>(acc, aA, fA, bb + 16 * mi, a + 16 * ni, aA, fA, a + 16 * ni, a + 16 * ni, 2 - ni, lane);
             warp_store16(acc, pX, fX, 32 * p + 16 * mi, 16 * ni, lane);
             __syncthreads();
             float acc2[2][4] = {};
-            warp_mm(acc2, aA, fA, bb + 16 * mi, bb, aX, fX, 32 * p, 16 * ni, 16 * mi + 16, lane);
+            warp_mm<2>(acc2, aA, fA, bb + 16 * mi, bb, aX, fX, 32 * p, 16 * ni, mi + 1, lane);
             warp_store16(acc2, pA, fA, bb + 16 * mi, a + 16 * ni, lane);
         }
         __syncthreads();
-        // 64 -> 128: the 64-blocks (64, 0); warp w takes 16 x 16 tiles w and w + 8
+        // 64 -> 128: the 64-blocks (64, 0).  X = Ap21 T11 takes 4 - ni k-steps for tile (mi, ni), so
+        // warp w takes tiles (w / 2, w % 2) and (w / 2, 3 - w % 2): five steps for every warp
+#pragma unroll
         for (int rep = 0; rep < 2; ++rep) {
-            const int idx = wid + 8 * rep, mi = idx >> 2, ni = idx & 3;
+            const int mi = wid >> 1, ni = rep ? 3 - (wid & 1) : (wid & 1);
             float acc[2][4] = {};
-            warp_mm(acc, aA, fA, 64 + 16 * mi, 16 * ni, aA, fA, 16 * ni, 16 * ni, 64 - 16 * ni, lane);
+            warp_mm<4>(acc, aA, fA, 64 + 16 * mi, 16 * ni, aA, fA, 16 * ni, 16 * ni, 4 - ni, lane);
             warp_store16(acc, pX, fX, 16 * mi, 16 * ni, lane);
         }
         __syncthreads();
+        // T21 = T22 X takes mi + 1 k-steps: warp w takes tiles (w % 2, w / 2) and (3 - w % 2, w / 2)
+#pragma unroll
         for (int rep = 0; rep < 2; ++rep) {
-            const int idx = wid + 8 * rep, mi = idx >> 2, ni = idx & 3;
+            const int ni = wid >> 1, mi = rep ? 3 - (wid & 1) : (wid & 1);
             float acc[2][4] = {};
-            warp_mm(acc, aA, fA, 64 + 16 * mi, 64, aX, fX, 0, 16 * ni, 16 * mi + 16, lane);
+            warp_mm<4>(acc, aA, fA, 64 + 16 * mi, 64, aX, fX, 0, 16 * ni, mi + 1, lane);
             warp_store16(acc, pA, fA, 64 + 16 * mi, 16 * ni, lane);
         }
     }
