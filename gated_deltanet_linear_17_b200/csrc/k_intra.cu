@@ -142,28 +142,30 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     float *gam = reinterpret_cast<float *>(smem + OFF_VEC);
     float *bet = gam + 128, *rkv = gam + 256, *kfe = gam + 384;
     const uint32_t bar_ld = sbase + OFF_BAR, bar_mma = sbase + OFF_BAR + 8, bar_d = sbase + OFF_BAR + 16;
+    const uint32_t bar_v = sbase + OFF_BAR + 48;  // the v rows (k rows on bar_ld)
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 24);
 
     if (tid == 0) {
         tc::mbar_init(bar_ld, 1);
+        tc::mbar_init(bar_v, 1);
         tc::mbar_init(bar_mma, 1);
         tc::mbar_init(bar_d, 1);
         tc::mbar_init_fence();
     }
     if (wid == 0) tc::tmem_alloc(smem_addr(tslot), 256);
     __syncthreads();
-    // raw k and v rows of the chunk (rows past T read as zero); load_k reloads the k rows (second phase)
+    // raw k rows (bar_ld) and v rows (bar_v) of the chunk, rows past T read as zero; load_k reloads
+    // the k rows (second phase of bar_ld)
     auto load_k = [&]() {
         tma::expect_tx(bar_ld, 32768);
         tma::load_2d(sbase + OFF_K, &tm_k, hq * D, t0, bar_ld);
         tma::load_2d(sbase + OFF_K + 16384, &tm_k, hq * D + 64, t0, bar_ld);
     };
-    if (tid == 0) {  // one arrival and 64 KiB for the first phase of bar_ld
-        tma::expect_tx(bar_ld, 65536);
-        tma::load_2d(sbase + OFF_V, &tm_v, h * D, t0, bar_ld);
-        tma::load_2d(sbase + OFF_V + 16384, &tm_v, h * D + 64, t0, bar_ld);
-        tma::load_2d(sbase + OFF_K, &tm_k, hq * D, t0, bar_ld);
-        tma::load_2d(sbase + OFF_K + 16384, &tm_k, hq * D + 64, t0, bar_ld);
+    if (tid == 0) {
+        load_k();
+        tma::expect_tx(bar_v, 32768);
+        tma::load_2d(sbase + OFF_V, &tm_v, h * D, t0, bar_v);
+        tma::load_2d(sbase + OFF_V + 16384, &tm_v, h * D + 64, t0, bar_v);
     }
     // chunk-local cumulative gate and beta while the rows load
     chunk_gamma(g, Nv, h, t0, n, gam, reinterpret_cast<float *>(smem + OFF_BAR + 32));
@@ -191,10 +193,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
         tc::fence_after_sync();
     };
     wait_bar(bar_ld, 0);
-    if (n < L) {
-        zero_tail(OFF_K);
-        zero_tail(OFF_V);
-    }
+    if (n < L) zero_tail(OFF_K);
     sync_operands();
     const uint32_t tmem = *tslot;
     const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -218,8 +217,6 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
         gcum_out[(size_t)h * T + t0 + tid] = gam[tid];
         betaf_out[(size_t)h * T + t0 + tid] = bet[tid];
     }
-    // ... and diag(beta) v in fp16, in place
-    scale_rows_f16(smem + OFF_V, tid, L, [&](int r) { return bet[r]; });
     __syncthreads();
     if (tid < 128) {
         kfe[tid] = rkv[tid] * __expf(gam[tid | 15] - gam[tid]);
@@ -314,6 +311,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
         }
         // diag(beta e^gamma rk) k in fp16, in place (the k k^T product is complete)
         scale_rows_f16(smem + OFF_K, tid, L, [&](int r) { return bet[r] * __expf(gam[r]) * rkv[r]; });
+        // diag(beta) v in fp16, in place; rows past the chunk (the next sequence's) as zeros
+        wait_bar(bar_v, 0);
+        scale_rows_f16(smem + OFF_V, tid, n, [&](int r) { return bet[r]; });
     }
     __syncthreads();
 
@@ -492,10 +492,11 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     } else if (tid == 0) {
         atomicOr(status + 2, 4);
         // copies and MMAs still in flight land before shared and tensor memory are released:
-        // a commit covers every MMA issued before it, and both loads were counted on bar_ld
+        // a commit covers every MMA issued before it; then every load issued
         tc::commit(bar_d);
         tc::mbar_wait_bounded(bar_d, 0);
         tc::mbar_wait_bounded(bar_ld, 0);
+        tc::mbar_wait_bounded(bar_v, 0);
         tc::mbar_wait_bounded(bar_ld, 1);
     }
     if (tid == 0) tma::wait_read_all();  // the stores have read shared memory (the grid's end publishes them)

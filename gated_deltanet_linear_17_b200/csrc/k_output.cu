@@ -51,8 +51,8 @@ constexpr int OO_Q = 0;        // q (bf16) -> Qw (fp16), K-major over Dk -> O (b
 constexpr int OO_K = 32768;    // k (bf16), K-major over Dk -> S_c (fp16) [Dk][Dv], MN-major B of Qw S_c
 constexpr int OO_X = 65536;    // W (fp16) [L][Dk], MN-major B of P W -> U (fp16) [L][Dv], MN-major B of P U
 constexpr int OO_VEC = 98304;  // gam, rqv, rkv, kfe (rk_j e^{gamma_je - gamma_j})
-constexpr int OO_BAR = OO_VEC + 4 * 512;  // mbarriers, TMEM slot, scan sums (64 bytes)
-constexpr int kOutSmem = OO_BAR + 64 + 1024;
+constexpr int OO_BAR = OO_VEC + 4 * 512;  // mbarriers, TMEM slot, scan sums (72 bytes)
+constexpr int kOutSmem = OO_BAR + 128 + 1024;
 
 // byte offset of 16-byte chunk c (0..15) of row r in a 128 x 128 tile
 __device__ __forceinline__ uint32_t t128(int r, int c) { return (uint32_t)((c >> 3) * 16384) + tc::sw128c(r, c & 7); }
@@ -80,6 +80,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     const uint32_t bar_ld = sbase + OO_BAR, bar_mma = sbase + OO_BAR + 8, bar_d = sbase + OO_BAR + 16;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + OO_BAR + 24);
     const uint32_t bar_s = sbase + OO_BAR + 48, bar_u = sbase + OO_BAR + 56;  // S_c and U loads
+    const uint32_t bar_w = sbase + OO_BAR + 64;                                 // W load (q, k on bar_ld)
     const int trow = (c * Nv + h) * L;  // first row of the chunk's tiles in the workspace
 
     if (tid == 0) {
@@ -88,18 +89,20 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         tc::mbar_init(bar_d, 1);
         tc::mbar_init(bar_s, 1);
         tc::mbar_init(bar_u, 1);
+        tc::mbar_init(bar_w, 1);
         tc::mbar_init_fence();
     }
     if (wid == 0) tc::tmem_alloc(smem_addr(tslot), 256);
     __syncthreads();
-    if (tid == 0) {  // one arrival and 96 KiB for the first phase of bar_ld
-        tma::expect_tx(bar_ld, 98304);
+    if (tid == 0) {  // q and k (64 KiB) on bar_ld, W (32 KiB) on bar_w
+        tma::expect_tx(bar_ld, 65536);
         tma::load_2d(sbase + OO_Q, &tm_q, hq * D, t0, bar_ld);
         tma::load_2d(sbase + OO_Q + 16384, &tm_q, hq * D + 64, t0, bar_ld);
         tma::load_2d(sbase + OO_K, &tm_k, hq * D, t0, bar_ld);
         tma::load_2d(sbase + OO_K + 16384, &tm_k, hq * D + 64, t0, bar_ld);
-        tma::load_2d(sbase + OO_X, &tm_w, 0, trow, bar_ld);
-        tma::load_2d(sbase + OO_X + 16384, &tm_w, 64, trow, bar_ld);
+        tma::expect_tx(bar_w, 32768);
+        tma::load_2d(sbase + OO_X, &tm_w, 0, trow, bar_w);
+        tma::load_2d(sbase + OO_X + 16384, &tm_w, 64, trow, bar_w);
     }
     // chunk-local cumulative gate while the rows load
     chunk_gamma(g, Nv, h, t0, n, gam, reinterpret_cast<float *>(smem + OO_BAR + 32));
@@ -241,16 +244,26 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     // ---- (3) S_c starts loading over the consumed k tile; Z = P W (P from TMEM) into TMEM columns
     // [0, 128); U then loads over the consumed W; Qw = diag(rq e^gamma) q - Z in fp16, in place of q
     const uint32_t idesc_n128 = tc::idesc_f16(128, 128, false, false, false, true);
-    if (ok && tid == 0) {
-        load_tile(sbase + OO_K, &tm_sc, bar_s);
-        s_issued = true;
-        const uint64_t dw = tc::desc_mn(sbase + OO_X, 16384, 1024, 2);
+    if (ok) {
+        bool w_ok = true;
+        if (tid == 0) {
+            load_tile(sbase + OO_K, &tm_sc, bar_s);
+            s_issued = true;
+            w_ok = tc::mbar_wait_bounded(bar_w, 0);  // W has landed
+            if (w_ok) {
+                const uint64_t dw = tc::desc_mn(sbase + OO_X, 16384, 1024, 2);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-            tc::mma_f16_ts(tmem, tmem + 128 + kk * 8, dw + (uint64_t)((kk * 2048) >> 4), idesc_n128, kk > 0 ? 1u : 0u);
-        tc::commit(bar_mma);
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_f16_ts(tmem, tmem + 128 + kk * 8, dw + (uint64_t)((kk * 2048) >> 4), idesc_n128,
+                                   kk > 0 ? 1u : 0u);
+            }
+            tc::commit(bar_mma);
+            w_ok = tc::mbar_wait_bounded(bar_mma, 1) && w_ok;  // second phase of bar_mma
+        }
+        tc::fence_before_sync();
+        ok = __syncthreads_and(w_ok) != 0 && ok;
+        tc::fence_after_sync();
     }
-    if (ok) wait_bar(bar_mma, 1);
     if (ok && tid == 0) {
         load_tile(sbase + OO_X, &tm_u, bar_u);
         u_issued = true;
@@ -343,6 +356,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         tc::commit(bar_d);
         tc::mbar_wait_bounded(bar_d, 0);
         tc::mbar_wait_bounded(bar_ld, 0);
+        tc::mbar_wait_bounded(bar_w, 0);
         if (s_issued) tc::mbar_wait_bounded(bar_s, 0);
         if (u_issued) tc::mbar_wait_bounded(bar_u, 0);
     }
