@@ -46,14 +46,56 @@ def flops_per_token(Nqk, Nv):
     return Nv * (4 * L * D + 2 * L * D + 6 * D * D) + Nqk * (4 * L * D)
 
 
-def stage_work(T, Nqk, Nv):
-    """Algorithmic work of one launch of each stage: (bound, amount, unit)."""
+def stage_work(T, Nqk, Nv, NC, B):
+    """Algorithmic work of one launch of each stage: {stage: (FLOP, HBM bytes)}.
+
+    FLOP: the dense tensor-core products of the stage (counted once per
+    qk-head where shared).  Bytes: what the stage must read and write in HBM
+    at least once, with NC chunks and 32 KiB fp16 tiles per (chunk, v-head):
+      intra  reads k, v, g, beta; writes U, W, Mk and the 528-byte factor
+             records (the inspection copies of gcum, betaf, rk not counted)
+      state  reads Mk, k, U, the factor records; writes S_c and the final state
+      output reads q, k, g, W, U, S_c; writes out."""
+    tile = L * D * 2
+    qk, v, g, beta = T * Nqk * D * 2, T * Nv * D * 2, T * Nv * 4, T * Nv * 2
+    fa = NC * Nv * 528
+    tiles = NC * Nv * tile
     return {
-        "chunk_map": ("hbm", 0.0, "GB/s"),
-        "intra": ("tensor", T * (Nv * (2 * L * D + 2 * L * D) + Nqk * 2 * L * D), "TFLOP/s"),
-        "state": ("tensor", T * Nv * 4 * D * D, "TFLOP/s"),
-        "output": ("tensor", T * (Nv * (2 * D * D + 2 * L * D) + Nqk * 2 * L * D), "TFLOP/s"),
+        "chunk_map": (0.0, 4.0 * (B + 1) + 16.0 * NC),
+        "intra": (T * (Nv * (2 * L * D + 2 * L * D) + Nqk * 2 * L * D), qk + v + g + beta + 3 * tiles + fa),
+        "state": (T * Nv * 4 * D * D, 2 * tiles + qk + fa + tiles + B * Nv * D * D * 4),
+        "output": (T * (Nv * (2 * D * D + 2 * L * D) + Nqk * 2 * L * D), 2 * qk + g + 3 * tiles + v),
     }
+
+
+def roofline_of(flop, nbytes, sec, peaks):
+    """The roofline that binds (the larger time at peak) and the fraction achieved on it."""
+    t_tc = flop / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    if t_hbm >= t_tc:
+        return {"bound": "hbm", "achieved": nbytes / sec / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": nbytes / sec / 1e9 / peaks["hbm_gbs"], "per_launch": f"{nbytes:.4g} bytes per launch"}
+    return {"bound": "tensor", "achieved": flop / sec / 1e12, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": flop / sec / 1e12 / peaks["bf16_tflops"], "per_launch": f"{flop:.4g} FLOP per launch"}
+
+
+def measured_traffic(kernel, units):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, scaled from the
+    captured workload to `units` (chunk, v-head) pairs; None when there is no capture or
+    the kernel's source has changed since it was taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "gated_deltanet_linear_17_b200", "csrc", rec["source"])
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+            return None
+    return rec["dram_bytes_per_launch"] * units / rec["units"]
 
 
 def short_bytes(inp):
@@ -253,24 +295,23 @@ def main():
     F = flops_per_token(Nqk, Nv)
     tc_frac = F * T / (ms / 1e3) / (peaks["bf16_tflops"] * 1e12)
 
-    work = stage_work(T, Nqk, Nv)
+    nchunks = sum((n + L - 1) // L for n in inp.seqlens)
+    work = stage_work(T, Nqk, Nv, nchunks, inp.B)
     dom = max(names, key=lambda n: stage_ms[n])
-    bound, amount, unit = work[dom]
-    sec = stage_ms[dom] / 1e3
-    if bound == "hbm":
-        achieved, peak = amount / sec / 1e9, peaks["hbm_gbs"]
-    else:
-        achieved, peak = amount / sec / 1e12, peaks["bf16_tflops"]
-    roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": achieved / peak, "traffic": None,
-                "peak_source": f"{peaks['source']} (burst bf16 / STREAM copy)",
-                "per_launch": f"{amount:.4g} {'bytes' if bound == 'hbm' else 'FLOP'} per launch"}
+    units = nchunks * Nv  # (chunk, v-head) pairs, the CTAs of the intra and output kernels
+    roofline = {"kernel": dom, **roofline_of(*work[dom], stage_ms[dom] / 1e3, peaks),
+                "traffic": measured_traffic(f"{dom}_kernel", units),
+                "peak_source": f"{peaks['source']} (burst bf16 / STREAM copy)"}
+    stage_roofline = {n: {k: (round(v, 4) if isinstance(v, float) else v) for k, v in
+                          roofline_of(*work[n], stage_ms[n] / 1e3, peaks).items() if k in ("bound", "frac")}
+                      for n in names if n != "chunk_map"}
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; see inputs.CONFIGS)",
             "config": workload_config(inp), "tc_frac": tc_frac,
             "stages_ms": {n: round(v, 5) for n, v in stage_ms.items()}, "roofline": roofline,
+            "stage_roofline": stage_roofline,
             "gpu_launches": len(names) * args.steps, "clocks": clocks}
 
     # ---- short-sequence state-pool pass (HBM-bound)
