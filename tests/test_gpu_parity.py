@@ -63,6 +63,13 @@ def test_short_pool_b256_both_paths():
         assert_close(fin, rf, f"short max_seqlen={ms} final_state")
 
 
+def test_short_path_without_pool_two_heads():
+    """Fused short kernel with a zero initial state, empty sequences and Nv = 2 (g, beta rows of 8 and 4 bytes)."""
+    inp = inputs.make([5, 1, 8, 0, 3, 16, 0], Nqk=1, Nv=2, seed=21)
+    out, fin = _gpu(inp, max_seqlen=16)
+    _check(inp, out, fin, what="short, no pool")
+
+
 @pytest.mark.slow
 def test_long_s128k_b2_sampled_heads():
     """Two 128K-token sequences with initial states, oracle on v-heads 0, 7, 16, 31."""
