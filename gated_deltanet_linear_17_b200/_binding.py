@@ -30,7 +30,8 @@ _lib = None
 
 class _Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
-                ("total", "status", "chunk_info", "seq_chunk0", "rq", "rk", "gcum", "betaf", "U", "W", "Mk", "Sc", "fa")] + \
+                ("total", "status", "chunk_info", "seq_chunk0", "rq", "rk", "gcum", "betaf", "U", "W", "Mk", "Sc", "fa",
+                 "carry")] + \
                [("max_chunks", ctypes.c_int64)]
 
 
@@ -192,6 +193,13 @@ def chunk_fwd_noalloc(q, k, v, g, beta, cu_seqlens, out, final_state=None, state
                                      _ptr(final_state), T, B, Nqk, Nv, P, int(max_seqlen), _stream(stream))
     _check(rc, "gdn_chunk_fwd_noalloc")
     return out, final_state
+
+
+def pipeline_ranges(T, B, Nqk=1, Nv=1):
+    """Number of chunk ranges gdn_chunk_fwd pipelines for these sizes (one carry slot per boundary
+    in the workspace layout)."""
+    lay = workspace_layout(T, B, Nqk, Nv)
+    return 1 + (lay["total"] - lay["carry"]) // (Nv * HEAD_DIM * HEAD_DIM * 4)
 
 
 def short_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None, scale=None, eps=1e-6,

@@ -1,7 +1,16 @@
 // Host side of the C ABI (include/gdn.h, include/gdn_stages.h): argument
-// checks, workspace layout and the launch sequence on the caller's stream.
+// checks, workspace layout and the launch sequence.  The chunked forward pass
+// splits the chunks into ranges and runs them as a pipeline: the intra-chunk
+// kernel on a low-priority stream, the state pass on a high-priority stream
+// (range r after the intra-chunk kernel of range r and the state pass of range
+// r - 1) and the output kernel on the caller's stream (range r after the state
+// pass of range r), so the state pass, which keeps only part of the GPU busy,
+// runs beside the other two kernels of neighbouring ranges.  The side streams
+// fork from and join back into the caller's stream within the call.
 #include <math.h>
 #include <string.h>
+
+#include <mutex>
 
 #include "gdn.h"
 #include "gdn_internal.h"
@@ -14,6 +23,38 @@ namespace {
 constexpr int kVersion = 100;  // 0.1.0
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// The pipeline's side streams and events, per device, created on first use and kept
+// until the process exits; g_pipe_lock serialises their use (a call's record / wait
+// pairs must not interleave with another host thread's).
+constexpr int kMaxPipeDevices = 64;
+struct SideStreams {
+    cudaStream_t intra = nullptr, state = nullptr;
+    cudaEvent_t ev[2 * gdn::kMaxRanges + 3] = {};
+    bool ready = false;
+};
+std::mutex g_pipe_lock;
+SideStreams g_side[kMaxPipeDevices];
+
+cudaError_t side_streams(SideStreams **out)
+{
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxPipeDevices) return cudaErrorInvalidDevice;
+    SideStreams &s = g_side[dev];
+    if (!s.ready) {
+        int least = 0, greatest = 0;
+        if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
+        if ((e = cudaStreamCreateWithPriority(&s.intra, cudaStreamNonBlocking, least)) != cudaSuccess) return e;
+        if ((e = cudaStreamCreateWithPriority(&s.state, cudaStreamNonBlocking, greatest)) != cudaSuccess) return e;
+        for (auto &x : s.ev)
+            if ((e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming)) != cudaSuccess) return e;
+        s.ready = true;
+    }
+    *out = &s;
+    return cudaSuccess;
+}
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -49,6 +90,9 @@ int fill_layout(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, gdn_workspace_lay
     off += (size_t)NC * Nv * tile;
     lay->fa = off;
     off += (size_t)NC * Nv * gdn::kFaStride * 4;
+    off = align256(off);
+    lay->carry = off;
+    off += (size_t)(gdn::pipeline_ranges(NC) - 1) * Nv * gdn::D * gdn::D * 4;
     lay->total = align256(off);
     lay->max_chunks = NC;
     return GDN_OK;
@@ -70,6 +114,7 @@ Workspace views(void *base, const gdn_workspace_layout_t &lay)
     w.Mk = reinterpret_cast<uint16_t *>(p + lay.Mk);
     w.Sc = reinterpret_cast<uint16_t *>(p + lay.Sc);
     w.fa = reinterpret_cast<float *>(p + lay.fa);
+    w.carry = reinterpret_cast<float *>(p + lay.carry);
     w.NC = static_cast<int>(lay.max_chunks);
     return w;
 }
@@ -194,7 +239,7 @@ int gdn_stage_intra(const uint16_t *k, const uint16_t *v, const float *g, const 
     if (!k || !v || !g || !beta) return GDN_ERR_NULL_ARG;
     if (!aligned16(k) || !aligned16(v)) return GDN_ERR_ALIGNMENT;
     const Workspace w = views(workspace, lay);
-    return cuda_status(gdn::launch_intra(k, v, g, beta, eps, (int)T, Nqk, Nv, w.NC, w, (cudaStream_t)stream));
+    return cuda_status(gdn::launch_intra(k, v, g, beta, eps, (int)T, Nqk, Nv, 0, w.NC, w, (cudaStream_t)stream));
 }
 
 int gdn_stage_state(const uint16_t *k, const float *state_pool, const int32_t *state_indices, float *final_state,
@@ -214,7 +259,7 @@ int gdn_stage_state(const uint16_t *k, const float *state_pool, const int32_t *s
     const size_t sbytes = (size_t)gdn::D * gdn::D * 4 * Nv;
     if (overlap(final_state, sbytes * B, state_pool, sbytes * P)) return GDN_ERR_OVERLAP;
     const Workspace w = views(workspace, lay);
-    return cuda_status(gdn::launch_state(k, state_pool, state_indices, final_state, (int)T, B, Nqk, Nv, w,
+    return cuda_status(gdn::launch_state(k, state_pool, state_indices, final_state, (int)T, B, Nqk, Nv, 0, w.NC, 0, w,
                                          (cudaStream_t)stream));
 }
 
@@ -230,7 +275,7 @@ int gdn_stage_output(const uint16_t *q, const uint16_t *k, const float *g, float
     if (!q || !k || !g || !out) return GDN_ERR_NULL_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(out)) return GDN_ERR_ALIGNMENT;
     const Workspace w = views(workspace, lay);
-    return cuda_status(gdn::launch_output(q, k, g, resolve_scale(scale), eps, out, (int)T, Nqk, Nv, w.NC, w,
+    return cuda_status(gdn::launch_output(q, k, g, resolve_scale(scale), eps, out, (int)T, Nqk, Nv, 0, w.NC, w,
                                           (cudaStream_t)stream));
 }
 
@@ -274,11 +319,50 @@ int gdn_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
         if (workspace_bytes < lay.total) return GDN_ERR_WORKSPACE;
     }
     const Workspace w = views(workspace, lay);
-    const int Ti = (int)T;
-    cudaError_t e = gdn::launch_chunk_map(cu_seqlens, B, Ti, w.NC, w, st);
-    if (e == cudaSuccess) e = gdn::launch_intra(k, v, g, beta, eps, Ti, Nqk, Nv, w.NC, w, st);
-    if (e == cudaSuccess) e = gdn::launch_state(k, state_pool, state_indices, final_state, Ti, B, Nqk, Nv, w, st);
-    if (e == cudaSuccess) e = gdn::launch_output(q, k, g, sc, eps, out, Ti, Nqk, Nv, w.NC, w, st);
+    const int Ti = (int)T, NC = w.NC;
+    cudaError_t e = gdn::launch_chunk_map(cu_seqlens, B, Ti, NC, w, st);
+    const int R = gdn::pipeline_ranges(NC);
+    if (e == cudaSuccess && R == 1) {
+        e = gdn::launch_intra(k, v, g, beta, eps, Ti, Nqk, Nv, 0, NC, w, st);
+        if (e == cudaSuccess)
+            e = gdn::launch_state(k, state_pool, state_indices, final_state, Ti, B, Nqk, Nv, 0, NC, 0, w, st);
+        if (e == cudaSuccess) e = gdn::launch_output(q, k, g, sc, eps, out, Ti, Nqk, Nv, 0, NC, w, st);
+    } else if (e == cudaSuccess) {
+        std::lock_guard<std::mutex> guard(g_pipe_lock);
+        SideStreams *ss = nullptr;
+        e = side_streams(&ss);
+        if (e == cudaSuccess) {
+            // ev[0]: fork; ev[1 + r]: intra-chunk of range r done; ev[1 + R + r]: state pass of range r done;
+            // ev[1 + 2R], ev[2 + 2R]: join
+            cudaEvent_t *ev = ss->ev;
+            auto c0 = [&](int r) { return gdn::range_begin(r, R, NC); };
+            auto c1 = [&](int r) { return gdn::range_begin(r + 1, R, NC); };
+            e = cudaEventRecord(ev[0], st);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->intra, ev[0], 0);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->state, ev[0], 0);
+            for (int r = 0; r < R && e == cudaSuccess; ++r) {
+                e = gdn::launch_intra(k, v, g, beta, eps, Ti, Nqk, Nv, c0(r), c1(r) - c0(r), w, ss->intra);
+                if (e == cudaSuccess) e = cudaEventRecord(ev[1 + r], ss->intra);
+            }
+            for (int r = 0; r < R && e == cudaSuccess; ++r) {
+                e = cudaStreamWaitEvent(ss->state, ev[1 + r], 0);
+                if (e == cudaSuccess)
+                    e = gdn::launch_state(k, state_pool, state_indices, final_state, Ti, B, Nqk, Nv, c0(r), c1(r), r,
+                                          w, ss->state);
+                if (e == cudaSuccess) e = cudaEventRecord(ev[1 + R + r], ss->state);
+            }
+            for (int r = 0; r < R && e == cudaSuccess; ++r) {
+                e = cudaStreamWaitEvent(st, ev[1 + R + r], 0);
+                if (e == cudaSuccess) e = gdn::launch_output(q, k, g, sc, eps, out, Ti, Nqk, Nv, c0(r), c1(r) - c0(r), w, st);
+            }
+            // join, also after a failed launch, so that nothing of this call runs outside `st` afterwards
+            cudaError_t j = cudaEventRecord(ev[1 + 2 * R], ss->intra);
+            if (j == cudaSuccess) j = cudaEventRecord(ev[2 + 2 * R], ss->state);
+            if (j == cudaSuccess) j = cudaStreamWaitEvent(st, ev[1 + 2 * R], 0);
+            if (j == cudaSuccess) j = cudaStreamWaitEvent(st, ev[2 + 2 * R], 0);
+            if (e == cudaSuccess) e = j;
+        }
+    }
     if (owned) {
         cudaError_t f = cudaFreeAsync(workspace, st);
         if (e == cudaSuccess) e = f;

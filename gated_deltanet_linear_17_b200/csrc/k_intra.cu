@@ -126,12 +126,12 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_w,
     const __grid_constant__ CUtensorMap tm_mk, const float *__restrict__ g, const uint16_t *__restrict__ beta,
     float eps, int T, int Nqk, int Nv, const int4 *__restrict__ info, float *__restrict__ rk_out,
-    float *__restrict__ gcum_out, float *__restrict__ betaf_out, float *__restrict__ fa, int32_t *__restrict__ status)
+    float *__restrict__ gcum_out, float *__restrict__ betaf_out, float *__restrict__ fa, int32_t *__restrict__ status, int c0)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
     const uint32_t sbase = smem_addr(smem);
-    const int c = blockIdx.x, h = blockIdx.y;
+    const int c = c0 + blockIdx.x, h = blockIdx.y;
     const ChunkInfo ci = load_chunk(info, c);
     if (ci.seq < 0) return;
     const int hq = h / (Nv / Nqk);
@@ -507,10 +507,11 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
 }
 
 cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, const float *g, const uint16_t *beta, float eps, int T,
-                         int Nqk, int Nv, int NC, const Workspace &ws, cudaStream_t st)
+                         int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st)
 {
-    if (NC == 0 || T == 0) return cudaSuccess;
-    const uint64_t trows = (uint64_t)NC * Nv * L;  // TMA coordinates are 32-bit signed
+    if (nc <= 0 || T == 0) return cudaSuccess;
+    if (c0 < 0 || c0 + nc > ws.NC) return cudaErrorInvalidValue;
+    const uint64_t trows = (uint64_t)ws.NC * Nv * L;  // TMA coordinates are 32-bit signed
     if ((uint64_t)T >= (1ull << 31) || trows >= (1ull << 31)) return cudaErrorInvalidValue;
     CUtensorMap m_k, m_v, m_u, m_w, m_mk;
     cudaError_t e = tma::map2d(&m_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, (uint64_t)Nqk * D, (uint64_t)T,
@@ -528,9 +529,9 @@ cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, const float *g, c
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kIntraSmem);
     if (e != cudaSuccess) return e;
-    intra_kernel<<<dim3(NC, Nv), kIntraThreads, kIntraSmem, st>>>(m_k, m_v, m_u, m_w, m_mk, g, beta, eps, T, Nqk, Nv,
+    intra_kernel<<<dim3(nc, Nv), kIntraThreads, kIntraSmem, st>>>(m_k, m_v, m_u, m_w, m_mk, g, beta, eps, T, Nqk, Nv,
                                                                    ws.chunk_info, ws.rk, ws.gcum, ws.betaf, ws.fa,
-                                                                   ws.status);
+                                                                   ws.status, c0);
     return cudaGetLastError();
 }
 

@@ -62,12 +62,12 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sc,
     const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_out, uint16_t *__restrict__ out,
     const float *__restrict__ g, float scale, float eps, int T, int Nqk, int Nv, const int4 *__restrict__ info,
-    float *__restrict__ rq_out, int32_t *__restrict__ status)
+    float *__restrict__ rq_out, int32_t *__restrict__ status, int c0)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
     const uint32_t sbase = smem_addr(smem);
-    const int c = blockIdx.x, h = blockIdx.y;
+    const int c = c0 + blockIdx.x, h = blockIdx.y;
     const ChunkInfo ci = load_chunk(info, c);
     if (ci.seq < 0) return;
     const int hq = h / (Nv / Nqk);
@@ -368,10 +368,11 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
 }
 
 cudaError_t launch_output(const uint16_t *q, const uint16_t *k, const float *g, float scale, float eps, uint16_t *out,
-                          int T, int Nqk, int Nv, int NC, const Workspace &ws, cudaStream_t st)
+                          int T, int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st)
 {
-    if (NC == 0 || T == 0) return cudaSuccess;
-    const uint64_t trows = (uint64_t)NC * Nv * L;  // TMA coordinates are 32-bit signed
+    if (nc <= 0 || T == 0) return cudaSuccess;
+    if (c0 < 0 || c0 + nc > ws.NC) return cudaErrorInvalidValue;
+    const uint64_t trows = (uint64_t)ws.NC * Nv * L;  // TMA coordinates are 32-bit signed
     if ((uint64_t)T >= (1ull << 31) || trows >= (1ull << 31)) return cudaErrorInvalidValue;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, HF = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
@@ -385,8 +386,8 @@ cudaError_t launch_output(const uint16_t *q, const uint16_t *k, const float *g, 
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
     if (e != cudaSuccess) return e;
-    output_kernel<<<dim3(NC, Nv), kOutThreads, kOutSmem, st>>>(m_q, m_k, m_w, m_sc, m_u, m_out, out, g, scale, eps, T,
-                                                                Nqk, Nv, ws.chunk_info, ws.rq, ws.status);
+    output_kernel<<<dim3(nc, Nv), kOutThreads, kOutSmem, st>>>(m_q, m_k, m_w, m_sc, m_u, m_out, out, g, scale, eps, T,
+                                                                Nqk, Nv, ws.chunk_info, ws.rq, ws.status, c0);
     return cudaGetLastError();
 }
 

@@ -1,9 +1,12 @@
 /*
  * gdn_stages.h -- the kernels of gdn_chunk_fwd as separate C-ABI calls.
  *
- * gdn_chunk_fwd (gdn.h) is exactly gdn_stage_chunk_map, gdn_stage_intra,
- * gdn_stage_state and gdn_stage_output enqueued in that order
- * on one stream with one workspace.  The stages are exposed so that each
+ * gdn_chunk_fwd (gdn.h) runs the same kernels as gdn_stage_chunk_map,
+ * gdn_stage_intra, gdn_stage_state and gdn_stage_output enqueued in that order
+ * on one stream with one workspace, with the same results: it splits the
+ * chunks into R ranges (see `carry`) and overlaps the ranges' kernels on
+ * streams of its own, which fork from and join back into the caller's stream
+ * within the call.  The stages run over all chunks.  They are exposed so that each
  * kernel can be checked against the chunked form's intermediates and timed on
  * its own.  Conventions (device pointers, bf16 as uint16_t bits, asynchronous
  * on `stream`, status codes, alignment) are those of gdn.h.  Every stage takes
@@ -54,6 +57,9 @@ extern "C" {
  *   Sc          fp16 [NC][Nv][128 (Dk)][128 (Dv)]: state entering each chunk
  *   fa          fp32 [NC][Nv][132]: per chunk rk_t e^{gamma_L - gamma_t} for its
  *               rows t < 128 (0 past the chunk), e^{gamma_L} at 128, zeros after
+ *   carry       fp32 [R-1][Nv][128][128]: the state of a sequence that crosses the
+ *               boundary after chunk range r (the forward pass runs R chunk ranges
+ *               as a pipeline: R = 2 from NC = 32 on, else 1; empty when R = 1)
  * The tensor-core products take fp16 operands (11-bit significand) with fp32
  * accumulation: the raw bf16 q, k, v convert to fp16 exactly (magnitudes in
  * [2^-14, 65504]), the L2 norms enter as fp32 scalings, and the state update's
@@ -75,6 +81,7 @@ typedef struct {
     size_t Mk;
     size_t Sc;
     size_t fa;
+    size_t carry;
     int64_t max_chunks;
 } gdn_workspace_layout_t;
 
@@ -107,7 +114,7 @@ int gdn_stage_intra(const uint16_t *k, const uint16_t *v, const float *g, const 
                     void *stream);
 
 /*
- * Inter-chunk state passing: per (sequence, v-head, 32-column slice of Dv),
+ * Inter-chunk state passing: per (sequence, v-head, 64-column slice of Dv),
  * serially over the sequence's chunks, S <- e^{gamma_last} S + k_gexp^T U - Mk S
  * ("State Update" with v' = W S regrouped), the state kept in fp32 on chip.
  * S starts from state_pool[state_indices[b]] (or slot b, or zero without a

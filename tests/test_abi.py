@@ -52,13 +52,17 @@ def test_status_strings(lib):
 def test_workspace_layout_regions_disjoint_and_aligned(lib):
     lay = gdn.workspace_layout(4048, 4, 4, 8)
     assert lay["max_chunks"] == (4048 + 127 * 4) // 128
-    regions = ["status", "chunk_info", "seq_chunk0", "rq", "rk", "gcum", "betaf", "U", "W", "Mk", "Sc", "fa"]
+    regions = ["status", "chunk_info", "seq_chunk0", "rq", "rk", "gcum", "betaf", "U", "W", "Mk", "Sc", "fa", "carry"]
     offs = [lay[r] for r in regions]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     tile = 128 * 128 * 2
     assert lay["W"] - lay["U"] == lay["max_chunks"] * 8 * tile
     assert lay["fa"] >= lay["Sc"] + lay["max_chunks"] * 8 * tile
-    assert lay["total"] >= lay["fa"] + lay["max_chunks"] * 8 * 132 * 4
+    assert lay["carry"] >= lay["fa"] + lay["max_chunks"] * 8 * 132 * 4
+    assert lay["total"] >= lay["carry"]  # few chunks: one range, no carry slots
+    big = gdn.workspace_layout(32768, 1, 16, 32)  # 256 chunks: 2 ranges, 1 carry slot
+    assert big["total"] >= big["carry"] + 32 * 128 * 128 * 4
+    assert gdn.pipeline_ranges(32768, 1, 16, 32) == 2 and gdn.pipeline_ranges(3000, 1, 16, 32) == 1
     assert gdn.workspace_bytes(4048, 4, 4, 8) == lay["total"]
 
 

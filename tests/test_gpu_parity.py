@@ -288,3 +288,35 @@ def test_workspace_given_or_internal_identical():
     assert rc == 0
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(f1, f2)
+
+
+# ------------------------------------------------------------------ the pipelined forward pass
+
+def _staged(inp):
+    d = inp.to(DEV)
+    st = gdn.Stages(inp.T, inp.B, inp.Nqk, inp.Nv, DEV)
+    out, fin = st.run_all(d.q, d.k, d.v, d.g, d.beta, d.cu_seqlens, d.state_pool, d.state_indices,
+                          scale=inp.scale, eps=inp.eps)
+    torch.cuda.synchronize()
+    return out, fin
+
+
+@pytest.mark.parametrize("lens", [[32768], [3000, 5000, 129, 0, 2600], [9000, 1, 7000], [2048, 2048]],
+                         ids=["one_seq", "boundary_inside_seq", "tiny_seq_between", "boundary_between_seqs"])
+def test_pipelined_equals_staged_bit_exact(lens):
+    """gdn_chunk_fwd runs chunk ranges as a pipeline over several streams, with the state of a
+    sequence that crosses a range boundary carried in fp32: it must equal the kernels run one
+    after another over all chunks, bit for bit."""
+    inp = inputs.make(lens, Nqk=4, Nv=8, state=("normal", 0.02, len(lens), "perm"), seed=31)
+    assert gdn.pipeline_ranges(inp.T, inp.B, inp.Nqk, inp.Nv) > 1
+    out, fin = _gpu(inp)
+    so, sf = _staged(inp)
+    assert torch.equal(out, so) and torch.equal(fin, sf)
+
+
+def test_pipelined_varlen_against_oracle():
+    """A range boundary inside a sequence, an empty sequence and a 2-chunk sequence, through the
+    pipelined call, against the oracle on a subset of v-heads."""
+    inp = inputs.make([3000, 5000, 129, 0, 2600], Nqk=4, Nv=8, state=("normal", 0.02, 5, "perm"), seed=32)
+    out, fin = _gpu(inp)
+    _check(inp, out, fin, heads=[0, 3, 5], what="pipelined varlen")
