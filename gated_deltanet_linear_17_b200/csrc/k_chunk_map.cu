@@ -59,17 +59,32 @@ __global__ void __launch_bounds__(kMapThreads) chunk_map_kernel(const int32_t *_
     const int base = (wid ? warp_tot[wid - 1] : 0) + incl - my;
     const int total = warp_tot[kMapThreads / 32 - 1];
 
-    int c = base;
-    for (int b = b0; b < b1; ++b) {
-        int s = cu[b], e = cu[b + 1];
-        s = min(max(s, 0), T);
-        e = min(max(e, s), T);
-        seq_chunk0[b] = min(c, NC);
-        for (int t = s, j = 0; t < e; t += L, ++j, ++c)
-            if (c < NC) info[c] = make_int4(b, t, min(L, e - t), j);
+    // first chunk of every sequence, then the chunks themselves spread over the block: chunk c
+    // belongs to the last sequence whose first chunk is <= c (binary search)
+    {
+        int c = base;
+        for (int b = b0; b < b1; ++b) {
+            int s = cu[b], e = cu[b + 1];
+            s = min(max(s, 0), T);
+            e = min(max(e, s), T);
+            seq_chunk0[b] = min(c, NC);
+            c += (e - s + L - 1) / L;
+        }
+    }
+    if (tid == 0) seq_chunk0[B] = min(total, NC);
+    __syncthreads();  // seq_chunk0 is complete (global writes of the block, ordered by the barrier)
+    for (int c = tid; c < min(total, NC); c += kMapThreads) {
+        int lo = 0, hi = B - 1;  // seq_chunk0[lo] <= c < seq_chunk0[hi + 1]
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (seq_chunk0[mid] <= c) lo = mid;
+            else hi = mid - 1;
+        }
+        const int s = min(max(cu[lo], 0), T), e = min(max(cu[lo + 1], s), T);
+        const int j = c - seq_chunk0[lo], t = s + j * L;
+        info[c] = make_int4(lo, t, min(L, e - t), j);
     }
     if (tid == 0) {
-        seq_chunk0[B] = min(total, NC);
         status[0] = err_bits;
         status[1] = total;
     }
