@@ -196,11 +196,11 @@ __device__ __forceinline__ ChunkInfo load_chunk(const int4 *info, int c)
 // value.  Every thread of the CTA calls it (it holds barriers); threads 0..127
 // produce gam[i]; wsum is 4 floats of shared scratch.  The kernels that need the
 // gate all use this function, so they see the same fp32 values bit for bit.
-__device__ __forceinline__ void chunk_gamma(const float *__restrict__ g, int Nv, int h, int t0, int n, float *gam,
-                                            float *wsum)
+// chunk_gamma_x takes the thread's gate value already loaded (0 for threads from n on and
+// from 128 on), so that a kernel can fetch it ahead of time.
+__device__ __forceinline__ void chunk_gamma_x(float x, float *gam, float *wsum)
 {
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    float x = (tid < 128 && tid < n) ? g[(size_t)(t0 + tid) * Nv + h] : 0.f;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const float y = __shfl_up_sync(0xffffffffu, x, o);
@@ -214,6 +214,13 @@ __device__ __forceinline__ void chunk_gamma(const float *__restrict__ g, int Nv,
         gam[tid] = x + pre;
     }
     __syncthreads();
+}
+
+__device__ __forceinline__ void chunk_gamma(const float *__restrict__ g, int Nv, int h, int t0, int n, float *gam,
+                                            float *wsum)
+{
+    const int tid = threadIdx.x;
+    chunk_gamma_x((tid < 128 && tid < n) ? g[(size_t)(t0 + tid) * Nv + h] : 0.f, gam, wsum);
 }
 
 // Largest gate span gamma_first - gamma_last of a 16-row block for which a row's
