@@ -157,6 +157,26 @@ __device__ __forceinline__ uint32_t bf2_to_h2(uint32_t x)
     return pack_h2(__uint_as_float(x << 16), __uint_as_float(x & 0xffff0000u));
 }
 
+// Packed fp32 pair arithmetic of sm_100 (one instruction for two lanes of a float2, each an
+// IEEE round-to-nearest operation, so the results equal two fmaf / two multiplications).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<const uint64_t *>(&a)), "l"(*reinterpret_cast<const uint64_t *>(&b)),
+          "l"(*reinterpret_cast<const uint64_t *>(&c)));
+    return *reinterpret_cast<const float2 *>(&d);
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b)
+{
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<const uint64_t *>(&a)), "l"(*reinterpret_cast<const uint64_t *>(&b)));
+    return *reinterpret_cast<const float2 *>(&d);
+}
+
 __device__ __forceinline__ float warp_sum(float x)
 {
 #pragma unroll

@@ -289,7 +289,7 @@ int gdn_short_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
                            Nqk, Nv, P);
     if (rc || B == 0) return rc;
     return cuda_status(gdn::launch_short(q, k, v, g, beta, cu_seqlens, state_pool, state_indices,
-                                         resolve_scale(scale), eps, out, final_state, (int)T, B, Nqk, Nv,
+                                         resolve_scale(scale), eps, out, final_state, (int)T, B, Nqk, Nv, 0,
                                          (cudaStream_t)stream));
 }
 
@@ -306,7 +306,7 @@ int gdn_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
     const float sc = resolve_scale(scale);
     if (max_seqlen >= 1 && max_seqlen <= GDN_SHORT_MAX)
         return cuda_status(gdn::launch_short(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, sc, eps,
-                                             out, final_state, (int)T, B, Nqk, Nv, st));
+                                             out, final_state, (int)T, B, Nqk, Nv, max_seqlen, st));
 
     gdn_workspace_layout_t lay;
     if ((rc = fill_layout(T, B, Nqk, Nv, &lay))) return rc;

@@ -53,6 +53,6 @@ cudaError_t launch_output(const uint16_t *q, const uint16_t *k, const float *g, 
 cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                          const uint16_t *beta, const int32_t *cu, const float *pool, const int32_t *idx,
                          float scale, float eps, uint16_t *out, float *final_state, int T, int B, int Nqk,
-                         int Nv, cudaStream_t st);
+                         int Nv, int max_seqlen, cudaStream_t st);
 
 }  // namespace gdn

@@ -7,14 +7,20 @@
 // against a few hundred bytes of q/k/v per token, so the kernel is a stream:
 // each CTA issues the loads of its state slice (warp w holds Dk rows
 // 32w..32w+31, lane j holds column j, one 128-byte row segment per warp load)
-// together with cp.async copies of the token data of up to kPre tokens (q and
-// k rows, the v slice, g), so that a single memory latency covers both; it then
-// applies the tokens from registers and shared memory,
+// together with cp.async copies of the token data of up to PRE tokens (q and
+// k rows, the v slice, g), so that a single memory latency covers both.  The q
+// and k rows are then normalised as in "L2 Normalization" into fp32 rows in
+// shared memory (q with the scale), and the tokens are applied from registers,
 //   S = e^g S;  kv = S^T kh;  S += kh (beta (v - kv))^T;  o = S^T qh,
-// with q and k normalised as in "L2 Normalization" and the cross-warp sums over
-// Dk going through shared memory, and writes the final slice from registers.
-// Tokens past kPre are read directly from global memory, so the kernel is exact
-// for any sequence length; it is only fast for short ones.
+// with the sums over Dk taken per warp and then across the four warps through
+// shared memory (two barriers per token, the partial sums double-buffered by
+// token parity), and the per-element work in packed fp32 pairs.  The final slice
+// is written from registers.  Tokens past PRE are read directly from global
+// memory, so the kernel is exact for any sequence length; it is only fast for
+// short ones.  PRE is 8 when every sequence is known to have at most 8 tokens,
+// else 16: the staging area then stays small enough for eight CTAs per SM (the
+// register file holds eight state slices), where 16 staged tokens leave room for
+// seven.
 #include "common.cuh"
 #include "gdn_internal.h"
 
@@ -22,29 +28,31 @@ namespace gdn {
 
 constexpr int kShortThreads = 128;
 constexpr int kTile = 32;  // Dv columns per CTA
-constexpr int kPre = 16;   // tokens staged together with the state
 
+template <int PRE>  // tokens staged together with the state
 struct ShortSmem {
-    uint16_t q[kPre][D], k[kPre][D];  // raw bf16 rows
-    uint16_t v[kPre][kTile];          // raw bf16 slice
-    float g[kPre], beta[kPre], rq[kPre], rk[kPre];
-    float red[4][32], red2[4][32];
+    float kh[PRE][D], qh[PRE][D];   // normalised rows, fp32 (qh includes the scale)
+    uint16_t q[PRE][D], k[PRE][D];  // raw bf16 rows
+    uint16_t v[PRE][kTile];         // raw bf16 slice
+    float g[PRE], dg[PRE], beta[PRE];
+    float red[2][4][32], red2[2][4][32];
 };
 
+template <int PRE>
 __global__ void __launch_bounds__(kShortThreads) short_kernel(
     const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, const uint16_t *__restrict__ v,
     const float *__restrict__ g, const uint16_t *__restrict__ beta, const int32_t *__restrict__ cu,
     const float *__restrict__ pool, const int32_t *__restrict__ idx, float scale, float eps,
     uint16_t *__restrict__ out, float *__restrict__ final_state, int T, int Nqk, int Nv)
 {
-    __shared__ __align__(16) ShortSmem sm;
+    __shared__ __align__(16) ShortSmem<PRE> sm;
     const int b = blockIdx.x, h = blockIdx.y, tl = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int col = tl * kTile + lane;
     const int hq = h / (Nv / Nqk);
     const int t0 = min(max(cu[b], 0), T);
     const int t1 = min(max(cu[b + 1], t0), T);
-    const int n = t1 - t0, npre = min(n, kPre);
+    const int n = t1 - t0, npre = min(n, PRE);
 
     // token data of the first kPre tokens: async copies
     for (int e = tid; e < npre * 16; e += kShortThreads) {
@@ -62,115 +70,145 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
     float bt_mine = 0.f;
     if (tid < npre) bt_mine = bf2f(beta[(size_t)(t0 + tid) * Nv + h]);
 
-    // the state slice, straight into registers
-    float s[32];
+    // the state slice, straight into registers: s2[m] holds rows 32 wid + 2m, 2m + 1
+    float2 s2[16];
     if (pool) {
         const int slot = idx ? idx[b] : b;
         const float *src = pool + (((size_t)slot * Nv + h) * D + wid * 32) * D + col;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[i] = __ldcs(src + (size_t)i * D);
+        for (int m = 0; m < 16; ++m) s2[m] = make_float2(__ldcs(src + (size_t)(2 * m) * D), __ldcs(src + (size_t)(2 * m + 1) * D));
     } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[i] = 0.f;
+        for (int m = 0; m < 16; ++m) s2[m] = make_float2(0.f, 0.f);
     }
 
     cp_async_wait<0>();
     if (tid < npre) sm.beta[tid] = bt_mine;
     __syncthreads();
-    // norms of the staged q and k rows: one warp per token
+    // normalised q and k rows in fp32 and the decay of every staged token: one warp per token,
+    // lane l at elements 4l .. 4l + 3
     for (int t = wid; t < npre; t += kShortThreads / 32) {
         const uint2 qa = *reinterpret_cast<const uint2 *>(&sm.q[t][lane * 4]);
         const uint2 ka = *reinterpret_cast<const uint2 *>(&sm.k[t][lane * 4]);
-        const uint32_t qw[2] = {qa.x, qa.y}, kw[2] = {ka.x, ka.y};
+        const float q4[4] = {__uint_as_float(qa.x << 16), __uint_as_float(qa.x & 0xffff0000u),
+                             __uint_as_float(qa.y << 16), __uint_as_float(qa.y & 0xffff0000u)};
+        const float k4[4] = {__uint_as_float(ka.x << 16), __uint_as_float(ka.x & 0xffff0000u),
+                             __uint_as_float(ka.y << 16), __uint_as_float(ka.y & 0xffff0000u)};
         float sq = 0.f, sk = 0.f;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const float q0 = __uint_as_float(qw[e] << 16), q1 = __uint_as_float(qw[e] & 0xffff0000u);
-            const float k0 = __uint_as_float(kw[e] << 16), k1 = __uint_as_float(kw[e] & 0xffff0000u);
-            sq += q0 * q0 + q1 * q1;
-            sk += k0 * k0 + k1 * k1;
+        for (int e = 0; e < 4; ++e) {
+            sq = fmaf(q4[e], q4[e], sq);
+            sk = fmaf(k4[e], k4[e], sk);
         }
         sq = warp_sum(sq);
         sk = warp_sum(sk);
-        if (lane == 0) {
-            sm.rq[t] = scale / sqrtf(sq + eps);
-            sm.rk[t] = 1.0f / sqrtf(sk + eps);
-        }
+        const float rq = scale / sqrtf(sq + eps), rk = 1.0f / sqrtf(sk + eps);
+        *reinterpret_cast<float4 *>(&sm.qh[t][lane * 4]) = make_float4(q4[0] * rq, q4[1] * rq, q4[2] * rq, q4[3] * rq);
+        *reinterpret_cast<float4 *>(&sm.kh[t][lane * 4]) = make_float4(k4[0] * rk, k4[1] * rk, k4[2] * rk, k4[3] * rk);
+        if (lane == 0) sm.dg[t] = __expf(sm.g[t]);
     }
+    __syncthreads();
 
-    for (int j = 0; j < n; ++j) {
-        // this warp's 32 rows of the token's k and q (raw bf16) and the token's scalars
-        const uint16_t *kr, *qr;
-        float vj, gt, bt, rks, rqs;
-        if (j < kPre) {
-            __syncthreads();  // norms (first token) / previous token's reductions are complete
-            kr = &sm.k[j][wid * 32];
-            qr = &sm.q[j][wid * 32];
-            vj = bf2f(sm.v[j][lane]);
-            gt = sm.g[j];
-            bt = sm.beta[j];
-            rks = sm.rk[j];
-            rqs = sm.rq[j];
-        } else {  // beyond the staged tokens: read directly
-            const int t = t0 + j;
-            const uint16_t *qrow = q + ((size_t)t * Nqk + hq) * D, *krow = k + ((size_t)t * Nqk + hq) * D;
-            float sq = 0.f, sk = 0.f;
+    for (int j = 0; j < npre; ++j) {
+        const int p = j & 1;
+        const float4 *kr = reinterpret_cast<const float4 *>(&sm.kh[j][wid * 32]);
+        const float4 *qr = reinterpret_cast<const float4 *>(&sm.qh[j][wid * 32]);
+        const float dg = sm.dg[j], bt = sm.beta[j], vj = bf2f(sm.v[j][lane]);
+        // this warp's part of S^T kh (the decay is applied to the sum)
+        float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float a = bf2f(qrow[lane + 32 * i]), c = bf2f(krow[lane + 32 * i]);
-                sq += a * a;
-                sk += c * c;
-            }
-            sq = warp_sum(sq);
-            sk = warp_sum(sk);
-            rqs = scale / sqrtf(sq + eps);
-            rks = 1.0f / sqrtf(sk + eps);
-            kr = krow + wid * 32;
-            qr = qrow + wid * 32;
-            vj = bf2f(v[((size_t)t * Nv + h) * D + col]);
-            gt = g[(size_t)t * Nv + h];
-            bt = bf2f(beta[(size_t)t * Nv + h]);
-            __syncthreads();  // previous token's reductions are complete
+        for (int c = 0; c < 8; ++c) {
+            const float4 kx = kr[c];
+            a0 = ffma2(s2[2 * c], make_float2(kx.x, kx.y), a0);
+            a1 = ffma2(s2[2 * c + 1], make_float2(kx.z, kx.w), a1);
         }
-        const float dg = __expf(gt);
-        float acc = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            s[i] *= dg;
-            acc += s[i] * bf2f(kr[i]);
-        }
-        sm.red[wid][lane] = acc;
+        sm.red[p][wid][lane] = (a0.x + a0.y) + (a1.x + a1.y);
         __syncthreads();
-        const float u = bt * (vj - rks * (sm.red[0][lane] + sm.red[1][lane] + sm.red[2][lane] + sm.red[3][lane]));
-        const float ku = u * rks;
-        float acc2 = 0.f;
+        const float kv = dg * ((sm.red[p][0][lane] + sm.red[p][1][lane]) + (sm.red[p][2][lane] + sm.red[p][3][lane]));
+        const float u = bt * (vj - kv);
+        const float2 dg2 = make_float2(dg, dg), u2 = make_float2(u, u);
+        // S = e^g S + kh u^T, then this warp's part of S^T qh
+        float2 b0 = make_float2(0.f, 0.f), b1 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            s[i] += bf2f(kr[i]) * ku;
-            acc2 += s[i] * bf2f(qr[i]);
+        for (int c = 0; c < 8; ++c) {
+            const float4 kx = kr[c], qx = qr[c];
+            s2[2 * c] = ffma2(make_float2(kx.x, kx.y), u2, fmul2(s2[2 * c], dg2));
+            s2[2 * c + 1] = ffma2(make_float2(kx.z, kx.w), u2, fmul2(s2[2 * c + 1], dg2));
+            b0 = ffma2(s2[2 * c], make_float2(qx.x, qx.y), b0);
+            b1 = ffma2(s2[2 * c + 1], make_float2(qx.z, qx.w), b1);
         }
-        sm.red2[wid][lane] = acc2;
+        sm.red2[p][wid][lane] = (b0.x + b0.y) + (b1.x + b1.y);
         __syncthreads();
         if (wid == 0)
             out[((size_t)(t0 + j) * Nv + h) * D + col] =
-                f2bf(rqs * (sm.red2[0][lane] + sm.red2[1][lane] + sm.red2[2][lane] + sm.red2[3][lane]));
+                f2bf((sm.red2[p][0][lane] + sm.red2[p][1][lane]) + (sm.red2[p][2][lane] + sm.red2[p][3][lane]));
+    }
+
+    // beyond the staged tokens (longer sequences than the fused path is meant for): read directly
+    for (int j = PRE; j < n; ++j) {
+        const int t = t0 + j, p = j & 1;
+        const uint16_t *qrow = q + ((size_t)t * Nqk + hq) * D, *krow = k + ((size_t)t * Nqk + hq) * D;
+        float sq = 0.f, sk = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float a = bf2f(qrow[lane + 32 * i]), c = bf2f(krow[lane + 32 * i]);
+            sq = fmaf(a, a, sq);
+            sk = fmaf(c, c, sk);
+        }
+        sq = warp_sum(sq);
+        sk = warp_sum(sk);
+        const float rq = scale / sqrtf(sq + eps), rk = 1.0f / sqrtf(sk + eps);
+        const float vj = bf2f(v[((size_t)t * Nv + h) * D + col]);
+        const float dg = __expf(g[(size_t)t * Nv + h]), bt = bf2f(beta[(size_t)t * Nv + h]);
+        const uint16_t *kr = krow + wid * 32, *qr = qrow + wid * 32;
+        float acc = 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            acc = fmaf(s2[m].x, bf2f(kr[2 * m]) * rk, acc);
+            acc = fmaf(s2[m].y, bf2f(kr[2 * m + 1]) * rk, acc);
+        }
+        sm.red[p][wid][lane] = acc;
+        __syncthreads();
+        const float kv = dg * ((sm.red[p][0][lane] + sm.red[p][1][lane]) + (sm.red[p][2][lane] + sm.red[p][3][lane]));
+        const float u = bt * (vj - kv);
+        float acc2 = 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            s2[m].x = fmaf(bf2f(kr[2 * m]) * rk, u, s2[m].x * dg);
+            s2[m].y = fmaf(bf2f(kr[2 * m + 1]) * rk, u, s2[m].y * dg);
+            acc2 = fmaf(s2[m].x, bf2f(qr[2 * m]) * rq, acc2);
+            acc2 = fmaf(s2[m].y, bf2f(qr[2 * m + 1]) * rq, acc2);
+        }
+        sm.red2[p][wid][lane] = acc2;
+        __syncthreads();
+        if (wid == 0)
+            out[((size_t)t * Nv + h) * D + col] =
+                f2bf((sm.red2[p][0][lane] + sm.red2[p][1][lane]) + (sm.red2[p][2][lane] + sm.red2[p][3][lane]));
     }
 
     if (final_state) {
         float *dst = final_state + (((size_t)b * Nv + h) * D + wid * 32) * D + col;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) __stcs(dst + (size_t)i * D, s[i]);
+        for (int m = 0; m < 16; ++m) {
+            __stcs(dst + (size_t)(2 * m) * D, s2[m].x);
+            __stcs(dst + (size_t)(2 * m + 1) * D, s2[m].y);
+        }
     }
 }
 
 cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                          const uint16_t *beta, const int32_t *cu, const float *pool, const int32_t *idx,
                          float scale, float eps, uint16_t *out, float *final_state, int T, int B, int Nqk,
-                         int Nv, cudaStream_t st)
+                         int Nv, int max_seqlen, cudaStream_t st)
 {
     if (B == 0) return cudaSuccess;
-    short_kernel<<<dim3(B, Nv, D / kTile), kShortThreads, 0, st>>>(q, k, v, g, beta, cu, pool, idx, scale, eps, out,
-                                                                    final_state, T, Nqk, Nv);
+    const dim3 grid(B, Nv, D / kTile);
+    if (max_seqlen >= 1 && max_seqlen <= 8)
+        short_kernel<8><<<grid, kShortThreads, 0, st>>>(q, k, v, g, beta, cu, pool, idx, scale, eps, out, final_state,
+                                                        T, Nqk, Nv);
+    else
+        short_kernel<16><<<grid, kShortThreads, 0, st>>>(q, k, v, g, beta, cu, pool, idx, scale, eps, out,
+                                                         final_state, T, Nqk, Nv);
     return cudaGetLastError();
 }
 

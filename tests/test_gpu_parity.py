@@ -63,6 +63,17 @@ def test_short_pool_b256_both_paths():
         assert_close(fin, rf, f"short max_seqlen={ms} final_state")
 
 
+def test_short_path_staging_depths():
+    """Sequences of 9..16 tokens from a pool: the fused kernel stages 16 tokens when max_seqlen says 16,
+    8 when it says 8 (an understated bound: the tokens past the eighth are read directly)."""
+    inp = inputs.make([9, 16, 1, 12, 8, 15], Nqk=2, Nv=4, state=("normal", 0.02, 8, "perm"), seed=23)
+    ro, rf = run_oracle(inp)
+    for ms in (16, 8):
+        out, fin = _gpu(inp, max_seqlen=ms)
+        assert_close(out, ro, f"short staging max_seqlen={ms} out")
+        assert_close(fin, rf, f"short staging max_seqlen={ms} final_state")
+
+
 def test_short_path_without_pool_two_heads():
     """Fused short kernel with a zero initial state, empty sequences and Nv = 2 (g, beta rows of 8 and 4 bytes)."""
     inp = inputs.make([5, 1, 8, 0, 3, 16, 0], Nqk=1, Nv=2, seed=21)
