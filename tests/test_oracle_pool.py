@@ -1,0 +1,141 @@
+"""Pins of the per-token-slot pool oracle (``oracle.pool.recurrent_pool``) to the
+independent C token recurrence (CPU only).
+
+The pool oracle restates the decode page's token loop in numpy with the slot
+semantics of "lite_boost.ops.recurrent_gated_delta_rule" (``ssm_state_indices``
+per token, ``num_accepted_tokens``, the updated pool ``state_out``).  It is
+checked against ``oracle.recurrent`` (C, pinned in test_oracle_pins.py) on the
+three cases that fix the semantics:
+
+* one slot per sequence, every token accepted: the plain recurrence with the
+  final state written back into that slot, every other slot untouched;
+* a distinct slot per token: slot j holds the recurrence's state after token j
+  (a prefix run of the C oracle);
+* ``num_accepted = a``: the sequence starts from the slot of its token a - 1.
+
+Planted mistakes in a copy of the pool oracle's source must each fail a pin.
+"""
+from __future__ import annotations
+
+import importlib.util
+import os
+import sys
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import pool as pool_oracle
+
+TOL = 1e-12
+POOL_SRC = os.path.join(os.path.dirname(os.path.abspath(oracle.__file__)), "pool.py")
+
+
+def _problem(seed, lens, Nqk=1, Nv=2, D=6, P=12):
+    r = np.random.default_rng(seed)
+    T = sum(lens)
+    return dict(q=r.standard_normal((T, Nqk, D)), k=r.standard_normal((T, Nqk, D)),
+                v=r.standard_normal((T, Nv, D)), g=-(r.random((T, Nv)) * 0.5 + 0.01),
+                beta=r.random((T, Nv)) * 0.9 + 0.05,
+                cu_seqlens=np.concatenate([[0], np.cumsum(lens)]).astype(np.int32),
+                state_pool=r.standard_normal((P, Nv, D, D)) * 0.3)
+
+
+def _close(a, b, what):
+    a, b = np.asarray(a), np.asarray(b)
+    err = float(np.max(np.abs(a - b))) if a.size else 0.0
+    scale = max(1.0, float(np.max(np.abs(b))) if b.size else 1.0)
+    assert err <= TOL * scale, f"{what}: max abs diff {err:.3e}"
+
+
+def _plain(p, lo, hi, init):
+    """C recurrence of tokens [lo, hi) of the problem as one sequence from state `init` [Nv, D, D]."""
+    sl = lambda x: x[lo:hi]
+    return oracle.recurrent(sl(p["q"]), sl(p["k"]), sl(p["v"]), sl(p["g"]), sl(p["beta"]),
+                            np.array([0, hi - lo], np.int32), state_pool=init[None])
+
+
+def pin_one_slot_per_sequence(fn):
+    lens = [3, 1, 5, 0, 2]
+    p = _problem(31, lens)
+    seq_slot = [7, 2, 10, 4, 0]
+    slots = np.concatenate([[s] * n for s, n in zip(seq_slot, lens)]).astype(np.int32)
+    out, pool = fn(**p, token_slots=slots)
+    ref_o, ref_f = oracle.recurrent(p["q"], p["k"], p["v"], p["g"], p["beta"], p["cu_seqlens"],
+                                    state_pool=p["state_pool"], state_indices=np.array(seq_slot, np.int32))
+    _close(out, ref_o, "one slot: out")
+    for b, (s, n) in enumerate(zip(seq_slot, lens)):
+        _close(pool[s], ref_f[b] if n else p["state_pool"][s], f"one slot: slot {s}")
+    untouched = [s for s in range(p["state_pool"].shape[0]) if s not in seq_slot]
+    _close(pool[untouched], p["state_pool"][untouched], "one slot: other slots")
+
+
+def pin_slot_per_token(fn):
+    lens = [4, 3]
+    p = _problem(32, lens)
+    slots = np.array([5, 9, 1, 3, 11, 6, 2], np.int32)
+    out, pool = fn(**p, token_slots=slots, num_accepted=np.array([2, 3], np.int32))
+    cu = p["cu_seqlens"]
+    for b in range(2):
+        t0, t1 = int(cu[b]), int(cu[b + 1])
+        init = p["state_pool"][slots[t0 + (2 if b == 0 else 3) - 1]]
+        ref_o, _ = _plain(p, t0, t1, init)
+        _close(out[t0:t1], ref_o, f"per token: out of sequence {b}")
+        for j in range(t1 - t0):
+            _, f = _plain(p, t0, t0 + j + 1, init)
+            _close(pool[slots[t0 + j]], f[0], f"per token: slot of token {t0 + j}")
+
+
+def pin_accepted_selects_start(fn):
+    lens = [5]
+    p = _problem(33, lens, Nv=1)
+    slots = np.array([0, 1, 2, 3, 4], np.int32)
+    for a in (1, 3, 5):
+        out, _ = fn(**p, token_slots=slots, num_accepted=np.array([a], np.int32))
+        ref_o, _ = _plain(p, 0, 5, p["state_pool"][a - 1])
+        _close(out, ref_o, f"accepted {a}: out")
+    # the start must matter
+    o1, _ = fn(**p, token_slots=slots, num_accepted=np.array([1], np.int32))
+    o5, _ = fn(**p, token_slots=slots, num_accepted=np.array([5], np.int32))
+    assert np.max(np.abs(o1 - o5)) > 1e-6
+
+
+PINS = [pin_one_slot_per_sequence, pin_slot_per_token, pin_accepted_selects_start]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
+def test_pool_oracle_pin(pin):
+    pin(pool_oracle.recurrent_pool)
+
+
+MUTANTS = [
+    ("start_from_first_token_slot", "starts.append(pool[slots[t0 + a - 1]].copy())",
+     "starts.append(pool[slots[t0]].copy())"),
+    ("start_from_last_token_slot", "starts.append(pool[slots[t0 + a - 1]].copy())",
+     "starts.append(pool[slots[t1 - 1]].copy())"),
+    ("write_to_sequence_start_slot", "pool_out[slots[t], h] = S", "pool_out[slots[t0], h] = S"),
+    ("no_decay", "S = S * math.exp(G[t, h])", "S = S"),
+    ("write_before_update", "                pool_out[slots[t], h] = S\n",
+     "                pool_out[slots[t], h] = starts[b][h]\n"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_pool_mistake_is_caught(name, old, new):
+    src = open(POOL_SRC).read()
+    assert src.count(old) == 1, name
+    spec = importlib.util.spec_from_loader(f"oracle._pool_mutant_{name}", loader=None)
+    mod = importlib.util.module_from_spec(spec)
+    mod.__dict__["__package__"] = "oracle"
+    sys.modules[spec.name] = mod
+    try:
+        exec(compile(src.replace(old, new), POOL_SRC, "exec"), mod.__dict__)
+        caught = 0
+        for pin in PINS:
+            try:
+                pin(mod.recurrent_pool)
+            except AssertionError:
+                caught += 1
+        assert caught >= 1, f"no pin fails for the planted mistake {name}"
+    finally:
+        del sys.modules[spec.name]
