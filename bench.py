@@ -14,6 +14,12 @@ i.e. per chunk and v-head: U = T (beta V), W = T (beta e^gamma K), W S, Q S,
 P U', K^T U'; per chunk and qk-head: K K^T and Q K^T.  The triangular solve
 and the masked halves are not counted.
 
+Two HBM-bound side workloads are timed in the same run (skipped with
+--no-short) and reported in the same line: ``short_seq`` (256 sequences of
+1..8 tokens from an fp32 state pool, gdn_chunk_fwd's fused short path) and
+``spec_decode`` (256 sequences of 4 draft tokens, a pool slot per token,
+gdn_recurrent_fwd updating the pool in place).
+
 Prints ONE JSON line (rank 0).  ``--impl reference`` times the fp64 CPU
 oracle (the reference arm) on a bounded sample of the same workload instead.
 """
@@ -363,6 +369,38 @@ def main():
                              "l2": "state traffic 1.07 GB per step > L2"}
         line["gpu_launches"] += args.steps
         del sh, so, sf
+
+        # speculative decoding on a pool updated in place (one slot per token; HBM-bound)
+        cfg = inputs.CONFIGS["spec_decode_b256x4"]
+        sp = inputs.config("spec_decode_b256x4", seed=cfg["seed"] + rank)
+        slots, acc = inputs.spec_slots(sp, seed=cfg["seed"] + 100 + rank)
+        sp, slots, acc = sp.to(dev), slots.to(dev), acc.to(dev)
+        spo = torch.empty(sp.T, sp.Nv, D, dtype=torch.bfloat16, device=dev)
+
+        def pstep():
+            gdn.recurrent_fwd(sp.q, sp.k, sp.v, sp.g, sp.beta, sp.cu_seqlens, sp.state_pool, slots,
+                              num_accepted=acc, scale=sp.scale, eps=sp.eps, max_seqlen=sp.max_seqlen, out=spo)
+        for _ in range(args.warmup):
+            pstep()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            pstep()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        pms = gdist.max_over_ranks(e0.elapsed_time(e1) / args.steps, device=dev)
+        sbytes = sp.Nv * D * D * 4
+        pb = sp.B * sbytes + sp.T * sbytes + (short_bytes(sp) - 2 * sp.B * sbytes)  # starts, per-token states, I/O
+        line["spec_decode"] = {"workload": f"spec_decode_b256x4: B={sp.B} x 4 draft tokens (T={sp.T}), Nqk={sp.Nqk}, "
+                                           f"Nv={sp.Nv}, a pool slot per token, accepted counts uniform 1..4, "
+                                           f"fp32 pool [{sp.state_pool.shape[0]},{sp.Nv},128,128] updated in place",
+                               "ms": pms, "bytes": pb, "GB/s": pb / (pms / 1e3) / 1e9,
+                               "hbm_frac": pb / (pms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                               "tokens/s": world * sp.T / (pms / 1e3), "kernel": "short_kernel (per-token slots)",
+                               "call": "gdn_recurrent_fwd"}
+        line["gpu_launches"] += args.steps
+        del sp, slots, acc, spo
 
     # ---- end to end from pinned host buffers through the public call
     if not args.no_e2e:

@@ -21,6 +21,16 @@
 // else 16: the staging area then stays small enough for eight CTAs per SM (the
 // register file holds eight state slices), where 16 staged tokens leave room for
 // seven.
+//
+// With SLOTS the pool is updated in place with one slot index per token (page
+// "lite_boost.ops.recurrent_gated_delta_rule": ssm_state_indices per token,
+// num_accepted_tokens, state_out): a sequence starts from the slot of its last
+// accepted token, slots[t0 + a - 1], and the state after token j is written to
+// slots[t0 + j] whenever the next token's slot differs or j is the last token
+// (a run of tokens on one slot keeps only its last state, so this writes every
+// slot's final value).  A CTA reads its slice of the starting slot before it
+// writes anything, and the slots of different sequences are disjoint, so the
+// in-place update is race-free.
 #include "common.cuh"
 #include "gdn_internal.h"
 
@@ -35,15 +45,17 @@ struct ShortSmem {
     uint16_t q[PRE][D], k[PRE][D];  // raw bf16 rows
     uint16_t v[PRE][kTile];         // raw bf16 slice
     float g[PRE], dg[PRE], beta[PRE];
+    int32_t slot[PRE + 1];  // token slots (SLOTS)
     float red[2][4][32], red2[2][4][32];
 };
 
-template <int PRE>
+template <int PRE, bool SLOTS>
 __global__ void __launch_bounds__(kShortThreads) short_kernel(
     const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, const uint16_t *__restrict__ v,
     const float *__restrict__ g, const uint16_t *__restrict__ beta, const int32_t *__restrict__ cu,
-    const float *__restrict__ pool, const int32_t *__restrict__ idx, float scale, float eps,
-    uint16_t *__restrict__ out, float *__restrict__ final_state, int T, int Nqk, int Nv)
+    const float *pool, const int32_t *__restrict__ idx, const int32_t *__restrict__ token_slots,
+    const int32_t *__restrict__ num_accepted, float *pool_w, float scale, float eps, uint16_t *__restrict__ out,
+    float *__restrict__ final_state, int T, int Nqk, int Nv)
 {
     __shared__ __align__(16) ShortSmem<PRE> sm;
     const int b = blockIdx.x, h = blockIdx.y, tl = blockIdx.z;
@@ -53,6 +65,7 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
     const int t0 = min(max(cu[b], 0), T);
     const int t1 = min(max(cu[b + 1], t0), T);
     const int n = t1 - t0, npre = min(n, PRE);
+    if (SLOTS && n == 0) return;  // no token: the pool keeps its slots
 
     // token data of the first kPre tokens: async copies
     for (int e = tid; e < npre * 16; e += kShortThreads) {
@@ -66,6 +79,7 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
         cp_async16(smem_addr(&sm.v[t][c * 8]), v + ((size_t)(t0 + t) * Nv + h) * D + tl * kTile + c * 8, true);
     }
     if (tid < npre) cp_async4(smem_addr(&sm.g[tid]), g + (size_t)(t0 + tid) * Nv + h);
+    if (SLOTS && tid <= PRE && tid < n) cp_async4(smem_addr(&sm.slot[tid]), token_slots + t0 + tid);
     cp_async_commit();
     float bt_mine = 0.f;
     if (tid < npre) bt_mine = bf2f(beta[(size_t)(t0 + tid) * Nv + h]);
@@ -73,7 +87,13 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
     // the state slice, straight into registers: s2[m] holds rows 32 wid + 2m, 2m + 1
     float2 s2[16];
     if (pool) {
-        const int slot = idx ? idx[b] : b;
+        int slot;
+        if (SLOTS) {  // the state after the last accepted token (n >= 1 here)
+            const int a = min(max(num_accepted ? num_accepted[b] : n, 1), n);
+            slot = token_slots[t0 + a - 1];
+        } else {
+            slot = idx ? idx[b] : b;
+        }
         const float *src = pool + (((size_t)slot * Nv + h) * D + wid * 32) * D + col;
 #pragma unroll
         for (int m = 0; m < 16; ++m) s2[m] = make_float2(__ldcs(src + (size_t)(2 * m) * D), __ldcs(src + (size_t)(2 * m + 1) * D));
@@ -81,6 +101,16 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
 #pragma unroll
         for (int m = 0; m < 16; ++m) s2[m] = make_float2(0.f, 0.f);
     }
+
+    // this thread's 32 values of the state into pool slot `slot` (SLOTS)
+    auto write_slot = [&](int slot) {
+        float *dst = pool_w + (((size_t)slot * Nv + h) * D + wid * 32) * D + col;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            __stcs(dst + (size_t)(2 * m) * D, s2[m].x);
+            __stcs(dst + (size_t)(2 * m + 1) * D, s2[m].y);
+        }
+    };
 
     cp_async_wait<0>();
     if (tid < npre) sm.beta[tid] = bt_mine;
@@ -138,6 +168,7 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
             b1 = ffma2(s2[2 * c + 1], make_float2(qx.z, qx.w), b1);
         }
         sm.red2[p][wid][lane] = (b0.x + b0.y) + (b1.x + b1.y);
+        if (SLOTS && (j == n - 1 || sm.slot[j + 1] != sm.slot[j])) write_slot(sm.slot[j]);
         __syncthreads();
         if (wid == 0)
             out[((size_t)(t0 + j) * Nv + h) * D + col] =
@@ -180,13 +211,17 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
             acc2 = fmaf(s2[m].y, bf2f(qr[2 * m + 1]) * rq, acc2);
         }
         sm.red2[p][wid][lane] = acc2;
+        if (SLOTS) {
+            const int sj = token_slots[t], sn = j + 1 < n ? token_slots[t + 1] : -1;
+            if (j == n - 1 || sn != sj) write_slot(sj);
+        }
         __syncthreads();
         if (wid == 0)
             out[((size_t)t * Nv + h) * D + col] =
                 f2bf((sm.red2[p][0][lane] + sm.red2[p][1][lane]) + (sm.red2[p][2][lane] + sm.red2[p][3][lane]));
     }
 
-    if (final_state) {
+    if (!SLOTS && final_state) {
         float *dst = final_state + (((size_t)b * Nv + h) * D + wid * 32) * D + col;
 #pragma unroll
         for (int m = 0; m < 16; ++m) {
@@ -198,17 +233,29 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
 
 cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                          const uint16_t *beta, const int32_t *cu, const float *pool, const int32_t *idx,
-                         float scale, float eps, uint16_t *out, float *final_state, int T, int B, int Nqk,
-                         int Nv, int max_seqlen, cudaStream_t st)
+                         const int32_t *token_slots, const int32_t *num_accepted, float *pool_w, float scale,
+                         float eps, uint16_t *out, float *final_state, int T, int B, int Nqk, int Nv, int max_seqlen,
+                         cudaStream_t st)
 {
     if (B == 0) return cudaSuccess;
     const dim3 grid(B, Nv, D / kTile);
-    if (max_seqlen >= 1 && max_seqlen <= 8)
-        short_kernel<8><<<grid, kShortThreads, 0, st>>>(q, k, v, g, beta, cu, pool, idx, scale, eps, out, final_state,
-                                                        T, Nqk, Nv);
-    else
-        short_kernel<16><<<grid, kShortThreads, 0, st>>>(q, k, v, g, beta, cu, pool, idx, scale, eps, out,
-                                                         final_state, T, Nqk, Nv);
+    const bool few = max_seqlen >= 1 && max_seqlen <= 8;
+    if (token_slots) {
+        if (few)
+            short_kernel<8, true><<<grid, kShortThreads, 0, st>>>(q, k, v, g, beta, cu, pool, idx, token_slots,
+                                                                   num_accepted, pool_w, scale, eps, out, final_state,
+                                                                   T, Nqk, Nv);
+        else
+            short_kernel<16, true><<<grid, kShortThreads, 0, st>>>(q, k, v, g, beta, cu, pool, idx, token_slots,
+                                                                    num_accepted, pool_w, scale, eps, out, final_state,
+                                                                    T, Nqk, Nv);
+    } else if (few) {
+        short_kernel<8, false><<<grid, kShortThreads, 0, st>>>(q, k, v, g, beta, cu, pool, idx, nullptr, nullptr,
+                                                                nullptr, scale, eps, out, final_state, T, Nqk, Nv);
+    } else {
+        short_kernel<16, false><<<grid, kShortThreads, 0, st>>>(q, k, v, g, beta, cu, pool, idx, nullptr, nullptr,
+                                                                 nullptr, scale, eps, out, final_state, T, Nqk, Nv);
+    }
     return cudaGetLastError();
 }
 

@@ -90,7 +90,25 @@ CONFIGS = {
     # two 128K-token sequences with initial states
     "long_s128k_b2": dict(lens=[131072, 131072], Nqk=16, Nv=32, g=("softplus", 0.05),
                           beta=("sigmoid",), state=("normal", 0.02, None, "identity"), seed=4),
+    # speculative decoding: 256 sequences of 4 draft tokens, a pool slot per token (see spec_slots)
+    "spec_decode_b256x4": dict(lens=[4] * 256, Nqk=16, Nv=32, g=("uniform_neg", 1.0, 0.01),
+                               beta=("uniform", 0.05, 0.95), state=("normal", 0.02, 1024, "perm"), seed=5),
 }
+
+
+def spec_slots(inp: GdnInputs, seed: int):
+    """Token slots and accepted counts for a speculative step: every token gets its own pool slot
+    (a random permutation of the pool's first T slots) and sequence b accepts a uniform 1..n_b of
+    its tokens.  Returns (token_slots int32 [T], num_accepted int32 [B]) on the CPU."""
+    gen = torch.Generator().manual_seed(seed)
+    T, B = inp.T, inp.B
+    P = inp.state_pool.shape[0]
+    if P < T:
+        raise ValueError("the pool needs a slot per token")
+    slots = torch.randperm(P, generator=gen)[:T].to(torch.int32)
+    n = (inp.cu_seqlens[1:] - inp.cu_seqlens[:-1]).to(torch.int64)
+    acc = (torch.floor(torch.rand(B, generator=gen) * n.clamp(min=1)).to(torch.int64) + 1).clamp(max=n.clamp(min=1))
+    return slots, acc.to(torch.int32)
 
 
 def _draw_lens(spec, gen):

@@ -153,6 +153,58 @@ int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *
                           float *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
                           int32_t max_seqlen, void *stream);
 
+/*
+ * gdn_recurrent_fwd -- token recurrence on a state pool updated in place, with
+ * one slot index per token (decode and speculative decoding).
+ *
+ * Page "lite_boost.ops.recurrent_gated_delta_rule": per token, in this order,
+ * S = S * exp(g); kv_mem = S^T k; S = S + k ((v - kv_mem) * beta)^T; o = S^T q,
+ * with q and k L2-normalised here (eps inside the square root) and q scaled
+ * after the normalisation; every token selects a slot of the state pool through
+ * its own index (ssm_state_indices), num_accepted_tokens marks how many tokens
+ * of a speculative step were accepted, and the updated pool is the result
+ * (state_out).  Where the page leaves the slot use open, this call takes:
+ *   - sequence b (tokens t0 = cu[b] .. t1 - 1, n = t1 - t0 >= 1) starts from
+ *     state_pool[token_slots[t0 + a - 1]], a = num_accepted[b] clamped to
+ *     1 .. n (a = n when num_accepted is NULL): the state after its last
+ *     accepted token;
+ *   - after token t the state is written to state_pool[token_slots[t]]; a run
+ *     of consecutive tokens on one slot writes only its last state, so every
+ *     slot ends holding the state after its sequence's last token on it;
+ *   - a sequence with no tokens reads and writes nothing.
+ * Ordinary decoding puts all tokens of sequence b on one slot (its state is
+ * then read from and written back to that slot).
+ *
+ *   q, k, v, g, beta, cu_seqlens   as for gdn_chunk_fwd
+ *   state_pool    device fp32 [P, Nv, 128 (Dk), 128 (Dv)], read and written in
+ *                 place (required)
+ *   token_slots   device int32 [T], each in [0, P) (not checked on the device);
+ *                 the slots used by different sequences, including each
+ *                 sequence's starting slot, must be disjoint
+ *   num_accepted  device int32 [B], or NULL
+ *   scale, eps    as for gdn_chunk_fwd
+ *   out           device bf16 [T, Nv, 128], written for every token; must not
+ *                 overlap any input or state_pool
+ *   T, B, Nqk, Nv, P   sizes (T = cu[B]); Nv % Nqk == 0; P >= 1
+ *   max_seqlen    longest sequence if known, else 0.  At most 8 selects the
+ *                 kernel variant that stages 8 tokens per sequence (eight CTAs
+ *                 per SM); any other value the one that stages 16.  Every
+ *                 length is exact; tokens past the staged ones are read from
+ *                 global memory one at a time (slower).
+ *
+ * Alignment: q, k, v, out, state_pool 16-byte aligned; g, cu_seqlens,
+ * token_slots, num_accepted 4-byte aligned; beta 2-byte aligned.  Errors:
+ * GDN_ERR_NULL_ARG, GDN_ERR_BAD_SHAPE, GDN_ERR_UNSUPPORTED, GDN_ERR_ALIGNMENT,
+ * GDN_ERR_OVERLAP before anything is enqueued; GDN_ERR_CUDA when the launch
+ * fails.  B == 0 or T == 0 is a no-op.  Asynchronous on `stream`; the library
+ * keeps no pointer after the call returns.
+ */
+int gdn_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                      const uint16_t *beta, const int32_t *cu_seqlens, float *state_pool,
+                      const int32_t *token_slots, const int32_t *num_accepted, float scale, float eps,
+                      uint16_t *out, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
+                      int32_t max_seqlen, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,108 @@
+"""GPU parity of gdn_recurrent_fwd (token recurrence on a pool updated in place,
+one slot per token) against the fp64 pool oracle.
+
+Tolerances as for the forward pass (relative L2 <= 1e-2, max-abs <= 2e-2 RMS,
+see helpers.assert_close); slots that no token writes must come back bit-exact.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import gated_deltanet_linear_17_b200 as gdn
+from gated_deltanet_linear_17_b200 import inputs
+from oracle.pool import recurrent_pool
+
+from helpers import assert_close
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _case(lens, Nqk, Nv, P, seed, per_token, accepted):
+    """Inputs, token slots [T] and accepted counts [B] (None: every token accepted)."""
+    inp = inputs.make(lens, Nqk=Nqk, Nv=Nv, state=("normal", 0.02, P, "perm"), seed=seed)
+    r = np.random.default_rng(seed + 1000)
+    cu = inp.cu_seqlens.numpy()
+    T, B = int(cu[-1]), len(lens)
+    if per_token:  # a distinct slot for every token
+        slots = r.permutation(P)[:T].astype(np.int32)
+    else:  # every token of sequence b on the sequence's slot
+        seq_slot = r.permutation(P)[:B]
+        slots = np.concatenate([np.full(n, seq_slot[b]) for b, n in enumerate(lens)] + [np.zeros(0)]).astype(np.int32)
+    acc = None
+    if accepted:
+        acc = np.array([r.integers(1, n + 1) if n > 0 else 0 for n in lens], np.int32)
+    return inp, slots, acc
+
+
+def _run_and_check(inp, slots, acc, max_seqlen, what):
+    ro, rpool = recurrent_pool(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, inp.state_pool, slots,
+                               num_accepted=acc, scale=inp.scale, eps=inp.eps)
+    d = inp.to(DEV)
+    pool = d.state_pool.clone()
+    ts = torch.from_numpy(slots).to(DEV)
+    na = None if acc is None else torch.from_numpy(acc).to(DEV)
+    out = gdn.recurrent_fwd(d.q, d.k, d.v, d.g, d.beta, d.cu_seqlens, pool, ts, num_accepted=na, scale=d.scale,
+                            eps=d.eps, max_seqlen=max_seqlen)
+    torch.cuda.synchronize()
+    assert_close(out, ro, f"{what} out")
+    written = np.unique(slots)
+    assert_close(pool[torch.from_numpy(written).to(DEV).long()], rpool[written], f"{what} written slots")
+    others = np.setdiff1d(np.arange(pool.shape[0]), written)
+    if others.size:
+        idx = torch.from_numpy(others).to(DEV).long()
+        assert torch.equal(pool[idx], d.state_pool[idx]), f"{what}: a slot no token names was changed"
+
+
+@pytest.mark.parametrize("max_seqlen", [4, 0])
+def test_recurrent_decode_one_slot_per_sequence(max_seqlen):
+    """Ordinary decoding: all tokens of a sequence on its slot, read and written back in place."""
+    r = np.random.default_rng(40)
+    lens = [int(x) for x in r.integers(1, 5, size=48)]
+    inp, slots, acc = _case(lens, Nqk=4, Nv=8, P=64, seed=41, per_token=False, accepted=False)
+    _run_and_check(inp, slots, acc, max_seqlen, f"decode max_seqlen={max_seqlen}")
+
+
+@pytest.mark.parametrize("max_seqlen", [5, 16])
+def test_recurrent_speculative_slot_per_token(max_seqlen):
+    """Speculative decoding: a slot per token, each sequence starting from its last accepted token's slot."""
+    r = np.random.default_rng(42)
+    lens = [int(x) for x in r.integers(1, 6, size=40)]
+    inp, slots, acc = _case(lens, Nqk=2, Nv=4, P=224, seed=43, per_token=True, accepted=True)
+    _run_and_check(inp, slots, acc, max_seqlen, f"speculative max_seqlen={max_seqlen}")
+
+
+@pytest.mark.parametrize("max_seqlen", [0, 8, 24])
+def test_recurrent_long_and_empty_sequences(max_seqlen):
+    """Sequences past the staged tokens (read directly), empty ones (nothing read or written)."""
+    lens = [0, 20, 3, 0, 17, 9]
+    inp, slots, acc = _case(lens, Nqk=1, Nv=2, P=64, seed=44, per_token=True, accepted=True)
+    _run_and_check(inp, slots, acc, max_seqlen, f"long/empty max_seqlen={max_seqlen}")
+
+
+def test_recurrent_runs_of_slots():
+    """Runs of tokens sharing a slot inside a sequence (A A B B B C): each slot keeps its run's last state."""
+    lens = [6, 4]
+    inp, _, _ = _case(lens, Nqk=1, Nv=2, P=16, seed=45, per_token=False, accepted=False)
+    slots = np.array([3, 3, 7, 7, 7, 1, 9, 9, 12, 12], np.int32)
+    acc = np.array([6, 2], np.int32)
+    _run_and_check(inp, slots, acc, 8, "runs of slots")
+
+
+def test_recurrent_matches_chunk_fwd_final_state():
+    """One slot per sequence equals the short path of gdn_chunk_fwd with its final states."""
+    lens = [3, 1, 8, 5]
+    inp, slots, _ = _case(lens, Nqk=2, Nv=4, P=8, seed=46, per_token=False, accepted=False)
+    d = inp.to(DEV)
+    cu = inp.cu_seqlens.numpy()
+    seq_slot = torch.tensor([int(slots[cu[b]]) for b in range(len(lens))], dtype=torch.int32, device=DEV)
+    out_c, fin_c = gdn.chunk_fwd(d.q, d.k, d.v, d.g, d.beta, d.cu_seqlens, d.state_pool, seq_slot, scale=d.scale,
+                                 eps=d.eps, max_seqlen=8)
+    pool = d.state_pool.clone()
+    out_r = gdn.recurrent_fwd(d.q, d.k, d.v, d.g, d.beta, d.cu_seqlens, pool, torch.from_numpy(slots).to(DEV),
+                              scale=d.scale, eps=d.eps, max_seqlen=8)
+    torch.cuda.synchronize()
+    assert torch.equal(out_r, out_c)
+    assert torch.equal(pool[seq_slot.long()], fin_c)
