@@ -19,11 +19,13 @@ and after each token j of the sequence the state is written to pool[slots[t0 + j
 (later writes to a slot supersede earlier ones).  Every initial state is read
 before any write of the call.  Per token, in the page's order:
 
-    S = S * exp(g);  kv_mem = S^T k;  S = S + k ((v - kv_mem) * beta)^T;  o = S^T q
+    S = S * exp(g) * exp(gk);  kv_mem = S^T k;  S = S + k ((v - kv_mem) * beta)^T;  o = S^T q
 
 with q and k normalised as in "Qwen3Next Samples", equation "L2 Normalization"
-(eps inside the square root) and q scaled after the normalisation.  Plain
-numpy, per token, for the small shapes of the tests.
+(eps inside the square root) and q scaled after the normalisation.  gk, when
+given, is the page's key-dimension gate: exp(gk) decays each key row of S (S is
+[Dk, Dv]) by its own factor; without gk that factor is 1.  Plain numpy, per
+token, for the small shapes of the tests.
 """
 from __future__ import annotations
 
@@ -41,16 +43,18 @@ def _ints(x) -> np.ndarray:
 
 
 def recurrent_pool(q, k, v, g, beta, cu_seqlens, state_pool, token_slots, num_accepted=None, scale=None,
-                   eps=1e-6):
+                   eps=1e-6, gk=None):
     """Token recurrence with per-token pool slots, in fp64.
 
     Shapes: q, k [T, Nqk, Dk]; v [T, Nv, Dv]; g, beta [T, Nv]; cu_seqlens [B+1];
-    state_pool [P, Nv, Dk, Dv]; token_slots [T]; num_accepted [B] or None.
+    state_pool [P, Nv, Dk, Dv]; token_slots [T]; num_accepted [B] or None;
+    gk [T, Nv, Dk] or None.
     Returns (out [T, Nv, Dv], pool_out [P, Nv, Dk, Dv]) as float64; pool_out is a
     copy of state_pool with the written slots replaced.
     """
     Q, K, V = as_numpy_exact(q), as_numpy_exact(k), as_numpy_exact(v)
     G, Bt = as_numpy_exact(g), as_numpy_exact(beta)
+    GK = None if gk is None else as_numpy_exact(gk)
     pool = as_numpy_exact(state_pool)
     cu, slots = _ints(cu_seqlens), _ints(token_slots)
     acc = None if num_accepted is None else _ints(num_accepted)
@@ -84,6 +88,8 @@ def recurrent_pool(q, k, v, g, beta, cu_seqlens, state_pool, token_slots, num_ac
                 kh = K[t, hq] / math.sqrt(float(np.dot(K[t, hq], K[t, hq])) + eps)
                 qh = scale * Q[t, hq] / math.sqrt(float(np.dot(Q[t, hq], Q[t, hq])) + eps)
                 S = S * math.exp(G[t, h])
+                if GK is not None:
+                    S = S * np.exp(GK[t, h])[:, None]  # row i of S (key dimension i)
                 kv_mem = S.T @ kh
                 S = S + np.outer(kh, (V[t, h] - kv_mem) * Bt[t, h])
                 out[t, h] = S.T @ qh

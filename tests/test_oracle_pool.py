@@ -100,7 +100,52 @@ def pin_accepted_selects_start(fn):
     assert np.max(np.abs(o1 - o5)) > 1e-6
 
 
-PINS = [pin_one_slot_per_sequence, pin_slot_per_token, pin_accepted_selects_start]
+def pin_key_gate_zero(fn):
+    """gk = 0 is the recurrence without a key gate."""
+    lens = [3, 4]
+    p = _problem(34, lens)
+    slots = np.array([0, 0, 0, 5, 5, 5, 5], np.int32)
+    o1, p1 = fn(**p, token_slots=slots)
+    o2, p2 = fn(**p, token_slots=slots, gk=np.zeros(p["k"].shape[:1] + (2, 6)))
+    _close(o2, o1, "gk = 0: out")
+    _close(p2, p1, "gk = 0: pool")
+
+
+def pin_key_gate_constant(fn):
+    """A gk equal to c in every key dimension is the recurrence with g + c (C oracle)."""
+    lens = [5]
+    p = _problem(35, lens)
+    slots = np.zeros(5, np.int32)
+    c = -0.3
+    out, pool = fn(**p, token_slots=slots, gk=np.full((5, 2, 6), c))
+    shifted = dict(p)
+    shifted["g"] = p["g"] + c
+    ref_o, ref_f = _plain(shifted, 0, 5, p["state_pool"][0])
+    _close(out, ref_o, "gk = c: out")
+    _close(pool[0], ref_f[0], "gk = c: state")
+
+
+def pin_key_gate_rows_closed_form(fn):
+    """beta = 0: S_t = diag(exp(sum (g + gk))) S_0 row by row, o_t = S_t^T qh (Dk = 3, Dv = 5)."""
+    r = np.random.default_rng(36)
+    T, Dk, Dv = 4, 3, 5
+    q, k = r.standard_normal((T, 1, Dk)), r.standard_normal((T, 1, Dk))
+    v = r.standard_normal((T, 1, Dv))
+    g = -(r.random((T, 1)) * 0.5 + 0.01)
+    gk = -(r.random((T, 1, Dk)) * 0.7 + 0.01)
+    S0 = r.standard_normal((1, 1, Dk, Dv))
+    out, pool = fn(q, k, v, g, np.zeros((T, 1)), np.array([0, T], np.int32), S0, np.zeros(T, np.int32), gk=gk)
+    scale = 1.0 / np.sqrt(Dk)
+    for t in range(T):
+        rows = np.exp(np.cumsum(g[:t + 1, 0])[-1] + np.cumsum(gk[:t + 1, 0], axis=0)[-1])
+        St = rows[:, None] * S0[0, 0]
+        qh = scale * q[t, 0] / np.sqrt(np.dot(q[t, 0], q[t, 0]) + 1e-6)
+        _close(out[t, 0], St.T @ qh, f"closed form: out {t}")
+    _close(pool[0, 0], St, "closed form: state")
+
+
+PINS = [pin_one_slot_per_sequence, pin_slot_per_token, pin_accepted_selects_start, pin_key_gate_zero,
+        pin_key_gate_constant, pin_key_gate_rows_closed_form]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -117,6 +162,9 @@ MUTANTS = [
     ("no_decay", "S = S * math.exp(G[t, h])", "S = S"),
     ("write_before_update", "                pool_out[slots[t], h] = S\n",
      "                pool_out[slots[t], h] = starts[b][h]\n"),
+    ("key_gate_on_columns", "S = S * np.exp(GK[t, h])[:, None]", "S = S * np.exp(GK[t, h])[:S.shape[1]][None, :]"),
+    ("key_gate_sign", "S = S * np.exp(GK[t, h])[:, None]", "S = S * np.exp(-GK[t, h])[:, None]"),
+    ("key_gate_ignored", "S = S * np.exp(GK[t, h])[:, None]", "S = S"),
 ]
 
 
@@ -134,7 +182,7 @@ def test_planted_pool_mistake_is_caught(name, old, new):
         for pin in PINS:
             try:
                 pin(mod.recurrent_pool)
-            except AssertionError:
+            except Exception:  # a wrong value or a shape the mistake cannot handle
                 caught += 1
         assert caught >= 1, f"no pin fails for the planted mistake {name}"
     finally:
