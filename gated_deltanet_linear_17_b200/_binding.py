@@ -59,7 +59,8 @@ def lib():
         L.gdn_short_fwd.restype = ctypes.c_int
         L.gdn_short_fwd.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, p]
         L.gdn_recurrent_fwd.restype = ctypes.c_int
-        L.gdn_recurrent_fwd.argtypes = [p, p, p, p, p, p, p, p, p, f32, f32, p, i64, i32, i32, i32, i32, i32, p]
+        L.gdn_recurrent_fwd.argtypes = [p, p, p, p, p, p, p, p, i32, p, p, f32, f32, p, i64, i32, i32, i32, i32, i32,
+                                        p]
         L.gdn_stage_chunk_map.restype = ctypes.c_int
         L.gdn_stage_chunk_map.argtypes = [p, i64, i32, i32, i32, p, sz, p]
         L.gdn_stage_intra.restype = ctypes.c_int
@@ -221,24 +222,32 @@ def short_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None,
 
 
 def recurrent_fwd(q, k, v, g, beta, cu_seqlens, state_pool, token_slots, num_accepted=None, scale=None, eps=1e-6,
-                  max_seqlen: int = 0, out=None, stream=None):
+                  gk=None, max_seqlen: int = 0, out=None, stream=None):
     """Token recurrence with the pool updated in place, one slot per token (``gdn_recurrent_fwd``).
 
-    ``token_slots`` [T] int32 gives each token's slot; sequence b starts from the slot of its
-    token ``num_accepted[b] - 1`` (its last token when ``num_accepted`` is None).  Returns ``out``;
-    ``state_pool`` holds the updated states afterwards."""
+    ``state_pool`` [P, Nv, 128, 128] fp32 or bf16; ``token_slots`` [T] int32 gives each token's
+    slot; sequence b starts from the slot of its token ``num_accepted[b] - 1`` (its last token when
+    ``num_accepted`` is None); ``gk`` [T, Nv, 128] fp32 is the optional key-dimension gate.
+    Returns ``out``; ``state_pool`` holds the updated states afterwards."""
     if state_pool is None or token_slots is None:
         raise ValueError("recurrent_fwd needs a state pool and a slot per token")
-    T, B, Nqk, Nv, P, dev = _resolve(q, k, v, g, beta, cu_seqlens, state_pool, None)
+    if state_pool.dtype not in (torch.float32, torch.bfloat16):
+        raise RuntimeError(f"state_pool must be float32 or bfloat16 (got {state_pool.dtype})")
+    bf16_pool = state_pool.dtype == torch.bfloat16
+    T, B, Nqk, Nv, P, dev = _resolve(q, k, v, g, beta, cu_seqlens, None, None)
+    P = state_pool.shape[0]
+    _need(state_pool, "state_pool", state_pool.dtype, (P, Nv, HEAD_DIM, HEAD_DIM), dev)
     _need(token_slots, "token_slots", torch.int32, (T,), dev)
     if num_accepted is not None:
         _need(num_accepted, "num_accepted", torch.int32, (B,), dev)
+    if gk is not None:
+        _need(gk, "gk", torch.float32, (T, Nv, HEAD_DIM), dev)
     if out is None:
         out = torch.empty(T, Nv, HEAD_DIM, dtype=torch.bfloat16, device=dev)
     sc = 0.0 if scale is None else float(scale)
-    rc = lib().gdn_recurrent_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), _ptr(state_pool),
-                                 _ptr(token_slots), _ptr(num_accepted), sc, float(eps), _ptr(out), T, B, Nqk, Nv, P,
-                                 int(max_seqlen), _stream(stream))
+    rc = lib().gdn_recurrent_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(gk), _ptr(cu_seqlens),
+                                 _ptr(state_pool), int(bf16_pool), _ptr(token_slots), _ptr(num_accepted), sc,
+                                 float(eps), _ptr(out), T, B, Nqk, Nv, P, int(max_seqlen), _stream(stream))
     _check(rc, "gdn_recurrent_fwd")
     return out
 

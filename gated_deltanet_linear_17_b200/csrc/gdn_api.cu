@@ -288,29 +288,33 @@ int gdn_short_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
     int rc = check_forward(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, out, final_state, T, B,
                            Nqk, Nv, P);
     if (rc || B == 0) return rc;
-    return cuda_status(gdn::launch_short(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, nullptr,
-                                         nullptr, nullptr, resolve_scale(scale), eps, out, final_state, (int)T, B,
-                                         Nqk, Nv, 0, (cudaStream_t)stream));
+    return cuda_status(gdn::launch_short(q, k, v, g, beta, cu_seqlens, state_pool, state_indices,
+                                         resolve_scale(scale), eps, out, final_state, (int)T, B, Nqk, Nv, 0,
+                                         (cudaStream_t)stream));
 }
 
 int gdn_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
-                      const uint16_t *beta, const int32_t *cu_seqlens, float *state_pool,
-                      const int32_t *token_slots, const int32_t *num_accepted, float scale, float eps,
-                      uint16_t *out, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
+                      const uint16_t *beta, const float *gk, const int32_t *cu_seqlens, void *state_pool,
+                      int32_t state_bf16, const int32_t *token_slots, const int32_t *num_accepted, float scale,
+                      float eps, uint16_t *out, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
                       int32_t max_seqlen, void *stream)
 {
-    int rc = check_forward(q, k, v, g, beta, cu_seqlens, state_pool, nullptr, out, nullptr, T, B, Nqk, Nv, P);
+    int rc = check_forward(q, k, v, g, beta, cu_seqlens, static_cast<const float *>(state_pool), nullptr, out,
+                           nullptr, T, B, Nqk, Nv, P);
     if (rc || B == 0) return rc;
     if (!state_pool || (T > 0 && !token_slots)) return GDN_ERR_NULL_ARG;
-    if (P <= 0) return GDN_ERR_BAD_SHAPE;
-    if ((reinterpret_cast<uintptr_t>(token_slots) & 3u) || (reinterpret_cast<uintptr_t>(num_accepted) & 3u))
+    if (P <= 0 || (state_bf16 != 0 && state_bf16 != 1)) return GDN_ERR_BAD_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(token_slots) & 3u) || (reinterpret_cast<uintptr_t>(num_accepted) & 3u) ||
+        !aligned16(gk))
         return GDN_ERR_ALIGNMENT;
     const size_t obytes = (size_t)T * Nv * gdn::D * 2;
-    if (overlap(out, obytes, state_pool, (size_t)gdn::D * gdn::D * 4 * Nv * P)) return GDN_ERR_OVERLAP;
+    const size_t pbytes = (size_t)gdn::D * gdn::D * (state_bf16 ? 2 : 4) * Nv * P;
+    if (overlap(out, obytes, state_pool, pbytes) || overlap(out, obytes, gk, (size_t)T * Nv * gdn::D * 4))
+        return GDN_ERR_OVERLAP;
     if (T == 0) return GDN_OK;
-    return cuda_status(gdn::launch_short(q, k, v, g, beta, cu_seqlens, state_pool, nullptr, token_slots,
-                                         num_accepted, state_pool, resolve_scale(scale), eps, out, nullptr, (int)T,
-                                         B, Nqk, Nv, max_seqlen, (cudaStream_t)stream));
+    return cuda_status(gdn::launch_recurrent(q, k, v, g, beta, gk, cu_seqlens, state_pool, state_bf16 != 0,
+                                             token_slots, num_accepted, resolve_scale(scale), eps, out, (int)T, B, Nqk,
+                                             Nv, max_seqlen, (cudaStream_t)stream));
 }
 
 int gdn_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
@@ -325,9 +329,8 @@ int gdn_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
     const cudaStream_t st = (cudaStream_t)stream;
     const float sc = resolve_scale(scale);
     if (max_seqlen >= 1 && max_seqlen <= GDN_SHORT_MAX)
-        return cuda_status(gdn::launch_short(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, nullptr,
-                                             nullptr, nullptr, sc, eps, out, final_state, (int)T, B, Nqk, Nv,
-                                             max_seqlen, st));
+        return cuda_status(gdn::launch_short(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, sc, eps,
+                                             out, final_state, (int)T, B, Nqk, Nv, max_seqlen, st));
 
     gdn_workspace_layout_t lay;
     if ((rc = fill_layout(T, B, Nqk, Nv, &lay))) return rc;

@@ -50,14 +50,17 @@ cudaError_t launch_state(const uint16_t *k, const float *pool, const int32_t *id
                          int Nqk, int Nv, int c_lo, int c_hi, int range, const Workspace &ws, cudaStream_t st);
 cudaError_t launch_output(const uint16_t *q, const uint16_t *k, const float *g, float scale, float eps, uint16_t *out,
                           int T, int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st);
-// Fused short-sequence kernel.  token_slots == nullptr: sequence b starts from
-// pool[idx ? idx[b] : b] (or zero without a pool) and ends in final_state[b].
-// token_slots != nullptr: the pool (pool == pool_w) is updated in place, one slot
-// index per token, the start taken from the last accepted token's slot.
+// Fused short-sequence kernel: sequence b starts from pool[idx ? idx[b] : b] (or
+// zero without a pool) and ends in final_state[b].
 cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
-                         const uint16_t *beta, const int32_t *cu, const float *pool, const int32_t *idx,
-                         const int32_t *token_slots, const int32_t *num_accepted, float *pool_w, float scale,
+                         const uint16_t *beta, const int32_t *cu, const float *pool, const int32_t *idx, float scale,
                          float eps, uint16_t *out, float *final_state, int T, int B, int Nqk, int Nv, int max_seqlen,
                          cudaStream_t st);
+// The same kernel on a pool updated in place (fp32, or bf16 when bf16_pool), one slot per token,
+// the start taken from the last accepted token's slot; gk [T, Nv, 128] or nullptr.
+cudaError_t launch_recurrent(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                             const uint16_t *beta, const float *gk, const int32_t *cu, void *pool, bool bf16_pool,
+                             const int32_t *token_slots, const int32_t *num_accepted, float scale, float eps,
+                             uint16_t *out, int T, int B, int Nqk, int Nv, int max_seqlen, cudaStream_t st);
 
 }  // namespace gdn

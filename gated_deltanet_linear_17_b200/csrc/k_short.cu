@@ -30,7 +30,12 @@
 // (a run of tokens on one slot keeps only its last state, so this writes every
 // slot's final value).  A CTA reads its slice of the starting slot before it
 // writes anything, and the slots of different sequences are disjoint, so the
-// in-place update is race-free.
+// in-place update is race-free.  Two more options of that page's operator: a
+// bf16 state pool (SBF: the state is widened to fp32 on load and rounded to bf16
+// when written) and the key-dimension gate gk (GK: S = S e^g e^gk, row i of S
+// decayed by e^{g + gk_i}; the 128 factors of each staged token are computed once
+// per CTA into shared memory, and the state rows are decayed before the sum
+// S^T kh).
 #include "common.cuh"
 #include "gdn_internal.h"
 
@@ -39,9 +44,10 @@ namespace gdn {
 constexpr int kShortThreads = 128;
 constexpr int kTile = 32;  // Dv columns per CTA
 
-template <int PRE>  // tokens staged together with the state
+template <int PRE, bool GK>  // tokens staged together with the state; key gate
 struct ShortSmem {
     float kh[PRE][D], qh[PRE][D];   // normalised rows, fp32 (qh includes the scale)
+    float gkd[GK ? PRE : 1][D];     // gk rows, then the row decays e^{g + gk} (GK)
     uint16_t q[PRE][D], k[PRE][D];  // raw bf16 rows
     uint16_t v[PRE][kTile];         // raw bf16 slice
     float g[PRE], dg[PRE], beta[PRE];
@@ -49,15 +55,15 @@ struct ShortSmem {
     float red[2][4][32], red2[2][4][32];
 };
 
-template <int PRE, bool SLOTS>
+template <int PRE, bool SLOTS, bool GK, bool SBF>
 __global__ void __launch_bounds__(kShortThreads) short_kernel(
     const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, const uint16_t *__restrict__ v,
-    const float *__restrict__ g, const uint16_t *__restrict__ beta, const int32_t *__restrict__ cu,
-    const float *pool, const int32_t *__restrict__ idx, const int32_t *__restrict__ token_slots,
-    const int32_t *__restrict__ num_accepted, float *pool_w, float scale, float eps, uint16_t *__restrict__ out,
-    float *__restrict__ final_state, int T, int Nqk, int Nv)
+    const float *__restrict__ g, const uint16_t *__restrict__ beta, const float *__restrict__ gk,
+    const int32_t *__restrict__ cu, const void *pool, const int32_t *__restrict__ idx,
+    const int32_t *__restrict__ token_slots, const int32_t *__restrict__ num_accepted, void *pool_w, float scale,
+    float eps, uint16_t *__restrict__ out, float *__restrict__ final_state, int T, int Nqk, int Nv)
 {
-    __shared__ __align__(16) ShortSmem<PRE> sm;
+    __shared__ __align__(16) ShortSmem<PRE, GK> sm;
     const int b = blockIdx.x, h = blockIdx.y, tl = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int col = tl * kTile + lane;
@@ -80,6 +86,12 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
     }
     if (tid < npre) cp_async4(smem_addr(&sm.g[tid]), g + (size_t)(t0 + tid) * Nv + h);
     if (SLOTS && tid <= PRE && tid < n) cp_async4(smem_addr(&sm.slot[tid]), token_slots + t0 + tid);
+    if (GK) {
+        for (int e = tid; e < npre * 32; e += kShortThreads) {
+            const int t = e >> 5, c = e & 31;
+            cp_async16(smem_addr(&sm.gkd[t][c * 4]), gk + ((size_t)(t0 + t) * Nv + h) * D + c * 4, true);
+        }
+    }
     cp_async_commit();
     float bt_mine = 0.f;
     if (tid < npre) bt_mine = bf2f(beta[(size_t)(t0 + tid) * Nv + h]);
@@ -94,9 +106,18 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
         } else {
             slot = idx ? idx[b] : b;
         }
-        const float *src = pool + (((size_t)slot * Nv + h) * D + wid * 32) * D + col;
+        const size_t off = (((size_t)slot * Nv + h) * D + wid * 32) * D + col;
+        if (SBF) {
+            const unsigned short *src = static_cast<const unsigned short *>(pool) + off;
 #pragma unroll
-        for (int m = 0; m < 16; ++m) s2[m] = make_float2(__ldcs(src + (size_t)(2 * m) * D), __ldcs(src + (size_t)(2 * m + 1) * D));
+            for (int m = 0; m < 16; ++m)
+                s2[m] = make_float2(bf2f(__ldcs(src + (size_t)(2 * m) * D)), bf2f(__ldcs(src + (size_t)(2 * m + 1) * D)));
+        } else {
+            const float *src = static_cast<const float *>(pool) + off;
+#pragma unroll
+            for (int m = 0; m < 16; ++m)
+                s2[m] = make_float2(__ldcs(src + (size_t)(2 * m) * D), __ldcs(src + (size_t)(2 * m + 1) * D));
+        }
     } else {
 #pragma unroll
         for (int m = 0; m < 16; ++m) s2[m] = make_float2(0.f, 0.f);
@@ -104,11 +125,21 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
 
     // this thread's 32 values of the state into pool slot `slot` (SLOTS)
     auto write_slot = [&](int slot) {
-        float *dst = pool_w + (((size_t)slot * Nv + h) * D + wid * 32) * D + col;
+        const size_t off = (((size_t)slot * Nv + h) * D + wid * 32) * D + col;
+        if (SBF) {
+            unsigned short *dst = static_cast<unsigned short *>(pool_w) + off;
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            __stcs(dst + (size_t)(2 * m) * D, s2[m].x);
-            __stcs(dst + (size_t)(2 * m + 1) * D, s2[m].y);
+            for (int m = 0; m < 16; ++m) {
+                __stcs(dst + (size_t)(2 * m) * D, (unsigned short)f2bf(s2[m].x));
+                __stcs(dst + (size_t)(2 * m + 1) * D, (unsigned short)f2bf(s2[m].y));
+            }
+        } else {
+            float *dst = static_cast<float *>(pool_w) + off;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                __stcs(dst + (size_t)(2 * m) * D, s2[m].x);
+                __stcs(dst + (size_t)(2 * m + 1) * D, s2[m].y);
+            }
         }
     };
 
@@ -137,14 +168,31 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
         *reinterpret_cast<float4 *>(&sm.kh[t][lane * 4]) = make_float4(k4[0] * rk, k4[1] * rk, k4[2] * rk, k4[3] * rk);
         if (lane == 0) sm.dg[t] = __expf(sm.g[t]);
     }
+    if (GK) {  // the row decays e^{g + gk_i} of every staged token, in place over gk
+        for (int e = tid; e < npre * D; e += kShortThreads) {
+            const int t = e >> 7, i = e & (D - 1);
+            sm.gkd[t][i] = __expf(sm.g[t] + sm.gkd[t][i]);
+        }
+    }
     __syncthreads();
 
     for (int j = 0; j < npre; ++j) {
         const int p = j & 1;
         const float4 *kr = reinterpret_cast<const float4 *>(&sm.kh[j][wid * 32]);
         const float4 *qr = reinterpret_cast<const float4 *>(&sm.qh[j][wid * 32]);
-        const float dg = sm.dg[j], bt = sm.beta[j], vj = bf2f(sm.v[j][lane]);
-        // this warp's part of S^T kh (the decay is applied to the sum)
+        // the decay as one factor (applied to the sum S^T kh and in the update), or per row (GK: applied
+        // to the state rows first)
+        const float dg = GK ? 1.f : sm.dg[j], bt = sm.beta[j], vj = bf2f(sm.v[j][lane]);
+        if (GK) {
+            const float4 *dr = reinterpret_cast<const float4 *>(&sm.gkd[j][wid * 32]);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float4 d4 = dr[c];
+                s2[2 * c] = fmul2(s2[2 * c], make_float2(d4.x, d4.y));
+                s2[2 * c + 1] = fmul2(s2[2 * c + 1], make_float2(d4.z, d4.w));
+            }
+        }
+        // this warp's part of S^T kh
         float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -157,13 +205,18 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
         const float kv = dg * ((sm.red[p][0][lane] + sm.red[p][1][lane]) + (sm.red[p][2][lane] + sm.red[p][3][lane]));
         const float u = bt * (vj - kv);
         const float2 dg2 = make_float2(dg, dg), u2 = make_float2(u, u);
-        // S = e^g S + kh u^T, then this warp's part of S^T qh
+        // S = e^g S + kh u^T (GK: S already decayed), then this warp's part of S^T qh
         float2 b0 = make_float2(0.f, 0.f), b1 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const float4 kx = kr[c], qx = qr[c];
-            s2[2 * c] = ffma2(make_float2(kx.x, kx.y), u2, fmul2(s2[2 * c], dg2));
-            s2[2 * c + 1] = ffma2(make_float2(kx.z, kx.w), u2, fmul2(s2[2 * c + 1], dg2));
+            if (GK) {
+                s2[2 * c] = ffma2(make_float2(kx.x, kx.y), u2, s2[2 * c]);
+                s2[2 * c + 1] = ffma2(make_float2(kx.z, kx.w), u2, s2[2 * c + 1]);
+            } else {
+                s2[2 * c] = ffma2(make_float2(kx.x, kx.y), u2, fmul2(s2[2 * c], dg2));
+                s2[2 * c + 1] = ffma2(make_float2(kx.z, kx.w), u2, fmul2(s2[2 * c + 1], dg2));
+            }
             b0 = ffma2(s2[2 * c], make_float2(qx.x, qx.y), b0);
             b1 = ffma2(s2[2 * c + 1], make_float2(qx.z, qx.w), b1);
         }
@@ -190,7 +243,16 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
         sk = warp_sum(sk);
         const float rq = scale / sqrtf(sq + eps), rk = 1.0f / sqrtf(sk + eps);
         const float vj = bf2f(v[((size_t)t * Nv + h) * D + col]);
-        const float dg = __expf(g[(size_t)t * Nv + h]), bt = bf2f(beta[(size_t)t * Nv + h]);
+        const float gt = g[(size_t)t * Nv + h], bt = bf2f(beta[(size_t)t * Nv + h]);
+        const float dg = GK ? 1.f : __expf(gt);
+        if (GK) {  // this thread's 32 rows decayed by e^{g + gk_i}
+            const float *gr = gk + ((size_t)t * Nv + h) * D + wid * 32;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                s2[m].x *= __expf(gt + gr[2 * m]);
+                s2[m].y *= __expf(gt + gr[2 * m + 1]);
+            }
+        }
         const uint16_t *kr = krow + wid * 32, *qr = qrow + wid * 32;
         float acc = 0.f;
 #pragma unroll
@@ -231,31 +293,66 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
     }
 }
 
+template <int PRE, bool SLOTS, bool GK, bool SBF>
+static void launch_variant(dim3 grid, cudaStream_t st, const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                           const float *g, const uint16_t *beta, const float *gk, const int32_t *cu, const void *pool,
+                           const int32_t *idx, const int32_t *token_slots, const int32_t *num_accepted, void *pool_w,
+                           float scale, float eps, uint16_t *out, float *final_state, int T, int Nqk, int Nv)
+{
+    short_kernel<PRE, SLOTS, GK, SBF><<<grid, kShortThreads, 0, st>>>(q, k, v, g, beta, gk, cu, pool, idx, token_slots,
+                                                                      num_accepted, pool_w, scale, eps, out,
+                                                                      final_state, T, Nqk, Nv);
+}
+
+template <int PRE>
+static void launch_slots(bool has_gk, bool bf16_pool, dim3 grid, cudaStream_t st, const uint16_t *q,
+                         const uint16_t *k, const uint16_t *v, const float *g, const uint16_t *beta, const float *gk,
+                         const int32_t *cu, const void *pool, const int32_t *token_slots, const int32_t *num_accepted,
+                         void *pool_w, float scale, float eps, uint16_t *out, int T, int Nqk, int Nv)
+{
+    if (has_gk && bf16_pool)
+        launch_variant<PRE, true, true, true>(grid, st, q, k, v, g, beta, gk, cu, pool, nullptr, token_slots,
+                                              num_accepted, pool_w, scale, eps, out, nullptr, T, Nqk, Nv);
+    else if (has_gk)
+        launch_variant<PRE, true, true, false>(grid, st, q, k, v, g, beta, gk, cu, pool, nullptr, token_slots,
+                                               num_accepted, pool_w, scale, eps, out, nullptr, T, Nqk, Nv);
+    else if (bf16_pool)
+        launch_variant<PRE, true, false, true>(grid, st, q, k, v, g, beta, nullptr, cu, pool, nullptr, token_slots,
+                                               num_accepted, pool_w, scale, eps, out, nullptr, T, Nqk, Nv);
+    else
+        launch_variant<PRE, true, false, false>(grid, st, q, k, v, g, beta, nullptr, cu, pool, nullptr, token_slots,
+                                                num_accepted, pool_w, scale, eps, out, nullptr, T, Nqk, Nv);
+}
+
 cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
-                         const uint16_t *beta, const int32_t *cu, const float *pool, const int32_t *idx,
-                         const int32_t *token_slots, const int32_t *num_accepted, float *pool_w, float scale,
+                         const uint16_t *beta, const int32_t *cu, const float *pool, const int32_t *idx, float scale,
                          float eps, uint16_t *out, float *final_state, int T, int B, int Nqk, int Nv, int max_seqlen,
                          cudaStream_t st)
 {
     if (B == 0) return cudaSuccess;
     const dim3 grid(B, Nv, D / kTile);
-    const bool few = max_seqlen >= 1 && max_seqlen <= 8;
-    if (token_slots) {
-        if (few)
-            short_kernel<8, true><<<grid, kShortThreads, 0, st>>>(q, k, v, g, beta, cu, pool, idx, token_slots,
-                                                                   num_accepted, pool_w, scale, eps, out, final_state,
-                                                                   T, Nqk, Nv);
-        else
-            short_kernel<16, true><<<grid, kShortThreads, 0, st>>>(q, k, v, g, beta, cu, pool, idx, token_slots,
-                                                                    num_accepted, pool_w, scale, eps, out, final_state,
-                                                                    T, Nqk, Nv);
-    } else if (few) {
-        short_kernel<8, false><<<grid, kShortThreads, 0, st>>>(q, k, v, g, beta, cu, pool, idx, nullptr, nullptr,
-                                                                nullptr, scale, eps, out, final_state, T, Nqk, Nv);
-    } else {
-        short_kernel<16, false><<<grid, kShortThreads, 0, st>>>(q, k, v, g, beta, cu, pool, idx, nullptr, nullptr,
-                                                                 nullptr, scale, eps, out, final_state, T, Nqk, Nv);
-    }
+    if (max_seqlen >= 1 && max_seqlen <= 8)
+        launch_variant<8, false, false, false>(grid, st, q, k, v, g, beta, nullptr, cu, pool, idx, nullptr, nullptr,
+                                               nullptr, scale, eps, out, final_state, T, Nqk, Nv);
+    else
+        launch_variant<16, false, false, false>(grid, st, q, k, v, g, beta, nullptr, cu, pool, idx, nullptr, nullptr,
+                                                nullptr, scale, eps, out, final_state, T, Nqk, Nv);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_recurrent(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                             const uint16_t *beta, const float *gk, const int32_t *cu, void *pool, bool bf16_pool,
+                             const int32_t *token_slots, const int32_t *num_accepted, float scale, float eps,
+                             uint16_t *out, int T, int B, int Nqk, int Nv, int max_seqlen, cudaStream_t st)
+{
+    if (B == 0) return cudaSuccess;
+    const dim3 grid(B, Nv, D / kTile);
+    if (max_seqlen >= 1 && max_seqlen <= 8)
+        launch_slots<8>(gk != nullptr, bf16_pool, grid, st, q, k, v, g, beta, gk, cu, pool, token_slots, num_accepted,
+                        pool, scale, eps, out, T, Nqk, Nv);
+    else
+        launch_slots<16>(gk != nullptr, bf16_pool, grid, st, q, k, v, g, beta, gk, cu, pool, token_slots, num_accepted,
+                         pool, scale, eps, out, T, Nqk, Nv);
     return cudaGetLastError();
 }
 

@@ -90,6 +90,9 @@ CONFIGS = {
     # two 128K-token sequences with initial states
     "long_s128k_b2": dict(lens=[131072, 131072], Nqk=16, Nv=32, g=("softplus", 0.05),
                           beta=("sigmoid",), state=("normal", 0.02, None, "identity"), seed=4),
+    # decode step: 256 sequences of one token on a bf16 pool, with the key-dimension gate (key_gate)
+    "decode_b256_bf16": dict(lens=[1] * 256, Nqk=16, Nv=32, g=("uniform_neg", 1.0, 0.01),
+                             beta=("uniform", 0.05, 0.95), state=("normal", 0.02, 512, "perm"), seed=6),
     # speculative decoding: 256 sequences of 4 draft tokens, a pool slot per token (see spec_slots)
     "spec_decode_b256x4": dict(lens=[4] * 256, Nqk=16, Nv=32, g=("uniform_neg", 1.0, 0.01),
                                beta=("uniform", 0.05, 0.95), state=("normal", 0.02, 1024, "perm"), seed=5),
@@ -171,3 +174,10 @@ def config(name: str, device="cpu", seed: Optional[int] = None) -> GdnInputs:
     if seed is not None:
         rec["seed"] = seed
     return make(name=name, device=device, **rec)
+
+
+def key_gate(inp: GdnInputs, seed: int) -> torch.Tensor:
+    """The decode page's key-dimension gate for a batch: gk [T, Nv, 128] fp32 = -(U + 0.01) * 0.5
+    (the page's example draws -(U + 0.01); the factor keeps e^gk away from tiny values)."""
+    gen = torch.Generator().manual_seed(seed)
+    return -(torch.rand(inp.T, inp.Nv, D, generator=gen) + 0.01) * 0.5

@@ -158,7 +158,8 @@ int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *
  * one slot index per token (decode and speculative decoding).
  *
  * Page "lite_boost.ops.recurrent_gated_delta_rule": per token, in this order,
- * S = S * exp(g); kv_mem = S^T k; S = S + k ((v - kv_mem) * beta)^T; o = S^T q,
+ * S = S * exp(g) * exp(gk); kv_mem = S^T k; S = S + k ((v - kv_mem) * beta)^T;
+ * o = S^T q, where exp(gk) decays row i of S (key dimension i) by its own factor,
  * with q and k L2-normalised here (eps inside the square root) and q scaled
  * after the normalisation; every token selects a slot of the state pool through
  * its own index (ssm_state_indices), num_accepted_tokens marks how many tokens
@@ -176,8 +177,12 @@ int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *
  * then read from and written back to that slot).
  *
  *   q, k, v, g, beta, cu_seqlens   as for gdn_chunk_fwd
- *   state_pool    device fp32 [P, Nv, 128 (Dk), 128 (Dv)], read and written in
- *                 place (required)
+ *   gk            device fp32 [T, Nv, 128 (Dk)], the key-dimension gate
+ *                 (expected <= 0, not checked), or NULL for none
+ *   state_pool    device [P, Nv, 128 (Dk), 128 (Dv)], read and written in place
+ *                 (required): fp32 when state_bf16 == 0, bf16 when state_bf16 == 1
+ *                 (the page's pool dtype: widened to fp32 on load, the fp32 result
+ *                 rounded to nearest even when written)
  *   token_slots   device int32 [T], each in [0, P) (not checked on the device);
  *                 the slots used by different sequences, including each
  *                 sequence's starting slot, must be disjoint
@@ -192,17 +197,17 @@ int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *
  *                 length is exact; tokens past the staged ones are read from
  *                 global memory one at a time (slower).
  *
- * Alignment: q, k, v, out, state_pool 16-byte aligned; g, cu_seqlens,
+ * Alignment: q, k, v, out, state_pool, gk 16-byte aligned; g, cu_seqlens,
  * token_slots, num_accepted 4-byte aligned; beta 2-byte aligned.  Errors:
  * GDN_ERR_NULL_ARG, GDN_ERR_BAD_SHAPE, GDN_ERR_UNSUPPORTED, GDN_ERR_ALIGNMENT,
- * GDN_ERR_OVERLAP before anything is enqueued; GDN_ERR_CUDA when the launch
- * fails.  B == 0 or T == 0 is a no-op.  Asynchronous on `stream`; the library
+ * GDN_ERR_OVERLAP before anything is enqueued (state_bf16 other than 0 or 1 is
+ * GDN_ERR_BAD_SHAPE); GDN_ERR_CUDA when the launch fails.  B == 0 or T == 0 is a no-op.  Asynchronous on `stream`; the library
  * keeps no pointer after the call returns.
  */
 int gdn_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
-                      const uint16_t *beta, const int32_t *cu_seqlens, float *state_pool,
-                      const int32_t *token_slots, const int32_t *num_accepted, float scale, float eps,
-                      uint16_t *out, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
+                      const uint16_t *beta, const float *gk, const int32_t *cu_seqlens, void *state_pool,
+                      int32_t state_bf16, const int32_t *token_slots, const int32_t *num_accepted, float scale,
+                      float eps, uint16_t *out, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
                       int32_t max_seqlen, void *stream);
 
 #ifdef __cplusplus

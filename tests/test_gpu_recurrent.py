@@ -37,15 +37,21 @@ def _case(lens, Nqk, Nv, P, seed, per_token, accepted):
     return inp, slots, acc
 
 
-def _run_and_check(inp, slots, acc, max_seqlen, what):
-    ro, rpool = recurrent_pool(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, inp.state_pool, slots,
-                               num_accepted=acc, scale=inp.scale, eps=inp.eps)
+def _key_gate(inp, seed):
+    return inputs.key_gate(inp, seed)
+
+
+def _run_and_check(inp, slots, acc, max_seqlen, what, gk=None, bf16_pool=False):
+    pool0 = inp.state_pool.to(torch.bfloat16) if bf16_pool else inp.state_pool
+    ro, rpool = recurrent_pool(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, pool0, slots,
+                               num_accepted=acc, scale=inp.scale, eps=inp.eps, gk=gk)
     d = inp.to(DEV)
-    pool = d.state_pool.clone()
+    pool = pool0.to(DEV).clone()
+    start = pool.clone()
     ts = torch.from_numpy(slots).to(DEV)
     na = None if acc is None else torch.from_numpy(acc).to(DEV)
     out = gdn.recurrent_fwd(d.q, d.k, d.v, d.g, d.beta, d.cu_seqlens, pool, ts, num_accepted=na, scale=d.scale,
-                            eps=d.eps, max_seqlen=max_seqlen)
+                            eps=d.eps, gk=None if gk is None else gk.to(DEV), max_seqlen=max_seqlen)
     torch.cuda.synchronize()
     assert_close(out, ro, f"{what} out")
     written = np.unique(slots)
@@ -53,7 +59,7 @@ def _run_and_check(inp, slots, acc, max_seqlen, what):
     others = np.setdiff1d(np.arange(pool.shape[0]), written)
     if others.size:
         idx = torch.from_numpy(others).to(DEV).long()
-        assert torch.equal(pool[idx], d.state_pool[idx]), f"{what}: a slot no token names was changed"
+        assert torch.equal(pool[idx], start[idx]), f"{what}: a slot no token names was changed"
 
 
 @pytest.mark.parametrize("max_seqlen", [4, 0])
@@ -106,3 +112,40 @@ def test_recurrent_matches_chunk_fwd_final_state():
     torch.cuda.synchronize()
     assert torch.equal(out_r, out_c)
     assert torch.equal(pool[seq_slot.long()], fin_c)
+
+
+@pytest.mark.parametrize("max_seqlen", [4, 0])
+def test_recurrent_key_gate(max_seqlen):
+    """The decode page's key-dimension gate: each key row of S decays by e^{g + gk_i}."""
+    r = np.random.default_rng(47)
+    lens = [int(x) for x in r.integers(1, 5, size=32)]
+    inp, slots, acc = _case(lens, Nqk=4, Nv=8, P=48, seed=48, per_token=False, accepted=False)
+    _run_and_check(inp, slots, acc, max_seqlen, f"key gate max_seqlen={max_seqlen}", gk=_key_gate(inp, 49))
+
+
+@pytest.mark.parametrize("max_seqlen", [8, 16])
+def test_recurrent_bf16_pool(max_seqlen):
+    """A bf16 state pool: widened on load, the fp32 state rounded when written."""
+    r = np.random.default_rng(50)
+    lens = [int(x) for x in r.integers(1, 9, size=32)]
+    inp, slots, acc = _case(lens, Nqk=2, Nv=4, P=40, seed=51, per_token=False, accepted=False)
+    _run_and_check(inp, slots, acc, max_seqlen, f"bf16 pool max_seqlen={max_seqlen}", bf16_pool=True)
+
+
+def test_recurrent_decode_page_operator():
+    """Everything of the decode page at once: bf16 pool, key gate, a slot per token, accepted counts."""
+    r = np.random.default_rng(52)
+    lens = [int(x) for x in r.integers(1, 6, size=36)]
+    inp, slots, acc = _case(lens, Nqk=4, Nv=8, P=224, seed=53, per_token=True, accepted=True)
+    _run_and_check(inp, slots, acc, 5, "decode page operator", gk=_key_gate(inp, 54), bf16_pool=True)
+
+
+@pytest.mark.parametrize("max_seqlen", [0, 8])
+def test_recurrent_key_gate_past_staged_tokens(max_seqlen):
+    """Key gate on tokens read directly (past the staged ones), fp32 and bf16 pools."""
+    lens = [19, 2, 11]
+    inp, slots, acc = _case(lens, Nqk=1, Nv=2, P=40, seed=55, per_token=True, accepted=True)
+    gk = _key_gate(inp, 56)
+    _run_and_check(inp, slots, acc, max_seqlen, f"key gate, long, max_seqlen={max_seqlen}", gk=gk)
+    _run_and_check(inp, slots, acc, max_seqlen, f"key gate, long, bf16, max_seqlen={max_seqlen}", gk=gk,
+                   bf16_pool=True)
