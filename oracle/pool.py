@@ -26,6 +26,12 @@ with q and k normalised as in "Qwen3Next Samples", equation "L2 Normalization"
 given, is the page's key-dimension gate: exp(gk) decays each key row of S (S is
 [Dk, Dv]) by its own factor; without gk that factor is 1.  Plain numpy, per
 token, for the small shapes of the tests.
+
+``rule`` selects one of the four update rules of the page "com.microsoft.
+LinearAttention" (attribute update_rule): ``gated_delta`` (the rule above),
+``delta`` (no decay: the gates are not used), ``gated`` (S = S exp(g) exp(gk)
++ k v^T: no retrieval, beta not used) and ``linear`` (S = S + k v^T).  q and k
+are normalised in every rule, as this operator defines them.
 """
 from __future__ import annotations
 
@@ -42,8 +48,11 @@ def _ints(x) -> np.ndarray:
     return np.asarray(x, dtype=np.int64)
 
 
+RULES = ("gated_delta", "delta", "gated", "linear")
+
+
 def recurrent_pool(q, k, v, g, beta, cu_seqlens, state_pool, token_slots, num_accepted=None, scale=None,
-                   eps=1e-6, gk=None):
+                   eps=1e-6, gk=None, rule="gated_delta"):
     """Token recurrence with per-token pool slots, in fp64.
 
     Shapes: q, k [T, Nqk, Dk]; v [T, Nv, Dv]; g, beta [T, Nv]; cu_seqlens [B+1];
@@ -52,8 +61,12 @@ def recurrent_pool(q, k, v, g, beta, cu_seqlens, state_pool, token_slots, num_ac
     Returns (out [T, Nv, Dv], pool_out [P, Nv, Dk, Dv]) as float64; pool_out is a
     copy of state_pool with the written slots replaced.
     """
+    if rule not in RULES:
+        raise ValueError(f"unknown update rule {rule}")
+    decay, delta = rule in ("gated_delta", "gated"), rule in ("gated_delta", "delta")
     Q, K, V = as_numpy_exact(q), as_numpy_exact(k), as_numpy_exact(v)
-    G, Bt = as_numpy_exact(g), as_numpy_exact(beta)
+    G = as_numpy_exact(g) if decay else None
+    Bt = as_numpy_exact(beta) if delta else None
     GK = None if gk is None else as_numpy_exact(gk)
     pool = as_numpy_exact(state_pool)
     cu, slots = _ints(cu_seqlens), _ints(token_slots)
@@ -87,11 +100,15 @@ def recurrent_pool(q, k, v, g, beta, cu_seqlens, state_pool, token_slots, num_ac
             for t in range(t0, t1):
                 kh = K[t, hq] / math.sqrt(float(np.dot(K[t, hq], K[t, hq])) + eps)
                 qh = scale * Q[t, hq] / math.sqrt(float(np.dot(Q[t, hq], Q[t, hq])) + eps)
-                S = S * math.exp(G[t, h])
-                if GK is not None:
-                    S = S * np.exp(GK[t, h])[:, None]  # row i of S (key dimension i)
-                kv_mem = S.T @ kh
-                S = S + np.outer(kh, (V[t, h] - kv_mem) * Bt[t, h])
+                if decay:
+                    S = S * math.exp(G[t, h])
+                    if GK is not None:
+                        S = S * np.exp(GK[t, h])[:, None]  # row i of S (key dimension i)
+                if delta:
+                    kv_mem = S.T @ kh
+                    S = S + np.outer(kh, (V[t, h] - kv_mem) * Bt[t, h])
+                else:
+                    S = S + np.outer(kh, V[t, h])
                 out[t, h] = S.T @ qh
                 pool_out[slots[t], h] = S
     return out, pool_out

@@ -144,8 +144,63 @@ def pin_key_gate_rows_closed_form(fn):
     _close(pool[0, 0], St, "closed form: state")
 
 
+def _sum_closed_form(p, T, decay):
+    """The gated / linear rules summed out: S_t = D_t S_0 + sum_{j <= t} D_t D_j^-1 kh_j v_j^T, with
+    D_t = diag(exp(sum_{i <= t} (g_i + gk_i))) (identity for the linear rule); o_t = S_t^T qh_t."""
+    q, k, v, g, gk = p["q"][:, 0], p["k"][:, 0], p["v"][:, 0], p["g"][:, 0], p["gk"][:, 0]
+    S0 = p["state_pool"][0, 0]
+    cum = np.cumsum(g[:, None] + gk, axis=0) if decay else np.zeros_like(gk)
+    kh = k / np.sqrt(np.sum(k * k, axis=1, keepdims=True) + 1e-6)
+    qh = (q / np.sqrt(np.sum(q * q, axis=1, keepdims=True) + 1e-6)) / np.sqrt(q.shape[1])
+    outs, S = [], None
+    for t in range(T):
+        S = np.exp(cum[t])[:, None] * S0
+        for j in range(t + 1):
+            S = S + np.exp(cum[t] - cum[j])[:, None] * np.outer(kh[j], v[j])
+        outs.append(S.T @ qh[t])
+    return np.array(outs), S
+
+
+def _rule_problem(seed):
+    r = np.random.default_rng(seed)
+    T, Dk, Dv = 5, 3, 4
+    return dict(q=r.standard_normal((T, 1, Dk)), k=r.standard_normal((T, 1, Dk)), v=r.standard_normal((T, 1, Dv)),
+                g=-(r.random((T, 1)) * 0.5 + 0.01), beta=r.random((T, 1)) * 0.9 + 0.05,
+                cu_seqlens=np.array([0, T], np.int32), state_pool=r.standard_normal((1, 1, Dk, Dv)),
+                gk=-(r.random((T, 1, Dk)) * 0.4 + 0.01))
+
+
+def pin_rule_gated_closed_form(fn):
+    p = _rule_problem(37)
+    out, pool = fn(**p, token_slots=np.zeros(5, np.int32), rule="gated")
+    ro, rs = _sum_closed_form(p, 5, decay=True)
+    _close(out[:, 0], ro, "gated: out")
+    _close(pool[0, 0], rs, "gated: state")
+
+
+def pin_rule_linear_closed_form(fn):
+    p = _rule_problem(38)
+    out, pool = fn(**p, token_slots=np.zeros(5, np.int32), rule="linear")
+    ro, rs = _sum_closed_form(p, 5, decay=False)
+    _close(out[:, 0], ro, "linear: out")
+    _close(pool[0, 0], rs, "linear: state")
+
+
+def pin_rule_delta_is_zero_gate(fn):
+    """The delta rule is the C recurrence with g = 0 (the gates given are not used)."""
+    p = _problem(39, [6])
+    slots = np.zeros(6, np.int32)
+    out, pool = fn(**p, token_slots=slots, gk=np.full((6, 2, 6), -0.7), rule="delta")
+    zero = dict(p)
+    zero["g"] = np.zeros_like(p["g"])
+    ro, rf = _plain(zero, 0, 6, p["state_pool"][0])
+    _close(out, ro, "delta: out")
+    _close(pool[0], rf[0], "delta: state")
+
+
 PINS = [pin_one_slot_per_sequence, pin_slot_per_token, pin_accepted_selects_start, pin_key_gate_zero,
-        pin_key_gate_constant, pin_key_gate_rows_closed_form]
+        pin_key_gate_constant, pin_key_gate_rows_closed_form, pin_rule_gated_closed_form,
+        pin_rule_linear_closed_form, pin_rule_delta_is_zero_gate]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -165,6 +220,10 @@ MUTANTS = [
     ("key_gate_on_columns", "S = S * np.exp(GK[t, h])[:, None]", "S = S * np.exp(GK[t, h])[:S.shape[1]][None, :]"),
     ("key_gate_sign", "S = S * np.exp(GK[t, h])[:, None]", "S = S * np.exp(-GK[t, h])[:, None]"),
     ("key_gate_ignored", "S = S * np.exp(GK[t, h])[:, None]", "S = S"),
+    ("gated_rule_without_decay", 'decay, delta = rule in ("gated_delta", "gated")', 'decay, delta = rule in ("gated_delta",)'),
+    ("delta_rule_with_decay", 'decay, delta = rule in ("gated_delta", "gated")', 'decay, delta = rule in ("gated_delta", "gated", "delta")'),
+    ("linear_rule_uses_beta", "S = S + np.outer(kh, V[t, h])", "S = S + np.outer(kh, V[t, h] * 0.5)"),
+    ("rules_without_retrieval_retrieve", 'rule in ("gated_delta", "delta")\n', 'rule in ("gated_delta", "delta", "gated")\n'),
 ]
 
 
