@@ -400,6 +400,28 @@ def main():
                                "hbm_frac": pb / (pms / 1e3) / 1e9 / peaks["hbm_gbs"],
                                "tokens/s": world * sp.T / (pms / 1e3), "kernel": "short_kernel (per-token slots)",
                                "call": "gdn_recurrent_fwd"}
+        # the same workload under each update rule of the LinearAttention page (GB/s counts the same bytes)
+        rules = {}
+        for rule in ("gated_delta", "delta", "gated", "linear"):
+            decay, delta = rule in ("gated_delta", "gated"), rule in ("gated_delta", "delta")
+
+            def rstep():
+                gdn.recurrent_fwd(sp.q, sp.k, sp.v, sp.g if decay else None, sp.beta if delta else None,
+                                  sp.cu_seqlens, sp.state_pool, slots, num_accepted=acc, scale=sp.scale, eps=sp.eps,
+                                  update_rule=rule, max_seqlen=sp.max_seqlen, out=spo)
+            for _ in range(args.warmup):
+                rstep()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                rstep()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            rms_ = gdist.max_over_ranks(e0.elapsed_time(e1) / args.steps, device=dev)
+            rules[rule] = {"ms": rms_, "hbm_frac": pb / (rms_ / 1e3) / 1e9 / peaks["hbm_gbs"]}
+            line["gpu_launches"] += args.steps
+        line["spec_decode"]["update_rules"] = rules
         line["gpu_launches"] += args.steps
         del sp, slots, acc, spo
 

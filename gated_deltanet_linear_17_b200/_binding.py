@@ -59,8 +59,8 @@ def lib():
         L.gdn_short_fwd.restype = ctypes.c_int
         L.gdn_short_fwd.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, p]
         L.gdn_recurrent_fwd.restype = ctypes.c_int
-        L.gdn_recurrent_fwd.argtypes = [p, p, p, p, p, p, p, p, i32, p, p, f32, f32, p, i64, i32, i32, i32, i32, i32,
-                                        p]
+        L.gdn_recurrent_fwd.argtypes = [p, p, p, p, p, p, p, p, i32, i32, p, p, f32, f32, p, i64, i32, i32, i32, i32,
+                                        i32, p]
         L.gdn_stage_chunk_map.restype = ctypes.c_int
         L.gdn_stage_chunk_map.argtypes = [p, i64, i32, i32, i32, p, sz, p]
         L.gdn_stage_intra.restype = ctypes.c_int
@@ -221,20 +221,38 @@ def short_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None,
     return out, final_state
 
 
+UPDATE_RULES = {"gated_delta": 0, "delta": 1, "gated": 2, "linear": 3}
+
+
 def recurrent_fwd(q, k, v, g, beta, cu_seqlens, state_pool, token_slots, num_accepted=None, scale=None, eps=1e-6,
-                  gk=None, max_seqlen: int = 0, out=None, stream=None):
+                  gk=None, update_rule="gated_delta", max_seqlen: int = 0, out=None, stream=None):
     """Token recurrence with the pool updated in place, one slot per token (``gdn_recurrent_fwd``).
 
     ``state_pool`` [P, Nv, 128, 128] fp32 or bf16; ``token_slots`` [T] int32 gives each token's
     slot; sequence b starts from the slot of its token ``num_accepted[b] - 1`` (its last token when
-    ``num_accepted`` is None); ``gk`` [T, Nv, 128] fp32 is the optional key-dimension gate.
+    ``num_accepted`` is None); ``gk`` [T, Nv, 128] fp32 is the optional key-dimension gate;
+    ``update_rule`` is one of gated_delta, delta, gated, linear (g and gk are not needed by
+    delta and linear, beta not by gated and linear: pass None).
     Returns ``out``; ``state_pool`` holds the updated states afterwards."""
     if state_pool is None or token_slots is None:
         raise ValueError("recurrent_fwd needs a state pool and a slot per token")
     if state_pool.dtype not in (torch.float32, torch.bfloat16):
         raise RuntimeError(f"state_pool must be float32 or bfloat16 (got {state_pool.dtype})")
     bf16_pool = state_pool.dtype == torch.bfloat16
-    T, B, Nqk, Nv, P, dev = _resolve(q, k, v, g, beta, cu_seqlens, None, None)
+    if update_rule not in UPDATE_RULES:
+        raise ValueError(f"update_rule must be one of {sorted(UPDATE_RULES)}")
+    rule = UPDATE_RULES[update_rule]
+    decay, delta = rule in (0, 2), rule in (0, 1)
+    if not decay:
+        g = gk = None
+    if not delta:
+        beta = None
+    if q.dim() != 3 or v.dim() != 3:
+        raise ValueError("q/k must be [T, Nqk, 128] and v [T, Nv, 128]")
+    T, Nv = q.shape[0], v.shape[1]
+    dummy_g = g if g is not None else torch.empty(T, Nv, dtype=torch.float32, device=q.device)
+    dummy_b = beta if beta is not None else torch.empty(T, Nv, dtype=torch.bfloat16, device=q.device)
+    T, B, Nqk, Nv, P, dev = _resolve(q, k, v, dummy_g, dummy_b, cu_seqlens, None, None)
     P = state_pool.shape[0]
     _need(state_pool, "state_pool", state_pool.dtype, (P, Nv, HEAD_DIM, HEAD_DIM), dev)
     _need(token_slots, "token_slots", torch.int32, (T,), dev)
@@ -246,7 +264,7 @@ def recurrent_fwd(q, k, v, g, beta, cu_seqlens, state_pool, token_slots, num_acc
         out = torch.empty(T, Nv, HEAD_DIM, dtype=torch.bfloat16, device=dev)
     sc = 0.0 if scale is None else float(scale)
     rc = lib().gdn_recurrent_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(gk), _ptr(cu_seqlens),
-                                 _ptr(state_pool), int(bf16_pool), _ptr(token_slots), _ptr(num_accepted), sc,
+                                 _ptr(state_pool), int(bf16_pool), rule, _ptr(token_slots), _ptr(num_accepted), sc,
                                  float(eps), _ptr(out), T, B, Nqk, Nv, P, int(max_seqlen), _stream(stream))
     _check(rc, "gdn_recurrent_fwd")
     return out

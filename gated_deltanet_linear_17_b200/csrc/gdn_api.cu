@@ -154,14 +154,14 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA
 int check_forward(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                   const uint16_t *beta, const int32_t *cu, const float *pool, const int32_t *idx,
                   const uint16_t *out, const float *final_state, int64_t T, int32_t B, int32_t Nqk,
-                  int32_t Nv, int32_t P)
+                  int32_t Nv, int32_t P, bool need_g = true, bool need_beta = true)
 {
     int rc = check_sizes(T, B, Nqk, Nv);
     if (rc) return rc;
     if (P < 0) return GDN_ERR_BAD_SHAPE;
     if (B == 0) return GDN_OK;
     if (!cu) return GDN_ERR_NULL_ARG;
-    if (T > 0 && (!q || !k || !v || !g || !beta || !out)) return GDN_ERR_NULL_ARG;
+    if (T > 0 && (!q || !k || !v || (need_g && !g) || (need_beta && !beta) || !out)) return GDN_ERR_NULL_ARG;
     if (pool && P == 0) return GDN_ERR_BAD_SHAPE;
     if (pool && !idx && P < B) return GDN_ERR_BAD_SHAPE;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(pool) ||
@@ -295,12 +295,17 @@ int gdn_short_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
 
 int gdn_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                       const uint16_t *beta, const float *gk, const int32_t *cu_seqlens, void *state_pool,
-                      int32_t state_bf16, const int32_t *token_slots, const int32_t *num_accepted, float scale,
-                      float eps, uint16_t *out, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
-                      int32_t max_seqlen, void *stream)
+                      int32_t state_bf16, int32_t update_rule, const int32_t *token_slots,
+                      const int32_t *num_accepted, float scale, float eps, uint16_t *out, int64_t T, int32_t B,
+                      int32_t Nqk, int32_t Nv, int32_t P, int32_t max_seqlen, void *stream)
 {
+    if (update_rule < GDN_RULE_GATED_DELTA || update_rule > GDN_RULE_LINEAR) return GDN_ERR_BAD_SHAPE;
+    const bool decay = update_rule == GDN_RULE_GATED_DELTA || update_rule == GDN_RULE_GATED;
+    const bool delta = update_rule == GDN_RULE_GATED_DELTA || update_rule == GDN_RULE_DELTA;
+    if (!decay) g = nullptr, gk = nullptr;  // not read by this rule
+    if (!delta) beta = nullptr;
     int rc = check_forward(q, k, v, g, beta, cu_seqlens, static_cast<const float *>(state_pool), nullptr, out,
-                           nullptr, T, B, Nqk, Nv, P);
+                           nullptr, T, B, Nqk, Nv, P, decay, delta);
     if (rc || B == 0) return rc;
     if (!state_pool || (T > 0 && !token_slots)) return GDN_ERR_NULL_ARG;
     if (P <= 0 || (state_bf16 != 0 && state_bf16 != 1)) return GDN_ERR_BAD_SHAPE;
@@ -313,8 +318,8 @@ int gdn_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, c
         return GDN_ERR_OVERLAP;
     if (T == 0) return GDN_OK;
     return cuda_status(gdn::launch_recurrent(q, k, v, g, beta, gk, cu_seqlens, state_pool, state_bf16 != 0,
-                                             token_slots, num_accepted, resolve_scale(scale), eps, out, (int)T, B, Nqk,
-                                             Nv, max_seqlen, (cudaStream_t)stream));
+                                             update_rule, token_slots, num_accepted, resolve_scale(scale), eps, out,
+                                             (int)T, B, Nqk, Nv, max_seqlen, (cudaStream_t)stream));
 }
 
 int gdn_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,

@@ -35,7 +35,10 @@
 // when written) and the key-dimension gate gk (GK: S = S e^g e^gk, row i of S
 // decayed by e^{g + gk_i}; the 128 factors of each staged token are computed once
 // per CTA into shared memory, and the state rows are decayed before the sum
-// S^T kh).
+// S^T kh).  DECAY and DELTA select the update rule of the page
+// "com.microsoft.LinearAttention" (update_rule): gated_delta (both), delta (no
+// decay: g and gk unused), gated (S = e^g S + kh v^T: no retrieval, beta unused)
+// and linear (S = S + kh v^T); without the retrieval a token needs one barrier.
 #include "common.cuh"
 #include "gdn_internal.h"
 
@@ -55,7 +58,7 @@ struct ShortSmem {
     float red[2][4][32], red2[2][4][32];
 };
 
-template <int PRE, bool SLOTS, bool GK, bool SBF>
+template <int PRE, bool SLOTS, bool GK, bool SBF, bool DECAY, bool DELTA>
 __global__ void __launch_bounds__(kShortThreads) short_kernel(
     const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, const uint16_t *__restrict__ v,
     const float *__restrict__ g, const uint16_t *__restrict__ beta, const float *__restrict__ gk,
@@ -84,7 +87,7 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
         const int t = e >> 2, c = e & 3;
         cp_async16(smem_addr(&sm.v[t][c * 8]), v + ((size_t)(t0 + t) * Nv + h) * D + tl * kTile + c * 8, true);
     }
-    if (tid < npre) cp_async4(smem_addr(&sm.g[tid]), g + (size_t)(t0 + tid) * Nv + h);
+    if (DECAY && tid < npre) cp_async4(smem_addr(&sm.g[tid]), g + (size_t)(t0 + tid) * Nv + h);
     if (SLOTS && tid <= PRE && tid < n) cp_async4(smem_addr(&sm.slot[tid]), token_slots + t0 + tid);
     if (GK) {
         for (int e = tid; e < npre * 32; e += kShortThreads) {
@@ -94,7 +97,7 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
     }
     cp_async_commit();
     float bt_mine = 0.f;
-    if (tid < npre) bt_mine = bf2f(beta[(size_t)(t0 + tid) * Nv + h]);
+    if (DELTA && tid < npre) bt_mine = bf2f(beta[(size_t)(t0 + tid) * Nv + h]);
 
     // the state slice, straight into registers: s2[m] holds rows 32 wid + 2m, 2m + 1
     float2 s2[16];
@@ -166,7 +169,7 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
         const float rq = scale / sqrtf(sq + eps), rk = 1.0f / sqrtf(sk + eps);
         *reinterpret_cast<float4 *>(&sm.qh[t][lane * 4]) = make_float4(q4[0] * rq, q4[1] * rq, q4[2] * rq, q4[3] * rq);
         *reinterpret_cast<float4 *>(&sm.kh[t][lane * 4]) = make_float4(k4[0] * rk, k4[1] * rk, k4[2] * rk, k4[3] * rk);
-        if (lane == 0) sm.dg[t] = __expf(sm.g[t]);
+        if (lane == 0) sm.dg[t] = DECAY ? __expf(sm.g[t]) : 1.f;
     }
     if (GK) {  // the row decays e^{g + gk_i} of every staged token, in place over gk
         for (int e = tid; e < npre * D; e += kShortThreads) {
@@ -182,7 +185,7 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
         const float4 *qr = reinterpret_cast<const float4 *>(&sm.qh[j][wid * 32]);
         // the decay as one factor (applied to the sum S^T kh and in the update), or per row (GK: applied
         // to the state rows first)
-        const float dg = GK ? 1.f : sm.dg[j], bt = sm.beta[j], vj = bf2f(sm.v[j][lane]);
+        const float dg = (GK || !DECAY) ? 1.f : sm.dg[j], vj = bf2f(sm.v[j][lane]);
         if (GK) {
             const float4 *dr = reinterpret_cast<const float4 *>(&sm.gkd[j][wid * 32]);
 #pragma unroll
@@ -192,25 +195,28 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
                 s2[2 * c + 1] = fmul2(s2[2 * c + 1], make_float2(d4.z, d4.w));
             }
         }
-        // this warp's part of S^T kh
-        float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+        float u = vj;
+        if (DELTA) {  // this warp's part of S^T kh, then u = beta (v - S^T kh)
+            float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const float4 kx = kr[c];
-            a0 = ffma2(s2[2 * c], make_float2(kx.x, kx.y), a0);
-            a1 = ffma2(s2[2 * c + 1], make_float2(kx.z, kx.w), a1);
+            for (int c = 0; c < 8; ++c) {
+                const float4 kx = kr[c];
+                a0 = ffma2(s2[2 * c], make_float2(kx.x, kx.y), a0);
+                a1 = ffma2(s2[2 * c + 1], make_float2(kx.z, kx.w), a1);
+            }
+            sm.red[p][wid][lane] = (a0.x + a0.y) + (a1.x + a1.y);
+            __syncthreads();
+            const float kv =
+                dg * ((sm.red[p][0][lane] + sm.red[p][1][lane]) + (sm.red[p][2][lane] + sm.red[p][3][lane]));
+            u = sm.beta[j] * (vj - kv);
         }
-        sm.red[p][wid][lane] = (a0.x + a0.y) + (a1.x + a1.y);
-        __syncthreads();
-        const float kv = dg * ((sm.red[p][0][lane] + sm.red[p][1][lane]) + (sm.red[p][2][lane] + sm.red[p][3][lane]));
-        const float u = bt * (vj - kv);
         const float2 dg2 = make_float2(dg, dg), u2 = make_float2(u, u);
         // S = e^g S + kh u^T (GK: S already decayed), then this warp's part of S^T qh
         float2 b0 = make_float2(0.f, 0.f), b1 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const float4 kx = kr[c], qx = qr[c];
-            if (GK) {
+            if (GK || !DECAY) {
                 s2[2 * c] = ffma2(make_float2(kx.x, kx.y), u2, s2[2 * c]);
                 s2[2 * c + 1] = ffma2(make_float2(kx.z, kx.w), u2, s2[2 * c + 1]);
             } else {
@@ -243,8 +249,8 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
         sk = warp_sum(sk);
         const float rq = scale / sqrtf(sq + eps), rk = 1.0f / sqrtf(sk + eps);
         const float vj = bf2f(v[((size_t)t * Nv + h) * D + col]);
-        const float gt = g[(size_t)t * Nv + h], bt = bf2f(beta[(size_t)t * Nv + h]);
-        const float dg = GK ? 1.f : __expf(gt);
+        const float gt = DECAY ? g[(size_t)t * Nv + h] : 0.f, bt = DELTA ? bf2f(beta[(size_t)t * Nv + h]) : 1.f;
+        const float dg = (GK || !DECAY) ? 1.f : __expf(gt);
         if (GK) {  // this thread's 32 rows decayed by e^{g + gk_i}
             const float *gr = gk + ((size_t)t * Nv + h) * D + wid * 32;
 #pragma unroll
@@ -254,16 +260,20 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
             }
         }
         const uint16_t *kr = krow + wid * 32, *qr = qrow + wid * 32;
-        float acc = 0.f;
+        float u = vj;
+        if (DELTA) {
+            float acc = 0.f;
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            acc = fmaf(s2[m].x, bf2f(kr[2 * m]) * rk, acc);
-            acc = fmaf(s2[m].y, bf2f(kr[2 * m + 1]) * rk, acc);
+            for (int m = 0; m < 16; ++m) {
+                acc = fmaf(s2[m].x, bf2f(kr[2 * m]) * rk, acc);
+                acc = fmaf(s2[m].y, bf2f(kr[2 * m + 1]) * rk, acc);
+            }
+            sm.red[p][wid][lane] = acc;
+            __syncthreads();
+            const float kv =
+                dg * ((sm.red[p][0][lane] + sm.red[p][1][lane]) + (sm.red[p][2][lane] + sm.red[p][3][lane]));
+            u = bt * (vj - kv);
         }
-        sm.red[p][wid][lane] = acc;
-        __syncthreads();
-        const float kv = dg * ((sm.red[p][0][lane] + sm.red[p][1][lane]) + (sm.red[p][2][lane] + sm.red[p][3][lane]));
-        const float u = bt * (vj - kv);
         float acc2 = 0.f;
 #pragma unroll
         for (int m = 0; m < 16; ++m) {
@@ -293,35 +303,67 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
     }
 }
 
-template <int PRE, bool SLOTS, bool GK, bool SBF>
+template <int PRE, bool SLOTS, bool GK, bool SBF, bool DECAY, bool DELTA>
 static void launch_variant(dim3 grid, cudaStream_t st, const uint16_t *q, const uint16_t *k, const uint16_t *v,
                            const float *g, const uint16_t *beta, const float *gk, const int32_t *cu, const void *pool,
                            const int32_t *idx, const int32_t *token_slots, const int32_t *num_accepted, void *pool_w,
                            float scale, float eps, uint16_t *out, float *final_state, int T, int Nqk, int Nv)
 {
-    short_kernel<PRE, SLOTS, GK, SBF><<<grid, kShortThreads, 0, st>>>(q, k, v, g, beta, gk, cu, pool, idx, token_slots,
-                                                                      num_accepted, pool_w, scale, eps, out,
-                                                                      final_state, T, Nqk, Nv);
+    short_kernel<PRE, SLOTS, GK, SBF, DECAY, DELTA><<<grid, kShortThreads, 0, st>>>(
+        q, k, v, g, beta, gk, cu, pool, idx, token_slots, num_accepted, pool_w, scale, eps, out, final_state, T, Nqk,
+        Nv);
+}
+
+// the pool variants of one staging depth and update rule; a key gate only with a decaying rule
+template <int PRE, bool DECAY, bool DELTA>
+static void launch_rule(bool has_gk, bool bf16_pool, dim3 grid, cudaStream_t st, const uint16_t *q,
+                        const uint16_t *k, const uint16_t *v, const float *g, const uint16_t *beta, const float *gk,
+                        const int32_t *cu, void *pool, const int32_t *token_slots, const int32_t *num_accepted,
+                        float scale, float eps, uint16_t *out, int T, int Nqk, int Nv)
+{
+    if (DECAY && has_gk) {
+        if (bf16_pool)
+            launch_variant<PRE, true, DECAY, true, DECAY, DELTA>(grid, st, q, k, v, g, beta, gk, cu, pool, nullptr,
+                                                                 token_slots, num_accepted, pool, scale, eps, out,
+                                                                 nullptr, T, Nqk, Nv);
+        else
+            launch_variant<PRE, true, DECAY, false, DECAY, DELTA>(grid, st, q, k, v, g, beta, gk, cu, pool, nullptr,
+                                                                  token_slots, num_accepted, pool, scale, eps, out,
+                                                                  nullptr, T, Nqk, Nv);
+    } else if (bf16_pool) {
+        launch_variant<PRE, true, false, true, DECAY, DELTA>(grid, st, q, k, v, g, beta, nullptr, cu, pool, nullptr,
+                                                             token_slots, num_accepted, pool, scale, eps, out,
+                                                             nullptr, T, Nqk, Nv);
+    } else {
+        launch_variant<PRE, true, false, false, DECAY, DELTA>(grid, st, q, k, v, g, beta, nullptr, cu, pool, nullptr,
+                                                              token_slots, num_accepted, pool, scale, eps, out,
+                                                              nullptr, T, Nqk, Nv);
+    }
 }
 
 template <int PRE>
-static void launch_slots(bool has_gk, bool bf16_pool, dim3 grid, cudaStream_t st, const uint16_t *q,
+static void launch_slots(int rule, bool has_gk, bool bf16_pool, dim3 grid, cudaStream_t st, const uint16_t *q,
                          const uint16_t *k, const uint16_t *v, const float *g, const uint16_t *beta, const float *gk,
-                         const int32_t *cu, const void *pool, const int32_t *token_slots, const int32_t *num_accepted,
-                         void *pool_w, float scale, float eps, uint16_t *out, int T, int Nqk, int Nv)
+                         const int32_t *cu, void *pool, const int32_t *token_slots, const int32_t *num_accepted,
+                         float scale, float eps, uint16_t *out, int T, int Nqk, int Nv)
 {
-    if (has_gk && bf16_pool)
-        launch_variant<PRE, true, true, true>(grid, st, q, k, v, g, beta, gk, cu, pool, nullptr, token_slots,
-                                              num_accepted, pool_w, scale, eps, out, nullptr, T, Nqk, Nv);
-    else if (has_gk)
-        launch_variant<PRE, true, true, false>(grid, st, q, k, v, g, beta, gk, cu, pool, nullptr, token_slots,
-                                               num_accepted, pool_w, scale, eps, out, nullptr, T, Nqk, Nv);
-    else if (bf16_pool)
-        launch_variant<PRE, true, false, true>(grid, st, q, k, v, g, beta, nullptr, cu, pool, nullptr, token_slots,
-                                               num_accepted, pool_w, scale, eps, out, nullptr, T, Nqk, Nv);
-    else
-        launch_variant<PRE, true, false, false>(grid, st, q, k, v, g, beta, nullptr, cu, pool, nullptr, token_slots,
-                                                num_accepted, pool_w, scale, eps, out, nullptr, T, Nqk, Nv);
+    switch (rule) {
+    case kRuleDelta:
+        launch_rule<PRE, false, true>(has_gk, bf16_pool, grid, st, q, k, v, g, beta, gk, cu, pool, token_slots,
+                                      num_accepted, scale, eps, out, T, Nqk, Nv);
+        break;
+    case kRuleGated:
+        launch_rule<PRE, true, false>(has_gk, bf16_pool, grid, st, q, k, v, g, beta, gk, cu, pool, token_slots,
+                                      num_accepted, scale, eps, out, T, Nqk, Nv);
+        break;
+    case kRuleLinear:
+        launch_rule<PRE, false, false>(has_gk, bf16_pool, grid, st, q, k, v, g, beta, gk, cu, pool, token_slots,
+                                       num_accepted, scale, eps, out, T, Nqk, Nv);
+        break;
+    default:
+        launch_rule<PRE, true, true>(has_gk, bf16_pool, grid, st, q, k, v, g, beta, gk, cu, pool, token_slots,
+                                     num_accepted, scale, eps, out, T, Nqk, Nv);
+    }
 }
 
 cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
@@ -332,27 +374,28 @@ cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v
     if (B == 0) return cudaSuccess;
     const dim3 grid(B, Nv, D / kTile);
     if (max_seqlen >= 1 && max_seqlen <= 8)
-        launch_variant<8, false, false, false>(grid, st, q, k, v, g, beta, nullptr, cu, pool, idx, nullptr, nullptr,
-                                               nullptr, scale, eps, out, final_state, T, Nqk, Nv);
+        launch_variant<8, false, false, false, true, true>(grid, st, q, k, v, g, beta, nullptr, cu, pool, idx, nullptr,
+                                                           nullptr, nullptr, scale, eps, out, final_state, T, Nqk, Nv);
     else
-        launch_variant<16, false, false, false>(grid, st, q, k, v, g, beta, nullptr, cu, pool, idx, nullptr, nullptr,
-                                                nullptr, scale, eps, out, final_state, T, Nqk, Nv);
+        launch_variant<16, false, false, false, true, true>(grid, st, q, k, v, g, beta, nullptr, cu, pool, idx,
+                                                            nullptr, nullptr, nullptr, scale, eps, out, final_state, T,
+                                                            Nqk, Nv);
     return cudaGetLastError();
 }
 
 cudaError_t launch_recurrent(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                              const uint16_t *beta, const float *gk, const int32_t *cu, void *pool, bool bf16_pool,
-                             const int32_t *token_slots, const int32_t *num_accepted, float scale, float eps,
-                             uint16_t *out, int T, int B, int Nqk, int Nv, int max_seqlen, cudaStream_t st)
+                             int rule, const int32_t *token_slots, const int32_t *num_accepted, float scale,
+                             float eps, uint16_t *out, int T, int B, int Nqk, int Nv, int max_seqlen, cudaStream_t st)
 {
     if (B == 0) return cudaSuccess;
     const dim3 grid(B, Nv, D / kTile);
     if (max_seqlen >= 1 && max_seqlen <= 8)
-        launch_slots<8>(gk != nullptr, bf16_pool, grid, st, q, k, v, g, beta, gk, cu, pool, token_slots, num_accepted,
-                        pool, scale, eps, out, T, Nqk, Nv);
+        launch_slots<8>(rule, gk != nullptr, bf16_pool, grid, st, q, k, v, g, beta, gk, cu, pool, token_slots,
+                        num_accepted, scale, eps, out, T, Nqk, Nv);
     else
-        launch_slots<16>(gk != nullptr, bf16_pool, grid, st, q, k, v, g, beta, gk, cu, pool, token_slots, num_accepted,
-                         pool, scale, eps, out, T, Nqk, Nv);
+        launch_slots<16>(rule, gk != nullptr, bf16_pool, grid, st, q, k, v, g, beta, gk, cu, pool, token_slots,
+                         num_accepted, scale, eps, out, T, Nqk, Nv);
     return cudaGetLastError();
 }
 

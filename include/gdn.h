@@ -51,6 +51,12 @@ extern "C" {
 #define GDN_SHORT_MAX 16 /* max_seqlen at or below which the fused short-sequence kernel runs */
 #define GDN_NOALLOC_SCRATCH_BYTES (64u << 20) /* static workspace of gdn_chunk_fwd_noalloc, per GPU */
 
+/* update rules of gdn_recurrent_fwd */
+#define GDN_RULE_GATED_DELTA 0
+#define GDN_RULE_DELTA 1
+#define GDN_RULE_GATED 2
+#define GDN_RULE_LINEAR 3
+
 typedef enum {
     GDN_OK = 0,
     GDN_ERR_NULL_ARG = 1,    /* a required pointer is NULL                              */
@@ -179,6 +185,13 @@ int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *
  *   q, k, v, g, beta, cu_seqlens   as for gdn_chunk_fwd
  *   gk            device fp32 [T, Nv, 128 (Dk)], the key-dimension gate
  *                 (expected <= 0, not checked), or NULL for none
+ *   update_rule   GDN_RULE_GATED_DELTA (the rule above), GDN_RULE_DELTA (no decay:
+ *                 g and gk are not read and may be NULL), GDN_RULE_GATED
+ *                 (S = S * exp(g) * exp(gk) + k v^T: no retrieval, beta not read,
+ *                 may be NULL) or GDN_RULE_LINEAR (S = S + k v^T: g, gk and beta
+ *                 not read) -- the update rules of the page "com.microsoft.
+ *                 LinearAttention" (update_rule); q and k are normalised in
+ *                 every rule
  *   state_pool    device [P, Nv, 128 (Dk), 128 (Dv)], read and written in place
  *                 (required): fp32 when state_bf16 == 0, bf16 when state_bf16 == 1
  *                 (the page's pool dtype: widened to fp32 on load, the fp32 result
@@ -200,15 +213,16 @@ int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *
  * Alignment: q, k, v, out, state_pool, gk 16-byte aligned; g, cu_seqlens,
  * token_slots, num_accepted 4-byte aligned; beta 2-byte aligned.  Errors:
  * GDN_ERR_NULL_ARG, GDN_ERR_BAD_SHAPE, GDN_ERR_UNSUPPORTED, GDN_ERR_ALIGNMENT,
- * GDN_ERR_OVERLAP before anything is enqueued (state_bf16 other than 0 or 1 is
- * GDN_ERR_BAD_SHAPE); GDN_ERR_CUDA when the launch fails.  B == 0 or T == 0 is a no-op.  Asynchronous on `stream`; the library
+ * GDN_ERR_OVERLAP before anything is enqueued (state_bf16 other than 0 or 1, or
+ * an unknown update_rule, is GDN_ERR_BAD_SHAPE); GDN_ERR_CUDA when the launch
+ * fails.  B == 0 or T == 0 is a no-op.  Asynchronous on `stream`; the library
  * keeps no pointer after the call returns.
  */
 int gdn_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                       const uint16_t *beta, const float *gk, const int32_t *cu_seqlens, void *state_pool,
-                      int32_t state_bf16, const int32_t *token_slots, const int32_t *num_accepted, float scale,
-                      float eps, uint16_t *out, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
-                      int32_t max_seqlen, void *stream);
+                      int32_t state_bf16, int32_t update_rule, const int32_t *token_slots,
+                      const int32_t *num_accepted, float scale, float eps, uint16_t *out, int64_t T, int32_t B,
+                      int32_t Nqk, int32_t Nv, int32_t P, int32_t max_seqlen, void *stream);
 
 #ifdef __cplusplus
 }

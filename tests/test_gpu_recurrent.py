@@ -41,17 +41,20 @@ def _key_gate(inp, seed):
     return inputs.key_gate(inp, seed)
 
 
-def _run_and_check(inp, slots, acc, max_seqlen, what, gk=None, bf16_pool=False):
+def _run_and_check(inp, slots, acc, max_seqlen, what, gk=None, bf16_pool=False, rule="gated_delta"):
     pool0 = inp.state_pool.to(torch.bfloat16) if bf16_pool else inp.state_pool
     ro, rpool = recurrent_pool(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, pool0, slots,
-                               num_accepted=acc, scale=inp.scale, eps=inp.eps, gk=gk)
+                               num_accepted=acc, scale=inp.scale, eps=inp.eps, gk=gk, rule=rule)
     d = inp.to(DEV)
     pool = pool0.to(DEV).clone()
     start = pool.clone()
     ts = torch.from_numpy(slots).to(DEV)
     na = None if acc is None else torch.from_numpy(acc).to(DEV)
-    out = gdn.recurrent_fwd(d.q, d.k, d.v, d.g, d.beta, d.cu_seqlens, pool, ts, num_accepted=na, scale=d.scale,
-                            eps=d.eps, gk=None if gk is None else gk.to(DEV), max_seqlen=max_seqlen)
+    decay, delta = rule in ("gated_delta", "gated"), rule in ("gated_delta", "delta")
+    out = gdn.recurrent_fwd(d.q, d.k, d.v, d.g if decay else None, d.beta if delta else None, d.cu_seqlens, pool,
+                            ts, num_accepted=na, scale=d.scale, eps=d.eps,
+                            gk=None if gk is None or not decay else gk.to(DEV), update_rule=rule,
+                            max_seqlen=max_seqlen)
     torch.cuda.synchronize()
     assert_close(out, ro, f"{what} out")
     written = np.unique(slots)
@@ -149,3 +152,20 @@ def test_recurrent_key_gate_past_staged_tokens(max_seqlen):
     _run_and_check(inp, slots, acc, max_seqlen, f"key gate, long, max_seqlen={max_seqlen}", gk=gk)
     _run_and_check(inp, slots, acc, max_seqlen, f"key gate, long, bf16, max_seqlen={max_seqlen}", gk=gk,
                    bf16_pool=True)
+
+
+@pytest.mark.parametrize("rule", ["delta", "gated", "linear"])
+@pytest.mark.parametrize("max_seqlen", [8, 0])
+def test_recurrent_update_rules(rule, max_seqlen):
+    """The LinearAttention page's other update rules, a slot per token, staged and direct-read tokens."""
+    lens = [3, 1, 6, 0, 18, 2]
+    inp, slots, acc = _case(lens, Nqk=2, Nv=4, P=40, seed=57, per_token=True, accepted=True)
+    _run_and_check(inp, slots, acc, max_seqlen, f"rule {rule} max_seqlen={max_seqlen}", rule=rule)
+
+
+def test_recurrent_gated_rule_key_gate_bf16():
+    """The gated rule with the key-dimension gate on a bf16 pool (ordinary decoding)."""
+    r = np.random.default_rng(58)
+    lens = [int(x) for x in r.integers(1, 5, size=24)]
+    inp, slots, acc = _case(lens, Nqk=4, Nv=8, P=32, seed=59, per_token=False, accepted=False)
+    _run_and_check(inp, slots, acc, 4, "gated rule, gk, bf16", gk=_key_gate(inp, 60), bf16_pool=True, rule="gated")
