@@ -18,8 +18,9 @@ Two HBM-bound side workloads are timed in the same run (skipped with
 --no-short) and reported in the same line: ``short_seq`` (256 sequences of
 1..8 tokens from an fp32 state pool, gdn_chunk_fwd's fused short path) and
 ``spec_decode`` (256 sequences of 4 draft tokens, a pool slot per token,
-gdn_recurrent_fwd updating the pool in place) and ``decode_bf16`` (one token
-for each of 256 sequences on a bf16 pool with the key-dimension gate).
+gdn_recurrent_fwd updating the pool in place) and ``decode_bf16`` /
+``decode_bf16_dk64_dv512`` (one token per sequence on a bf16 pool with the
+key-dimension gate, at Dk = Dv = 128 and at the decode page's Dk = 64, Dv = 512).
 
 Prints ONE JSON line (rank 0).  ``--impl reference`` times the fp64 CPU
 oracle (the reference arm) on a bounded sample of the same workload instead.
@@ -425,38 +426,41 @@ def main():
         line["gpu_launches"] += args.steps
         del sp, slots, acc, spo
 
-        # one decode step on a bf16 pool with the key-dimension gate (the decode page's operator)
-        cfg = inputs.CONFIGS["decode_b256_bf16"]
-        dc = inputs.config("decode_b256_bf16", seed=cfg["seed"] + rank)
-        dgk = inputs.key_gate(dc, seed=cfg["seed"] + 200 + rank).to(dev)
-        dslots = dc.state_indices.clone()  # one token per sequence: its slot is the sequence's
-        dc = dc.to(dev)
-        dpool = dc.state_pool.to(torch.bfloat16)
-        dslots = dslots.to(dev)
-        dco = torch.empty(dc.T, dc.Nv, D, dtype=torch.bfloat16, device=dev)
+        # one decode step on a bf16 pool with the key-dimension gate (the decode page's operator), at the
+        # bench's head size and at the page's example shape
+        def decode_line(name):
+            cfg = inputs.CONFIGS[name]
+            dc = inputs.config(name, seed=cfg["seed"] + rank)
+            dgk = inputs.key_gate(dc, seed=cfg["seed"] + 200 + rank).to(dev)
+            dslots = dc.state_indices.clone().to(dev)  # one token per sequence: its slot is the sequence's
+            dc = dc.to(dev)
+            dpool = dc.state_pool.to(torch.bfloat16)
+            Dk, Dv = dc.q.shape[2], dc.v.shape[2]
+            dco = torch.empty(dc.T, dc.Nv, Dv, dtype=torch.bfloat16, device=dev)
 
-        def dstep():
-            gdn.recurrent_fwd(dc.q, dc.k, dc.v, dc.g, dc.beta, dc.cu_seqlens, dpool, dslots, scale=dc.scale,
-                              eps=dc.eps, gk=dgk, max_seqlen=1, out=dco)
-        for _ in range(args.warmup):
-            dstep()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            dstep()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        dms = gdist.max_over_ranks(e0.elapsed_time(e1) / args.steps, device=dev)
-        db = 2 * dc.B * dc.Nv * D * D * 2 + (short_bytes(dc) - 2 * dc.B * dc.Nv * D * D * 4) + dc.T * dc.Nv * D * 4
-        line["decode_bf16"] = {"workload": f"decode_b256_bf16: B={dc.B} x 1 token, Nqk={dc.Nqk}, Nv={dc.Nv}, bf16 pool "
-                                           f"[{dpool.shape[0]},{dc.Nv},128,128] updated in place, key gate gk",
-                               "ms": dms, "bytes": db, "GB/s": db / (dms / 1e3) / 1e9,
-                               "hbm_frac": db / (dms / 1e3) / 1e9 / peaks["hbm_gbs"],
-                               "tokens/s": world * dc.T / (dms / 1e3), "kernel": "short_kernel (slots, gk, bf16 pool)",
-                               "call": "gdn_recurrent_fwd"}
-        line["gpu_launches"] += args.steps
-        del dc, dgk, dslots, dpool, dco
+            def dstep():
+                gdn.recurrent_fwd(dc.q, dc.k, dc.v, dc.g, dc.beta, dc.cu_seqlens, dpool, dslots, scale=dc.scale,
+                                  eps=dc.eps, gk=dgk, max_seqlen=1, out=dco)
+            for _ in range(args.warmup):
+                dstep()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                dstep()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            dms = gdist.max_over_ranks(e0.elapsed_time(e1) / args.steps, device=dev)
+            per_tok = 2 * dc.Nqk * Dk * 2 + dc.Nv * Dv * 2 + dc.Nv * 4 + dc.Nv * 2 + dc.Nv * Dv * 2 + dc.Nv * Dk * 4
+            db = 2 * dc.B * dc.Nv * Dk * Dv * 2 + dc.T * per_tok  # bf16 states in and out, token I/O with gk
+            line["gpu_launches"] += args.steps
+            return {"workload": f"{name}: B={dc.B} x 1 token, Nqk={dc.Nqk}, Nv={dc.Nv}, Dk={Dk}, Dv={Dv}, bf16 pool "
+                                f"[{dpool.shape[0]},{dc.Nv},{Dk},{Dv}] updated in place, key gate gk",
+                    "ms": dms, "bytes": db, "GB/s": db / (dms / 1e3) / 1e9,
+                    "hbm_frac": db / (dms / 1e3) / 1e9 / peaks["hbm_gbs"], "tokens/s": world * dc.T / (dms / 1e3),
+                    "kernel": "short_kernel (slots, gk, bf16 pool)", "call": "gdn_recurrent_fwd"}
+        line["decode_bf16"] = decode_line("decode_b256_bf16")
+        line["decode_bf16_dk64_dv512"] = decode_line("decode_dk64_dv512")
 
     # ---- end to end from pinned host buffers through the public call
     if not args.no_e2e:

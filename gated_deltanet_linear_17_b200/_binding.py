@@ -59,8 +59,10 @@ def lib():
         L.gdn_short_fwd.restype = ctypes.c_int
         L.gdn_short_fwd.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, p]
         L.gdn_recurrent_fwd.restype = ctypes.c_int
+        # q k v g beta gk cu pool | state_bf16 rule | slots accepted | scale eps | out | T | B Nqk Nv Dk Dv P
+        # max_seqlen | stream
         L.gdn_recurrent_fwd.argtypes = [p, p, p, p, p, p, p, p, i32, i32, p, p, f32, f32, p, i64, i32, i32, i32, i32,
-                                        i32, p]
+                                        i32, i32, i32, p]
         L.gdn_stage_chunk_map.restype = ctypes.c_int
         L.gdn_stage_chunk_map.argtypes = [p, i64, i32, i32, i32, p, sz, p]
         L.gdn_stage_intra.restype = ctypes.c_int
@@ -228,7 +230,8 @@ def recurrent_fwd(q, k, v, g, beta, cu_seqlens, state_pool, token_slots, num_acc
                   gk=None, update_rule="gated_delta", max_seqlen: int = 0, out=None, stream=None):
     """Token recurrence with the pool updated in place, one slot per token (``gdn_recurrent_fwd``).
 
-    ``state_pool`` [P, Nv, 128, 128] fp32 or bf16; ``token_slots`` [T] int32 gives each token's
+    q, k [T, Nqk, Dk], v [T, Nv, Dv] with Dk 64 or 128 and Dv a multiple of 32;
+    ``state_pool`` [P, Nv, Dk, Dv] fp32 or bf16; ``token_slots`` [T] int32 gives each token's
     slot; sequence b starts from the slot of its token ``num_accepted[b] - 1`` (its last token when
     ``num_accepted`` is None); ``gk`` [T, Nv, 128] fp32 is the optional key-dimension gate;
     ``update_rule`` is one of gated_delta, delta, gated, linear (g and gk are not needed by
@@ -248,24 +251,34 @@ def recurrent_fwd(q, k, v, g, beta, cu_seqlens, state_pool, token_slots, num_acc
     if not delta:
         beta = None
     if q.dim() != 3 or v.dim() != 3:
-        raise ValueError("q/k must be [T, Nqk, 128] and v [T, Nv, 128]")
-    T, Nv = q.shape[0], v.shape[1]
-    dummy_g = g if g is not None else torch.empty(T, Nv, dtype=torch.float32, device=q.device)
-    dummy_b = beta if beta is not None else torch.empty(T, Nv, dtype=torch.bfloat16, device=q.device)
-    T, B, Nqk, Nv, P, dev = _resolve(q, k, v, dummy_g, dummy_b, cu_seqlens, None, None)
+        raise ValueError("q/k must be [T, Nqk, Dk] and v [T, Nv, Dv]")
+    T, Nqk, Dk = q.shape
+    Nv, Dv = v.shape[1], v.shape[2]
+    if Nv % Nqk != 0:
+        raise ValueError(f"Nv ({Nv}) must be a multiple of Nqk ({Nqk})")
+    B = cu_seqlens.shape[0] - 1
+    dev = q.device
+    _need(q, "q", torch.bfloat16, (T, Nqk, Dk), dev)
+    _need(k, "k", torch.bfloat16, (T, Nqk, Dk), dev)
+    _need(v, "v", torch.bfloat16, (T, Nv, Dv), dev)
+    if g is not None:
+        _need(g, "g", torch.float32, (T, Nv), dev)
+    if beta is not None:
+        _need(beta, "beta", torch.bfloat16, (T, Nv), dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), dev)
     P = state_pool.shape[0]
-    _need(state_pool, "state_pool", state_pool.dtype, (P, Nv, HEAD_DIM, HEAD_DIM), dev)
+    _need(state_pool, "state_pool", state_pool.dtype, (P, Nv, Dk, Dv), dev)
     _need(token_slots, "token_slots", torch.int32, (T,), dev)
     if num_accepted is not None:
         _need(num_accepted, "num_accepted", torch.int32, (B,), dev)
     if gk is not None:
-        _need(gk, "gk", torch.float32, (T, Nv, HEAD_DIM), dev)
+        _need(gk, "gk", torch.float32, (T, Nv, Dk), dev)
     if out is None:
-        out = torch.empty(T, Nv, HEAD_DIM, dtype=torch.bfloat16, device=dev)
+        out = torch.empty(T, Nv, Dv, dtype=torch.bfloat16, device=dev)
     sc = 0.0 if scale is None else float(scale)
     rc = lib().gdn_recurrent_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(gk), _ptr(cu_seqlens),
                                  _ptr(state_pool), int(bf16_pool), rule, _ptr(token_slots), _ptr(num_accepted), sc,
-                                 float(eps), _ptr(out), T, B, Nqk, Nv, P, int(max_seqlen), _stream(stream))
+                                 float(eps), _ptr(out), T, B, Nqk, Nv, Dk, Dv, P, int(max_seqlen), _stream(stream))
     _check(rc, "gdn_recurrent_fwd")
     return out
 

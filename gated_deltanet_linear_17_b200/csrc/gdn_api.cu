@@ -297,29 +297,39 @@ int gdn_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, c
                       const uint16_t *beta, const float *gk, const int32_t *cu_seqlens, void *state_pool,
                       int32_t state_bf16, int32_t update_rule, const int32_t *token_slots,
                       const int32_t *num_accepted, float scale, float eps, uint16_t *out, int64_t T, int32_t B,
-                      int32_t Nqk, int32_t Nv, int32_t P, int32_t max_seqlen, void *stream)
+                      int32_t Nqk, int32_t Nv, int32_t Dk, int32_t Dv, int32_t P, int32_t max_seqlen, void *stream)
 {
+    int rc = check_sizes(T, B, Nqk, Nv);
+    if (rc) return rc;
     if (update_rule < GDN_RULE_GATED_DELTA || update_rule > GDN_RULE_LINEAR) return GDN_ERR_BAD_SHAPE;
+    if (P <= 0 || (state_bf16 != 0 && state_bf16 != 1)) return GDN_ERR_BAD_SHAPE;
+    if (Dk <= 0 || Dv <= 0) return GDN_ERR_BAD_SHAPE;
+    if ((Dk != 64 && Dk != 128) || Dv % 32 != 0 || Dv > 1024) return GDN_ERR_UNSUPPORTED;
+    if (B == 0) return GDN_OK;
     const bool decay = update_rule == GDN_RULE_GATED_DELTA || update_rule == GDN_RULE_GATED;
     const bool delta = update_rule == GDN_RULE_GATED_DELTA || update_rule == GDN_RULE_DELTA;
     if (!decay) g = nullptr, gk = nullptr;  // not read by this rule
     if (!delta) beta = nullptr;
-    int rc = check_forward(q, k, v, g, beta, cu_seqlens, static_cast<const float *>(state_pool), nullptr, out,
-                           nullptr, T, B, Nqk, Nv, P, decay, delta);
-    if (rc || B == 0) return rc;
-    if (!state_pool || (T > 0 && !token_slots)) return GDN_ERR_NULL_ARG;
-    if (P <= 0 || (state_bf16 != 0 && state_bf16 != 1)) return GDN_ERR_BAD_SHAPE;
-    if ((reinterpret_cast<uintptr_t>(token_slots) & 3u) || (reinterpret_cast<uintptr_t>(num_accepted) & 3u) ||
+    if (!cu_seqlens || !state_pool) return GDN_ERR_NULL_ARG;
+    if (T > 0 && (!q || !k || !v || !out || !token_slots || (decay && !g) || (delta && !beta)))
+        return GDN_ERR_NULL_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(state_pool) ||
         !aligned16(gk))
         return GDN_ERR_ALIGNMENT;
-    const size_t obytes = (size_t)T * Nv * gdn::D * 2;
-    const size_t pbytes = (size_t)gdn::D * gdn::D * (state_bf16 ? 2 : 4) * Nv * P;
-    if (overlap(out, obytes, state_pool, pbytes) || overlap(out, obytes, gk, (size_t)T * Nv * gdn::D * 4))
+    if ((reinterpret_cast<uintptr_t>(g) & 3u) || (reinterpret_cast<uintptr_t>(beta) & 1u) ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(token_slots) & 3u) ||
+        (reinterpret_cast<uintptr_t>(num_accepted) & 3u))
+        return GDN_ERR_ALIGNMENT;
+    const size_t obytes = (size_t)T * Nv * Dv * 2, qbytes = (size_t)T * Nqk * Dk * 2;
+    const size_t pbytes = (size_t)Dk * Dv * (state_bf16 ? 2 : 4) * Nv * P;
+    if (overlap(out, obytes, q, qbytes) || overlap(out, obytes, k, qbytes) || overlap(out, obytes, v, obytes) ||
+        overlap(out, obytes, state_pool, pbytes) || overlap(out, obytes, gk, (size_t)T * Nv * Dk * 4))
         return GDN_ERR_OVERLAP;
     if (T == 0) return GDN_OK;
+    const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)Dk);
     return cuda_status(gdn::launch_recurrent(q, k, v, g, beta, gk, cu_seqlens, state_pool, state_bf16 != 0,
-                                             update_rule, token_slots, num_accepted, resolve_scale(scale), eps, out,
-                                             (int)T, B, Nqk, Nv, max_seqlen, (cudaStream_t)stream));
+                                             update_rule, token_slots, num_accepted, sc, eps, out, (int)T, B, Nqk, Nv,
+                                             Dk, Dv, max_seqlen, (cudaStream_t)stream));
 }
 
 int gdn_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,

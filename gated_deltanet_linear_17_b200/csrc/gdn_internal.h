@@ -57,13 +57,14 @@ cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v
                          float eps, uint16_t *out, float *final_state, int T, int B, int Nqk, int Nv, int max_seqlen,
                          cudaStream_t st);
 // The same kernel on a pool updated in place (fp32, or bf16 when bf16_pool), one slot per token,
-// the start taken from the last accepted token's slot; gk [T, Nv, 128] or nullptr (read only by the
-// decaying rules).
+// the start taken from the last accepted token's slot; key dimension Dk (64 or 128), value dimension
+// Dv (a multiple of 32); gk [T, Nv, Dk] or nullptr (read only by the decaying rules).
 // update rules of gdn_recurrent_fwd (GDN_RULE_* in gdn.h)
 constexpr int kRuleGatedDelta = 0, kRuleDelta = 1, kRuleGated = 2, kRuleLinear = 3;
 cudaError_t launch_recurrent(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                              const uint16_t *beta, const float *gk, const int32_t *cu, void *pool, bool bf16_pool,
                              int rule, const int32_t *token_slots, const int32_t *num_accepted, float scale,
-                             float eps, uint16_t *out, int T, int B, int Nqk, int Nv, int max_seqlen, cudaStream_t st);
+                             float eps, uint16_t *out, int T, int B, int Nqk, int Nv, int Dk, int Dv, int max_seqlen,
+                             cudaStream_t st);
 
 }  // namespace gdn

@@ -44,29 +44,40 @@
 
 namespace gdn {
 
-constexpr int kShortThreads = 128;
 constexpr int kTile = 32;  // Dv columns per CTA
 
-template <int PRE, bool GK>  // tokens staged together with the state; key gate
+// DK: key dimension (64 or 128); the CTA has DK threads, warp w holding state rows 32w .. 32w + 31
+template <int PRE, bool GK, int DK>  // tokens staged together with the state; key gate
 struct ShortSmem {
-    float kh[PRE][D], qh[PRE][D];   // normalised rows, fp32 (qh includes the scale)
-    float gkd[GK ? PRE : 1][D];     // gk rows, then the row decays e^{g + gk} (GK)
-    uint16_t q[PRE][D], k[PRE][D];  // raw bf16 rows
-    uint16_t v[PRE][kTile];         // raw bf16 slice
+    float kh[PRE][DK], qh[PRE][DK];   // normalised rows, fp32 (qh includes the scale)
+    float gkd[GK ? PRE : 1][DK];      // gk rows, then the row decays e^{g + gk} (GK)
+    uint16_t q[PRE][DK], k[PRE][DK];  // raw bf16 rows
+    uint16_t v[PRE][kTile];           // raw bf16 slice
     float g[PRE], dg[PRE], beta[PRE];
     int32_t slot[PRE + 1];  // token slots (SLOTS)
-    float red[2][4][32], red2[2][4][32];
+    float red[2][DK / 32][32], red2[2][DK / 32][32];
 };
 
-template <int PRE, bool SLOTS, bool GK, bool SBF, bool DECAY, bool DELTA>
-__global__ void __launch_bounds__(kShortThreads) short_kernel(
+// sum over the warps of a [DK / 32][32] partial-sum array at this lane's column
+template <int NW>
+__device__ __forceinline__ float sum_warps(const float (&r)[NW][32], int lane)
+{
+    float a = r[0][lane];
+#pragma unroll
+    for (int w = 1; w < NW; ++w) a += r[w][lane];
+    return a;
+}
+
+template <int PRE, bool SLOTS, bool GK, bool SBF, bool DECAY, bool DELTA, int DK>
+__global__ void __launch_bounds__(DK) short_kernel(
     const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, const uint16_t *__restrict__ v,
     const float *__restrict__ g, const uint16_t *__restrict__ beta, const float *__restrict__ gk,
     const int32_t *__restrict__ cu, const void *pool, const int32_t *__restrict__ idx,
     const int32_t *__restrict__ token_slots, const int32_t *__restrict__ num_accepted, void *pool_w, float scale,
-    float eps, uint16_t *__restrict__ out, float *__restrict__ final_state, int T, int Nqk, int Nv)
+    float eps, uint16_t *__restrict__ out, float *__restrict__ final_state, int T, int Nqk, int Nv, int Dv)
 {
-    __shared__ __align__(16) ShortSmem<PRE, GK> sm;
+    constexpr int NW = DK / 32, EL = DK / 32;  // warps; elements of a q/k row per lane
+    __shared__ __align__(16) ShortSmem<PRE, GK, DK> sm;
     const int b = blockIdx.x, h = blockIdx.y, tl = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int col = tl * kTile + lane;
@@ -77,22 +88,22 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
     if (SLOTS && n == 0) return;  // no token: the pool keeps its slots
 
     // token data of the first kPre tokens: async copies
-    for (int e = tid; e < npre * 16; e += kShortThreads) {
-        const int t = e >> 4, c = e & 15;
-        const size_t off = ((size_t)(t0 + t) * Nqk + hq) * D + c * 8;
+    for (int e = tid; e < npre * (DK / 8); e += DK) {
+        const int t = e / (DK / 8), c = e % (DK / 8);
+        const size_t off = ((size_t)(t0 + t) * Nqk + hq) * DK + c * 8;
         cp_async16(smem_addr(&sm.q[t][c * 8]), q + off, true);
         cp_async16(smem_addr(&sm.k[t][c * 8]), k + off, true);
     }
-    for (int e = tid; e < npre * 4; e += kShortThreads) {
+    for (int e = tid; e < npre * 4; e += DK) {
         const int t = e >> 2, c = e & 3;
-        cp_async16(smem_addr(&sm.v[t][c * 8]), v + ((size_t)(t0 + t) * Nv + h) * D + tl * kTile + c * 8, true);
+        cp_async16(smem_addr(&sm.v[t][c * 8]), v + ((size_t)(t0 + t) * Nv + h) * Dv + tl * kTile + c * 8, true);
     }
     if (DECAY && tid < npre) cp_async4(smem_addr(&sm.g[tid]), g + (size_t)(t0 + tid) * Nv + h);
     if (SLOTS && tid <= PRE && tid < n) cp_async4(smem_addr(&sm.slot[tid]), token_slots + t0 + tid);
     if (GK) {
-        for (int e = tid; e < npre * 32; e += kShortThreads) {
-            const int t = e >> 5, c = e & 31;
-            cp_async16(smem_addr(&sm.gkd[t][c * 4]), gk + ((size_t)(t0 + t) * Nv + h) * D + c * 4, true);
+        for (int e = tid; e < npre * (DK / 4); e += DK) {
+            const int t = e / (DK / 4), c = e % (DK / 4);
+            cp_async16(smem_addr(&sm.gkd[t][c * 4]), gk + ((size_t)(t0 + t) * Nv + h) * DK + c * 4, true);
         }
     }
     cp_async_commit();
@@ -109,17 +120,17 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
         } else {
             slot = idx ? idx[b] : b;
         }
-        const size_t off = (((size_t)slot * Nv + h) * D + wid * 32) * D + col;
+        const size_t off = (((size_t)slot * Nv + h) * DK + wid * 32) * Dv + col;
         if (SBF) {
             const unsigned short *src = static_cast<const unsigned short *>(pool) + off;
 #pragma unroll
             for (int m = 0; m < 16; ++m)
-                s2[m] = make_float2(bf2f(__ldcs(src + (size_t)(2 * m) * D)), bf2f(__ldcs(src + (size_t)(2 * m + 1) * D)));
+                s2[m] = make_float2(bf2f(__ldcs(src + (size_t)(2 * m) * Dv)), bf2f(__ldcs(src + (size_t)(2 * m + 1) * Dv)));
         } else {
             const float *src = static_cast<const float *>(pool) + off;
 #pragma unroll
             for (int m = 0; m < 16; ++m)
-                s2[m] = make_float2(__ldcs(src + (size_t)(2 * m) * D), __ldcs(src + (size_t)(2 * m + 1) * D));
+                s2[m] = make_float2(__ldcs(src + (size_t)(2 * m) * Dv), __ldcs(src + (size_t)(2 * m + 1) * Dv));
         }
     } else {
 #pragma unroll
@@ -128,20 +139,20 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
 
     // this thread's 32 values of the state into pool slot `slot` (SLOTS)
     auto write_slot = [&](int slot) {
-        const size_t off = (((size_t)slot * Nv + h) * D + wid * 32) * D + col;
+        const size_t off = (((size_t)slot * Nv + h) * DK + wid * 32) * Dv + col;
         if (SBF) {
             unsigned short *dst = static_cast<unsigned short *>(pool_w) + off;
 #pragma unroll
             for (int m = 0; m < 16; ++m) {
-                __stcs(dst + (size_t)(2 * m) * D, (unsigned short)f2bf(s2[m].x));
-                __stcs(dst + (size_t)(2 * m + 1) * D, (unsigned short)f2bf(s2[m].y));
+                __stcs(dst + (size_t)(2 * m) * Dv, (unsigned short)f2bf(s2[m].x));
+                __stcs(dst + (size_t)(2 * m + 1) * Dv, (unsigned short)f2bf(s2[m].y));
             }
         } else {
             float *dst = static_cast<float *>(pool_w) + off;
 #pragma unroll
             for (int m = 0; m < 16; ++m) {
-                __stcs(dst + (size_t)(2 * m) * D, s2[m].x);
-                __stcs(dst + (size_t)(2 * m + 1) * D, s2[m].y);
+                __stcs(dst + (size_t)(2 * m) * Dv, s2[m].x);
+                __stcs(dst + (size_t)(2 * m + 1) * Dv, s2[m].y);
             }
         }
     };
@@ -150,32 +161,36 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
     if (tid < npre) sm.beta[tid] = bt_mine;
     __syncthreads();
     // normalised q and k rows in fp32 and the decay of every staged token: one warp per token,
-    // lane l at elements 4l .. 4l + 3
-    for (int t = wid; t < npre; t += kShortThreads / 32) {
-        const uint2 qa = *reinterpret_cast<const uint2 *>(&sm.q[t][lane * 4]);
-        const uint2 ka = *reinterpret_cast<const uint2 *>(&sm.k[t][lane * 4]);
-        const float q4[4] = {__uint_as_float(qa.x << 16), __uint_as_float(qa.x & 0xffff0000u),
-                             __uint_as_float(qa.y << 16), __uint_as_float(qa.y & 0xffff0000u)};
-        const float k4[4] = {__uint_as_float(ka.x << 16), __uint_as_float(ka.x & 0xffff0000u),
-                             __uint_as_float(ka.y << 16), __uint_as_float(ka.y & 0xffff0000u)};
+    // lane l at elements EL l .. EL l + EL - 1
+    for (int t = wid; t < npre; t += NW) {
+        float qe[EL], ke[EL];
         float sq = 0.f, sk = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            sq = fmaf(q4[e], q4[e], sq);
-            sk = fmaf(k4[e], k4[e], sk);
+        for (int e2 = 0; e2 < EL / 2; ++e2) {
+            const uint32_t qw = reinterpret_cast<const uint32_t *>(&sm.q[t][lane * EL])[e2];
+            const uint32_t kw = reinterpret_cast<const uint32_t *>(&sm.k[t][lane * EL])[e2];
+            qe[2 * e2] = __uint_as_float(qw << 16);
+            qe[2 * e2 + 1] = __uint_as_float(qw & 0xffff0000u);
+            ke[2 * e2] = __uint_as_float(kw << 16);
+            ke[2 * e2 + 1] = __uint_as_float(kw & 0xffff0000u);
+        }
+#pragma unroll
+        for (int e = 0; e < EL; ++e) {
+            sq = fmaf(qe[e], qe[e], sq);
+            sk = fmaf(ke[e], ke[e], sk);
         }
         sq = warp_sum(sq);
         sk = warp_sum(sk);
         const float rq = scale / sqrtf(sq + eps), rk = 1.0f / sqrtf(sk + eps);
-        *reinterpret_cast<float4 *>(&sm.qh[t][lane * 4]) = make_float4(q4[0] * rq, q4[1] * rq, q4[2] * rq, q4[3] * rq);
-        *reinterpret_cast<float4 *>(&sm.kh[t][lane * 4]) = make_float4(k4[0] * rk, k4[1] * rk, k4[2] * rk, k4[3] * rk);
+#pragma unroll
+        for (int e2 = 0; e2 < EL / 2; ++e2) {
+            reinterpret_cast<float2 *>(&sm.qh[t][lane * EL])[e2] = make_float2(qe[2 * e2] * rq, qe[2 * e2 + 1] * rq);
+            reinterpret_cast<float2 *>(&sm.kh[t][lane * EL])[e2] = make_float2(ke[2 * e2] * rk, ke[2 * e2 + 1] * rk);
+        }
         if (lane == 0) sm.dg[t] = DECAY ? __expf(sm.g[t]) : 1.f;
     }
-    if (GK) {  // the row decays e^{g + gk_i} of every staged token, in place over gk
-        for (int e = tid; e < npre * D; e += kShortThreads) {
-            const int t = e >> 7, i = e & (D - 1);
-            sm.gkd[t][i] = __expf(sm.g[t] + sm.gkd[t][i]);
-        }
+    if (GK) {  // the row decays e^{g + gk_i} of every staged token, in place over gk (thread i: row i)
+        for (int t = 0; t < npre; ++t) sm.gkd[t][tid] = __expf(sm.g[t] + sm.gkd[t][tid]);
     }
     __syncthreads();
 
@@ -206,8 +221,7 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
             }
             sm.red[p][wid][lane] = (a0.x + a0.y) + (a1.x + a1.y);
             __syncthreads();
-            const float kv =
-                dg * ((sm.red[p][0][lane] + sm.red[p][1][lane]) + (sm.red[p][2][lane] + sm.red[p][3][lane]));
+            const float kv = dg * sum_warps<NW>(sm.red[p], lane);
             u = sm.beta[j] * (vj - kv);
         }
         const float2 dg2 = make_float2(dg, dg), u2 = make_float2(u, u);
@@ -230,17 +244,16 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
         if (SLOTS && (j == n - 1 || sm.slot[j + 1] != sm.slot[j])) write_slot(sm.slot[j]);
         __syncthreads();
         if (wid == 0)
-            out[((size_t)(t0 + j) * Nv + h) * D + col] =
-                f2bf((sm.red2[p][0][lane] + sm.red2[p][1][lane]) + (sm.red2[p][2][lane] + sm.red2[p][3][lane]));
+            out[((size_t)(t0 + j) * Nv + h) * Dv + col] = f2bf(sum_warps<NW>(sm.red2[p], lane));
     }
 
     // beyond the staged tokens (longer sequences than the fused path is meant for): read directly
     for (int j = PRE; j < n; ++j) {
         const int t = t0 + j, p = j & 1;
-        const uint16_t *qrow = q + ((size_t)t * Nqk + hq) * D, *krow = k + ((size_t)t * Nqk + hq) * D;
+        const uint16_t *qrow = q + ((size_t)t * Nqk + hq) * DK, *krow = k + ((size_t)t * Nqk + hq) * DK;
         float sq = 0.f, sk = 0.f;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < EL; ++i) {
             const float a = bf2f(qrow[lane + 32 * i]), c = bf2f(krow[lane + 32 * i]);
             sq = fmaf(a, a, sq);
             sk = fmaf(c, c, sk);
@@ -248,11 +261,11 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
         sq = warp_sum(sq);
         sk = warp_sum(sk);
         const float rq = scale / sqrtf(sq + eps), rk = 1.0f / sqrtf(sk + eps);
-        const float vj = bf2f(v[((size_t)t * Nv + h) * D + col]);
+        const float vj = bf2f(v[((size_t)t * Nv + h) * Dv + col]);
         const float gt = DECAY ? g[(size_t)t * Nv + h] : 0.f, bt = DELTA ? bf2f(beta[(size_t)t * Nv + h]) : 1.f;
         const float dg = (GK || !DECAY) ? 1.f : __expf(gt);
         if (GK) {  // this thread's 32 rows decayed by e^{g + gk_i}
-            const float *gr = gk + ((size_t)t * Nv + h) * D + wid * 32;
+            const float *gr = gk + ((size_t)t * Nv + h) * DK + wid * 32;
 #pragma unroll
             for (int m = 0; m < 16; ++m) {
                 s2[m].x *= __expf(gt + gr[2 * m]);
@@ -270,8 +283,7 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
             }
             sm.red[p][wid][lane] = acc;
             __syncthreads();
-            const float kv =
-                dg * ((sm.red[p][0][lane] + sm.red[p][1][lane]) + (sm.red[p][2][lane] + sm.red[p][3][lane]));
+            const float kv = dg * sum_warps<NW>(sm.red[p], lane);
             u = bt * (vj - kv);
         }
         float acc2 = 0.f;
@@ -289,80 +301,71 @@ __global__ void __launch_bounds__(kShortThreads) short_kernel(
         }
         __syncthreads();
         if (wid == 0)
-            out[((size_t)t * Nv + h) * D + col] =
-                f2bf((sm.red2[p][0][lane] + sm.red2[p][1][lane]) + (sm.red2[p][2][lane] + sm.red2[p][3][lane]));
+            out[((size_t)t * Nv + h) * Dv + col] = f2bf(sum_warps<NW>(sm.red2[p], lane));
     }
 
     if (!SLOTS && final_state) {
-        float *dst = final_state + (((size_t)b * Nv + h) * D + wid * 32) * D + col;
+        float *dst = final_state + (((size_t)b * Nv + h) * DK + wid * 32) * Dv + col;
 #pragma unroll
         for (int m = 0; m < 16; ++m) {
-            __stcs(dst + (size_t)(2 * m) * D, s2[m].x);
-            __stcs(dst + (size_t)(2 * m + 1) * D, s2[m].y);
+            __stcs(dst + (size_t)(2 * m) * Dv, s2[m].x);
+            __stcs(dst + (size_t)(2 * m + 1) * Dv, s2[m].y);
         }
     }
 }
 
-template <int PRE, bool SLOTS, bool GK, bool SBF, bool DECAY, bool DELTA>
+template <int PRE, bool SLOTS, bool GK, bool SBF, bool DECAY, bool DELTA, int DK>
 static void launch_variant(dim3 grid, cudaStream_t st, const uint16_t *q, const uint16_t *k, const uint16_t *v,
                            const float *g, const uint16_t *beta, const float *gk, const int32_t *cu, const void *pool,
                            const int32_t *idx, const int32_t *token_slots, const int32_t *num_accepted, void *pool_w,
-                           float scale, float eps, uint16_t *out, float *final_state, int T, int Nqk, int Nv)
+                           float scale, float eps, uint16_t *out, float *final_state, int T, int Nqk, int Nv, int Dv)
 {
-    short_kernel<PRE, SLOTS, GK, SBF, DECAY, DELTA><<<grid, kShortThreads, 0, st>>>(
+    short_kernel<PRE, SLOTS, GK, SBF, DECAY, DELTA, DK><<<grid, DK, 0, st>>>(
         q, k, v, g, beta, gk, cu, pool, idx, token_slots, num_accepted, pool_w, scale, eps, out, final_state, T, Nqk,
-        Nv);
+        Nv, Dv);
 }
 
-// the pool variants of one staging depth and update rule; a key gate only with a decaying rule
-template <int PRE, bool DECAY, bool DELTA>
-static void launch_rule(bool has_gk, bool bf16_pool, dim3 grid, cudaStream_t st, const uint16_t *q,
-                        const uint16_t *k, const uint16_t *v, const float *g, const uint16_t *beta, const float *gk,
-                        const int32_t *cu, void *pool, const int32_t *token_slots, const int32_t *num_accepted,
-                        float scale, float eps, uint16_t *out, int T, int Nqk, int Nv)
+// Arguments of one pool-updating launch
+struct RecArgs {
+    const uint16_t *q, *k, *v;
+    const float *g;
+    const uint16_t *beta;
+    const float *gk;
+    const int32_t *cu;
+    void *pool;
+    const int32_t *token_slots, *num_accepted;
+    float scale, eps;
+    uint16_t *out;
+    int T, Nqk, Nv, Dv;
+};
+
+template <int PRE, bool GK, bool SBF, bool DECAY, bool DELTA, int DK>
+static void launch_pool(const RecArgs &a, dim3 grid, cudaStream_t st)
 {
-    if (DECAY && has_gk) {
-        if (bf16_pool)
-            launch_variant<PRE, true, DECAY, true, DECAY, DELTA>(grid, st, q, k, v, g, beta, gk, cu, pool, nullptr,
-                                                                 token_slots, num_accepted, pool, scale, eps, out,
-                                                                 nullptr, T, Nqk, Nv);
-        else
-            launch_variant<PRE, true, DECAY, false, DECAY, DELTA>(grid, st, q, k, v, g, beta, gk, cu, pool, nullptr,
-                                                                  token_slots, num_accepted, pool, scale, eps, out,
-                                                                  nullptr, T, Nqk, Nv);
-    } else if (bf16_pool) {
-        launch_variant<PRE, true, false, true, DECAY, DELTA>(grid, st, q, k, v, g, beta, nullptr, cu, pool, nullptr,
-                                                             token_slots, num_accepted, pool, scale, eps, out,
-                                                             nullptr, T, Nqk, Nv);
-    } else {
-        launch_variant<PRE, true, false, false, DECAY, DELTA>(grid, st, q, k, v, g, beta, nullptr, cu, pool, nullptr,
-                                                              token_slots, num_accepted, pool, scale, eps, out,
-                                                              nullptr, T, Nqk, Nv);
-    }
+    launch_variant<PRE, true, GK, SBF, DECAY, DELTA, DK>(grid, st, a.q, a.k, a.v, a.g, a.beta, a.gk, a.cu, a.pool,
+                                                         nullptr, a.token_slots, a.num_accepted, a.pool, a.scale,
+                                                         a.eps, a.out, nullptr, a.T, a.Nqk, a.Nv, a.Dv);
 }
 
-template <int PRE>
-static void launch_slots(int rule, bool has_gk, bool bf16_pool, dim3 grid, cudaStream_t st, const uint16_t *q,
-                         const uint16_t *k, const uint16_t *v, const float *g, const uint16_t *beta, const float *gk,
-                         const int32_t *cu, void *pool, const int32_t *token_slots, const int32_t *num_accepted,
-                         float scale, float eps, uint16_t *out, int T, int Nqk, int Nv)
+// the pool variants of one staging depth, update rule and key dimension; a key gate only with a decaying rule
+template <int PRE, bool DECAY, bool DELTA, int DK>
+static void launch_rule(const RecArgs &a, bool bf16_pool, dim3 grid, cudaStream_t st)
+{
+    const bool gk = DECAY && a.gk != nullptr;
+    if (gk && bf16_pool) launch_pool<PRE, DECAY, true, DECAY, DELTA, DK>(a, grid, st);
+    else if (gk) launch_pool<PRE, DECAY, false, DECAY, DELTA, DK>(a, grid, st);
+    else if (bf16_pool) launch_pool<PRE, false, true, DECAY, DELTA, DK>(a, grid, st);
+    else launch_pool<PRE, false, false, DECAY, DELTA, DK>(a, grid, st);
+}
+
+template <int PRE, int DK>
+static void launch_slots(const RecArgs &a, int rule, bool bf16_pool, dim3 grid, cudaStream_t st)
 {
     switch (rule) {
-    case kRuleDelta:
-        launch_rule<PRE, false, true>(has_gk, bf16_pool, grid, st, q, k, v, g, beta, gk, cu, pool, token_slots,
-                                      num_accepted, scale, eps, out, T, Nqk, Nv);
-        break;
-    case kRuleGated:
-        launch_rule<PRE, true, false>(has_gk, bf16_pool, grid, st, q, k, v, g, beta, gk, cu, pool, token_slots,
-                                      num_accepted, scale, eps, out, T, Nqk, Nv);
-        break;
-    case kRuleLinear:
-        launch_rule<PRE, false, false>(has_gk, bf16_pool, grid, st, q, k, v, g, beta, gk, cu, pool, token_slots,
-                                       num_accepted, scale, eps, out, T, Nqk, Nv);
-        break;
-    default:
-        launch_rule<PRE, true, true>(has_gk, bf16_pool, grid, st, q, k, v, g, beta, gk, cu, pool, token_slots,
-                                     num_accepted, scale, eps, out, T, Nqk, Nv);
+    case kRuleDelta: launch_rule<PRE, false, true, DK>(a, bf16_pool, grid, st); break;
+    case kRuleGated: launch_rule<PRE, true, false, DK>(a, bf16_pool, grid, st); break;
+    case kRuleLinear: launch_rule<PRE, false, false, DK>(a, bf16_pool, grid, st); break;
+    default: launch_rule<PRE, true, true, DK>(a, bf16_pool, grid, st);
     }
 }
 
@@ -374,28 +377,34 @@ cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v
     if (B == 0) return cudaSuccess;
     const dim3 grid(B, Nv, D / kTile);
     if (max_seqlen >= 1 && max_seqlen <= 8)
-        launch_variant<8, false, false, false, true, true>(grid, st, q, k, v, g, beta, nullptr, cu, pool, idx, nullptr,
-                                                           nullptr, nullptr, scale, eps, out, final_state, T, Nqk, Nv);
+        launch_variant<8, false, false, false, true, true, D>(grid, st, q, k, v, g, beta, nullptr, cu, pool, idx,
+                                                              nullptr, nullptr, nullptr, scale, eps, out, final_state,
+                                                              T, Nqk, Nv, D);
     else
-        launch_variant<16, false, false, false, true, true>(grid, st, q, k, v, g, beta, nullptr, cu, pool, idx,
-                                                            nullptr, nullptr, nullptr, scale, eps, out, final_state, T,
-                                                            Nqk, Nv);
+        launch_variant<16, false, false, false, true, true, D>(grid, st, q, k, v, g, beta, nullptr, cu, pool, idx,
+                                                               nullptr, nullptr, nullptr, scale, eps, out, final_state,
+                                                               T, Nqk, Nv, D);
     return cudaGetLastError();
 }
 
 cudaError_t launch_recurrent(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                              const uint16_t *beta, const float *gk, const int32_t *cu, void *pool, bool bf16_pool,
                              int rule, const int32_t *token_slots, const int32_t *num_accepted, float scale,
-                             float eps, uint16_t *out, int T, int B, int Nqk, int Nv, int max_seqlen, cudaStream_t st)
+                             float eps, uint16_t *out, int T, int B, int Nqk, int Nv, int Dk, int Dv, int max_seqlen,
+                             cudaStream_t st)
 {
     if (B == 0) return cudaSuccess;
-    const dim3 grid(B, Nv, D / kTile);
-    if (max_seqlen >= 1 && max_seqlen <= 8)
-        launch_slots<8>(rule, gk != nullptr, bf16_pool, grid, st, q, k, v, g, beta, gk, cu, pool, token_slots,
-                        num_accepted, scale, eps, out, T, Nqk, Nv);
-    else
-        launch_slots<16>(rule, gk != nullptr, bf16_pool, grid, st, q, k, v, g, beta, gk, cu, pool, token_slots,
-                         num_accepted, scale, eps, out, T, Nqk, Nv);
+    if ((Dk != 64 && Dk != 128) || Dv <= 0 || Dv % kTile != 0) return cudaErrorInvalidValue;
+    const RecArgs a{q, k, v, g, beta, gk, cu, pool, token_slots, num_accepted, scale, eps, out, T, Nqk, Nv, Dv};
+    const dim3 grid(B, Nv, Dv / kTile);
+    const bool few = max_seqlen >= 1 && max_seqlen <= 8;
+    if (Dk == 64) {
+        if (few) launch_slots<8, 64>(a, rule, bf16_pool, grid, st);
+        else launch_slots<16, 64>(a, rule, bf16_pool, grid, st);
+    } else {
+        if (few) launch_slots<8, 128>(a, rule, bf16_pool, grid, st);
+        else launch_slots<16, 128>(a, rule, bf16_pool, grid, st);
+    }
     return cudaGetLastError();
 }
 

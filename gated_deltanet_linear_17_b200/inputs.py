@@ -93,6 +93,10 @@ CONFIGS = {
     # decode step: 256 sequences of one token on a bf16 pool, with the key-dimension gate (key_gate)
     "decode_b256_bf16": dict(lens=[1] * 256, Nqk=16, Nv=32, g=("uniform_neg", 1.0, 0.01),
                              beta=("uniform", 0.05, 0.95), state=("normal", 0.02, 512, "perm"), seed=6),
+    # the decode page's example shape (Dk = 64, Dv = 512, 64 heads), one token for each of 128 sequences
+    "decode_dk64_dv512": dict(lens=[1] * 128, Nqk=64, Nv=64, g=("uniform_neg", 1.0, 0.01),
+                              beta=("uniform", 0.05, 0.95), state=("normal", 0.02, 256, "perm"), seed=7,
+                              Dk=64, Dv=512),
     # speculative decoding: 256 sequences of 4 draft tokens, a pool slot per token (see spec_slots)
     "spec_decode_b256x4": dict(lens=[4] * 256, Nqk=16, Nv=32, g=("uniform_neg", 1.0, 0.01),
                                beta=("uniform", 0.05, 0.95), state=("normal", 0.02, 1024, "perm"), seed=5),
@@ -122,8 +126,9 @@ def _draw_lens(spec, gen):
 
 
 def make(lens, Nqk, Nv, g=("uniform_neg", 0.5, 0.01), beta=("uniform", 0.05, 0.95), state=None,
-         seed=0, name="custom", scale=None, eps=1e-6, device="cpu") -> GdnInputs:
-    """Draw one batch.  See CONFIGS for the recipe keys."""
+         seed=0, name="custom", scale=None, eps=1e-6, device="cpu", Dk=D, Dv=D) -> GdnInputs:
+    """Draw one batch.  See CONFIGS for the recipe keys.  Dk, Dv: head dimensions (the chunked path
+    takes 128 only; the token recurrence on a pool also takes Dk = 64 and other Dv)."""
     gen = torch.Generator().manual_seed(seed)
     seqlens = _draw_lens(lens, gen)
     B = len(seqlens)
@@ -131,9 +136,9 @@ def make(lens, Nqk, Nv, g=("uniform_neg", 0.5, 0.01), beta=("uniform", 0.05, 0.9
     cu = torch.zeros(B + 1, dtype=torch.int32)
     if B:
         cu[1:] = torch.tensor(seqlens, dtype=torch.int64).cumsum(0).to(torch.int32)
-    q = torch.randn(T, Nqk, D, generator=gen).to(torch.bfloat16)
-    k = torch.randn(T, Nqk, D, generator=gen).to(torch.bfloat16)
-    v = torch.randn(T, Nv, D, generator=gen).to(torch.bfloat16)
+    q = torch.randn(T, Nqk, Dk, generator=gen).to(torch.bfloat16)
+    k = torch.randn(T, Nqk, Dk, generator=gen).to(torch.bfloat16)
+    v = torch.randn(T, Nv, Dv, generator=gen).to(torch.bfloat16)
     if g[0] == "uniform_neg":
         gg = -(torch.rand(T, Nv, generator=gen) * g[1] + g[2])
     elif g[0] == "softplus":
@@ -154,7 +159,7 @@ def make(lens, Nqk, Nv, g=("uniform_neg", 0.5, 0.01), beta=("uniform", 0.05, 0.9
     if state is not None:
         _, std, P, mode = state
         P = B if P is None else P
-        pool = torch.randn(P, Nv, D, D, generator=gen) * std
+        pool = torch.randn(P, Nv, Dk, Dv, generator=gen) * std
         if mode == "identity":
             idx = torch.arange(B, dtype=torch.int32)
         elif mode == "perm":
@@ -162,7 +167,7 @@ def make(lens, Nqk, Nv, g=("uniform_neg", 0.5, 0.01), beta=("uniform", 0.05, 0.9
         else:
             raise ValueError(mode)
     if scale is None:
-        scale = 1.0 / math.sqrt(D)
+        scale = 1.0 / math.sqrt(Dk)
     inp = GdnInputs(name, q, k, v, gg.float().contiguous(), bb.to(torch.bfloat16), cu, pool, idx,
                     float(scale), float(eps), seqlens)
     return inp if str(device) == "cpu" else inp.to(device)
@@ -177,7 +182,7 @@ def config(name: str, device="cpu", seed: Optional[int] = None) -> GdnInputs:
 
 
 def key_gate(inp: GdnInputs, seed: int) -> torch.Tensor:
-    """The decode page's key-dimension gate for a batch: gk [T, Nv, 128] fp32 = -(U + 0.01) * 0.5
+    """The decode page's key-dimension gate for a batch: gk [T, Nv, Dk] fp32 = -(U + 0.01) * 0.5
     (the page's example draws -(U + 0.01); the factor keeps e^gk away from tiny values)."""
     gen = torch.Generator().manual_seed(seed)
-    return -(torch.rand(inp.T, inp.Nv, D, generator=gen) + 0.01) * 0.5
+    return -(torch.rand(inp.T, inp.Nv, inp.q.shape[2], generator=gen) + 0.01) * 0.5

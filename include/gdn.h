@@ -182,8 +182,10 @@ int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *
  * Ordinary decoding puts all tokens of sequence b on one slot (its state is
  * then read from and written back to that slot).
  *
- *   q, k, v, g, beta, cu_seqlens   as for gdn_chunk_fwd
- *   gk            device fp32 [T, Nv, 128 (Dk)], the key-dimension gate
+ *   q, k          device bf16 [T, Nqk, Dk]
+ *   v             device bf16 [T, Nv, Dv]
+ *   g, beta, cu_seqlens   as for gdn_chunk_fwd
+ *   gk            device fp32 [T, Nv, Dk], the key-dimension gate
  *                 (expected <= 0, not checked), or NULL for none
  *   update_rule   GDN_RULE_GATED_DELTA (the rule above), GDN_RULE_DELTA (no decay:
  *                 g and gk are not read and may be NULL), GDN_RULE_GATED
@@ -192,7 +194,7 @@ int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *
  *                 not read) -- the update rules of the page "com.microsoft.
  *                 LinearAttention" (update_rule); q and k are normalised in
  *                 every rule
- *   state_pool    device [P, Nv, 128 (Dk), 128 (Dv)], read and written in place
+ *   state_pool    device [P, Nv, Dk, Dv], read and written in place
  *                 (required): fp32 when state_bf16 == 0, bf16 when state_bf16 == 1
  *                 (the page's pool dtype: widened to fp32 on load, the fp32 result
  *                 rounded to nearest even when written)
@@ -200,10 +202,14 @@ int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *
  *                 the slots used by different sequences, including each
  *                 sequence's starting slot, must be disjoint
  *   num_accepted  device int32 [B], or NULL
- *   scale, eps    as for gdn_chunk_fwd
- *   out           device bf16 [T, Nv, 128], written for every token; must not
+ *   scale         query scale; <= 0 selects 1/sqrt(Dk)
+ *   eps           as for gdn_chunk_fwd
+ *   out           device bf16 [T, Nv, Dv], written for every token; must not
  *                 overlap any input or state_pool
  *   T, B, Nqk, Nv, P   sizes (T = cu[B]); Nv % Nqk == 0; P >= 1
+ *   Dk, Dv        key and value head dimensions: Dk 64 or 128, Dv a multiple
+ *                 of 32 up to 1024 (other values: GDN_ERR_UNSUPPORTED); the
+ *                 decode page's example has Dk = 64, Dv = 512
  *   max_seqlen    longest sequence if known, else 0.  At most 8 selects the
  *                 kernel variant that stages 8 tokens per sequence (eight CTAs
  *                 per SM); any other value the one that stages 16.  Every
@@ -222,7 +228,8 @@ int gdn_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, c
                       const uint16_t *beta, const float *gk, const int32_t *cu_seqlens, void *state_pool,
                       int32_t state_bf16, int32_t update_rule, const int32_t *token_slots,
                       const int32_t *num_accepted, float scale, float eps, uint16_t *out, int64_t T, int32_t B,
-                      int32_t Nqk, int32_t Nv, int32_t P, int32_t max_seqlen, void *stream);
+                      int32_t Nqk, int32_t Nv, int32_t Dk, int32_t Dv, int32_t P, int32_t max_seqlen,
+                      void *stream);
 
 #ifdef __cplusplus
 }

@@ -112,13 +112,14 @@ def test_argument_errors_before_any_launch(lib):
 def _call_recurrent(lib, **over):
     M = 1 << 20  # fake, disjoint, aligned addresses; every call below returns before any launch
     a = dict(q=1 * M, k=2 * M, v=3 * M, g=4 * M, beta=5 * M, gk=None, cu=6 * M, pool=9 * M, bf16=0, rule=0,
-             slots=10 * M, acc=None, scale=0.0, eps=1e-6, out=7 * M, T=8, B=1, Nqk=2, Nv=4, P=2, max_seqlen=0,
-             stream=None)
+             slots=10 * M, acc=None, scale=0.0, eps=1e-6, out=7 * M, T=8, B=1, Nqk=2, Nv=4, Dk=128, Dv=128, P=2,
+             max_seqlen=0, stream=None)
     a.update(over)
     vp = lambda x: None if x is None else ctypes.c_void_p(x)
     return lib.gdn_recurrent_fwd(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["g"]), vp(a["beta"]), vp(a["gk"]),
                                  vp(a["cu"]), vp(a["pool"]), a["bf16"], a["rule"], vp(a["slots"]), vp(a["acc"]), a["scale"],
-                                 a["eps"], vp(a["out"]), a["T"], a["B"], a["Nqk"], a["Nv"], a["P"], a["max_seqlen"],
+                                 a["eps"], vp(a["out"]), a["T"], a["B"], a["Nqk"], a["Nv"], a["Dk"], a["Dv"], a["P"],
+                                 a["max_seqlen"],
                                  vp(a["stream"]))
 
 
@@ -130,6 +131,10 @@ def test_recurrent_argument_errors_before_any_launch(lib):
     assert _call_recurrent(lib, Nv=3) == B.GDN_ERR_BAD_SHAPE
     assert _call_recurrent(lib, bf16=2) == B.GDN_ERR_BAD_SHAPE
     assert _call_recurrent(lib, rule=4) == B.GDN_ERR_BAD_SHAPE
+    assert _call_recurrent(lib, Dk=96) == B.GDN_ERR_UNSUPPORTED
+    assert _call_recurrent(lib, Dv=48) == B.GDN_ERR_UNSUPPORTED
+    assert _call_recurrent(lib, Dv=0) == B.GDN_ERR_BAD_SHAPE
+    assert _call_recurrent(lib, Dk=64, Dv=512, slots=10 * M + 2) == B.GDN_ERR_ALIGNMENT  # accepted sizes
     assert _call_recurrent(lib, g=None) == B.GDN_ERR_NULL_ARG             # the gated delta rule reads g
     # rules that do not read g / beta accept NULL there (each call still stops at a later check)
     assert _call_recurrent(lib, beta=None, rule=2, slots=10 * M + 2) == B.GDN_ERR_ALIGNMENT

@@ -20,9 +20,9 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _case(lens, Nqk, Nv, P, seed, per_token, accepted):
+def _case(lens, Nqk, Nv, P, seed, per_token, accepted, Dk=128, Dv=128):
     """Inputs, token slots [T] and accepted counts [B] (None: every token accepted)."""
-    inp = inputs.make(lens, Nqk=Nqk, Nv=Nv, state=("normal", 0.02, P, "perm"), seed=seed)
+    inp = inputs.make(lens, Nqk=Nqk, Nv=Nv, state=("normal", 0.02, P, "perm"), seed=seed, Dk=Dk, Dv=Dv)
     r = np.random.default_rng(seed + 1000)
     cu = inp.cu_seqlens.numpy()
     T, B = int(cu[-1]), len(lens)
@@ -169,3 +169,13 @@ def test_recurrent_gated_rule_key_gate_bf16():
     lens = [int(x) for x in r.integers(1, 5, size=24)]
     inp, slots, acc = _case(lens, Nqk=4, Nv=8, P=32, seed=59, per_token=False, accepted=False)
     _run_and_check(inp, slots, acc, 4, "gated rule, gk, bf16", gk=_key_gate(inp, 60), bf16_pool=True, rule="gated")
+
+
+@pytest.mark.parametrize("Dk,Dv", [(64, 512), (64, 64), (128, 64), (128, 256)])
+def test_recurrent_head_dimensions(Dk, Dv):
+    """Key and value dimensions other than 128 (the decode page's example: Dk = 64, Dv = 512), with the
+    key gate, a bf16 pool, a slot per token and a sequence past the staged tokens."""
+    lens = [1, 4, 2, 19, 3]
+    inp, slots, acc = _case(lens, Nqk=2, Nv=4, P=40, seed=61, per_token=True, accepted=True, Dk=Dk, Dv=Dv)
+    _run_and_check(inp, slots, acc, 0, f"Dk={Dk} Dv={Dv}", gk=_key_gate(inp, 62), bf16_pool=True)
+    _run_and_check(inp, slots, acc, 4, f"Dk={Dk} Dv={Dv} fp32 delta", rule="delta")
