@@ -342,6 +342,26 @@ def main():
             "staged_ms_per_step": staged_ms, "pipeline_ranges": gdn.pipeline_ranges(T, B),
             "gpu_launches": (1 + 3 * gdn.pipeline_ranges(T, B)) * args.steps, "clocks": clocks}
 
+    # ---- the same prefill under the LinearAttention page's other update rules (gdn_chunk_fwd_rule)
+    rule_lines = {}
+    for rule in ("delta", "gated", "linear"):
+        def rstep():
+            gdn.chunk_fwd(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, inp.state_pool, inp.state_indices,
+                          scale=inp.scale, eps=inp.eps, out=out, final_state=fin, workspace=ws, update_rule=rule)
+        for _ in range(args.warmup):
+            rstep()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            rstep()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        rms_ = gdist.max_over_ranks(e0.elapsed_time(e1) / args.steps, device=dev)
+        rule_lines[rule] = {"ms_per_step": rms_, "tokens/s": world * T / (rms_ / 1e3)}
+        line["gpu_launches"] += (1 + 3 * gdn.pipeline_ranges(T, B, inp.Nqk, inp.Nv)) * args.steps
+    line["prefill_update_rules"] = rule_lines
+
     # ---- short-sequence state-pool pass (HBM-bound)
     if not args.no_short:
         sh = inputs.config("short_pool_b256", seed=inputs.CONFIGS["short_pool_b256"]["seed"] + rank).to(dev)

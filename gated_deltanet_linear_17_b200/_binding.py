@@ -24,6 +24,8 @@ GDN_OK, GDN_ERR_NULL_ARG, GDN_ERR_BAD_SHAPE, GDN_ERR_UNSUPPORTED = 0, 1, 2, 3
 GDN_ERR_ALIGNMENT, GDN_ERR_WORKSPACE, GDN_ERR_CUDA, GDN_ERR_OVERLAP = 4, 5, 6, 7
 GDN_ERR_SCRATCH_LIMIT = 8
 NOALLOC_SCRATCH_BYTES = 64 << 20
+# update rules of gdn_chunk_fwd_rule and gdn_recurrent_fwd (GDN_RULE_* in gdn.h)
+UPDATE_RULES = {"gated_delta": 0, "delta": 1, "gated": 2, "linear": 3}
 
 _lib = None
 
@@ -52,6 +54,9 @@ def lib():
         L.gdn_workspace_layout.argtypes = [i64, i32, i32, i32, ctypes.POINTER(_Layout)]
         L.gdn_chunk_fwd.restype = ctypes.c_int
         L.gdn_chunk_fwd.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, i32, p, sz, p]
+        L.gdn_chunk_fwd_rule.restype = ctypes.c_int
+        L.gdn_chunk_fwd_rule.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, i32, i32, p,
+                                         sz, p]
         L.gdn_chunk_fwd_noalloc.restype = ctypes.c_int
         L.gdn_chunk_fwd_noalloc.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, i32, p]
         L.gdn_selftest_umma.restype = ctypes.c_int
@@ -151,14 +156,27 @@ def _resolve(q, k, v, g, beta, cu_seqlens, state_pool, state_indices):
 
 def chunk_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None, scale=None, eps=1e-6,
               max_seqlen: int = 0, out=None, final_state=None, output_final_state=True, workspace=None,
-              stream=None):
-    """Gated Delta Rule forward through ``gdn_chunk_fwd``; returns (out, final_state).
+              stream=None, update_rule="gated_delta"):
+    """Gated Delta Rule forward through ``gdn_chunk_fwd`` (``gdn_chunk_fwd_rule`` for another
+    ``update_rule``: delta, gated or linear); returns (out, final_state).
 
     q, k [T, Nqk, 128] bf16; v [T, Nv, 128] bf16; g [T, Nv] fp32; beta [T, Nv]
     bf16; cu_seqlens [B+1] int32; state_pool [P, Nv, 128, 128] fp32 or None;
     state_indices [B] int32 or None.  All on one CUDA device.  ``max_seqlen``
-    in 1..16 selects the fused short-sequence kernel."""
-    T, B, Nqk, Nv, P, dev = _resolve(q, k, v, g, beta, cu_seqlens, state_pool, state_indices)
+    in 1..16 selects the fused short-sequence kernel.  g is not needed by the
+    delta and linear rules, beta not by the gated and linear rules (pass None)."""
+    if update_rule not in UPDATE_RULES:
+        raise ValueError(f"update_rule must be one of {sorted(UPDATE_RULES)}")
+    rule = UPDATE_RULES[update_rule]
+    if rule in (1, 3):
+        g = None
+    if rule in (2, 3):
+        beta = None
+    if q.dim() != 3 or v.dim() != 3:
+        raise ValueError("q/k must be [T, Nqk, 128] and v [T, Nv, 128]")
+    gg = g if g is not None else torch.empty(q.shape[0], v.shape[1], dtype=torch.float32, device=q.device)
+    bb = beta if beta is not None else torch.empty(q.shape[0], v.shape[1], dtype=torch.bfloat16, device=q.device)
+    T, B, Nqk, Nv, P, dev = _resolve(q, k, v, gg, bb, cu_seqlens, state_pool, state_indices)
     if out is None:
         out = torch.empty(T, Nv, HEAD_DIM, dtype=torch.bfloat16, device=dev)
     else:
@@ -172,10 +190,17 @@ def chunk_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None,
         workspace = torch.empty(workspace_bytes(T, B, Nqk, Nv), dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     sc = 0.0 if scale is None else float(scale)
-    rc = lib().gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), _ptr(state_pool),
-                             _ptr(state_indices), sc, float(eps), _ptr(out), _ptr(final_state), T, B, Nqk, Nv, P,
-                             int(max_seqlen), _ptr(workspace), ws_bytes, _stream(stream))
-    _check(rc, "gdn_chunk_fwd")
+    if rule == 0:
+        rc = lib().gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), _ptr(state_pool),
+                                 _ptr(state_indices), sc, float(eps), _ptr(out), _ptr(final_state), T, B, Nqk, Nv, P,
+                                 int(max_seqlen), _ptr(workspace), ws_bytes, _stream(stream))
+        _check(rc, "gdn_chunk_fwd")
+    else:
+        rc = lib().gdn_chunk_fwd_rule(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+                                      _ptr(state_pool), _ptr(state_indices), sc, float(eps), _ptr(out),
+                                      _ptr(final_state), T, B, Nqk, Nv, P, rule, int(max_seqlen), _ptr(workspace),
+                                      ws_bytes, _stream(stream))
+        _check(rc, "gdn_chunk_fwd_rule")
     return out, final_state
 
 
@@ -221,9 +246,6 @@ def short_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None,
                              _stream(stream))
     _check(rc, "gdn_short_fwd")
     return out, final_state
-
-
-UPDATE_RULES = {"gated_delta": 0, "delta": 1, "gated": 2, "linear": 3}
 
 
 def recurrent_fwd(q, k, v, g, beta, cu_seqlens, state_pool, token_slots, num_accepted=None, scale=None, eps=1e-6,

@@ -240,7 +240,7 @@ __device__ __forceinline__ void chunk_gamma(const float *__restrict__ g, int Nv,
                                             float *wsum)
 {
     const int tid = threadIdx.x;
-    chunk_gamma_x((tid < 128 && tid < n) ? g[(size_t)(t0 + tid) * Nv + h] : 0.f, gam, wsum);
+    chunk_gamma_x((g && tid < 128 && tid < n) ? g[(size_t)(t0 + tid) * Nv + h] : 0.f, gam, wsum);  // g null: zero
 }
 
 // Largest gate span gamma_first - gamma_last of a 16-row block for which a row's

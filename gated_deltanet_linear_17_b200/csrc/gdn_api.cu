@@ -338,14 +338,30 @@ int gdn_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
                   float *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
                   int32_t max_seqlen, void *workspace, size_t workspace_bytes, void *stream)
 {
+    return gdn_chunk_fwd_rule(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, scale, eps, out, final_state,
+                              T, B, Nqk, Nv, P, GDN_RULE_GATED_DELTA, max_seqlen, workspace, workspace_bytes, stream);
+}
+
+int gdn_chunk_fwd_rule(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                       const uint16_t *beta, const int32_t *cu_seqlens, const float *state_pool,
+                       const int32_t *state_indices, float scale, float eps, uint16_t *out,
+                       float *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
+                       int32_t update_rule, int32_t max_seqlen, void *workspace, size_t workspace_bytes,
+                       void *stream)
+{
+    if (update_rule < GDN_RULE_GATED_DELTA || update_rule > GDN_RULE_LINEAR) return GDN_ERR_BAD_SHAPE;
+    const bool decay = update_rule == GDN_RULE_GATED_DELTA || update_rule == GDN_RULE_GATED;
+    const bool delta = update_rule == GDN_RULE_GATED_DELTA || update_rule == GDN_RULE_DELTA;
+    if (!decay) g = nullptr;  // a zero gate
+    if (!delta) beta = nullptr;
     int rc = check_forward(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, out, final_state, T, B,
-                           Nqk, Nv, P);
+                           Nqk, Nv, P, decay, delta);
     if (rc || B == 0) return rc;
     const cudaStream_t st = (cudaStream_t)stream;
     const float sc = resolve_scale(scale);
     if (max_seqlen >= 1 && max_seqlen <= GDN_SHORT_MAX)
         return cuda_status(gdn::launch_short(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, sc, eps,
-                                             out, final_state, (int)T, B, Nqk, Nv, max_seqlen, st));
+                                             out, final_state, (int)T, B, Nqk, Nv, max_seqlen, st, update_rule));
 
     gdn_workspace_layout_t lay;
     if ((rc = fill_layout(T, B, Nqk, Nv, &lay))) return rc;
@@ -362,10 +378,10 @@ int gdn_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
     cudaError_t e = gdn::launch_chunk_map(cu_seqlens, B, Ti, NC, w, st);
     const int R = gdn::pipeline_ranges(NC);
     if (e == cudaSuccess && R == 1) {
-        e = gdn::launch_intra(k, v, g, beta, eps, Ti, Nqk, Nv, 0, NC, w, st);
+        e = gdn::launch_intra(k, v, g, beta, eps, Ti, Nqk, Nv, 0, NC, w, st, delta);
         if (e == cudaSuccess)
-            e = gdn::launch_state(k, state_pool, state_indices, final_state, Ti, B, Nqk, Nv, 0, NC, 0, w, st);
-        if (e == cudaSuccess) e = gdn::launch_output(q, k, g, sc, eps, out, Ti, Nqk, Nv, 0, NC, w, st);
+            e = gdn::launch_state(k, state_pool, state_indices, final_state, Ti, B, Nqk, Nv, 0, NC, 0, w, st, delta);
+        if (e == cudaSuccess) e = gdn::launch_output(q, k, g, sc, eps, out, Ti, Nqk, Nv, 0, NC, w, st, delta);
     } else if (e == cudaSuccess) {
         std::lock_guard<std::mutex> guard(g_pipe_lock);
         SideStreams *ss = nullptr;
@@ -380,19 +396,20 @@ int gdn_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
             if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->intra, ev[0], 0);
             if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->state, ev[0], 0);
             for (int r = 0; r < R && e == cudaSuccess; ++r) {
-                e = gdn::launch_intra(k, v, g, beta, eps, Ti, Nqk, Nv, c0(r), c1(r) - c0(r), w, ss->intra);
+                e = gdn::launch_intra(k, v, g, beta, eps, Ti, Nqk, Nv, c0(r), c1(r) - c0(r), w, ss->intra, delta);
                 if (e == cudaSuccess) e = cudaEventRecord(ev[1 + r], ss->intra);
             }
             for (int r = 0; r < R && e == cudaSuccess; ++r) {
                 e = cudaStreamWaitEvent(ss->state, ev[1 + r], 0);
                 if (e == cudaSuccess)
                     e = gdn::launch_state(k, state_pool, state_indices, final_state, Ti, B, Nqk, Nv, c0(r), c1(r), r,
-                                          w, ss->state);
+                                          w, ss->state, delta);
                 if (e == cudaSuccess) e = cudaEventRecord(ev[1 + R + r], ss->state);
             }
             for (int r = 0; r < R && e == cudaSuccess; ++r) {
                 e = cudaStreamWaitEvent(st, ev[1 + R + r], 0);
-                if (e == cudaSuccess) e = gdn::launch_output(q, k, g, sc, eps, out, Ti, Nqk, Nv, c0(r), c1(r) - c0(r), w, st);
+                if (e == cudaSuccess)
+                    e = gdn::launch_output(q, k, g, sc, eps, out, Ti, Nqk, Nv, c0(r), c1(r) - c0(r), w, st, delta);
             }
             // join, also after a failed launch, so that nothing of this call runs outside `st` afterwards
             cudaError_t j = cudaEventRecord(ev[1 + 2 * R], ss->intra);

@@ -45,17 +45,19 @@ cudaError_t launch_chunk_map(const int32_t *cu, int B, int T, int NC, const Work
                              cudaStream_t st);
 // intra and output run over chunks [c0, c0 + nc); the state pass over [c_lo, c_hi), range index `range`
 cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, const float *g, const uint16_t *beta, float eps, int T,
-                         int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st);
+                         int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st, bool delta = true);
 cudaError_t launch_state(const uint16_t *k, const float *pool, const int32_t *idx, float *final_state, int T, int B,
-                         int Nqk, int Nv, int c_lo, int c_hi, int range, const Workspace &ws, cudaStream_t st);
+                         int Nqk, int Nv, int c_lo, int c_hi, int range, const Workspace &ws, cudaStream_t st, bool delta = true);
 cudaError_t launch_output(const uint16_t *q, const uint16_t *k, const float *g, float scale, float eps, uint16_t *out,
-                          int T, int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st);
+                          int T, int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st, bool delta = true);
+// delta == false (launch_intra / launch_state / launch_output): an update rule without the
+// retrieval (U = v, no W or Mk); g == nullptr: a zero gate.
 // Fused short-sequence kernel: sequence b starts from pool[idx ? idx[b] : b] (or
 // zero without a pool) and ends in final_state[b].
 cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                          const uint16_t *beta, const int32_t *cu, const float *pool, const int32_t *idx, float scale,
                          float eps, uint16_t *out, float *final_state, int T, int B, int Nqk, int Nv, int max_seqlen,
-                         cudaStream_t st);
+                         cudaStream_t st, int rule = 0);
 // The same kernel on a pool updated in place (fp32, or bf16 when bf16_pool), one slot per token,
 // the start taken from the last accepted token's slot; key dimension Dk (64 or 128), value dimension
 // Dv (a multiple of 32); gk [T, Nv, Dk] or nullptr (read only by the decaying rules).

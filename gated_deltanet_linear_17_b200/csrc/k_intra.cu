@@ -30,7 +30,10 @@
 // product runs, the CTA loads the next item's k rows into the tile that held T
 // and U (the two tiles swap roles) and, once Mk is done, its v rows; the next
 // item's gate and beta values are fetched into registers at the start of the
-// current one.  Each wait is bounded; if one gives up, the CTA sets bit 2 of
+// current one.  For an update rule without the retrieval (`delta` = 0: the
+// LinearAttention page's gated and linear rules) the CTA takes one item, stores
+// U = v in fp16 and the factor records, and skips T, W and Mk.  Each wait is
+// bounded; if one gives up, the CTA sets bit 2 of
 // status[2], lets its MMAs and open loads drain and stops.
 #include "common.cuh"
 #include "gdn_internal.h"
@@ -145,7 +148,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     const __grid_constant__ CUtensorMap tm_mk, const float *__restrict__ g, const uint16_t *__restrict__ beta,
     float eps, int T, int Nqk, int Nv, const int4 *__restrict__ info, float *__restrict__ rk_out,
     float *__restrict__ gcum_out, float *__restrict__ betaf_out, float *__restrict__ fa, int32_t *__restrict__ status,
-    int c0, int nc)
+    int c0, int nc, int delta)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
@@ -199,9 +202,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     }
     // this thread's gate and beta of the current item (threads 0..127, zero past the chunk)
     float xg = 0.f, xb = 0.f;
-    if (tid < 128 && tid < ci.len) {
-        xg = g[(size_t)(ci.start + tid) * Nv + h];
-        xb = bf2f(beta[(size_t)(ci.start + tid) * Nv + h]);
+    if (tid < 128 && tid < ci.len) {  // g == nullptr: a zero gate; beta == nullptr: not read (no retrieval)
+        xg = g ? g[(size_t)(ci.start + tid) * Nv + h] : 0.f;
+        xb = beta ? bf2f(beta[(size_t)(ci.start + tid) * Nv + h]) : 0.f;
     }
     bool ok = true;
     uint32_t mma_phase = 0, v_par = 0, ld_par = 0;
@@ -239,8 +242,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
             const int nh = nit / nc;
             const ChunkInfo nci = load_chunk(info, c0 + nit % nc);
             if (tid < 128 && tid < nci.len) {
-                ng = g[(size_t)(nci.start + tid) * Nv + nh];
-                nb = bf2f(beta[(size_t)(nci.start + tid) * Nv + nh]);
+                ng = g ? g[(size_t)(nci.start + tid) * Nv + nh] : 0.f;
+                nb = beta ? bf2f(beta[(size_t)(nci.start + tid) * Nv + nh]) : 0.f;
             }
         }
         // chunk-local cumulative gate and beta while the rows load
@@ -293,6 +296,37 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
             if (tid < n && h % grp == 0) rk_out[(size_t)hq * T + t0 + tid] = rkv[tid];
         }
         __syncthreads();
+
+        if (!delta) {
+            // An update rule without the retrieval (the LinearAttention page's gated and linear rules):
+            // S_new = e^{g_last} S + k_gexp^T v and o = Q'S + P v, so U = v in fp16 (rows past the chunk
+            // zero) and there is no T, W or Mk.  One item per CTA in this mode.
+            if (ok) wait_bar(bar_v, v_par);
+            if (ok) {
+                v_pend = false;
+                scale_rows_f16<kIntraThreads>(smem + OFF_T1, tid, n, [&](int) { return 1.f; });
+                if (tid < kFaStride) {
+                    const float gl = gam[127];
+                    fa[(size_t)(c * Nv + h) * kFaStride + tid] =
+                        tid < 128 ? rkv[tid] * __expf(gl - gam[tid]) : (tid == 128 ? __expf(gl) : 0.f);
+                }
+            }
+            tc::fence_proxy_async();
+            __syncthreads();
+            if (ok && tid == 0) {
+                const int urow = (c * Nv + h) * L;
+                tma::store_2d(&tm_u, 0, urow, sbase + OFF_T1);
+                tma::store_2d(&tm_u, 64, urow, sbase + OFF_T1 + 16384);
+                tma::commit_group();
+            } else if (!ok && tid == 0) {
+                atomicOr(status + 2, 4);
+                tc::commit(bar_d);
+                tc::mbar_wait_bounded(bar_d, 0);
+                if (ld_pend) tc::mbar_wait_bounded(bar_ld, ld_par);
+                if (v_pend) tc::mbar_wait_bounded(bar_v, v_par);
+            }
+            break;
+        }
 
         // ---- (2) Ap = -strict_tril(diag(beta rk) (k k^T) diag(rk) (.) Gamma): this thread's row and 64 columns.
         // Blocks left of the row's diagonal 16-block go to the A tile in fp16; the diagonal block goes to the
@@ -614,7 +648,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
 }
 
 cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, const float *g, const uint16_t *beta, float eps, int T,
-                         int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st)
+                         int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st, bool delta)
 {
     if (nc <= 0 || T == 0) return cudaSuccess;
     if (c0 < 0 || c0 + nc > ws.NC) return cudaErrorInvalidValue;
@@ -637,10 +671,11 @@ cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, const float *g, c
     e = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kIntraSmem);
     if (e != cudaSuccess) return e;
     const int items = nc * Nv;  // below 2^31: nc Nv L rows are addressable
-    const int grid = (items + kIntraItemsPerCta - 1) / kIntraItemsPerCta;
+    const int per = delta ? kIntraItemsPerCta : 1;
+    const int grid = (items + per - 1) / per;
     intra_kernel<<<grid, kIntraThreads, kIntraSmem, st>>>(m_k, m_v, m_u, m_w, m_mk, g, beta, eps, T, Nqk, Nv,
                                                            ws.chunk_info, ws.rk, ws.gcum, ws.betaf, ws.fa, ws.status,
-                                                           c0, nc);
+                                                           c0, nc, delta ? 1 : 0);
     return cudaGetLastError();
 }
 

@@ -33,6 +33,9 @@
 //   5. O in bf16 is staged over the consumed Qw tile and leaves by TMA for a
 //      full chunk; a short chunk's rows are stored by the threads, so rows of
 //      the next sequence are never written.
+// For an update rule without the retrieval (`delta` = 0: the LinearAttention
+// page's gated and linear rules) W is zero: it is not loaded, Z is not formed and
+// Qw = diag(rq e^gamma) q.
 // One thread issues the MMAs and copies and waits for their completion
 // (mbarriers, bounded waits); a CTA barrier passes the outcome on.  If a wait
 // gives up, the CTA sets bit 1 of status[2] in the workspace and skips the rest
@@ -62,7 +65,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sc,
     const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_out, uint16_t *__restrict__ out,
     const float *__restrict__ g, float scale, float eps, int T, int Nqk, int Nv, const int4 *__restrict__ info,
-    float *__restrict__ rq_out, int32_t *__restrict__ status, int c0)
+    float *__restrict__ rq_out, int32_t *__restrict__ status, int c0, int delta)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
@@ -100,9 +103,11 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         tma::load_2d(sbase + OO_Q + 16384, &tm_q, hq * D + 64, t0, bar_ld);
         tma::load_2d(sbase + OO_K, &tm_k, hq * D, t0, bar_ld);
         tma::load_2d(sbase + OO_K + 16384, &tm_k, hq * D + 64, t0, bar_ld);
-        tma::expect_tx(bar_w, 32768);
-        tma::load_2d(sbase + OO_X, &tm_w, 0, trow, bar_w);
-        tma::load_2d(sbase + OO_X + 16384, &tm_w, 64, trow, bar_w);
+        if (delta) {  // W enters only the rules with the retrieval
+            tma::expect_tx(bar_w, 32768);
+            tma::load_2d(sbase + OO_X, &tm_w, 0, trow, bar_w);
+            tma::load_2d(sbase + OO_X + 16384, &tm_w, 64, trow, bar_w);
+        }
     }
     // chunk-local cumulative gate while the rows load
     chunk_gamma(g, Nv, h, t0, n, gam, reinterpret_cast<float *>(smem + OO_BAR + 32));
@@ -249,15 +254,15 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         if (tid == 0) {
             load_tile(sbase + OO_K, &tm_sc, bar_s);
             s_issued = true;
-            w_ok = tc::mbar_wait_bounded(bar_w, 0);  // W has landed
-            if (w_ok) {
+            if (delta) w_ok = tc::mbar_wait_bounded(bar_w, 0);  // W has landed
+            if (w_ok && delta) {
                 const uint64_t dw = tc::desc_mn(sbase + OO_X, 16384, 1024, 2);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_f16_ts(tmem, tmem + 128 + kk * 8, dw + (uint64_t)((kk * 2048) >> 4), idesc_n128,
                                    kk > 0 ? 1u : 0u);
             }
-            tc::commit(bar_mma);
+            tc::commit(bar_mma);  // (without the retrieval nothing new: the phase closes at once)
             w_ok = tc::mbar_wait_bounded(bar_mma, 1) && w_ok;  // second phase of bar_mma
         }
         tc::fence_before_sync();
@@ -273,7 +278,12 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
 #pragma unroll 1
         for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
             float z[32];
-            tc::tmem_ld32(t_row + j0, z);
+            if (delta) {
+                tc::tmem_ld32(t_row + j0, z);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) z[e] = 0.f;
+            }
             uint4 qv[4];
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) qv[c4] = *reinterpret_cast<const uint4 *>(smem + OO_Q + t128(row, (j0 >> 3) + c4));
@@ -356,7 +366,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         tc::commit(bar_d);
         tc::mbar_wait_bounded(bar_d, 0);
         tc::mbar_wait_bounded(bar_ld, 0);
-        tc::mbar_wait_bounded(bar_w, 0);
+        if (delta) tc::mbar_wait_bounded(bar_w, 0);
         if (s_issued) tc::mbar_wait_bounded(bar_s, 0);
         if (u_issued) tc::mbar_wait_bounded(bar_u, 0);
     }
@@ -368,7 +378,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
 }
 
 cudaError_t launch_output(const uint16_t *q, const uint16_t *k, const float *g, float scale, float eps, uint16_t *out,
-                          int T, int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st)
+                          int T, int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st, bool delta)
 {
     if (nc <= 0 || T == 0) return cudaSuccess;
     if (c0 < 0 || c0 + nc > ws.NC) return cudaErrorInvalidValue;
@@ -387,7 +397,8 @@ cudaError_t launch_output(const uint16_t *q, const uint16_t *k, const float *g, 
     e = cudaFuncSetAttribute(output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
     if (e != cudaSuccess) return e;
     output_kernel<<<dim3(nc, Nv), kOutThreads, kOutSmem, st>>>(m_q, m_k, m_w, m_sc, m_u, m_out, out, g, scale, eps, T,
-                                                                Nqk, Nv, ws.chunk_info, ws.rq, ws.status, c0);
+                                                                Nqk, Nv, ws.chunk_info, ws.rq, ws.status, c0,
+                                                                delta ? 1 : 0);
     return cudaGetLastError();
 }
 

@@ -40,6 +40,8 @@
 // decay: g and gk unused), gated (S = e^g S + kh v^T: no retrieval, beta unused)
 // and linear (S = S + kh v^T); without the retrieval a token needs one barrier.
 #include "common.cuh"
+
+#include <type_traits>
 #include "gdn_internal.h"
 
 namespace gdn {
@@ -372,18 +374,26 @@ static void launch_slots(const RecArgs &a, int rule, bool bf16_pool, dim3 grid, 
 cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                          const uint16_t *beta, const int32_t *cu, const float *pool, const int32_t *idx, float scale,
                          float eps, uint16_t *out, float *final_state, int T, int B, int Nqk, int Nv, int max_seqlen,
-                         cudaStream_t st)
+                         cudaStream_t st, int rule)
 {
     if (B == 0) return cudaSuccess;
     const dim3 grid(B, Nv, D / kTile);
-    if (max_seqlen >= 1 && max_seqlen <= 8)
-        launch_variant<8, false, false, false, true, true, D>(grid, st, q, k, v, g, beta, nullptr, cu, pool, idx,
-                                                              nullptr, nullptr, nullptr, scale, eps, out, final_state,
-                                                              T, Nqk, Nv, D);
-    else
-        launch_variant<16, false, false, false, true, true, D>(grid, st, q, k, v, g, beta, nullptr, cu, pool, idx,
-                                                               nullptr, nullptr, nullptr, scale, eps, out, final_state,
-                                                               T, Nqk, Nv, D);
+    const bool few = max_seqlen >= 1 && max_seqlen <= 8;
+    auto go = [&](auto pre, auto decay, auto delta) {
+        launch_variant<decltype(pre)::value, false, false, false, decltype(decay)::value, decltype(delta)::value, D>(
+            grid, st, q, k, v, g, beta, nullptr, cu, pool, idx, nullptr, nullptr, nullptr, scale, eps, out, final_state,
+            T, Nqk, Nv, D);
+    };
+    using P8 = std::integral_constant<int, 8>;
+    using P16 = std::integral_constant<int, 16>;
+    using Y = std::true_type;
+    using N = std::false_type;
+    switch (rule) {
+    case kRuleDelta: few ? go(P8{}, N{}, Y{}) : go(P16{}, N{}, Y{}); break;
+    case kRuleGated: few ? go(P8{}, Y{}, N{}) : go(P16{}, Y{}, N{}); break;
+    case kRuleLinear: few ? go(P8{}, N{}, N{}) : go(P16{}, N{}, N{}); break;
+    default: few ? go(P8{}, Y{}, Y{}) : go(P16{}, Y{}, Y{});
+    }
     return cudaGetLastError();
 }
 

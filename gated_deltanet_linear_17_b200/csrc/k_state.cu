@@ -34,7 +34,10 @@
 // One launch passes the chunks in a range [c_lo, c_hi): the forward pass runs
 // the ranges one after another on a stream of its own (so that the other
 // kernels of neighbouring ranges run beside it), and a sequence that crosses a
-// range boundary carries its fp32 state through a workspace slot.
+// range boundary carries its fp32 state through a workspace slot.  For an update
+// rule without the retrieval (the LinearAttention page's gated and linear rules,
+// `delta` = 0) the chain has no Mk S term: S_{c+1} = e^{g_last} S_c + Kt_c, and
+// neither Mk nor its product is loaded or issued.
 // The k rows of a chunk that ends before 128 tokens are zeroed after their TMA
 // load, so the next sequence's rows never enter a product.  Every wait is
 // bounded: if one gives up, the CTA sets bit 0 of status[2] in the workspace,
@@ -80,7 +83,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
     const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_sc,
     const float *__restrict__ pool, const int32_t *__restrict__ idx, float *__restrict__ final_state, int Nqk,
     int Nv, const int4 *__restrict__ info, const int32_t *__restrict__ seq_chunk0, const float *__restrict__ fa,
-    int32_t *__restrict__ status, int c_lo, int c_hi, int range, float *__restrict__ carry)
+    int32_t *__restrict__ status, int c_lo, int c_hi, int range, float *__restrict__ carry, int delta)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
@@ -124,9 +127,11 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
         const uint32_t base = sbase + st * kStage, full = bar_full + 8 * st;
         const int trow = (c * Nv + h) * L;  // first row of the chunk's tiles in the workspace
         const int cstart = seq_t0 + (c - c_begin) * L;
-        tma::expect_tx(full, kStageTx);
-        tma::load_2d(base + SG_MK, &tm_mk, 0, trow, full);
-        tma::load_2d(base + SG_MK + 16384, &tm_mk, 64, trow, full);
+        tma::expect_tx(full, delta ? kStageTx : kStageTx - 32768);
+        if (delta) {  // Mk enters only the rules with the retrieval
+            tma::load_2d(base + SG_MK, &tm_mk, 0, trow, full);
+            tma::load_2d(base + SG_MK + 16384, &tm_mk, 64, trow, full);
+        }
         tma::load_2d(base + SG_K, &tm_k, hq * D, cstart, full);
         tma::load_2d(base + SG_K + 16384, &tm_k, hq * D + 64, cstart, full);
         tma::load_2d(base + SG_U, &tm_u, col0, trow, full);
@@ -243,11 +248,13 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
             if (lane == 0) {
                 if (it == 0) issue_kt(0);  // the first chunk's Kt, before its chain product
                 const uint64_t so = (uint64_t)((st * kStage) >> 4), sb = (uint64_t)((st * 16384) >> 4);
+                if (delta) {
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_f16(tmem + st * 128, dMk0 + so + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                                dS0 + sb + (uint64_t)((kk * 2048) >> 4), idesc_mk, 1u);
-                tc::commit(bar_m);
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_f16(tmem + st * 128, dMk0 + so + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                                    dS0 + sb + (uint64_t)((kk * 2048) >> 4), idesc_mk, 1u);
+                }
+                tc::commit(bar_m);  // chunk c's products: Kt (issued before) and -Mk S
                 issued = true;
             }
             __syncwarp();
@@ -319,7 +326,8 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
 }
 
 cudaError_t launch_state(const uint16_t *k, const float *pool, const int32_t *idx, float *final_state, int T, int B,
-                         int Nqk, int Nv, int c_lo, int c_hi, int range, const Workspace &ws, cudaStream_t st)
+                         int Nqk, int Nv, int c_lo, int c_hi, int range, const Workspace &ws, cudaStream_t st,
+                         bool delta)
 {
     if (B == 0) return cudaSuccess;
     if (range < 0 || range >= kMaxRanges || c_lo < 0 || c_hi < c_lo) return cudaErrorInvalidValue;
@@ -344,7 +352,7 @@ cudaError_t launch_state(const uint16_t *k, const float *pool, const int32_t *id
     if (e != cudaSuccess) return e;
     state_kernel<<<dim3(B, Nv, D / DVT), kStateThreads, kStateSmem, st>>>(
         m_mk, m_k, m_u, m_sc, pool, idx, final_state, Nqk, Nv, ws.chunk_info, ws.seq_chunk0, ws.fa, ws.status, c_lo,
-        c_hi, range, ws.carry);
+        c_hi, range, ws.carry, delta ? 1 : 0);
     return cudaGetLastError();
 }
 

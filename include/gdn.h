@@ -51,7 +51,7 @@ extern "C" {
 #define GDN_SHORT_MAX 16 /* max_seqlen at or below which the fused short-sequence kernel runs */
 #define GDN_NOALLOC_SCRATCH_BYTES (64u << 20) /* static workspace of gdn_chunk_fwd_noalloc, per GPU */
 
-/* update rules of gdn_recurrent_fwd */
+/* update rules of gdn_chunk_fwd_rule and gdn_recurrent_fwd */
 #define GDN_RULE_GATED_DELTA 0
 #define GDN_RULE_DELTA 1
 #define GDN_RULE_GATED 2
@@ -122,6 +122,30 @@ int gdn_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
                   const int32_t *state_indices, float scale, float eps, uint16_t *out,
                   float *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
                   int32_t max_seqlen, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * gdn_chunk_fwd_rule -- gdn_chunk_fwd with the update rule of the page
+ * "com.microsoft.LinearAttention" (attribute update_rule) as an argument;
+ * gdn_chunk_fwd is this call with GDN_RULE_GATED_DELTA.
+ *
+ *   update_rule   GDN_RULE_GATED_DELTA   S = e^g S + k (beta (v - S^T k))^T
+ *                 GDN_RULE_DELTA         S = S + k (beta (v - S^T k))^T; g not read (may be NULL)
+ *                 GDN_RULE_GATED         S = e^g S + k v^T; beta not read (may be NULL)
+ *                 GDN_RULE_LINEAR        S = S + k v^T; g and beta not read
+ *                 q and k are L2-normalised in every rule; o = S^T q after the update.
+ *
+ * The chunked form of the rules without the retrieval (gated, linear) has no
+ * triangular inverse: U = V, W = 0, so S_new = e^{g_last} S + k_gexp^T V and
+ * o = (e^gamma Q) S + P V; the kernels skip the products with W and Mk.  Every
+ * other argument, limit and error as for gdn_chunk_fwd; an update_rule outside
+ * 0..3 is GDN_ERR_BAD_SHAPE.
+ */
+int gdn_chunk_fwd_rule(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                       const uint16_t *beta, const int32_t *cu_seqlens, const float *state_pool,
+                       const int32_t *state_indices, float scale, float eps, uint16_t *out,
+                       float *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
+                       int32_t update_rule, int32_t max_seqlen, void *workspace, size_t workspace_bytes,
+                       void *stream);
 
 /*
  * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd for callers that cannot allocate
