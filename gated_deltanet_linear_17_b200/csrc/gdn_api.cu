@@ -304,7 +304,8 @@ int gdn_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, c
     if (update_rule < GDN_RULE_GATED_DELTA || update_rule > GDN_RULE_LINEAR) return GDN_ERR_BAD_SHAPE;
     if (P <= 0 || (state_bf16 != 0 && state_bf16 != 1)) return GDN_ERR_BAD_SHAPE;
     if (Dk <= 0 || Dv <= 0) return GDN_ERR_BAD_SHAPE;
-    if ((Dk != 64 && Dk != 128) || Dv % 32 != 0 || Dv > 1024) return GDN_ERR_UNSUPPORTED;
+    if ((Dk != 64 && Dk != 128) || Dv % 32 != 0 || Dv > 1024 || (state_bf16 && Dv % 64 != 0))
+        return GDN_ERR_UNSUPPORTED;
     if (B == 0) return GDN_OK;
     const bool decay = update_rule == GDN_RULE_GATED_DELTA || update_rule == GDN_RULE_GATED;
     const bool delta = update_rule == GDN_RULE_GATED_DELTA || update_rule == GDN_RULE_DELTA;

@@ -1,4 +1,5 @@
-// Fused short-sequence forward: one CTA per (sequence, v-head, 32-column slice of Dv).
+// Fused short-sequence forward: one CTA per (sequence, v-head, 32-column slice of Dv;
+// 64 columns with a bf16 pool).
 //
 // The decode page ("lite_boost.ops.recurrent_gated_delta_rule", algorithm
 // flow) runs the Gated Delta Rule token by token for a few tokens per call,
@@ -49,12 +50,14 @@ namespace gdn {
 constexpr int kTile = 32;  // Dv columns per CTA
 
 // DK: key dimension (64 or 128); the CTA has DK threads, warp w holding state rows 32w .. 32w + 31
-template <int PRE, bool GK, int DK>  // tokens staged together with the state; key gate
+// SBF: a bf16 pool; the CTA then covers 64 columns, its slice staged in shared memory (sst)
+template <int PRE, bool GK, int DK, bool SBF>  // tokens staged together with the state; key gate
 struct ShortSmem {
     float kh[PRE][DK], qh[PRE][DK];   // normalised rows, fp32 (qh includes the scale)
     float gkd[GK ? PRE : 1][DK];      // gk rows, then the row decays e^{g + gk} (GK)
+    uint16_t sst[SBF ? DK : 1][SBF ? 64 : 8];  // the bf16 state slice (SBF)
     uint16_t q[PRE][DK], k[PRE][DK];  // raw bf16 rows
-    uint16_t v[PRE][kTile];           // raw bf16 slice
+    uint16_t v[PRE][SBF ? 64 : 32];   // raw bf16 slice
     float g[PRE], dg[PRE], beta[PRE];
     int32_t slot[PRE + 1];  // token slots (SLOTS)
     float red[2][DK / 32][32], red2[2][DK / 32][32];
@@ -79,10 +82,14 @@ __global__ void __launch_bounds__(DK) short_kernel(
     float eps, uint16_t *__restrict__ out, float *__restrict__ final_state, int T, int Nqk, int Nv, int Dv)
 {
     constexpr int NW = DK / 32, EL = DK / 32;  // warps; elements of a q/k row per lane
-    __shared__ __align__(16) ShortSmem<PRE, GK, DK> sm;
+    // Dv columns per CTA: with a bf16 pool 64, the slice (16 KiB at Dk = 128) fetched by cp.async into
+    // shared memory and the tokens applied to one 32-column half after the other, so a CTA keeps twice
+    // the bytes in flight with the same registers
+    constexpr int CW = SBF ? 64 : 32;
+    __shared__ __align__(16) ShortSmem<PRE, GK, DK, SBF> sm;
     const int b = blockIdx.x, h = blockIdx.y, tl = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int col = tl * kTile + lane;
+    int col = tl * CW + lane;
     const int hq = h / (Nv / Nqk);
     const int t0 = min(max(cu[b], 0), T);
     const int t1 = min(max(cu[b + 1], t0), T);
@@ -96,9 +103,9 @@ __global__ void __launch_bounds__(DK) short_kernel(
         cp_async16(smem_addr(&sm.q[t][c * 8]), q + off, true);
         cp_async16(smem_addr(&sm.k[t][c * 8]), k + off, true);
     }
-    for (int e = tid; e < npre * 4; e += DK) {
-        const int t = e >> 2, c = e & 3;
-        cp_async16(smem_addr(&sm.v[t][c * 8]), v + ((size_t)(t0 + t) * Nv + h) * Dv + tl * kTile + c * 8, true);
+    for (int e = tid; e < npre * (CW / 8); e += DK) {
+        const int t = e / (CW / 8), c = e % (CW / 8);
+        cp_async16(smem_addr(&sm.v[t][c * 8]), v + ((size_t)(t0 + t) * Nv + h) * Dv + tl * CW + c * 8, true);
     }
     if (DECAY && tid < npre) cp_async4(smem_addr(&sm.g[tid]), g + (size_t)(t0 + tid) * Nv + h);
     if (SLOTS && tid <= PRE && tid < n) cp_async4(smem_addr(&sm.slot[tid]), token_slots + t0 + tid);
@@ -108,27 +115,33 @@ __global__ void __launch_bounds__(DK) short_kernel(
             cp_async16(smem_addr(&sm.gkd[t][c * 4]), gk + ((size_t)(t0 + t) * Nv + h) * DK + c * 4, true);
         }
     }
+    // the starting slot
+    int slot0 = 0;
+    if (pool) {
+        if (SLOTS) {  // the state after the last accepted token (n >= 1 here)
+            const int a = min(max(num_accepted ? num_accepted[b] : n, 1), n);
+            slot0 = token_slots[t0 + a - 1];
+        } else {
+            slot0 = idx ? idx[b] : b;
+        }
+    }
+    if (SBF && pool) {  // the bf16 slice [DK][64] (128-byte row segments) into shared memory
+        const unsigned short *src = static_cast<const unsigned short *>(pool) + ((size_t)slot0 * Nv + h) * DK * Dv + tl * CW;
+        for (int e = tid; e < DK * 8; e += DK) {
+            const int r = e >> 3, c = e & 7;
+            cp_async16(smem_addr(&sm.sst[r][c * 8]), src + (size_t)r * Dv + c * 8, true);
+        }
+    }
     cp_async_commit();
     float bt_mine = 0.f;
     if (DELTA && tid < npre) bt_mine = bf2f(beta[(size_t)(t0 + tid) * Nv + h]);
 
-    // the state slice, straight into registers: s2[m] holds rows 32 wid + 2m, 2m + 1
+    // fp32 pool: the state slice straight into registers, s2[m] holding rows 32 wid + 2m, 2m + 1
+    // (bf16 pool: from shared memory, one half at a time, below)
     float2 s2[16];
-    if (pool) {
-        int slot;
-        if (SLOTS) {  // the state after the last accepted token (n >= 1 here)
-            const int a = min(max(num_accepted ? num_accepted[b] : n, 1), n);
-            slot = token_slots[t0 + a - 1];
-        } else {
-            slot = idx ? idx[b] : b;
-        }
-        const size_t off = (((size_t)slot * Nv + h) * DK + wid * 32) * Dv + col;
-        if (SBF) {
-            const unsigned short *src = static_cast<const unsigned short *>(pool) + off;
-#pragma unroll
-            for (int m = 0; m < 16; ++m)
-                s2[m] = make_float2(bf2f(__ldcs(src + (size_t)(2 * m) * Dv)), bf2f(__ldcs(src + (size_t)(2 * m + 1) * Dv)));
-        } else {
+    if (pool && !SBF) {
+        const size_t off = (((size_t)slot0 * Nv + h) * DK + wid * 32) * Dv + col;
+        {
             const float *src = static_cast<const float *>(pool) + off;
 #pragma unroll
             for (int m = 0; m < 16; ++m)
@@ -196,13 +209,30 @@ __global__ void __launch_bounds__(DK) short_kernel(
     }
     __syncthreads();
 
+#pragma unroll 1
+    for (int half = 0; half < CW / 32; ++half) {
+    if (SBF) {
+        col = tl * CW + half * 32 + lane;
+        if (half) __syncthreads();  // the previous half's last partial sums have been read
+        if (pool) {
+#pragma unroll
+            for (int m = 0; m < 16; ++m)
+                s2[m] = make_float2(bf2f(sm.sst[wid * 32 + 2 * m][half * 32 + lane]),
+                                    bf2f(sm.sst[wid * 32 + 2 * m + 1][half * 32 + lane]));
+        } else {
+#pragma unroll
+            for (int m = 0; m < 16; ++m) s2[m] = make_float2(0.f, 0.f);
+        }
+    }
+    const int vc = half * 32 + lane;  // this thread's column in the staged v slice
+
     for (int j = 0; j < npre; ++j) {
         const int p = j & 1;
         const float4 *kr = reinterpret_cast<const float4 *>(&sm.kh[j][wid * 32]);
         const float4 *qr = reinterpret_cast<const float4 *>(&sm.qh[j][wid * 32]);
         // the decay as one factor (applied to the sum S^T kh and in the update), or per row (GK: applied
         // to the state rows first)
-        const float dg = (GK || !DECAY) ? 1.f : sm.dg[j], vj = bf2f(sm.v[j][lane]);
+        const float dg = (GK || !DECAY) ? 1.f : sm.dg[j], vj = bf2f(sm.v[j][vc]);
         if (GK) {
             const float4 *dr = reinterpret_cast<const float4 *>(&sm.gkd[j][wid * 32]);
 #pragma unroll
@@ -314,6 +344,7 @@ __global__ void __launch_bounds__(DK) short_kernel(
             __stcs(dst + (size_t)(2 * m + 1) * Dv, s2[m].y);
         }
     }
+    }  // half
 }
 
 template <int PRE, bool SLOTS, bool GK, bool SBF, bool DECAY, bool DELTA, int DK>
@@ -344,19 +375,23 @@ struct RecArgs {
 template <int PRE, bool GK, bool SBF, bool DECAY, bool DELTA, int DK>
 static void launch_pool(const RecArgs &a, dim3 grid, cudaStream_t st)
 {
+    grid.z = a.Dv / (SBF ? 64 : 32);  // Dv columns per CTA
     launch_variant<PRE, true, GK, SBF, DECAY, DELTA, DK>(grid, st, a.q, a.k, a.v, a.g, a.beta, a.gk, a.cu, a.pool,
                                                          nullptr, a.token_slots, a.num_accepted, a.pool, a.scale,
                                                          a.eps, a.out, nullptr, a.T, a.Nqk, a.Nv, a.Dv);
 }
 
 // the pool variants of one staging depth, update rule and key dimension; a key gate only with a decaying rule
+// (a bf16 pool stages 8 tokens: the decode page's operator takes at most 8 per call, and 16 with the
+// 64-column slice would not fit the static shared memory; longer sequences stay exact, their later
+// tokens read directly)
 template <int PRE, bool DECAY, bool DELTA, int DK>
 static void launch_rule(const RecArgs &a, bool bf16_pool, dim3 grid, cudaStream_t st)
 {
     const bool gk = DECAY && a.gk != nullptr;
-    if (gk && bf16_pool) launch_pool<PRE, DECAY, true, DECAY, DELTA, DK>(a, grid, st);
+    if (gk && bf16_pool) launch_pool<8, DECAY, true, DECAY, DELTA, DK>(a, grid, st);
     else if (gk) launch_pool<PRE, DECAY, false, DECAY, DELTA, DK>(a, grid, st);
-    else if (bf16_pool) launch_pool<PRE, false, true, DECAY, DELTA, DK>(a, grid, st);
+    else if (bf16_pool) launch_pool<8, false, true, DECAY, DELTA, DK>(a, grid, st);
     else launch_pool<PRE, false, false, DECAY, DELTA, DK>(a, grid, st);
 }
 

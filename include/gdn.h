@@ -232,8 +232,9 @@ int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *
  *                 overlap any input or state_pool
  *   T, B, Nqk, Nv, P   sizes (T = cu[B]); Nv % Nqk == 0; P >= 1
  *   Dk, Dv        key and value head dimensions: Dk 64 or 128, Dv a multiple
- *                 of 32 up to 1024 (other values: GDN_ERR_UNSUPPORTED); the
- *                 decode page's example has Dk = 64, Dv = 512
+ *                 of 32 (of 64 with a bf16 pool) up to 1024 (other values:
+ *                 GDN_ERR_UNSUPPORTED); the decode page's example has Dk = 64,
+ *                 Dv = 512
  *   max_seqlen    longest sequence if known, else 0.  At most 8 selects the
  *                 kernel variant that stages 8 tokens per sequence (eight CTAs
  *                 per SM); any other value the one that stages 16.  Every
