@@ -133,6 +133,7 @@ def test_recurrent_argument_errors_before_any_launch(lib):
     assert _call_recurrent(lib, rule=4) == B.GDN_ERR_BAD_SHAPE
     assert _call_recurrent(lib, Dk=96) == B.GDN_ERR_UNSUPPORTED
     assert _call_recurrent(lib, Dv=48) == B.GDN_ERR_UNSUPPORTED
+    assert _call_recurrent(lib, Dv=96, bf16=1) == B.GDN_ERR_UNSUPPORTED   # a bf16 pool: Dv a multiple of 64
     assert _call_recurrent(lib, Dv=0) == B.GDN_ERR_BAD_SHAPE
     assert _call_recurrent(lib, Dk=64, Dv=512, slots=10 * M + 2) == B.GDN_ERR_ALIGNMENT  # accepted sizes
     assert _call_recurrent(lib, g=None) == B.GDN_ERR_NULL_ARG             # the gated delta rule reads g
