@@ -1,7 +1,7 @@
 // Tensor Memory Accelerator (TMA) helpers for sm_100a: 2-D tiled tensor maps
 // encoded on the host, bulk tensor copies global <-> shared memory completing
 // on an mbarrier (loads) or a bulk group (stores), and 1-D bulk copies.
-// No copy here uses cluster multicast.
+// Every copy is issued by one CTA for that CTA alone.
 //
 // A 2-D map describes `rows` rows of `cols` elements, rows `row_bytes` apart
 // (a multiple of 16).  A copy moves a box of box_cols x box_rows elements whose
