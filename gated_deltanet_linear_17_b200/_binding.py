@@ -26,6 +26,8 @@ GDN_ERR_SCRATCH_LIMIT = 8
 NOALLOC_SCRATCH_BYTES = 64 << 20
 # update rules of gdn_chunk_fwd_rule and gdn_recurrent_fwd (GDN_RULE_* in gdn.h)
 UPDATE_RULES = {"gated_delta": 0, "delta": 1, "gated": 2, "linear": 3}
+# element types of gdn_recurrent_fwd (GDN_DTYPE_* in gdn.h)
+DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 
 _lib = None
 
@@ -64,10 +66,10 @@ def lib():
         L.gdn_short_fwd.restype = ctypes.c_int
         L.gdn_short_fwd.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, p]
         L.gdn_recurrent_fwd.restype = ctypes.c_int
-        # q k v g beta gk cu pool | state_bf16 rule | slots accepted | scale eps | out | T | B Nqk Nv Dk Dv P
-        # max_seqlen | stream
-        L.gdn_recurrent_fwd.argtypes = [p, p, p, p, p, p, p, p, i32, i32, p, p, f32, f32, p, i64, i32, i32, i32, i32,
-                                        i32, i32, i32, p]
+        # q k v g beta gk cu pool | act_dtype state_dtype rule | slots accepted | scale eps | out | T |
+        # B Nqk Nv Dk Dv P max_seqlen | stream
+        L.gdn_recurrent_fwd.argtypes = [p, p, p, p, p, p, p, p, i32, i32, i32, p, p, f32, f32, p, i64, i32, i32, i32,
+                                        i32, i32, i32, i32, p]
         L.gdn_stage_chunk_map.restype = ctypes.c_int
         L.gdn_stage_chunk_map.argtypes = [p, i64, i32, i32, i32, p, sz, p]
         L.gdn_stage_intra.restype = ctypes.c_int
@@ -252,8 +254,9 @@ def recurrent_fwd(q, k, v, g, beta, cu_seqlens, state_pool, token_slots, num_acc
                   gk=None, update_rule="gated_delta", max_seqlen: int = 0, out=None, stream=None):
     """Token recurrence with the pool updated in place, one slot per token (``gdn_recurrent_fwd``).
 
-    q, k [T, Nqk, Dk], v [T, Nv, Dv] with Dk 64 or 128 and Dv a multiple of 32;
-    ``state_pool`` [P, Nv, Dk, Dv] fp32 or bf16; ``token_slots`` [T] int32 gives each token's
+    q, k [T, Nqk, Dk], v [T, Nv, Dv] with Dk 64 or 128 and Dv a multiple of 32, all bf16 (with an
+    fp32 or bf16 pool) or all fp16 / fp32 (with an fp16 or fp32 pool, Dk = 128); ``out`` has their
+    type; ``state_pool`` [P, Nv, Dk, Dv]; ``token_slots`` [T] int32 gives each token's
     slot; sequence b starts from the slot of its token ``num_accepted[b] - 1`` (its last token when
     ``num_accepted`` is None); ``gk`` [T, Nv, 128] fp32 is the optional key-dimension gate;
     ``update_rule`` is one of gated_delta, delta, gated, linear (g and gk are not needed by
@@ -261,9 +264,10 @@ def recurrent_fwd(q, k, v, g, beta, cu_seqlens, state_pool, token_slots, num_acc
     Returns ``out``; ``state_pool`` holds the updated states afterwards."""
     if state_pool is None or token_slots is None:
         raise ValueError("recurrent_fwd needs a state pool and a slot per token")
-    if state_pool.dtype not in (torch.float32, torch.bfloat16):
-        raise RuntimeError(f"state_pool must be float32 or bfloat16 (got {state_pool.dtype})")
-    bf16_pool = state_pool.dtype == torch.bfloat16
+    if state_pool.dtype not in DTYPES or q.dtype not in DTYPES:
+        raise RuntimeError(f"q/k/v and state_pool must be float32, bfloat16 or float16 (got {q.dtype}, "
+                           f"{state_pool.dtype})")
+    adt = q.dtype
     if update_rule not in UPDATE_RULES:
         raise ValueError(f"update_rule must be one of {sorted(UPDATE_RULES)}")
     rule = UPDATE_RULES[update_rule]
@@ -280,9 +284,9 @@ def recurrent_fwd(q, k, v, g, beta, cu_seqlens, state_pool, token_slots, num_acc
         raise ValueError(f"Nv ({Nv}) must be a multiple of Nqk ({Nqk})")
     B = cu_seqlens.shape[0] - 1
     dev = q.device
-    _need(q, "q", torch.bfloat16, (T, Nqk, Dk), dev)
-    _need(k, "k", torch.bfloat16, (T, Nqk, Dk), dev)
-    _need(v, "v", torch.bfloat16, (T, Nv, Dv), dev)
+    _need(q, "q", adt, (T, Nqk, Dk), dev)
+    _need(k, "k", adt, (T, Nqk, Dk), dev)
+    _need(v, "v", adt, (T, Nv, Dv), dev)
     if g is not None:
         _need(g, "g", torch.float32, (T, Nv), dev)
     if beta is not None:
@@ -296,10 +300,13 @@ def recurrent_fwd(q, k, v, g, beta, cu_seqlens, state_pool, token_slots, num_acc
     if gk is not None:
         _need(gk, "gk", torch.float32, (T, Nv, Dk), dev)
     if out is None:
-        out = torch.empty(T, Nv, Dv, dtype=torch.bfloat16, device=dev)
+        out = torch.empty(T, Nv, Dv, dtype=adt, device=dev)
+    else:
+        _need(out, "out", adt, (T, Nv, Dv), dev)
     sc = 0.0 if scale is None else float(scale)
     rc = lib().gdn_recurrent_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(gk), _ptr(cu_seqlens),
-                                 _ptr(state_pool), int(bf16_pool), rule, _ptr(token_slots), _ptr(num_accepted), sc,
+                                 _ptr(state_pool), DTYPES[adt], DTYPES[state_pool.dtype], rule, _ptr(token_slots),
+                                 _ptr(num_accepted), sc,
                                  float(eps), _ptr(out), T, B, Nqk, Nv, Dk, Dv, P, int(max_seqlen), _stream(stream))
     _check(rc, "gdn_recurrent_fwd")
     return out

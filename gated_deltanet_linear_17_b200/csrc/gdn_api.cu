@@ -293,18 +293,23 @@ int gdn_short_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
                                          (cudaStream_t)stream));
 }
 
-int gdn_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
-                      const uint16_t *beta, const float *gk, const int32_t *cu_seqlens, void *state_pool,
-                      int32_t state_bf16, int32_t update_rule, const int32_t *token_slots,
-                      const int32_t *num_accepted, float scale, float eps, uint16_t *out, int64_t T, int32_t B,
+int gdn_recurrent_fwd(const void *q, const void *k, const void *v, const float *g, const uint16_t *beta,
+                      const float *gk, const int32_t *cu_seqlens, void *state_pool, int32_t act_dtype,
+                      int32_t state_dtype, int32_t update_rule, const int32_t *token_slots,
+                      const int32_t *num_accepted, float scale, float eps, void *out, int64_t T, int32_t B,
                       int32_t Nqk, int32_t Nv, int32_t Dk, int32_t Dv, int32_t P, int32_t max_seqlen, void *stream)
 {
     int rc = check_sizes(T, B, Nqk, Nv);
     if (rc) return rc;
     if (update_rule < GDN_RULE_GATED_DELTA || update_rule > GDN_RULE_LINEAR) return GDN_ERR_BAD_SHAPE;
-    if (P <= 0 || (state_bf16 != 0 && state_bf16 != 1)) return GDN_ERR_BAD_SHAPE;
-    if (Dk <= 0 || Dv <= 0) return GDN_ERR_BAD_SHAPE;
-    if ((Dk != 64 && Dk != 128) || Dv % 32 != 0 || Dv > 1024 || (state_bf16 && Dv % 64 != 0))
+    if (P <= 0 || Dk <= 0 || Dv <= 0) return GDN_ERR_BAD_SHAPE;
+    const auto known = [](int32_t d) { return d == GDN_DTYPE_FP32 || d == GDN_DTYPE_BF16 || d == GDN_DTYPE_FP16; };
+    if (!known(act_dtype) || !known(state_dtype)) return GDN_ERR_BAD_SHAPE;
+    // bf16 activations take an fp32 or bf16 pool; fp16 / fp32 activations an fp16 or fp32 pool at Dk = 128
+    const bool types_ok = act_dtype == GDN_DTYPE_BF16 ? state_dtype != GDN_DTYPE_FP16
+                                                      : state_dtype != GDN_DTYPE_BF16 && Dk == 128;
+    const bool pool16 = state_dtype != GDN_DTYPE_FP32;
+    if (!types_ok || (Dk != 64 && Dk != 128) || Dv % 32 != 0 || Dv > 1024 || (pool16 && Dv % 64 != 0))
         return GDN_ERR_UNSUPPORTED;
     if (B == 0) return GDN_OK;
     const bool decay = update_rule == GDN_RULE_GATED_DELTA || update_rule == GDN_RULE_GATED;
@@ -321,14 +326,15 @@ int gdn_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, c
         (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(token_slots) & 3u) ||
         (reinterpret_cast<uintptr_t>(num_accepted) & 3u))
         return GDN_ERR_ALIGNMENT;
-    const size_t obytes = (size_t)T * Nv * Dv * 2, qbytes = (size_t)T * Nqk * Dk * 2;
-    const size_t pbytes = (size_t)Dk * Dv * (state_bf16 ? 2 : 4) * Nv * P;
+    const size_t ae = act_dtype == GDN_DTYPE_FP32 ? 4 : 2;
+    const size_t obytes = (size_t)T * Nv * Dv * ae, qbytes = (size_t)T * Nqk * Dk * ae;
+    const size_t pbytes = (size_t)Dk * Dv * (pool16 ? 2 : 4) * Nv * P;
     if (overlap(out, obytes, q, qbytes) || overlap(out, obytes, k, qbytes) || overlap(out, obytes, v, obytes) ||
         overlap(out, obytes, state_pool, pbytes) || overlap(out, obytes, gk, (size_t)T * Nv * Dk * 4))
         return GDN_ERR_OVERLAP;
     if (T == 0) return GDN_OK;
     const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)Dk);
-    return cuda_status(gdn::launch_recurrent(q, k, v, g, beta, gk, cu_seqlens, state_pool, state_bf16 != 0,
+    return cuda_status(gdn::launch_recurrent(q, k, v, g, beta, gk, cu_seqlens, state_pool, act_dtype, state_dtype,
                                              update_rule, token_slots, num_accepted, sc, eps, out, (int)T, B, Nqk, Nv,
                                              Dk, Dv, max_seqlen, (cudaStream_t)stream));
 }

@@ -58,15 +58,15 @@ cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v
                          const uint16_t *beta, const int32_t *cu, const float *pool, const int32_t *idx, float scale,
                          float eps, uint16_t *out, float *final_state, int T, int B, int Nqk, int Nv, int max_seqlen,
                          cudaStream_t st, int rule = 0);
-// The same kernel on a pool updated in place (fp32, or bf16 when bf16_pool), one slot per token,
+// The same kernel on a pool updated in place (dtype codes: 0 fp32, 1 bf16, 2 fp16 for the activations
+// q, k, v, out and for the pool), one slot per token,
 // the start taken from the last accepted token's slot; key dimension Dk (64 or 128), value dimension
 // Dv (a multiple of 32); gk [T, Nv, Dk] or nullptr (read only by the decaying rules).
 // update rules of gdn_recurrent_fwd (GDN_RULE_* in gdn.h)
 constexpr int kRuleGatedDelta = 0, kRuleDelta = 1, kRuleGated = 2, kRuleLinear = 3;
-cudaError_t launch_recurrent(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
-                             const uint16_t *beta, const float *gk, const int32_t *cu, void *pool, bool bf16_pool,
-                             int rule, const int32_t *token_slots, const int32_t *num_accepted, float scale,
-                             float eps, uint16_t *out, int T, int B, int Nqk, int Nv, int Dk, int Dv, int max_seqlen,
-                             cudaStream_t st);
+cudaError_t launch_recurrent(const void *q, const void *k, const void *v, const float *g, const uint16_t *beta,
+                             const float *gk, const int32_t *cu, void *pool, int act_dtype, int state_dtype, int rule,
+                             const int32_t *token_slots, const int32_t *num_accepted, float scale, float eps, void *out,
+                             int T, int B, int Nqk, int Nv, int Dk, int Dv, int max_seqlen, cudaStream_t st);
 
 }  // namespace gdn

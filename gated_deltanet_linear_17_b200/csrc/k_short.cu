@@ -49,15 +49,55 @@ namespace gdn {
 
 constexpr int kTile = 32;  // Dv columns per CTA
 
-// DK: key dimension (64 or 128); the CTA has DK threads, warp w holding state rows 32w .. 32w + 31
-// SBF: a bf16 pool; the CTA then covers 64 columns, its slice staged in shared memory (sst)
-template <int PRE, bool GK, int DK, bool SBF>  // tokens staged together with the state; key gate
+// element types of the activations (q, k, v, out) and of the state pool
+constexpr int kF32 = 0, kBF16 = 1, kF16 = 2;
+
+template <int DT>  // a 16-bit value of type DT widened to fp32
+__device__ __forceinline__ float wide16(uint16_t x)
+{
+    if constexpr (DT == kBF16) return bf2f(x);
+    else return __half2float(__ushort_as_half(x));
+}
+template <int DT>  // fp32 rounded to nearest even in the 16-bit type DT
+__device__ __forceinline__ uint16_t narrow16(float x)
+{
+    if constexpr (DT == kBF16) return f2bf(x);
+    else return __half_as_ushort(__float2half_rn(x));
+}
+template <int DT>  // element i of an activation array of type DT
+__device__ __forceinline__ float ld_act(const void *p, size_t i)
+{
+    if constexpr (DT == kF32) return static_cast<const float *>(p)[i];
+    else return wide16<DT>(static_cast<const uint16_t *>(p)[i]);
+}
+template <int DT>
+__device__ __forceinline__ void st_act(void *p, size_t i, float x)
+{
+    if constexpr (DT == kF32) static_cast<float *>(p)[i] = x;
+    else static_cast<uint16_t *>(p)[i] = narrow16<DT>(x);
+}
+template <int DT>  // elements 2e, 2e + 1 of a staged row of type DT
+__device__ __forceinline__ float2 pair_at(const uint16_t *row, int e)
+{
+    if constexpr (DT == kF32) return reinterpret_cast<const float2 *>(row)[e];
+    else if constexpr (DT == kF16) return __half22float2(reinterpret_cast<const __half2 *>(row)[e]);
+    else {
+        const uint32_t w = reinterpret_cast<const uint32_t *>(row)[e];
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+}
+
+// DK: key dimension (64 or 128); the CTA has DK threads, warp w holding state rows 32w .. 32w + 31.
+// SDT: the pool's type; with a 16-bit pool the CTA covers 64 columns, its slice staged in shared
+// memory (sst).  ADT: the activations' type (raw rows staged as bytes, 16-bit units).
+template <int PRE, bool GK, int DK, int SDT, int ADT>  // tokens staged together with the state; key gate
 struct ShortSmem {
+    static constexpr int AU = ADT == kF32 ? 2 : 1;  // 16-bit units per activation element
     float kh[PRE][DK], qh[PRE][DK];   // normalised rows, fp32 (qh includes the scale)
     float gkd[GK ? PRE : 1][DK];      // gk rows, then the row decays e^{g + gk} (GK)
-    uint16_t sst[SBF ? DK : 1][SBF ? 64 : 8];  // the bf16 state slice (SBF)
-    uint16_t q[PRE][DK], k[PRE][DK];  // raw bf16 rows
-    uint16_t v[PRE][SBF ? 64 : 32];   // raw bf16 slice
+    uint16_t sst[SDT != kF32 ? DK : 1][SDT != kF32 ? 64 : 8];  // the 16-bit state slice
+    uint16_t q[PRE][DK * AU], k[PRE][DK * AU];                  // raw rows
+    uint16_t v[PRE][(SDT != kF32 ? 64 : 32) * AU];              // raw slice
     float g[PRE], dg[PRE], beta[PRE];
     int32_t slot[PRE + 1];  // token slots (SLOTS)
     float red[2][DK / 32][32], red2[2][DK / 32][32];
@@ -73,20 +113,22 @@ __device__ __forceinline__ float sum_warps(const float (&r)[NW][32], int lane)
     return a;
 }
 
-template <int PRE, bool SLOTS, bool GK, bool SBF, bool DECAY, bool DELTA, int DK>
+template <int PRE, bool SLOTS, bool GK, int SDT, bool DECAY, bool DELTA, int DK, int ADT>
 __global__ void __launch_bounds__(DK) short_kernel(
-    const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, const uint16_t *__restrict__ v,
+    const void *__restrict__ q, const void *__restrict__ k, const void *__restrict__ v,
     const float *__restrict__ g, const uint16_t *__restrict__ beta, const float *__restrict__ gk,
     const int32_t *__restrict__ cu, const void *pool, const int32_t *__restrict__ idx,
     const int32_t *__restrict__ token_slots, const int32_t *__restrict__ num_accepted, void *pool_w, float scale,
-    float eps, uint16_t *__restrict__ out, float *__restrict__ final_state, int T, int Nqk, int Nv, int Dv)
+    float eps, void *__restrict__ out, float *__restrict__ final_state, int T, int Nqk, int Nv, int Dv)
 {
+    constexpr bool SBF = SDT != kF32;          // a 16-bit pool
+    constexpr int AES = ADT == kF32 ? 4 : 2;   // activation element bytes
     constexpr int NW = DK / 32, EL = DK / 32;  // warps; elements of a q/k row per lane
     // Dv columns per CTA: with a bf16 pool 64, the slice (16 KiB at Dk = 128) fetched by cp.async into
     // shared memory and the tokens applied to one 32-column half after the other, so a CTA keeps twice
     // the bytes in flight with the same registers
     constexpr int CW = SBF ? 64 : 32;
-    __shared__ __align__(16) ShortSmem<PRE, GK, DK, SBF> sm;
+    __shared__ __align__(16) ShortSmem<PRE, GK, DK, SDT, ADT> sm;
     const int b = blockIdx.x, h = blockIdx.y, tl = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     int col = tl * CW + lane;
@@ -97,15 +139,17 @@ __global__ void __launch_bounds__(DK) short_kernel(
     if (SLOTS && n == 0) return;  // no token: the pool keeps its slots
 
     // token data of the first kPre tokens: async copies
-    for (int e = tid; e < npre * (DK / 8); e += DK) {
-        const int t = e / (DK / 8), c = e % (DK / 8);
-        const size_t off = ((size_t)(t0 + t) * Nqk + hq) * DK + c * 8;
-        cp_async16(smem_addr(&sm.q[t][c * 8]), q + off, true);
-        cp_async16(smem_addr(&sm.k[t][c * 8]), k + off, true);
+    constexpr int QC = DK * AES / 16, VC = CW * AES / 16;  // 16-byte pieces of a q/k row, of the v slice
+    for (int e = tid; e < npre * QC; e += DK) {
+        const int t = e / QC, c = e % QC;
+        const size_t off = (((size_t)(t0 + t) * Nqk + hq) * DK) * AES + c * 16;
+        cp_async16(smem_addr(&sm.q[t][c * 8]), static_cast<const char *>(q) + off, true);
+        cp_async16(smem_addr(&sm.k[t][c * 8]), static_cast<const char *>(k) + off, true);
     }
-    for (int e = tid; e < npre * (CW / 8); e += DK) {
-        const int t = e / (CW / 8), c = e % (CW / 8);
-        cp_async16(smem_addr(&sm.v[t][c * 8]), v + ((size_t)(t0 + t) * Nv + h) * Dv + tl * CW + c * 8, true);
+    for (int e = tid; e < npre * VC; e += DK) {
+        const int t = e / VC, c = e % VC;
+        const size_t off = (((size_t)(t0 + t) * Nv + h) * Dv + tl * CW) * AES + c * 16;
+        cp_async16(smem_addr(&sm.v[t][c * 8]), static_cast<const char *>(v) + off, true);
     }
     if (DECAY && tid < npre) cp_async4(smem_addr(&sm.g[tid]), g + (size_t)(t0 + tid) * Nv + h);
     if (SLOTS && tid <= PRE && tid < n) cp_async4(smem_addr(&sm.slot[tid]), token_slots + t0 + tid);
@@ -159,8 +203,8 @@ __global__ void __launch_bounds__(DK) short_kernel(
             unsigned short *dst = static_cast<unsigned short *>(pool_w) + off;
 #pragma unroll
             for (int m = 0; m < 16; ++m) {
-                __stcs(dst + (size_t)(2 * m) * Dv, (unsigned short)f2bf(s2[m].x));
-                __stcs(dst + (size_t)(2 * m + 1) * Dv, (unsigned short)f2bf(s2[m].y));
+                __stcs(dst + (size_t)(2 * m) * Dv, (unsigned short)narrow16<SDT>(s2[m].x));
+                __stcs(dst + (size_t)(2 * m + 1) * Dv, (unsigned short)narrow16<SDT>(s2[m].y));
             }
         } else {
             float *dst = static_cast<float *>(pool_w) + off;
@@ -182,12 +226,12 @@ __global__ void __launch_bounds__(DK) short_kernel(
         float sq = 0.f, sk = 0.f;
 #pragma unroll
         for (int e2 = 0; e2 < EL / 2; ++e2) {
-            const uint32_t qw = reinterpret_cast<const uint32_t *>(&sm.q[t][lane * EL])[e2];
-            const uint32_t kw = reinterpret_cast<const uint32_t *>(&sm.k[t][lane * EL])[e2];
-            qe[2 * e2] = __uint_as_float(qw << 16);
-            qe[2 * e2 + 1] = __uint_as_float(qw & 0xffff0000u);
-            ke[2 * e2] = __uint_as_float(kw << 16);
-            ke[2 * e2 + 1] = __uint_as_float(kw & 0xffff0000u);
+            const float2 qp = pair_at<ADT>(&sm.q[t][0], lane * EL / 2 + e2);
+            const float2 kp = pair_at<ADT>(&sm.k[t][0], lane * EL / 2 + e2);
+            qe[2 * e2] = qp.x;
+            qe[2 * e2 + 1] = qp.y;
+            ke[2 * e2] = kp.x;
+            ke[2 * e2 + 1] = kp.y;
         }
 #pragma unroll
         for (int e = 0; e < EL; ++e) {
@@ -217,8 +261,8 @@ __global__ void __launch_bounds__(DK) short_kernel(
         if (pool) {
 #pragma unroll
             for (int m = 0; m < 16; ++m)
-                s2[m] = make_float2(bf2f(sm.sst[wid * 32 + 2 * m][half * 32 + lane]),
-                                    bf2f(sm.sst[wid * 32 + 2 * m + 1][half * 32 + lane]));
+                s2[m] = make_float2(wide16<SDT>(sm.sst[wid * 32 + 2 * m][half * 32 + lane]),
+                                    wide16<SDT>(sm.sst[wid * 32 + 2 * m + 1][half * 32 + lane]));
         } else {
 #pragma unroll
             for (int m = 0; m < 16; ++m) s2[m] = make_float2(0.f, 0.f);
@@ -232,7 +276,10 @@ __global__ void __launch_bounds__(DK) short_kernel(
         const float4 *qr = reinterpret_cast<const float4 *>(&sm.qh[j][wid * 32]);
         // the decay as one factor (applied to the sum S^T kh and in the update), or per row (GK: applied
         // to the state rows first)
-        const float dg = (GK || !DECAY) ? 1.f : sm.dg[j], vj = bf2f(sm.v[j][vc]);
+        const float dg = (GK || !DECAY) ? 1.f : sm.dg[j];
+        float vj;
+        if constexpr (ADT == kF32) vj = reinterpret_cast<const float *>(&sm.v[j][0])[vc];
+        else vj = wide16<ADT>(sm.v[j][vc]);
         if (GK) {
             const float4 *dr = reinterpret_cast<const float4 *>(&sm.gkd[j][wid * 32]);
 #pragma unroll
@@ -276,24 +323,24 @@ __global__ void __launch_bounds__(DK) short_kernel(
         if (SLOTS && (j == n - 1 || sm.slot[j + 1] != sm.slot[j])) write_slot(sm.slot[j]);
         __syncthreads();
         if (wid == 0)
-            out[((size_t)(t0 + j) * Nv + h) * Dv + col] = f2bf(sum_warps<NW>(sm.red2[p], lane));
+            st_act<ADT>(out, ((size_t)(t0 + j) * Nv + h) * Dv + col, sum_warps<NW>(sm.red2[p], lane));
     }
 
     // beyond the staged tokens (longer sequences than the fused path is meant for): read directly
     for (int j = PRE; j < n; ++j) {
         const int t = t0 + j, p = j & 1;
-        const uint16_t *qrow = q + ((size_t)t * Nqk + hq) * DK, *krow = k + ((size_t)t * Nqk + hq) * DK;
+        const size_t qrow = ((size_t)t * Nqk + hq) * DK;  // first element of the token's q and k rows
         float sq = 0.f, sk = 0.f;
 #pragma unroll
         for (int i = 0; i < EL; ++i) {
-            const float a = bf2f(qrow[lane + 32 * i]), c = bf2f(krow[lane + 32 * i]);
+            const float a = ld_act<ADT>(q, qrow + lane + 32 * i), c = ld_act<ADT>(k, qrow + lane + 32 * i);
             sq = fmaf(a, a, sq);
             sk = fmaf(c, c, sk);
         }
         sq = warp_sum(sq);
         sk = warp_sum(sk);
         const float rq = scale / sqrtf(sq + eps), rk = 1.0f / sqrtf(sk + eps);
-        const float vj = bf2f(v[((size_t)t * Nv + h) * Dv + col]);
+        const float vj = ld_act<ADT>(v, ((size_t)t * Nv + h) * Dv + col);
         const float gt = DECAY ? g[(size_t)t * Nv + h] : 0.f, bt = DELTA ? bf2f(beta[(size_t)t * Nv + h]) : 1.f;
         const float dg = (GK || !DECAY) ? 1.f : __expf(gt);
         if (GK) {  // this thread's 32 rows decayed by e^{g + gk_i}
@@ -304,14 +351,14 @@ __global__ void __launch_bounds__(DK) short_kernel(
                 s2[m].y *= __expf(gt + gr[2 * m + 1]);
             }
         }
-        const uint16_t *kr = krow + wid * 32, *qr = qrow + wid * 32;
+        const size_t kr = qrow + wid * 32, qr = qrow + wid * 32;  // this warp's 32 rows
         float u = vj;
         if (DELTA) {
             float acc = 0.f;
 #pragma unroll
             for (int m = 0; m < 16; ++m) {
-                acc = fmaf(s2[m].x, bf2f(kr[2 * m]) * rk, acc);
-                acc = fmaf(s2[m].y, bf2f(kr[2 * m + 1]) * rk, acc);
+                acc = fmaf(s2[m].x, ld_act<ADT>(k, kr + 2 * m) * rk, acc);
+                acc = fmaf(s2[m].y, ld_act<ADT>(k, kr + 2 * m + 1) * rk, acc);
             }
             sm.red[p][wid][lane] = acc;
             __syncthreads();
@@ -321,10 +368,10 @@ __global__ void __launch_bounds__(DK) short_kernel(
         float acc2 = 0.f;
 #pragma unroll
         for (int m = 0; m < 16; ++m) {
-            s2[m].x = fmaf(bf2f(kr[2 * m]) * rk, u, s2[m].x * dg);
-            s2[m].y = fmaf(bf2f(kr[2 * m + 1]) * rk, u, s2[m].y * dg);
-            acc2 = fmaf(s2[m].x, bf2f(qr[2 * m]) * rq, acc2);
-            acc2 = fmaf(s2[m].y, bf2f(qr[2 * m + 1]) * rq, acc2);
+            s2[m].x = fmaf(ld_act<ADT>(k, kr + 2 * m) * rk, u, s2[m].x * dg);
+            s2[m].y = fmaf(ld_act<ADT>(k, kr + 2 * m + 1) * rk, u, s2[m].y * dg);
+            acc2 = fmaf(s2[m].x, ld_act<ADT>(q, qr + 2 * m) * rq, acc2);
+            acc2 = fmaf(s2[m].y, ld_act<ADT>(q, qr + 2 * m + 1) * rq, acc2);
         }
         sm.red2[p][wid][lane] = acc2;
         if (SLOTS) {
@@ -333,7 +380,7 @@ __global__ void __launch_bounds__(DK) short_kernel(
         }
         __syncthreads();
         if (wid == 0)
-            out[((size_t)t * Nv + h) * Dv + col] = f2bf(sum_warps<NW>(sm.red2[p], lane));
+            st_act<ADT>(out, ((size_t)t * Nv + h) * Dv + col, sum_warps<NW>(sm.red2[p], lane));
     }
 
     if (!SLOTS && final_state) {
@@ -347,20 +394,20 @@ __global__ void __launch_bounds__(DK) short_kernel(
     }  // half
 }
 
-template <int PRE, bool SLOTS, bool GK, bool SBF, bool DECAY, bool DELTA, int DK>
-static void launch_variant(dim3 grid, cudaStream_t st, const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                           const float *g, const uint16_t *beta, const float *gk, const int32_t *cu, const void *pool,
+template <int PRE, bool SLOTS, bool GK, int SDT, bool DECAY, bool DELTA, int DK, int ADT>
+static void launch_variant(dim3 grid, cudaStream_t st, const void *q, const void *k, const void *v, const float *g,
+                           const uint16_t *beta, const float *gk, const int32_t *cu, const void *pool,
                            const int32_t *idx, const int32_t *token_slots, const int32_t *num_accepted, void *pool_w,
-                           float scale, float eps, uint16_t *out, float *final_state, int T, int Nqk, int Nv, int Dv)
+                           float scale, float eps, void *out, float *final_state, int T, int Nqk, int Nv, int Dv)
 {
-    short_kernel<PRE, SLOTS, GK, SBF, DECAY, DELTA, DK><<<grid, DK, 0, st>>>(
+    short_kernel<PRE, SLOTS, GK, SDT, DECAY, DELTA, DK, ADT><<<grid, DK, 0, st>>>(
         q, k, v, g, beta, gk, cu, pool, idx, token_slots, num_accepted, pool_w, scale, eps, out, final_state, T, Nqk,
         Nv, Dv);
 }
 
 // Arguments of one pool-updating launch
 struct RecArgs {
-    const uint16_t *q, *k, *v;
+    const void *q, *k, *v;
     const float *g;
     const uint16_t *beta;
     const float *gk;
@@ -368,41 +415,57 @@ struct RecArgs {
     void *pool;
     const int32_t *token_slots, *num_accepted;
     float scale, eps;
-    uint16_t *out;
+    void *out;
     int T, Nqk, Nv, Dv;
 };
 
-template <int PRE, bool GK, bool SBF, bool DECAY, bool DELTA, int DK>
+template <int PRE, bool GK, int SDT, bool DECAY, bool DELTA, int DK, int ADT>
 static void launch_pool(const RecArgs &a, dim3 grid, cudaStream_t st)
 {
-    grid.z = a.Dv / (SBF ? 64 : 32);  // Dv columns per CTA
-    launch_variant<PRE, true, GK, SBF, DECAY, DELTA, DK>(grid, st, a.q, a.k, a.v, a.g, a.beta, a.gk, a.cu, a.pool,
-                                                         nullptr, a.token_slots, a.num_accepted, a.pool, a.scale,
-                                                         a.eps, a.out, nullptr, a.T, a.Nqk, a.Nv, a.Dv);
+    grid.z = a.Dv / (SDT != kF32 ? 64 : 32);  // Dv columns per CTA
+    launch_variant<PRE, true, GK, SDT, DECAY, DELTA, DK, ADT>(grid, st, a.q, a.k, a.v, a.g, a.beta, a.gk, a.cu, a.pool,
+                                                              nullptr, a.token_slots, a.num_accepted, a.pool, a.scale,
+                                                              a.eps, a.out, nullptr, a.T, a.Nqk, a.Nv, a.Dv);
 }
 
-// the pool variants of one staging depth, update rule and key dimension; a key gate only with a decaying rule
-// (a bf16 pool stages 8 tokens: the decode page's operator takes at most 8 per call, and 16 with the
-// 64-column slice would not fit the static shared memory; longer sequences stay exact, their later
-// tokens read directly)
-template <int PRE, bool DECAY, bool DELTA, int DK>
-static void launch_rule(const RecArgs &a, bool bf16_pool, dim3 grid, cudaStream_t st)
+// one activation type and pool type; a key gate only with a decaying rule.  A 16-bit pool stages 8
+// tokens (the decode page's operator takes at most 8 per call, and 16 with the 64-column slice would not
+// fit the static shared memory; longer sequences stay exact, their later tokens read directly)
+template <int PRE, bool DECAY, bool DELTA, int DK, int ADT, int SDT>
+static void launch_types(const RecArgs &a, dim3 grid, cudaStream_t st)
 {
-    const bool gk = DECAY && a.gk != nullptr;
-    if (gk && bf16_pool) launch_pool<8, DECAY, true, DECAY, DELTA, DK>(a, grid, st);
-    else if (gk) launch_pool<PRE, DECAY, false, DECAY, DELTA, DK>(a, grid, st);
-    else if (bf16_pool) launch_pool<8, false, true, DECAY, DELTA, DK>(a, grid, st);
-    else launch_pool<PRE, false, false, DECAY, DELTA, DK>(a, grid, st);
+    constexpr int P = SDT != kF32 ? 8 : PRE;
+    if (DECAY && a.gk) launch_pool<P, DECAY, SDT, DECAY, DELTA, DK, ADT>(a, grid, st);
+    else launch_pool<P, false, SDT, DECAY, DELTA, DK, ADT>(a, grid, st);
+}
+
+// the type combinations: bf16 activations with an fp32 or bf16 pool (the decode page), fp16 or fp32
+// activations with an fp16 or fp32 pool (the LinearAttention page; Dk = 128 only)
+template <int PRE, bool DECAY, bool DELTA, int DK>
+static void launch_rule(const RecArgs &a, int adt, int sdt, dim3 grid, cudaStream_t st)
+{
+    if (adt == kBF16) {
+        if (sdt == kBF16) launch_types<PRE, DECAY, DELTA, DK, kBF16, kBF16>(a, grid, st);
+        else launch_types<PRE, DECAY, DELTA, DK, kBF16, kF32>(a, grid, st);
+    } else if constexpr (DK == 128) {
+        if (adt == kF16) {
+            if (sdt == kF16) launch_types<16, DECAY, DELTA, DK, kF16, kF16>(a, grid, st);
+            else launch_types<16, DECAY, DELTA, DK, kF16, kF32>(a, grid, st);
+        } else {
+            if (sdt == kF16) launch_types<16, DECAY, DELTA, DK, kF32, kF16>(a, grid, st);
+            else launch_types<16, DECAY, DELTA, DK, kF32, kF32>(a, grid, st);
+        }
+    }
 }
 
 template <int PRE, int DK>
-static void launch_slots(const RecArgs &a, int rule, bool bf16_pool, dim3 grid, cudaStream_t st)
+static void launch_slots(const RecArgs &a, int rule, int adt, int sdt, dim3 grid, cudaStream_t st)
 {
     switch (rule) {
-    case kRuleDelta: launch_rule<PRE, false, true, DK>(a, bf16_pool, grid, st); break;
-    case kRuleGated: launch_rule<PRE, true, false, DK>(a, bf16_pool, grid, st); break;
-    case kRuleLinear: launch_rule<PRE, false, false, DK>(a, bf16_pool, grid, st); break;
-    default: launch_rule<PRE, true, true, DK>(a, bf16_pool, grid, st);
+    case kRuleDelta: launch_rule<PRE, false, true, DK>(a, adt, sdt, grid, st); break;
+    case kRuleGated: launch_rule<PRE, true, false, DK>(a, adt, sdt, grid, st); break;
+    case kRuleLinear: launch_rule<PRE, false, false, DK>(a, adt, sdt, grid, st); break;
+    default: launch_rule<PRE, true, true, DK>(a, adt, sdt, grid, st);
     }
 }
 
@@ -415,9 +478,9 @@ cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v
     const dim3 grid(B, Nv, D / kTile);
     const bool few = max_seqlen >= 1 && max_seqlen <= 8;
     auto go = [&](auto pre, auto decay, auto delta) {
-        launch_variant<decltype(pre)::value, false, false, false, decltype(decay)::value, decltype(delta)::value, D>(
-            grid, st, q, k, v, g, beta, nullptr, cu, pool, idx, nullptr, nullptr, nullptr, scale, eps, out, final_state,
-            T, Nqk, Nv, D);
+        launch_variant<decltype(pre)::value, false, false, kF32, decltype(decay)::value, decltype(delta)::value, D,
+                       kBF16>(grid, st, q, k, v, g, beta, nullptr, cu, pool, idx, nullptr, nullptr, nullptr, scale, eps,
+                              out, final_state, T, Nqk, Nv, D);
     };
     using P8 = std::integral_constant<int, 8>;
     using P16 = std::integral_constant<int, 16>;
@@ -432,23 +495,23 @@ cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v
     return cudaGetLastError();
 }
 
-cudaError_t launch_recurrent(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
-                             const uint16_t *beta, const float *gk, const int32_t *cu, void *pool, bool bf16_pool,
-                             int rule, const int32_t *token_slots, const int32_t *num_accepted, float scale,
-                             float eps, uint16_t *out, int T, int B, int Nqk, int Nv, int Dk, int Dv, int max_seqlen,
-                             cudaStream_t st)
+cudaError_t launch_recurrent(const void *q, const void *k, const void *v, const float *g, const uint16_t *beta,
+                             const float *gk, const int32_t *cu, void *pool, int act_dtype, int state_dtype, int rule,
+                             const int32_t *token_slots, const int32_t *num_accepted, float scale, float eps, void *out,
+                             int T, int B, int Nqk, int Nv, int Dk, int Dv, int max_seqlen, cudaStream_t st)
 {
     if (B == 0) return cudaSuccess;
     if ((Dk != 64 && Dk != 128) || Dv <= 0 || Dv % kTile != 0) return cudaErrorInvalidValue;
+    if (act_dtype != kBF16 && Dk != 128) return cudaErrorInvalidValue;
     const RecArgs a{q, k, v, g, beta, gk, cu, pool, token_slots, num_accepted, scale, eps, out, T, Nqk, Nv, Dv};
     const dim3 grid(B, Nv, Dv / kTile);
     const bool few = max_seqlen >= 1 && max_seqlen <= 8;
     if (Dk == 64) {
-        if (few) launch_slots<8, 64>(a, rule, bf16_pool, grid, st);
-        else launch_slots<16, 64>(a, rule, bf16_pool, grid, st);
+        if (few) launch_slots<8, 64>(a, rule, act_dtype, state_dtype, grid, st);
+        else launch_slots<16, 64>(a, rule, act_dtype, state_dtype, grid, st);
     } else {
-        if (few) launch_slots<8, 128>(a, rule, bf16_pool, grid, st);
-        else launch_slots<16, 128>(a, rule, bf16_pool, grid, st);
+        if (few) launch_slots<8, 128>(a, rule, act_dtype, state_dtype, grid, st);
+        else launch_slots<16, 128>(a, rule, act_dtype, state_dtype, grid, st);
     }
     return cudaGetLastError();
 }

@@ -51,6 +51,11 @@ extern "C" {
 #define GDN_SHORT_MAX 16 /* max_seqlen at or below which the fused short-sequence kernel runs */
 #define GDN_NOALLOC_SCRATCH_BYTES (64u << 20) /* static workspace of gdn_chunk_fwd_noalloc, per GPU */
 
+/* element types of gdn_recurrent_fwd's activations and state pool */
+#define GDN_DTYPE_FP32 0
+#define GDN_DTYPE_BF16 1
+#define GDN_DTYPE_FP16 2
+
 /* update rules of gdn_chunk_fwd_rule and gdn_recurrent_fwd */
 #define GDN_RULE_GATED_DELTA 0
 #define GDN_RULE_DELTA 1
@@ -206,8 +211,8 @@ int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *
  * Ordinary decoding puts all tokens of sequence b on one slot (its state is
  * then read from and written back to that slot).
  *
- *   q, k          device bf16 [T, Nqk, Dk]
- *   v             device bf16 [T, Nv, Dv]
+ *   q, k          device [T, Nqk, Dk] of act_dtype
+ *   v             device [T, Nv, Dv] of act_dtype
  *   g, beta, cu_seqlens   as for gdn_chunk_fwd
  *   gk            device fp32 [T, Nv, Dk], the key-dimension gate
  *                 (expected <= 0, not checked), or NULL for none
@@ -218,21 +223,26 @@ int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *
  *                 not read) -- the update rules of the page "com.microsoft.
  *                 LinearAttention" (update_rule); q and k are normalised in
  *                 every rule
- *   state_pool    device [P, Nv, Dk, Dv], read and written in place
- *                 (required): fp32 when state_bf16 == 0, bf16 when state_bf16 == 1
- *                 (the page's pool dtype: widened to fp32 on load, the fp32 result
- *                 rounded to nearest even when written)
+ *   state_pool    device [P, Nv, Dk, Dv] of state_dtype, read and written in
+ *                 place (required); a 16-bit pool is widened to fp32 on load and
+ *                 the fp32 result rounded to nearest even when written
+ *   act_dtype, state_dtype   GDN_DTYPE_FP32 / _BF16 / _FP16.  bf16 activations
+ *                 (the decode page) take an fp32 or bf16 pool; fp16 or fp32
+ *                 activations (the LinearAttention page: activations and state
+ *                 each fp16 or fp32) take an fp16 or fp32 pool and need Dk = 128;
+ *                 other pairs are GDN_ERR_UNSUPPORTED.  g stays fp32 and beta bf16
+ *                 in every combination
  *   token_slots   device int32 [T], each in [0, P) (not checked on the device);
  *                 the slots used by different sequences, including each
  *                 sequence's starting slot, must be disjoint
  *   num_accepted  device int32 [B], or NULL
  *   scale         query scale; <= 0 selects 1/sqrt(Dk)
  *   eps           as for gdn_chunk_fwd
- *   out           device bf16 [T, Nv, Dv], written for every token; must not
+ *   out           device [T, Nv, Dv] of act_dtype, written for every token; must not
  *                 overlap any input or state_pool
  *   T, B, Nqk, Nv, P   sizes (T = cu[B]); Nv % Nqk == 0; P >= 1
  *   Dk, Dv        key and value head dimensions: Dk 64 or 128, Dv a multiple
- *                 of 32 (of 64 with a bf16 pool) up to 1024 (other values:
+ *                 of 32 (of 64 with a 16-bit pool) up to 1024 (other values:
  *                 GDN_ERR_UNSUPPORTED); the decode page's example has Dk = 64,
  *                 Dv = 512
  *   max_seqlen    longest sequence if known, else 0.  At most 8 selects the
@@ -244,15 +254,14 @@ int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *
  * Alignment: q, k, v, out, state_pool, gk 16-byte aligned; g, cu_seqlens,
  * token_slots, num_accepted 4-byte aligned; beta 2-byte aligned.  Errors:
  * GDN_ERR_NULL_ARG, GDN_ERR_BAD_SHAPE, GDN_ERR_UNSUPPORTED, GDN_ERR_ALIGNMENT,
- * GDN_ERR_OVERLAP before anything is enqueued (state_bf16 other than 0 or 1, or
- * an unknown update_rule, is GDN_ERR_BAD_SHAPE); GDN_ERR_CUDA when the launch
- * fails.  B == 0 or T == 0 is a no-op.  Asynchronous on `stream`; the library
+ * GDN_ERR_OVERLAP before anything is enqueued (an unknown dtype code or
+ * update_rule is GDN_ERR_BAD_SHAPE); GDN_ERR_CUDA when the launch fails.  B == 0 or T == 0 is a no-op.  Asynchronous on `stream`; the library
  * keeps no pointer after the call returns.
  */
-int gdn_recurrent_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
-                      const uint16_t *beta, const float *gk, const int32_t *cu_seqlens, void *state_pool,
-                      int32_t state_bf16, int32_t update_rule, const int32_t *token_slots,
-                      const int32_t *num_accepted, float scale, float eps, uint16_t *out, int64_t T, int32_t B,
+int gdn_recurrent_fwd(const void *q, const void *k, const void *v, const float *g, const uint16_t *beta,
+                      const float *gk, const int32_t *cu_seqlens, void *state_pool, int32_t act_dtype,
+                      int32_t state_dtype, int32_t update_rule, const int32_t *token_slots,
+                      const int32_t *num_accepted, float scale, float eps, void *out, int64_t T, int32_t B,
                       int32_t Nqk, int32_t Nv, int32_t Dk, int32_t Dv, int32_t P, int32_t max_seqlen,
                       void *stream);
 

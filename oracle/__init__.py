@@ -80,7 +80,15 @@ def _typed(x):
 
 
 def as_numpy_exact(x) -> np.ndarray:
-    """Widen a tensor/array exactly to float64 (bf16 and fp32 values are representable)."""
+    """Widen a tensor/array exactly to float64 (bf16, fp16 and fp32 values are representable)."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor) and x.dtype == torch.float16:
+            return x.detach().cpu().numpy().astype(np.float64)
+    except ImportError:  # pragma: no cover
+        pass
+    if isinstance(x, np.ndarray) and x.dtype == np.float16:
+        return x.astype(np.float64)
     a, tag = _typed(x)
     if tag == _BF16:
         return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)

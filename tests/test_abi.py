@@ -111,13 +111,14 @@ def test_argument_errors_before_any_launch(lib):
 
 def _call_recurrent(lib, **over):
     M = 1 << 20  # fake, disjoint, aligned addresses; every call below returns before any launch
-    a = dict(q=1 * M, k=2 * M, v=3 * M, g=4 * M, beta=5 * M, gk=None, cu=6 * M, pool=9 * M, bf16=0, rule=0,
+    a = dict(q=1 * M, k=2 * M, v=3 * M, g=4 * M, beta=5 * M, gk=None, cu=6 * M, pool=9 * M, act=1, bf16=0, rule=0,
              slots=10 * M, acc=None, scale=0.0, eps=1e-6, out=7 * M, T=8, B=1, Nqk=2, Nv=4, Dk=128, Dv=128, P=2,
              max_seqlen=0, stream=None)
     a.update(over)
     vp = lambda x: None if x is None else ctypes.c_void_p(x)
     return lib.gdn_recurrent_fwd(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["g"]), vp(a["beta"]), vp(a["gk"]),
-                                 vp(a["cu"]), vp(a["pool"]), a["bf16"], a["rule"], vp(a["slots"]), vp(a["acc"]), a["scale"],
+                                 vp(a["cu"]), vp(a["pool"]), a["act"], a["bf16"], a["rule"], vp(a["slots"]), vp(a["acc"]),
+                                 a["scale"],
                                  a["eps"], vp(a["out"]), a["T"], a["B"], a["Nqk"], a["Nv"], a["Dk"], a["Dv"], a["P"],
                                  a["max_seqlen"],
                                  vp(a["stream"]))
@@ -129,7 +130,12 @@ def test_recurrent_argument_errors_before_any_launch(lib):
     assert _call_recurrent(lib, slots=None) == B.GDN_ERR_NULL_ARG
     assert _call_recurrent(lib, P=0) == B.GDN_ERR_BAD_SHAPE
     assert _call_recurrent(lib, Nv=3) == B.GDN_ERR_BAD_SHAPE
-    assert _call_recurrent(lib, bf16=2) == B.GDN_ERR_BAD_SHAPE
+    assert _call_recurrent(lib, bf16=3) == B.GDN_ERR_BAD_SHAPE             # unknown pool type code
+    assert _call_recurrent(lib, act=5) == B.GDN_ERR_BAD_SHAPE              # unknown activation type code
+    assert _call_recurrent(lib, act=1, bf16=2) == B.GDN_ERR_UNSUPPORTED     # bf16 activations, fp16 pool
+    assert _call_recurrent(lib, act=2, bf16=1) == B.GDN_ERR_UNSUPPORTED     # fp16 activations, bf16 pool
+    assert _call_recurrent(lib, act=0, Dk=64) == B.GDN_ERR_UNSUPPORTED      # fp32 activations need Dk = 128
+    assert _call_recurrent(lib, act=2, bf16=2, slots=10 * M + 2) == B.GDN_ERR_ALIGNMENT  # accepted pair
     assert _call_recurrent(lib, rule=4) == B.GDN_ERR_BAD_SHAPE
     assert _call_recurrent(lib, Dk=96) == B.GDN_ERR_UNSUPPORTED
     assert _call_recurrent(lib, Dv=48) == B.GDN_ERR_UNSUPPORTED

@@ -179,3 +179,34 @@ def test_recurrent_head_dimensions(Dk, Dv):
     inp, slots, acc = _case(lens, Nqk=2, Nv=4, P=40, seed=61, per_token=True, accepted=True, Dk=Dk, Dv=Dv)
     _run_and_check(inp, slots, acc, 0, f"Dk={Dk} Dv={Dv}", gk=_key_gate(inp, 62), bf16_pool=True)
     _run_and_check(inp, slots, acc, 4, f"Dk={Dk} Dv={Dv} fp32 delta", rule="delta")
+
+
+@pytest.mark.parametrize("act,state", [(torch.float16, torch.float32), (torch.float16, torch.float16),
+                                       (torch.float32, torch.float32), (torch.float32, torch.float16)])
+def test_recurrent_linear_attention_types(act, state):
+    """The LinearAttention page's element types: activations and state each fp16 or fp32, with the key
+    gate, a slot per token, accepted counts and tokens past the staged ones.  The activations carry bits
+    beyond bf16 (a small fp32 perturbation), so a narrowed path would show."""
+    lens = [3, 1, 6, 19, 2]
+    inp, slots, acc = _case(lens, Nqk=2, Nv=4, P=40, seed=63, per_token=True, accepted=True)
+    gen = torch.Generator().manual_seed(64)
+    widen = lambda x: (x.float() + 1e-3 * torch.randn(x.shape, generator=gen)).to(act)
+    q, k, v = widen(inp.q), widen(inp.k), widen(inp.v)
+    pool0 = inp.state_pool.to(state)
+    gk = _key_gate(inp, 65)
+    ro, rpool = recurrent_pool(q, k, v, inp.g, inp.beta, inp.cu_seqlens, pool0, slots, num_accepted=acc,
+                               scale=inp.scale, eps=inp.eps, gk=gk)
+    d = inp.to(DEV)
+    pool = pool0.to(DEV).clone()
+    start = pool.clone()
+    out = gdn.recurrent_fwd(q.to(DEV), k.to(DEV), v.to(DEV), d.g, d.beta, d.cu_seqlens, pool,
+                            torch.from_numpy(slots).to(DEV), num_accepted=torch.from_numpy(acc).to(DEV),
+                            scale=d.scale, eps=d.eps, gk=gk.to(DEV), max_seqlen=0)
+    torch.cuda.synchronize()
+    what = f"act {act} state {state}"
+    assert out.dtype == act
+    assert_close(out, ro, f"{what} out")
+    written = np.unique(slots)
+    assert_close(pool[torch.from_numpy(written).to(DEV).long()], rpool[written], f"{what} written slots")
+    others = torch.from_numpy(np.setdiff1d(np.arange(pool.shape[0]), written)).to(DEV).long()
+    assert torch.equal(pool[others], start[others])

@@ -246,3 +246,13 @@ def test_planted_pool_mistake_is_caught(name, old, new):
         assert caught >= 1, f"no pin fails for the planted mistake {name}"
     finally:
         del sys.modules[spec.name]
+
+
+def test_fp16_inputs_widen_exactly():
+    """fp16 activations and states enter the oracle exactly: the smallest subnormal, the smallest normal,
+    the largest finite value and a rounded decimal keep their exact binary values."""
+    import torch
+    x = torch.tensor([2.0 ** -24, -(2.0 ** -14), 65504.0, 0.1], dtype=torch.float16)
+    got = oracle.as_numpy_exact(x)
+    assert got.dtype == np.float64
+    assert list(got) == [2.0 ** -24, -(2.0 ** -14), 65504.0, 1638.0 / 16384.0]  # 0.1 rounds to 1638 * 2^-14
