@@ -113,8 +113,10 @@ __device__ __forceinline__ float sum_warps(const float (&r)[NW][32], int lane)
     return a;
 }
 
+// gdn_chunk_fwd's short path (no SLOTS) is held to 64 registers, eight CTAs per SM: the register file
+// then holds eight state slices in flight (without the bound the compiler takes 78 and fits six)
 template <int PRE, bool SLOTS, bool GK, int SDT, bool DECAY, bool DELTA, int DK, int ADT>
-__global__ void __launch_bounds__(DK) short_kernel(
+__global__ void __launch_bounds__(DK, SLOTS ? 1 : 1024 / DK) short_kernel(
     const void *__restrict__ q, const void *__restrict__ k, const void *__restrict__ v,
     const float *__restrict__ g, const uint16_t *__restrict__ beta, const float *__restrict__ gk,
     const int32_t *__restrict__ cu, const void *pool, const int32_t *__restrict__ idx,
