@@ -113,10 +113,13 @@ __device__ __forceinline__ float sum_warps(const float (&r)[NW][32], int lane)
     return a;
 }
 
-// gdn_chunk_fwd's short path (no SLOTS) is held to 64 registers, eight CTAs per SM: the register file
-// then holds eight state slices in flight (without the bound the compiler takes 78 and fits six)
+// The kernel body, entered through two kernels that differ only in their register budget:
+// gdn_chunk_fwd's short path is held to 64 registers, eight CTAs per SM (without a bound the compiler
+// takes 78 and fits six); the pool-slot variants keep the compiler's own choice (an explicit minimum of
+// one CTA per SM makes it spend up to 142 registers and fit three; other explicit budgets measured
+// slower at Dk = 64).
 template <int PRE, bool SLOTS, bool GK, int SDT, bool DECAY, bool DELTA, int DK, int ADT>
-__global__ void __launch_bounds__(DK, SLOTS ? 1 : 1024 / DK) short_kernel(
+__device__ __forceinline__ void short_body(
     const void *__restrict__ q, const void *__restrict__ k, const void *__restrict__ v,
     const float *__restrict__ g, const uint16_t *__restrict__ beta, const float *__restrict__ gk,
     const int32_t *__restrict__ cu, const void *pool, const int32_t *__restrict__ idx,
@@ -396,15 +399,42 @@ __global__ void __launch_bounds__(DK, SLOTS ? 1 : 1024 / DK) short_kernel(
     }  // half
 }
 
+#define GDN_SHORT_PARAMS                                                                                           \
+    const void *__restrict__ q, const void *__restrict__ k, const void *__restrict__ v,                          \
+        const float *__restrict__ g, const uint16_t *__restrict__ beta, const float *__restrict__ gk,            \
+        const int32_t *__restrict__ cu, const void *pool, const int32_t *__restrict__ idx,                       \
+        const int32_t *__restrict__ token_slots, const int32_t *__restrict__ num_accepted, void *pool_w,         \
+        float scale, float eps, void *__restrict__ out, float *__restrict__ final_state, int T, int Nqk, int Nv, \
+        int Dv
+#define GDN_SHORT_ARGS \
+    q, k, v, g, beta, gk, cu, pool, idx, token_slots, num_accepted, pool_w, scale, eps, out, final_state, T, Nqk, Nv, Dv
+
+template <int PRE, bool GK, int SDT, bool DECAY, bool DELTA, int DK, int ADT>
+__global__ void __launch_bounds__(DK) short_kernel_slots(GDN_SHORT_PARAMS)
+{
+    short_body<PRE, true, GK, SDT, DECAY, DELTA, DK, ADT>(GDN_SHORT_ARGS);
+}
+
+template <int PRE, bool DECAY, bool DELTA>
+__global__ void __launch_bounds__(D, 8) short_kernel(GDN_SHORT_PARAMS)
+{
+    short_body<PRE, false, false, kF32, DECAY, DELTA, D, kBF16>(GDN_SHORT_ARGS);
+}
+
 template <int PRE, bool SLOTS, bool GK, int SDT, bool DECAY, bool DELTA, int DK, int ADT>
 static void launch_variant(dim3 grid, cudaStream_t st, const void *q, const void *k, const void *v, const float *g,
                            const uint16_t *beta, const float *gk, const int32_t *cu, const void *pool,
                            const int32_t *idx, const int32_t *token_slots, const int32_t *num_accepted, void *pool_w,
                            float scale, float eps, void *out, float *final_state, int T, int Nqk, int Nv, int Dv)
 {
-    short_kernel<PRE, SLOTS, GK, SDT, DECAY, DELTA, DK, ADT><<<grid, DK, 0, st>>>(
-        q, k, v, g, beta, gk, cu, pool, idx, token_slots, num_accepted, pool_w, scale, eps, out, final_state, T, Nqk,
-        Nv, Dv);
+    if constexpr (SLOTS)
+        short_kernel_slots<PRE, GK, SDT, DECAY, DELTA, DK, ADT><<<grid, DK, 0, st>>>(
+            q, k, v, g, beta, gk, cu, pool, idx, token_slots, num_accepted, pool_w, scale, eps, out, final_state, T,
+            Nqk, Nv, Dv);
+    else
+        short_kernel<PRE, DECAY, DELTA><<<grid, DK, 0, st>>>(q, k, v, g, beta, gk, cu, pool, idx, token_slots,
+                                                               num_accepted, pool_w, scale, eps, out, final_state, T,
+                                                               Nqk, Nv, Dv);
 }
 
 // Arguments of one pool-updating launch
