@@ -4,7 +4,7 @@ TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` are the only callers.  The CUDA path never
 imports this package and this package never imports the CUDA path.
 
-Three independent statements of the same computation live here:
+Independent statements of the computation live here:
 
 * ``recurrent``   -- the token recurrence (C, fp64), the definition that the
   GPU is compared against ("lite_boost.ops.recurrent_gated_delta_rule",
@@ -13,6 +13,8 @@ Three independent statements of the same computation live here:
   (chunk_gated_delta_rule, "Mathematical Formulas") in numpy fp64, with the
   chunk size as a parameter, exposing its per-chunk intermediates.
 * ``transition``  -- brute-force affine transition matrices for tiny shapes.
+* ``pool``, ``window`` -- the token loop with per-token pool slots (decode page)
+  and with a window of recent states (LinearAttention page, state_window).
 """
 from __future__ import annotations
 
