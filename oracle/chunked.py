@@ -4,15 +4,15 @@ Written from the page "Qwen3Next Samples" (chunk_gated_delta_rule,
 "Mathematical Formulas"), step by step in that page's order and names:
 gate cumulative sum -> decay mask -> pre-attention matrix A -> matrix
 inversion -> value and key cumulative decay -> recurrent state attention ->
-state update.  The chunk size C is a parameter ("chunk_size does not affect
-the result" on the LinearAttention operator page), so C = 1 reduces to the
-token recurrence and any C must agree with it.
+state update.  The chunk size C is a parameter (on the LinearAttention
+operator page the chunk size is an attribute with no effect on the output), so
+C = 1 reduces to the token recurrence and any C must agree with it.
 
 Readings where the page is silent or garbled (each also listed with the design notes):
 * The state is kept as S[Dk, Dv] (the decode page's layout); the page's
   ``S^T`` products therefore appear here as plain products with S.
-* M_mask ("lower triangular negative value mask") is -1 strictly below the
-  diagonal and 0 elsewhere, so the inverse is (I - A)^-1 of a strictly lower
+* M_mask (described on the page as a negative mask on the lower triangle) is
+  -1 strictly below the diagonal and 0 elsewhere, so the inverse is (I - A)^-1 of a strictly lower
   triangular A; T_tril (lower triangle of ones) includes the diagonal.
 * The garbled row recurrence of "Matrix Inversion" is read as forward
   substitution: X[i, :i] = A[i, :i] + A[i, :i] X[:i, :i], inverse = I + X.
