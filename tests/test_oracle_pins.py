@@ -345,3 +345,47 @@ def test_state_update_split_into_state_free_parts():
         Mk = k_gexp.T @ r["k_cumdecay"]
         S = r["S_in"]
         _close(np.exp(r["g_cum"][-1]) * S + N - Mk @ S, r["S_new"], 1e-12, "regrouped state update")
+
+
+def _unequal_problem(seed, lens, Dk, Dv, Nqk=1, Nv=2, P=3):
+    r = _rng(seed)
+    T = sum(lens)
+    return dict(q=r.standard_normal((T, Nqk, Dk)), k=r.standard_normal((T, Nqk, Dk)),
+                v=r.standard_normal((T, Nv, Dv)), g=-(r.random((T, Nv)) * 0.5 + 0.01),
+                beta=r.random((T, Nv)) * 0.9 + 0.05,
+                cu_seqlens=np.concatenate([[0], np.cumsum(lens)]).astype(np.int32),
+                state_pool=r.standard_normal((P, Nv, Dk, Dv)) * 0.3,
+                state_indices=r.permutation(P)[:len(lens)].astype(np.int32))
+
+
+@pytest.mark.parametrize("Dk,Dv", [(3, 5), (6, 2), (4, 16)])
+def test_unequal_head_dims_three_forms_agree(Dk, Dv):
+    """Dk != Dv (the decode page's example shape has Dk = 64, Dv = 512): the C recurrence, the chunked
+    form at several chunk sizes and the dense transition matrices give one result, the state kept as
+    [Dk, Dv] (a transposed state or a swapped head dimension cannot pass with Dk != Dv)."""
+    p = _unequal_problem(24, [9, 1, 20], Dk, Dv)
+    o1, f1 = oracle.recurrent(**p, scale=0.7, eps=1e-4)
+    assert o1.shape == (30, 2, Dv) and f1.shape == (3, 2, Dk, Dv)
+    o2, f2 = oracle.transition(**p, scale=0.7, eps=1e-4)
+    _close(o1, o2, 1e-12, "transition o")
+    _close(f1, f2, 1e-12, "transition state")
+    for C in (1, 4, 16):
+        o3, f3 = oracle.chunked(**p, scale=0.7, eps=1e-4, C=C)
+        _close(o3, o1, 1e-10, f"chunked o C={C}")
+        _close(f3, f1, 1e-10, f"chunked state C={C}")
+
+
+def test_unequal_head_dims_beta_zero_closed_form():
+    """beta = 0 with Dk != Dv: S_t = e^{sum g} S_0 and o_t = S_t^T qh_t, in both the C recurrence and
+    the chunked form."""
+    p = _unequal_problem(25, [7], 4, 9, Nv=1, P=1)
+    p["beta"] = np.zeros_like(p["beta"])
+    S0 = p["state_pool"][0, 0]
+    cum = np.cumsum(p["g"][:, 0])
+    q = p["q"][:, 0]
+    qh = 0.5 * q / np.sqrt(np.sum(q * q, axis=1, keepdims=True) + 1e-6)
+    ref = np.stack([(math.exp(cum[t]) * S0).T @ qh[t] for t in range(7)])
+    for name, fn in (("recurrence", oracle.recurrent), ("chunked", functools.partial(oracle.chunked, C=4))):
+        o, f = fn(**p, scale=0.5, eps=1e-6)
+        _close(o[:, 0], ref, 1e-12, f"{name}: o")
+        _close(f[0, 0], math.exp(cum[-1]) * S0, 1e-12, f"{name}: state")
