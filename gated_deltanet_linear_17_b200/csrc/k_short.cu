@@ -409,6 +409,13 @@ __device__ __forceinline__ void short_body(
 #define GDN_SHORT_ARGS \
     q, k, v, g, beta, gk, cu, pool, idx, token_slots, num_accepted, pool_w, scale, eps, out, final_state, T, Nqk, Nv, Dv
 
+// Two entry kernels around one body, each with its own register budget.  The pool
+// pass of the chunked forward (bf16 activations, fp32 state, one slot per sequence)
+// is held to 64 registers, eight CTAs per SM: the register file then holds eight
+// 32-column state slices, the most in flight.  The per-token-slot variants (key gate,
+// 16-bit pools, other activation types and head dimensions) keep the compiler's own
+// choice: capped at 64 they spill, and a minimum of one CTA per SM lets the compiler
+// take so many registers that only three fit.
 template <int PRE, bool GK, int SDT, bool DECAY, bool DELTA, int DK, int ADT>
 __global__ void __launch_bounds__(DK) short_kernel_slots(GDN_SHORT_PARAMS)
 {
