@@ -54,37 +54,48 @@ def flops_per_token(Nqk, Nv):
     return Nv * (4 * L * D + 2 * L * D + 6 * D * D) + Nqk * (4 * L * D)
 
 
-def stage_work(T, Nqk, Nv, NC, B):
-    """Algorithmic work of one launch of each stage: {stage: (FLOP, HBM bytes)}.
+def stage_work(T, Nqk, Nv, NC, B, B_init=0):
+    """Algorithmic work of one launch of each kernel: {kernel: (FLOP, HBM bytes)}.
 
-    FLOP: the dense tensor-core products of the stage (counted once per
-    qk-head where shared).  Bytes: what the stage must read and write in HBM
-    at least once, with NC chunks and 32 KiB fp16 tiles per (chunk, v-head):
-      intra  reads k, v, g, beta; writes U, W, Mk and the 528-byte factor
-             records (the inspection copies of gcum, betaf, rk not counted)
-      state  reads Mk, k, U, the factor records; writes S_c and the final state
-      output reads q, k, g, W, U, S_c; writes out."""
-    tile = L * D * 2
+    Both follow the operator's own counts, not this implementation's data flow.
+    FLOP: the kernel's share of the dense products of the chunked form (the
+    per-token formula above, split by the kernel that computes each product):
+      intra  U = T (beta V), W = T (beta e^gamma K) per v-head, K K^T per qk-head
+      state  W S and K~^T U' per v-head
+      output Q S and P U' per v-head, Q K^T per qk-head
+    Bytes: the operator inputs and outputs the kernel reads or writes (q, k, v,
+    g, beta, out, initial and final state), each once; the per-chunk tiles this
+    implementation passes between its kernels (U, W, Mk, S_c and the factor
+    records) are not algorithmic and are not counted:
+      intra  k, v, g, beta;  state  k, g, the initial and the final states;
+      output q, k, g, out."""
     qk, v, g, beta = T * Nqk * D * 2, T * Nv * D * 2, T * Nv * 4, T * Nv * 2
-    fa = NC * Nv * 528
-    tiles = NC * Nv * tile
+    states = (B_init + B) * Nv * D * D * 4
     return {
-        "chunk_map": (0.0, 4.0 * (B + 1) + 16.0 * NC),
-        "intra": (T * (Nv * (2 * L * D + 2 * L * D) + Nqk * 2 * L * D), qk + v + g + beta + 3 * tiles + fa),
-        "state": (T * Nv * 4 * D * D, 2 * tiles + qk + fa + tiles + B * Nv * D * D * 4),
-        "output": (T * (Nv * (2 * D * D + 2 * L * D) + Nqk * 2 * L * D), 2 * qk + g + 3 * tiles + v),
+        "chunk_map": (0.0, 4.0 * (B + 1)),
+        "intra": (T * (Nv * (2 * L * D + 2 * L * D) + Nqk * 2 * L * D), qk + v + g + beta),
+        "state": (T * Nv * 4 * D * D, qk + g + states),
+        "output": (T * (Nv * (2 * D * D + 2 * L * D) + Nqk * 2 * L * D), 2 * qk + g + v),
     }
 
 
+def step_bytes(T, Nqk, Nv, B, B_init=0):
+    """Algorithmic HBM bytes of one whole forward pass: every input read once, every output written once."""
+    return T * (2 * Nqk * D * 2 + Nv * D * 2 + Nv * 4 + Nv * 2 + Nv * D * 2) + (B_init + B) * Nv * D * D * 4
+
+
 def roofline_of(flop, nbytes, sec, peaks):
-    """The roofline that binds (the larger time at peak) and the fraction achieved on it."""
+    """The roofline that binds (the larger time at peak) and the fraction achieved on it; the other
+    side's fraction is reported beside it."""
     t_tc = flop / (peaks["bf16_tflops"] * 1e12)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    tc = {"achieved": flop / sec / 1e12, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+          "frac": flop / sec / 1e12 / peaks["bf16_tflops"], "per_launch": f"{flop:.4g} FLOP per launch"}
+    hbm = {"achieved": nbytes / sec / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+           "frac": nbytes / sec / 1e9 / peaks["hbm_gbs"], "per_launch": f"{nbytes:.4g} bytes per launch"}
     if t_hbm >= t_tc:
-        return {"bound": "hbm", "achieved": nbytes / sec / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": nbytes / sec / 1e9 / peaks["hbm_gbs"], "per_launch": f"{nbytes:.4g} bytes per launch"}
-    return {"bound": "tensor", "achieved": flop / sec / 1e12, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": flop / sec / 1e12 / peaks["bf16_tflops"], "per_launch": f"{flop:.4g} FLOP per launch"}
+        return {"bound": "hbm", **hbm, "other": {"bound": "tensor", "frac": tc["frac"]}}
+    return {"bound": "tensor", **tc, "other": {"bound": "hbm", "frac": hbm["frac"]}}
 
 
 def measured_traffic(kernel, units):
@@ -323,20 +334,31 @@ def main():
     tc_frac = F * T / (ms / 1e3) / (peaks["bf16_tflops"] * 1e12)
 
     nchunks = sum((n + L - 1) // L for n in inp.seqlens)
-    work = stage_work(T, Nqk, Nv, nchunks, inp.B)
+    b_init = inp.B if inp.state_pool is not None else 0
+    work = stage_work(T, Nqk, Nv, nchunks, inp.B, b_init)
     dom = max(names, key=lambda n: stage_ms[n])
     units = nchunks * Nv  # (chunk, v-head) pairs, the CTAs of the intra and output kernels
-    roofline = {"kernel": dom, **roofline_of(*work[dom], stage_ms[dom] / 1e3, peaks),
-                "traffic": measured_traffic(f"{dom}_kernel", units),
-                "peak_source": f"{peaks['source']} (burst bf16 / STREAM copy)"}
-    stage_roofline = {n: {k: (round(v, 4) if isinstance(v, float) else v) for k, v in
-                          roofline_of(*work[n], stage_ms[n] / 1e3, peaks).items() if k in ("bound", "frac")}
-                      for n in names if n != "chunk_map"}
+    traffic = measured_traffic(f"{dom}_kernel", units)
+    roofline = {"kernel": dom, **roofline_of(*work[dom], stage_ms[dom] / 1e3, peaks), "traffic": traffic,
+                "traffic_over_algorithmic": None if traffic is None else traffic / work[dom][1],
+                "peak_source": f"{peaks['source']} (burst bf16 / STREAM copy)",
+                "work": "FLOP and bytes of the operator's chunked form (see stage_work), no intermediate tiles"}
+    stage_roofline = {n: {"bound": r["bound"], "frac": round(r["frac"], 4), "other_frac": round(r["other"]["frac"], 4)}
+                      for n in names if n != "chunk_map"
+                      for r in [roofline_of(*work[n], stage_ms[n] / 1e3, peaks)]}
+    # the whole forward pass: the headline fraction of the tensor roofline, and the HBM side
+    sbytes = step_bytes(T, Nqk, Nv, inp.B, b_init)
+    step_traffic = [measured_traffic(f"{n}_kernel", units) for n in ("intra", "state", "output")]
+    step_roofline = {"tc_frac": tc_frac, "flop": F * T, "bytes": sbytes,
+                     "hbm_frac": sbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                     "floor_ms": 1e3 * max(F * T / (peaks["bf16_tflops"] * 1e12), sbytes / (peaks["hbm_gbs"] * 1e9)),
+                     "dram_traffic": None if None in step_traffic else sum(step_traffic),
+                     "traffic_over_algorithmic": None if None in step_traffic else sum(step_traffic) / sbytes}
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; see inputs.CONFIGS)",
-            "config": workload_config(inp), "tc_frac": tc_frac,
+            "config": workload_config(inp), "tc_frac": tc_frac, "step_roofline": step_roofline,
             "stages_ms": {n: round(v, 5) for n, v in stage_ms.items()}, "roofline": roofline,
             "stage_roofline": stage_roofline,
             "staged_ms_per_step": staged_ms, "pipeline_ranges": gdn.pipeline_ranges(T, B),

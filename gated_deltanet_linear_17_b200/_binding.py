@@ -24,6 +24,12 @@ GDN_OK, GDN_ERR_NULL_ARG, GDN_ERR_BAD_SHAPE, GDN_ERR_UNSUPPORTED = 0, 1, 2, 3
 GDN_ERR_ALIGNMENT, GDN_ERR_WORKSPACE, GDN_ERR_CUDA, GDN_ERR_OVERLAP = 4, 5, 6, 7
 GDN_ERR_SCRATCH_LIMIT = 8
 NOALLOC_SCRATCH_BYTES = 64 << 20
+# bits of the device status words (GDN_DEV_* in gdn.h): word 0 cu_seqlens, word 2 waits, word 3 fp16 range
+DEV_BITS = {0: {1: "cu[0] != 0", 2: "cu_seqlens decreasing", 4: "cu[B] != T"},
+            2: {1: "a wait of the state pass gave up", 2: "a wait of the output kernel gave up",
+                4: "a wait of the intra-chunk kernel gave up", 8: "the self-test wait gave up"},
+            3: {1: "U (or beta v) beyond the fp16 range", 2: "the state beyond the fp16 range",
+                4: "the output kernel's fp16 operand beyond the fp16 range"}}
 # update rules of gdn_chunk_fwd_rule and gdn_recurrent_fwd (GDN_RULE_* in gdn.h)
 UPDATE_RULES = {"gated_delta": 0, "delta": 1, "gated": 2, "linear": 3}
 # element types of gdn_recurrent_fwd (GDN_DTYPE_* in gdn.h)
@@ -63,6 +69,12 @@ def lib():
         L.gdn_chunk_fwd_noalloc.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, i32, p]
         L.gdn_selftest_umma.restype = ctypes.c_int
         L.gdn_selftest_umma.argtypes = [p, p, p, i32, i32, i32, i32, i32, p, p]
+        L.gdn_selftest_wait.restype = ctypes.c_int
+        L.gdn_selftest_wait.argtypes = [i32, i32, p, sz, p]
+        L.gdn_read_status.restype = ctypes.c_int
+        L.gdn_read_status.argtypes = [p, p, p]
+        L.gdn_noalloc_read_status.restype = ctypes.c_int
+        L.gdn_noalloc_read_status.argtypes = [p, p]
         L.gdn_short_fwd.restype = ctypes.c_int
         L.gdn_short_fwd.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, p]
         L.gdn_recurrent_fwd.restype = ctypes.c_int
@@ -158,7 +170,7 @@ def _resolve(q, k, v, g, beta, cu_seqlens, state_pool, state_indices):
 
 def chunk_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None, scale=None, eps=1e-6,
               max_seqlen: int = 0, out=None, final_state=None, output_final_state=True, workspace=None,
-              stream=None, update_rule="gated_delta"):
+              stream=None, update_rule="gated_delta", check_status=False):
     """Gated Delta Rule forward through ``gdn_chunk_fwd`` (``gdn_chunk_fwd_rule`` for another
     ``update_rule``: delta, gated or linear); returns (out, final_state).
 
@@ -166,7 +178,10 @@ def chunk_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None,
     bf16; cu_seqlens [B+1] int32; state_pool [P, Nv, 128, 128] fp32 or None;
     state_indices [B] int32 or None.  All on one CUDA device.  ``max_seqlen``
     in 1..16 selects the fused short-sequence kernel.  g is not needed by the
-    delta and linear rules, beta not by the gated and linear rules (pass None)."""
+    delta and linear rules, beta not by the gated and linear rules (pass None).
+    ``check_status`` waits for the call and raises RuntimeError when the device
+    status words of the chunked path report a malformed cu_seqlens, a wait that
+    gave up or a value beyond the fp16 range (see ``read_status``)."""
     if update_rule not in UPDATE_RULES:
         raise ValueError(f"update_rule must be one of {sorted(UPDATE_RULES)}")
     rule = UPDATE_RULES[update_rule]
@@ -203,6 +218,10 @@ def chunk_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None,
                                       _ptr(final_state), T, B, Nqk, Nv, P, rule, int(max_seqlen), _ptr(workspace),
                                       ws_bytes, _stream(stream))
         _check(rc, "gdn_chunk_fwd_rule")
+    if check_status and workspace is not None and not short:
+        found = decode_status(read_status(workspace, stream))
+        if found:
+            raise RuntimeError("gdn_chunk_fwd: " + "; ".join(found))
     return out, final_state
 
 
@@ -225,6 +244,31 @@ def chunk_fwd_noalloc(q, k, v, g, beta, cu_seqlens, out, final_state=None, state
                                      _ptr(final_state), T, B, Nqk, Nv, P, int(max_seqlen), _stream(stream))
     _check(rc, "gdn_chunk_fwd_noalloc")
     return out, final_state
+
+
+def decode_status(words) -> list:
+    """Human-readable findings of the four device status words (empty when all is well)."""
+    words = [int(w) for w in words]
+    return [msg for w, bits in DEV_BITS.items() for b, msg in bits.items() if words[w] & b]
+
+
+def read_status(workspace, stream=None) -> list:
+    """The workspace's four device status words (``gdn_read_status``), after the stream's work is done."""
+    st = torch.cuda.current_stream() if stream is None else stream
+    dst = torch.zeros(4, dtype=torch.int32, device=workspace.device)
+    _check(lib().gdn_read_status(_ptr(workspace), _ptr(dst), _stream(st)), "gdn_read_status")
+    st.synchronize()
+    return dst.cpu().tolist()
+
+
+def noalloc_status(stream=None) -> list:
+    """The four device status words of the allocation-free entry's scratch (``gdn_noalloc_read_status``),
+    copied into pinned host memory without any device allocation."""
+    st = torch.cuda.current_stream() if stream is None else stream
+    dst = torch.zeros(4, dtype=torch.int32, pin_memory=True)
+    _check(lib().gdn_noalloc_read_status(_ptr(dst), _stream(st)), "gdn_noalloc_read_status")
+    st.synchronize()
+    return dst.tolist()
 
 
 def pipeline_ranges(T, B, Nqk=1, Nv=1):

@@ -249,6 +249,19 @@ __device__ __forceinline__ void chunk_gamma(const float *__restrict__ g, int Nv,
 // Wider spans take e^{gamma_i - gamma_j} element by element.
 constexpr float kSpanMax = 64.f;
 
+// Largest finite fp16 magnitude: an fp32 value above it does not fit an fp16 operand tile
+// (the kernels record that in status word 3 instead of computing on an infinity silently).
+constexpr float kFp16Max = 65504.f;
+// max(m, |x|) that keeps a NaN (a NaN operand never fits either), so that
+// out_of_fp16(m) also catches NaN and infinite values
+__device__ __forceinline__ float absmax_nan(float m, float x)
+{
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(m), "f"(fabsf(x)));
+    return r;
+}
+__device__ __forceinline__ bool out_of_fp16(float m) { return !(m <= kFp16Max); }
+
 // d[0..N) = s[0..N) from shared memory in 16-byte loads (s 16-byte aligned).  Loading
 // a row's per-column factors into registers ahead of the row's stores keeps the
 // loads from being ordered after stores the compiler cannot tell apart from them.

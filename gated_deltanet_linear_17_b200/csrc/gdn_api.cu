@@ -20,7 +20,7 @@ using gdn::Workspace;
 
 namespace {
 
-constexpr int kVersion = 100;  // 0.1.0
+constexpr int kVersion = 200;  // 0.2.0
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -201,6 +201,14 @@ const char *gdn_status_string(int status)
 }
 
 int gdn_version(void) { return kVersion; }
+
+int gdn_read_status(const void *workspace, int32_t *status_out, void *stream)
+{
+    if (!workspace || !status_out) return GDN_ERR_NULL_ARG;
+    if (!aligned16(workspace) || (reinterpret_cast<uintptr_t>(status_out) & 3u)) return GDN_ERR_ALIGNMENT;
+    return cuda_status(cudaMemcpyAsync(status_out, workspace, 4 * sizeof(int32_t), cudaMemcpyDefault,
+                                       (cudaStream_t)stream));
+}
 
 int gdn_workspace_layout(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, gdn_workspace_layout_t *layout)
 {

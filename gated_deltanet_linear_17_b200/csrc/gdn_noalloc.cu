@@ -44,18 +44,29 @@ extern "C" int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const
                                      float *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
                                      int32_t max_seqlen, void *stream)
 {
+    // sizes that gdn_chunk_fwd refuses get its code, before the scratch limit is looked at
+    if (T < 0 || B < 0 || Nqk <= 0 || Nv <= 0 || P < 0 || Nv % Nqk != 0) return GDN_ERR_BAD_SHAPE;
+    if (T >= (int64_t(1) << 31) || Nqk > 64 || Nv > 256) return GDN_ERR_UNSUPPORTED;
     const bool short_path = max_seqlen >= 1 && max_seqlen <= GDN_SHORT_MAX;
-    if (!short_path && T >= 0 && B >= 0 && Nqk > 0 && Nv > 0) {
-        // reject sizes whose workspace does not fit, before anything is enqueued
-        if (gdn_chunk_fwd_workspace_bytes(T, B, Nqk, Nv) > (size_t)GDN_NOALLOC_SCRATCH_BYTES)
-            return GDN_ERR_SCRATCH_LIMIT;
-    }
+    // reject sizes whose workspace does not fit, before anything is enqueued
+    if (!short_path && gdn_chunk_fwd_workspace_bytes(T, B, Nqk, Nv) > (size_t)GDN_NOALLOC_SCRATCH_BYTES)
+        return GDN_ERR_SCRATCH_LIMIT;
     void *scratch = nullptr;
     const int rc = scratch_address(&scratch);
     if (rc != GDN_OK) return rc;
-    // Nothing in the workspace has to start at zero: every region a kernel
-    // reads is written earlier in the same call, so the previous call's
-    // leftovers are never used.  A non-NULL workspace means no allocation.
+    // Nothing in the workspace has to start at zero: the chunk-table kernel
+    // clears the status words first, and every other region a kernel reads is
+    // written earlier in the same call, so the previous call's leftovers are
+    // never used.  A non-NULL workspace means no allocation.
     return gdn_chunk_fwd(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, scale, eps, out, final_state, T,
                          B, Nqk, Nv, P, max_seqlen, scratch, (size_t)GDN_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+extern "C" int gdn_noalloc_read_status(int32_t *status_out, void *stream)
+{
+    if (!status_out) return GDN_ERR_NULL_ARG;
+    void *scratch = nullptr;
+    const int rc = scratch_address(&scratch);
+    if (rc != GDN_OK) return rc;
+    return gdn_read_status(scratch, status_out, stream);
 }

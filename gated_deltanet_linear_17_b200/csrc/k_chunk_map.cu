@@ -85,8 +85,12 @@ __global__ void __launch_bounds__(kMapThreads) chunk_map_kernel(const int32_t *_
         info[c] = make_int4(lo, t, min(L, e - t), j);
     }
     if (tid == 0) {
+        // this kernel runs first in every chunked call, on the caller's stream: the wait and
+        // range bits of an earlier call on this workspace are cleared before any kernel can set them
         status[0] = err_bits;
         status[1] = total;
+        status[2] = 0;
+        status[3] = 0;
     }
     for (int i = total + tid; i < NC; i += kMapThreads) info[i] = make_int4(-1, 0, 0, 0);
 }

@@ -36,6 +36,7 @@
 // bounded; if one gives up, the CTA sets bit 2 of
 // status[2], lets its MMAs and open loads drain and stops.
 #include "common.cuh"
+#include "gdn.h"
 #include "gdn_internal.h"
 #include "tc100.cuh"
 #include "tma.cuh"
@@ -112,9 +113,9 @@ __device__ __forceinline__ void warp_store16(const float (&acc)[2][4], uint8_t *
 // Rewrite a 128 x 128 tile of raw bf16 rows in place as fp16 rows scaled by fac(r),
 // rows from nvalid on as zeros; NT threads (t = 0 .. NT - 1), thread t at chunk t % 16 of
 // rows t / 16 + (NT / 16) i, eight rows at a time with their loads issued before any
-// conversion
-template <int NT, typename F>
-__device__ __forceinline__ void scale_rows_f16(uint8_t *tile, int t, int nvalid, F fac)
+// conversion.  With TRACK, vmax keeps the largest magnitude written (fp16 range check).
+template <int NT, bool TRACK = false, typename F>
+__device__ __forceinline__ void scale_rows_f16(uint8_t *tile, int t, int nvalid, F fac, float *vmax = nullptr)
 {
     constexpr int kStep = NT / 16, kRows = 128 / kStep;
 #pragma unroll 1
@@ -131,6 +132,14 @@ __device__ __forceinline__ void scale_rows_f16(uint8_t *tile, int t, int nvalid,
         for (int i = 0; i < 8; ++i) {
             const int r = (t >> 4) + kStep * (b + i);
             const float m = f[i];
+            if (TRACK && r < nvalid) {
+                const uint32_t w4[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+                float mx = 0.f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    mx = absmax_nan(absmax_nan(mx, __uint_as_float(w4[e] << 16)), __uint_as_float(w4[e] & 0xffff0000u));
+                *vmax = absmax_nan(*vmax, mx * m);
+            }
             *reinterpret_cast<uint4 *>(tile + t128(r, t & 15)) =
                 r < nvalid
                     ? make_uint4(pack_h2(__uint_as_float(x[i].x << 16) * m, __uint_as_float(x[i].x & 0xffff0000u) * m),
@@ -207,6 +216,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
         xb = beta ? bf2f(beta[(size_t)(ci.start + tid) * Nv + h]) : 0.f;
     }
     bool ok = true;
+    float vmax = 0.f;  // largest magnitude of the fp16 U tiles (range check; a NaN is kept)
     uint32_t mma_phase = 0, v_par = 0, ld_par = 0;
     bool ld_pend = true, v_pend = true;  // a load phase issued and not yet waited on
     auto wait_bar = [&](uint32_t bar, uint32_t parity) {  // bounded, outcome shared with the CTA
@@ -304,7 +314,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
             if (ok) wait_bar(bar_v, v_par);
             if (ok) {
                 v_pend = false;
-                scale_rows_f16<kIntraThreads>(smem + OFF_T1, tid, n, [&](int) { return 1.f; });
+                scale_rows_f16<kIntraThreads, true>(smem + OFF_T1, tid, n, [&](int) { return 1.f; }, &vmax);  // U = v
                 if (tid < kFaStride) {
                     const float gl = gam[127];
                     fa[(size_t)(c * Nv + h) * kFaStride + tid] =
@@ -319,7 +329,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
                 tma::store_2d(&tm_u, 64, urow, sbase + OFF_T1 + 16384);
                 tma::commit_group();
             } else if (!ok && tid == 0) {
-                atomicOr(status + 2, 4);
+                atomicOr(status + 2, GDN_DEV_WAIT_INTRA);
                 tc::commit(bar_d);
                 tc::mbar_wait_bounded(bar_d, 0);
                 if (ld_pend) tc::mbar_wait_bounded(bar_ld, ld_par);
@@ -542,6 +552,12 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
             for (int j0 = 0; j0 < 128; j0 += 32) {
                 float a[32];
                 tc::tmem_ld32(t_row + half * 128 + j0, a);
+                // U (v-derived; an out-of-range beta v shows up here as inf or NaN); W and Mk are bounded
+                // by T, since their other factors have entries of magnitude <= 1
+                if (half != wsel) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) vmax = absmax_nan(vmax, a[e]);
+                }
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8)
                     *reinterpret_cast<uint4 *>(dst + t128(row, (j0 >> 3) + q8)) =
@@ -622,7 +638,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
         }
         if (!ok) {
             if (tid == 0) {
-                atomicOr(status + 2, 4);
+                atomicOr(status + 2, GDN_DEV_WAIT_INTRA);
                 // MMAs and loads still in flight land before shared and tensor memory are released: a
                 // commit covers every MMA issued before it; each barrier has at most one load phase open
                 tc::commit(bar_d);
@@ -641,6 +657,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
         xb = nb;
     }
     if (tid == 0) tma::wait_read_all();  // the stores have read shared memory (the grid's end publishes them)
+    if (__any_sync(0xffffffffu, out_of_fp16(vmax)) && lane == 0) atomicOr(status + 3, GDN_DEV_RANGE_INTRA);
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();

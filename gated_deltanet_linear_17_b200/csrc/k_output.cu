@@ -41,6 +41,7 @@
 // gives up, the CTA sets bit 1 of status[2] in the workspace and skips the rest
 // of its chunk after letting its copies and MMAs drain.
 #include "common.cuh"
+#include "gdn.h"
 #include "gdn_internal.h"
 #include "tc100.cuh"
 #include "tma.cuh"
@@ -273,6 +274,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         load_tile(sbase + OO_X, &tm_u, bar_u);
         u_issued = true;
     }
+    float vmax = 0.f;  // largest magnitude of Qw (fp16 range check)
     if (ok) {
         const float qf = rqv[row] * __expf(gam[row]);
 #pragma unroll 1
@@ -294,9 +296,12 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
                 const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
                 uint32_t o4[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    o4[e] = pack_h2(__uint_as_float(w4[e] << 16) * qf - z[c4 * 8 + 2 * e],
-                                    __uint_as_float(w4[e] & 0xffff0000u) * qf - z[c4 * 8 + 2 * e + 1]);
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = __uint_as_float(w4[e] << 16) * qf - z[c4 * 8 + 2 * e];
+                    const float x1 = __uint_as_float(w4[e] & 0xffff0000u) * qf - z[c4 * 8 + 2 * e + 1];
+                    vmax = absmax_nan(absmax_nan(vmax, x0), x1);
+                    o4[e] = pack_h2(x0, x1);
+                }
                 *p = make_uint4(o4[0], o4[1], o4[2], o4[3]);
             }
         }
@@ -360,7 +365,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
             }
         }
     } else if (tid == 0) {
-        atomicOr(status + 2, 2);
+        atomicOr(status + 2, GDN_DEV_WAIT_OUTPUT);
         // copies and MMAs still in flight land before shared and tensor memory are released:
         // a commit covers every MMA issued before it; then the last load phase issued
         tc::commit(bar_d);
@@ -371,6 +376,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         if (u_issued) tc::mbar_wait_bounded(bar_u, 0);
     }
     if (tid == 0) tma::wait_read_all();  // the stores have read shared memory (the grid's end publishes them)
+    if (__any_sync(0xffffffffu, out_of_fp16(vmax)) && lane == 0) atomicOr(status + 3, GDN_DEV_RANGE_OUTPUT);
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();

@@ -98,7 +98,31 @@ __global__ void __launch_bounds__(128, 1)
     if (wid == 0) tc::tmem_dealloc(tmem, ncols);
 }
 
+// The bounded wait on an mbarrier that (without `arrive`) no one arrives on: it
+// gives up after max_polls polls and the thread records that in status word 2.
+__global__ void wait_selftest_kernel(uint32_t max_polls, int arrive, int32_t *__restrict__ status)
+{
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_addr(&bar);
+    tc::mbar_init(b, 1);
+    tc::mbar_init_fence();
+    if (arrive) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(b) : "memory");
+    if (!tc::mbar_wait_bounded(b, 0, max_polls)) atomicOr(status + 2, GDN_DEV_WAIT_SELFTEST);
+}
+
 }  // namespace gdn
+
+extern "C" int gdn_selftest_wait(int32_t max_polls, int32_t arrive, void *workspace, size_t workspace_bytes,
+                                 void *stream)
+{
+    if (!workspace) return GDN_ERR_NULL_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 15u) return GDN_ERR_ALIGNMENT;
+    if (workspace_bytes < 16) return GDN_ERR_WORKSPACE;
+    if (max_polls < 1 || max_polls > (1 << 22)) return GDN_ERR_BAD_SHAPE;
+    gdn::wait_selftest_kernel<<<1, 1, 0, (cudaStream_t)stream>>>((uint32_t)max_polls, arrive,
+                                                                 static_cast<int32_t *>(workspace));
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
 
 extern "C" int gdn_selftest_umma(const uint16_t *A, const uint16_t *B, float *C, int32_t N, int32_t K,
                                  int32_t bf16, int32_t a_mn, int32_t b_mn, int32_t *status, void *stream)

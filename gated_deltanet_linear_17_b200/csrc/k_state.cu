@@ -43,6 +43,7 @@
 // bounded: if one gives up, the CTA sets bit 0 of status[2] in the workspace,
 // stops, lets its copies and MMAs drain and frees its tensor memory.
 #include "common.cuh"
+#include "gdn.h"
 #include "gdn_internal.h"
 #include "tc100.cuh"
 #include "tma.cuh"
@@ -189,7 +190,9 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
 #pragma unroll
         for (int j = 0; j < 32; ++j) s[j] = 0.f;
     }
-    // S in fp16 as the MN-major B operand (buffer buf): row `row`, 16-byte chunks cbase/8 .. cbase/8 + 3
+    // S in fp16 as the MN-major B operand (buffer buf): row `row`, 16-byte chunks cbase/8 .. cbase/8 + 3;
+    // vmax keeps the largest magnitude converted (fp16 range check)
+    float vmax = 0.f;
     auto store_state_operand = [&](int buf) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -197,6 +200,8 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
             *reinterpret_cast<uint4 *>(smem + OFF_S + buf * 16384 + tc::sw128c(row, (cbase >> 3) + j)) =
                 make_uint4(pack_h2(v8[0], v8[1]), pack_h2(v8[2], v8[3]), pack_h2(v8[4], v8[5]), pack_h2(v8[6], v8[7]));
         }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) vmax = absmax_nan(vmax, s[j]);
     };
 
     bool ok = true;
@@ -311,8 +316,9 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
         tc::commit(bar_d);
         tc::mbar_wait_bounded(bar_d, 0);
     }
+    if (epi && __any_sync(0xffffffffu, out_of_fp16(vmax)) && lane == 0) atomicOr(status + 3, GDN_DEV_RANGE_STATE);
     if (!ok) {
-        if (tid == 0) atomicOr(status + 2, 1);
+        if (tid == 0) atomicOr(status + 2, GDN_DEV_WAIT_STATE);
     } else if (epi && (final_state || to_carry)) {
         float *base = to_carry ? carry + (size_t)range * Nv * D * D : final_state + (size_t)b * Nv * D * D;
         float4 *dst = reinterpret_cast<float4 *>(base + ((size_t)h * D + row) * D + col0 + cbase);

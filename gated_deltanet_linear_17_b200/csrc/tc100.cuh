@@ -185,9 +185,9 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t addr, uint32_t parity)
 // thousand); kMaxPolls bounds the wait to well under a second.  Returns false
 // when it gives up.
 constexpr uint32_t kMaxPolls = 1u << 22;
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t addr, uint32_t parity)
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t addr, uint32_t parity, uint32_t max_polls = kMaxPolls)
 {
-    for (uint32_t i = 0; i < kMaxPolls; ++i) {
+    for (uint32_t i = 0; i < max_polls; ++i) {
         if (mbar_test_wait(addr, parity)) return true;
         if (i > 4096) __nanosleep(64);
     }

@@ -34,7 +34,50 @@
  *     beta in [0, 1] (the decode page leaves both unchecked on purpose, since
  *     a reduction over the inputs would cost a pass on the inference path);
  *     state_indices must lie in [0, P).
- *   - Return value: a gdn_status_t code (0 = success).
+ *   - Return value: a gdn_status_t code (0 = success).  It covers what the host
+ *     can see when it enqueues.  What only the device can see (a malformed
+ *     cu_seqlens, a bounded wait that gave up, a value outside the fp16 range)
+ *     goes to the status words of the chunked path's workspace, which
+ *     gdn_read_status copies out (see "Device status" below).
+ *
+ * Device status (the chunked path: gdn_chunk_fwd, gdn_chunk_fwd_rule, the
+ * stage calls of gdn_stages.h and gdn_chunk_fwd_noalloc).  The decode page's
+ * operator raises ValueError for bad arguments and RuntimeError when
+ * execution fails; here the host checks come back as the return code and the
+ * device-side findings as four int32 words at the start of the workspace:
+ *   [0] cu_seqlens errors: GDN_DEV_CU_FIRST (cu[0] != 0), GDN_DEV_CU_DECREASING,
+ *       GDN_DEV_CU_TOTAL (cu[B] != T).  The chunk table clamps every token range
+ *       to [0, T), so nothing is read or written out of bounds, but the
+ *       results are those of the clamped lengths.
+ *   [1] the number of chunks.
+ *   [2] bounded waits that gave up: GDN_DEV_WAIT_STATE, GDN_DEV_WAIT_OUTPUT,
+ *       GDN_DEV_WAIT_INTRA (GDN_DEV_WAIT_SELFTEST: the test hook of
+ *       gdn_testing.h).  Every wait of a kernel on the tensor core or on a TMA
+ *       copy gives up after about 0.3 s instead of hanging; the CTA then stops,
+ *       lets its copies drain and frees its tensor memory.
+ *   [3] values outside the fp16 range (|x| > 65504) in an fp16 intermediate:
+ *       GDN_DEV_RANGE_INTRA (U, or beta v, which shows up in U),
+ *       GDN_DEV_RANGE_STATE (the state's fp16 operand copy),
+ *       GDN_DEV_RANGE_OUTPUT (the output kernel's fp16 operand).  A NaN in
+ *       one of them also sets the bit.  See "fp16 intermediates" below.
+ * Words 0, 2 and 3 are cleared at the start of every chunked call (by the
+ * chunk-table kernel, on `stream`, before any kernel that sets a bit), so the
+ * words describe the last chunked call on that workspace.  A nonzero word 2 or
+ * 3 means that call's out and final_state are not valid.  The fused
+ * short-sequence path (1 <= max_seqlen <= GDN_SHORT_MAX) computes in fp32,
+ * has no waits and no workspace, and writes no status.
+ *
+ * fp16 intermediates.  The chunked path's tensor-core operands other than the
+ * raw q and k rows are fp16 with fp32 accumulation (11 significant bits
+ * against bf16's 8).  Values derived from v and from the initial state (U, the
+ * state, the output before its bf16 rounding) must therefore stay within
+ * +-65504; beyond that the result is not valid and word 3 says so.  Far below
+ * 2^-14 (about 6e-5) fp16 loses significant bits and the result loses
+ * accuracy without a flag.  The operator is linear in (v, initial state)
+ * jointly, so a caller whose v and states are far outside 1e-3 .. 1e3 in
+ * magnitude can scale both by a power of two and scale out and final_state
+ * back.  The fused short-sequence path and gdn_recurrent_fwd compute in fp32
+ * and have neither limit.
  */
 #ifndef GDN_H_
 #define GDN_H_
@@ -62,6 +105,18 @@ extern "C" {
 #define GDN_RULE_GATED 2
 #define GDN_RULE_LINEAR 3
 
+/* bits of the device status words (see "Device status" above) */
+#define GDN_DEV_CU_FIRST 1      /* word 0: cu[0] != 0                  */
+#define GDN_DEV_CU_DECREASING 2 /* word 0: cu[b+1] < cu[b] for some b   */
+#define GDN_DEV_CU_TOTAL 4      /* word 0: cu[B] != T                   */
+#define GDN_DEV_WAIT_STATE 1    /* word 2: a wait of the state pass gave up     */
+#define GDN_DEV_WAIT_OUTPUT 2   /* word 2: a wait of the output kernel gave up  */
+#define GDN_DEV_WAIT_INTRA 4    /* word 2: a wait of the intra-chunk kernel gave up */
+#define GDN_DEV_WAIT_SELFTEST 8 /* word 2: the wait of gdn_selftest_wait gave up */
+#define GDN_DEV_RANGE_INTRA 1   /* word 3: U (or beta v) beyond +-65504         */
+#define GDN_DEV_RANGE_STATE 2   /* word 3: the state beyond +-65504             */
+#define GDN_DEV_RANGE_OUTPUT 4  /* word 3: the output kernel's fp16 operand beyond +-65504 */
+
 typedef enum {
     GDN_OK = 0,
     GDN_ERR_NULL_ARG = 1,    /* a required pointer is NULL                              */
@@ -80,6 +135,22 @@ const char *gdn_status_string(int status);
 
 /* Library ABI version: major * 10000 + minor * 100 + patch. */
 int gdn_version(void);
+
+/*
+ * gdn_read_status -- copy the four device status words (see "Device status")
+ * of a chunked-path workspace into status_out, in order on `stream`.
+ *
+ *   workspace    the device workspace the chunked call ran on (16-byte aligned)
+ *   status_out   int32[4], device memory or host memory (pinned host memory
+ *                keeps the copy asynchronous; pageable memory makes the call
+ *                wait for `stream`); valid once the copy has completed on
+ *                `stream`
+ * Errors: GDN_ERR_NULL_ARG, GDN_ERR_ALIGNMENT, GDN_ERR_CUDA.  A call of
+ * gdn_chunk_fwd with workspace == NULL frees its internal workspace before it
+ * returns, so there is nothing to read afterwards: pass a workspace to read
+ * the status.
+ */
+int gdn_read_status(const void *workspace, int32_t *status_out, void *stream);
 
 /*
  * Bytes of device workspace that the chunked path of gdn_chunk_fwd needs for
@@ -115,7 +186,8 @@ size_t gdn_chunk_fwd_workspace_bytes(int64_t T, int32_t B, int32_t Nqk, int32_t 
  *                 only chooses the faster one.
  *   workspace     device buffer of workspace_bytes >= gdn_chunk_fwd_workspace_bytes,
  *                 or NULL: the call then allocates and frees it stream-ordered
- *                 (cudaMallocAsync / cudaFreeAsync on `stream`).
+ *                 (cudaMallocAsync / cudaFreeAsync on `stream`).  Its first 16
+ *                 bytes receive the device status words (gdn_read_status).
  *
  * Alignment: q, k, v, out, state_pool, final_state and workspace 16-byte aligned.
  * Limits: T < 2^31, Nqk <= 64, Nv <= 256 (else GDN_ERR_UNSUPPORTED).
@@ -169,24 +241,42 @@ int gdn_chunk_fwd_rule(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
  *
  * Limit: sizes whose chunked-path workspace (gdn_chunk_fwd_workspace_bytes)
  * exceeds 64 MiB are rejected with GDN_ERR_SCRATCH_LIMIT before anything is
- * enqueued (at Nqk = 16, Nv = 32 that is about 1500 tokens in one sequence).
- * The fused short-sequence path (1 <= max_seqlen <= GDN_SHORT_MAX) uses no
- * workspace and has no such limit.
+ * enqueued (at B = 1, Nqk = 16, Nv = 32 the longest sequence that fits is
+ * 1920 tokens, 15 chunks; for other sizes compare
+ * gdn_chunk_fwd_workspace_bytes with GDN_NOALLOC_SCRATCH_BYTES).  Arguments
+ * that gdn_chunk_fwd would refuse (a bad shape, unsupported sizes) get that
+ * code first.  The fused short-sequence path (1 <= max_seqlen <=
+ * GDN_SHORT_MAX) uses no workspace and has no such limit.
  *
  * The buffer used is the one of the calling thread's current device; `stream`
  * must belong to that device.  The first call on a device looks up the
- * buffer's device address (cudaGetSymbolAddress) and keeps it; make that first
- * call before any stream capture.  All calls on one device share the buffer,
- * which keeps whatever the previous call left in it (no call depends on it
- * starting at zero): calls that can overlap on the GPU (unordered streams,
- * several host threads) race on it and corrupt each other's results, so
- * order them on one stream.
+ * buffer's device address (cudaGetSymbolAddress) and keeps it for the life of
+ * the process; make that first call before any stream capture.  The kept
+ * address belongs to the device's primary context, which the CUDA runtime
+ * uses: a caller that switches the thread to another driver context, or calls
+ * cudaDeviceReset after the first call, must not use this entry afterwards.
+ * All calls on one device share the buffer,
+ * which keeps whatever the previous call left in it (every call clears the
+ * status words and writes every other region before reading it, so no call
+ * depends on what an earlier one left): calls that can overlap on the GPU
+ * (unordered streams, several host threads) race on it and corrupt each
+ * other's results, so order them on one stream.  gdn_noalloc_read_status
+ * copies the scratch's device status words (see "Device status") of the last
+ * chunked call out, without allocating.
  */
 int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
                           const uint16_t *beta, const int32_t *cu_seqlens, const float *state_pool,
                           const int32_t *state_indices, float scale, float eps, uint16_t *out,
                           float *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
                           int32_t max_seqlen, void *stream);
+
+/*
+ * gdn_noalloc_read_status -- gdn_read_status for the static scratch of
+ * gdn_chunk_fwd_noalloc on the current device: copies its four status words
+ * into status_out (int32[4], device or host memory) in order on `stream`.
+ * Allocates nothing.  GDN_ERR_NULL_ARG, GDN_ERR_CUDA.
+ */
+int gdn_noalloc_read_status(int32_t *status_out, void *stream);
 
 /*
  * gdn_recurrent_fwd -- token recurrence on a state pool updated in place, with

@@ -18,6 +18,7 @@
 #ifndef GDN_TESTING_H_
 #define GDN_TESTING_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #include "gdn.h"
@@ -28,6 +29,20 @@ extern "C" {
 
 int gdn_selftest_umma(const uint16_t *A, const uint16_t *B, float *C, int32_t N, int32_t K, int32_t bf16,
                       int32_t a_mn, int32_t b_mn, int32_t *status, void *stream);
+
+/*
+ * gdn_selftest_wait: the bounded mbarrier wait of the kernels, run out on
+ * purpose without faulting or hanging.  One thread initialises an mbarrier
+ * that expects one arrival, arrives on it if `arrive` is nonzero, and waits
+ * for its phase with at most `max_polls` polls (the kernels use 2^22, about
+ * 0.3 s).  Without the arrival the wait gives up, and the thread sets
+ * GDN_DEV_WAIT_SELFTEST in status word 2 of `workspace` (the word that the
+ * chunked kernels use for their own waits; read it with gdn_read_status).
+ * Nothing else is touched: no copy or tensor-core work is in flight.
+ *   max_polls   1 .. 2^22
+ *   workspace   device, 16-byte aligned, at least 16 bytes
+ */
+int gdn_selftest_wait(int32_t max_polls, int32_t arrive, void *workspace, size_t workspace_bytes, void *stream);
 
 #ifdef __cplusplus
 }

@@ -34,7 +34,8 @@ def lib():
 def test_headers_declare_entry_points():
     names = _declared()
     for n in ("gdn_chunk_fwd", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string", "gdn_short_fwd",
-              "gdn_stage_intra", "gdn_stage_state", "gdn_stage_output"):
+              "gdn_stage_intra", "gdn_stage_state", "gdn_stage_output", "gdn_read_status",
+              "gdn_noalloc_read_status", "gdn_selftest_wait"):
         assert n in names
 
 
@@ -174,3 +175,51 @@ def test_python_layer_refuses_cpu_tensors():
     inp = inputs.make([5], 1, 2, seed=0)
     with pytest.raises(RuntimeError):
         gdn.chunk_fwd(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens)
+
+
+def _noalloc(lib, **over):
+    M = 1 << 20  # fake, disjoint, 16-byte aligned addresses; every call below returns before any launch
+    a = dict(T=8, B=1, Nqk=2, Nv=4, P=0, max_seqlen=0)
+    a.update(over)
+    vp = ctypes.c_void_p
+    return lib.gdn_chunk_fwd_noalloc(vp(M), vp(2 * M), vp(3 * M), vp(4 * M), vp(5 * M), vp(6 * M), None, None, 0.0,
+                                     1e-6, vp(7 * M), None, a["T"], a["B"], a["Nqk"], a["Nv"], a["P"],
+                                     a["max_seqlen"], None)
+
+
+def test_noalloc_refuses_bad_shapes_before_the_scratch_limit(lib):
+    # sizes large enough to exceed the scratch, but invalid for gdn_chunk_fwd too: the shape code wins
+    assert _noalloc(lib, T=1 << 20, Nqk=2, Nv=3) == B.GDN_ERR_BAD_SHAPE
+    assert _noalloc(lib, T=1 << 20, Nqk=128, Nv=128) == B.GDN_ERR_UNSUPPORTED
+    assert _noalloc(lib, T=1 << 20, P=-1) == B.GDN_ERR_BAD_SHAPE
+    assert _noalloc(lib, T=1 << 20, Nqk=16, Nv=32) == B.GDN_ERR_SCRATCH_LIMIT
+    # the stated limit: one sequence of 1920 tokens at Nqk = 16, Nv = 32 fits, 1921 does not
+    assert gdn.workspace_bytes(1920, 1, 16, 32) <= B.NOALLOC_SCRATCH_BYTES < gdn.workspace_bytes(1921, 1, 16, 32)
+    assert _noalloc(lib, T=1921, Nqk=16, Nv=32) == B.GDN_ERR_SCRATCH_LIMIT
+    assert "1920 tokens" in open(os.path.join(ROOT, "include", "gdn.h")).read()
+
+
+def test_status_entry_argument_errors(lib):
+    vp = ctypes.c_void_p
+    assert lib.gdn_read_status(None, vp(1 << 20), None) == B.GDN_ERR_NULL_ARG
+    assert lib.gdn_read_status(vp(1 << 20), None, None) == B.GDN_ERR_NULL_ARG
+    assert lib.gdn_read_status(vp((1 << 20) + 8), vp(2 << 20), None) == B.GDN_ERR_ALIGNMENT
+    assert lib.gdn_read_status(vp(1 << 20), vp((2 << 20) + 2), None) == B.GDN_ERR_ALIGNMENT
+    assert lib.gdn_noalloc_read_status(None, None) == B.GDN_ERR_NULL_ARG
+    assert lib.gdn_selftest_wait(16, 0, None, 16, None) == B.GDN_ERR_NULL_ARG
+    assert lib.gdn_selftest_wait(16, 0, vp((1 << 20) + 4), 16, None) == B.GDN_ERR_ALIGNMENT
+    assert lib.gdn_selftest_wait(16, 0, vp(1 << 20), 8, None) == B.GDN_ERR_WORKSPACE
+    assert lib.gdn_selftest_wait(0, 0, vp(1 << 20), 16, None) == B.GDN_ERR_BAD_SHAPE
+    assert lib.gdn_selftest_wait((1 << 22) + 1, 0, vp(1 << 20), 16, None) == B.GDN_ERR_BAD_SHAPE
+
+
+def test_status_bits_match_the_header():
+    text = open(os.path.join(ROOT, "include", "gdn.h")).read()
+    macros = {m.group(1): int(m.group(2)) for m in re.finditer(r"#define (GDN_DEV_\w+) (\d+)", text)}
+    word = {"CU": 0, "WAIT": 2, "RANGE": 3}
+    for name, bit in macros.items():
+        assert bit in B.DEV_BITS[word[name.split("_")[2]]], name
+    assert sum(len(v) for v in B.DEV_BITS.values()) == len(macros)
+    assert gdn.decode_status([0, 5, 0, 0]) == []
+    assert gdn.decode_status([2, 5, 4, 2]) == ["cu_seqlens decreasing", "a wait of the intra-chunk kernel gave up",
+                                               "the state beyond the fp16 range"]
