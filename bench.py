@@ -504,16 +504,52 @@ def main():
         line["decode_bf16"] = decode_line("decode_b256_bf16")
         line["decode_bf16_dk64_dv512"] = decode_line("decode_dk64_dv512")
 
+        # a state window of the LinearAttention page (gdn_recurrent_window_fwd): 256 sequences of 2 tokens, W = 4
+        W = 4
+        wc = inputs.make([2] * 256, Nqk=16, Nv=32, g=("uniform_neg", 1.0, 0.01), seed=8 + rank, name="window")
+        wgen = torch.Generator(device=dev).manual_seed(9 + rank)
+        win = torch.randn(W, wc.B, wc.Nv, D, D, device=dev, generator=wgen) * 0.02
+        wc = wc.to(dev)
+        wo = torch.empty(wc.T, wc.Nv, D, dtype=torch.bfloat16, device=dev)
+
+        def wstep():
+            gdn.recurrent_window_fwd(wc.q, wc.k, wc.v, wc.g, wc.beta, wc.cu_seqlens, win, W, scale=wc.scale,
+                                     eps=wc.eps, max_seqlen=2, out=wo)
+        for _ in range(args.warmup):
+            wstep()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            wstep()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        wms = gdist.max_over_ranks(e0.elapsed_time(e1) / args.steps, device=dev)
+        sb = wc.Nv * D * D * 4
+        # per sequence: the shift reads entries 2, 3 and writes 0, 1; the recurrence reads entry 3 and writes 2, 3
+        wb = wc.B * 7 * sb + (short_bytes(wc) - 2 * wc.B * sb)
+        line["state_window"] = {"workload": f"window_b256_w{W}: B={wc.B} x 2 tokens, Nqk={wc.Nqk}, Nv={wc.Nv}, "
+                                            f"fp32 window [{W},{wc.B},{wc.Nv},128,128] updated in place",
+                                "ms": wms, "bytes": wb, "GB/s": wb / (wms / 1e3) / 1e9,
+                                "hbm_frac": wb / (wms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                                "tokens/s": world * wc.T / (wms / 1e3),
+                                "kernel": "window_shift_kernel + short_kernel (window slots)",
+                                "call": "gdn_recurrent_window_fwd"}
+        line["gpu_launches"] += 2 * args.steps
+        del win, wc, wo
+
     # ---- end to end from pinned host buffers through the public call
     if not args.no_e2e:
         pin = lambda t: None if t is None else t.pin_memory()
         hq, hk, hv, hg, hb, hc = (pin(getattr(host, n)) for n in ("q", "k", "v", "g", "beta", "cu_seqlens"))
         oh = torch.empty(T, Nv, D, dtype=torch.bfloat16, pin_memory=True)
         fh = torch.empty(B, Nv, D, D, dtype=torch.float32, pin_memory=True)
-        ws = st.ws
+        del st, ws  # the host entry brings its own device buffer
+        dbuf = torch.empty(gdn.host_buffer_bytes(hc, Nqk, Nv, False), dtype=torch.uint8, device=dev)
+        plan = gdn.host_plan(hc)
         for _ in range(max(1, args.warmup // 2)):
             gdn.chunk_fwd_host(hq, hk, hv, hg, hb, hc, scale=host.scale, eps=host.eps, device=dev,
-                               out_host=oh, final_host=fh, workspace=ws)
+                               out_host=oh, final_host=fh, device_buffer=dbuf)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         gdist.barrier()
@@ -521,13 +557,18 @@ def main():
         h2d = d2h = 0
         for _ in range(args.steps):
             _, _, h2d, d2h = gdn.chunk_fwd_host(hq, hk, hv, hg, hb, hc, scale=host.scale, eps=host.eps, device=dev,
-                                                out_host=oh, final_host=fh, workspace=ws)
+                                                out_host=oh, final_host=fh, device_buffer=dbuf)
         e1.record(stream)
         torch.cuda.synchronize()
         ems = gdist.max_over_ranks(e0.elapsed_time(e1) / args.steps, device=dev)
         line["e2e"] = {"value": world * T / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                       "d2h_bytes_per_step": d2h, "ms_per_step": ems}
-        line["gpu_launches"] += 5 * args.steps
+                       "d2h_bytes_per_step": d2h, "ms_per_step": ems,
+                       "call": f"gdn_chunk_fwd_host from pinned host buffers, {len(plan)} pieces, uploads and "
+                               f"downloads overlapped with the compute",
+                       "h2d_GB/s": h2d / (ems / 1e3) / 1e9, "d2h_GB/s": d2h / (ems / 1e3) / 1e9}
+        # per piece: one chunk table, the pipelined kernels and the cu kernel
+        line["gpu_launches"] += args.steps * sum(2 + 3 * gdn.pipeline_ranges(r[4] - r[3], r[2], Nqk, Nv)
+                                                 for r in plan)
 
     # ---- CPU oracle baseline (rank 0, one GPU only)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -6,9 +6,9 @@ Importing the package does not load the library; the first call does, and
 raises if the library has not been built.
 """
 from ._binding import (CHUNK, HEAD_DIM, SHORT_MAX, Stages, chunk_fwd, chunk_fwd_host, chunk_fwd_noalloc,
-                       decode_status, lib, noalloc_status, pipeline_ranges, read_status, recurrent_fwd, short_fwd,
+                       decode_status, host_buffer_bytes, host_plan, lib, noalloc_status, pipeline_ranges, read_status, recurrent_fwd, recurrent_window_fwd, short_fwd,
                        status_string, workspace_bytes, workspace_layout)
 
-__all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_fwd_noalloc", "recurrent_fwd", "short_fwd", "pipeline_ranges",
+__all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_fwd_noalloc", "recurrent_fwd", "recurrent_window_fwd", "short_fwd", "pipeline_ranges",
            "Stages", "workspace_bytes", "workspace_layout", "lib", "status_string", "read_status", "noalloc_status",
-           "decode_status", "HEAD_DIM", "CHUNK", "SHORT_MAX"]
+           "decode_status", "host_buffer_bytes", "host_plan", "HEAD_DIM", "CHUNK", "SHORT_MAX"]

@@ -71,6 +71,13 @@ def lib():
         L.gdn_selftest_umma.argtypes = [p, p, p, i32, i32, i32, i32, i32, p, p]
         L.gdn_selftest_wait.restype = ctypes.c_int
         L.gdn_selftest_wait.argtypes = [i32, i32, p, sz, p]
+        L.gdn_chunk_fwd_host_bytes.restype = sz
+        L.gdn_chunk_fwd_host_bytes.argtypes = [p, i64, i32, i32, i32, i32, i32]
+        L.gdn_chunk_fwd_host.restype = ctypes.c_int
+        L.gdn_chunk_fwd_host.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, i32, p, sz,
+                                         p]
+        L.gdn_testing_host_plan.restype = ctypes.c_int
+        L.gdn_testing_host_plan.argtypes = [p, i64, i32, i32, p, i32]
         L.gdn_read_status.restype = ctypes.c_int
         L.gdn_read_status.argtypes = [p, p, p]
         L.gdn_noalloc_read_status.restype = ctypes.c_int
@@ -82,6 +89,10 @@ def lib():
         # B Nqk Nv Dk Dv P max_seqlen | stream
         L.gdn_recurrent_fwd.argtypes = [p, p, p, p, p, p, p, p, i32, i32, i32, p, p, f32, f32, p, i64, i32, i32, i32,
                                         i32, i32, i32, i32, p]
+        L.gdn_recurrent_window_fwd.restype = ctypes.c_int
+        # q k v g beta gk cu window | W act_dtype state_dtype rule | scale eps | out | T | B Nqk Nv Dk Dv | max_seqlen
+        L.gdn_recurrent_window_fwd.argtypes = [p, p, p, p, p, p, p, p, i32, i32, i32, i32, f32, f32, p, i64, i32, i32,
+                                               i32, i32, i32, i32, p]
         L.gdn_stage_chunk_map.restype = ctypes.c_int
         L.gdn_stage_chunk_map.argtypes = [p, i64, i32, i32, i32, p, sz, p]
         L.gdn_stage_intra.restype = ctypes.c_int
@@ -356,6 +367,55 @@ def recurrent_fwd(q, k, v, g, beta, cu_seqlens, state_pool, token_slots, num_acc
     return out
 
 
+def recurrent_window_fwd(q, k, v, g, beta, cu_seqlens, state_window, window, scale=None, eps=1e-6, gk=None,
+                         update_rule="gated_delta", max_seqlen: int = 0, out=None, stream=None):
+    """Token recurrence keeping the ``window`` most recent states (``gdn_recurrent_window_fwd``).
+
+    ``state_window`` [max(window, 1), B, Nv, Dk, Dv] holds the past window on entry (entry window - 1
+    the newest; zeros for an absent past) and the present window afterwards; every other argument
+    as for ``recurrent_fwd``.  Returns ``out``."""
+    if update_rule not in UPDATE_RULES:
+        raise ValueError(f"update_rule must be one of {sorted(UPDATE_RULES)}")
+    rule = UPDATE_RULES[update_rule]
+    decay, delta = rule in (0, 2), rule in (0, 1)
+    if not decay:
+        g = gk = None
+    if not delta:
+        beta = None
+    if state_window is None or state_window.dtype not in DTYPES or q.dtype not in DTYPES:
+        raise RuntimeError("state_window and q/k/v must be float32, bfloat16 or float16 tensors")
+    if q.dim() != 3 or v.dim() != 3:
+        raise ValueError("q/k must be [T, Nqk, Dk] and v [T, Nv, Dv]")
+    T, Nqk, Dk = q.shape
+    Nv, Dv = v.shape[1], v.shape[2]
+    B = cu_seqlens.shape[0] - 1
+    W = max(int(window), 1)
+    dev = q.device
+    adt = q.dtype
+    _need(q, "q", adt, (T, Nqk, Dk), dev)
+    _need(k, "k", adt, (T, Nqk, Dk), dev)
+    _need(v, "v", adt, (T, Nv, Dv), dev)
+    if g is not None:
+        _need(g, "g", torch.float32, (T, Nv), dev)
+    if beta is not None:
+        _need(beta, "beta", torch.bfloat16, (T, Nv), dev)
+    if gk is not None:
+        _need(gk, "gk", torch.float32, (T, Nv, Dk), dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), dev)
+    _need(state_window, "state_window", state_window.dtype, (W, B, Nv, Dk, Dv), dev)
+    if out is None:
+        out = torch.empty(T, Nv, Dv, dtype=adt, device=dev)
+    else:
+        _need(out, "out", adt, (T, Nv, Dv), dev)
+    sc = 0.0 if scale is None else float(scale)
+    rc = lib().gdn_recurrent_window_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(gk), _ptr(cu_seqlens),
+                                        _ptr(state_window), int(window), DTYPES[adt], DTYPES[state_window.dtype], rule,
+                                        sc, float(eps), _ptr(out), T, B, Nqk, Nv, Dk, Dv, int(max_seqlen),
+                                        _stream(stream))
+    _check(rc, "gdn_recurrent_window_fwd")
+    return out
+
+
 class Stages:
     """The four kernels of the chunked path as separate calls on one workspace.
 
@@ -449,20 +509,76 @@ class Stages:
         return out, final_state
 
 
+def _host_tensor(t, name, dtype, shape):
+    if not isinstance(t, torch.Tensor) or t.device.type != "cpu":
+        raise RuntimeError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}")
+
+
+def host_plan(cu_seqlens, segments=0):
+    """The cut of ``gdn_chunk_fwd_host`` into pieces (``gdn_testing_host_plan``): rows of (segment, first
+    sequence, sequences, first token, end token, initial-state source, final-state target)."""
+    cu = cu_seqlens.to(torch.int32).contiguous()
+    B = cu.shape[0] - 1
+    cap = 4 * (B + 64) + 8 * max(segments, 8)
+    rows = torch.zeros(cap, 7, dtype=torch.int32)
+    n = lib().gdn_testing_host_plan(_ptr(cu), int(cu[-1]), B, int(segments), _ptr(rows), cap)
+    if n < 0:
+        raise ValueError("invalid cu_seqlens for gdn_chunk_fwd_host")
+    return rows[:n].tolist()
+
+
+def host_buffer_bytes(cu_seqlens, Nqk, Nv, with_pool, segments=0) -> int:
+    cu = cu_seqlens.to(torch.int32).contiguous()
+    return int(lib().gdn_chunk_fwd_host_bytes(_ptr(cu), int(cu[-1]), cu.shape[0] - 1, Nqk, Nv, int(bool(with_pool)),
+                                              int(segments)))
+
+
 def chunk_fwd_host(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None, scale=None, eps=1e-6,
-                   max_seqlen: int = 0, device="cuda", out_host=None, final_host=None, workspace=None):
-    """End-to-end call from host tensors: copies the inputs to the device,
-    runs ``gdn_chunk_fwd`` and copies out and final_state back (into the given
-    pinned host buffers when provided).  Returns (out, final_state, h2d_bytes, d2h_bytes)."""
-    host = [q, k, v, g, beta, cu_seqlens, state_pool, state_indices]
-    dev = [None if t is None else t.to(device, non_blocking=True) for t in host]
-    h2d = sum(t.numel() * t.element_size() for t in host if t is not None)
-    o, f = chunk_fwd(*dev, scale=scale, eps=eps, max_seqlen=max_seqlen, workspace=workspace)
+                   device="cuda", out_host=None, final_host=None, device_buffer=None, segments=0, stream=None):
+    """End-to-end forward from host tensors through ``gdn_chunk_fwd_host``: the library streams the
+    batch through the GPU in pieces, its uploads and downloads overlapped with the compute, and writes
+    out and final_state into host tensors (pinned ones keep the copies asynchronous).  ``device_buffer``
+    (uint8 on ``device``, at least ``host_buffer_bytes`` long) is allocated here when not given.
+    Returns (out_host, final_host, h2d_bytes, d2h_bytes); the host tensors are complete once the
+    stream has reached the end of the call (the stream is synchronised here)."""
+    if q.dim() != 3 or v.dim() != 3:
+        raise ValueError("q/k must be [T, Nqk, 128] and v [T, Nv, 128]")
+    T, Nqk, _ = q.shape
+    Nv = v.shape[1]
+    Bn = cu_seqlens.shape[0] - 1
+    _host_tensor(q, "q", torch.bfloat16, (T, Nqk, HEAD_DIM))
+    _host_tensor(k, "k", torch.bfloat16, (T, Nqk, HEAD_DIM))
+    _host_tensor(v, "v", torch.bfloat16, (T, Nv, HEAD_DIM))
+    _host_tensor(g, "g", torch.float32, (T, Nv))
+    _host_tensor(beta, "beta", torch.bfloat16, (T, Nv))
+    _host_tensor(cu_seqlens, "cu_seqlens", torch.int32, (Bn + 1,))
+    P = 0
+    if state_pool is not None:
+        P = state_pool.shape[0]
+        _host_tensor(state_pool, "state_pool", torch.float32, (P, Nv, HEAD_DIM, HEAD_DIM))
+    if state_indices is not None:
+        _host_tensor(state_indices, "state_indices", torch.int32, (Bn,))
     if out_host is None:
-        out_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        out_host = torch.empty(T, Nv, HEAD_DIM, dtype=torch.bfloat16, pin_memory=True)
     if final_host is None:
-        final_host = torch.empty(f.shape, dtype=f.dtype, pin_memory=True)
-    out_host.copy_(o, non_blocking=True)
-    final_host.copy_(f, non_blocking=True)
-    d2h = o.numel() * o.element_size() + f.numel() * f.element_size()
+        final_host = torch.empty(Bn, Nv, HEAD_DIM, HEAD_DIM, dtype=torch.float32, pin_memory=True)
+    _host_tensor(out_host, "out_host", torch.bfloat16, (T, Nv, HEAD_DIM))
+    _host_tensor(final_host, "final_host", torch.float32, (Bn, Nv, HEAD_DIM, HEAD_DIM))
+    need = host_buffer_bytes(cu_seqlens, Nqk, Nv, state_pool is not None, segments)
+    if device_buffer is None or device_buffer.numel() < need:
+        device_buffer = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+    st = torch.cuda.current_stream(device_buffer.device) if stream is None else stream
+    sc = 0.0 if scale is None else float(scale)
+    rc = lib().gdn_chunk_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+                                  _ptr(state_pool), _ptr(state_indices), sc, float(eps), _ptr(out_host),
+                                  _ptr(final_host), T, Bn, Nqk, Nv, P, int(segments), _ptr(device_buffer),
+                                  device_buffer.numel(), _stream(st))
+    _check(rc, "gdn_chunk_fwd_host")
+    st.synchronize()
+    sbytes = Nv * HEAD_DIM * HEAD_DIM * 4
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v, g, beta, cu_seqlens)) + \
+        (Bn * sbytes if state_pool is not None else 0)
+    d2h = out_host.numel() * out_host.element_size() + final_host.numel() * final_host.element_size()
     return out_host, final_host, h2d, d2h

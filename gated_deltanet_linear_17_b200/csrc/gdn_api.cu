@@ -8,6 +8,7 @@
 // runs beside the other two kernels of neighbouring ranges.  The side streams
 // fork from and join back into the caller's stream within the call.
 #include <math.h>
+#include <algorithm>
 #include <string.h>
 
 #include <mutex>
@@ -301,11 +302,17 @@ int gdn_short_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
                                          (cudaStream_t)stream));
 }
 
-int gdn_recurrent_fwd(const void *q, const void *k, const void *v, const float *g, const uint16_t *beta,
-                      const float *gk, const int32_t *cu_seqlens, void *state_pool, int32_t act_dtype,
-                      int32_t state_dtype, int32_t update_rule, const int32_t *token_slots,
-                      const int32_t *num_accepted, float scale, float eps, void *out, int64_t T, int32_t B,
-                      int32_t Nqk, int32_t Nv, int32_t Dk, int32_t Dv, int32_t P, int32_t max_seqlen, void *stream)
+}  // extern "C"
+
+namespace {
+
+// Checks and launch shared by gdn_recurrent_fwd (win = 0: a pool of P slots, one slot per token) and
+// gdn_recurrent_window_fwd (win >= 1: a window buffer of win * B slots, P = win * B, no token slots).
+int recurrent_call(const void *q, const void *k, const void *v, const float *g, const uint16_t *beta,
+                   const float *gk, const int32_t *cu_seqlens, void *state_pool, int32_t act_dtype,
+                   int32_t state_dtype, int32_t update_rule, const int32_t *token_slots, const int32_t *num_accepted,
+                   float scale, float eps, void *out, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t Dk,
+                   int32_t Dv, int64_t P, int32_t max_seqlen, void *stream, int win)
 {
     int rc = check_sizes(T, B, Nqk, Nv);
     if (rc) return rc;
@@ -319,13 +326,15 @@ int gdn_recurrent_fwd(const void *q, const void *k, const void *v, const float *
     const bool pool16 = state_dtype != GDN_DTYPE_FP32;
     if (!types_ok || (Dk != 64 && Dk != 128) || Dv % 32 != 0 || Dv > 1024 || (pool16 && Dv % 64 != 0))
         return GDN_ERR_UNSUPPORTED;
+    if (win > 0 && (int64_t)win * B >= (int64_t(1) << 31) / 256) return GDN_ERR_UNSUPPORTED;
     if (B == 0) return GDN_OK;
     const bool decay = update_rule == GDN_RULE_GATED_DELTA || update_rule == GDN_RULE_GATED;
     const bool delta = update_rule == GDN_RULE_GATED_DELTA || update_rule == GDN_RULE_DELTA;
     if (!decay) g = nullptr, gk = nullptr;  // not read by this rule
     if (!delta) beta = nullptr;
+    if (win > 0) token_slots = nullptr, num_accepted = nullptr;  // the window decides the slots
     if (!cu_seqlens || !state_pool) return GDN_ERR_NULL_ARG;
-    if (T > 0 && (!q || !k || !v || !out || !token_slots || (decay && !g) || (delta && !beta)))
+    if (T > 0 && (!q || !k || !v || !out || (win == 0 && !token_slots) || (decay && !g) || (delta && !beta)))
         return GDN_ERR_NULL_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(state_pool) ||
         !aligned16(gk))
@@ -344,7 +353,34 @@ int gdn_recurrent_fwd(const void *q, const void *k, const void *v, const float *
     const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)Dk);
     return cuda_status(gdn::launch_recurrent(q, k, v, g, beta, gk, cu_seqlens, state_pool, act_dtype, state_dtype,
                                              update_rule, token_slots, num_accepted, sc, eps, out, (int)T, B, Nqk, Nv,
-                                             Dk, Dv, max_seqlen, (cudaStream_t)stream));
+                                             Dk, Dv, max_seqlen, (cudaStream_t)stream, win));
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn_recurrent_fwd(const void *q, const void *k, const void *v, const float *g, const uint16_t *beta,
+                      const float *gk, const int32_t *cu_seqlens, void *state_pool, int32_t act_dtype,
+                      int32_t state_dtype, int32_t update_rule, const int32_t *token_slots,
+                      const int32_t *num_accepted, float scale, float eps, void *out, int64_t T, int32_t B,
+                      int32_t Nqk, int32_t Nv, int32_t Dk, int32_t Dv, int32_t P, int32_t max_seqlen, void *stream)
+{
+    return recurrent_call(q, k, v, g, beta, gk, cu_seqlens, state_pool, act_dtype, state_dtype, update_rule,
+                          token_slots, num_accepted, scale, eps, out, T, B, Nqk, Nv, Dk, Dv, P, max_seqlen, stream, 0);
+}
+
+int gdn_recurrent_window_fwd(const void *q, const void *k, const void *v, const float *g, const uint16_t *beta,
+                             const float *gk, const int32_t *cu_seqlens, void *state_window, int32_t window,
+                             int32_t act_dtype, int32_t state_dtype, int32_t update_rule, float scale, float eps,
+                             void *out, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t Dk, int32_t Dv,
+                             int32_t max_seqlen, void *stream)
+{
+    if (window < 0 || window > GDN_MAX_STATE_WINDOW) return GDN_ERR_BAD_SHAPE;
+    const int W = window > 0 ? window : 1;  // no window axis: the current state alone, one entry
+    return recurrent_call(q, k, v, g, beta, gk, cu_seqlens, state_window, act_dtype, state_dtype, update_rule,
+                          nullptr, nullptr, scale, eps, out, T, B, Nqk, Nv, Dk, Dv, std::max<int64_t>((int64_t)W * B, 1),
+                          max_seqlen, stream, W);
 }
 
 int gdn_chunk_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,

@@ -67,6 +67,9 @@ constexpr int kRuleGatedDelta = 0, kRuleDelta = 1, kRuleGated = 2, kRuleLinear =
 cudaError_t launch_recurrent(const void *q, const void *k, const void *v, const float *g, const uint16_t *beta,
                              const float *gk, const int32_t *cu, void *pool, int act_dtype, int state_dtype, int rule,
                              const int32_t *token_slots, const int32_t *num_accepted, float scale, float eps, void *out,
-                             int T, int B, int Nqk, int Nv, int Dk, int Dv, int max_seqlen, cudaStream_t st);
+                             int T, int B, int Nqk, int Nv, int Dk, int Dv, int max_seqlen, cudaStream_t st,
+                             int win = 0);
+// win > 0: the pool is a state window [win, B, Nv, Dk, Dv] updated in place (token_slots and
+// num_accepted unused); see gdn_recurrent_window_fwd in gdn.h.
 
 }  // namespace gdn

@@ -36,7 +36,13 @@
 // when written) and the key-dimension gate gk (GK: S = S e^g e^gk, row i of S
 // decayed by e^{g + gk_i}; the 128 factors of each staged token are computed once
 // per CTA into shared memory, and the state rows are decayed before the sum
-// S^T kh).  DECAY and DELTA select the update rule of the page
+// S^T kh).  With a state window (`win` = W > 0, the LinearAttention page's
+// state_window) the pool is the window buffer [W, B, ...] seen as W B slots,
+// slot w B + b holding entry w of sequence b: the sequence starts from entry
+// W - 1 and the state after token j of its n goes to entry W - n + j when that
+// is >= 0 (earlier tokens' states leave the window and are not written); the
+// entries that a sequence shorter than the window keeps were moved down by
+// window_shift_kernel before this kernel runs.  DECAY and DELTA select the update rule of the page
 // "com.microsoft.LinearAttention" (update_rule): gated_delta (both), delta (no
 // decay: g and gk unused), gated (S = e^g S + kh v^T: no retrieval, beta unused)
 // and linear (S = S + kh v^T); without the retrieval a token needs one barrier.
@@ -124,7 +130,8 @@ __device__ __forceinline__ void short_body(
     const float *__restrict__ g, const uint16_t *__restrict__ beta, const float *__restrict__ gk,
     const int32_t *__restrict__ cu, const void *pool, const int32_t *__restrict__ idx,
     const int32_t *__restrict__ token_slots, const int32_t *__restrict__ num_accepted, void *pool_w, float scale,
-    float eps, void *__restrict__ out, float *__restrict__ final_state, int T, int Nqk, int Nv, int Dv)
+    float eps, void *__restrict__ out, float *__restrict__ final_state, int T, int Nqk, int Nv, int Dv, int win,
+    int Bw)
 {
     constexpr bool SBF = SDT != kF32;          // a 16-bit pool
     constexpr int AES = ADT == kF32 ? 4 : 2;   // activation element bytes
@@ -157,7 +164,12 @@ __device__ __forceinline__ void short_body(
         cp_async16(smem_addr(&sm.v[t][c * 8]), static_cast<const char *>(v) + off, true);
     }
     if (DECAY && tid < npre) cp_async4(smem_addr(&sm.g[tid]), g + (size_t)(t0 + tid) * Nv + h);
-    if (SLOTS && tid <= PRE && tid < n) cp_async4(smem_addr(&sm.slot[tid]), token_slots + t0 + tid);
+    // the window slot of token j (-1: its state leaves the window and is not written)
+    auto win_slot = [&](int j) { return j >= n - win ? (win - n + j) * Bw + b : -1; };
+    if (SLOTS && tid <= PRE && tid < n) {
+        if (win > 0) sm.slot[tid] = win_slot(tid);
+        else cp_async4(smem_addr(&sm.slot[tid]), token_slots + t0 + tid);
+    }
     if (GK) {
         for (int e = tid; e < npre * (DK / 4); e += DK) {
             const int t = e / (DK / 4), c = e % (DK / 4);
@@ -167,7 +179,9 @@ __device__ __forceinline__ void short_body(
     // the starting slot
     int slot0 = 0;
     if (pool) {
-        if (SLOTS) {  // the state after the last accepted token (n >= 1 here)
+        if (SLOTS && win > 0) {  // the window's newest entry
+            slot0 = (win - 1) * Bw + b;
+        } else if (SLOTS) {  // the state after the last accepted token (n >= 1 here)
             const int a = min(max(num_accepted ? num_accepted[b] : n, 1), n);
             slot0 = token_slots[t0 + a - 1];
         } else {
@@ -325,7 +339,7 @@ __device__ __forceinline__ void short_body(
             b1 = ffma2(s2[2 * c + 1], make_float2(qx.z, qx.w), b1);
         }
         sm.red2[p][wid][lane] = (b0.x + b0.y) + (b1.x + b1.y);
-        if (SLOTS && (j == n - 1 || sm.slot[j + 1] != sm.slot[j])) write_slot(sm.slot[j]);
+        if (SLOTS && sm.slot[j] >= 0 && (j == n - 1 || sm.slot[j + 1] != sm.slot[j])) write_slot(sm.slot[j]);
         __syncthreads();
         if (wid == 0)
             st_act<ADT>(out, ((size_t)(t0 + j) * Nv + h) * Dv + col, sum_warps<NW>(sm.red2[p], lane));
@@ -380,8 +394,9 @@ __device__ __forceinline__ void short_body(
         }
         sm.red2[p][wid][lane] = acc2;
         if (SLOTS) {
-            const int sj = token_slots[t], sn = j + 1 < n ? token_slots[t + 1] : -1;
-            if (j == n - 1 || sn != sj) write_slot(sj);
+            const int sj = win > 0 ? win_slot(j) : token_slots[t];
+            const int sn = j + 1 < n ? (win > 0 ? win_slot(j + 1) : token_slots[t + 1]) : -1;
+            if (sj >= 0 && (j == n - 1 || sn != sj)) write_slot(sj);
         }
         __syncthreads();
         if (wid == 0)
@@ -405,9 +420,10 @@ __device__ __forceinline__ void short_body(
         const int32_t *__restrict__ cu, const void *pool, const int32_t *__restrict__ idx,                       \
         const int32_t *__restrict__ token_slots, const int32_t *__restrict__ num_accepted, void *pool_w,         \
         float scale, float eps, void *__restrict__ out, float *__restrict__ final_state, int T, int Nqk, int Nv, \
-        int Dv
-#define GDN_SHORT_ARGS \
-    q, k, v, g, beta, gk, cu, pool, idx, token_slots, num_accepted, pool_w, scale, eps, out, final_state, T, Nqk, Nv, Dv
+        int Dv, int win, int Bw
+#define GDN_SHORT_ARGS                                                                                              \
+    q, k, v, g, beta, gk, cu, pool, idx, token_slots, num_accepted, pool_w, scale, eps, out, final_state, T, Nqk, Nv, \
+        Dv, win, Bw
 
 // Two entry kernels around one body, each with its own register budget.  The pool
 // pass of the chunked forward (bf16 activations, fp32 state, one slot per sequence)
@@ -432,16 +448,17 @@ template <int PRE, bool SLOTS, bool GK, int SDT, bool DECAY, bool DELTA, int DK,
 static void launch_variant(dim3 grid, cudaStream_t st, const void *q, const void *k, const void *v, const float *g,
                            const uint16_t *beta, const float *gk, const int32_t *cu, const void *pool,
                            const int32_t *idx, const int32_t *token_slots, const int32_t *num_accepted, void *pool_w,
-                           float scale, float eps, void *out, float *final_state, int T, int Nqk, int Nv, int Dv)
+                           float scale, float eps, void *out, float *final_state, int T, int Nqk, int Nv, int Dv,
+                           int win = 0, int Bw = 0)
 {
     if constexpr (SLOTS)
         short_kernel_slots<PRE, GK, SDT, DECAY, DELTA, DK, ADT><<<grid, DK, 0, st>>>(
             q, k, v, g, beta, gk, cu, pool, idx, token_slots, num_accepted, pool_w, scale, eps, out, final_state, T,
-            Nqk, Nv, Dv);
+            Nqk, Nv, Dv, win, Bw);
     else
         short_kernel<PRE, DECAY, DELTA><<<grid, DK, 0, st>>>(q, k, v, g, beta, gk, cu, pool, idx, token_slots,
                                                                num_accepted, pool_w, scale, eps, out, final_state, T,
-                                                               Nqk, Nv, Dv);
+                                                               Nqk, Nv, Dv, 0, 0);
 }
 
 // Arguments of one pool-updating launch
@@ -456,6 +473,7 @@ struct RecArgs {
     float scale, eps;
     void *out;
     int T, Nqk, Nv, Dv;
+    int win, Bw;  // state window (0: none) and the number of sequences
 };
 
 template <int PRE, bool GK, int SDT, bool DECAY, bool DELTA, int DK, int ADT>
@@ -464,7 +482,8 @@ static void launch_pool(const RecArgs &a, dim3 grid, cudaStream_t st)
     grid.z = a.Dv / (SDT != kF32 ? 64 : 32);  // Dv columns per CTA
     launch_variant<PRE, true, GK, SDT, DECAY, DELTA, DK, ADT>(grid, st, a.q, a.k, a.v, a.g, a.beta, a.gk, a.cu, a.pool,
                                                               nullptr, a.token_slots, a.num_accepted, a.pool, a.scale,
-                                                              a.eps, a.out, nullptr, a.T, a.Nqk, a.Nv, a.Dv);
+                                                              a.eps, a.out, nullptr, a.T, a.Nqk, a.Nv, a.Dv, a.win,
+                                                              a.Bw);
 }
 
 // one activation type and pool type; a key gate only with a decaying rule.  A 16-bit pool stages 8
@@ -534,15 +553,37 @@ cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v
     return cudaGetLastError();
 }
 
+// The window entries that a sequence of 1 <= n < W tokens keeps, moved n places towards entry 0 before
+// the recurrence writes entries W - n .. W - 1: entry w <- entry w + n for w = 0 .. W - n - 1, in that
+// order (each source is read before it is overwritten, and entry W - 1, the start of the recurrence, is
+// not written here).  Grid (B, Nv, 16-byte pieces of a state / 256): each thread moves one 16-byte piece
+// of the state through the entries.
+__global__ void __launch_bounds__(256) window_shift_kernel(const int32_t *__restrict__ cu, uint4 *pool, int T, int B,
+                                                           int Nv, int win, int pieces)
+{
+    const int b = blockIdx.x, h = blockIdx.y, i = blockIdx.z * 256 + threadIdx.x;
+    const int t0 = min(max(cu[b], 0), T), n = min(max(cu[b + 1], t0), T) - t0;
+    if (n < 1 || n >= win || i >= pieces) return;
+    for (int w = 0; w + n < win; ++w)
+        pool[(((size_t)w * B + b) * Nv + h) * pieces + i] = pool[(((size_t)(w + n) * B + b) * Nv + h) * pieces + i];
+}
+
 cudaError_t launch_recurrent(const void *q, const void *k, const void *v, const float *g, const uint16_t *beta,
                              const float *gk, const int32_t *cu, void *pool, int act_dtype, int state_dtype, int rule,
                              const int32_t *token_slots, const int32_t *num_accepted, float scale, float eps, void *out,
-                             int T, int B, int Nqk, int Nv, int Dk, int Dv, int max_seqlen, cudaStream_t st)
+                             int T, int B, int Nqk, int Nv, int Dk, int Dv, int max_seqlen, cudaStream_t st, int win)
 {
     if (B == 0) return cudaSuccess;
     if ((Dk != 64 && Dk != 128) || Dv <= 0 || Dv % kTile != 0) return cudaErrorInvalidValue;
     if (act_dtype != kBF16 && Dk != 128) return cudaErrorInvalidValue;
-    const RecArgs a{q, k, v, g, beta, gk, cu, pool, token_slots, num_accepted, scale, eps, out, T, Nqk, Nv, Dv};
+    if (win > 1) {
+        const int pieces = Dk * Dv * (state_dtype == kF32 ? 4 : 2) / 16;
+        window_shift_kernel<<<dim3(B, Nv, (pieces + 255) / 256), 256, 0, st>>>(cu, static_cast<uint4 *>(pool), T, B,
+                                                                                Nv, win, pieces);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    const RecArgs a{q, k, v, g, beta, gk, cu, pool, token_slots, num_accepted, scale, eps, out, T, Nqk, Nv, Dv, win, B};
     const dim3 grid(B, Nv, Dv / kTile);
     const bool few = max_seqlen >= 1 && max_seqlen <= 8;
     if (Dk == 64) {

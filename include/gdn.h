@@ -93,6 +93,7 @@ extern "C" {
 #define GDN_CHUNK 128    /* L */
 #define GDN_SHORT_MAX 16 /* max_seqlen at or below which the fused short-sequence kernel runs */
 #define GDN_NOALLOC_SCRATCH_BYTES (64u << 20) /* static workspace of gdn_chunk_fwd_noalloc, per GPU */
+#define GDN_MAX_STATE_WINDOW 8 /* largest state_window of gdn_recurrent_window_fwd */
 
 /* element types of gdn_recurrent_fwd's activations and state pool */
 #define GDN_DTYPE_FP32 0
@@ -279,6 +280,50 @@ int gdn_chunk_fwd_noalloc(const uint16_t *q, const uint16_t *k, const uint16_t *
 int gdn_noalloc_read_status(int32_t *status_out, void *stream);
 
 /*
+ * gdn_chunk_fwd_host -- gdn_chunk_fwd from host buffers, with the host <-> device
+ * copies overlapped with the compute.
+ *
+ * The prefill page's operator reuses the state across sequence chunks for
+ * streaming inference; this call uses that to stream a batch through the GPU.
+ * It cuts the tokens into `segments` pieces at 128-token chunk starts of the
+ * sequences (a cut never splits a chunk) and, for each piece, uploads its
+ * tokens on a copy stream of the library, runs gdn_chunk_fwd on `stream` once
+ * they have landed, and downloads its output rows (and the final states of the
+ * sequences that end in it) on a second copy stream, so that piece s+1 uploads
+ * while s computes and s-1 downloads.  A sequence cut between two pieces
+ * resumes from its fp32 state, exactly as a state crosses a chunk range inside
+ * one call: out and final_state equal those of one gdn_chunk_fwd call bit for
+ * bit.
+ *
+ *   q, k, v, g, beta   host, layouts as for gdn_chunk_fwd.  Pinned (page-locked)
+ *                 memory lets the copies run asynchronously; pageable memory
+ *                 works but each copy then waits for the host.
+ *   cu_seqlens    host int32 [B+1]: cu[0] = 0, non-decreasing, cu[B] = T
+ *                 (checked on the host: GDN_ERR_BAD_SHAPE otherwise)
+ *   state_pool    host fp32 [P, Nv, 128, 128] or NULL; only the B slots named by
+ *                 state_indices (host int32 [B], each in [0, P), checked; NULL
+ *                 for slot b) are uploaded
+ *   out           host bf16 [T, Nv, 128]; final_state host fp32 [B, Nv, 128, 128]
+ *                 or NULL.  Both are complete once `stream` has reached the
+ *                 point after this call.
+ *   segments      number of pieces (> 0), or 0 for 8 from 32768 tokens on, 4
+ *                 from 4096 on, else 1
+ *   device_buffer device memory of device_bytes >= gdn_chunk_fwd_host_bytes(...)
+ *                 with the same cu_seqlens and segments, 256-byte aligned: it
+ *                 holds the device copies, the per-piece workspace and the
+ *                 carried states (GDN_ERR_WORKSPACE when too small)
+ * Same limits as gdn_chunk_fwd.  Asynchronous on `stream` (and on the library's
+ * two copy streams, which fork from and join back into `stream` within the call).
+ */
+size_t gdn_chunk_fwd_host_bytes(const int32_t *cu_seqlens, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
+                                int32_t with_pool, int32_t segments);
+int gdn_chunk_fwd_host(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
+                       const uint16_t *beta, const int32_t *cu_seqlens, const float *state_pool,
+                       const int32_t *state_indices, float scale, float eps, uint16_t *out,
+                       float *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
+                       int32_t segments, void *device_buffer, size_t device_bytes, void *stream);
+
+/*
  * gdn_recurrent_fwd -- token recurrence on a state pool updated in place, with
  * one slot index per token (decode and speculative decoding).
  *
@@ -354,6 +399,48 @@ int gdn_recurrent_fwd(const void *q, const void *k, const void *v, const float *
                       const int32_t *num_accepted, float scale, float eps, void *out, int64_t T, int32_t B,
                       int32_t Nqk, int32_t Nv, int32_t Dk, int32_t Dv, int32_t P, int32_t max_seqlen,
                       void *stream);
+
+/*
+ * gdn_recurrent_window_fwd -- the token recurrence of gdn_recurrent_fwd keeping
+ * a window of the most recent states, updated in place.
+ *
+ * Page "com.microsoft.LinearAttention": attribute state_window (0 to 8) is the
+ * number of recent recurrent states kept in present_state, and with a window
+ * past_state and present_state carry a leading window axis, shape (W, B, H_kv,
+ * d_k, d_v), so that a caller can roll back (for example to undo rejected
+ * speculative tokens).  The page gives neither the order of the window nor
+ * where a step starts; this call takes a first-in-first-out window in time
+ * order:
+ *   - entry W - 1 is the newest state, and sequence b continues from
+ *     state_window[W - 1, b];
+ *   - after each token the new state is appended and the oldest entry leaves,
+ *     so after n tokens the window holds the last W of [past entries 0 ..
+ *     W - 1, S_1, .., S_n]: with n >= W the states after tokens n - W + 1 ..
+ *     n, with n < W the W - n newest past entries moved n places towards
+ *     entry 0 followed by S_1 .. S_n; a sequence with no tokens keeps its
+ *     window;
+ *   - rolling back r tokens of the step is reading entry W - 1 - r.
+ * An absent past_state is a window of zero states (the page's default): the
+ * caller zero-fills the buffer before the first step.  window = 0 (the page's
+ * value for no window axis) keeps only the current state: the buffer is then
+ * [B, Nv, Dk, Dv], the same as a window of 1.
+ *
+ *   state_window  device [max(window, 1), B, Nv, Dk, Dv] of state_dtype, read as
+ *                 past_state and overwritten as present_state (required)
+ *   window        0 .. GDN_MAX_STATE_WINDOW
+ *   every other argument as for gdn_recurrent_fwd (no token slots, no accepted
+ *   counts: the window decides where each state goes)
+ * Cost: besides the recurrence, a sequence of 1 <= n < W tokens moves W - n of
+ * its states inside the buffer before the tokens are applied (a kernel ahead
+ * of the recurrence on `stream`); the page's layout puts the newest entry
+ * last, which makes that move part of every short step.  Errors as for
+ * gdn_recurrent_fwd; a window outside 0 .. 8 is GDN_ERR_BAD_SHAPE.
+ */
+int gdn_recurrent_window_fwd(const void *q, const void *k, const void *v, const float *g, const uint16_t *beta,
+                             const float *gk, const int32_t *cu_seqlens, void *state_window, int32_t window,
+                             int32_t act_dtype, int32_t state_dtype, int32_t update_rule, float scale, float eps,
+                             void *out, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t Dk, int32_t Dv,
+                             int32_t max_seqlen, void *stream);
 
 #ifdef __cplusplus
 }

@@ -44,6 +44,19 @@ int gdn_selftest_umma(const uint16_t *A, const uint16_t *B, float *C, int32_t N,
  */
 int gdn_selftest_wait(int32_t max_polls, int32_t arrive, void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * gdn_testing_host_plan: the cut of gdn_chunk_fwd_host into pieces and calls,
+ * on the host only (no CUDA call).  For host int32 cu_seqlens [B+1] and
+ * `segments` (as for gdn_chunk_fwd_host) it writes up to max_calls rows of 7
+ * int32 into calls: segment, first sequence, number of sequences, first token,
+ * end token, initial-state source (1 the sequence's own initial state, 2 the
+ * state carried from the previous piece), final-state target (0 the final
+ * row, 1 carried to the next piece).  Returns the number of calls, or -1 for
+ * invalid arguments or too small a max_calls.
+ */
+int gdn_testing_host_plan(const int32_t *cu_seqlens, int64_t T, int32_t B, int32_t segments, int32_t *calls,
+                          int32_t max_calls);
+
 #ifdef __cplusplus
 }
 #endif

@@ -223,3 +223,28 @@ def test_status_bits_match_the_header():
     assert gdn.decode_status([0, 5, 0, 0]) == []
     assert gdn.decode_status([2, 5, 4, 2]) == ["cu_seqlens decreasing", "a wait of the intra-chunk kernel gave up",
                                                "the state beyond the fp16 range"]
+
+
+def test_window_entry_argument_errors(lib):
+    M = 1 << 20  # fake, disjoint, aligned addresses; every call below returns before any launch
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+
+    def call(**over):
+        a = dict(q=M, k=2 * M, v=3 * M, g=4 * M, beta=5 * M, gk=None, cu=6 * M, win=9 * M, W=4, act=1, sdt=0,
+                 rule=0, out=7 * M, T=8, B=1, Nqk=2, Nv=4, Dk=128, Dv=128)
+        a.update(over)
+        return lib.gdn_recurrent_window_fwd(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["g"]), vp(a["beta"]),
+                                            vp(a["gk"]), vp(a["cu"]), vp(a["win"]), a["W"], a["act"], a["sdt"],
+                                            a["rule"], 0.0, 1e-6, vp(a["out"]), a["T"], a["B"], a["Nqk"], a["Nv"],
+                                            a["Dk"], a["Dv"], 0, None)
+    assert call(W=9) == B.GDN_ERR_BAD_SHAPE and call(W=-1) == B.GDN_ERR_BAD_SHAPE
+    assert call(win=None) == B.GDN_ERR_NULL_ARG
+    assert call(Nv=3) == B.GDN_ERR_BAD_SHAPE
+    assert call(act=2, sdt=1) == B.GDN_ERR_UNSUPPORTED
+    assert call(win=9 * M + 8) == B.GDN_ERR_ALIGNMENT
+    entry = 1 * 4 * 128 * 128 * 4  # bytes of one window entry at B = 1, Nv = 4, fp32
+    assert call(out=9 * M) == B.GDN_ERR_OVERLAP                    # out inside the window buffer
+    assert call(out=9 * M + 3 * entry) == B.GDN_ERR_OVERLAP        # inside entry 3 of a 4-entry window
+    assert call(out=9 * M + 3 * entry, W=3, g=None) == B.GDN_ERR_NULL_ARG  # past a 3-entry window: later checks
+    assert call(B=0) == B.GDN_OK and call(T=0) == B.GDN_OK
+    assert call(W=0, g=None) == B.GDN_ERR_NULL_ARG                  # the gated delta rule reads g
