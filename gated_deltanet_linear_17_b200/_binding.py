@@ -29,7 +29,8 @@ DEV_BITS = {0: {1: "cu[0] != 0", 2: "cu_seqlens decreasing", 4: "cu[B] != T"},
             2: {1: "a wait of the state pass gave up", 2: "a wait of the output kernel gave up",
                 4: "a wait of the intra-chunk kernel gave up", 8: "the self-test wait gave up"},
             3: {1: "U (or beta v) beyond the fp16 range", 2: "the state beyond the fp16 range",
-                4: "the output kernel's fp16 operand beyond the fp16 range"}}
+                4: "the output kernel's fp16 operand beyond the fp16 range",
+                8: "an fp32 activation beyond the fp16 range"}}
 # update rules of gdn_chunk_fwd_rule and gdn_recurrent_fwd (GDN_RULE_* in gdn.h)
 UPDATE_RULES = {"gated_delta": 0, "delta": 1, "gated": 2, "linear": 3}
 # element types of gdn_recurrent_fwd (GDN_DTYPE_* in gdn.h)
@@ -41,7 +42,7 @@ _lib = None
 class _Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("total", "status", "chunk_info", "seq_chunk0", "rq", "rk", "gcum", "betaf", "U", "W", "Mk", "Sc", "fa",
-                 "carry")] + \
+                 "carry", "act16")] + \
                [("max_chunks", ctypes.c_int64)]
 
 
@@ -65,6 +66,13 @@ def lib():
         L.gdn_chunk_fwd_rule.restype = ctypes.c_int
         L.gdn_chunk_fwd_rule.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, i32, i32, p,
                                          sz, p]
+        L.gdn_chunk_fwd_typed_workspace_bytes.restype = sz
+        L.gdn_chunk_fwd_typed_workspace_bytes.argtypes = [i64, i32, i32, i32, i32]
+        L.gdn_chunk_fwd_typed.restype = ctypes.c_int
+        # q k v g beta cu pool idx | scale eps | out final | T B Nqk Nv P | rule act_dtype state_dtype max_seqlen |
+        # workspace bytes stream
+        L.gdn_chunk_fwd_typed.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, i32, i32,
+                                          i32, i32, p, sz, p]
         L.gdn_chunk_fwd_noalloc.restype = ctypes.c_int
         L.gdn_chunk_fwd_noalloc.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, i32, p]
         L.gdn_selftest_umma.restype = ctypes.c_int
@@ -153,7 +161,7 @@ def workspace_layout(T: int, B: int, Nqk: int, Nv: int) -> dict:
     return {n: getattr(lay, n) for n, _ in _Layout._fields_}
 
 
-def _resolve(q, k, v, g, beta, cu_seqlens, state_pool, state_indices):
+def _resolve(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, act=torch.bfloat16, state=torch.float32):
     if q.dim() != 3 or v.dim() != 3:
         raise ValueError("q/k must be [T, Nqk, 128] and v [T, Nv, 128]")
     T, Nqk, Dk = q.shape
@@ -164,16 +172,16 @@ def _resolve(q, k, v, g, beta, cu_seqlens, state_pool, state_indices):
         raise ValueError(f"Nv ({Nv}) must be a multiple of Nqk ({Nqk})")
     B = cu_seqlens.shape[0] - 1
     dev = q.device
-    _need(q, "q", torch.bfloat16, (T, Nqk, HEAD_DIM), dev)
-    _need(k, "k", torch.bfloat16, (T, Nqk, HEAD_DIM), dev)
-    _need(v, "v", torch.bfloat16, (T, Nv, HEAD_DIM), dev)
+    _need(q, "q", act, (T, Nqk, HEAD_DIM), dev)
+    _need(k, "k", act, (T, Nqk, HEAD_DIM), dev)
+    _need(v, "v", act, (T, Nv, HEAD_DIM), dev)
     _need(g, "g", torch.float32, (T, Nv), dev)
     _need(beta, "beta", torch.bfloat16, (T, Nv), dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), dev)
     P = 0
     if state_pool is not None:
         P = state_pool.shape[0]
-        _need(state_pool, "state_pool", torch.float32, (P, Nv, HEAD_DIM, HEAD_DIM), dev)
+        _need(state_pool, "state_pool", state, (P, Nv, HEAD_DIM, HEAD_DIM), dev)
     if state_indices is not None:
         _need(state_indices, "state_indices", torch.int32, (B,), dev)
     return T, B, Nqk, Nv, P, dev
@@ -181,7 +189,7 @@ def _resolve(q, k, v, g, beta, cu_seqlens, state_pool, state_indices):
 
 def chunk_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None, scale=None, eps=1e-6,
               max_seqlen: int = 0, out=None, final_state=None, output_final_state=True, workspace=None,
-              stream=None, update_rule="gated_delta", check_status=False):
+              stream=None, update_rule="gated_delta", check_status=False, state_dtype=None):
     """Gated Delta Rule forward through ``gdn_chunk_fwd`` (``gdn_chunk_fwd_rule`` for another
     ``update_rule``: delta, gated or linear); returns (out, final_state).
 
@@ -192,7 +200,13 @@ def chunk_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None,
     delta and linear rules, beta not by the gated and linear rules (pass None).
     ``check_status`` waits for the call and raises RuntimeError when the device
     status words of the chunked path report a malformed cu_seqlens, a wait that
-    gave up or a value beyond the fp16 range (see ``read_status``)."""
+    gave up or a value beyond the fp16 range (see ``read_status``).
+
+    Element types (the LinearAttention page: activations and state each fp16 or
+    fp32): q, k, v and out share one type, bf16, fp16 or fp32; the state pool and
+    final_state share another, fp32, fp16 or bf16 (``state_dtype`` sets it when
+    there is no pool; fp32 by default).  Anything but bf16 activations with an
+    fp32 state goes through ``gdn_chunk_fwd_typed``."""
     if update_rule not in UPDATE_RULES:
         raise ValueError(f"update_rule must be one of {sorted(UPDATE_RULES)}")
     rule = UPDATE_RULES[update_rule]
@@ -202,23 +216,35 @@ def chunk_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None,
         beta = None
     if q.dim() != 3 or v.dim() != 3:
         raise ValueError("q/k must be [T, Nqk, 128] and v [T, Nv, 128]")
+    act = q.dtype
+    state = state_pool.dtype if state_pool is not None else (state_dtype or torch.float32)
+    if act not in DTYPES or state not in DTYPES:
+        raise RuntimeError(f"activations and states must be bfloat16, float16 or float32 (got {act}, {state})")
     gg = g if g is not None else torch.empty(q.shape[0], v.shape[1], dtype=torch.float32, device=q.device)
     bb = beta if beta is not None else torch.empty(q.shape[0], v.shape[1], dtype=torch.bfloat16, device=q.device)
-    T, B, Nqk, Nv, P, dev = _resolve(q, k, v, gg, bb, cu_seqlens, state_pool, state_indices)
+    T, B, Nqk, Nv, P, dev = _resolve(q, k, v, gg, bb, cu_seqlens, state_pool, state_indices, act, state)
     if out is None:
-        out = torch.empty(T, Nv, HEAD_DIM, dtype=torch.bfloat16, device=dev)
+        out = torch.empty(T, Nv, HEAD_DIM, dtype=act, device=dev)
     else:
-        _need(out, "out", torch.bfloat16, (T, Nv, HEAD_DIM), dev)
+        _need(out, "out", act, (T, Nv, HEAD_DIM), dev)
     if final_state is None and output_final_state:
-        final_state = torch.empty(B, Nv, HEAD_DIM, HEAD_DIM, dtype=torch.float32, device=dev)
+        final_state = torch.empty(B, Nv, HEAD_DIM, HEAD_DIM, dtype=state, device=dev)
     elif final_state is not None:
-        _need(final_state, "final_state", torch.float32, (B, Nv, HEAD_DIM, HEAD_DIM), dev)
-    short = 1 <= int(max_seqlen) <= SHORT_MAX
+        _need(final_state, "final_state", state, (B, Nv, HEAD_DIM, HEAD_DIM), dev)
+    typed = act != torch.bfloat16 or state != torch.float32
+    short = 1 <= int(max_seqlen) <= SHORT_MAX and not typed
     if workspace is None and not short and B > 0:
-        workspace = torch.empty(workspace_bytes(T, B, Nqk, Nv), dtype=torch.uint8, device=dev)
+        nbytes = lib().gdn_chunk_fwd_typed_workspace_bytes(T, B, Nqk, Nv, DTYPES[act])
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     sc = 0.0 if scale is None else float(scale)
-    if rule == 0:
+    if typed:
+        rc = lib().gdn_chunk_fwd_typed(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+                                       _ptr(state_pool), _ptr(state_indices), sc, float(eps), _ptr(out),
+                                       _ptr(final_state), T, B, Nqk, Nv, P, rule, DTYPES[act], DTYPES[state],
+                                       int(max_seqlen), _ptr(workspace), ws_bytes, _stream(stream))
+        _check(rc, "gdn_chunk_fwd_typed")
+    elif rule == 0:
         rc = lib().gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), _ptr(state_pool),
                                  _ptr(state_indices), sc, float(eps), _ptr(out), _ptr(final_state), T, B, Nqk, Nv, P,
                                  int(max_seqlen), _ptr(workspace), ws_bytes, _stream(stream))
@@ -286,7 +312,7 @@ def pipeline_ranges(T, B, Nqk=1, Nv=1):
     """Number of chunk ranges gdn_chunk_fwd pipelines for these sizes (one carry slot per boundary
     in the workspace layout)."""
     lay = workspace_layout(T, B, Nqk, Nv)
-    return 1 + (lay["total"] - lay["carry"]) // (Nv * HEAD_DIM * HEAD_DIM * 4)
+    return 1 + (lay["act16"] - lay["carry"]) // (Nv * HEAD_DIM * HEAD_DIM * 4)
 
 
 def short_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None, scale=None, eps=1e-6,

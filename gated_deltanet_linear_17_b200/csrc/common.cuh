@@ -200,6 +200,34 @@ __device__ __forceinline__ void split_bf2(float x0, float x1, uint32_t &hi, uint
     lo = pack_bf2(x0 - h0, x1 - h1);
 }
 
+// ---------------------------------------------------------------- 16-bit activation types
+// The chunked kernels take q, k, v as raw 16-bit rows, bf16 (F16 = false) or fp16 (F16 = true); both
+// are exact tensor-core operands of kind::f16, and these helpers widen a packed pair of either type.
+template <bool F16>
+__device__ __forceinline__ float2 unpack2(uint32_t w)
+{
+    if constexpr (F16) return unpack_h2(w);
+    else return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+// split x into a pair (hi, lo) of the 16-bit type with hi + lo = x to about twice its significand
+template <bool F16>
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t &hi, uint32_t &lo)
+{
+    if constexpr (F16) {
+        hi = pack_h2(x0, x1);
+        const float2 h = unpack_h2(hi);
+        lo = pack_h2(x0 - h.x, x1 - h.y);
+    } else {
+        split_bf2(x0, x1, hi, lo);
+    }
+}
+template <bool F16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi)
+{
+    if constexpr (F16) return pack_h2(lo, hi);
+    else return pack_bf2(lo, hi);
+}
+
 // chunk table row: sequence, first token, tokens, chunk index within the sequence
 struct ChunkInfo {
     int seq, start, len, idx;
@@ -278,13 +306,14 @@ __device__ __forceinline__ void lds_vec(float (&d)[N], const float *s)
     }
 }
 
-// 1 / sqrt(|x_r|^2 + eps) for row r of a 128 x 128 16-bit tile of raw bf16 rows
+// 1 / sqrt(|x_r|^2 + eps) for row r of a 128 x 128 16-bit tile of raw bf16 (fp16 with F16) rows
 // stored as two 64-column halves of 128-byte rows with the 128-byte swizzle
 // ("L2 Normalization", eps inside the square root).  Two adjacent lanes share a
 // row (part = lane & 1): part 0 sums the first 64 columns, part 1 the last 64, each
 // 16-byte chunk in an order that keeps a quarter-warp on eight distinct bank
 // groups, with four partial sums; both lanes get the result.  Same summation
 // order in every kernel that calls it.
+template <bool F16 = false>
 __device__ __forceinline__ float row_inv_norm_pair(const uint8_t *tile, int r, int part, float eps)
 {
     float s[4] = {0.f, 0.f, 0.f, 0.f};
@@ -295,8 +324,8 @@ __device__ __forceinline__ float row_inv_norm_pair(const uint8_t *tile, int r, i
         const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float a = __uint_as_float(w4[e] << 16), b = __uint_as_float(w4[e] & 0xffff0000u);
-            s[e] = fmaf(b, b, fmaf(a, a, s[e]));
+            const float2 ab = unpack2<F16>(w4[e]);
+            s[e] = fmaf(ab.y, ab.y, fmaf(ab.x, ab.x, s[e]));
         }
     }
     float t = (s[0] + s[1]) + (s[2] + s[3]);

@@ -61,7 +61,9 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 int64_t max_chunks(int64_t T, int32_t B) { return (T + 127 * (int64_t)B) / gdn::L; }
 
-int fill_layout(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, gdn_workspace_layout_t *lay)
+// act_dtype: the activations' type; fp32 activations add the act16 region (their fp16 copies)
+int fill_layout(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, gdn_workspace_layout_t *lay,
+                int32_t act_dtype = GDN_DTYPE_BF16)
 {
     if (T < 0 || B < 0 || Nqk <= 0 || Nv <= 0) return GDN_ERR_BAD_SHAPE;
     const int64_t NC = max_chunks(T, B);
@@ -94,6 +96,9 @@ int fill_layout(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, gdn_workspace_lay
     off = align256(off);
     lay->carry = off;
     off += (size_t)(gdn::pipeline_ranges(NC) - 1) * Nv * gdn::D * gdn::D * 4;
+    off = align256(off);
+    lay->act16 = off;
+    if (act_dtype == GDN_DTYPE_FP32) off += (size_t)(2 * Nqk + Nv) * T * gdn::D * 2;
     lay->total = align256(off);
     lay->max_chunks = NC;
     return GDN_OK;
@@ -116,6 +121,7 @@ Workspace views(void *base, const gdn_workspace_layout_t &lay)
     w.Sc = reinterpret_cast<uint16_t *>(p + lay.Sc);
     w.fa = reinterpret_cast<float *>(p + lay.fa);
     w.carry = reinterpret_cast<float *>(p + lay.carry);
+    w.act16 = lay.total > lay.act16 ? reinterpret_cast<uint16_t *>(p + lay.act16) : nullptr;
     w.NC = static_cast<int>(lay.max_chunks);
     return w;
 }
@@ -151,11 +157,12 @@ float resolve_scale(float scale) { return scale > 0.f ? scale : 1.0f / sqrtf((fl
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
 
-// arguments of the whole forward (shared by gdn_chunk_fwd and gdn_short_fwd)
-int check_forward(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,
-                  const uint16_t *beta, const int32_t *cu, const float *pool, const int32_t *idx,
-                  const uint16_t *out, const float *final_state, int64_t T, int32_t B, int32_t Nqk,
-                  int32_t Nv, int32_t P, bool need_g = true, bool need_beta = true)
+// arguments of the whole forward (shared by gdn_chunk_fwd and gdn_short_fwd); ae / se: bytes per
+// activation / state element
+int check_forward(const void *q, const void *k, const void *v, const float *g,
+                  const uint16_t *beta, const int32_t *cu, const void *pool, const int32_t *idx,
+                  const void *out, const void *final_state, int64_t T, int32_t B, int32_t Nqk,
+                  int32_t Nv, int32_t P, bool need_g = true, bool need_beta = true, size_t ae = 2, size_t se = 4)
 {
     int rc = check_sizes(T, B, Nqk, Nv);
     if (rc) return rc;
@@ -171,11 +178,11 @@ int check_forward(const uint16_t *q, const uint16_t *k, const uint16_t *v, const
     if ((reinterpret_cast<uintptr_t>(g) & 3u) || (reinterpret_cast<uintptr_t>(beta) & 1u) ||
         (reinterpret_cast<uintptr_t>(cu) & 3u) || (reinterpret_cast<uintptr_t>(idx) & 3u))
         return GDN_ERR_ALIGNMENT;
-    const size_t sbytes = (size_t)gdn::D * gdn::D * 4 * Nv;
+    const size_t sbytes = (size_t)gdn::D * gdn::D * se * Nv;
     if (overlap(final_state, sbytes * B, pool, sbytes * P)) return GDN_ERR_OVERLAP;
-    const size_t obytes = (size_t)T * Nv * gdn::D * 2;
-    if (overlap(out, obytes, q, (size_t)T * Nqk * gdn::D * 2) ||
-        overlap(out, obytes, k, (size_t)T * Nqk * gdn::D * 2) || overlap(out, obytes, v, obytes))
+    const size_t obytes = (size_t)T * Nv * gdn::D * ae;
+    if (overlap(out, obytes, q, (size_t)T * Nqk * gdn::D * ae) ||
+        overlap(out, obytes, k, (size_t)T * Nqk * gdn::D * ae) || overlap(out, obytes, v, obytes))
         return GDN_ERR_OVERLAP;
     return GDN_OK;
 }
@@ -400,22 +407,49 @@ int gdn_chunk_fwd_rule(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
                        int32_t update_rule, int32_t max_seqlen, void *workspace, size_t workspace_bytes,
                        void *stream)
 {
+    return gdn_chunk_fwd_typed(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, scale, eps, out, final_state,
+                               T, B, Nqk, Nv, P, update_rule, GDN_DTYPE_BF16, GDN_DTYPE_FP32, max_seqlen, workspace,
+                               workspace_bytes, stream);
+}
+
+size_t gdn_chunk_fwd_typed_workspace_bytes(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t act_dtype)
+{
+    gdn_workspace_layout_t lay;
+    if (fill_layout(T, B, Nqk, Nv, &lay, act_dtype)) return 0;
+    return lay.total;
+}
+
+int gdn_chunk_fwd_typed(const void *q, const void *k, const void *v, const float *g, const uint16_t *beta,
+                        const int32_t *cu_seqlens, const void *state_pool, const int32_t *state_indices, float scale,
+                        float eps, void *out, void *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
+                        int32_t P, int32_t update_rule, int32_t act_dtype, int32_t state_dtype, int32_t max_seqlen,
+                        void *workspace, size_t workspace_bytes, void *stream)
+{
     if (update_rule < GDN_RULE_GATED_DELTA || update_rule > GDN_RULE_LINEAR) return GDN_ERR_BAD_SHAPE;
+    const auto known = [](int32_t d) { return d == GDN_DTYPE_FP32 || d == GDN_DTYPE_BF16 || d == GDN_DTYPE_FP16; };
+    if (!known(act_dtype) || !known(state_dtype)) return GDN_ERR_BAD_SHAPE;
     const bool decay = update_rule == GDN_RULE_GATED_DELTA || update_rule == GDN_RULE_GATED;
     const bool delta = update_rule == GDN_RULE_GATED_DELTA || update_rule == GDN_RULE_DELTA;
     if (!decay) g = nullptr;  // a zero gate
     if (!delta) beta = nullptr;
-    int rc = check_forward(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, out, final_state, T, B,
-                           Nqk, Nv, P, decay, delta);
+    const size_t ae = act_dtype == GDN_DTYPE_FP32 ? 4 : 2, se = state_dtype == GDN_DTYPE_FP32 ? 4 : 2;
+    int rc = check_forward(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, out, final_state, T, B, Nqk, Nv,
+                           P, decay, delta, ae, se);
     if (rc || B == 0) return rc;
     const cudaStream_t st = (cudaStream_t)stream;
     const float sc = resolve_scale(scale);
-    if (max_seqlen >= 1 && max_seqlen <= GDN_SHORT_MAX)
-        return cuda_status(gdn::launch_short(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, sc, eps,
-                                             out, final_state, (int)T, B, Nqk, Nv, max_seqlen, st, update_rule));
+    // the fused short-sequence kernel takes bf16 activations and an fp32 state; other types take the
+    // chunked kernels whatever the lengths
+    const bool short_ok = act_dtype == GDN_DTYPE_BF16 && state_dtype == GDN_DTYPE_FP32;
+    if (short_ok && max_seqlen >= 1 && max_seqlen <= GDN_SHORT_MAX)
+        return cuda_status(gdn::launch_short(static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(k),
+                                             static_cast<const uint16_t *>(v), g, beta, cu_seqlens,
+                                             static_cast<const float *>(state_pool), state_indices, sc, eps,
+                                             static_cast<uint16_t *>(out), static_cast<float *>(final_state), (int)T,
+                                             B, Nqk, Nv, max_seqlen, st, update_rule));
 
     gdn_workspace_layout_t lay;
-    if ((rc = fill_layout(T, B, Nqk, Nv, &lay))) return rc;
+    if ((rc = fill_layout(T, B, Nqk, Nv, &lay, act_dtype))) return rc;
     bool owned = false;
     if (!workspace) {
         if (cudaMallocAsync(&workspace, lay.total, st) != cudaSuccess) return GDN_ERR_CUDA;
@@ -426,13 +460,25 @@ int gdn_chunk_fwd_rule(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
     }
     const Workspace w = views(workspace, lay);
     const int Ti = (int)T, NC = w.NC;
+    const bool f16 = act_dtype != GDN_DTYPE_BF16;  // fp16 rows (fp32 activations: their fp16 copies)
+    const int sdt = state_dtype, odt = act_dtype;
+    const uint16_t *q16 = static_cast<const uint16_t *>(q), *k16 = static_cast<const uint16_t *>(k),
+                   *v16 = static_cast<const uint16_t *>(v);
     cudaError_t e = gdn::launch_chunk_map(cu_seqlens, B, Ti, NC, w, st);
+    if (e == cudaSuccess && act_dtype == GDN_DTYPE_FP32 && T > 0) {
+        uint16_t *aq = w.act16, *ak = aq + (size_t)T * Nqk * gdn::D, *av = ak + (size_t)T * Nqk * gdn::D;
+        e = gdn::launch_act_to_f16(static_cast<const float *>(q), static_cast<const float *>(k),
+                                   static_cast<const float *>(v), aq, ak, av, Ti, Nqk, Nv, w.status, st);
+        q16 = aq, k16 = ak, v16 = av;
+    }
     const int R = gdn::pipeline_ranges(NC);
     if (e == cudaSuccess && R == 1) {
-        e = gdn::launch_intra(k, v, g, beta, eps, Ti, Nqk, Nv, 0, NC, w, st, delta);
+        e = gdn::launch_intra(k16, v16, g, beta, eps, Ti, Nqk, Nv, 0, NC, w, st, delta, f16);
         if (e == cudaSuccess)
-            e = gdn::launch_state(k, state_pool, state_indices, final_state, Ti, B, Nqk, Nv, 0, NC, 0, w, st, delta);
-        if (e == cudaSuccess) e = gdn::launch_output(q, k, g, sc, eps, out, Ti, Nqk, Nv, 0, NC, w, st, delta);
+            e = gdn::launch_state(k16, state_pool, state_indices, final_state, Ti, B, Nqk, Nv, 0, NC, 0, w, st, delta,
+                                  f16, sdt);
+        if (e == cudaSuccess)
+            e = gdn::launch_output(q16, k16, g, sc, eps, out, Ti, Nqk, Nv, 0, NC, w, st, delta, f16, odt);
     } else if (e == cudaSuccess) {
         std::lock_guard<std::mutex> guard(g_pipe_lock);
         SideStreams *ss = nullptr;
@@ -447,20 +493,22 @@ int gdn_chunk_fwd_rule(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
             if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->intra, ev[0], 0);
             if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->state, ev[0], 0);
             for (int r = 0; r < R && e == cudaSuccess; ++r) {
-                e = gdn::launch_intra(k, v, g, beta, eps, Ti, Nqk, Nv, c0(r), c1(r) - c0(r), w, ss->intra, delta);
+                e = gdn::launch_intra(k16, v16, g, beta, eps, Ti, Nqk, Nv, c0(r), c1(r) - c0(r), w, ss->intra, delta,
+                                      f16);
                 if (e == cudaSuccess) e = cudaEventRecord(ev[1 + r], ss->intra);
             }
             for (int r = 0; r < R && e == cudaSuccess; ++r) {
                 e = cudaStreamWaitEvent(ss->state, ev[1 + r], 0);
                 if (e == cudaSuccess)
-                    e = gdn::launch_state(k, state_pool, state_indices, final_state, Ti, B, Nqk, Nv, c0(r), c1(r), r,
-                                          w, ss->state, delta);
+                    e = gdn::launch_state(k16, state_pool, state_indices, final_state, Ti, B, Nqk, Nv, c0(r), c1(r), r,
+                                          w, ss->state, delta, f16, sdt);
                 if (e == cudaSuccess) e = cudaEventRecord(ev[1 + R + r], ss->state);
             }
             for (int r = 0; r < R && e == cudaSuccess; ++r) {
                 e = cudaStreamWaitEvent(st, ev[1 + R + r], 0);
                 if (e == cudaSuccess)
-                    e = gdn::launch_output(q, k, g, sc, eps, out, Ti, Nqk, Nv, c0(r), c1(r) - c0(r), w, st, delta);
+                    e = gdn::launch_output(q16, k16, g, sc, eps, out, Ti, Nqk, Nv, c0(r), c1(r) - c0(r), w, st, delta,
+                                           f16, odt);
             }
             // join, also after a failed launch, so that nothing of this call runs outside `st` afterwards
             cudaError_t j = cudaEventRecord(ev[1 + 2 * R], ss->intra);

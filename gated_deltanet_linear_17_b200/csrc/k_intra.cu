@@ -10,8 +10,9 @@
 // page's inverse_pto does, T is built from the inverses of its 16-row diagonal
 // blocks, merged two at a time (16 -> 32 -> 64 -> 128): the inverse of
 // [[M11, 0], [M21, M22]] with M = I - Ap is [[T11, 0], [T22 Ap21 T11, T22]].
-// Steps, with the raw bf16 k and v rows staged by TMA:
-//   1. k k^T     -- tcgen05.mma M=128, N=128, K=128, bf16 (exact inputs); the L2
+// Steps, with the raw k and v rows (bf16, or fp16 when the caller's activations are
+// fp16) staged by TMA:
+//   1. k k^T     -- tcgen05.mma M=128, N=128, K=128 on the raw rows (exact inputs); the L2
 //                   norms enter as the fp32 factors rk, taken from its diagonal.
 //   2. Ap from TMEM in fp16 (the diagonal 16x16 blocks in fp32); the decay is
 //      factored per 16-column block as in the output kernel, the diagonal
@@ -53,8 +54,8 @@ constexpr int kIntraItemsPerCta = 2;
 
 // shared memory (bytes), relative to a 1024-byte aligned base; 128 x 128 16-bit
 // tiles are two 64-column halves of 128-byte rows with the 128-byte swizzle
-// Three tiles.  Tile 1 always holds raw v (bf16) -> diag(beta) v (fp16) -> W (fp16).  Of tiles 0 and 2,
-// the item's k tile holds raw k (bf16) -> diag(beta e^gamma rk) k (fp16) -> raw k again -> k_gexp (fp16)
+// Three tiles.  Tile 1 always holds raw v -> diag(beta) v (fp16) -> W (fp16).  Of tiles 0 and 2,
+// the item's k tile holds raw k -> diag(beta e^gamma rk) k (fp16) -> raw k again -> k_gexp (fp16)
 // -> Mk (fp16), and its A tile Ap (fp16) -> T (fp16), rows i, columns j -> U (fp16); the two swap roles
 // from one item of a CTA to the next.
 constexpr int OFF_T0 = 0;
@@ -110,11 +111,11 @@ __device__ __forceinline__ void warp_store16(const float (&acc)[2][4], uint8_t *
         }
 }
 
-// Rewrite a 128 x 128 tile of raw bf16 rows in place as fp16 rows scaled by fac(r),
+// Rewrite a 128 x 128 tile of raw bf16 (F16: fp16) rows in place as fp16 rows scaled by fac(r),
 // rows from nvalid on as zeros; NT threads (t = 0 .. NT - 1), thread t at chunk t % 16 of
 // rows t / 16 + (NT / 16) i, eight rows at a time with their loads issued before any
 // conversion.  With TRACK, vmax keeps the largest magnitude written (fp16 range check).
-template <int NT, bool TRACK = false, typename F>
+template <int NT, bool F16, bool TRACK = false, typename F>
 __device__ __forceinline__ void scale_rows_f16(uint8_t *tile, int t, int nvalid, F fac, float *vmax = nullptr)
 {
     constexpr int kStep = NT / 16, kRows = 128 / kStep;
@@ -137,20 +138,23 @@ __device__ __forceinline__ void scale_rows_f16(uint8_t *tile, int t, int nvalid,
                 float mx = 0.f;
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    mx = absmax_nan(absmax_nan(mx, __uint_as_float(w4[e] << 16)), __uint_as_float(w4[e] & 0xffff0000u));
+                {
+                    const float2 p = unpack2<F16>(w4[e]);
+                    mx = absmax_nan(absmax_nan(mx, p.x), p.y);
+                }
                 *vmax = absmax_nan(*vmax, mx * m);
             }
+            const float2 p0 = unpack2<F16>(x[i].x), p1 = unpack2<F16>(x[i].y), p2 = unpack2<F16>(x[i].z),
+                         p3 = unpack2<F16>(x[i].w);
             *reinterpret_cast<uint4 *>(tile + t128(r, t & 15)) =
-                r < nvalid
-                    ? make_uint4(pack_h2(__uint_as_float(x[i].x << 16) * m, __uint_as_float(x[i].x & 0xffff0000u) * m),
-                                 pack_h2(__uint_as_float(x[i].y << 16) * m, __uint_as_float(x[i].y & 0xffff0000u) * m),
-                                 pack_h2(__uint_as_float(x[i].z << 16) * m, __uint_as_float(x[i].z & 0xffff0000u) * m),
-                                 pack_h2(__uint_as_float(x[i].w << 16) * m, __uint_as_float(x[i].w & 0xffff0000u) * m))
-                    : make_uint4(0, 0, 0, 0);
+                r < nvalid ? make_uint4(pack_h2(p0.x * m, p0.y * m), pack_h2(p1.x * m, p1.y * m),
+                                        pack_h2(p2.x * m, p2.y * m), pack_h2(p3.x * m, p3.y * m))
+                           : make_uint4(0, 0, 0, 0);
         }
     }
 }
 
+template <bool F16>  // raw q/k/v rows of fp16 (else bf16)
 __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_w,
@@ -274,7 +278,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
         // ---- (1) k k^T into TMEM columns [0, 128)
         if (ok && tid == 0) {
             const uint64_t dk = tc::desc_k128(sbase + tk);
-            const uint32_t idesc = tc::idesc_f16(128, 128, true, true);
+            const uint32_t idesc = tc::idesc_f16(128, 128, !F16, !F16);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) tc::mma_f16(tmem, kmaj(dk, kk), kmaj(dk, kk), idesc, kk > 0 ? 1u : 0u);
             tc::commit(bar_mma);
@@ -289,7 +293,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
             mma_phase ^= 1;
         }
         // 1/|k_i| ("L2 Normalization") from the diagonal of k k^T, the fp32 sum of the exact squares of
-        // the bf16 entries: warp q < 4 reads its 32 rows' diagonal block of columns and keeps lane l's
+        // the raw 16-bit entries: warp q < 4 reads its 32 rows' diagonal block of columns and keeps lane l's
         // column l
         if (ok && half == 0) {
             float a[32];
@@ -314,7 +318,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
             if (ok) wait_bar(bar_v, v_par);
             if (ok) {
                 v_pend = false;
-                scale_rows_f16<kIntraThreads, true>(smem + OFF_T1, tid, n, [&](int) { return 1.f; }, &vmax);  // U = v
+                scale_rows_f16<kIntraThreads, F16, true>(smem + OFF_T1, tid, n, [&](int) { return 1.f; }, &vmax);  // U = v
                 if (tid < kFaStride) {
                     const float gl = gam[127];
                     fa[(size_t)(c * Nv + h) * kFaStride + tid] =
@@ -423,14 +427,14 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
                 }
             }
             // diag(beta e^gamma rk) k in fp16, in place (the k k^T product is complete)
-            scale_rows_f16<kIntraThreads>(smem + tk, tid, L, [&](int r) { return bet[r] * __expf(gam[r]) * rkv[r]; });
+            scale_rows_f16<kIntraThreads, F16>(smem + tk, tid, L, [&](int r) { return bet[r] * __expf(gam[r]) * rkv[r]; });
             // diag(beta) v in fp16, in place; rows past the chunk (the next sequence's) as zeros
             wait_bar(bar_v, v_par);
             if (ok) {
                 v_pend = false;
                 v_par ^= 1;
             }
-            scale_rows_f16<kIntraThreads>(smem + OFF_T1, tid, n, [&](int r) { return bet[r]; });
+            scale_rows_f16<kIntraThreads, F16>(smem + OFF_T1, tid, n, [&](int r) { return bet[r]; });
         }
         __syncthreads();
 
@@ -586,7 +590,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
 
         // ---- (5) k_gexp = fp16(rk e^{g_last - gamma} k) over the reloaded k rows (zero past the chunk), then Mk
         if (ok) wait_bar(bar_ld, 1);
-        if (ok) scale_rows_f16<kIntraThreads>(smem + tk, tid, n, [&](int r) { return kfe[r]; });
+        if (ok) scale_rows_f16<kIntraThreads, F16>(smem + tk, tid, n, [&](int r) { return kfe[r]; });
         sync_operands();
         // Mk = k_gexp^T W: A = k_gexp read MN-major (Dk contiguous), B = W MN-major; TMEM columns [0, 128)
         if (ok && tid == 0) {
@@ -665,18 +669,19 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
 }
 
 cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, const float *g, const uint16_t *beta, float eps, int T,
-                         int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st, bool delta)
+                         int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st, bool delta, bool f16)
 {
     if (nc <= 0 || T == 0) return cudaSuccess;
     if (c0 < 0 || c0 + nc > ws.NC) return cudaErrorInvalidValue;
     const uint64_t trows = (uint64_t)ws.NC * Nv * L;  // TMA coordinates are 32-bit signed
     if ((uint64_t)T >= (1ull << 31) || trows >= (1ull << 31)) return cudaErrorInvalidValue;
     CUtensorMap m_k, m_v, m_u, m_w, m_mk;
-    cudaError_t e = tma::map2d(&m_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, (uint64_t)Nqk * D, (uint64_t)T,
-                               (uint64_t)Nqk * D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    const auto AT = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    cudaError_t e = tma::map2d(&m_k, AT, k, (uint64_t)Nqk * D, (uint64_t)T, (uint64_t)Nqk * D * 2, 64, 128,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
     if (e == cudaSuccess)
-        e = tma::map2d(&m_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, (uint64_t)Nv * D, (uint64_t)T, (uint64_t)Nv * D * 2,
-                       64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+        e = tma::map2d(&m_v, AT, v, (uint64_t)Nv * D, (uint64_t)T, (uint64_t)Nv * D * 2, 64, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
     if (e == cudaSuccess)
         e = tma::map2d(&m_u, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws.U, D, trows, D * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     if (e == cudaSuccess)
@@ -685,14 +690,14 @@ cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, const float *g, c
         e = tma::map2d(&m_mk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws.Mk, D, trows, D * 2, 64, 128,
                        CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kIntraSmem);
+    auto kern = f16 ? intra_kernel<true> : intra_kernel<false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kIntraSmem);
     if (e != cudaSuccess) return e;
     const int items = nc * Nv;  // below 2^31: nc Nv L rows are addressable
     const int per = delta ? kIntraItemsPerCta : 1;
     const int grid = (items + per - 1) / per;
-    intra_kernel<<<grid, kIntraThreads, kIntraSmem, st>>>(m_k, m_v, m_u, m_w, m_mk, g, beta, eps, T, Nqk, Nv,
-                                                           ws.chunk_info, ws.rk, ws.gcum, ws.betaf, ws.fa, ws.status,
-                                                           c0, nc, delta ? 1 : 0);
+    kern<<<grid, kIntraThreads, kIntraSmem, st>>>(m_k, m_v, m_u, m_w, m_mk, g, beta, eps, T, Nqk, Nv, ws.chunk_info,
+                                                   ws.rk, ws.gcum, ws.betaf, ws.fa, ws.status, c0, nc, delta ? 1 : 0);
     return cudaGetLastError();
 }
 

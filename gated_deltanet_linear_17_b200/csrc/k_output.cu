@@ -12,8 +12,8 @@
 // 32(w%4)..32(w%4)+31 and, in the epilogues, one half of the columns.  Steps:
 //   0. TMA loads of the raw q and k rows and of W; rows past a short chunk are
 //      zeroed after the load.
-//   1. q k^T     -- tcgen05.mma M=128, N=128, K=128 on the raw bf16 rows (exact
-//                   inputs), both K-major; fp32 accumulator in TMEM.
+//   1. q k^T     -- tcgen05.mma M=128, N=128, K=128 on the raw 16-bit rows (bf16
+//                   or fp16: exact inputs), both K-major; fp32 accumulator in TMEM.
 //   2. P = rq_i rk_j exp(gamma_i - gamma_j) (q k^T)_ij for j <= i, else 0, read
 //      from TMEM and written back to TMEM in fp16 pairs, where it is the A
 //      operand of both products with P.  Since the gates are <= 0, gamma does not increase along the
@@ -30,9 +30,10 @@
 //      into W's tile, and Qw = diag(rq e^gamma) q - Z in fp16, in place of q.
 //   4. O = Qw S_c + P U -- 16 tcgen05.mma (N = 128); the eight on U are issued
 //      once it has landed, while the eight on S_c run.
-//   5. O in bf16 is staged over the consumed Qw tile and leaves by TMA for a
-//      full chunk; a short chunk's rows are stored by the threads, so rows of
-//      the next sequence are never written.
+//   5. O in out's type (bf16, fp16 or fp32): a full chunk of a 16-bit type is
+//      staged over the consumed Qw tile and leaves by TMA; a short chunk's rows,
+//      and fp32 rows, are stored by the threads, so rows of the next sequence are
+//      never written.
 // For an update rule without the retrieval (`delta` = 0: the LinearAttention
 // page's gated and linear rules) W is zero: it is not loaded, Z is not formed and
 // Qw = diag(rq e^gamma) q.
@@ -61,10 +62,13 @@ constexpr int kOutSmem = OO_BAR + 128 + 1024;
 // byte offset of 16-byte chunk c (0..15) of row r in a 128 x 128 tile
 __device__ __forceinline__ uint32_t t128(int r, int c) { return (uint32_t)((c >> 3) * 16384) + tc::sw128c(r, c & 7); }
 
+// F16: the raw q and k rows are fp16 (else bf16); ODT: out's type (kTypeBF16 or kTypeF16 through a TMA
+// store of the staged tile, kTypeF32 written by the threads)
+template <bool F16, int ODT>
 __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sc,
-    const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_out, uint16_t *__restrict__ out,
+    const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_out, void *__restrict__ out,
     const float *__restrict__ g, float scale, float eps, int T, int Nqk, int Nv, const int4 *__restrict__ info,
     float *__restrict__ rq_out, int32_t *__restrict__ status, int c0, int delta)
 {
@@ -151,7 +155,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     // ---- (1) q k^T
     if (ok && tid == 0) {
         const uint64_t dq = tc::desc_k128(sbase + OO_Q), dk = tc::desc_k128(sbase + OO_K);
-        const uint32_t idesc = tc::idesc_f16(128, 128, true, true);
+        const uint32_t idesc = tc::idesc_f16(128, 128, !F16, !F16);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) tc::mma_f16(tmem, kmaj(dq, kk), kmaj(dk, kk), idesc, kk > 0 ? 1u : 0u);
         tc::commit(bar_mma);
@@ -159,8 +163,8 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     // while it runs: scale/|q| and 1/|k| of the valid rows ("L2 Normalization") and the decay factors
     {
         const int r = tid >> 1;  // two lanes per row
-        const float xq = row_inv_norm_pair(smem + OO_Q, r, tid & 1, eps);
-        const float xk = row_inv_norm_pair(smem + OO_K, r, tid & 1, eps);
+        const float xq = row_inv_norm_pair<F16>(smem + OO_Q, r, tid & 1, eps);
+        const float xk = row_inv_norm_pair<F16>(smem + OO_K, r, tid & 1, eps);
         if ((tid & 1) == 0) {
             rqv[r] = r < n ? scale * xq : 0.f;
             rkv[r] = r < n ? xk : 0.f;
@@ -297,8 +301,9 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
                 uint32_t o4[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float x0 = __uint_as_float(w4[e] << 16) * qf - z[c4 * 8 + 2 * e];
-                    const float x1 = __uint_as_float(w4[e] & 0xffff0000u) * qf - z[c4 * 8 + 2 * e + 1];
+                    const float2 qp = unpack2<F16>(w4[e]);
+                    const float x0 = qp.x * qf - z[c4 * 8 + 2 * e];
+                    const float x1 = qp.y * qf - z[c4 * 8 + 2 * e + 1];
                     vmax = absmax_nan(absmax_nan(vmax, x0), x1);
                     o4[e] = pack_h2(x0, x1);
                 }
@@ -333,24 +338,34 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         tc::fence_after_sync();
     }
 
-    // ---- (5) O to bf16: a full chunk through shared memory (over Qw) and TMA, a short one row by row
+    // ---- (5) O in out's type: a full chunk of a 16-bit type through shared memory (over Qw) and TMA, a
+    // short one, or fp32, row by row
     if (ok) {
-        const bool full = n == L;
+        const bool full = n == L && ODT != kTypeF32;
 #pragma unroll 1
         for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
             float a[32];
             tc::tmem_ld32(t_row + j0, a);
+            if constexpr (ODT == kTypeF32) {
+                if (row < n) {
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(out) + ((size_t)(t0 + row) * Nv + h) * D + j0);
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4) dst[q4] = make_float4(a[4 * q4], a[4 * q4 + 1], a[4 * q4 + 2], a[4 * q4 + 3]);
+                }
+                continue;
+            }
+            constexpr bool OF16 = ODT == kTypeF16;
             uint4 w[4];
 #pragma unroll
             for (int q8 = 0; q8 < 4; ++q8)
-                w[q8] = make_uint4(pack_bf2(a[q8 * 8], a[q8 * 8 + 1]), pack_bf2(a[q8 * 8 + 2], a[q8 * 8 + 3]),
-                                   pack_bf2(a[q8 * 8 + 4], a[q8 * 8 + 5]), pack_bf2(a[q8 * 8 + 6], a[q8 * 8 + 7]));
+                w[q8] = make_uint4(pack2<OF16>(a[q8 * 8], a[q8 * 8 + 1]), pack2<OF16>(a[q8 * 8 + 2], a[q8 * 8 + 3]),
+                                   pack2<OF16>(a[q8 * 8 + 4], a[q8 * 8 + 5]), pack2<OF16>(a[q8 * 8 + 6], a[q8 * 8 + 7]));
             if (full) {
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8)
                     *reinterpret_cast<uint4 *>(smem + OO_Q + t128(row, (j0 >> 3) + q8)) = w[q8];
             } else if (row < n) {
-                uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)(t0 + row) * Nv + h) * D + j0);
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + ((size_t)(t0 + row) * Nv + h) * D + j0);
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8) dst[q8] = w[q8];
             }
@@ -383,8 +398,9 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     if (wid == 0) tc::tmem_dealloc(tmem, 256);
 }
 
-cudaError_t launch_output(const uint16_t *q, const uint16_t *k, const float *g, float scale, float eps, uint16_t *out,
-                          int T, int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st, bool delta)
+cudaError_t launch_output(const uint16_t *q, const uint16_t *k, const float *g, float scale, float eps, void *out,
+                          int T, int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st, bool delta,
+                          bool f16, int out_type)
 {
     if (nc <= 0 || T == 0) return cudaSuccess;
     if (c0 < 0 || c0 + nc > ws.NC) return cudaErrorInvalidValue;
@@ -393,18 +409,27 @@ cudaError_t launch_output(const uint16_t *q, const uint16_t *k, const float *g, 
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, HF = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
     CUtensorMap m_q, m_k, m_w, m_sc, m_u, m_out;
-    cudaError_t e = tma::map2d(&m_q, BF, q, (uint64_t)Nqk * D, (uint64_t)T, (uint64_t)Nqk * D * 2, 64, 128, SW);
-    if (e == cudaSuccess) e = tma::map2d(&m_k, BF, k, (uint64_t)Nqk * D, (uint64_t)T, (uint64_t)Nqk * D * 2, 64, 128, SW);
+    const auto AT = f16 ? HF : BF;
+    cudaError_t e = tma::map2d(&m_q, AT, q, (uint64_t)Nqk * D, (uint64_t)T, (uint64_t)Nqk * D * 2, 64, 128, SW);
+    if (e == cudaSuccess) e = tma::map2d(&m_k, AT, k, (uint64_t)Nqk * D, (uint64_t)T, (uint64_t)Nqk * D * 2, 64, 128, SW);
     if (e == cudaSuccess) e = tma::map2d(&m_w, HF, ws.W, D, trows, D * 2, 64, 128, SW);
     if (e == cudaSuccess) e = tma::map2d(&m_sc, HF, ws.Sc, D, trows, D * 2, 64, 128, SW);
     if (e == cudaSuccess) e = tma::map2d(&m_u, HF, ws.U, D, trows, D * 2, 64, 128, SW);
-    if (e == cudaSuccess) e = tma::map2d(&m_out, BF, out, (uint64_t)Nv * D, (uint64_t)T, (uint64_t)Nv * D * 2, 64, 128, SW);
+    if (e == cudaSuccess) {
+        if (out_type == kTypeF32)  // written by the threads: the map is never used
+            e = tma::map2d(&m_out, HF, ws.U, D, trows, D * 2, 64, 128, SW);
+        else
+            e = tma::map2d(&m_out, out_type == kTypeF16 ? HF : BF, out, (uint64_t)Nv * D, (uint64_t)T,
+                           (uint64_t)Nv * D * 2, 64, 128, SW);
+    }
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
+    auto kern = out_type == kTypeF32 ? (f16 ? output_kernel<true, kTypeF32> : output_kernel<false, kTypeF32>)
+              : out_type == kTypeF16 ? (f16 ? output_kernel<true, kTypeF16> : output_kernel<false, kTypeF16>)
+                                     : (f16 ? output_kernel<true, kTypeBF16> : output_kernel<false, kTypeBF16>);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
     if (e != cudaSuccess) return e;
-    output_kernel<<<dim3(nc, Nv), kOutThreads, kOutSmem, st>>>(m_q, m_k, m_w, m_sc, m_u, m_out, out, g, scale, eps, T,
-                                                                Nqk, Nv, ws.chunk_info, ws.rq, ws.status, c0,
-                                                                delta ? 1 : 0);
+    kern<<<dim3(nc, Nv), kOutThreads, kOutSmem, st>>>(m_q, m_k, m_w, m_sc, m_u, m_out, out, g, scale, eps, T, Nqk, Nv,
+                                                       ws.chunk_info, ws.rq, ws.status, c0, delta ? 1 : 0);
     return cudaGetLastError();
 }
 

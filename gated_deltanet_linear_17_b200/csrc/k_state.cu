@@ -9,8 +9,9 @@
 // regrouped as
 //   S_new = e^{g_last} S + Kt - Mk S,   Kt = k_gexp^T U,  Mk = k_gexp^T W.
 // Mk and the row factors f_t = rk_t e^{g_last - gamma_t} come from the
-// intra-chunk kernel.  Kt is taken exactly as the raw bf16 k rows times
-// Ub = diag(f) U split into bf16 hi + lo (about 16 significant bits).  Only
+// intra-chunk kernel.  Kt is taken exactly as the raw 16-bit k rows times
+// Ub = diag(f) U split into hi + lo halves of k's 16-bit type (about 16 significant
+// bits with bf16, 22 with fp16).  Only
 // Mk S depends on the state, so the serial chain over a sequence's chunks is
 // one product per chunk; it accumulates -Mk S (the instruction negates A)
 // onto the hi half of Kt, computed while the previous chunk's state update
@@ -22,7 +23,7 @@
 //               A = Mk K-major, B = S_c MN-major as the threads store it),
 //               committed to an mbarrier; then, once the epilogue warps have
 //               staged its operand, Kt of chunk c+1 = K^T [Ub_hi | Ub_lo]
-//               (M=128, N=128, K=128, bf16; A = the raw k tile read MN-major)
+//               (M=128, N=128, K=128, k's type; A = the raw k tile read MN-major)
 //               into the other accumulator.
 //   data warp:  a TMA store of S_c (fp16) to Sc; once chunk c's products have
 //               completed, TMA loads of chunk c+2 (Mk, the raw k rows, the U
@@ -79,10 +80,13 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int lan
     return __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
 }
 
+// F16: the raw k rows are fp16 (else bf16), and Ub's halves take the same type; SDT: the type of the
+// pool and of the final state (kTypeF32, kTypeBF16 or kTypeF16; the carried state is always fp32)
+template <bool F16, int SDT>
 __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
     const __grid_constant__ CUtensorMap tm_mk, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_sc,
-    const float *__restrict__ pool, const int32_t *__restrict__ idx, float *__restrict__ final_state, int Nqk,
+    const void *__restrict__ pool, const int32_t *__restrict__ idx, void *__restrict__ final_state, int Nqk,
     int Nv, const int4 *__restrict__ info, const int32_t *__restrict__ seq_chunk0, const float *__restrict__ fa,
     int32_t *__restrict__ status, int c_lo, int c_hi, int range, float *__restrict__ carry, int delta)
 {
@@ -164,7 +168,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float2 u = unpack_h2(x4[e]);
-                split_bf2(u.x * f, u.y * f, h4[e], l4[e]);
+                split2<F16>(u.x * f, u.y * f, h4[e], l4[e]);
             }
             const uint32_t off = tc::sw128c(row, (cbase >> 3) + j);
             *reinterpret_cast<uint4 *>(base + SG_U + off) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
@@ -175,9 +179,11 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
 
     // initial state: this thread's 32 values
     float s[32];
-    if (epi && (pool || from_carry)) {
-        const float *base = from_carry ? carry + (size_t)(range - 1) * Nv * D * D : pool + (size_t)(idx ? idx[b] : b) * Nv * D * D;
-        const float4 *src = reinterpret_cast<const float4 *>(base + ((size_t)h * D + row) * D + col0 + cbase);
+    const size_t s_off = ((size_t)h * D + row) * D + col0 + cbase;  // this thread's 32 values in a state
+    if (epi && (from_carry || (pool && SDT == kTypeF32))) {
+        const float *base = from_carry ? carry + (size_t)(range - 1) * Nv * D * D
+                                       : static_cast<const float *>(pool) + (size_t)(idx ? idx[b] : b) * Nv * D * D;
+        const float4 *src = reinterpret_cast<const float4 *>(base + s_off);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const float4 v4 = src[j];
@@ -185,6 +191,20 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
             s[4 * j + 1] = v4.y;
             s[4 * j + 2] = v4.z;
             s[4 * j + 3] = v4.w;
+        }
+    } else if (epi && pool) {  // a 16-bit pool, widened exactly
+        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(pool) +
+                                                           (size_t)(idx ? idx[b] : b) * Nv * D * D + s_off);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint4 w = src[j];
+            const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 p = unpack2<SDT == kTypeF16>(w4[e]);
+                s[8 * j + 2 * e] = p.x;
+                s[8 * j + 2 * e + 1] = p.y;
+            }
         }
     } else {
 #pragma unroll
@@ -229,7 +249,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
 
     const uint32_t tmem = *tslot;
     const uint32_t t_mine = tmem + ((uint32_t)(quarter * 32) << 16) + cbase;
-    const uint32_t idesc_kt = tc::idesc_f16(128, 128, true, true, true, true);
+    const uint32_t idesc_kt = tc::idesc_f16(128, 128, !F16, !F16, true, true);
     const uint32_t idesc_mk = tc::idesc_f16(128, 64, false, false, false, true) | (1u << 13);  // A negated
     // Operand descriptors of k step 0; the start-address field holds (byte
     // address >> 4) and every address stays below 256 KiB, so the descriptor
@@ -319,11 +339,20 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
     if (epi && __any_sync(0xffffffffu, out_of_fp16(vmax)) && lane == 0) atomicOr(status + 3, GDN_DEV_RANGE_STATE);
     if (!ok) {
         if (tid == 0) atomicOr(status + 2, GDN_DEV_WAIT_STATE);
-    } else if (epi && (final_state || to_carry)) {
-        float *base = to_carry ? carry + (size_t)range * Nv * D * D : final_state + (size_t)b * Nv * D * D;
-        float4 *dst = reinterpret_cast<float4 *>(base + ((size_t)h * D + row) * D + col0 + cbase);
+    } else if (epi && (to_carry || (final_state && SDT == kTypeF32))) {
+        float *base = to_carry ? carry + (size_t)range * Nv * D * D
+                               : static_cast<float *>(final_state) + (size_t)b * Nv * D * D;
+        float4 *dst = reinterpret_cast<float4 *>(base + s_off);
 #pragma unroll
         for (int j = 0; j < 8; ++j) dst[j] = make_float4(s[4 * j], s[4 * j + 1], s[4 * j + 2], s[4 * j + 3]);
+    } else if (epi && final_state) {  // a 16-bit final state, rounded to nearest even
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(final_state) + (size_t)b * Nv * D * D + s_off);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float *v8 = s + 8 * j;
+            dst[j] = make_uint4(pack2<SDT == kTypeF16>(v8[0], v8[1]), pack2<SDT == kTypeF16>(v8[2], v8[3]),
+                                pack2<SDT == kTypeF16>(v8[4], v8[5]), pack2<SDT == kTypeF16>(v8[6], v8[7]));
+        }
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -331,9 +360,9 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
     if (wid == 0) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
-cudaError_t launch_state(const uint16_t *k, const float *pool, const int32_t *idx, float *final_state, int T, int B,
+cudaError_t launch_state(const uint16_t *k, const void *pool, const int32_t *idx, void *final_state, int T, int B,
                          int Nqk, int Nv, int c_lo, int c_hi, int range, const Workspace &ws, cudaStream_t st,
-                         bool delta)
+                         bool delta, bool f16, int state_type)
 {
     if (B == 0) return cudaSuccess;
     if (range < 0 || range >= kMaxRanges || c_lo < 0 || c_hi < c_lo) return cudaErrorInvalidValue;
@@ -347,16 +376,19 @@ cudaError_t launch_state(const uint16_t *k, const float *pool, const int32_t *id
     cudaError_t e = tma::map2d(&m_mk, HF, ws.Mk, D, rows, D * 2, 64, 128, SW);
     if (e == cudaSuccess) {
         if (T > 0)
-            e = tma::map2d(&m_k, BF, k, (uint64_t)Nqk * D, (uint64_t)T, (uint64_t)Nqk * D * 2, 64, 128, SW);
+            e = tma::map2d(&m_k, f16 ? HF : BF, k, (uint64_t)Nqk * D, (uint64_t)T, (uint64_t)Nqk * D * 2, 64, 128, SW);
         else  // no chunk exists, so the map is never used
             e = tma::map2d(&m_k, BF, ws.Mk, D, rows, D * 2, 64, 128, SW);
     }
     if (e == cudaSuccess) e = tma::map2d(&m_u, HF, ws.U, D, rows, D * 2, DVT, 128, SW);
     if (e == cudaSuccess) e = tma::map2d(&m_sc, HF, ws.Sc, D, rows, D * 2, DVT, 128, SW);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStateSmem);
+    auto kern = state_type == kTypeF16 ? (f16 ? state_kernel<true, kTypeF16> : state_kernel<false, kTypeF16>)
+              : state_type == kTypeBF16 ? (f16 ? state_kernel<true, kTypeBF16> : state_kernel<false, kTypeBF16>)
+                                        : (f16 ? state_kernel<true, kTypeF32> : state_kernel<false, kTypeF32>);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStateSmem);
     if (e != cudaSuccess) return e;
-    state_kernel<<<dim3(B, Nv, D / DVT), kStateThreads, kStateSmem, st>>>(
+    kern<<<dim3(B, Nv, D / DVT), kStateThreads, kStateSmem, st>>>(
         m_mk, m_k, m_u, m_sc, pool, idx, final_state, Nqk, Nv, ws.chunk_info, ws.seq_chunk0, ws.fa, ws.status, c_lo,
         c_hi, range, ws.carry, delta ? 1 : 0);
     return cudaGetLastError();

@@ -58,8 +58,10 @@
  *   [3] values outside the fp16 range (|x| > 65504) in an fp16 intermediate:
  *       GDN_DEV_RANGE_INTRA (U, or beta v, which shows up in U),
  *       GDN_DEV_RANGE_STATE (the state's fp16 operand copy),
- *       GDN_DEV_RANGE_OUTPUT (the output kernel's fp16 operand).  A NaN in
- *       one of them also sets the bit.  See "fp16 intermediates" below.
+ *       GDN_DEV_RANGE_OUTPUT (the output kernel's fp16 operand),
+ *       GDN_DEV_RANGE_INPUT (an fp32 q, k or v element of gdn_chunk_fwd_typed,
+ *       which the chunked path rounds to fp16).  A NaN in one of them also
+ *       sets the bit.  See "fp16 intermediates" below.
  * Words 0, 2 and 3 are cleared at the start of every chunked call (by the
  * chunk-table kernel, on `stream`, before any kernel that sets a bit), so the
  * words describe the last chunked call on that workspace.  A nonzero word 2 or
@@ -95,7 +97,8 @@ extern "C" {
 #define GDN_NOALLOC_SCRATCH_BYTES (64u << 20) /* static workspace of gdn_chunk_fwd_noalloc, per GPU */
 #define GDN_MAX_STATE_WINDOW 8 /* largest state_window of gdn_recurrent_window_fwd */
 
-/* element types of gdn_recurrent_fwd's activations and state pool */
+/* element types of the activations and states of gdn_chunk_fwd_typed, gdn_recurrent_fwd and
+   gdn_recurrent_window_fwd */
 #define GDN_DTYPE_FP32 0
 #define GDN_DTYPE_BF16 1
 #define GDN_DTYPE_FP16 2
@@ -117,6 +120,7 @@ extern "C" {
 #define GDN_DEV_RANGE_INTRA 1   /* word 3: U (or beta v) beyond +-65504         */
 #define GDN_DEV_RANGE_STATE 2   /* word 3: the state beyond +-65504             */
 #define GDN_DEV_RANGE_OUTPUT 4  /* word 3: the output kernel's fp16 operand beyond +-65504 */
+#define GDN_DEV_RANGE_INPUT 8   /* word 3: an fp32 activation beyond +-65504 (gdn_chunk_fwd_typed) */
 
 typedef enum {
     GDN_OK = 0,
@@ -224,6 +228,37 @@ int gdn_chunk_fwd_rule(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
                        float *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t P,
                        int32_t update_rule, int32_t max_seqlen, void *workspace, size_t workspace_bytes,
                        void *stream);
+
+/*
+ * gdn_chunk_fwd_typed -- gdn_chunk_fwd_rule with the element types of the page
+ * "com.microsoft.LinearAttention" ("Activations and state may independently
+ * use float16 or float32"), beside the decode page's bf16 activations and bf16
+ * state; gdn_chunk_fwd_rule is this call with bf16 activations and an fp32
+ * state.
+ *
+ *   act_dtype     GDN_DTYPE_BF16, GDN_DTYPE_FP16 or GDN_DTYPE_FP32: the type of
+ *                 q, k, v and out (each laid out as for gdn_chunk_fwd)
+ *   state_dtype   GDN_DTYPE_FP32, GDN_DTYPE_FP16 or GDN_DTYPE_BF16: the type of
+ *                 state_pool and final_state (the state itself is carried in
+ *                 fp32 on the chip; a 16-bit pool is widened exactly, a 16-bit
+ *                 final state rounded to nearest even)
+ *   g, beta       fp32 and bf16 as for gdn_chunk_fwd, in every combination
+ *   workspace     >= gdn_chunk_fwd_typed_workspace_bytes(T, B, Nqk, Nv, act_dtype),
+ *                 or NULL (allocated and freed stream-ordered)
+ * bf16 and fp16 rows enter the tensor core as they are (both exact operands);
+ * fp32 q, k and v are first rounded to fp16 in the workspace (11 significant
+ * bits; an element beyond +-65504 sets GDN_DEV_RANGE_INPUT, see "Device
+ * status").  The fused short-sequence kernel serves bf16 activations with an
+ * fp32 state; other types run the chunked kernels for any max_seqlen.  Every
+ * other argument, limit and error as for gdn_chunk_fwd_rule; an unknown type
+ * code is GDN_ERR_BAD_SHAPE.
+ */
+size_t gdn_chunk_fwd_typed_workspace_bytes(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t act_dtype);
+int gdn_chunk_fwd_typed(const void *q, const void *k, const void *v, const float *g, const uint16_t *beta,
+                        const int32_t *cu_seqlens, const void *state_pool, const int32_t *state_indices, float scale,
+                        float eps, void *out, void *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
+                        int32_t P, int32_t update_rule, int32_t act_dtype, int32_t state_dtype, int32_t max_seqlen,
+                        void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd for callers that cannot allocate

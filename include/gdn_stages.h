@@ -60,6 +60,9 @@ extern "C" {
  *   carry       fp32 [R-1][Nv][128][128]: the state of a sequence that crosses the
  *               boundary after chunk range r (the forward pass runs R chunk ranges
  *               as a pipeline: R = 2 from NC = 32 on, else 1; empty when R = 1)
+ *   act16       fp16 q [T][Nqk][128], k [T][Nqk][128], v [T][Nv][128]: fp32
+ *               activations of gdn_chunk_fwd_typed rounded to fp16 (empty for
+ *               16-bit activations and in gdn_workspace_layout)
  * The tensor-core products take fp16 operands (11-bit significand) with fp32
  * accumulation: the raw bf16 q, k, v convert to fp16 exactly (magnitudes in
  * [2^-14, 65504]), the L2 norms enter as fp32 scalings, and the state update's
@@ -82,6 +85,7 @@ typedef struct {
     size_t Sc;
     size_t fa;
     size_t carry;
+    size_t act16;
     int64_t max_chunks;
 } gdn_workspace_layout_t;
 

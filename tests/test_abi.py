@@ -248,3 +248,28 @@ def test_window_entry_argument_errors(lib):
     assert call(out=9 * M + 3 * entry, W=3, g=None) == B.GDN_ERR_NULL_ARG  # past a 3-entry window: later checks
     assert call(B=0) == B.GDN_OK and call(T=0) == B.GDN_OK
     assert call(W=0, g=None) == B.GDN_ERR_NULL_ARG                  # the gated delta rule reads g
+
+
+def test_typed_entry_argument_errors(lib):
+    M = 1 << 20  # fake, disjoint, aligned addresses; every call below returns before any launch
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+
+    def call(**over):
+        a = dict(q=M, k=2 * M, v=3 * M, g=4 * M, beta=5 * M, cu=6 * M, pool=None, out=7 * M, fin=None, T=8, B=1,
+                 Nqk=2, Nv=4, P=0, rule=0, act=2, sdt=0, ws=None, wsb=0)
+        a.update(over)
+        return lib.gdn_chunk_fwd_typed(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["g"]), vp(a["beta"]), vp(a["cu"]),
+                                       vp(a["pool"]), None, 0.0, 1e-6, vp(a["out"]), vp(a["fin"]), a["T"], a["B"],
+                                       a["Nqk"], a["Nv"], a["P"], a["rule"], a["act"], a["sdt"], 0, vp(a["ws"]),
+                                       a["wsb"], None)
+    assert call(act=3) == B.GDN_ERR_BAD_SHAPE and call(sdt=-1) == B.GDN_ERR_BAD_SHAPE
+    assert call(rule=4) == B.GDN_ERR_BAD_SHAPE
+    assert call(Nv=3) == B.GDN_ERR_BAD_SHAPE
+    assert call(q=None) == B.GDN_ERR_NULL_ARG
+    # fp32 activations: out (4 bytes per element) overlaps v when 16 KiB apart
+    assert call(act=0, out=3 * M + 8 * 4 * 128 * 2) == B.GDN_ERR_OVERLAP
+    assert call(ws=8 << 20, wsb=10) == B.GDN_ERR_WORKSPACE
+    # the fp32-activation workspace holds their fp16 copies on top of the 16-bit one
+    w16 = lib.gdn_chunk_fwd_typed_workspace_bytes(4096, 2, 4, 8, 2)
+    w32 = lib.gdn_chunk_fwd_typed_workspace_bytes(4096, 2, 4, 8, 0)
+    assert w16 == gdn.workspace_bytes(4096, 2, 4, 8) and w32 >= w16 + (2 * 4 + 8) * 4096 * 128 * 2
