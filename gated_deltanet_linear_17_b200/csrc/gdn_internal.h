@@ -83,5 +83,12 @@ cudaError_t launch_recurrent(const void *q, const void *k, const void *v, const 
                              int win = 0);
 // win > 0: the pool is a state window [win, B, Nv, Dk, Dv] updated in place (token_slots and
 // num_accepted unused); see gdn_recurrent_window_fwd in gdn.h.
+// The one-token decode kernel (k_decode.cu): launch_recurrent routes to it when max_seqlen == 1 and
+// decode_supported() holds (bf16 activations, an fp32 or bf16 pool, Dk 64 or 128, no window).
+bool decode_supported(int act_dtype, int state_dtype, int Dk, int Dv, int win);
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g, const uint16_t *beta,
+                          const float *gk, const int32_t *cu, void *pool, int state_dtype, int rule,
+                          const int32_t *token_slots, const int32_t *num_accepted, float scale, float eps, void *out,
+                          int T, int B, int Nqk, int Nv, int Dk, int Dv, cudaStream_t st);
 
 }  // namespace gdn

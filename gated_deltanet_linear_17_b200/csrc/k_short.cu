@@ -583,6 +583,9 @@ cudaError_t launch_recurrent(const void *q, const void *k, const void *v, const 
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
+    if (max_seqlen == 1 && decode_supported(act_dtype, state_dtype, Dk, Dv, win))
+        return launch_decode(q, k, v, g, beta, gk, cu, pool, state_dtype, rule, token_slots, num_accepted, scale, eps,
+                             out, T, B, Nqk, Nv, Dk, Dv, st);
     const RecArgs a{q, k, v, g, beta, gk, cu, pool, token_slots, num_accepted, scale, eps, out, T, Nqk, Nv, Dv, win, B};
     const dim3 grid(B, Nv, Dv / kTile);
     const bool few = max_seqlen >= 1 && max_seqlen <= 8;

@@ -210,3 +210,36 @@ def test_recurrent_linear_attention_types(act, state):
     assert_close(pool[torch.from_numpy(written).to(DEV).long()], rpool[written], f"{what} written slots")
     others = torch.from_numpy(np.setdiff1d(np.arange(pool.shape[0]), written)).to(DEV).long()
     assert torch.equal(pool[others], start[others])
+
+
+@pytest.mark.parametrize("bf16_pool", [False, True])
+@pytest.mark.parametrize("rule", ["gated_delta", "delta", "gated", "linear"])
+def test_recurrent_one_token_decode_kernel(bf16_pool, rule):
+    """max_seqlen = 1 (one token per sequence, the decode page's common call) takes the streaming decode
+    kernel: a token per sequence, empty sequences, some sequences moved to another slot, the key gate on
+    the decaying rules."""
+    r = np.random.default_rng(110)
+    lens = [int(x) for x in r.choice([0, 1, 1, 1], size=70)]
+    inp, slots, acc = _case(lens, Nqk=4, Nv=8, P=160, seed=111, per_token=True, accepted=False)
+    gk = _key_gate(inp, 112) if rule in ("gated_delta", "gated") else None
+    _run_and_check(inp, slots, acc, 1, f"decode kernel {rule} bf16_pool={bf16_pool}", gk=gk, bf16_pool=bf16_pool,
+                   rule=rule)
+
+
+@pytest.mark.parametrize("Dk,Dv", [(64, 512), (64, 64), (128, 256)])
+def test_recurrent_one_token_decode_head_dimensions(Dk, Dv):
+    r = np.random.default_rng(113)
+    lens = [int(x) for x in r.choice([0, 1], size=40, p=[0.1, 0.9])]
+    inp, slots, acc = _case(lens, Nqk=2, Nv=4, P=60, seed=114, per_token=False, accepted=False, Dk=Dk, Dv=Dv)
+    _run_and_check(inp, slots, acc, 1, f"decode kernel Dk={Dk} Dv={Dv} bf16", gk=_key_gate(inp, 115), bf16_pool=True)
+    _run_and_check(inp, slots, acc, 1, f"decode kernel Dk={Dk} Dv={Dv} fp32")
+
+
+@pytest.mark.parametrize("bf16_pool", [False, True])
+def test_recurrent_decode_hint_too_small_stays_exact(bf16_pool):
+    """max_seqlen = 1 understated: sequences of 2..6 tokens with per-token slots and accepted counts run
+    the decode kernel's fp32 register path and still match the oracle."""
+    lens = [1, 3, 0, 6, 1, 2, 5]
+    inp, slots, acc = _case(lens, Nqk=2, Nv=4, P=40, seed=116, per_token=True, accepted=True)
+    _run_and_check(inp, slots, acc, 1, f"decode kernel understated hint bf16_pool={bf16_pool}",
+                   gk=_key_gate(inp, 117), bf16_pool=bf16_pool)
