@@ -67,12 +67,12 @@ def lib():
         L.gdn_chunk_fwd_rule.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, i32, i32, p,
                                          sz, p]
         L.gdn_chunk_fwd_typed_workspace_bytes.restype = sz
-        L.gdn_chunk_fwd_typed_workspace_bytes.argtypes = [i64, i32, i32, i32, i32]
+        L.gdn_chunk_fwd_typed_workspace_bytes.argtypes = [i64, i32, i32, i32, i32, i32, i32]
         L.gdn_chunk_fwd_typed.restype = ctypes.c_int
-        # q k v g beta cu pool idx | scale eps | out final | T B Nqk Nv P | rule act_dtype state_dtype max_seqlen |
-        # workspace bytes stream
+        # q k v g beta cu pool idx | scale eps | out final | T B Nqk Nv P | rule act_dtype state_dtype Dk Dv
+        # max_seqlen | workspace bytes stream
         L.gdn_chunk_fwd_typed.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, i32, i32,
-                                          i32, i32, p, sz, p]
+                                          i32, i32, i32, i32, p, sz, p]
         L.gdn_chunk_fwd_noalloc.restype = ctypes.c_int
         L.gdn_chunk_fwd_noalloc.argtypes = [p, p, p, p, p, p, p, p, f32, f32, p, p, i64, i32, i32, i32, i32, i32, p]
         L.gdn_selftest_umma.restype = ctypes.c_int
@@ -161,27 +161,29 @@ def workspace_layout(T: int, B: int, Nqk: int, Nv: int) -> dict:
     return {n: getattr(lay, n) for n, _ in _Layout._fields_}
 
 
-def _resolve(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, act=torch.bfloat16, state=torch.float32):
+def _resolve(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, act=torch.bfloat16, state=torch.float32,
+             dims=False):
+    """Shapes of a chunked call; ``dims`` allows head dimensions other than 128 (the typed entry)."""
     if q.dim() != 3 or v.dim() != 3:
-        raise ValueError("q/k must be [T, Nqk, 128] and v [T, Nv, 128]")
+        raise ValueError("q/k must be [T, Nqk, Dk] and v [T, Nv, Dv]")
     T, Nqk, Dk = q.shape
-    Nv = v.shape[1]
-    if Dk != HEAD_DIM or v.shape[2] != HEAD_DIM:
+    Nv, Dv = v.shape[1], v.shape[2]
+    if not dims and (Dk != HEAD_DIM or Dv != HEAD_DIM):
         raise ValueError(f"head dimension must be {HEAD_DIM}")
     if Nv % Nqk != 0:
         raise ValueError(f"Nv ({Nv}) must be a multiple of Nqk ({Nqk})")
     B = cu_seqlens.shape[0] - 1
     dev = q.device
-    _need(q, "q", act, (T, Nqk, HEAD_DIM), dev)
-    _need(k, "k", act, (T, Nqk, HEAD_DIM), dev)
-    _need(v, "v", act, (T, Nv, HEAD_DIM), dev)
+    _need(q, "q", act, (T, Nqk, Dk), dev)
+    _need(k, "k", act, (T, Nqk, Dk), dev)
+    _need(v, "v", act, (T, Nv, Dv), dev)
     _need(g, "g", torch.float32, (T, Nv), dev)
     _need(beta, "beta", torch.bfloat16, (T, Nv), dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), dev)
     P = 0
     if state_pool is not None:
         P = state_pool.shape[0]
-        _need(state_pool, "state_pool", state, (P, Nv, HEAD_DIM, HEAD_DIM), dev)
+        _need(state_pool, "state_pool", state, (P, Nv, Dk, Dv), dev)
     if state_indices is not None:
         _need(state_indices, "state_indices", torch.int32, (B,), dev)
     return T, B, Nqk, Nv, P, dev
@@ -205,8 +207,10 @@ def chunk_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None,
     Element types (the LinearAttention page: activations and state each fp16 or
     fp32): q, k, v and out share one type, bf16, fp16 or fp32; the state pool and
     final_state share another, fp32, fp16 or bf16 (``state_dtype`` sets it when
-    there is no pool; fp32 by default).  Anything but bf16 activations with an
-    fp32 state goes through ``gdn_chunk_fwd_typed``."""
+    there is no pool; fp32 by default).  Head dimensions: Dk (q, k) 64 or 128,
+    Dv (v, out, states [.., Dk, Dv]) a multiple of 128 up to 512.  Anything but
+    bf16 activations with an fp32 state and 128 x 128 heads goes through
+    ``gdn_chunk_fwd_typed``."""
     if update_rule not in UPDATE_RULES:
         raise ValueError(f"update_rule must be one of {sorted(UPDATE_RULES)}")
     rule = UPDATE_RULES[update_rule]
@@ -222,26 +226,29 @@ def chunk_fwd(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None,
         raise RuntimeError(f"activations and states must be bfloat16, float16 or float32 (got {act}, {state})")
     gg = g if g is not None else torch.empty(q.shape[0], v.shape[1], dtype=torch.float32, device=q.device)
     bb = beta if beta is not None else torch.empty(q.shape[0], v.shape[1], dtype=torch.bfloat16, device=q.device)
-    T, B, Nqk, Nv, P, dev = _resolve(q, k, v, gg, bb, cu_seqlens, state_pool, state_indices, act, state)
+    T, B, Nqk, Nv, P, dev = _resolve(q, k, v, gg, bb, cu_seqlens, state_pool, state_indices, act, state, dims=True)
+    Dk, Dv = q.shape[2], v.shape[2]
     if out is None:
-        out = torch.empty(T, Nv, HEAD_DIM, dtype=act, device=dev)
+        out = torch.empty(T, Nv, Dv, dtype=act, device=dev)
     else:
-        _need(out, "out", act, (T, Nv, HEAD_DIM), dev)
+        _need(out, "out", act, (T, Nv, Dv), dev)
     if final_state is None and output_final_state:
-        final_state = torch.empty(B, Nv, HEAD_DIM, HEAD_DIM, dtype=state, device=dev)
+        final_state = torch.empty(B, Nv, Dk, Dv, dtype=state, device=dev)
     elif final_state is not None:
-        _need(final_state, "final_state", state, (B, Nv, HEAD_DIM, HEAD_DIM), dev)
-    typed = act != torch.bfloat16 or state != torch.float32
+        _need(final_state, "final_state", state, (B, Nv, Dk, Dv), dev)
+    typed = act != torch.bfloat16 or state != torch.float32 or Dk != HEAD_DIM or Dv != HEAD_DIM
     short = 1 <= int(max_seqlen) <= SHORT_MAX and not typed
     if workspace is None and not short and B > 0:
-        nbytes = lib().gdn_chunk_fwd_typed_workspace_bytes(T, B, Nqk, Nv, DTYPES[act])
+        nbytes = lib().gdn_chunk_fwd_typed_workspace_bytes(T, B, Nqk, Nv, DTYPES[act], Dk, Dv)
+        if nbytes == 0:
+            raise ValueError(f"unsupported head dimensions Dk={Dk}, Dv={Dv}")
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     sc = 0.0 if scale is None else float(scale)
     if typed:
         rc = lib().gdn_chunk_fwd_typed(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
                                        _ptr(state_pool), _ptr(state_indices), sc, float(eps), _ptr(out),
-                                       _ptr(final_state), T, B, Nqk, Nv, P, rule, DTYPES[act], DTYPES[state],
+                                       _ptr(final_state), T, B, Nqk, Nv, P, rule, DTYPES[act], DTYPES[state], Dk, Dv,
                                        int(max_seqlen), _ptr(workspace), ws_bytes, _stream(stream))
         _check(rc, "gdn_chunk_fwd_typed")
     elif rule == 0:

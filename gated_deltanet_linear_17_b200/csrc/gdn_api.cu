@@ -61,9 +61,10 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 int64_t max_chunks(int64_t T, int32_t B) { return (T + 127 * (int64_t)B) / gdn::L; }
 
-// act_dtype: the activations' type; fp32 activations add the act16 region (their fp16 copies)
+// act_dtype: the activations' type; fp32 activations add the act16 region (their fp16 copies, q and k
+// rows of Dk elements); Nv counts 128-column sub-heads (Nv Dv / 128 for a value dimension Dv)
 int fill_layout(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, gdn_workspace_layout_t *lay,
-                int32_t act_dtype = GDN_DTYPE_BF16)
+                int32_t act_dtype = GDN_DTYPE_BF16, int32_t Dk = gdn::D)
 {
     if (T < 0 || B < 0 || Nqk <= 0 || Nv <= 0) return GDN_ERR_BAD_SHAPE;
     const int64_t NC = max_chunks(T, B);
@@ -98,7 +99,7 @@ int fill_layout(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, gdn_workspace_lay
     off += (size_t)(gdn::pipeline_ranges(NC) - 1) * Nv * gdn::D * gdn::D * 4;
     off = align256(off);
     lay->act16 = off;
-    if (act_dtype == GDN_DTYPE_FP32) off += (size_t)(2 * Nqk + Nv) * T * gdn::D * 2;
+    if (act_dtype == GDN_DTYPE_FP32) off += ((size_t)2 * Nqk * Dk + (size_t)Nv * gdn::D) * T * 2;
     lay->total = align256(off);
     lay->max_chunks = NC;
     return GDN_OK;
@@ -158,11 +159,12 @@ float resolve_scale(float scale) { return scale > 0.f ? scale : 1.0f / sqrtf((fl
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
 
 // arguments of the whole forward (shared by gdn_chunk_fwd and gdn_short_fwd); ae / se: bytes per
-// activation / state element
+// activation / state element; Dk, Dv: head dimensions
 int check_forward(const void *q, const void *k, const void *v, const float *g,
                   const uint16_t *beta, const int32_t *cu, const void *pool, const int32_t *idx,
                   const void *out, const void *final_state, int64_t T, int32_t B, int32_t Nqk,
-                  int32_t Nv, int32_t P, bool need_g = true, bool need_beta = true, size_t ae = 2, size_t se = 4)
+                  int32_t Nv, int32_t P, bool need_g = true, bool need_beta = true, size_t ae = 2, size_t se = 4,
+                  int32_t Dk = gdn::D, int32_t Dv = gdn::D)
 {
     int rc = check_sizes(T, B, Nqk, Nv);
     if (rc) return rc;
@@ -178,11 +180,11 @@ int check_forward(const void *q, const void *k, const void *v, const float *g,
     if ((reinterpret_cast<uintptr_t>(g) & 3u) || (reinterpret_cast<uintptr_t>(beta) & 1u) ||
         (reinterpret_cast<uintptr_t>(cu) & 3u) || (reinterpret_cast<uintptr_t>(idx) & 3u))
         return GDN_ERR_ALIGNMENT;
-    const size_t sbytes = (size_t)gdn::D * gdn::D * se * Nv;
+    const size_t sbytes = (size_t)Dk * Dv * se * Nv;
     if (overlap(final_state, sbytes * B, pool, sbytes * P)) return GDN_ERR_OVERLAP;
-    const size_t obytes = (size_t)T * Nv * gdn::D * ae;
-    if (overlap(out, obytes, q, (size_t)T * Nqk * gdn::D * ae) ||
-        overlap(out, obytes, k, (size_t)T * Nqk * gdn::D * ae) || overlap(out, obytes, v, obytes))
+    const size_t obytes = (size_t)T * Nv * Dv * ae;
+    if (overlap(out, obytes, q, (size_t)T * Nqk * Dk * ae) ||
+        overlap(out, obytes, k, (size_t)T * Nqk * Dk * ae) || overlap(out, obytes, v, obytes))
         return GDN_ERR_OVERLAP;
     return GDN_OK;
 }
@@ -408,39 +410,47 @@ int gdn_chunk_fwd_rule(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
                        void *stream)
 {
     return gdn_chunk_fwd_typed(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, scale, eps, out, final_state,
-                               T, B, Nqk, Nv, P, update_rule, GDN_DTYPE_BF16, GDN_DTYPE_FP32, max_seqlen, workspace,
-                               workspace_bytes, stream);
+                               T, B, Nqk, Nv, P, update_rule, GDN_DTYPE_BF16, GDN_DTYPE_FP32, GDN_HEAD_DIM, GDN_HEAD_DIM,
+                               max_seqlen, workspace, workspace_bytes, stream);
 }
 
-size_t gdn_chunk_fwd_typed_workspace_bytes(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t act_dtype)
+size_t gdn_chunk_fwd_typed_workspace_bytes(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t act_dtype, int32_t Dk,
+                                           int32_t Dv)
 {
+    if ((Dk != 64 && Dk != 128) || Dv <= 0 || Dv % 128 != 0 || Dv > 512 || Nv <= 0) return 0;
     gdn_workspace_layout_t lay;
-    if (fill_layout(T, B, Nqk, Nv, &lay, act_dtype)) return 0;
+    if (fill_layout(T, B, Nqk, Nv * (Dv / 128), &lay, act_dtype, Dk)) return 0;
     return lay.total;
 }
 
 int gdn_chunk_fwd_typed(const void *q, const void *k, const void *v, const float *g, const uint16_t *beta,
                         const int32_t *cu_seqlens, const void *state_pool, const int32_t *state_indices, float scale,
                         float eps, void *out, void *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
-                        int32_t P, int32_t update_rule, int32_t act_dtype, int32_t state_dtype, int32_t max_seqlen,
-                        void *workspace, size_t workspace_bytes, void *stream)
+                        int32_t P, int32_t update_rule, int32_t act_dtype, int32_t state_dtype, int32_t Dk, int32_t Dv,
+                        int32_t max_seqlen, void *workspace, size_t workspace_bytes, void *stream)
 {
     if (update_rule < GDN_RULE_GATED_DELTA || update_rule > GDN_RULE_LINEAR) return GDN_ERR_BAD_SHAPE;
     const auto known = [](int32_t d) { return d == GDN_DTYPE_FP32 || d == GDN_DTYPE_BF16 || d == GDN_DTYPE_FP16; };
     if (!known(act_dtype) || !known(state_dtype)) return GDN_ERR_BAD_SHAPE;
+    if (Dk <= 0 || Dv <= 0) return GDN_ERR_BAD_SHAPE;
+    if ((Dk != 64 && Dk != 128) || Dv % 128 != 0 || Dv > 512) return GDN_ERR_UNSUPPORTED;
+    gdn::Dims dims;
+    dims.Dk = Dk, dims.Dv = Dv, dims.m = Dv / 128;
+    if (Nv > 0 && (int64_t)Nv * dims.m > 256) return GDN_ERR_UNSUPPORTED;
     const bool decay = update_rule == GDN_RULE_GATED_DELTA || update_rule == GDN_RULE_GATED;
     const bool delta = update_rule == GDN_RULE_GATED_DELTA || update_rule == GDN_RULE_DELTA;
     if (!decay) g = nullptr;  // a zero gate
     if (!delta) beta = nullptr;
     const size_t ae = act_dtype == GDN_DTYPE_FP32 ? 4 : 2, se = state_dtype == GDN_DTYPE_FP32 ? 4 : 2;
     int rc = check_forward(q, k, v, g, beta, cu_seqlens, state_pool, state_indices, out, final_state, T, B, Nqk, Nv,
-                           P, decay, delta, ae, se);
+                           P, decay, delta, ae, se, Dk, Dv);
     if (rc || B == 0) return rc;
     const cudaStream_t st = (cudaStream_t)stream;
-    const float sc = resolve_scale(scale);
-    // the fused short-sequence kernel takes bf16 activations and an fp32 state; other types take the
-    // chunked kernels whatever the lengths
-    const bool short_ok = act_dtype == GDN_DTYPE_BF16 && state_dtype == GDN_DTYPE_FP32;
+    const float sc = resolve_scale(scale > 0.f ? scale : 1.0f / sqrtf((float)Dk));
+    // the fused short-sequence kernel takes bf16 activations, an fp32 state and 128 x 128 heads; other
+    // types and sizes take the chunked kernels whatever the lengths
+    const bool short_ok = act_dtype == GDN_DTYPE_BF16 && state_dtype == GDN_DTYPE_FP32 && Dk == gdn::D &&
+                          Dv == gdn::D;
     if (short_ok && max_seqlen >= 1 && max_seqlen <= GDN_SHORT_MAX)
         return cuda_status(gdn::launch_short(static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(k),
                                              static_cast<const uint16_t *>(v), g, beta, cu_seqlens,
@@ -448,8 +458,9 @@ int gdn_chunk_fwd_typed(const void *q, const void *k, const void *v, const float
                                              static_cast<uint16_t *>(out), static_cast<float *>(final_state), (int)T,
                                              B, Nqk, Nv, max_seqlen, st, update_rule));
 
+    const int32_t Nvs = Nv * dims.m;  // the kernels' head count: 128-column sub-heads
     gdn_workspace_layout_t lay;
-    if ((rc = fill_layout(T, B, Nqk, Nv, &lay, act_dtype))) return rc;
+    if ((rc = fill_layout(T, B, Nqk, Nvs, &lay, act_dtype, Dk))) return rc;
     bool owned = false;
     if (!workspace) {
         if (cudaMallocAsync(&workspace, lay.total, st) != cudaSuccess) return GDN_ERR_CUDA;
@@ -466,19 +477,19 @@ int gdn_chunk_fwd_typed(const void *q, const void *k, const void *v, const float
                    *v16 = static_cast<const uint16_t *>(v);
     cudaError_t e = gdn::launch_chunk_map(cu_seqlens, B, Ti, NC, w, st);
     if (e == cudaSuccess && act_dtype == GDN_DTYPE_FP32 && T > 0) {
-        uint16_t *aq = w.act16, *ak = aq + (size_t)T * Nqk * gdn::D, *av = ak + (size_t)T * Nqk * gdn::D;
+        uint16_t *aq = w.act16, *ak = aq + (size_t)T * Nqk * Dk, *av = ak + (size_t)T * Nqk * Dk;
         e = gdn::launch_act_to_f16(static_cast<const float *>(q), static_cast<const float *>(k),
-                                   static_cast<const float *>(v), aq, ak, av, Ti, Nqk, Nv, w.status, st);
+                                   static_cast<const float *>(v), aq, ak, av, Ti, Nqk, Nvs, w.status, st, dims);
         q16 = aq, k16 = ak, v16 = av;
     }
     const int R = gdn::pipeline_ranges(NC);
     if (e == cudaSuccess && R == 1) {
-        e = gdn::launch_intra(k16, v16, g, beta, eps, Ti, Nqk, Nv, 0, NC, w, st, delta, f16);
+        e = gdn::launch_intra(k16, v16, g, beta, eps, Ti, Nqk, Nvs, 0, NC, w, st, delta, f16, dims);
         if (e == cudaSuccess)
-            e = gdn::launch_state(k16, state_pool, state_indices, final_state, Ti, B, Nqk, Nv, 0, NC, 0, w, st, delta,
-                                  f16, sdt);
+            e = gdn::launch_state(k16, state_pool, state_indices, final_state, Ti, B, Nqk, Nvs, 0, NC, 0, w, st, delta,
+                                  f16, sdt, dims);
         if (e == cudaSuccess)
-            e = gdn::launch_output(q16, k16, g, sc, eps, out, Ti, Nqk, Nv, 0, NC, w, st, delta, f16, odt);
+            e = gdn::launch_output(q16, k16, g, sc, eps, out, Ti, Nqk, Nvs, 0, NC, w, st, delta, f16, odt, dims);
     } else if (e == cudaSuccess) {
         std::lock_guard<std::mutex> guard(g_pipe_lock);
         SideStreams *ss = nullptr;
@@ -493,22 +504,22 @@ int gdn_chunk_fwd_typed(const void *q, const void *k, const void *v, const float
             if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->intra, ev[0], 0);
             if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->state, ev[0], 0);
             for (int r = 0; r < R && e == cudaSuccess; ++r) {
-                e = gdn::launch_intra(k16, v16, g, beta, eps, Ti, Nqk, Nv, c0(r), c1(r) - c0(r), w, ss->intra, delta,
-                                      f16);
+                e = gdn::launch_intra(k16, v16, g, beta, eps, Ti, Nqk, Nvs, c0(r), c1(r) - c0(r), w, ss->intra, delta,
+                                      f16, dims);
                 if (e == cudaSuccess) e = cudaEventRecord(ev[1 + r], ss->intra);
             }
             for (int r = 0; r < R && e == cudaSuccess; ++r) {
                 e = cudaStreamWaitEvent(ss->state, ev[1 + r], 0);
                 if (e == cudaSuccess)
-                    e = gdn::launch_state(k16, state_pool, state_indices, final_state, Ti, B, Nqk, Nv, c0(r), c1(r), r,
-                                          w, ss->state, delta, f16, sdt);
+                    e = gdn::launch_state(k16, state_pool, state_indices, final_state, Ti, B, Nqk, Nvs, c0(r), c1(r), r,
+                                          w, ss->state, delta, f16, sdt, dims);
                 if (e == cudaSuccess) e = cudaEventRecord(ev[1 + R + r], ss->state);
             }
             for (int r = 0; r < R && e == cudaSuccess; ++r) {
                 e = cudaStreamWaitEvent(st, ev[1 + R + r], 0);
                 if (e == cudaSuccess)
-                    e = gdn::launch_output(q16, k16, g, sc, eps, out, Ti, Nqk, Nv, c0(r), c1(r) - c0(r), w, st, delta,
-                                           f16, odt);
+                    e = gdn::launch_output(q16, k16, g, sc, eps, out, Ti, Nqk, Nvs, c0(r), c1(r) - c0(r), w, st, delta,
+                                           f16, odt, dims);
             }
             // join, also after a failed launch, so that nothing of this call runs outside `st` afterwards
             cudaError_t j = cudaEventRecord(ev[1 + 2 * R], ss->intra);

@@ -45,25 +45,35 @@ struct Workspace {
 cudaError_t launch_chunk_map(const int32_t *cu, int B, int T, int NC, const Workspace &ws,
                              cudaStream_t st);
 // intra and output run over chunks [c0, c0 + nc); the state pass over [c_lo, c_hi), range index `range`
+// Head dimensions of the chunked path.  The kernels work on 128 x 128 states; a key dimension Dk of 64
+// reads as 128 with the last 64 columns zero (the TMA copies of q and k fill them, and the state rows
+// past Dk stay zero), and a value dimension Dv = 128 m runs as m sub-heads of 128 columns per v-head,
+// which share the v-head's gate, beta and qk-head (the columns of the state evolve independently).
+// Every kernel's Nv argument then counts sub-heads (Nv m).
+struct Dims {
+    int Dk = 128, Dv = 128, m = 1;
+};
+
 // element types of the chunked path: kActBF16 / kActF16 raw 16-bit q, k, v rows; outputs and states
 // also kTypeF32 (the dtype codes of gdn.h: 0 fp32, 1 bf16, 2 fp16)
 constexpr int kTypeF32 = 0, kTypeBF16 = 1, kTypeF16 = 2;
 cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, const float *g, const uint16_t *beta, float eps, int T,
                          int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st, bool delta = true,
-                         bool f16 = false);
+                         bool f16 = false, Dims dims = Dims());
 cudaError_t launch_state(const uint16_t *k, const void *pool, const int32_t *idx, void *final_state, int T, int B,
                          int Nqk, int Nv, int c_lo, int c_hi, int range, const Workspace &ws, cudaStream_t st,
-                         bool delta = true, bool f16 = false, int state_type = kTypeF32);
+                         bool delta = true, bool f16 = false, int state_type = kTypeF32, Dims dims = Dims());
 cudaError_t launch_output(const uint16_t *q, const uint16_t *k, const float *g, float scale, float eps, void *out,
                           int T, int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st,
-                          bool delta = true, bool f16 = false, int out_type = kTypeBF16);
+                          bool delta = true, bool f16 = false, int out_type = kTypeBF16, Dims dims = Dims());
 // delta == false (launch_intra / launch_state / launch_output): an update rule without the
 // retrieval (U = v, no W or Mk); g == nullptr: a zero gate.  f16: q, k, v are fp16 rows (else bf16);
 // state_type: the pool's and final state's type (fp32, bf16 or fp16); out_type: out's type.
 // fp32 q, k, v rows rounded to fp16 (round to nearest even) into act16 [T][Nqk | Nqk | Nv][128]
 // (the workspace's act16 region), before the fp16 kernels run
 cudaError_t launch_act_to_f16(const float *q, const float *k, const float *v, uint16_t *q16, uint16_t *k16,
-                              uint16_t *v16, int T, int Nqk, int Nv, int32_t *status, cudaStream_t st);
+                              uint16_t *v16, int T, int Nqk, int Nv, int32_t *status, cudaStream_t st,
+                              Dims dims = Dims());
 // Fused short-sequence kernel: sequence b starts from pool[idx ? idx[b] : b] (or
 // zero without a pool) and ends in final_state[b].
 cudaError_t launch_short(const uint16_t *q, const uint16_t *k, const uint16_t *v, const float *g,

@@ -27,9 +27,10 @@ __global__ void __launch_bounds__(256) act_to_f16_kernel(const float4 *__restric
 }
 
 cudaError_t launch_act_to_f16(const float *q, const float *k, const float *v, uint16_t *q16, uint16_t *k16,
-                              uint16_t *v16, int T, int Nqk, int Nv, int32_t *status, cudaStream_t st)
+                              uint16_t *v16, int T, int Nqk, int Nv, int32_t *status, cudaStream_t st, Dims dims)
 {
-    const size_t nqk = (size_t)T * Nqk * D / 8, nv = (size_t)T * Nv * D / 8;
+    // q, k [T][Nqk][Dk]; v [T][Nv][128] with Nv counting 128-column sub-heads
+    const size_t nqk = (size_t)T * Nqk * dims.Dk / 8, nv = (size_t)T * Nv * D / 8;
     const struct { const float *s; uint16_t *d; size_t n8; } parts[3] = {{q, q16, nqk}, {k, k16, nqk}, {v, v16, nv}};
     for (const auto &p : parts) {
         if (p.n8 == 0) continue;

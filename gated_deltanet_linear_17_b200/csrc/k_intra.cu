@@ -161,8 +161,11 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     const __grid_constant__ CUtensorMap tm_mk, const float *__restrict__ g, const uint16_t *__restrict__ beta,
     float eps, int T, int Nqk, int Nv, const int4 *__restrict__ info, float *__restrict__ rk_out,
     float *__restrict__ gcum_out, float *__restrict__ betaf_out, float *__restrict__ fa, int32_t *__restrict__ status,
-    int c0, int nc, int delta)
+    int c0, int nc, int delta, int m)
 {
+    // Nv counts 128-column sub-heads: a v-head of Dv = 128 m columns is m sub-heads that share its gate,
+    // beta and qk-head; g and beta are indexed by the v-head, Nv / m of them per token
+    const int Nvr = Nv / m;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
     const uint32_t sbase = smem_addr(smem);
@@ -201,8 +204,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     // once; a load is issued only after the barrier's previous phase has been waited on.
     auto load_k = [&](uint32_t dst, int hq_, int t0_) {
         tma::expect_tx(bar_ld, 32768);
-        tma::load_2d(sbase + dst, &tm_k, hq_ * D, t0_, bar_ld);
-        tma::load_2d(sbase + dst + 16384, &tm_k, hq_ * D + 64, t0_, bar_ld);
+        tma::load_3d(sbase + dst, &tm_k, 0, hq_, t0_, bar_ld);  // columns past Dk (= 64) read as zero
+        tma::load_3d(sbase + dst + 16384, &tm_k, 64, hq_, t0_, bar_ld);
     };
     auto load_v = [&](int h_, int t0_) {
         tma::expect_tx(bar_v, 32768);
@@ -216,8 +219,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
     // this thread's gate and beta of the current item (threads 0..127, zero past the chunk)
     float xg = 0.f, xb = 0.f;
     if (tid < 128 && tid < ci.len) {  // g == nullptr: a zero gate; beta == nullptr: not read (no retrieval)
-        xg = g ? g[(size_t)(ci.start + tid) * Nv + h] : 0.f;
-        xb = beta ? bf2f(beta[(size_t)(ci.start + tid) * Nv + h]) : 0.f;
+        xg = g ? g[(size_t)(ci.start + tid) * Nvr + h / m] : 0.f;
+        xb = beta ? bf2f(beta[(size_t)(ci.start + tid) * Nvr + h / m]) : 0.f;
     }
     bool ok = true;
     float vmax = 0.f;  // largest magnitude of the fp16 U tiles (range check; a NaN is kept)
@@ -256,8 +259,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
             const int nh = nit / nc;
             const ChunkInfo nci = load_chunk(info, c0 + nit % nc);
             if (tid < 128 && tid < nci.len) {
-                ng = g ? g[(size_t)(nci.start + tid) * Nv + nh] : 0.f;
-                nb = beta ? bf2f(beta[(size_t)(nci.start + tid) * Nv + nh]) : 0.f;
+                ng = g ? g[(size_t)(nci.start + tid) * Nvr + nh / m] : 0.f;
+                nb = beta ? bf2f(beta[(size_t)(nci.start + tid) * Nvr + nh / m]) : 0.f;
             }
         }
         // chunk-local cumulative gate and beta while the rows load
@@ -669,7 +672,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
 }
 
 cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, const float *g, const uint16_t *beta, float eps, int T,
-                         int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st, bool delta, bool f16)
+                         int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st, bool delta, bool f16,
+                         Dims dims)
 {
     if (nc <= 0 || T == 0) return cudaSuccess;
     if (c0 < 0 || c0 + nc > ws.NC) return cudaErrorInvalidValue;
@@ -677,8 +681,7 @@ cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, const float *g, c
     if ((uint64_t)T >= (1ull << 31) || trows >= (1ull << 31)) return cudaErrorInvalidValue;
     CUtensorMap m_k, m_v, m_u, m_w, m_mk;
     const auto AT = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    cudaError_t e = tma::map2d(&m_k, AT, k, (uint64_t)Nqk * D, (uint64_t)T, (uint64_t)Nqk * D * 2, 64, 128,
-                               CU_TENSOR_MAP_SWIZZLE_128B);
+    cudaError_t e = tma::map_heads(&m_k, AT, k, (uint64_t)dims.Dk, (uint64_t)Nqk, (uint64_t)T, 128);
     if (e == cudaSuccess)
         e = tma::map2d(&m_v, AT, v, (uint64_t)Nv * D, (uint64_t)T, (uint64_t)Nv * D * 2, 64, 128,
                        CU_TENSOR_MAP_SWIZZLE_128B);
@@ -697,7 +700,8 @@ cudaError_t launch_intra(const uint16_t *k, const uint16_t *v, const float *g, c
     const int per = delta ? kIntraItemsPerCta : 1;
     const int grid = (items + per - 1) / per;
     kern<<<grid, kIntraThreads, kIntraSmem, st>>>(m_k, m_v, m_u, m_w, m_mk, g, beta, eps, T, Nqk, Nv, ws.chunk_info,
-                                                   ws.rk, ws.gcum, ws.betaf, ws.fa, ws.status, c0, nc, delta ? 1 : 0);
+                                                   ws.rk, ws.gcum, ws.betaf, ws.fa, ws.status, c0, nc, delta ? 1 : 0,
+                                                   dims.m);
     return cudaGetLastError();
 }
 

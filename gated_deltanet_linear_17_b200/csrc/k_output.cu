@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sc,
     const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_out, void *__restrict__ out,
     const float *__restrict__ g, float scale, float eps, int T, int Nqk, int Nv, const int4 *__restrict__ info,
-    float *__restrict__ rq_out, int32_t *__restrict__ status, int c0, int delta)
+    float *__restrict__ rq_out, int32_t *__restrict__ status, int c0, int delta, int m)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
@@ -104,10 +104,11 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
     __syncthreads();
     if (tid == 0) {  // q and k (64 KiB) on bar_ld, W (32 KiB) on bar_w
         tma::expect_tx(bar_ld, 65536);
-        tma::load_2d(sbase + OO_Q, &tm_q, hq * D, t0, bar_ld);
-        tma::load_2d(sbase + OO_Q + 16384, &tm_q, hq * D + 64, t0, bar_ld);
-        tma::load_2d(sbase + OO_K, &tm_k, hq * D, t0, bar_ld);
-        tma::load_2d(sbase + OO_K + 16384, &tm_k, hq * D + 64, t0, bar_ld);
+        // q and k of the qk-head (columns past Dk = 64 read as zero)
+        tma::load_3d(sbase + OO_Q, &tm_q, 0, hq, t0, bar_ld);
+        tma::load_3d(sbase + OO_Q + 16384, &tm_q, 64, hq, t0, bar_ld);
+        tma::load_3d(sbase + OO_K, &tm_k, 0, hq, t0, bar_ld);
+        tma::load_3d(sbase + OO_K + 16384, &tm_k, 64, hq, t0, bar_ld);
         if (delta) {  // W enters only the rules with the retrieval
             tma::expect_tx(bar_w, 32768);
             tma::load_2d(sbase + OO_X, &tm_w, 0, trow, bar_w);
@@ -115,7 +116,8 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
         }
     }
     // chunk-local cumulative gate while the rows load
-    chunk_gamma(g, Nv, h, t0, n, gam, reinterpret_cast<float *>(smem + OO_BAR + 32));
+    // the gate of the v-head (Nv counts sub-heads of 128 columns, m per v-head)
+    chunk_gamma(g, Nv / m, h / m, t0, n, gam, reinterpret_cast<float *>(smem + OO_BAR + 32));
     // S_c, then U, as MN-major [128][128] tiles (two 64-column halves), each on its own barrier (thread 0)
     bool s_issued = false, u_issued = false;
     auto load_tile = [&](uint32_t dst, const CUtensorMap *m, uint32_t bar) {
@@ -400,7 +402,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
 
 cudaError_t launch_output(const uint16_t *q, const uint16_t *k, const float *g, float scale, float eps, void *out,
                           int T, int Nqk, int Nv, int c0, int nc, const Workspace &ws, cudaStream_t st, bool delta,
-                          bool f16, int out_type)
+                          bool f16, int out_type, Dims dims)
 {
     if (nc <= 0 || T == 0) return cudaSuccess;
     if (c0 < 0 || c0 + nc > ws.NC) return cudaErrorInvalidValue;
@@ -410,8 +412,8 @@ cudaError_t launch_output(const uint16_t *q, const uint16_t *k, const float *g, 
     const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
     CUtensorMap m_q, m_k, m_w, m_sc, m_u, m_out;
     const auto AT = f16 ? HF : BF;
-    cudaError_t e = tma::map2d(&m_q, AT, q, (uint64_t)Nqk * D, (uint64_t)T, (uint64_t)Nqk * D * 2, 64, 128, SW);
-    if (e == cudaSuccess) e = tma::map2d(&m_k, AT, k, (uint64_t)Nqk * D, (uint64_t)T, (uint64_t)Nqk * D * 2, 64, 128, SW);
+    cudaError_t e = tma::map_heads(&m_q, AT, q, (uint64_t)dims.Dk, (uint64_t)Nqk, (uint64_t)T, 128);
+    if (e == cudaSuccess) e = tma::map_heads(&m_k, AT, k, (uint64_t)dims.Dk, (uint64_t)Nqk, (uint64_t)T, 128);
     if (e == cudaSuccess) e = tma::map2d(&m_w, HF, ws.W, D, trows, D * 2, 64, 128, SW);
     if (e == cudaSuccess) e = tma::map2d(&m_sc, HF, ws.Sc, D, trows, D * 2, 64, 128, SW);
     if (e == cudaSuccess) e = tma::map2d(&m_u, HF, ws.U, D, trows, D * 2, 64, 128, SW);
@@ -429,7 +431,7 @@ cudaError_t launch_output(const uint16_t *q, const uint16_t *k, const float *g, 
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
     if (e != cudaSuccess) return e;
     kern<<<dim3(nc, Nv), kOutThreads, kOutSmem, st>>>(m_q, m_k, m_w, m_sc, m_u, m_out, out, g, scale, eps, T, Nqk, Nv,
-                                                       ws.chunk_info, ws.rq, ws.status, c0, delta ? 1 : 0);
+                                                       ws.chunk_info, ws.rq, ws.status, c0, delta ? 1 : 0, dims.m);
     return cudaGetLastError();
 }
 

@@ -88,7 +88,8 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
     const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_sc,
     const void *__restrict__ pool, const int32_t *__restrict__ idx, void *__restrict__ final_state, int Nqk,
     int Nv, const int4 *__restrict__ info, const int32_t *__restrict__ seq_chunk0, const float *__restrict__ fa,
-    int32_t *__restrict__ status, int c_lo, int c_hi, int range, float *__restrict__ carry, int delta)
+    int32_t *__restrict__ status, int c_lo, int c_hi, int range, float *__restrict__ carry, int delta, int Dk, int Dv,
+    int m)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
@@ -137,8 +138,8 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
             tma::load_2d(base + SG_MK, &tm_mk, 0, trow, full);
             tma::load_2d(base + SG_MK + 16384, &tm_mk, 64, trow, full);
         }
-        tma::load_2d(base + SG_K, &tm_k, hq * D, cstart, full);
-        tma::load_2d(base + SG_K + 16384, &tm_k, hq * D + 64, cstart, full);
+        tma::load_3d(base + SG_K, &tm_k, 0, hq, cstart, full);  // columns past Dk (= 64) read as zero
+        tma::load_3d(base + SG_K + 16384, &tm_k, 64, hq, cstart, full);
         tma::load_2d(base + SG_U, &tm_u, col0, trow, full);
         tma::load_1d(sbase + OFF_F + st * kFaStride * 4, fa + (size_t)(c * Nv + h) * kFaStride, kFaStride * 4,
                      full);
@@ -178,12 +179,18 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
     };
 
     // initial state: this thread's 32 values
+    // this thread's 32 values: in a carry slot [Nv sub-heads][128][128], and in a pool slot or a final
+    // state [Nv / m v-heads][Dk][Dv] (sub-head h is columns 128 (h % m) .. of v-head h / m); state rows
+    // past Dk stay zero and are neither read nor written
     float s[32];
-    const size_t s_off = ((size_t)h * D + row) * D + col0 + cbase;  // this thread's 32 values in a state
-    if (epi && (from_carry || (pool && SDT == kTypeF32))) {
-        const float *base = from_carry ? carry + (size_t)(range - 1) * Nv * D * D
-                                       : static_cast<const float *>(pool) + (size_t)(idx ? idx[b] : b) * Nv * D * D;
-        const float4 *src = reinterpret_cast<const float4 *>(base + s_off);
+    const size_t s_off = ((size_t)h * D + row) * D + col0 + cbase;
+    const size_t p_off = ((size_t)(h / m) * Dk + row) * Dv + (size_t)(h % m) * D + col0 + cbase;
+    const size_t p_slot = (size_t)(Nv / m) * Dk * Dv;  // elements of a pool slot
+    const bool in_dk = row < Dk;
+    if (epi && (from_carry || (pool && in_dk && SDT == kTypeF32))) {
+        const float *src4 = from_carry ? carry + (size_t)(range - 1) * Nv * D * D + s_off
+                                       : static_cast<const float *>(pool) + (size_t)(idx ? idx[b] : b) * p_slot + p_off;
+        const float4 *src = reinterpret_cast<const float4 *>(src4);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const float4 v4 = src[j];
@@ -192,9 +199,9 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
             s[4 * j + 2] = v4.z;
             s[4 * j + 3] = v4.w;
         }
-    } else if (epi && pool) {  // a 16-bit pool, widened exactly
+    } else if (epi && pool && in_dk) {  // a 16-bit pool, widened exactly
         const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(pool) +
-                                                           (size_t)(idx ? idx[b] : b) * Nv * D * D + s_off);
+                                                           (size_t)(idx ? idx[b] : b) * p_slot + p_off);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const uint4 w = src[j];
@@ -339,14 +346,14 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
     if (epi && __any_sync(0xffffffffu, out_of_fp16(vmax)) && lane == 0) atomicOr(status + 3, GDN_DEV_RANGE_STATE);
     if (!ok) {
         if (tid == 0) atomicOr(status + 2, GDN_DEV_WAIT_STATE);
-    } else if (epi && (to_carry || (final_state && SDT == kTypeF32))) {
-        float *base = to_carry ? carry + (size_t)range * Nv * D * D
-                               : static_cast<float *>(final_state) + (size_t)b * Nv * D * D;
-        float4 *dst = reinterpret_cast<float4 *>(base + s_off);
+    } else if (epi && (to_carry || (final_state && in_dk && SDT == kTypeF32))) {
+        float *dst4 = to_carry ? carry + (size_t)range * Nv * D * D + s_off
+                               : static_cast<float *>(final_state) + (size_t)b * p_slot + p_off;
+        float4 *dst = reinterpret_cast<float4 *>(dst4);
 #pragma unroll
         for (int j = 0; j < 8; ++j) dst[j] = make_float4(s[4 * j], s[4 * j + 1], s[4 * j + 2], s[4 * j + 3]);
-    } else if (epi && final_state) {  // a 16-bit final state, rounded to nearest even
-        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(final_state) + (size_t)b * Nv * D * D + s_off);
+    } else if (epi && final_state && in_dk) {  // a 16-bit final state, rounded to nearest even
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(final_state) + (size_t)b * p_slot + p_off);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const float *v8 = s + 8 * j;
@@ -362,7 +369,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
 
 cudaError_t launch_state(const uint16_t *k, const void *pool, const int32_t *idx, void *final_state, int T, int B,
                          int Nqk, int Nv, int c_lo, int c_hi, int range, const Workspace &ws, cudaStream_t st,
-                         bool delta, bool f16, int state_type)
+                         bool delta, bool f16, int state_type, Dims dims)
 {
     if (B == 0) return cudaSuccess;
     if (range < 0 || range >= kMaxRanges || c_lo < 0 || c_hi < c_lo) return cudaErrorInvalidValue;
@@ -376,9 +383,9 @@ cudaError_t launch_state(const uint16_t *k, const void *pool, const int32_t *idx
     cudaError_t e = tma::map2d(&m_mk, HF, ws.Mk, D, rows, D * 2, 64, 128, SW);
     if (e == cudaSuccess) {
         if (T > 0)
-            e = tma::map2d(&m_k, f16 ? HF : BF, k, (uint64_t)Nqk * D, (uint64_t)T, (uint64_t)Nqk * D * 2, 64, 128, SW);
+            e = tma::map_heads(&m_k, f16 ? HF : BF, k, (uint64_t)dims.Dk, (uint64_t)Nqk, (uint64_t)T, 128);
         else  // no chunk exists, so the map is never used
-            e = tma::map2d(&m_k, BF, ws.Mk, D, rows, D * 2, 64, 128, SW);
+            e = tma::map_heads(&m_k, BF, ws.Mk, D, 1, rows, 128);
     }
     if (e == cudaSuccess) e = tma::map2d(&m_u, HF, ws.U, D, rows, D * 2, DVT, 128, SW);
     if (e == cudaSuccess) e = tma::map2d(&m_sc, HF, ws.Sc, D, rows, D * 2, DVT, 128, SW);
@@ -390,7 +397,7 @@ cudaError_t launch_state(const uint16_t *k, const void *pool, const int32_t *idx
     if (e != cudaSuccess) return e;
     kern<<<dim3(B, Nv, D / DVT), kStateThreads, kStateSmem, st>>>(
         m_mk, m_k, m_u, m_sc, pool, idx, final_state, Nqk, Nv, ws.chunk_info, ws.seq_chunk0, ws.fa, ws.status, c_lo,
-        c_hi, range, ws.carry, delta ? 1 : 0);
+        c_hi, range, ws.carry, delta ? 1 : 0, dims.Dk, dims.Dv, dims.m);
     return cudaGetLastError();
 }
 

@@ -24,6 +24,13 @@ namespace tma {
 cudaError_t map2d(CUtensorMap *m, CUtensorMapDataType dtype, const void *base, uint64_t cols, uint64_t rows,
                   uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle);
 
+// Host: a 3-D tiled map of rows of `heads` heads of `dim` elements (a [rows][heads][dim] tensor of
+// 16-bit elements, row stride heads * dim elements), box of 64 elements x 1 head x box_rows rows with
+// the 128-byte swizzle: box (x, head, row) lands as box_rows rows of 64 elements, the layout of one K
+// half.  A head narrower than 128 elements reads its second half (x = 64) as zeros past dim.
+cudaError_t map_heads(CUtensorMap *m, CUtensorMapDataType dtype, const void *base, uint64_t dim, uint64_t heads,
+                      uint64_t rows, uint32_t box_rows);
+
 __device__ __forceinline__ void prefetch_map(const CUtensorMap *m)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -42,6 +49,16 @@ __device__ __forceinline__ void load_2d(uint32_t dst, const CUtensorMap *m, int 
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
             "r"(dst),
         "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(mbar)
+        : "memory");
+}
+
+// box at (x, head, y) of a 3-D map (map_heads) -> shared memory at dst; completes on mbar
+__device__ __forceinline__ void load_3d(uint32_t dst, const CUtensorMap *m, int x, int head, int y, uint32_t mbar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(head), "r"(y), "r"(mbar)
         : "memory");
 }
 

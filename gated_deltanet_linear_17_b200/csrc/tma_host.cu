@@ -34,5 +34,20 @@ cudaError_t map2d(CUtensorMap *m, CUtensorMapDataType dtype, const void *base, u
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t map_heads(CUtensorMap *m, CUtensorMapDataType dtype, const void *base, uint64_t dim, uint64_t heads,
+                      uint64_t rows, uint32_t box_rows)
+{
+    auto fn = encoder();
+    if (!fn || !base || dim == 0 || heads == 0 || rows == 0) return cudaErrorInvalidValue;
+    const cuuint64_t dims[3] = {dim, heads, rows};
+    const cuuint64_t strides[2] = {dim * 2, heads * dim * 2};  // bytes; 16-bit elements
+    const cuuint32_t box[3] = {64, 1, box_rows};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, dtype, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace tma
 }  // namespace gdn

@@ -233,32 +233,44 @@ int gdn_chunk_fwd_rule(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
  * gdn_chunk_fwd_typed -- gdn_chunk_fwd_rule with the element types of the page
  * "com.microsoft.LinearAttention" ("Activations and state may independently
  * use float16 or float32"), beside the decode page's bf16 activations and bf16
- * state; gdn_chunk_fwd_rule is this call with bf16 activations and an fp32
- * state.
+ * state, and with other head dimensions (the decode page's example has
+ * Dk = 64, Dv = 512); gdn_chunk_fwd_rule is this call with bf16 activations,
+ * an fp32 state and Dk = Dv = 128.
  *
  *   act_dtype     GDN_DTYPE_BF16, GDN_DTYPE_FP16 or GDN_DTYPE_FP32: the type of
- *                 q, k, v and out (each laid out as for gdn_chunk_fwd)
+ *                 q, k, v and out
  *   state_dtype   GDN_DTYPE_FP32, GDN_DTYPE_FP16 or GDN_DTYPE_BF16: the type of
  *                 state_pool and final_state (the state itself is carried in
  *                 fp32 on the chip; a 16-bit pool is widened exactly, a 16-bit
  *                 final state rounded to nearest even)
+ *   Dk, Dv        head dimensions: Dk 64 or 128, Dv 128, 256, 384 or 512, with
+ *                 Nv * Dv / 128 <= 256 (else GDN_ERR_UNSUPPORTED).  Layouts:
+ *                 q, k [T, Nqk, Dk]; v, out [T, Nv, Dv]; state_pool [P, Nv, Dk, Dv];
+ *                 final_state [B, Nv, Dk, Dv].  The kernels compute on 128 x 128
+ *                 states: Dk = 64 runs as 128 with the extra key columns zero
+ *                 (exact, at the cost of Dk = 128), and a head of Dv = 128 m runs
+ *                 as m heads of 128 value columns that share its q, k, gate and
+ *                 beta (the columns of the state evolve independently), so the
+ *                 work of T, W and Mk is repeated m times.  scale <= 0 selects
+ *                 1/sqrt(Dk).
  *   g, beta       fp32 and bf16 as for gdn_chunk_fwd, in every combination
- *   workspace     >= gdn_chunk_fwd_typed_workspace_bytes(T, B, Nqk, Nv, act_dtype),
- *                 or NULL (allocated and freed stream-ordered)
+ *   workspace     >= gdn_chunk_fwd_typed_workspace_bytes(T, B, Nqk, Nv, act_dtype,
+ *                 Dk, Dv), or NULL (allocated and freed stream-ordered)
  * bf16 and fp16 rows enter the tensor core as they are (both exact operands);
  * fp32 q, k and v are first rounded to fp16 in the workspace (11 significant
  * bits; an element beyond +-65504 sets GDN_DEV_RANGE_INPUT, see "Device
  * status").  The fused short-sequence kernel serves bf16 activations with an
- * fp32 state; other types run the chunked kernels for any max_seqlen.  Every
- * other argument, limit and error as for gdn_chunk_fwd_rule; an unknown type
- * code is GDN_ERR_BAD_SHAPE.
+ * fp32 state and Dk = Dv = 128; everything else runs the chunked kernels for
+ * any max_seqlen.  Every other argument, limit and error as for
+ * gdn_chunk_fwd_rule; an unknown type code is GDN_ERR_BAD_SHAPE.
  */
-size_t gdn_chunk_fwd_typed_workspace_bytes(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t act_dtype);
+size_t gdn_chunk_fwd_typed_workspace_bytes(int64_t T, int32_t B, int32_t Nqk, int32_t Nv, int32_t act_dtype,
+                                           int32_t Dk, int32_t Dv);
 int gdn_chunk_fwd_typed(const void *q, const void *k, const void *v, const float *g, const uint16_t *beta,
                         const int32_t *cu_seqlens, const void *state_pool, const int32_t *state_indices, float scale,
                         float eps, void *out, void *final_state, int64_t T, int32_t B, int32_t Nqk, int32_t Nv,
-                        int32_t P, int32_t update_rule, int32_t act_dtype, int32_t state_dtype, int32_t max_seqlen,
-                        void *workspace, size_t workspace_bytes, void *stream);
+                        int32_t P, int32_t update_rule, int32_t act_dtype, int32_t state_dtype, int32_t Dk, int32_t Dv,
+                        int32_t max_seqlen, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd for callers that cannot allocate

@@ -256,12 +256,12 @@ def test_typed_entry_argument_errors(lib):
 
     def call(**over):
         a = dict(q=M, k=2 * M, v=3 * M, g=4 * M, beta=5 * M, cu=6 * M, pool=None, out=7 * M, fin=None, T=8, B=1,
-                 Nqk=2, Nv=4, P=0, rule=0, act=2, sdt=0, ws=None, wsb=0)
+                 Nqk=2, Nv=4, P=0, rule=0, act=2, sdt=0, Dk=128, Dv=128, ws=None, wsb=0)
         a.update(over)
         return lib.gdn_chunk_fwd_typed(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["g"]), vp(a["beta"]), vp(a["cu"]),
                                        vp(a["pool"]), None, 0.0, 1e-6, vp(a["out"]), vp(a["fin"]), a["T"], a["B"],
-                                       a["Nqk"], a["Nv"], a["P"], a["rule"], a["act"], a["sdt"], 0, vp(a["ws"]),
-                                       a["wsb"], None)
+                                       a["Nqk"], a["Nv"], a["P"], a["rule"], a["act"], a["sdt"], a["Dk"], a["Dv"], 0,
+                                       vp(a["ws"]), a["wsb"], None)
     assert call(act=3) == B.GDN_ERR_BAD_SHAPE and call(sdt=-1) == B.GDN_ERR_BAD_SHAPE
     assert call(rule=4) == B.GDN_ERR_BAD_SHAPE
     assert call(Nv=3) == B.GDN_ERR_BAD_SHAPE
@@ -270,6 +270,15 @@ def test_typed_entry_argument_errors(lib):
     assert call(act=0, out=3 * M + 8 * 4 * 128 * 2) == B.GDN_ERR_OVERLAP
     assert call(ws=8 << 20, wsb=10) == B.GDN_ERR_WORKSPACE
     # the fp32-activation workspace holds their fp16 copies on top of the 16-bit one
-    w16 = lib.gdn_chunk_fwd_typed_workspace_bytes(4096, 2, 4, 8, 2)
-    w32 = lib.gdn_chunk_fwd_typed_workspace_bytes(4096, 2, 4, 8, 0)
+    w16 = lib.gdn_chunk_fwd_typed_workspace_bytes(4096, 2, 4, 8, 2, 128, 128)
+    w32 = lib.gdn_chunk_fwd_typed_workspace_bytes(4096, 2, 4, 8, 0, 128, 128)
     assert w16 == gdn.workspace_bytes(4096, 2, 4, 8) and w32 >= w16 + (2 * 4 + 8) * 4096 * 128 * 2
+    # head dimensions: Dv = 512 runs as four 128-column sub-heads per v-head; Dk 64 or 128 only
+    assert lib.gdn_chunk_fwd_typed_workspace_bytes(4096, 2, 4, 8, 2, 64, 512) == gdn.workspace_bytes(4096, 2, 4, 32)
+    assert lib.gdn_chunk_fwd_typed_workspace_bytes(4096, 2, 4, 8, 2, 96, 128) == 0
+    assert lib.gdn_chunk_fwd_typed_workspace_bytes(4096, 2, 4, 8, 2, 128, 192) == 0
+    assert call(Dk=96) == B.GDN_ERR_UNSUPPORTED and call(Dv=640) == B.GDN_ERR_UNSUPPORTED
+    assert call(Dv=192) == B.GDN_ERR_UNSUPPORTED and call(Dk=0) == B.GDN_ERR_BAD_SHAPE
+    assert call(Nqk=64, Nv=128, Dv=512) == B.GDN_ERR_UNSUPPORTED  # 512 sub-heads of 128 columns
+    # out of a Dv = 512 call (4 bytes per fp32 element) overlaps v when 64 KiB apart
+    assert call(act=0, Dk=64, Dv=512, out=3 * M + 8 * 4 * 512 * 2) == B.GDN_ERR_OVERLAP

@@ -1,6 +1,7 @@
 """GPU parity of the chunked path with the LinearAttention page's element types (gdn_chunk_fwd_typed):
 activations (q, k, v, out) fp16 or fp32 and the state (pool, final state) fp16 or fp32, beside the
-decode page's bf16 activations and bf16 state, against the fp64 oracle.
+decode page's bf16 activations and bf16 state, and with head dimensions other than 128 (Dk 64 or 128,
+Dv up to 512), against the fp64 oracle.
 
 The activations carry bits beyond bf16 (a small fp32 perturbation of the seeded values), so a path that
 narrowed them to bf16 would show; fp16 rows enter the tensor core exactly, fp32 rows are rounded to
@@ -38,7 +39,7 @@ def _oracle(q, k, v, inp, pool, rule="gated_delta"):
     P = pool.shape[0] if pool is not None else inp.B
     idx = inp.state_indices if inp.state_indices is not None else torch.arange(inp.B, dtype=torch.int32)
     slots = torch.cat([torch.full((n,), int(idx[b])) for b, n in enumerate(inp.seqlens)]).numpy().astype("int32")
-    p0 = pool if pool is not None else torch.zeros(P, inp.Nv, 128, 128)
+    p0 = pool if pool is not None else torch.zeros(P, inp.Nv, inp.q.shape[2], inp.v.shape[2])
     ro, rpool = recurrent_pool(q, k, v, inp.g, inp.beta, inp.cu_seqlens, p0, slots, scale=inp.scale, eps=inp.eps,
                                rule=rule)
     return ro, rpool[idx.long().numpy()]
@@ -95,10 +96,43 @@ def test_fp32_activation_beyond_fp16_range_is_reported():
     q, k, v = _widen(inp, F32, 102)
     v[5, 1, 7] = 1.0e6  # cannot be held in fp16
     d = inp.to(DEV)
-    ws = torch.empty(gdn.lib().gdn_chunk_fwd_typed_workspace_bytes(d.T, d.B, d.Nqk, d.Nv, 0), dtype=torch.uint8,
+    ws = torch.empty(gdn.lib().gdn_chunk_fwd_typed_workspace_bytes(d.T, d.B, d.Nqk, d.Nv, 0, 128, 128), dtype=torch.uint8,
                      device=DEV)
     gdn.chunk_fwd(q.to(DEV), k.to(DEV), v.to(DEV), d.g, d.beta, d.cu_seqlens, scale=d.scale, eps=d.eps,
                   workspace=ws)
     words = gdn.read_status(ws)
     assert words[3] & 8, words
     assert "an fp32 activation beyond the fp16 range" in gdn.decode_status(words)
+
+
+@pytest.mark.parametrize("Dk,Dv,act,state", [(64, 512, BF16, F32), (128, 256, BF16, F32), (64, 128, BF16, F32),
+                                             (64, 256, F16, BF16), (128, 384, F32, F16)])
+def test_head_dimensions_chunked(Dk, Dv, act, state):
+    """Dk != Dv in the chunked path (the decode page's example has Dk = 64, Dv = 512): Dk = 64 runs as 128
+    with zero key columns, Dv = 128 m as m sub-heads per v-head sharing q, k, gate and beta."""
+    inp = inputs.make([300, 129, 1, 700, 0, 64], Nqk=2, Nv=4, state=("normal", 0.02, 8, "perm"), seed=103,
+                      Dk=Dk, Dv=Dv)
+    q, k, v = _widen(inp, act, 104) if act != BF16 else (inp.q, inp.k, inp.v)
+    pool = inp.state_pool.to(state)
+    ro, rf = _oracle(q, k, v, inp, pool)
+    d = inp.to(DEV)
+    out, fin = gdn.chunk_fwd(q.to(DEV), k.to(DEV), v.to(DEV), d.g, d.beta, d.cu_seqlens, pool.to(DEV),
+                             d.state_indices, scale=d.scale, eps=d.eps, check_status=True)
+    torch.cuda.synchronize()
+    assert out.shape == (inp.T, 4, Dv) and fin.shape == (inp.B, 4, Dk, Dv)
+    assert_close(out, ro, f"Dk={Dk} Dv={Dv} {act}/{state} out")
+    assert_close(fin, rf, f"Dk={Dk} Dv={Dv} {act}/{state} final_state")
+
+
+def test_head_dimensions_pipelined_and_rules():
+    """Dk = 64, Dv = 512 over two pipelined chunk ranges (a carried state per sub-head), and the gated rule."""
+    inp = inputs.make([3000, 1500, 7], Nqk=1, Nv=2, state=("normal", 0.02, 3, "perm"), seed=105, Dk=64, Dv=512)
+    d = inp.to(DEV)
+    assert gdn.pipeline_ranges(d.T, d.B, d.Nqk, d.Nv * 4) == 2
+    for rule in ("gated_delta", "gated"):
+        ro, rf = _oracle(inp.q, inp.k, inp.v, inp, inp.state_pool, rule)
+        out, fin = gdn.chunk_fwd(d.q, d.k, d.v, d.g, d.beta, d.cu_seqlens, d.state_pool, d.state_indices,
+                                 scale=d.scale, eps=d.eps, update_rule=rule)
+        torch.cuda.synchronize()
+        assert_close(out, ro, f"Dk=64 Dv=512 {rule} out")
+        assert_close(fin, rf, f"Dk=64 Dv=512 {rule} final_state")
