@@ -25,9 +25,10 @@
 //               staged its operand, Kt of chunk c+1 = K^T [Ub_hi | Ub_lo]
 //               (M=128, N=128, K=128, k's type; A = the raw k tile read MN-major)
 //               into the other accumulator.
-//   data warp:  a TMA store of S_c (fp16) to Sc; once chunk c's products have
-//               completed, TMA loads of chunk c+2 (Mk, the raw k rows, the U
-//               slice and the factors) into the freed stage.
+//   data warp:  a TMA store of S_c (fp16) to Sc; TMA loads of chunk c+2 into
+//               the stage chunk c leaves: its raw k rows, U slice and factors
+//               as soon as Kt of chunk c has completed (early in the chunk),
+//               its Mk once the chain product of chunk c has.
 //   epilogue:   stage Ub of chunk c+1 (hi over its U slice, lo beside it);
 //               wait for the products of chunk c; S_{c+1} = e^{g_last} S_c +
 //               D_hi + D_lo, whose fp16 copy is the next B operand (the other
@@ -61,11 +62,11 @@ constexpr int SG_K = 32768;    // bf16 k [L][Dk] in two 64-column blocks (MN-maj
 constexpr int SG_U = 65536;    // fp16 U slice [L][64] -> bf16 Ub_hi (MN-major B, first 64 columns)
 constexpr int SG_UL = 81920;   // bf16 Ub_lo [L][64] (MN-major B, last 64 columns)
 constexpr int kStage = 98304;  // a multiple of 1024
-constexpr uint32_t kStageTx = 32768 + 32768 + 16384 + kFaStride * 4;  // bytes per stage fill
+constexpr uint32_t kKUTx = 32768 + 16384 + kFaStride * 4;  // bytes of a stage's k / U / factor fill
 constexpr int OFF_S = 2 * kStage;            // 2 x fp16 S [Dk][64] (MN-major B)
 constexpr int OFF_F = OFF_S + 2 * 16384;     // 2 x fp32 factors: f_t (t < 128), e^{g_last} at 128
-constexpr int OFF_BAR = OFF_F + 2 * kFaStride * 4;  // full[2], chain, drain mbarriers; TMEM address slot
-constexpr int kStateSmem = OFF_BAR + 64 + 1024;     // + alignment slack
+constexpr int OFF_BAR = OFF_F + 2 * kFaStride * 4;  // mbarriers; TMEM address slot
+constexpr int kStateSmem = OFF_BAR + 96 + 1024;     // + alignment slack
 constexpr int kTmemCols = 256;  // two accumulators [D_hi | D_lo], D_hi = Kt_hi - Mk S
 
 // named barrier 1: the epilogue warps arrive once Ub is staged, the issue warp waits
@@ -114,36 +115,40 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
     const int seq_t1 = c_begin < c_end ? info[c_end - 1].y + info[c_end - 1].z : 0;
     auto chunk_len = [&](int c) { return min(L, seq_t1 - (seq_t0 + (c - c_begin) * L)); };
 
-    const uint32_t bar_full = sbase + OFF_BAR;  // + 8 s: stage s holds its chunk
-    const uint32_t bar_m = sbase + OFF_BAR + 16, bar_d = sbase + OFF_BAR + 24;  // chunk products; drain on error
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 32);
+    // mbarriers (+ 8 s for stage s): ku (the stage's k rows, U slice and factors have landed), mk (its Mk
+    // has landed), kt (the Kt product of the stage's chunk has completed); m (a chunk's chain product and
+    // every product before it); d (drain on error)
+    const uint32_t bar_ku = sbase + OFF_BAR, bar_mk = bar_ku + 16, bar_kt = bar_ku + 32;
+    const uint32_t bar_m = bar_ku + 48, bar_d = bar_ku + 56;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 64);
     if (tid == 0) {
-        tc::mbar_init(bar_full, 1);
-        tc::mbar_init(bar_full + 8, 1);
-        tc::mbar_init(bar_m, 1);
-        tc::mbar_init(bar_d, 1);
+        for (int i = 0; i < 8; ++i) tc::mbar_init(bar_ku + 8 * i, 1);
         tc::mbar_init_fence();
     }
     if (wid == 0) tc::tmem_alloc(smem_addr(tslot), kTmemCols);
     __syncthreads();
 
-    // TMA fill of stage st with chunk c (data lane)
-    int fills[2] = {0, 0};
-    auto fill = [&](int c, int st) {
-        const uint32_t base = sbase + st * kStage, full = bar_full + 8 * st;
+    // TMA fills of stage st with chunk c (data lane): its k rows, U slice and factors; its Mk
+    int fills_ku[2] = {0, 0}, fills_mk[2] = {0, 0};
+    auto fill_ku = [&](int c, int st) {
+        const uint32_t base = sbase + st * kStage, full = bar_ku + 8 * st;
         const int trow = (c * Nv + h) * L;  // first row of the chunk's tiles in the workspace
         const int cstart = seq_t0 + (c - c_begin) * L;
-        tma::expect_tx(full, delta ? kStageTx : kStageTx - 32768);
-        if (delta) {  // Mk enters only the rules with the retrieval
-            tma::load_2d(base + SG_MK, &tm_mk, 0, trow, full);
-            tma::load_2d(base + SG_MK + 16384, &tm_mk, 64, trow, full);
-        }
+        tma::expect_tx(full, kKUTx);
         tma::load_3d(base + SG_K, &tm_k, 0, hq, cstart, full);  // columns past Dk (= 64) read as zero
         tma::load_3d(base + SG_K + 16384, &tm_k, 64, hq, cstart, full);
         tma::load_2d(base + SG_U, &tm_u, col0, trow, full);
         tma::load_1d(sbase + OFF_F + st * kFaStride * 4, fa + (size_t)(c * Nv + h) * kFaStride, kFaStride * 4,
                      full);
-        ++fills[st];
+        ++fills_ku[st];
+    };
+    auto fill_mk = [&](int c, int st) {  // Mk enters only the rules with the retrieval
+        const uint32_t base = sbase + st * kStage, full = bar_mk + 8 * st;
+        const int trow = (c * Nv + h) * L;
+        tma::expect_tx(full, 32768);
+        tma::load_2d(base + SG_MK, &tm_mk, 0, trow, full);
+        tma::load_2d(base + SG_MK + 16384, &tm_mk, 64, trow, full);
+        ++fills_mk[st];
     };
     // After stage st has landed with chunk c (epilogue warps): zero the k rows
     // past a short chunk, and stage Ub = diag(f) U as bf16 hi (over U) and lo.
@@ -239,13 +244,15 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
             tma::prefetch_map(&tm_k);
             tma::prefetch_map(&tm_u);
             tma::prefetch_map(&tm_sc);
-            if (lo < hi) fill(lo, 0);
-            if (lo + 1 < hi) fill(lo + 1, 1);
+            for (int j = 0; j < 2 && lo + j < hi; ++j) {
+                fill_ku(lo + j, j);
+                if (delta) fill_mk(lo + j, j);
+            }
         }
     } else if (epi) {
         store_state_operand(0);
         if (lo < hi) {
-            ok = warp_wait(bar_full, 0, lane);
+            ok = warp_wait(bar_ku, 0, lane);
             dg = stage_ub(lo, 0);
         }
     }
@@ -263,13 +270,14 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
     // of a k step is the base descriptor plus (byte offset >> 4).
     const uint64_t dMk0 = tc::desc_k128(sbase + SG_MK), dK0 = tc::desc_mn(sbase + SG_K, 16384, 1024, 2);
     const uint64_t dUb0 = tc::desc_mn(sbase + SG_U, 16384, 1024, 2), dS0 = tc::desc_mn(sbase + OFF_S, 0, 1024, 2);
-    // Kt of the chunk in stage st into accumulator st (issue lane)
+    // Kt of the chunk in stage st into accumulator st (issue lane), tracked by kt[st]
     auto issue_kt = [&](int st) {
         const uint64_t so = (uint64_t)((st * kStage) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
             tc::mma_f16(tmem + st * 128, dK0 + so + (uint64_t)((kk * 2048) >> 4),
                         dUb0 + so + (uint64_t)((kk * 2048) >> 4), idesc_kt, kk > 0 ? 1u : 0u);
+        tc::commit(bar_kt + 8 * st);
     };
     bool issued = false;  // issue lane: any MMA in flight
 
@@ -277,19 +285,25 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
         const int st = it & 1;  // stage, accumulator and S buffer of chunk c
         const bool has_next = c + 1 < hi;
         if (issuer) {
+            bool w_ok = true;
             if (lane == 0) {
                 if (it == 0) issue_kt(0);  // the first chunk's Kt, before its chain product
                 const uint64_t so = (uint64_t)((st * kStage) >> 4), sb = (uint64_t)((st * 16384) >> 4);
                 if (delta) {
+                    w_ok = tc::mbar_wait_bounded(bar_mk + 8 * st, (uint32_t)((it >> 1) & 1));  // Mk of chunk c
+                    tc::fence_after_sync();
+                    if (w_ok) {
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_f16(tmem + st * 128, dMk0 + so + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                                    dS0 + sb + (uint64_t)((kk * 2048) >> 4), idesc_mk, 1u);
+                        for (int kk = 0; kk < 8; ++kk)
+                            tc::mma_f16(tmem + st * 128,
+                                        dMk0 + so + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                                        dS0 + sb + (uint64_t)((kk * 2048) >> 4), idesc_mk, 1u);
+                    }
                 }
                 tc::commit(bar_m);  // chunk c's products: Kt (issued before) and -Mk S
                 issued = true;
             }
-            __syncwarp();
+            ok = __shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0) != 0 && ok;
             if (has_next) {
                 named_sync(1, 288);  // Ub of chunk c + 1 is staged
                 if (lane == 0) issue_kt(st ^ 1);
@@ -301,16 +315,23 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
                 // the state entering chunk c, from its operand copy
                 tma::store_2d(&tm_sc, col0, (c * Nv + h) * L, sbase + OFF_S + st * 16384);
                 tma::commit_group();
-                // stage st is free once chunk c's products have completed
-                w_ok = tc::mbar_wait_bounded(bar_m, (uint32_t)(it & 1));
-                if (w_ok && c + 2 < hi) fill(c + 2, st);
+                // stage st takes chunk c + 2: its k rows, U slice and factors once chunk c's Kt has read the
+                // stage's (Kt was issued during the previous chunk), its Mk once chunk c's chain product has
+                // read Mk
+                if (c + 2 < hi) {
+                    w_ok = tc::mbar_wait_bounded(bar_kt + 8 * st, (uint32_t)((it >> 1) & 1));
+                    if (w_ok) fill_ku(c + 2, st);
+                }
+                const bool m_ok = tc::mbar_wait_bounded(bar_m, (uint32_t)(it & 1));
+                w_ok = w_ok && m_ok;
+                if (w_ok && delta && c + 2 < hi) fill_mk(c + 2, st);
                 tma::wait_read_all();  // the store of S_c has read its buffer
             }
             ok = __shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0) != 0;
         } else {  // epilogue warps
             float dg_next = 1.f;
             if (has_next) {
-                const bool f_ok = warp_wait(bar_full + 8 * (st ^ 1), (uint32_t)(((it + 1) >> 1) & 1), lane);
+                const bool f_ok = warp_wait(bar_ku + 8 * (st ^ 1), (uint32_t)(((it + 1) >> 1) & 1), lane);
                 ok = ok && f_ok;
                 dg_next = stage_ub(c + 1, st ^ 1);
                 tc::fence_proxy_async();
@@ -335,8 +356,10 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
 
     // copies and MMAs still in flight land before shared and tensor memory are released
     if (producer && lane == 0) {
-        for (int st = 0; st < 2; ++st)
-            if (fills[st] > 0) tc::mbar_wait_bounded(bar_full + 8 * st, (uint32_t)((fills[st] - 1) & 1));
+        for (int st = 0; st < 2; ++st) {
+            if (fills_ku[st] > 0) tc::mbar_wait_bounded(bar_ku + 8 * st, (uint32_t)((fills_ku[st] - 1) & 1));
+            if (fills_mk[st] > 0) tc::mbar_wait_bounded(bar_mk + 8 * st, (uint32_t)((fills_mk[st] - 1) & 1));
+        }
         tma::wait_read_all();  // the stores have read shared memory (the grid's end publishes them)
     }
     if (issuer && lane == 0 && !ok && issued) {  // a commit covers every MMA issued before it
