@@ -25,7 +25,8 @@ GDN_ERR_ALIGNMENT, GDN_ERR_WORKSPACE, GDN_ERR_CUDA, GDN_ERR_OVERLAP = 4, 5, 6, 7
 GDN_ERR_SCRATCH_LIMIT = 8
 NOALLOC_SCRATCH_BYTES = 64 << 20
 # bits of the device status words (GDN_DEV_* in gdn.h): word 0 cu_seqlens, word 2 waits, word 3 fp16 range
-DEV_BITS = {0: {1: "cu[0] != 0", 2: "cu_seqlens decreasing", 4: "cu[B] != T"},
+DEV_BITS = {0: {1: "cu[0] != 0", 2: "cu_seqlens decreasing", 4: "cu[B] != T", 8: "a gate that is not <= 0",
+                16: "a beta outside [0, 1]", 32: "a state index outside [0, P)"},
             2: {1: "a wait of the state pass gave up", 2: "a wait of the output kernel gave up",
                 4: "a wait of the intra-chunk kernel gave up", 8: "the self-test wait gave up"},
             3: {1: "U (or beta v) beyond the fp16 range", 2: "the state beyond the fp16 range",
@@ -88,6 +89,10 @@ def lib():
         L.gdn_testing_host_plan.argtypes = [p, i64, i32, i32, p, i32]
         L.gdn_read_status.restype = ctypes.c_int
         L.gdn_read_status.argtypes = [p, p, p]
+        L.gdn_check_values.restype = ctypes.c_int
+        L.gdn_check_values.argtypes = [p, p, p, i64, i32, i32, i32, p, p]
+        L.gdn_set_value_checks.restype = ctypes.c_int
+        L.gdn_set_value_checks.argtypes = [ctypes.c_int]
         L.gdn_noalloc_read_status.restype = ctypes.c_int
         L.gdn_noalloc_read_status.argtypes = [p, p]
         L.gdn_short_fwd.restype = ctypes.c_int
@@ -303,6 +308,36 @@ def read_status(workspace, stream=None) -> list:
     _check(lib().gdn_read_status(_ptr(workspace), _ptr(dst), _stream(st)), "gdn_read_status")
     st.synchronize()
     return dst.cpu().tolist()
+
+
+def check_values(g=None, beta=None, state_indices=None, P=0, stream=None) -> int:
+    """The value checks of ``gdn_check_values`` on device tensors g [T, Nv] fp32, beta [T, Nv] bf16 and
+    state_indices [B] int32 (each optional): the GDN_DEV_VAL_* bits found (0 when every value is in range),
+    after the stream's work is done."""
+    ref = next((t for t in (g, beta, state_indices) if t is not None), None)
+    if ref is None:
+        return 0
+    T, Nv = (g.shape[0], g.shape[1]) if g is not None else (beta.shape[0], beta.shape[1]) if beta is not None \
+        else (0, 1)
+    for t, dt in ((g, torch.float32), (beta, torch.bfloat16)):
+        if t is not None:
+            _need(t, "g" if dt == torch.float32 else "beta", dt, (T, Nv), ref.device)
+    B = 0
+    if state_indices is not None:
+        _need(state_indices, "state_indices", torch.int32, (state_indices.shape[0],), ref.device)
+        B = state_indices.shape[0]
+    st = torch.cuda.current_stream() if stream is None else stream
+    word = torch.zeros(1, dtype=torch.int32, device=ref.device)
+    _check(lib().gdn_check_values(_ptr(g), _ptr(beta), _ptr(state_indices), T, B, Nv, int(P), _ptr(word),
+                                  _stream(st)), "gdn_check_values")
+    st.synchronize()
+    return int(word.item())
+
+
+def set_value_checks(on: bool) -> bool:
+    """Switch the value checks of the chunked entry points on or off (``gdn_set_value_checks``); returns the
+    previous setting.  With the checks on, a chunked call's status word 0 also carries the GDN_DEV_VAL_* bits."""
+    return bool(lib().gdn_set_value_checks(1 if on else 0))
 
 
 def noalloc_status(stream=None) -> list:

@@ -11,6 +11,7 @@
 #include <algorithm>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "gdn.h"
@@ -191,6 +192,10 @@ int check_forward(const void *q, const void *k, const void *v, const float *g,
 
 }  // namespace
 
+namespace {
+std::atomic<int> g_value_checks{0};  // the process-wide switch of gdn_set_value_checks
+}  // namespace
+
 extern "C" {
 
 const char *gdn_status_string(int status)
@@ -211,6 +216,20 @@ const char *gdn_status_string(int status)
 }
 
 int gdn_version(void) { return kVersion; }
+
+int gdn_check_values(const float *g, const uint16_t *beta, const int32_t *state_indices, int64_t T, int32_t B,
+                     int32_t Nv, int32_t P, int32_t *status_word, void *stream)
+{
+    if (!status_word) return GDN_ERR_NULL_ARG;
+    if (T < 0 || B < 0 || Nv <= 0 || P < 0) return GDN_ERR_BAD_SHAPE;
+    if (T * (int64_t)Nv >= (int64_t(1) << 40)) return GDN_ERR_UNSUPPORTED;
+    const auto al = [](const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; };
+    if (!al(g, 4) || !al(status_word, 4) || !al(beta, 2) || !al(state_indices, 4)) return GDN_ERR_ALIGNMENT;
+    return cuda_status(gdn::launch_check_values(g, beta, state_indices, T, Nv, B, P, status_word,
+                                                (cudaStream_t)stream));
+}
+
+int gdn_set_value_checks(int on) { return g_value_checks.exchange(on ? 1 : 0); }
 
 int gdn_read_status(const void *workspace, int32_t *status_out, void *stream)
 {
@@ -476,6 +495,8 @@ int gdn_chunk_fwd_typed(const void *q, const void *k, const void *v, const float
     const uint16_t *q16 = static_cast<const uint16_t *>(q), *k16 = static_cast<const uint16_t *>(k),
                    *v16 = static_cast<const uint16_t *>(v);
     cudaError_t e = gdn::launch_chunk_map(cu_seqlens, B, Ti, NC, w, st);
+    if (e == cudaSuccess && g_value_checks.load(std::memory_order_relaxed))  // into word 0, after the table clears it
+        e = gdn::launch_check_values(g, beta, state_pool ? state_indices : nullptr, T, Nv, B, P, w.status, st);
     if (e == cudaSuccess && act_dtype == GDN_DTYPE_FP32 && T > 0) {
         uint16_t *aq = w.act16, *ak = aq + (size_t)T * Nqk * Dk, *av = ak + (size_t)T * Nqk * Dk;
         e = gdn::launch_act_to_f16(static_cast<const float *>(q), static_cast<const float *>(k),

@@ -42,6 +42,10 @@ struct Workspace {
     int NC;  // max chunks
 };
 
+// the value checks of gdn_check_values: bits GDN_DEV_VAL_* ORed into *word (g, beta [T][Nv] or null;
+// idx [B] or null)
+cudaError_t launch_check_values(const float *g, const uint16_t *beta, const int32_t *idx, long long T, int Nv, int B,
+                                int P, int32_t *word, cudaStream_t st);
 cudaError_t launch_chunk_map(const int32_t *cu, int B, int T, int NC, const Workspace &ws,
                              cudaStream_t st);
 // intra and output run over chunks [c0, c0 + nc); the state pass over [c_lo, c_hi), range index `range`

@@ -30,10 +30,12 @@
  *     Argument errors are returned before anything is enqueued.  A launch
  *     failure returns GDN_ERR_CUDA; a fault inside a kernel surfaces at the
  *     caller's next synchronisation, as with any CUDA launch.
- *   - Values are not validated on the device: gates are expected <= 0 and
+ *   - Values are not validated on the hot path: gates are expected <= 0 and
  *     beta in [0, 1] (the decode page leaves both unchecked on purpose, since
  *     a reduction over the inputs would cost a pass on the inference path);
- *     state_indices must lie in [0, P).
+ *     state_indices must lie in [0, P).  On request they are checked on the
+ *     device (gdn_check_values, and gdn_set_value_checks for the chunked
+ *     path), into status bits GDN_DEV_VAL_*.
  *   - Return value: a gdn_status_t code (0 = success).  It covers what the host
  *     can see when it enqueues.  What only the device can see (a malformed
  *     cu_seqlens, a bounded wait that gave up, a value outside the fp16 range)
@@ -45,10 +47,12 @@
  * operator raises ValueError for bad arguments and RuntimeError when
  * execution fails; here the host checks come back as the return code and the
  * device-side findings as four int32 words at the start of the workspace:
- *   [0] cu_seqlens errors: GDN_DEV_CU_FIRST (cu[0] != 0), GDN_DEV_CU_DECREASING,
- *       GDN_DEV_CU_TOTAL (cu[B] != T).  The chunk table clamps every token range
- *       to [0, T), so nothing is read or written out of bounds, but the
- *       results are those of the clamped lengths.
+ *   [0] input errors.  cu_seqlens: GDN_DEV_CU_FIRST (cu[0] != 0),
+ *       GDN_DEV_CU_DECREASING, GDN_DEV_CU_TOTAL (cu[B] != T); the chunk table
+ *       clamps every token range to [0, T), so nothing is read or written out
+ *       of bounds, but the results are those of the clamped lengths.  With
+ *       value checks switched on (gdn_set_value_checks): GDN_DEV_VAL_GATE,
+ *       GDN_DEV_VAL_BETA, GDN_DEV_VAL_INDEX (see gdn_check_values).
  *   [1] the number of chunks.
  *   [2] bounded waits that gave up: GDN_DEV_WAIT_STATE, GDN_DEV_WAIT_OUTPUT,
  *       GDN_DEV_WAIT_INTRA (GDN_DEV_WAIT_SELFTEST: the test hook of
@@ -113,6 +117,9 @@ extern "C" {
 #define GDN_DEV_CU_FIRST 1      /* word 0: cu[0] != 0                  */
 #define GDN_DEV_CU_DECREASING 2 /* word 0: cu[b+1] < cu[b] for some b   */
 #define GDN_DEV_CU_TOTAL 4      /* word 0: cu[B] != T                   */
+#define GDN_DEV_VAL_GATE 8      /* word 0: a gate that is not <= 0 (or a NaN)   */
+#define GDN_DEV_VAL_BETA 16     /* word 0: a beta outside [0, 1] (or a NaN)     */
+#define GDN_DEV_VAL_INDEX 32    /* word 0: a state index outside [0, P)         */
 #define GDN_DEV_WAIT_STATE 1    /* word 2: a wait of the state pass gave up     */
 #define GDN_DEV_WAIT_OUTPUT 2   /* word 2: a wait of the output kernel gave up  */
 #define GDN_DEV_WAIT_INTRA 4    /* word 2: a wait of the intra-chunk kernel gave up */
@@ -156,6 +163,34 @@ int gdn_version(void);
  * the status.
  */
 int gdn_read_status(const void *workspace, int32_t *status_out, void *stream);
+
+/*
+ * Value checks on the device (the decode page's "Raises" cases that concern
+ * values rather than shapes).  One pass over g and beta ([T, Nv], fp32 and
+ * bf16, each optional: NULL skips it) and state_indices ([B], int32, NULL
+ * skips it), ORing into the device int32 *status_word:
+ *   GDN_DEV_VAL_GATE  for a gate that is not <= 0 (a positive value or a NaN),
+ *   GDN_DEV_VAL_BETA  for a beta outside [0, 1] (or a NaN),
+ *   GDN_DEV_VAL_INDEX for an index outside [0, P).
+ * The word is not cleared first; the call enqueues one kernel on `stream` and
+ * returns.  It reads about 6 bytes per (token, v-head), which is why the hot
+ * path does not run it unless asked.  Errors: GDN_ERR_NULL_ARG (status_word),
+ * GDN_ERR_BAD_SHAPE (negative sizes, Nv <= 0, P < 0), GDN_ERR_ALIGNMENT (g or
+ * status_word not 4-byte aligned, beta not 2-byte aligned), GDN_ERR_CUDA.
+ */
+int gdn_check_values(const float *g, const uint16_t *beta, const int32_t *state_indices, int64_t T, int32_t B,
+                     int32_t Nv, int32_t P, int32_t *status_word, void *stream);
+
+/*
+ * Process-wide switch of the value checks for the chunked entry points
+ * (gdn_chunk_fwd, gdn_chunk_fwd_rule, gdn_chunk_fwd_typed, gdn_chunk_fwd_host,
+ * gdn_chunk_fwd_noalloc): when on (nonzero), each call runs gdn_check_values
+ * on its g, beta and state_indices (the pool's P) right after the chunk table,
+ * into status word 0 of its workspace, so gdn_read_status reports them.  The
+ * fused short-sequence path has no workspace and is not covered (call
+ * gdn_check_values directly).  Off by default.  Returns the previous setting.
+ */
+int gdn_set_value_checks(int on);
 
 /*
  * Bytes of device workspace that the chunked path of gdn_chunk_fwd needs for

@@ -35,7 +35,7 @@ def test_headers_declare_entry_points():
     names = _declared()
     for n in ("gdn_chunk_fwd", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string", "gdn_short_fwd",
               "gdn_stage_intra", "gdn_stage_state", "gdn_stage_output", "gdn_read_status",
-              "gdn_noalloc_read_status", "gdn_selftest_wait"):
+              "gdn_noalloc_read_status", "gdn_selftest_wait", "gdn_check_values", "gdn_set_value_checks"):
         assert n in names
 
 
@@ -213,10 +213,30 @@ def test_status_entry_argument_errors(lib):
     assert lib.gdn_selftest_wait((1 << 22) + 1, 0, vp(1 << 20), 16, None) == B.GDN_ERR_BAD_SHAPE
 
 
+def test_value_check_entry_argument_errors(lib):
+    """gdn_check_values refuses bad arguments before it enqueues anything; the switch of the chunked
+    entry points is process-wide and returns its previous setting."""
+    vp = ctypes.c_void_p
+    g, beta, idx, word = vp(1 << 20), vp(2 << 20), vp(3 << 20), vp(4 << 20)
+    assert lib.gdn_check_values(g, beta, idx, 100, 2, 4, 8, None, None) == B.GDN_ERR_NULL_ARG
+    assert lib.gdn_check_values(g, beta, idx, -1, 2, 4, 8, word, None) == B.GDN_ERR_BAD_SHAPE
+    assert lib.gdn_check_values(g, beta, idx, 100, -2, 4, 8, word, None) == B.GDN_ERR_BAD_SHAPE
+    assert lib.gdn_check_values(g, beta, idx, 100, 2, 0, 8, word, None) == B.GDN_ERR_BAD_SHAPE
+    assert lib.gdn_check_values(g, beta, idx, 100, 2, 4, -1, word, None) == B.GDN_ERR_BAD_SHAPE
+    assert lib.gdn_check_values(vp((1 << 20) + 2), beta, idx, 100, 2, 4, 8, word, None) == B.GDN_ERR_ALIGNMENT
+    assert lib.gdn_check_values(g, vp((2 << 20) + 1), idx, 100, 2, 4, 8, word, None) == B.GDN_ERR_ALIGNMENT
+    assert lib.gdn_check_values(g, beta, idx, 100, 2, 4, 8, vp((4 << 20) + 2), None) == B.GDN_ERR_ALIGNMENT
+    # nothing to check: no launch, GDN_OK
+    assert lib.gdn_check_values(None, None, None, 100, 0, 4, 8, word, None) == B.GDN_OK
+    assert gdn.set_value_checks(True) is False
+    assert gdn.set_value_checks(False) is True
+    assert gdn.set_value_checks(False) is False
+
+
 def test_status_bits_match_the_header():
     text = open(os.path.join(ROOT, "include", "gdn.h")).read()
     macros = {m.group(1): int(m.group(2)) for m in re.finditer(r"#define (GDN_DEV_\w+) (\d+)", text)}
-    word = {"CU": 0, "WAIT": 2, "RANGE": 3}
+    word = {"CU": 0, "VAL": 0, "WAIT": 2, "RANGE": 3}
     for name, bit in macros.items():
         assert bit in B.DEV_BITS[word[name.split("_")[2]]], name
     assert sum(len(v) for v in B.DEV_BITS.values()) == len(macros)

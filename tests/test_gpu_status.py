@@ -8,7 +8,10 @@ status words of the workspace, read with gdn_read_status:
   - a bounded wait that gave up (word 2), run out here on purpose through the
     self-test hook, which waits on an mbarrier that nothing arrives on: no
     fault, no trap, no hang, and the bit comes back set;
-  - a value beyond the fp16 range in an fp16 intermediate (word 3).
+  - a value beyond the fp16 range in an fp16 intermediate (word 3);
+  - with the value checks switched on, a gate above 0, a beta outside [0, 1]
+    or a slot index outside the pool (word 0, GDN_DEV_VAL_*), and the same
+    bits from gdn_check_values called on its own.
 """
 from __future__ import annotations
 
@@ -123,3 +126,73 @@ def test_fp16_range_large_values_match_or_report():
     gdn.chunk_fwd(d.q, d.k, d.v, d.g, d.beta, d.cu_seqlens, d.state_pool, d.state_indices, scale=d.scale,
                   eps=d.eps, workspace=ws)
     assert gdn.read_status(ws)[2:] == [0, 0]
+
+
+VAL_GATE, VAL_BETA, VAL_INDEX = 8, 16, 32
+
+
+def _bf16_bits(x):
+    return torch.tensor([x], dtype=torch.float32).to(torch.bfloat16).view(torch.int16).item()
+
+
+@pytest.mark.parametrize("plant,bits", [
+    (None, 0),
+    ("gate_positive", VAL_GATE),
+    ("gate_nan", VAL_GATE),
+    ("beta_above_one", VAL_BETA),
+    ("beta_negative", VAL_BETA),
+    ("beta_nan", VAL_BETA),
+    ("index_at_P", VAL_INDEX),
+    ("index_negative", VAL_INDEX),
+])
+def test_check_values_finds_each_case(plant, bits):
+    inp = inputs.make([300, 129, 1, 700], Nqk=2, Nv=4, state=("normal", 0.02, 6, "perm"), seed=111)
+    d = inp.to(DEV)
+    g, beta, idx = d.g.clone(), d.beta.clone(), d.state_indices.clone()
+    P = inp.state_pool.shape[0]
+    if plant == "gate_positive":
+        g[777, 3] = 0.25
+    elif plant == "gate_nan":
+        g[5, 0] = float("nan")
+    elif plant == "beta_above_one":
+        beta[1000, 2] = 1.5
+    elif plant == "beta_negative":
+        beta[0, 1] = -0.125
+    elif plant == "beta_nan":
+        beta.view(torch.int16)[42, 3] = 0x7FC0
+    elif plant == "index_at_P":
+        idx[2] = P
+    elif plant == "index_negative":
+        idx[0] = -1
+    assert gdn.check_values(g, beta, idx, P) == bits
+    assert gdn.check_values(g=g) == bits & VAL_GATE
+    assert gdn.check_values(beta=beta) == bits & VAL_BETA
+    assert gdn.check_values(state_indices=idx, P=P) == bits & VAL_INDEX
+
+
+def test_value_checks_switch_reports_through_the_workspace():
+    """With the switch on, a chunked call's status word 0 carries the value bits (and its results are
+    those of the call without the checks); with it off, nothing is checked."""
+    inp = inputs.make([300, 129, 1, 700], Nqk=2, Nv=4, state=("normal", 0.02, 6, "perm"), seed=113)
+    d = inp.to(DEV)
+    g = d.g.clone()
+    g[100, 2] = 0.5  # a gate above 0
+    ws = torch.empty(gdn.workspace_bytes(d.T, d.B, d.Nqk, d.Nv), dtype=torch.uint8, device=DEV)
+    run = lambda: gdn.chunk_fwd(d.q, d.k, d.v, g, d.beta, d.cu_seqlens, d.state_pool, d.state_indices,
+                                scale=d.scale, eps=d.eps, workspace=ws)
+    out0, fin0 = run()
+    assert gdn.read_status(ws)[0] == 0
+    prev = gdn.set_value_checks(True)
+    try:
+        out1, fin1 = run()
+        words = gdn.read_status(ws)
+        assert words[0] == VAL_GATE, words
+        assert "a gate that is not <= 0" in gdn.decode_status(words)
+        # a clean call on the same workspace: the chunk table clears the word first
+        gdn.chunk_fwd(d.q, d.k, d.v, d.g, d.beta, d.cu_seqlens, d.state_pool, d.state_indices,
+                                scale=d.scale, eps=d.eps, workspace=ws)
+        assert gdn.read_status(ws)[0] == 0
+    finally:
+        gdn.set_value_checks(prev)
+    torch.cuda.synchronize()
+    assert torch.equal(out0, out1) and torch.equal(fin0, fin1)
