@@ -177,6 +177,23 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b)
     return *reinterpret_cast<const float2 *>(&d);
 }
 
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<const uint64_t *>(&a)), "l"(*reinterpret_cast<const uint64_t *>(&b)));
+    return *reinterpret_cast<const float2 *>(&d);
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b)
+{
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<const uint64_t *>(&a)), "l"(*reinterpret_cast<const uint64_t *>(&b)));
+    return *reinterpret_cast<const float2 *>(&d);
+}
+
 __device__ __forceinline__ float warp_sum(float x)
 {
 #pragma unroll

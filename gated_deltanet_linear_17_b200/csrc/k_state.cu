@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
         }
         const float *fr = reinterpret_cast<const float *>(smem + OFF_F + st * kFaStride * 4);
         const float f = fr[row];
+        const float2 ff = make_float2(f, f);
         uint4 x[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) x[j] = *reinterpret_cast<const uint4 *>(base + SG_U + tc::sw128c(row, (cbase >> 3) + j));
@@ -172,9 +173,11 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
             const uint32_t x4[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
             uint32_t h4[4], l4[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 u = unpack_h2(x4[e]);
-                split2<F16>(u.x * f, u.y * f, h4[e], l4[e]);
+            for (int e = 0; e < 4; ++e) {  // split2 in packed fp32 pairs (the same roundings)
+                const float2 u = fmul2(unpack_h2(x4[e]), ff);
+                h4[e] = pack2<F16>(u.x, u.y);
+                const float2 r = fsub2(u, unpack2<F16>(h4[e]));
+                l4[e] = pack2<F16>(r.x, r.y);
             }
             const uint32_t off = tc::sw128c(row, (cbase >> 3) + j);
             *reinterpret_cast<uint4 *>(base + SG_U + off) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
@@ -343,8 +346,14 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
             float dh[32], dl[32];
             tc::tmem_ld32(t_mine + st * 128, dh);
             tc::tmem_ld32(t_mine + st * 128 + 64, dl);
+            const float2 dg2 = make_float2(dg, dg);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) s[j] = fmaf(dg, s[j], dh[j] + dl[j]);
+            for (int j = 0; j < 32; j += 2) {  // s = dg s + (dh + dl), in packed fp32 pairs
+                const float2 r = ffma2(dg2, make_float2(s[j], s[j + 1]),
+                                       fadd2(make_float2(dh[j], dh[j + 1]), make_float2(dl[j], dl[j + 1])));
+                s[j] = r.x;
+                s[j + 1] = r.y;
+            }
             store_state_operand(st ^ 1);
             tc::fence_proxy_async();
             dg = dg_next;
