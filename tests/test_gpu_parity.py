@@ -181,6 +181,19 @@ def test_ragged_lengths_with_empty_sequences():
         assert torch.equal(fin[b].cpu(), inp.state_pool[inp.state_indices[b]])
 
 
+def test_largest_head_counts():
+    """The largest head counts the boundary accepts (Nqk = 64, Nv = 256, GQA group 4) on ragged sequences
+    that span several chunks, with a pool: the kernels' head indexing at their widest grid; the oracle on a
+    spread of v-heads, the first and last of qk-head groups among them."""
+    inp = inputs.make([300, 129, 1, 260], Nqk=64, Nv=256, state=("normal", 0.02, 5, "perm"), seed=121)
+    for ms in (0, inp.max_seqlen):  # the chunked kernels, then the same call with a length hint
+        out, fin = _gpu(inp, max_seqlen=ms)
+        _check(inp, out, fin, heads=[0, 3, 4, 127, 128, 200, 255], what=f"Nqk=64 Nv=256 max_seqlen={ms}")
+    short = inputs.make([3, 1, 8, 5], Nqk=64, Nv=256, state=("normal", 0.02, 6, "perm"), seed=122)
+    out, fin = _gpu(short, max_seqlen=short.max_seqlen)  # the fused short-sequence kernel
+    _check(short, out, fin, heads=[0, 63, 64, 255], what="short Nqk=64 Nv=256")
+
+
 def test_all_sequences_empty():
     inp = inputs.make([0, 0, 0], Nqk=1, Nv=2, state=("normal", 0.02, 3, "perm"), seed=7)
     out, fin = _gpu(inp)
