@@ -147,6 +147,7 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi)
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
 }
+__device__ __forceinline__ uint32_t pack_h2f(float2 v) { return pack_h2(v.x, v.y); }
 __device__ __forceinline__ float2 unpack_h2(uint32_t x)
 {
     return __half22float2(*reinterpret_cast<const __half2 *>(&x));

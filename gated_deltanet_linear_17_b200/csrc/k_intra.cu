@@ -144,11 +144,12 @@ __device__ __forceinline__ void scale_rows_f16(uint8_t *tile, int t, int nvalid,
                 }
                 *vmax = absmax_nan(*vmax, mx * m);
             }
-            const float2 p0 = unpack2<F16>(x[i].x), p1 = unpack2<F16>(x[i].y), p2 = unpack2<F16>(x[i].z),
-                         p3 = unpack2<F16>(x[i].w);
+            const float2 mm = make_float2(m, m);  // packed fp32 pairs: the same products
+            const float2 p0 = fmul2(unpack2<F16>(x[i].x), mm), p1 = fmul2(unpack2<F16>(x[i].y), mm),
+                         p2 = fmul2(unpack2<F16>(x[i].z), mm), p3 = fmul2(unpack2<F16>(x[i].w), mm);
             *reinterpret_cast<uint4 *>(tile + t128(r, t & 15)) =
-                r < nvalid ? make_uint4(pack_h2(p0.x * m, p0.y * m), pack_h2(p1.x * m, p1.y * m),
-                                        pack_h2(p2.x * m, p2.y * m), pack_h2(p3.x * m, p3.y * m))
+                r < nvalid ? make_uint4(pack_h2(p0.x, p0.y), pack_h2(p1.x, p1.y), pack_h2(p2.x, p2.y),
+                                        pack_h2(p3.x, p3.y))
                            : make_uint4(0, 0, 0, 0);
         }
     }
@@ -401,7 +402,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int jj = (q8 & 1) * 8 + 2 * e;
-                            w4[e] = (q8 < 2 && hi) ? pack_h2(eb * kf[jj] * a[jj], eb * kf[jj + 1] * a[jj + 1]) : 0u;
+                            w4[e] = (q8 < 2 && hi) ? pack_h2f(fmul2(fmul2(make_float2(eb, eb), make_float2(kf[jj], kf[jj + 1])),
+                                                                    make_float2(a[jj], a[jj + 1])))
+                                                   : 0u;
                         }
                         *reinterpret_cast<uint4 *>(smem + ta + t128(row, (j0 >> 3) + q8)) =
                             make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -422,7 +425,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int jj = q16 * 16 + q8 * 8 + 2 * e;
-                            w4[e] = pack_h2(eb * kf[jj] * a[jj], eb * kf[jj + 1] * a[jj + 1]);
+                            w4[e] = pack_h2f(fmul2(fmul2(make_float2(eb, eb), make_float2(kf[jj], kf[jj + 1])),
+                                                   make_float2(a[jj], a[jj + 1])));
                         }
                         *reinterpret_cast<uint4 *>(smem + ta + t128(row, (jb >> 3) + q8)) =
                             make_uint4(w4[0], w4[1], w4[2], w4[3]);

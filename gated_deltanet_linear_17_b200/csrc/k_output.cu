@@ -226,7 +226,8 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int jj = q8 * 8 + 2 * e, d = jj & 15;
-                        const uint32_t left = pack_h2(eb * kf[d] * a[jj], eb * kf[d + 1] * a[jj + 1]);
+                        const uint32_t left = pack_h2f(fmul2(fmul2(make_float2(eb, eb), make_float2(kf[d], kf[d + 1])),
+                                                             make_float2(a[jj], a[jj + 1])));
                         const uint32_t dg = pack_h2(pd[d], pd[d + 1]);
                         pw[q8 * 4 + e] = q8 < 2 ? (hi ? left : dg) : (hi ? dg : 0u);
                     }
@@ -244,7 +245,8 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int jj = q16 * 16 + 2 * e;
-                    pw[q16 * 8 + e] = pack_h2(eb * kf[jj] * a[jj], eb * kf[jj + 1] * a[jj + 1]);
+                    pw[q16 * 8 + e] = pack_h2f(fmul2(fmul2(make_float2(eb, eb), make_float2(kf[jj], kf[jj + 1])),
+                                                     make_float2(a[jj], a[jj + 1])));
                 }
             }
             tc::tmem_st16(t_p, pw);
