@@ -381,7 +381,12 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
                         lds_vec(kd, kfe + rb);
                         const float ed = fr * __expf(gi - gl);
 #pragma unroll
-                        for (int jj = 0; jj < 16; ++jj) dv[jj] = rb + jj < row ? ed * kd[jj] * (hi ? a[16 + jj] : a[jj]) : 0.f;
+                        for (int jj = 0; jj < 16; jj += 2) {
+                            const float2 x = fmul2(fmul2(make_float2(ed, ed), make_float2(kd[jj], kd[jj + 1])),
+                                                   hi ? make_float2(a[16 + jj], a[17 + jj]) : make_float2(a[jj], a[jj + 1]));
+                            dv[jj] = rb + jj < row ? x.x : 0.f;
+                            dv[jj + 1] = rb + jj + 1 < row ? x.y : 0.f;
+                        }
                     } else {
                         float rkj[16], gmj[16];
                         lds_vec(rkj, rkv + rb);
@@ -462,15 +467,13 @@ __global__ void __launch_bounds__(kIntraThreads, 2) intra_kernel(
                         nr[4 * q + 2] = x.z;
                         nr[4 * q + 3] = x.w;
                     }
-                float s0 = i == cidx ? 1.f : 0.f, s1 = 0.f;
+                // even j into the first lane of the pair, odd j into the second (packed fp32 pairs)
+                float2 s2 = make_float2(i == cidx ? 1.f : 0.f, 0.f);
 #pragma unroll
-                for (int j = 0; j < i; ++j) {
-                    if (j & 1)
-                        s1 = fmaf(nr[j], tcol[j], s1);
-                    else
-                        s0 = fmaf(nr[j], tcol[j], s0);
-                }
-                tcol[i] = i < cidx ? 0.f : s0 + s1;
+                for (int j = 0; j + 1 < i; j += 2)
+                    s2 = ffma2(make_float2(nr[j], nr[j + 1]), make_float2(tcol[j], tcol[j + 1]), s2);
+                if (i & 1) s2.x = fmaf(nr[i - 1], tcol[i - 1], s2.x);
+                tcol[i] = i < cidx ? 0.f : s2.x + s2.y;
             }
             const int col = wid * 16 + cidx;
 #pragma unroll

@@ -211,7 +211,12 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
                     lds_vec(kd, kfe + rb);
                     const float ed = fr * __expf(gi - gl);
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) pd[jj] = rb + jj <= row ? ed * kd[jj] * (hi ? a[16 + jj] : a[jj]) : 0.f;
+                    for (int jj = 0; jj < 16; jj += 2) {
+                        const float2 x = fmul2(fmul2(make_float2(ed, ed), make_float2(kd[jj], kd[jj + 1])),
+                                               hi ? make_float2(a[16 + jj], a[17 + jj]) : make_float2(a[jj], a[jj + 1]));
+                        pd[jj] = rb + jj <= row ? x.x : 0.f;
+                        pd[jj + 1] = rb + jj + 1 <= row ? x.y : 0.f;
+                    }
                 } else {
                     float rkj[16], gmj[16];
                     lds_vec(rkj, rkv + rb);
@@ -304,12 +309,11 @@ __global__ void __launch_bounds__(kOutThreads, 2) output_kernel(
                 const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
                 uint32_t o4[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 qp = unpack2<F16>(w4[e]);
-                    const float x0 = qp.x * qf - z[c4 * 8 + 2 * e];
-                    const float x1 = qp.y * qf - z[c4 * 8 + 2 * e + 1];
-                    vmax = absmax_nan(absmax_nan(vmax, x0), x1);
-                    o4[e] = pack_h2(x0, x1);
+                for (int e = 0; e < 4; ++e) {  // q qf - z as one fused multiply-add per element, in pairs
+                    const float2 x = ffma2(unpack2<F16>(w4[e]), make_float2(qf, qf),
+                                           make_float2(-z[c4 * 8 + 2 * e], -z[c4 * 8 + 2 * e + 1]));
+                    vmax = absmax_nan(absmax_nan(vmax, x.x), x.y);
+                    o4[e] = pack_h2(x.x, x.y);
                 }
                 *p = make_uint4(o4[0], o4[1], o4[2], o4[3]);
             }
