@@ -225,9 +225,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
 #pragma unroll
         for (int j = 0; j < 32; ++j) s[j] = 0.f;
     }
-    // S in fp16 as the MN-major B operand (buffer buf): row `row`, 16-byte chunks cbase/8 .. cbase/8 + 3;
-    // vmax keeps the largest magnitude converted (fp16 range check)
-    float vmax = 0.f;
+    // S in fp16 as the MN-major B operand (buffer buf): row `row`, 16-byte chunks cbase/8 .. cbase/8 + 3
     auto store_state_operand = [&](int buf) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -235,6 +233,11 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
             *reinterpret_cast<uint4 *>(smem + OFF_S + buf * 16384 + tc::sw128c(row, (cbase >> 3) + j)) =
                 make_uint4(pack_h2(v8[0], v8[1]), pack_h2(v8[2], v8[3]), pack_h2(v8[4], v8[5]), pack_h2(v8[6], v8[7]));
         }
+    };
+    // vmax: the largest magnitude of the states converted to fp16 (range check), taken over each state
+    // after its copy is stored, off the chain (at the start of the next chunk, and after the last)
+    float vmax = 0.f;
+    auto track_range = [&]() {
 #pragma unroll
         for (int j = 0; j < 32; ++j) vmax = absmax_nan(vmax, s[j]);
     };
@@ -332,6 +335,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
             }
             ok = __shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0) != 0;
         } else {  // epilogue warps
+            track_range();  // the state stored by the previous chunk (or the initial one), while loads land
             float dg_next = 1.f;
             if (has_next) {
                 const bool f_ok = warp_wait(bar_ku + 8 * (st ^ 1), (uint32_t)(((it + 1) >> 1) & 1), lane);
@@ -375,6 +379,7 @@ __global__ void __launch_bounds__(kStateThreads, 1) state_kernel(
         tc::commit(bar_d);
         tc::mbar_wait_bounded(bar_d, 0);
     }
+    if (epi) track_range();  // the last state stored (a repeat of the initial one when no chunk ran is harmless)
     if (epi && __any_sync(0xffffffffu, out_of_fp16(vmax)) && lane == 0) atomicOr(status + 3, GDN_DEV_RANGE_STATE);
     if (!ok) {
         if (tid == 0) atomicOr(status + 2, GDN_DEV_WAIT_STATE);
