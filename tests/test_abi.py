@@ -177,6 +177,17 @@ def test_python_layer_refuses_cpu_tensors():
         gdn.chunk_fwd(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens)
 
 
+def test_value_checks_refuse_cpu_tensors():
+    import torch
+    from gated_deltanet_linear_17_b200 import inputs
+    inp = inputs.make([5, 3], 1, 2, state=("normal", 0.02, 2, "perm"), seed=0)
+    with pytest.raises(RuntimeError):
+        gdn.check_values(inp.g, inp.beta)
+    with pytest.raises(RuntimeError):
+        gdn.check_values(state_indices=inp.state_indices, P=2)
+    assert gdn.check_values() == 0  # nothing to check
+
+
 def _noalloc(lib, **over):
     M = 1 << 20  # fake, disjoint, 16-byte aligned addresses; every call below returns before any launch
     a = dict(T=8, B=1, Nqk=2, Nv=4, P=0, max_seqlen=0)
