@@ -604,13 +604,16 @@ def host_buffer_bytes(cu_seqlens, Nqk, Nv, with_pool, segments=0) -> int:
 
 
 def chunk_fwd_host(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=None, scale=None, eps=1e-6,
-                   device="cuda", out_host=None, final_host=None, device_buffer=None, segments=0, stream=None):
+                   device="cuda", out_host=None, final_host=None, device_buffer=None, segments=0, stream=None,
+                   check_status=False):
     """End-to-end forward from host tensors through ``gdn_chunk_fwd_host``: the library streams the
     batch through the GPU in pieces, its uploads and downloads overlapped with the compute, and writes
     out and final_state into host tensors (pinned ones keep the copies asynchronous).  ``device_buffer``
     (uint8 on ``device``, at least ``host_buffer_bytes`` long) is allocated here when not given.
     Returns (out_host, final_host, h2d_bytes, d2h_bytes); the host tensors are complete once the
-    stream has reached the end of the call (the stream is synchronised here)."""
+    stream has reached the end of the call (the stream is synchronised here).  The call's device status
+    words, folded over its pieces, sit at the start of ``device_buffer`` (``read_status(device_buffer)``);
+    ``check_status`` raises RuntimeError when they report a problem."""
     if q.dim() != 3 or v.dim() != 3:
         raise ValueError("q/k must be [T, Nqk, 128] and v [T, Nv, 128]")
     T, Nqk, _ = q.shape
@@ -645,6 +648,10 @@ def chunk_fwd_host(q, k, v, g, beta, cu_seqlens, state_pool=None, state_indices=
                                   device_buffer.numel(), _stream(st))
     _check(rc, "gdn_chunk_fwd_host")
     st.synchronize()
+    if check_status:
+        found = decode_status(read_status(device_buffer, st))
+        if found:
+            raise RuntimeError("gdn_chunk_fwd_host: " + "; ".join(found))
     sbytes = Nv * HEAD_DIM * HEAD_DIM * 4
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v, g, beta, cu_seqlens)) + \
         (Bn * sbytes if state_pool is not None else 0)

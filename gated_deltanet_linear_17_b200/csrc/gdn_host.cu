@@ -21,6 +21,7 @@
 
 #include "gdn.h"
 #include "gdn_internal.h"
+#include "gdn_stages.h"
 #include "gdn_testing.h"
 
 namespace {
@@ -34,6 +35,17 @@ size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 __global__ void call_cu_kernel(const int32_t *__restrict__ cu, int b0, int nb, int t0, int t1, int32_t *__restrict__ dst)
 {
     for (int i = threadIdx.x; i <= nb; i += blockDim.x) dst[i] = min(max(cu[b0 + i], t0), t1) - t0;
+}
+
+// the call's status words: those of one piece's workspace folded in (bits ORed, chunk counts added)
+__global__ void status_fold_kernel(const int32_t *__restrict__ w, int32_t *__restrict__ acc)
+{
+    if (threadIdx.x == 0) {
+        acc[0] |= w[0];
+        acc[1] += w[1];
+        acc[2] |= w[2];
+        acc[3] |= w[3];
+    }
 }
 
 struct Streams {
@@ -133,7 +145,7 @@ Plan make_plan(const int32_t *cu, int64_t T, int B, int segments)
 }
 
 struct Regions {
-    size_t q, k, v, g, beta, cu, callcu, out, init, fin, carry, ws, ws_bytes, total;
+    size_t status, q, k, v, g, beta, cu, callcu, out, init, fin, carry, ws, ws_bytes, total;
 };
 
 Regions layout(int64_t T, int B, int Nqk, int Nv, bool pool, const Plan &p)
@@ -142,6 +154,7 @@ Regions layout(int64_t T, int B, int Nqk, int Nv, bool pool, const Plan &p)
     size_t off = 0;
     auto take = [&](size_t n) { const size_t o = off; off = up256(off + n); return o; };
     const size_t sbytes = (size_t)Nv * kD * kD * 4;
+    r.status = take(16);  // at offset 0: the call's four status words, read with gdn_read_status
     r.q = take((size_t)T * Nqk * kD * 2);
     r.k = take((size_t)T * Nqk * kD * 2);
     r.v = take((size_t)T * Nv * kD * 2);
@@ -230,6 +243,10 @@ extern "C" int gdn_chunk_fwd_host(const uint16_t *q, const uint16_t *k, const ui
     auto dinit = reinterpret_cast<float *>(base + r.init), dfin = reinterpret_cast<float *>(base + r.fin);
     auto dcarry = reinterpret_cast<float *>(base + r.carry);
     void *dws = base + r.ws;
+    auto dstatus = reinterpret_cast<int32_t *>(base + r.status);
+    gdn_workspace_layout_t wlay;
+    gdn_workspace_layout(p.max_call_tokens, std::max(p.max_call_seqs, 1), Nqk, Nv, &wlay);
+    const int32_t *ws_status = reinterpret_cast<const int32_t *>(static_cast<char *>(dws) + wlay.status);
     const size_t sfl = (size_t)Nv * kD * kD;  // floats per state
 
     const cudaStream_t st = (cudaStream_t)stream;
@@ -250,6 +267,7 @@ extern "C" int gdn_chunk_fwd_host(const uint16_t *q, const uint16_t *k, const ui
     auto record = [&](cudaEvent_t x, cudaStream_t s) { if (e == cudaSuccess) e = cudaEventRecord(x, s); };
     auto wait = [&](cudaStream_t s, cudaEvent_t x) { if (e == cudaSuccess) e = cudaStreamWaitEvent(s, x, 0); };
 
+    if ((e = cudaMemsetAsync(dstatus, 0, 16, st)) != cudaSuccess) return GDN_ERR_CUDA;
     // the copy streams start after the work the caller already enqueued on `stream`
     record(ev[2 * S], st);
     wait(ss->up, ev[2 * S]);
@@ -284,6 +302,10 @@ extern "C" int gdn_chunk_fwd_host(const uint16_t *q, const uint16_t *k, const ui
             rc = gdn_chunk_fwd(dq + t0 * Nqk * kD, dk + t0 * Nqk * kD, dv + t0 * Nv * kD, dg + t0 * Nv,
                                db + t0 * Nv, ccu, pool, nullptr, scale, eps, dout + t0 * Nv * kD, fin, c.t1 - c.t0,
                                c.nb, Nqk, Nv, pool ? c.nb : 0, 0, dws, r.ws_bytes, stream);
+            if (rc == GDN_OK) {  // this piece's status words, before the next piece clears them
+                status_fold_kernel<<<1, 32, 0, st>>>(ws_status, dstatus);
+                e = cudaGetLastError();
+            }
             if (c.dst == 1) carry_in ^= 1;  // the next segment's first call resumes from this slot
         }
         record(ev[S + s], st);

@@ -393,7 +393,11 @@ int gdn_noalloc_read_status(int32_t *status_out, void *stream);
  *   device_buffer device memory of device_bytes >= gdn_chunk_fwd_host_bytes(...)
  *                 with the same cu_seqlens and segments, 256-byte aligned: it
  *                 holds the device copies, the per-piece workspace and the
- *                 carried states (GDN_ERR_WORKSPACE when too small)
+ *                 carried states (GDN_ERR_WORKSPACE when too small).  Its first
+ *                 16 bytes hold the call's four device status words ("Device
+ *                 status"), folded over its pieces (words 0, 2 and 3 ORed, word 1
+ *                 the total number of chunks): gdn_read_status(device_buffer, ...)
+ *                 reads them once the call's work is done
  * Same limits as gdn_chunk_fwd.  Asynchronous on `stream` (and on the library's
  * two copy streams, which fork from and join back into `stream` within the call).
  */

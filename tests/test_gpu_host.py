@@ -57,3 +57,27 @@ def test_host_entry_full_prefill_workload():
     out, fin, _, _ = gdn.chunk_fwd_host(q, k, v, g, beta, cu, pool, idx, scale=inp.scale, eps=inp.eps, device=DEV)
     assert torch.equal(out, ref_out)
     assert torch.equal(fin, ref_fin)
+
+
+def test_host_entry_status_folded_over_pieces():
+    """The call's device status words sit at the start of the device buffer, folded over the pieces:
+    the chunk counts add up to the batch's, and a value beyond the fp16 range in the first piece is still
+    reported after the later, clean pieces have run (each piece's chunk table clears its own words)."""
+    lens = [1000, 513, 128, 2407]
+    inp = inputs.make(lens, Nqk=2, Nv=4, state=("normal", 0.02, 6, "perm"), seed=63)
+    q, k, v, g, beta, cu, pool, idx = _pinned(inp)
+    need = gdn.host_buffer_bytes(cu, 2, 4, True, 4)
+    buf = torch.empty(need, dtype=torch.uint8, device=DEV)
+    gdn.chunk_fwd_host(q, k, v, g, beta, cu, pool, idx, scale=inp.scale, eps=inp.eps, device=DEV, segments=4,
+                       device_buffer=buf, check_status=True)
+    words = gdn.read_status(buf)
+    assert words[0] == 0 and words[2] == 0 and words[3] == 0, words
+    assert words[1] == sum((n + 127) // 128 for n in lens)
+    rows = gdn.host_plan(inp.cu_seqlens, 4)
+    assert len({r[0] for r in rows}) > 1  # the batch really runs in several pieces
+    big = v.clone()
+    big[:200] *= 2.0 ** 20  # beta v beyond +-65504 in the first sequence, the first piece
+    with pytest.raises(RuntimeError, match="fp16 range"):
+        gdn.chunk_fwd_host(q, k, big, g, beta, cu, pool, idx, scale=inp.scale, eps=inp.eps, device=DEV,
+                           segments=4, device_buffer=buf, check_status=True)
+    assert gdn.read_status(buf)[3] & 1
