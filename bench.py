@@ -566,8 +566,8 @@ def main():
                        "call": f"gdn_chunk_fwd_host from pinned host buffers, {len(plan)} pieces, uploads and "
                                f"downloads overlapped with the compute",
                        "h2d_GB/s": h2d / (ems / 1e3) / 1e9, "d2h_GB/s": d2h / (ems / 1e3) / 1e9}
-        # per piece: one chunk table, the pipelined kernels and the cu kernel
-        line["gpu_launches"] += args.steps * sum(2 + 3 * gdn.pipeline_ranges(r[4] - r[3], r[2], Nqk, Nv)
+        # per piece: the cu kernel, one chunk table, the pipelined kernels and the status fold
+        line["gpu_launches"] += args.steps * sum(3 + 3 * gdn.pipeline_ranges(r[4] - r[3], r[2], Nqk, Nv)
                                                  for r in plan)
 
     # ---- CPU oracle baseline (rank 0, one GPU only)
